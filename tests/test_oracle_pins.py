@@ -1,0 +1,337 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each test checks the token-by-token oracle (``oracle.fwd`` / ``bwd`` /
+``decode``) against something fixed by "Gated DeltaNet-2: Decoupling Erase and
+Write in Linear Attention" or by plain mathematics:
+  * brute-force dense unrolling of the product form
+    S_t = (I - k_t (b_t*k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t*v_t)^T   (tiny sizes);
+  * a hand-worked example (tests/golden/tiny_d2_t3.json);
+  * the two reductions the pages state (README "Strict Generalization" bullet,
+    arXiv abstract): KDA when b_t = w_t = beta_t * 1, Gated DeltaNet when the
+    decay is also a scalar;
+  * closed forms: b = 0 gives gated linear attention, plus alpha = 1 plain
+    causal linear attention; w = 0 with S0 = 0 gives zero;
+  * the delta rule's exact retrieval (abstract: "subtract the current read
+    before writing"): with b = 1, ||k_t|| = 1 and q_t = k_t, o_t = w_t*v_t;
+  * structure: linearity in (v, S0), causality, head/batch/column independence;
+  * the fp64 chunkwise restatement (oracle.chunkwise) equals the token oracle at
+    chunk sizes 16/32/64 and ragged lengths, forward and backward;
+  * fp64 central finite differences of L = <dout, o> + <dST, S_T> for every
+    gradient, also through the KDA reduction;
+  * T decode steps equal the forward over the same T tokens.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from conftest import rel_l2
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rand_inputs(seed, B, T, H, Dk, Dv, S0=True, unit_keys=True):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, H, Dk))
+    k = rng.standard_normal((B, T, H, Dk))
+    if unit_keys:
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, H, Dv))
+    la = -np.logaddexp(0, rng.standard_normal((B, T, H, Dk))) / 4.0
+    b = 1 / (1 + np.exp(-rng.standard_normal((B, T, H, Dk))))
+    w = 1 / (1 + np.exp(-rng.standard_normal((B, T, H, Dv))))
+    s0 = 0.3 * rng.standard_normal((B, H, Dk, Dv)) if S0 else None
+    return dict(q=q, k=k, v=v, log_alpha=la, b=b, w=w), s0
+
+
+# ---------------------------------------------------------------- brute force
+
+def brute_force(q, k, v, la, b, w, S0):
+    """Dense unrolling of the product form with explicit d_k x d_k matrices.
+
+    M_t = (I - k_t e_t^T) Diag(alpha_t), e_t = b_t*k_t, u_t = w_t*v_t;
+    S_t = M_t...M_1 S0 + sum_{s<=t} M_t...M_{s+1} k_s u_s^T;  o_t = S_t^T q_t.
+    """
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    o = np.zeros((B, T, H, Dv))
+    ST = np.zeros((B, H, Dk, Dv))
+    I = np.eye(Dk)
+    for bb in range(B):
+        for hh in range(H):
+            M = [(I - np.outer(k[bb, t, hh], b[bb, t, hh] * k[bb, t, hh])) @ np.diag(np.exp(la[bb, t, hh]))
+                 for t in range(T)]
+            for t in range(T):
+                Phi = I.copy()                       # M_t ... M_1
+                for s in range(t, -1, -1):
+                    Phi = Phi @ M[s]
+                St = Phi @ S0[bb, hh]
+                for s in range(t + 1):
+                    Ps = I.copy()                    # M_t ... M_{s+1}
+                    for r in range(t, s, -1):
+                        Ps = Ps @ M[r]
+                    St = St + Ps @ np.outer(k[bb, s, hh], w[bb, s, hh] * v[bb, s, hh])
+                o[bb, t, hh] = St.T @ q[bb, t, hh]
+                if t == T - 1:
+                    ST[bb, hh] = St
+    return o, ST
+
+
+@pytest.mark.parametrize("Dk,Dv,T", [(4, 4, 12), (4, 3, 9), (3, 5, 7)])
+def test_bruteforce_dense_unroll(oracle_mod, Dk, Dv, T):
+    x, S0 = rand_inputs(1, 2, T, 2, Dk, Dv, unit_keys=False)
+    o_ref, ST_ref = brute_force(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], S0)
+    o, ST = oracle_mod.fwd(**x, S0=S0)
+    assert np.max(np.abs(o - o_ref)) <= 1e-12 * max(1.0, np.max(np.abs(o_ref)))
+    assert np.max(np.abs(ST - ST_ref)) <= 1e-12 * max(1.0, np.max(np.abs(ST_ref)))
+
+
+def test_golden_hand_worked(oracle_mod):
+    with open(os.path.join(GOLDEN, "tiny_d2_t3.json")) as f:
+        g = json.load(f)
+    arr = {n: np.array(g["inputs"][n], dtype=np.float64)[None, :, None, :]
+           for n in ("q", "k", "v", "b", "w")}
+    arr["log_alpha"] = np.log(np.array(g["inputs"]["alpha"], dtype=np.float64))[None, :, None, :]
+    o, ST = oracle_mod.fwd(**arr)
+    np.testing.assert_allclose(o[0, :, 0, :], np.array(g["expected"]["o"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(ST[0, 0], np.array(g["expected"]["S_T"]), rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- reductions
+
+def kda_reference(q, k, v, la, beta, S0):
+    """KDA: S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T, o_t = S_t^T q_t."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    o = np.zeros((B, T, H, Dv))
+    S = S0.copy()
+    for t in range(T):
+        for bb in range(B):
+            for hh in range(H):
+                kt = k[bb, t, hh]
+                bt = beta[bb, t, hh]
+                S[bb, hh] = (np.eye(Dk) - bt * np.outer(kt, kt)) @ (np.exp(la[bb, t, hh])[:, None] * S[bb, hh]) \
+                    + bt * np.outer(kt, v[bb, t, hh])
+                o[bb, t, hh] = S[bb, hh].T @ q[bb, t, hh]
+    return o, S
+
+
+def gdn_reference(q, k, v, log_a, beta, S0T):
+    """Gated DeltaNet in its published transposed form, state d_v x d_k:
+    S_t = a_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t."""
+    B, T, H, Dk = q.shape
+    o = np.zeros((B, T, H, v.shape[-1]))
+    S = S0T.copy()
+    for t in range(T):
+        for bb in range(B):
+            for hh in range(H):
+                kt = k[bb, t, hh]
+                bt = beta[bb, t, hh]
+                S[bb, hh] = np.exp(log_a[bb, t, hh]) * S[bb, hh] @ (np.eye(Dk) - bt * np.outer(kt, kt)) \
+                    + bt * np.outer(v[bb, t, hh], kt)
+                o[bb, t, hh] = S[bb, hh] @ q[bb, t, hh]
+    return o, S
+
+
+def test_reduces_to_kda(oracle_mod):
+    x, S0 = rand_inputs(2, 2, 17, 3, 6, 5)
+    beta = np.random.default_rng(3).uniform(0, 1, size=(2, 17, 3))
+    x["b"] = np.repeat(beta[..., None], 6, axis=-1)
+    x["w"] = np.repeat(beta[..., None], 5, axis=-1)
+    o, ST = oracle_mod.fwd(**x, S0=S0)
+    o_ref, ST_ref = kda_reference(x["q"], x["k"], x["v"], x["log_alpha"], beta, S0)
+    assert rel_l2(o, o_ref) < 1e-13 and rel_l2(ST, ST_ref) < 1e-13
+
+
+def test_reduces_to_gated_deltanet(oracle_mod):
+    x, S0 = rand_inputs(4, 1, 19, 2, 5, 7)
+    rng = np.random.default_rng(5)
+    beta = rng.uniform(0, 1, size=(1, 19, 2))
+    log_a = -rng.uniform(0, 0.5, size=(1, 19, 2))
+    x["b"] = np.repeat(beta[..., None], 5, axis=-1)
+    x["w"] = np.repeat(beta[..., None], 7, axis=-1)
+    x["log_alpha"] = np.repeat(log_a[..., None], 5, axis=-1)
+    o, ST = oracle_mod.fwd(**x, S0=S0)
+    o_ref, STT_ref = gdn_reference(x["q"], x["k"], x["v"], log_a, beta, np.swapaxes(S0, -1, -2))
+    assert rel_l2(o, o_ref) < 1e-13
+    assert rel_l2(ST, np.swapaxes(STT_ref, -1, -2)) < 1e-13
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_no_erase_is_gated_linear_attention(oracle_mod):
+    """b = 0: o_t = S0^T (g_t*q_t) + sum_{s<=t} ((g_t/g_s)*q_t . k_s) (w_s*v_s), g = cumprod(alpha)."""
+    x, S0 = rand_inputs(6, 1, 23, 2, 6, 4)
+    x["b"] = np.zeros_like(x["b"])
+    o, _ = oracle_mod.fwd(**x, S0=S0)
+    G = np.cumsum(x["log_alpha"], axis=1)
+    ref = np.zeros_like(o)
+    T = o.shape[1]
+    for t in range(T):
+        ref[:, t] = np.einsum("bhkv,bhk->bhv", S0, np.exp(G[:, t]) * x["q"][:, t])
+        for s in range(t + 1):
+            coef = np.sum(np.exp(G[:, t] - G[:, s]) * x["q"][:, t] * x["k"][:, s], axis=-1)
+            ref[:, t] += coef[..., None] * x["w"][:, s] * x["v"][:, s]
+    assert rel_l2(o, ref) < 1e-13
+
+
+def test_no_erase_no_decay_is_linear_attention(oracle_mod):
+    x, _ = rand_inputs(7, 1, 15, 1, 4, 4, S0=False)
+    x["b"] = np.zeros_like(x["b"])
+    x["log_alpha"] = np.zeros_like(x["log_alpha"])
+    x["w"] = np.ones_like(x["w"])
+    o, _ = oracle_mod.fwd(**x)
+    q, k, v = x["q"][0, :, 0], x["k"][0, :, 0], x["v"][0, :, 0]
+    scores = np.tril(q @ k.T)
+    assert rel_l2(o[0, :, 0], scores @ v) < 1e-13
+
+
+def test_zero_write_zero_state(oracle_mod):
+    x, _ = rand_inputs(8, 2, 11, 2, 5, 5, S0=False)
+    x["w"] = np.zeros_like(x["w"])
+    o, ST = oracle_mod.fwd(**x)
+    assert np.all(o == 0) and np.all(ST == 0)
+
+
+def test_exact_retrieval(oracle_mod):
+    """b = 1, unit k_t, q_t = k_t: the read after the update returns exactly w_t*v_t."""
+    x, S0 = rand_inputs(9, 2, 21, 2, 8, 6)
+    x["b"] = np.ones_like(x["b"])
+    x["q"] = x["k"].copy()
+    o, _ = oracle_mod.fwd(**x, S0=S0)
+    np.testing.assert_allclose(o, x["w"] * x["v"], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- structure
+
+def test_linear_in_values_and_state(oracle_mod):
+    x, S0 = rand_inputs(10, 1, 13, 2, 5, 4)
+    y, S1 = rand_inputs(11, 1, 13, 2, 5, 4)
+    c = 0.7
+    o1, T1 = oracle_mod.fwd(**x, S0=S0)
+    x2 = dict(x, v=y["v"])
+    o2, T2 = oracle_mod.fwd(**x2, S0=S1)
+    x3 = dict(x, v=x["v"] + c * y["v"])
+    o3, T3 = oracle_mod.fwd(**x3, S0=S0 + c * S1)
+    assert rel_l2(o3, o1 + c * o2) < 1e-13 and rel_l2(T3, T1 + c * T2) < 1e-13
+
+
+def test_causal(oracle_mod):
+    x, S0 = rand_inputs(12, 1, 16, 2, 5, 4)
+    o, _ = oracle_mod.fwd(**x, S0=S0)
+    y = {n: a.copy() for n, a in x.items()}
+    rng = np.random.default_rng(13)
+    for n in y:
+        y[n][:, 9:] = rng.uniform(0.1, 0.9, size=y[n][:, 9:].shape)
+    o2, _ = oracle_mod.fwd(**y, S0=S0)
+    assert np.array_equal(o[:, :9], o2[:, :9])
+    assert not np.allclose(o[:, 9:], o2[:, 9:])
+
+
+def test_heads_batches_columns_independent(oracle_mod):
+    x, S0 = rand_inputs(14, 3, 10, 4, 5, 6)
+    o, ST = oracle_mod.fwd(**x, S0=S0)
+    pb, ph = [2, 0, 1], [3, 1, 0, 2]
+    xp = {n: a[pb][:, :, ph] for n, a in x.items()}
+    op, STp = oracle_mod.fwd(**xp, S0=S0[pb][:, ph])
+    assert np.array_equal(op, o[pb][:, :, ph]) and np.array_equal(STp, ST[pb][:, ph])
+    cols = [4, 1]
+    xc = dict(x, v=x["v"][..., cols], w=x["w"][..., cols])
+    oc, STc = oracle_mod.fwd(**xc, S0=np.ascontiguousarray(S0[..., cols]))
+    assert np.array_equal(oc, o[..., cols]) and np.array_equal(STc, ST[..., cols])
+
+
+# ---------------------------------------------------------------- chunk algebra
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("T", [1, 37, 64, 150])
+def test_chunkwise_forward_equals_token(oracle_mod, chunk, T):
+    from oracle import chunkwise
+    x, S0 = rand_inputs(20 + T, 2, T, 2, 16, 12)
+    o, ST = oracle_mod.fwd(**x, S0=S0)
+    oc, STc = chunkwise.fwd(**x, S0=S0, chunk=chunk)
+    assert rel_l2(oc, o) < 1e-10 and rel_l2(STc, ST) < 1e-10
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("T", [5, 70, 128])
+def test_chunkwise_backward_equals_token(oracle_mod, chunk, T):
+    from oracle import chunkwise
+    x, S0 = rand_inputs(40 + T, 1, T, 2, 16, 12)
+    rng = np.random.default_rng(T)
+    dout = rng.standard_normal(x["v"].shape)
+    dST = rng.standard_normal(S0.shape)
+    g = oracle_mod.bwd(**x, dout=dout, S0=S0, dST=dST)
+    gc = chunkwise.bwd(**x, dout=dout, S0=S0, dST=dST, chunk=chunk)
+    for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "dS0"):
+        assert rel_l2(gc[n], g[n]) < 1e-9, n
+
+
+# ---------------------------------------------------------------- gradients
+
+def _loss(oracle_mod, x, S0, dout, dST):
+    o, ST = oracle_mod.fwd(**x, S0=S0)
+    return float(np.sum(o * dout) + np.sum(ST * dST))
+
+
+def test_finite_differences_all_gradients(oracle_mod):
+    x, S0 = rand_inputs(50, 1, 20, 1, 8, 6)
+    rng = np.random.default_rng(51)
+    dout = rng.standard_normal(x["v"].shape)
+    dST = rng.standard_normal(S0.shape)
+    g = oracle_mod.bwd(**x, dout=dout, S0=S0, dST=dST)
+    h = 1e-6
+    names = {"q": "dq", "k": "dk", "v": "dv", "log_alpha": "dlog_alpha", "b": "db", "w": "dw"}
+    for name, gname in names.items():
+        fd = np.zeros_like(x[name])
+        for idx in np.ndindex(x[name].shape):
+            xp = {n: a.copy() for n, a in x.items()}
+            xm = {n: a.copy() for n, a in x.items()}
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            fd[idx] = (_loss(oracle_mod, xp, S0, dout, dST) - _loss(oracle_mod, xm, S0, dout, dST)) / (2 * h)
+        assert rel_l2(g[gname], fd) < 1e-6, gname
+    fd = np.zeros_like(S0)
+    for idx in np.ndindex(S0.shape):
+        Sp, Sm = S0.copy(), S0.copy()
+        Sp[idx] += h
+        Sm[idx] -= h
+        fd[idx] = (_loss(oracle_mod, x, Sp, dout, dST) - _loss(oracle_mod, x, Sm, dout, dST)) / (2 * h)
+    assert rel_l2(g["dS0"], fd) < 1e-6
+
+
+def test_gradient_through_kda_reduction(oracle_mod):
+    """With b = w = beta*1, dL/dbeta_t = sum_i db_t,i + sum_j dw_t,j must match
+    finite differences of the separately written KDA recurrence."""
+    x, S0 = rand_inputs(60, 1, 9, 1, 5, 4)
+    beta = np.random.default_rng(61).uniform(0.1, 0.9, size=(1, 9, 1))
+    x["b"] = np.repeat(beta[..., None], 5, axis=-1)
+    x["w"] = np.repeat(beta[..., None], 4, axis=-1)
+    rng = np.random.default_rng(62)
+    dout = rng.standard_normal(x["v"].shape)
+    g = oracle_mod.bwd(**x, dout=dout, S0=S0)
+    dbeta = g["db"].sum(-1) + g["dw"].sum(-1)
+    h = 1e-6
+    fd = np.zeros_like(beta)
+    for idx in np.ndindex(beta.shape):
+        bp, bm = beta.copy(), beta.copy()
+        bp[idx] += h
+        bm[idx] -= h
+        op, _ = kda_reference(x["q"], x["k"], x["v"], x["log_alpha"], bp, S0)
+        om, _ = kda_reference(x["q"], x["k"], x["v"], x["log_alpha"], bm, S0)
+        fd[idx] = (np.sum(op * dout) - np.sum(om * dout)) / (2 * h)
+    assert rel_l2(dbeta, fd) < 1e-6
+
+
+# ---------------------------------------------------------------- decode
+
+def test_decode_steps_equal_forward(oracle_mod):
+    x, S0 = rand_inputs(70, 2, 14, 3, 6, 5)
+    o, ST = oracle_mod.fwd(**x, S0=S0)
+    S = S0.copy()
+    for t in range(14):
+        ot, S = oracle_mod.decode(*(x[n][:, t] for n in ("q", "k", "v", "log_alpha", "b", "w")), S)
+        assert np.array_equal(ot, o[:, t])
+    assert np.array_equal(S, ST)
