@@ -1,0 +1,320 @@
+"""Throughput benchmark of the Gated Delta Rule-2 operator (forward + gate-aware backward).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = gdn2_fwd (keeping the chunk-start states) + gdn2_bwd on one batch of
+the 1.3B training-layer shape: B=4, H=16, T=4096, d_k=d_v=128, bf16 inputs,
+fp32 state, chunk 64, synthetic seeded inputs resident in HBM. For N > 1 (one
+process per GPU under torchrun) every rank runs its own batch: heads and batch
+entries never interact, so there is no data-path collective (weak scaling).
+Rank 0 prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN-2 fwd+bwd tokens/s (H16 d128 T4K bf16, 1×B200); % of roofline"
+WORKLOAD = "fwdbwd-bf16-b4h16t4096d128"
+
+# Algorithmic work per token and head (C = 64, d = 128): forward reads q, k, v,
+# log_alpha, b, w and writes o (7 x 256 B); the backward re-reads the six inputs,
+# reads dout and writes six gradients (13 x 256 B). Flops: forward 180,224
+# (the chunk contractions), backward counted as twice the forward.
+BYTES_PER_TOKEN_HEAD = {"fwd": 1792, "bwd": 3328}
+FLOPS_PER_TOKEN_HEAD = {"fwd": 180224, "bwd": 2 * 180224}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index, path):
+        self.path, self.index, self.proc = path, index, None
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def make_host_inputs(rank):
+    from linear_attention_delta_gdn_b200.inputs import WORKLOADS, make_inputs
+    wl = WORKLOADS[WORKLOAD]
+    return wl, make_inputs(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, wl.seed + 7919 * rank, wl.dtype, with_do=True)
+
+
+def cpu_baseline(wl, x, budget_s=20.0, steps=1):
+    """Time the fp64 oracle (fwd + bwd) on a bounded sample of the workload."""
+    import oracle
+    from linear_attention_delta_gdn_b200.inputs import to_f64
+    cores = oracle.threads()
+    nheads = max(1, min(wl.B * wl.H, 2 * cores))
+    T = wl.T
+    # pick nheads (b, h) sequences, first T tokens
+    heads = [(i // wl.H, i % wl.H) for i in range(nheads)]
+    g = {n: to_f64(t) for n, t in x.items()}
+    sub = {n: np.stack([g[n][b, :T, h] for b, h in heads])[:, :, None] for n in g}
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    # shrink the sample until one step fits the budget (estimate from a short probe)
+    t0 = time.perf_counter()
+    probe_T = min(T, 256)
+    probe = {n: np.ascontiguousarray(a[:, :probe_T]) for n, a in sub.items()}
+    oracle.fwd(*(probe[n] for n in names))
+    oracle.bwd(*(probe[n] for n in names), dout=probe["dout"])
+    est = (time.perf_counter() - t0) * T / probe_T
+    if est > budget_s:
+        T = max(probe_T, int(T * budget_s / est) // 64 * 64)
+        sub = {n: np.ascontiguousarray(a[:, :T]) for n, a in sub.items()}
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.fwd(*(sub[n] for n in names))
+        oracle.bwd(*(sub[n] for n in names), dout=sub["dout"])
+        times.append(time.perf_counter() - t0)
+    dt = statistics.median(times)
+    tokens = nheads * T / wl.H            # token = one position of the 16-head layer
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "fp64 oracle fwd+bwd on %d of %d (batch, head) sequences x %d tokens; tokens = "
+                      "sequences x tokens / %d heads" % (nheads, wl.B * wl.H, T, wl.H),
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl, x = make_host_inputs(0)
+    budget = float(os.environ.get("GDN2_REF_BUDGET_S", "8"))
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; warm-up steps are not repeated on the CPU
+    cb = cpu_baseline(wl, x, budget_s=budget, steps=max(1, args.steps))
+    line = {"metric": METRIC, "impl": "reference", "value": cb["value"], "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": wl.B, "T": wl.T, "H": wl.H, "Dk": wl.Dk, "Dv": wl.Dv,
+                       "chunk": wl.chunk, "global_batch": wl.B, "seq_len": wl.T, "parallelism": "host threads"},
+            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from linear_attention_delta_gdn_b200 import binding, build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    L = binding.lib()
+
+    wl, xh = make_host_inputs(rank)
+    B, T, H, Dk, Dv, chunk = wl.B, wl.T, wl.H, wl.Dk, wl.Dv, wl.chunk
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    pinned = {n: t.pin_memory() for n, t in xh.items()}
+    d = {n: t.to(dev, non_blocking=True) for n, t in pinned.items()}
+    o = torch.empty((B, T, H, Dv), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev)
+    grads = {n: torch.empty((B, T, H, Dk), dtype=torch.bfloat16, device=dev) for n in ("dq", "dk", "dlog_alpha", "db")}
+    grads.update({n: torch.empty((B, T, H, Dv), dtype=torch.bfloat16, device=dev) for n in ("dv", "dw")})
+    grads["dS0"] = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, binding.GDN2_BF16),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(inp):
+        binding.gdn2_fwd(*(inp[n] for n in names), None, chunk=chunk, save_states=True, ws=ws, o=o, ST=ST)
+        binding.gdn2_bwd(*(inp[n] for n in names), inp["dout"], None, None, chunk=chunk, states_saved=True,
+                         ws=ws, grads=grads)
+
+    for _ in range(max(3, args.warmup)):
+        step(d)
+    torch.cuda.synchronize(dev)
+
+    # ---- device-timed region: inputs resident in HBM (470 MB per step, larger than L2)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clock_log = os.path.join(ROOT, "gpurun_out", "bench_clocks_rank%d.csv" % rank)
+    os.makedirs(os.path.dirname(clock_log), exist_ok=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local, clock_log) as clocks:
+        time.sleep(0.3)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            binding.gdn2_fwd(*(d[n] for n in names), None, chunk=chunk, save_states=True, ws=ws, o=o, ST=ST)
+            e1.record(stream)
+            binding.gdn2_bwd(*(d[n] for n in names), d["dout"], None, None, chunk=chunk, states_saved=True,
+                             ws=ws, grads=grads)
+            e2.record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    bwd_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in ev)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = t.item()
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = B * T
+    value = world * tokens_per_step / (ms_per_step / 1e3)
+
+    # ---- end to end through host buffers: H2D inputs, fwd + bwd, D2H o and gradients
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    outs = [o] + [grads[n] for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw")]
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e_start.record(stream)
+    for _ in range(args.e2e_steps):
+        for n in pinned:
+            d[n].copy_(pinned[n], non_blocking=True)
+        step(d)
+        for h_, t in zip(host_out, outs):
+            h_.copy_(t, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e_start.elapsed_time(e_end) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e_value = world * tokens_per_step / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant call
+    pk = peaks()
+    th = B * T * H
+    calls = {"fwd": fwd_ms, "bwd": bwd_ms}
+    dom = max(calls, key=calls.get)
+    alg_bytes = th * BYTES_PER_TOKEN_HEAD[dom] + (B * H * Dk * Dv * 4 if dom == "bwd" else B * H * Dk * Dv * 4)
+    achieved = alg_bytes / (calls[dom] / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "gdn2_%s" % dom, "achieved": achieved, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "peak_source": pk["source"], "alg_bytes_per_launch": alg_bytes,
+                "call_ms": {"fwd": fwd_ms, "bwd": bwd_ms},
+                "step_frac": (th * sum(BYTES_PER_TOKEN_HEAD.values()) + 2 * B * H * Dk * Dv * 4)
+                / (ms_per_step / 1e3) / 1e9 / pk["hbm_gbs"]}
+
+    tc = binding.gdn2_workspace_size(binding.GDN2_OP_FWD_SAVE, B, T, H, Dk, Dv, chunk, binding.GDN2_BF16) \
+        < B * H * ((T + chunk - 1) // chunk) * Dk * Dv * 4
+    launches_per_step = (1 + 2) if tc else (1 + 1)
+
+    line = None
+    if rank == 0:
+        cb = None
+        if not args.no_cpu_baseline and world == 1:
+            cb = cpu_baseline(wl, xh)
+            cb = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "Dk": Dk, "Dv": Dv, "chunk": chunk,
+                           "global_batch": world * B, "seq_len": T,
+                           "parallelism": "dp%d (independent batches, no collective)" % world,
+                           "l2": "inputs larger than L2 (%.0f MB read per step)" % (h2d / 1e6),
+                           "path": "tensor-core chunkwise" if tc else "fp32 recurrent"},
+                "roofline": roofline, "cpu_baseline": cb, "clocks": clocks.summary(),
+                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches_per_step * args.steps}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,146 @@
+/*
+ * gdn2.h -- C ABI of libgdn2.so: the Gated Delta Rule-2 sequence-mixing
+ * operator of Gated DeltaNet-2 on NVIDIA B200 (sm_100a).
+ *
+ * The operator ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
+ * Attention"; GitHub README method bullets and arXiv abstract 2605.22791): per
+ * batch element and head, a d_k x d_v state S evolves with a channel-wise decay
+ * alpha_t, a channel-wise erase gate b_t in [0,1]^{d_k} acting on the key side
+ * of the decayed state and a channel-wise write gate w_t in [0,1]^{d_v} acting
+ * on the value side of the new content:
+ *
+ *     S_t = (I - k_t (b_t*k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t*v_t)^T
+ *     o_t = S_t^T q_t
+ *
+ * ('*' is the elementwise product; alpha_t = exp(log_alpha_t)). The README's
+ * "Hardware-efficient Training" bullet and the abstract name the method of
+ * computation: a chunkwise WY algorithm with the channel-wise decay absorbed
+ * into asymmetric erase factors, and a gate-aware backward.
+ *
+ * Conventions for every call below
+ *   - Pointers are DEVICE pointers to contiguous row-major tensors, unless a
+ *     comment says otherwise. Token tensors are [B, T, H, D]; single-token
+ *     (decode) tensors are [B, H, D]; states are [B, H, Dk, Dv] float32 with
+ *     rows indexing keys and columns indexing values.
+ *   - dt is the element type of q, k, v, log_alpha, b, w, o, dout and of the
+ *     token gradients dq, dk, dv, dlog_alpha, db, dw. States and their
+ *     gradients are always float32.
+ *   - stream is a cudaStream_t (NULL: the legacy default stream). All work is
+ *     enqueued on it; no call synchronises the host or allocates memory.
+ *   - The caller owns every buffer, including the workspace.
+ *   - Arguments are checked on the host before anything is launched. On an
+ *     error status nothing has been launched and no output was touched, except
+ *     GDN2_ERR_CUDA, which reports a launch failure or an earlier asynchronous
+ *     error of the device (outputs are then undefined).
+ *   - Gate values are not range-checked (that would cost a pass over HBM).
+ *   - Supported sizes: Dk, Dv in {16, 32, 64, 128}; chunk in {16, 32, 64};
+ *     any T >= 0 (a ragged last chunk is allowed); B, H >= 1.
+ *     The tensor-core path runs for dt = GDN2_BF16, Dk = Dv = 128, chunk = 64;
+ *     every other supported combination runs on the fp32 recurrent kernels.
+ *   - Thread safety: calls may be made from several host threads; error
+ *     detail strings are per thread.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn2_status {
+    GDN2_OK = 0,
+    GDN2_ERR_INVALID = 1,     /* null pointer, bad size or option; nothing launched */
+    GDN2_ERR_UNSUPPORTED = 2, /* valid but not built for this shape/dtype; nothing launched */
+    GDN2_ERR_WORKSPACE = 3,   /* workspace missing or too small; nothing launched */
+    GDN2_ERR_CUDA = 4,        /* CUDA runtime error (see gdn2_last_error) */
+    GDN2_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (reserved) */
+} gdn2_status;
+
+typedef enum gdn2_dtype {
+    GDN2_F32 = 0,
+    GDN2_BF16 = 1
+} gdn2_dtype;
+
+typedef enum gdn2_op {
+    GDN2_OP_FWD = 0,      /* gdn2_fwd with save_states = 0 */
+    GDN2_OP_FWD_SAVE = 1, /* gdn2_fwd with save_states = 1 */
+    GDN2_OP_BWD = 2       /* gdn2_bwd (either value of states_saved) */
+} gdn2_op;
+
+/*
+ * Bytes of device workspace that gdn2_fwd / gdn2_bwd need for one problem.
+ * The workspace of GDN2_OP_BWD starts with the region that GDN2_OP_FWD_SAVE
+ * fills, so one buffer of gdn2_workspace_size(GDN2_OP_BWD, ...) bytes serves a
+ * gdn2_fwd(save_states = 1) followed by a gdn2_bwd(states_saved = 1).
+ * Returns 0 for an invalid or unsupported problem (and for GDN2_OP_FWD, which
+ * needs none). The workspace must be 256-byte aligned.
+ */
+size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk,
+                           gdn2_dtype dt);
+
+/*
+ * Forward over whole sequences.
+ *   q, k, log_alpha, b : [B, T, H, Dk] dt      (query, key, log-decay, erase gate)
+ *   v, w               : [B, T, H, Dv] dt      (value, write gate)
+ *   S0                 : [B, H, Dk, Dv] float32, or NULL for a zero initial state
+ *   o                  : [B, T, H, Dv] dt       output, o_t = S_t^T q_t
+ *   ST                 : [B, H, Dk, Dv] float32 final state, or NULL
+ *   chunk              : chunk length of the WY algorithm (16, 32 or 64)
+ *   save_states        : nonzero -> keep the chunk-start states in ws for a
+ *                        later gdn2_bwd(states_saved = 1) on the same inputs
+ *   ws, ws_bytes       : workspace of >= gdn2_workspace_size(GDN2_OP_FWD[_SAVE])
+ *                        bytes (may be NULL when that size is 0)
+ * S0 and ST may alias (the state is updated in place).
+ */
+gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
+                     const void* b, const void* w, const float* S0, void* o, float* ST,
+                     int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt,
+                     int save_states, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Gate-aware backward of gdn2_fwd for the loss L = <dout, o> + <dST, S_T>.
+ *   q .. w, S0         : the forward's inputs (S0 may be NULL: zeros)
+ *   dout               : [B, T, H, Dv] dt, gradient of o
+ *   dST                : [B, H, Dk, Dv] float32 gradient of S_T, or NULL (zero)
+ *   dq, dk, dlog_alpha, db : [B, T, H, Dk] dt   (outputs)
+ *   dv, dw             : [B, T, H, Dv] dt       (outputs)
+ *   dS0                : [B, H, Dk, Dv] float32 gradient of S0, or NULL
+ *   states_saved       : nonzero -> ws holds the chunk-start states written by
+ *                        gdn2_fwd(save_states = 1) with the same inputs, S0,
+ *                        sizes and chunk; zero -> they are recomputed here
+ *   ws, ws_bytes       : >= gdn2_workspace_size(GDN2_OP_BWD, ...) bytes
+ * All six token gradients must be given; they must not alias the inputs.
+ */
+gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* log_alpha,
+                     const void* b, const void* w, const float* S0, const void* dout,
+                     const float* dST, void* dq, void* dk, void* dv, void* dlog_alpha, void* db,
+                     void* dw, float* dS0, int B, int T, int H, int Dk, int Dv, int chunk,
+                     gdn2_dtype dt, int states_saved, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One recurrent decode step for every (b, h), state updated in place -- the
+ * constant-memory decoding of the arXiv abstract.
+ *   q, k, log_alpha, b : [B, H, Dk] dt ;  v, w : [B, H, Dv] dt
+ *   S                  : [B, H, Dk, Dv] float32, read and overwritten with S_t
+ *   o                  : [B, H, Dv] dt, o = S_t^T q
+ */
+gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
+                             const void* b, const void* w, float* S, void* o, int B, int H,
+                             int Dk, int Dv, gdn2_dtype dt, void* stream);
+
+/* Static description of a status code. */
+const char* gdn2_status_string(gdn2_status s);
+
+/* Detail of the last non-OK status returned on the calling host thread. */
+const char* gdn2_last_error(void);
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+int gdn2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H */

@@ -1,0 +1,207 @@
+"""ctypes binding of libgdn2.so (the C ABI declared in include/gdn2.h).
+
+Argument marshalling only: every step of the operator runs in the library's
+CUDA kernels. torch supplies device memory (outputs and the workspace are
+allocated as torch tensors) and the current CUDA stream. There is no CPU or
+library fallback: if ``libgdn2.so`` is missing or a tensor is not on a CUDA
+device, these functions raise.
+
+Names mirror the C entry points: :func:`gdn2_fwd`, :func:`gdn2_bwd`,
+:func:`gdn2_decode_step`, :func:`gdn2_workspace_size`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn2.so")
+_lib = None
+
+GDN2_F32, GDN2_BF16 = 0, 1
+GDN2_OP_FWD, GDN2_OP_FWD_SAVE, GDN2_OP_BWD = 0, 1, 2
+STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_WORKSPACE",
+          4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT"}
+
+#: exported symbols, as declared in include/gdn2.h
+EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "gdn2_status_string",
+           "gdn2_last_error", "gdn2_version")
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, fn, status, detail):
+        super().__init__("%s -> %s: %s" % (fn, STATUS.get(status, status), detail))
+        self.status = status
+
+
+def lib(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libgdn2.so (built by ``python -m linear_attention_delta_gdn_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise FileNotFoundError("%s is missing: build it with `python -m linear_attention_delta_gdn_b200.build`" % p)
+    L = ctypes.CDLL(p)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.gdn2_workspace_size.argtypes = [I] * 8
+    L.gdn2_workspace_size.restype = Z
+    L.gdn2_fwd.argtypes = [P] * 9 + [I] * 8 + [P, Z, P]
+    L.gdn2_fwd.restype = I
+    L.gdn2_bwd.argtypes = [P] * 16 + [I] * 8 + [P, Z, P]
+    L.gdn2_bwd.restype = I
+    L.gdn2_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
+    L.gdn2_decode_step.restype = I
+    L.gdn2_status_string.argtypes = [I]
+    L.gdn2_status_string.restype = ctypes.c_char_p
+    L.gdn2_last_error.argtypes = []
+    L.gdn2_last_error.restype = ctypes.c_char_p
+    L.gdn2_version.argtypes = []
+    L.gdn2_version.restype = I
+    if path is None:
+        _lib = L
+    return L
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise Gdn2Error(fn, rc, lib().gdn2_last_error().decode(errors="replace"))
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN2_BF16
+    if t.dtype == torch.float32:
+        return GDN2_F32
+    raise TypeError("dtype %s is not supported (float32 or bfloat16)" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _state(t, like, B, H, Dk, Dv):
+    if t is None:
+        return None
+    if t.dtype != torch.float32 or tuple(t.shape) != (B, H, Dk, Dv):
+        raise ValueError("states must be float32 [B, H, Dk, Dv] = %s" % ((B, H, Dk, Dv),))
+    return t
+
+
+def gdn2_workspace_size(op: int, B: int, T: int, H: int, Dk: int, Dv: int, chunk: int, dt: int) -> int:
+    return int(lib().gdn2_workspace_size(op, B, T, H, Dk, Dv, chunk, dt))
+
+
+def gdn2_fwd(q, k, v, log_alpha, b, w, S0=None, chunk: int = 64, want_state: bool = True,
+             save_states: bool = False, ws: Optional[torch.Tensor] = None, o=None, ST=None):
+    """Forward. Tensors [B, T, H, D] (bf16 or fp32), S0 [B, H, Dk, Dv] fp32 or None.
+
+    Returns ``(o, ST)`` (``ST`` is None unless ``want_state``). With
+    ``save_states`` the chunk-start states are kept in ``ws`` (a uint8 CUDA tensor
+    of at least ``gdn2_workspace_size(GDN2_OP_FWD_SAVE, ...)`` bytes; allocated
+    if not given) for a later :func:`gdn2_bwd` with ``states_saved=True``.
+    """
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for name, t, D in (("k", k, Dk), ("v", v, Dv), ("log_alpha", log_alpha, Dk), ("b", b, Dk), ("w", w, Dv)):
+        if t.dtype != q.dtype or tuple(t.shape) != (B, T, H, D):
+            raise ValueError("%s must be %s [%d, %d, %d, %d]" % (name, q.dtype, B, T, H, D))
+    _state(S0, q, B, H, Dk, Dv)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
+    if ST is None and want_state:
+        ST = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    ws_bytes = 0
+    if save_states:
+        need = gdn2_workspace_size(GDN2_OP_FWD_SAVE, B, T, H, Dk, Dv, chunk, dt)
+        if ws is None:
+            ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+        ws_bytes = ws.numel()
+    rc = lib().gdn2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                        _ptr(ST), B, T, H, Dk, Dv, chunk, dt, int(save_states), _ptr(ws), ws_bytes,
+                        _stream(q.device))
+    _check("gdn2_fwd", rc)
+    return o, ST
+
+
+def gdn2_bwd(q, k, v, log_alpha, b, w, dout, S0=None, dST=None, chunk: int = 64, want_dS0: bool = True,
+             states_saved: bool = False, ws: Optional[torch.Tensor] = None, grads=None):
+    """Gate-aware backward for L = <dout, o> + <dST, S_T>.
+
+    Returns a dict with dq, dk, dv, dlog_alpha, db, dw (input dtype) and dS0 (fp32 or None).
+    """
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    _state(S0, q, B, H, Dk, Dv)
+    _state(dST, q, B, H, Dk, Dv)
+    if tuple(dout.shape) != (B, T, H, Dv) or dout.dtype != q.dtype:
+        raise ValueError("dout must be %s [%d, %d, %d, %d]" % (q.dtype, B, T, H, Dv))
+    if grads is None:
+        grads = {n: torch.empty_like(q) for n in ("dq", "dk", "dlog_alpha", "db")}
+        grads.update({n: torch.empty_like(v) for n in ("dv", "dw")})
+        grads["dS0"] = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device) if want_dS0 else None
+    need = gdn2_workspace_size(GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    g = grads
+    rc = lib().gdn2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(dout),
+                        _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]),
+                        _ptr(g["db"]), _ptr(g["dw"]), _ptr(g.get("dS0")), B, T, H, Dk, Dv, chunk, dt,
+                        int(states_saved), _ptr(ws), ws.numel(), _stream(q.device))
+    _check("gdn2_bwd", rc)
+    return grads
+
+
+def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None):
+    """One decode step: inputs [B, H, D]; S [B, H, Dk, Dv] fp32 is updated in place. Returns o."""
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _state(S, q, B, H, Dk, Dv)
+    if o is None:
+        o = torch.empty((B, H, Dv), dtype=q.dtype, device=q.device)
+    rc = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
+                                B, H, Dk, Dv, _dt(q), _stream(q.device))
+    _check("gdn2_decode_step", rc)
+    return o
+
+
+class GatedDeltaRule2(torch.autograd.Function):
+    """autograd wrapper: forward keeps the chunk-start states for the backward."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, log_alpha, b, w, S0, chunk):
+        B, T, H, Dk = q.shape
+        Dv = v.shape[-1]
+        need = gdn2_workspace_size(GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, _dt(q))
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+        o, ST = gdn2_fwd(q, k, v, log_alpha, b, w, S0, chunk=chunk, save_states=True, ws=ws)
+        ctx.save_for_backward(q, k, v, log_alpha, b, w, S0, ws)
+        ctx.chunk = chunk
+        return o, ST
+
+    @staticmethod
+    def backward(ctx, do, dST):
+        q, k, v, log_alpha, b, w, S0, ws = ctx.saved_tensors
+        g = gdn2_bwd(q, k, v, log_alpha, b, w, do.contiguous(), S0,
+                     None if dST is None else dST.contiguous(), chunk=ctx.chunk,
+                     want_dS0=S0 is not None, states_saved=True, ws=ws)
+        return g["dq"], g["dk"], g["dv"], g["dlog_alpha"], g["db"], g["dw"], g["dS0"], None
+
+
+def gated_delta_rule2(q, k, v, log_alpha, b, w, S0=None, chunk: int = 64):
+    """Differentiable Gated Delta Rule-2 operator. Returns ``(o, S_T)``."""
+    return GatedDeltaRule2.apply(q, k, v, log_alpha, b, w, S0, chunk)

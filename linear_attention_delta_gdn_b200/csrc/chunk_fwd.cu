@@ -1,0 +1,369 @@
+// chunk_fwd.cu -- chunkwise WY forward of the Gated Delta Rule-2 operator on
+// tcgen05 tensor cores (bf16 operands, fp32 TMEM accumulators, fp32 state).
+//
+// One CTA (128 threads) per (batch, head) walks the chunks in order; the state
+// is carried across chunks in TMEM as S^T (lane j = value channel, column i =
+// key channel) in fp32, with a bf16 copy in shared memory as the UMMA operand.
+// Per chunk ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
+// Attention", arXiv abstract: chunkwise WY algorithm, decay absorbed into
+// asymmetric erase factors):
+//   TMA      q, k, v, log_alpha, b, w tiles (64 tokens x 128, bf16, 128B swizzle)
+//   prep     Et = g*b*k, Qt = g*q, Kt = k/g, Kh = gC*Kt, U = w*v       (g = exp(cumsum log_alpha))
+//   M1       [A; P] = [Et; Qt] Kt^T                                     (M=128, N=64, K=128)
+//   solve    T = (I + strict_lower(A))^{-1}                            (fp32, 16x16 blocks)
+//   M2, M3   Wm^T = Et^T T^T ,  Delta^T := U^T T^T                      (M=128, N=64, K=64)
+//   M4, M5   Delta^T -= S^T Wm^T ,  O^T = S^T Qt^T                      (M=128, N=64, K=128)
+//   M6, M7   O^T += Delta^T P^T ,   S^T <- S^T Diag(gC) + Delta^T Kh    (N=64 / N=128, K=64)
+// Optionally the chunk-start states are written (bf16 tile images) for the backward.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "chunk_common.cuh"
+#include "internal.h"
+
+namespace gdn2 {
+namespace {
+
+using namespace chunk;
+
+// shared-memory layout (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_QE = 0;           // [128 x 128] rows 0..63: b -> Et, rows 64..127: q -> Qt
+constexpr uint32_t OFF_KH = 32768;       // [64 x 128] k -> Kh
+constexpr uint32_t OFF_KT = 49152;       // [64 x 128] log_alpha -> Kt
+constexpr uint32_t OFF_UU = 65536;       // [64 x 128] v -> U
+constexpr uint32_t OFF_WW = 81920;       // [64 x 128] w -> Wm
+constexpr uint32_t OFF_ST = 98304;       // [128 x 128] S^T (bf16)
+constexpr uint32_t OFF_DT = 131072;      // [128 x 64] Delta^T (bf16)  | fp32 A scratch [64 x 68]
+constexpr uint32_t OFF_TF = 148480;      // fp32 T [64 x 68]
+constexpr uint32_t OFF_X = 165888;       // fp32 solve temporaries (768)
+constexpr uint32_t OFF_TT = 178176;      // [64 x 64] T (bf16)
+constexpr uint32_t OFF_PP = 186368;      // [64 x 64] P (bf16)
+constexpr uint32_t OFF_GC = 194560;      // fp32 gC[128]
+constexpr uint32_t OFF_BAR = 195072;     // 2 mbarriers, tmem base, abort flag
+constexpr uint32_t SMEM_BYTES = 195136 + 1024;
+
+// TMEM columns
+constexpr uint32_t TM_S = 0, TM_AP = 128, TM_W = 192, TM_D = 256, TM_O = 320, TM_COLS = 512;
+
+constexpr uint32_t LOAD_BYTES = 6 * 64 * 128 * 2;
+
+__device__ unsigned int g_fwd_error;
+
+__global__ void __launch_bounds__(NT, 1)
+chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                 const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mla,
+                 const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
+                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
+                 unsigned char* __restrict__ states, int T, int H) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* QE = sm + OFF_QE;
+    unsigned char* KH = sm + OFF_KH;
+    unsigned char* KT = sm + OFF_KT;
+    unsigned char* UU = sm + OFF_UU;
+    unsigned char* WW = sm + OFF_WW;
+    unsigned char* STt = sm + OFF_ST;
+    unsigned char* DT = sm + OFF_DT;
+    float* sA = reinterpret_cast<float*>(sm + OFF_DT);
+    float* sTf = reinterpret_cast<float*>(sm + OFF_TF);
+    float* sX = reinterpret_cast<float*>(sm + OFF_X);
+    unsigned char* TT = sm + OFF_TT;
+    unsigned char* PP = sm + OFF_PP;
+    float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_mma = bar_load + 1;
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
+    int* abort_flag = reinterpret_cast<int*>(sm + OFF_BAR + 20);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int h = blockIdx.x % H, b = blockIdx.x / H;
+    const size_t head = blockIdx.x;
+    const int nc = (T + C - 1) / C;
+    const bool want_o = (o != nullptr);
+
+    if (tid == 0) {
+        tc::mbar_init(bar_load, 1);
+        tc::mbar_init(bar_mma, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&mq); tc::tma_prefetch_desc(&mk); tc::tma_prefetch_desc(&mv);
+        tc::tma_prefetch_desc(&mla); tc::tma_prefetch_desc(&mb); tc::tma_prefetch_desc(&mw);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_base_ptr, TM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_base_ptr;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lanes
+
+    // issue the first chunk's loads
+    auto issue_loads = [&](int c) {
+        const int t0 = c * C;
+        tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
+        tma_tile(QE, 2 * C, 0, &mb, b, h, t0, bar_load);
+        tma_tile(QE, 2 * C, C, &mq, b, h, t0, bar_load);
+        tma_tile(KH, C, 0, &mk, b, h, t0, bar_load);
+        tma_tile(KT, C, 0, &mla, b, h, t0, bar_load);
+        tma_tile(UU, C, 0, &mv, b, h, t0, bar_load);
+        tma_tile(WW, C, 0, &mw, b, h, t0, bar_load);
+    };
+    if (tid == 0 && nc > 0) issue_loads(0);
+
+    // initial state: S^T row j = column j of S0
+    {
+        const int j = tid;
+        float v[32];
+#pragma unroll 1
+        for (int i0 = 0; i0 < D; i0 += 32) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] = S0 ? S0[(head * D + i0 + u) * D + j] : 0.f;
+            tc::tmem_st32(lane_base + TM_S + i0, v);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+        }
+        tc::tmem_wait_st();
+    }
+    tc::fence_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (states && tid == 0) {
+        tc::bulk_store(states + (head * nc + 0) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
+        tc::bulk_commit();
+    }
+
+    const uint32_t sQE = tc::smem_u32(QE), sKH = tc::smem_u32(KH), sKT = tc::smem_u32(KT),
+                   sUU = tc::smem_u32(UU), sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt),
+                   sDT = tc::smem_u32(DT), sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
+    constexpr uint32_t ID_M1 = tc::idesc_bf16(128, 64, false, false);
+    constexpr uint32_t ID_M23 = tc::idesc_bf16(128, 64, true, false);
+    constexpr uint32_t ID_M4 = tc::idesc_bf16(128, 64, false, false, true);
+    constexpr uint32_t ID_M56 = tc::idesc_bf16(128, 64, false, false);
+    constexpr uint32_t ID_M7 = tc::idesc_bf16(128, 128, false, true);
+
+    uint32_t ph_load = 0, ph_mma = 0;
+    auto wait_mma = [&]() {
+        if (!tc::mbar_wait(bar_mma, ph_mma)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 1u); }
+        ph_mma ^= 1;
+        tc::tc_fence_after();
+    };
+
+    for (int c = 0; c < nc; ++c) {
+        const int t0 = c * C;
+        const int L = min(C, T - t0);
+        if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
+        ph_load ^= 1;
+
+        // ---- gate prep (thread = channel)
+        gate_prep(QE, KH, KT, UU, WW, sGC, tid, want_o, true);
+        tc::fence_async_smem();
+        __syncthreads();
+
+        // ---- M1: [A; P] = [Et; Qt] Kt^T
+        if (tid == 0) {
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
+            tc::mma_commit(bar_mma);
+        }
+        wait_mma();
+        {
+            float v[32];
+            if (warp < 2) {                      // A rows t = tid (strictly lower part is used)
+                const int t = tid;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    tc::tmem_ld32(lane_base + TM_AP + 32 * h2, v);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 32; u += 4)
+                        *reinterpret_cast<float4*>(&sA[t * SA_STRIDE + 32 * h2 + u]) =
+                            make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+                }
+            } else {                             // P rows t = tid - 64, causal (s <= t)
+                const int t = tid - 64;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    tc::tmem_ld32(lane_base + TM_AP + 32 * h2, v);
+                    tc::tmem_wait_ld();
+                    if (want_o) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) v[u] = (32 * h2 + u <= t) ? v[u] : 0.f;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, t, 4 * h2 + g, v + 8 * g);
+                    }
+                }
+            }
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+
+        // ---- T = (I + A)^{-1}
+        solve_unit_lower(sA, sTf, sX, TT, tid);
+        tc::fence_async_smem();
+        __syncthreads();
+
+        // ---- M2: Wm^T = Et^T T^T ;  M3: Delta^T := U^T T^T
+        if (tid == 0) {
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                tc::mma_bf16(tmem + TM_W, tc::desc_mn(sQE, 2 * C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M23, kk > 0);
+                tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M23, kk > 0);
+            }
+            tc::mma_commit(bar_mma);
+        }
+        wait_mma();
+        {   // Wm (row tile [t][i]) from Wm^T in TMEM (lane i)
+            const int i = tid;
+            float v[32];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                tc::tmem_ld32(lane_base + TM_W + 32 * h2, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) tc::st_bf16(WW, tc::tile_off(C, 32 * h2 + u, i), v[u]);
+            }
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+
+        // ---- M4: Delta^T -= S^T Wm^T ;  M5: O^T = S^T Qt^T
+        if (tid == 0) {
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWW, C, 0, kk), ID_M4, 1);
+                if (want_o)
+                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sST, D, 0, kk), tc::desc_k(sQE, 2 * C, C, kk), ID_M56, kk > 0);
+            }
+            tc::mma_commit(bar_mma);
+        }
+        wait_mma();
+        {   // Delta^T (lane j) -> bf16 row tile; scale the fp32 state by gC along its key columns
+            const int j = tid;
+            float v[32];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                tc::tmem_ld32(lane_base + TM_D + 32 * h2, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tc::st_row8(DT, D, j, 4 * h2 + g, v + 8 * g);
+            }
+#pragma unroll 1
+            for (int i0 = 0; i0 < D; i0 += 32) {
+                tc::tmem_ld32(lane_base + TM_S + i0, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
+                tc::tmem_st32(lane_base + TM_S + i0, v);
+            }
+            tc::tmem_wait_st();
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+
+        // ---- M6: O^T += Delta^T P^T ;  M7: S^T += Delta^T Kh
+        if (tid == 0) {
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                if (want_o)
+                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sDT, D, 0, kk), tc::desc_k(sPP, C, 0, kk), ID_M56, 1);
+                tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sKH, C, 0, kk), ID_M7, 1);
+            }
+            tc::mma_commit(bar_mma);
+        }
+        wait_mma();
+        // all smem tiles of this chunk are consumed: prefetch the next chunk
+        if (tid == 0 && c + 1 < nc) issue_loads(c + 1);
+
+        if (want_o) {   // o[t][j] for t < L from O^T (lane j)
+            const int j = tid;
+            float v[32];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                tc::tmem_ld32(lane_base + TM_O + 32 * h2, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int t = 32 * h2 + u;
+                    if (t < L) o[tok_off(b, t0 + t, h, T, H, D) + j] = __float2bfloat16_rn(v[u]);
+                }
+            }
+        }
+        {   // new state: bf16 copy for the next chunk's operands (and the saved image)
+            if (states && tid == 0) tc::bulk_wait_read();
+            __syncthreads();
+            const int j = tid;
+            float v[32];
+#pragma unroll 1
+            for (int i0 = 0; i0 < D; i0 += 32) {
+                tc::tmem_ld32(lane_base + TM_S + i0, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+            }
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+        if (states && tid == 0 && c + 1 < nc) {
+            tc::bulk_store(states + (head * nc + c + 1) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
+            tc::bulk_commit();
+        }
+        if (*abort_flag) break;
+    }
+
+    // final state (fp32): ST[i][j] from S^T (lane j)
+    if (ST) {
+        const int j = tid;
+        float v[32];
+#pragma unroll 1
+        for (int i0 = 0; i0 < D; i0 += 32) {
+            tc::tmem_ld32(lane_base + TM_S + i0, v);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) ST[(head * D + i0 + u) * D + j] = v[u];
+        }
+    }
+    if (states && tid == 0) tc::bulk_wait_all();
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+}  // namespace
+
+cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
+    const Dims& d = a.d;
+    if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
+    CUtensorMap mq, mk, mv, mla, mb, mw;
+    const void* ptrs[6] = {a.q, a.k, a.v, a.la, a.b, a.w};
+    CUtensorMap* maps[6] = {&mq, &mk, &mv, &mla, &mb, &mw};
+    for (int i = 0; i < 6; ++i)
+        if (make_token_map(maps[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    chunk_fwd_kernel<<<d.B * d.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mla, mb, mw, a.S0,
+                                                       static_cast<__nv_bfloat16*>(a.o), a.ST, a.states, d.T, d.H);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn2

@@ -1,0 +1,236 @@
+// gdn2_api.cu -- the C ABI of libgdn2.so (declared in include/gdn2.h).
+//
+// Host-side argument checks, workspace layout and dispatch between the
+// tensor-core chunkwise kernels (bf16, Dk = Dv = 128, chunk 64) and the fp32
+// token-recurrent kernels (everything else). Nothing here allocates memory or
+// synchronises; every launch goes to the caller's stream.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "gdn2.h"
+#include "internal.h"
+
+using namespace gdn2;
+
+namespace {
+
+thread_local char g_err[512];
+
+gdn2_status fail(gdn2_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+gdn2_status fail(gdn2_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+gdn2_status cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return GDN2_OK;
+    return fail(GDN2_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Checks sizes; returns GDN2_OK or an error status with detail.
+gdn2_status check_dims(int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt, bool seq) {
+    if (dt != GDN2_F32 && dt != GDN2_BF16) return fail(GDN2_ERR_INVALID, "dtype %d is not GDN2_F32 or GDN2_BF16", (int)dt);
+    if (B < 1 || H < 1) return fail(GDN2_ERR_INVALID, "B=%d and H=%d must be >= 1", B, H);
+    if (seq && T < 0) return fail(GDN2_ERR_INVALID, "T=%d must be >= 0", T);
+    if (!dim_ok(Dk) || !dim_ok(Dv))
+        return fail(GDN2_ERR_UNSUPPORTED, "Dk=%d, Dv=%d: each must be 16, 32, 64 or 128", Dk, Dv);
+    if (seq && !chunk_ok(chunk)) return fail(GDN2_ERR_UNSUPPORTED, "chunk=%d: must be 16, 32 or 64", chunk);
+    // element counts must stay well inside size_t and int grid limits
+    const double elems = (double)B * (seq ? (double)T : 1.0) * H * (Dk > Dv ? Dk : Dv);
+    if (elems > 4.0e15) return fail(GDN2_ERR_INVALID, "problem too large");
+    if ((double)B * H > 2147483647.0) return fail(GDN2_ERR_INVALID, "B*H too large");
+    return GDN2_OK;
+}
+
+size_t states_bytes(const Dims& d, gdn2_dtype dt) {
+    const size_t units = (size_t)d.B * d.H * (size_t)d.nchunks();
+    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * TC_STATE_BYTES : units * d.Dk * d.Dv * sizeof(float);
+}
+
+size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
+    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk)) return (size_t)d.B * d.H * (size_t)d.nchunks() * TC_STATE_BYTES;
+    const size_t seg = (size_t)d.B * d.H * d.chunk * d.Dk * d.Dv * sizeof(float);
+    const size_t del = (size_t)d.B * d.H * d.chunk * d.Dv * sizeof(float);
+    return align256(seg) + align256(del);
+}
+
+#define REQUIRE_PTR(p)                                                                      \
+    do {                                                                                    \
+        if (!(p)) return fail(GDN2_ERR_INVALID, "%s must not be NULL", #p);                 \
+        if (!aligned((p), 16)) return fail(GDN2_ERR_INVALID, "%s must be 16-byte aligned", #p); \
+    } while (0)
+#define OPTIONAL_PTR(p)                                                                     \
+    do {                                                                                    \
+        if ((p) && !aligned((p), 16)) return fail(GDN2_ERR_INVALID, "%s must be 16-byte aligned", #p); \
+    } while (0)
+
+// T == 0: the final state is the initial state and no token work exists.
+gdn2_status copy_or_zero_state(float* dst, const float* src, const Dims& d, cudaStream_t s) {
+    if (!dst || dst == src) return GDN2_OK;
+    const size_t bytes = (size_t)d.B * d.H * d.Dk * d.Dv * sizeof(float);
+    cudaError_t e = src ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(dst, 0, bytes, s);
+    return cuda_status(e, "state copy");
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn2_version(void) { return 100; }
+
+const char* gdn2_status_string(gdn2_status s) {
+    switch (s) {
+    case GDN2_OK: return "GDN2_OK";
+    case GDN2_ERR_INVALID: return "GDN2_ERR_INVALID: invalid argument";
+    case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED: shape or dtype not supported";
+    case GDN2_ERR_WORKSPACE: return "GDN2_ERR_WORKSPACE: workspace missing or too small";
+    case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA: CUDA runtime error";
+    case GDN2_ERR_TIMEOUT: return "GDN2_ERR_TIMEOUT: device-side wait gave up";
+    }
+    return "unknown gdn2_status";
+}
+
+const char* gdn2_last_error(void) { return g_err; }
+
+size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt) {
+    if (check_dims(B, T, H, Dk, Dv, chunk, dt, true) != GDN2_OK) return 0;
+    const Dims d{B, T, H, Dk, Dv, chunk};
+    switch (op) {
+    case GDN2_OP_FWD: return 0;
+    case GDN2_OP_FWD_SAVE: return align256(states_bytes(d, dt));
+    case GDN2_OP_BWD: return align256(states_bytes(d, dt)) + align256(bwd_extra_bytes(d, dt));
+    }
+    return 0;
+}
+
+gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                     const void* w, const float* S0, void* o, float* ST, int B, int T, int H, int Dk,
+                     int Dv, int chunk, gdn2_dtype dt, int save_states, void* ws, size_t ws_bytes,
+                     void* stream) {
+    gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
+    if (st != GDN2_OK) return st;
+    const Dims d{B, T, H, Dk, Dv, chunk};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    OPTIONAL_PTR(S0);
+    OPTIONAL_PTR(ST);
+    if (T == 0) return copy_or_zero_state(ST, S0, d, s);
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(log_alpha);
+    REQUIRE_PTR(b); REQUIRE_PTR(w); REQUIRE_PTR(o);
+    if (save_states) {
+        const size_t need = gdn2_workspace_size(GDN2_OP_FWD_SAVE, B, T, H, Dk, Dv, chunk, dt);
+        if (!ws || ws_bytes < need)
+            return fail(GDN2_ERR_WORKSPACE, "save_states needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
+        if (!aligned(ws, 256)) return fail(GDN2_ERR_INVALID, "ws must be 256-byte aligned");
+    }
+    if (save_states ? tc_train_path(dt, Dk, Dv, chunk) : tc_path(dt, Dk, Dv, chunk)) {
+        ChunkFwdArgs a{};
+        a.d = d;
+        a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
+        a.S0 = S0; a.o = o; a.ST = ST;
+        a.states = save_states ? static_cast<unsigned char*>(ws) : nullptr;
+        return cuda_status(chunk_fwd_launch(a, s), "gdn2_fwd (tensor-core path)");
+    }
+    RecurrentArgs a{};
+    a.op = RecurrentArgs::FWD;
+    a.dt = dt;
+    a.d = d;
+    a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
+    a.S0 = S0; a.o = o; a.ST = ST;
+    a.states = save_states ? static_cast<float*>(ws) : nullptr;
+    return cuda_status(recurrent_launch(a, s), "gdn2_fwd (recurrent path)");
+}
+
+gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                     const void* w, const float* S0, const void* dout, const float* dST, void* dq,
+                     void* dk, void* dv, void* dlog_alpha, void* db, void* dw, float* dS0, int B, int T,
+                     int H, int Dk, int Dv, int chunk, gdn2_dtype dt, int states_saved, void* ws,
+                     size_t ws_bytes, void* stream) {
+    gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
+    if (st != GDN2_OK) return st;
+    const Dims d{B, T, H, Dk, Dv, chunk};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    OPTIONAL_PTR(S0);
+    OPTIONAL_PTR(dST);
+    OPTIONAL_PTR(dS0);
+    if (T == 0) return copy_or_zero_state(dS0, dST, d, s);
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(log_alpha);
+    REQUIRE_PTR(b); REQUIRE_PTR(w); REQUIRE_PTR(dout);
+    REQUIRE_PTR(dq); REQUIRE_PTR(dk); REQUIRE_PTR(dv); REQUIRE_PTR(dlog_alpha);
+    REQUIRE_PTR(db); REQUIRE_PTR(dw);
+    const size_t need = gdn2_workspace_size(GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt);
+    if (!ws || ws_bytes < need)
+        return fail(GDN2_ERR_WORKSPACE, "gdn2_bwd needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
+    if (!aligned(ws, 256)) return fail(GDN2_ERR_INVALID, "ws must be 256-byte aligned");
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    unsigned char* extra = wsb + align256(states_bytes(d, dt));
+
+    if (tc_train_path(dt, Dk, Dv, chunk)) {
+        if (!states_saved) {
+            ChunkFwdArgs f{};
+            f.d = d;
+            f.q = q; f.k = k; f.v = v; f.la = log_alpha; f.b = b; f.w = w;
+            f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb;
+            gdn2_status e = cuda_status(chunk_fwd_launch(f, s), "gdn2_bwd state recompute");
+            if (e != GDN2_OK) return e;
+        }
+        ChunkBwdArgs a{};
+        a.d = d;
+        a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w; a.dout = dout;
+        a.dST = dST;
+        a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.db = db; a.dw = dw; a.dS0 = dS0;
+        a.states = wsb;
+        a.dstates = extra;
+        return cuda_status(chunk_bwd_launch(a, s), "gdn2_bwd (tensor-core path)");
+    }
+
+    RecurrentArgs a{};
+    a.dt = dt;
+    a.d = d;
+    a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
+    a.S0 = S0;
+    a.states = reinterpret_cast<float*>(wsb);
+    if (!states_saved) {
+        a.op = RecurrentArgs::FWD;
+        a.o = nullptr;
+        a.ST = nullptr;
+        gdn2_status e = cuda_status(recurrent_launch(a, s), "gdn2_bwd state recompute");
+        if (e != GDN2_OK) return e;
+    }
+    a.op = RecurrentArgs::BWD;
+    a.dout = dout; a.dST = dST;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.db = db; a.dw = dw; a.dS0 = dS0;
+    const size_t seg = (size_t)B * H * chunk * Dk * Dv * sizeof(float);
+    a.seg = reinterpret_cast<float*>(extra);
+    a.segdelta = reinterpret_cast<float*>(extra + align256(seg));
+    return cuda_status(recurrent_launch(a, s), "gdn2_bwd (recurrent path)");
+}
+
+gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
+                             const void* b, const void* w, float* S, void* o, int B, int H, int Dk,
+                             int Dv, gdn2_dtype dt, void* stream) {
+    gdn2_status st = check_dims(B, 1, H, Dk, Dv, 64, dt, false);
+    if (st != GDN2_OK) return st;
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(log_alpha);
+    REQUIRE_PTR(b); REQUIRE_PTR(w); REQUIRE_PTR(S); REQUIRE_PTR(o);
+    RecurrentArgs a{};
+    a.op = RecurrentArgs::DECODE;
+    a.dt = dt;
+    a.d = Dims{B, 1, H, Dk, Dv, 64};
+    a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
+    a.S = S; a.o = o;
+    return cuda_status(recurrent_launch(a, static_cast<cudaStream_t>(stream)), "gdn2_decode_step");
+}
+
+}  // extern "C"

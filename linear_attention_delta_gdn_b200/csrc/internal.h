@@ -1,0 +1,66 @@
+// internal.h -- launch interfaces between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace gdn2 {
+
+// fp32 token-recurrent kernels (recurrent.cu).
+struct RecurrentArgs {
+    enum Op { DECODE, FWD, BWD } op;
+    gdn2_dtype dt;
+    Dims d;
+    const void *q, *k, *v, *la, *b, *w, *dout;
+    const float *S0, *dST;
+    float* S;            // decode: state in/out
+    void* o;             // output (may be null in FWD: states only)
+    float *ST, *dS0;
+    void *dq, *dk, *dv, *dla, *db, *dw;
+    float* states;       // [B,H,NC,Dk,Dv] fp32 chunk-start states (FWD writes if non-null, BWD reads)
+    float* seg;          // BWD scratch [B,H,chunk,Dk,Dv]
+    float* segdelta;     // BWD scratch [B,H,chunk,Dv]
+};
+cudaError_t recurrent_launch(const RecurrentArgs& a, cudaStream_t s);
+
+// Tensor-core chunkwise kernels (chunk_fwd.cu, chunk_bwd.cu): bf16, Dk = Dv = 128, chunk = 64.
+constexpr int TC_D = 128;
+constexpr int TC_C = 64;
+// bytes of one saved state image (bf16 128 x 128, 128B-swizzled panels)
+constexpr size_t TC_STATE_BYTES = (size_t)TC_D * TC_D * 2;
+
+struct ChunkFwdArgs {
+    Dims d;
+    const void *q, *k, *v, *la, *b, *w;
+    const float* S0;
+    void* o;               // may be null: states only
+    float* ST;
+    unsigned char* states; // [B,H,NC] state images, or null
+};
+cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s);
+
+struct ChunkBwdArgs {
+    Dims d;
+    const void *q, *k, *v, *la, *b, *w, *dout;
+    const float *dST;
+    void *dq, *dk, *dv, *dla, *db, *dw;
+    float* dS0;
+    const unsigned char* states;  // [B,H,NC] chunk-start state images
+    unsigned char* dstates;       // [B,H,NC] images of dL/dS at each chunk end (scratch)
+};
+cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
+
+// Whether the tensor-core forward handles this problem.
+inline bool tc_path(gdn2_dtype dt, int Dk, int Dv, int chunk) {
+    return dt == GDN2_BF16 && Dk == TC_D && Dv == TC_D && chunk == TC_C;
+}
+// Whether the tensor-core backward is built.
+constexpr bool kTcBackward = false;
+// Whether training (fwd with saved states + bwd) runs on the tensor-core kernels.
+inline bool tc_train_path(gdn2_dtype dt, int Dk, int Dv, int chunk) {
+    return kTcBackward && tc_path(dt, Dk, Dv, chunk);
+}
+
+}  // namespace gdn2

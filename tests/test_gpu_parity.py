@@ -1,0 +1,262 @@
+"""GPU parity: libgdn2 (through its C ABI) against the fp64 oracle on the same
+seeded inputs.
+
+Tolerances (relative L2 over a whole tensor, ||x - ref|| / ||ref||):
+  fp32 inputs: o, S_T and every gradient <= 1e-4
+  bf16 inputs (fp32 state and accumulation): o, S_T <= 2e-2; gradients <= 3e-2
+The oracle consumes exactly the dtype-rounded inputs, widened to fp64. Full-size
+workloads are checked on sampled (batch, head) pairs, which the oracle computes
+independently of the others (heads never interact).
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import rel_l2
+from linear_attention_delta_gdn_b200 import binding
+from linear_attention_delta_gdn_b200.inputs import WORKLOADS, make_inputs, make_workload_inputs, make_decode_stream, to_f64
+
+pytestmark = pytest.mark.gpu
+
+TOL_OUT = {"f32": 1e-4, "bf16": 2e-2}
+TOL_GRAD = {"f32": 1e-4, "bf16": 3e-2}
+GRADS = ("dq", "dk", "dv", "dlog_alpha", "db", "dw")
+NAMES = ("q", "k", "v", "log_alpha", "b", "w")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from linear_attention_delta_gdn_b200 import build
+    build.build()
+
+
+def dev(x):
+    return {n: (t.cuda() if t is not None else None) for n, t in x.items()}
+
+
+def f64(x):
+    return {n: to_f64(t) for n, t in x.items() if t is not None}
+
+
+def heads_slice(a, heads, state=False):
+    """Stack the (b, h) slices of a [B, T, H, D] (or [B, H, Dk, Dv]) array as batch entries."""
+    if state:
+        return np.stack([a[b, h] for b, h in heads])[:, None]
+    return np.stack([a[b, :, h] for b, h in heads])[:, :, None]
+
+
+def oracle_fwd(oracle_mod, x, heads=None):
+    g = f64(x)
+    S0 = g.get("S0")
+    args = [g[n] for n in NAMES]
+    if heads is not None:
+        args = [heads_slice(a, heads) for a in args]
+        S0 = None if S0 is None else heads_slice(S0, heads, state=True)
+    return oracle_mod.fwd(*args, S0=S0)
+
+
+def oracle_bwd(oracle_mod, x, dST=None, heads=None):
+    g = f64(x)
+    S0 = g.get("S0")
+    args = [g[n] for n in NAMES]
+    dout = g["dout"]
+    if heads is not None:
+        args = [heads_slice(a, heads) for a in args]
+        dout = heads_slice(dout, heads)
+        S0 = None if S0 is None else heads_slice(S0, heads, state=True)
+        dST = None if dST is None else heads_slice(dST, heads, state=True)
+    return oracle_mod.bwd(*args, dout=dout, S0=S0, dST=dST)
+
+
+def gpu_fwd(x, chunk):
+    d = dev(x)
+    o, ST = binding.gdn2_fwd(*(d[n] for n in NAMES), d.get("S0"), chunk=chunk)
+    torch.cuda.synchronize()
+    return to_f64(o), to_f64(ST)
+
+
+def pick(arr, heads, state=False):
+    return heads_slice(arr, heads, state) if heads is not None else arr
+
+
+def check_fwd(oracle_mod, x, chunk, dtype, heads=None):
+    o, ST = gpu_fwd(x, chunk)
+    o_ref, ST_ref = oracle_fwd(oracle_mod, x, heads)
+    eo, es = rel_l2(pick(o, heads), o_ref), rel_l2(pick(ST, heads, True), ST_ref)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(ST))
+    assert eo <= TOL_OUT[dtype], "o rel err %.3g" % eo
+    assert es <= TOL_OUT[dtype], "S_T rel err %.3g" % es
+    return eo, es
+
+
+# ---------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("Dk,Dv", [(128, 128), (64, 64), (32, 128), (128, 16)])
+def test_decode_steps(oracle_mod, dtype, Dk, Dv):
+    x = make_inputs(3, 5, 2, Dk, Dv, seed=7 + Dk + Dv, dtype=dtype, with_S0=True)
+    d = dev(x)
+    S = d["S0"].clone()
+    Sref = to_f64(x["S0"])
+    g = f64(x)
+    for t in range(5):
+        o = binding.gdn2_decode_step(*(d[n][:, t].contiguous() for n in NAMES), S)
+        o_ref, Sref = oracle_mod.decode(*(g[n][:, t] for n in NAMES), Sref)
+        assert rel_l2(to_f64(o), o_ref) <= TOL_OUT[dtype]
+    assert rel_l2(to_f64(S), Sref) <= TOL_OUT[dtype] / 10
+
+
+def test_decode_workload_sampled(oracle_mod):
+    wl = WORKLOADS["decode-bf16-b256h16d128x1024"]
+    xs = make_decode_stream(wl.T, wl.B, wl.H, wl.Dk, wl.Dv, wl.seed, wl.dtype, device="cuda")
+    heads = [(0, 0), (17, 3), (100, 7), (128, 8), (200, 11), (255, 15), (64, 1), (31, 14)]
+    bi = torch.tensor([b for b, _ in heads], device="cuda")
+    hi = torch.tensor([h for _, h in heads], device="cuda")
+    S = xs["S0"].clone()
+    Sref = to_f64(xs["S0"][bi, hi])[:, None]
+    o_gpu = []
+    for t in range(wl.T):
+        o = binding.gdn2_decode_step(*(xs[n][t] for n in NAMES), S)
+        o_gpu.append(o[bi, hi])
+    o_gpu = to_f64(torch.stack(o_gpu))                    # [steps, 8, Dv]
+    sub = {n: to_f64(xs[n][:, bi, hi]) for n in NAMES}    # [steps, 8, D]
+    o_ref = np.zeros_like(o_gpu)
+    for t in range(wl.T):
+        o_t, Sref = oracle_mod.decode(*(sub[n][t][:, None] for n in NAMES), Sref)
+        o_ref[t] = o_t[:, 0]
+    assert rel_l2(o_gpu, o_ref) <= TOL_OUT["bf16"]
+    assert rel_l2(to_f64(S[bi, hi]), Sref[:, 0]) <= TOL_OUT["bf16"]
+
+
+# ---------------------------------------------------------------- forward
+
+@pytest.mark.parametrize("T", [1, 37, 64, 150])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("Dk,Dv", [(64, 64), (32, 128)])
+def test_fwd_fp32_small(oracle_mod, T, chunk, Dk, Dv):
+    x = make_inputs(2, T, 3, Dk, Dv, seed=T + chunk + Dk, dtype="f32", with_S0=(T % 2 == 1))
+    check_fwd(oracle_mod, x, chunk, "f32")
+
+
+@pytest.mark.parametrize("T", [1, 37, 64, 150, 333])
+@pytest.mark.parametrize("with_S0", [False, True])
+def test_fwd_bf16_d128(oracle_mod, T, with_S0):
+    x = make_inputs(2, T, 3, 128, 128, seed=100 + T, dtype="bf16", with_S0=with_S0)
+    check_fwd(oracle_mod, x, 64, "bf16")
+
+
+@pytest.mark.parametrize("Dk,Dv,chunk", [(64, 64, 64), (128, 128, 32), (64, 128, 16)])
+def test_fwd_bf16_other_shapes(oracle_mod, Dk, Dv, chunk):
+    x = make_inputs(2, 97, 2, Dk, Dv, seed=200 + Dk + chunk, dtype="bf16", with_S0=True)
+    check_fwd(oracle_mod, x, chunk, "bf16")
+
+
+def test_fwd_workload_fp32(oracle_mod):
+    wl = WORKLOADS["fwd-f32-b1h2t256d64"]
+    check_fwd(oracle_mod, make_workload_inputs(wl), wl.chunk, wl.dtype)
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("fwd-bf16-b4h16t4096d128", [(0, 0), (1, 7), (2, 13), (3, 15)]),
+    ("fwd-bf16-b1h16t65536d128-s0", [(0, 0), (0, 9), (0, 15)]),
+])
+def test_fwd_workload_sampled(oracle_mod, name, heads):
+    wl = WORKLOADS[name]
+    check_fwd(oracle_mod, make_workload_inputs(wl), wl.chunk, wl.dtype, heads=heads)
+
+
+def test_fwd_resume_from_state(oracle_mod):
+    """fwd over [0, T) equals fwd over [0, T1) then [T1, T) started from S_T1."""
+    x = make_inputs(2, 200, 2, 128, 128, seed=300, dtype="bf16", with_S0=True)
+    d = dev(x)
+    o, ST = binding.gdn2_fwd(*(d[n] for n in NAMES), d["S0"])
+    T1 = 128
+    first = {n: d[n][:, :T1].contiguous() for n in NAMES}
+    second = {n: d[n][:, T1:].contiguous() for n in NAMES}
+    o1, S1 = binding.gdn2_fwd(*(first[n] for n in NAMES), d["S0"])
+    o2, S2 = binding.gdn2_fwd(*(second[n] for n in NAMES), S1)
+    assert rel_l2(to_f64(torch.cat([o1, o2], 1)), to_f64(o)) < 1e-2
+    assert rel_l2(to_f64(S2), to_f64(ST)) < 1e-2
+
+
+def test_fwd_state_in_place(oracle_mod):
+    x = make_inputs(1, 70, 2, 128, 128, seed=301, dtype="bf16", with_S0=True)
+    d = dev(x)
+    _, ST = binding.gdn2_fwd(*(d[n] for n in NAMES), d["S0"])
+    S = d["S0"].clone()
+    binding.gdn2_fwd(*(d[n] for n in NAMES), S, ST=S)
+    assert torch.equal(S, ST)
+
+
+# ---------------------------------------------------------------- backward
+
+def check_bwd(oracle_mod, x, chunk, dtype, heads=None, with_dST=False, saved=False):
+    d = dev(x)
+    dST = None
+    if with_dST:
+        B, _, H, Dk = x["q"].shape
+        dST = torch.randn((B, H, Dk, x["v"].shape[-1]), generator=torch.Generator().manual_seed(5))
+    if saved:
+        B, T, H, Dk = x["q"].shape
+        Dv = x["v"].shape[-1]
+        need = binding.gdn2_workspace_size(binding.GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, binding._dt(d["q"]))
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        binding.gdn2_fwd(*(d[n] for n in NAMES), d.get("S0"), chunk=chunk, save_states=True, ws=ws)
+        g = binding.gdn2_bwd(*(d[n] for n in NAMES), d["dout"], d.get("S0"),
+                             None if dST is None else dST.cuda(), chunk=chunk, states_saved=True, ws=ws)
+    else:
+        g = binding.gdn2_bwd(*(d[n] for n in NAMES), d["dout"], d.get("S0"),
+                             None if dST is None else dST.cuda(), chunk=chunk)
+    torch.cuda.synchronize()
+    ref = oracle_bwd(oracle_mod, x, None if dST is None else dST.double().numpy(), heads)
+    errs = {}
+    for n in GRADS:
+        got = to_f64(g[n])
+        assert np.all(np.isfinite(got)), n
+        errs[n] = rel_l2(pick(got, heads), ref[n])
+    errs["dS0"] = rel_l2(pick(to_f64(g["dS0"]), heads, True), ref["dS0"])
+    bad = {n: e for n, e in errs.items() if e > TOL_GRAD[dtype]}
+    assert not bad, "gradient rel errors above %g: %s (all: %s)" % (TOL_GRAD[dtype], bad, errs)
+    return errs
+
+
+@pytest.mark.parametrize("T", [1, 37, 150])
+@pytest.mark.parametrize("chunk", [16, 64])
+def test_bwd_fp32_small(oracle_mod, T, chunk):
+    x = make_inputs(2, T, 2, 32, 64, seed=400 + T + chunk, dtype="f32", with_do=True, with_S0=True)
+    check_bwd(oracle_mod, x, chunk, "f32", with_dST=True)
+
+
+@pytest.mark.parametrize("T", [1, 37, 64, 150, 300])
+@pytest.mark.parametrize("with_S0", [False, True])
+def test_bwd_bf16_d128(oracle_mod, T, with_S0):
+    x = make_inputs(2, T, 2, 128, 128, seed=500 + T, dtype="bf16", with_do=True, with_S0=with_S0)
+    check_bwd(oracle_mod, x, 64, "bf16", with_dST=with_S0)
+
+
+@pytest.mark.parametrize("saved", [False, True])
+def test_bwd_saved_states(oracle_mod, saved):
+    x = make_inputs(1, 190, 3, 128, 128, seed=600, dtype="bf16", with_do=True, with_S0=True)
+    check_bwd(oracle_mod, x, 64, "bf16", with_dST=True, saved=saved)
+
+
+def test_bwd_workload_sampled(oracle_mod):
+    wl = WORKLOADS["fwdbwd-bf16-b4h16t4096d128"]
+    x = make_workload_inputs(wl)
+    errs = check_bwd(oracle_mod, x, wl.chunk, wl.dtype, heads=[(0, 0), (1, 6), (2, 11), (3, 15)], saved=True)
+    print("sampled-head gradient rel errors:", errs)
+
+
+def test_autograd_matches_direct():
+    x = make_inputs(2, 100, 2, 128, 128, seed=700, dtype="bf16", with_do=True, with_S0=True)
+    d = dev(x)
+    leaves = {n: d[n].clone().requires_grad_(True) for n in NAMES}
+    S0 = d["S0"].clone().requires_grad_(True)
+    o, ST = binding.gated_delta_rule2(*(leaves[n] for n in NAMES), S0)
+    (o.float() * d["dout"].float()).sum().backward()
+    g = binding.gdn2_bwd(*(d[n] for n in NAMES), d["dout"], d["S0"])
+    for n, gn in zip(NAMES, GRADS):
+        assert rel_l2(to_f64(leaves[n].grad), to_f64(g[gn])) < 1e-6, n
+    assert rel_l2(to_f64(S0.grad), to_f64(g["dS0"])) < 1e-6
