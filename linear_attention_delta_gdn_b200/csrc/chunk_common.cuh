@@ -30,8 +30,7 @@ namespace chunk {
 constexpr int D = 128;        // d_k = d_v
 constexpr int C = 64;         // chunk length
 constexpr int NT = 128;       // threads per CTA (one warpgroup; thread i <-> TMEM lane i)
-constexpr int TILE64 = C * 128 * 2 / 2;   // bytes of a [64 x 128] bf16 row tile (16 KB)
-constexpr int SA_STRIDE = 68;             // fp32 row stride of the solve scratch
+constexpr uint32_t TILE_64x128 = 64 * 128 * 2;    // bytes of a [64 x 128] bf16 row tile
 
 // ------------------------------------------------------------ host: TMA maps
 
@@ -100,11 +99,48 @@ __device__ __forceinline__ void gate_prep(unsigned char* QE, unsigned char* KH, 
     }
 }
 
-// (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32, row stride SA_STRIDE, in sA).
-// Writes the fp32 inverse to sTf (same stride; lower triangle incl. the unit
-// diagonal is valid) and the bf16 row tile T (64 x 64, zeros above the diagonal).
+// fp32 64 x 64 scratch matrices (A and its inverse) are stored with row stride
+// 64 and the column index XOR-ed with (row % 32): row-wise and column-wise
+// accesses by a warp are then both free of bank conflicts.
+__device__ __forceinline__ int sq_idx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+
+// Copy the strictly lower part of [A; P] from TMEM (lanes 0..63 = A, 64..127 = P,
+// 64 columns at tm_ap) into the fp32 scratch sA (warps 0, 1) and, if want_p,
+// the causal part of P into the bf16 row tile PP (warps 2, 3).
+__device__ __forceinline__ void extract_AP(uint32_t lane_base_ap, float* sA, unsigned char* PP, bool want_p,
+                                           int tid) {
+    float v[32];
+    if (tid < 64) {
+        const int t = tid;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            tc::tmem_ld32(lane_base_ap + 32 * h2, v);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) sA[sq_idx(t, 32 * h2 + u)] = v[u];
+        }
+    } else {
+        const int t = tid - 64;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            tc::tmem_ld32(lane_base_ap + 32 * h2, v);
+            tc::tmem_wait_ld();
+            if (want_p) {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] = (32 * h2 + u <= t) ? v[u] : 0.f;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, t, 4 * h2 + g, v + 8 * g);
+            }
+        }
+    }
+}
+
+// (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32 scratch sA).
+// Writes the fp32 inverse to sTf (lower triangle incl. the unit diagonal is
+// valid) and the bf16 row tile T (64 x 64, zeros above the diagonal).
 // 16 x 16 diagonal blocks by forward substitution (one warp per block), then the
 // off-diagonal blocks by diagonals: T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj.
+// sX (768 floats) may alias the T tile: it is dead before T is written.
 __device__ __forceinline__ void solve_unit_lower(const float* sA, float* sTf, float* sX, unsigned char* Ttile,
                                                  int tid) {
     const int warp = tid >> 5, lane = tid & 31;
@@ -115,9 +151,9 @@ __device__ __forceinline__ void solve_unit_lower(const float* sA, float* sTf, fl
         for (int r = 0; r < 16; ++r) {
             float acc = (r == s) ? 1.f : 0.f;
 #pragma unroll
-            for (int m = 0; m < r; ++m) acc -= sA[(base + r) * SA_STRIDE + base + m] * x[m];
+            for (int m = 0; m < r; ++m) acc -= sA[sq_idx(base + r, base + m)] * x[m];
             x[r] = acc;
-            sTf[(base + r) * SA_STRIDE + base + s] = acc;
+            sTf[sq_idx(base + r, base + s)] = acc;
         }
     }
     __syncthreads();
@@ -130,7 +166,7 @@ __device__ __forceinline__ void solve_unit_lower(const float* sA, float* sTf, fl
             for (int kb = j; kb < i; ++kb) {
 #pragma unroll
                 for (int m = 0; m < 16; ++m)
-                    acc += sA[(16 * i + r) * SA_STRIDE + 16 * kb + m] * sTf[(16 * kb + m) * SA_STRIDE + 16 * j + c];
+                    acc += sA[sq_idx(16 * i + r, 16 * kb + m)] * sTf[sq_idx(16 * kb + m, 16 * j + c)];
             }
             sX[e] = acc;
         }
@@ -138,8 +174,8 @@ __device__ __forceinline__ void solve_unit_lower(const float* sA, float* sTf, fl
         for (int e = tid; e < nb * 256; e += NT) {
             const int j = e >> 8, i = j + d, r = (e >> 4) & 15, c = e & 15;
             float acc = 0.f;
-            for (int m = 0; m <= r; ++m) acc += sTf[(16 * i + r) * SA_STRIDE + 16 * i + m] * sX[(j << 8) + m * 16 + c];
-            sTf[(16 * i + r) * SA_STRIDE + 16 * j + c] = -acc;
+            for (int m = 0; m <= r; ++m) acc += sTf[sq_idx(16 * i + r, 16 * i + m)] * sX[(j << 8) + m * 16 + c];
+            sTf[sq_idx(16 * i + r, 16 * j + c)] = -acc;
         }
         __syncthreads();
     }
@@ -151,11 +187,52 @@ __device__ __forceinline__ void solve_unit_lower(const float* sA, float* sTf, fl
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int s = 8 * g + u;
-                x[u] = (s <= t) ? sTf[t * SA_STRIDE + s] : 0.f;
+                x[u] = (s <= t) ? sTf[sq_idx(t, s)] : 0.f;
             }
             tc::st_row8(Ttile, C, t, g, x);
         }
     }
+}
+
+// Transpose a [128 lanes x 64 columns] fp32 TMEM accumulator (lane = channel,
+// column = token) into the bf16 row tile dst [64 tokens x 128 channels].
+__device__ __forceinline__ void tmem_to_tile_transposed(uint32_t lane_base_col, unsigned char* dst, int tid) {
+    float v[32];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        tc::tmem_ld32(lane_base_col + 32 * h2, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) tc::st_bf16(dst, tc::tile_off(C, 32 * h2 + u, tid), v[u]);
+    }
+}
+
+// Copy a [128 lanes x ncol] fp32 TMEM accumulator into a bf16 row tile of 128
+// rows (row = lane), ncol in {64, 128}.
+template <int NCOL>
+__device__ __forceinline__ void tmem_to_tile_rows(uint32_t lane_base_col, unsigned char* dst, int tid) {
+    float v[32];
+#pragma unroll
+    for (int c0 = 0; c0 < NCOL; c0 += 32) {
+        tc::tmem_ld32(lane_base_col + c0, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) tc::st_row8(dst, 128, tid, (c0 >> 3) + g, v + 8 * g);
+    }
+}
+
+// Multiply a [128 lanes x 128 columns] fp32 TMEM state by gC[column] in place.
+__device__ __forceinline__ void tmem_scale_columns(uint32_t lane_base_col, const float* gC) {
+    float v[32];
+#pragma unroll 1
+    for (int i0 = 0; i0 < D; i0 += 32) {
+        tc::tmem_ld32(lane_base_col + i0, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] *= gC[i0 + u];
+        tc::tmem_st32(lane_base_col + i0, v);
+    }
+    tc::tmem_wait_st();
 }
 
 }  // namespace chunk

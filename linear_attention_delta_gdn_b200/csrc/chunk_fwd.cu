@@ -35,14 +35,13 @@ constexpr uint32_t OFF_KT = 49152;       // [64 x 128] log_alpha -> Kt
 constexpr uint32_t OFF_UU = 65536;       // [64 x 128] v -> U
 constexpr uint32_t OFF_WW = 81920;       // [64 x 128] w -> Wm
 constexpr uint32_t OFF_ST = 98304;       // [128 x 128] S^T (bf16)
-constexpr uint32_t OFF_DT = 131072;      // [128 x 64] Delta^T (bf16)  | fp32 A scratch [64 x 68]
-constexpr uint32_t OFF_TF = 148480;      // fp32 T [64 x 68]
-constexpr uint32_t OFF_X = 165888;       // fp32 solve temporaries (768)
-constexpr uint32_t OFF_TT = 178176;      // [64 x 64] T (bf16)
-constexpr uint32_t OFF_PP = 186368;      // [64 x 64] P (bf16)
-constexpr uint32_t OFF_GC = 194560;      // fp32 gC[128]
-constexpr uint32_t OFF_BAR = 195072;     // 2 mbarriers, tmem base, abort flag
-constexpr uint32_t SMEM_BYTES = 195136 + 1024;
+constexpr uint32_t OFF_DT = 131072;      // [128 x 64] Delta^T (bf16)  | fp32 A scratch [64 x 64]
+constexpr uint32_t OFF_TF = 147456;      // fp32 T [64 x 64]
+constexpr uint32_t OFF_TT = 163840;      // [64 x 64] T (bf16)  | solve temporaries (768 floats)
+constexpr uint32_t OFF_PP = 172032;      // [64 x 64] P (bf16)
+constexpr uint32_t OFF_GC = 180224;      // fp32 gC[128]
+constexpr uint32_t OFF_BAR = 180736;     // 2 mbarriers, tmem base, abort flag
+constexpr uint32_t SMEM_BYTES = 180800 + 1024;
 
 // TMEM columns
 constexpr uint32_t TM_S = 0, TM_AP = 128, TM_W = 192, TM_D = 256, TM_O = 320, TM_COLS = 512;
@@ -68,7 +67,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     unsigned char* DT = sm + OFF_DT;
     float* sA = reinterpret_cast<float*>(sm + OFF_DT);
     float* sTf = reinterpret_cast<float*>(sm + OFF_TF);
-    float* sX = reinterpret_cast<float*>(sm + OFF_X);
+    float* sX = reinterpret_cast<float*>(sm + OFF_TT);
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
@@ -173,34 +172,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        {
-            float v[32];
-            if (warp < 2) {                      // A rows t = tid (strictly lower part is used)
-                const int t = tid;
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    tc::tmem_ld32(lane_base + TM_AP + 32 * h2, v);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 32; u += 4)
-                        *reinterpret_cast<float4*>(&sA[t * SA_STRIDE + 32 * h2 + u]) =
-                            make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
-                }
-            } else {                             // P rows t = tid - 64, causal (s <= t)
-                const int t = tid - 64;
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    tc::tmem_ld32(lane_base + TM_AP + 32 * h2, v);
-                    tc::tmem_wait_ld();
-                    if (want_o) {
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) v[u] = (32 * h2 + u <= t) ? v[u] : 0.f;
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, t, 4 * h2 + g, v + 8 * g);
-                    }
-                }
-            }
-        }
+        extract_AP(lane_base + TM_AP, sA, PP, want_o, tid);
         tc::tc_fence_before();
         __syncthreads();
 
@@ -220,17 +192,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        {   // Wm (row tile [t][i]) from Wm^T in TMEM (lane i)
-            const int i = tid;
-            float v[32];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                tc::tmem_ld32(lane_base + TM_W + 32 * h2, v);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 32; ++u) tc::st_bf16(WW, tc::tile_off(C, 32 * h2 + u, i), v[u]);
-            }
-        }
+        tmem_to_tile_transposed(lane_base + TM_W, WW, tid);   // Wm [t][i] from Wm^T (lane i)
         tc::fence_async_smem();
         tc::tc_fence_before();
         __syncthreads();
@@ -247,26 +209,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        {   // Delta^T (lane j) -> bf16 row tile; scale the fp32 state by gC along its key columns
-            const int j = tid;
-            float v[32];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                tc::tmem_ld32(lane_base + TM_D + 32 * h2, v);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(DT, D, j, 4 * h2 + g, v + 8 * g);
-            }
-#pragma unroll 1
-            for (int i0 = 0; i0 < D; i0 += 32) {
-                tc::tmem_ld32(lane_base + TM_S + i0, v);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
-                tc::tmem_st32(lane_base + TM_S + i0, v);
-            }
-            tc::tmem_wait_st();
-        }
+        tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);       // Delta^T (lane j) -> bf16 rows
+        tmem_scale_columns(lane_base + TM_S, sGC);               // S^T <- S^T Diag(gC)
         tc::fence_async_smem();
         tc::tc_fence_before();
         __syncthreads();
@@ -300,19 +244,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 }
             }
         }
-        {   // new state: bf16 copy for the next chunk's operands (and the saved image)
-            if (states && tid == 0) tc::bulk_wait_read();
-            __syncthreads();
-            const int j = tid;
-            float v[32];
-#pragma unroll 1
-            for (int i0 = 0; i0 < D; i0 += 32) {
-                tc::tmem_ld32(lane_base + TM_S + i0, v);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
-            }
-        }
+        // new state: bf16 copy for the next chunk's operands (and the saved image)
+        if (states && tid == 0) tc::bulk_wait_read();
+        __syncthreads();
+        tmem_to_tile_rows<128>(lane_base + TM_S, STt, tid);
         tc::fence_async_smem();
         tc::tc_fence_before();
         __syncthreads();

@@ -57,7 +57,7 @@ inline bool tc_path(gdn2_dtype dt, int Dk, int Dv, int chunk) {
     return dt == GDN2_BF16 && Dk == TC_D && Dv == TC_D && chunk == TC_C;
 }
 // Whether the tensor-core backward is built.
-constexpr bool kTcBackward = false;
+constexpr bool kTcBackward = true;
 // Whether training (fwd with saved states + bwd) runs on the tensor-core kernels.
 inline bool tc_train_path(gdn2_dtype dt, int Dk, int Dv, int chunk) {
     return kTcBackward && tc_path(dt, Dk, Dv, chunk);
