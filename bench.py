@@ -98,9 +98,12 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def make_host_inputs(rank):
+def make_host_inputs(rank, B=None, T=None):
+    import dataclasses
     from linear_attention_delta_gdn_b200.inputs import WORKLOADS, make_inputs
     wl = WORKLOADS[WORKLOAD]
+    if B or T:
+        wl = dataclasses.replace(wl, name="%s-B%d-T%d" % (wl.name, B or wl.B, T or wl.T), B=B or wl.B, T=T or wl.T)
     return wl, make_inputs(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, wl.seed + 7919 * rank, wl.dtype, with_do=True)
 
 
@@ -169,6 +172,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--B", type=int, default=None, help="override the batch size (small profiling cases)")
+    ap.add_argument("--T", type=int, default=None, help="override the sequence length (small profiling cases)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -191,7 +196,7 @@ def main():
         dist.barrier()
     L = binding.lib()
 
-    wl, xh = make_host_inputs(rank)
+    wl, xh = make_host_inputs(rank, args.B, args.T)
     B, T, H, Dk, Dv, chunk = wl.B, wl.T, wl.H, wl.Dk, wl.Dv, wl.chunk
     names = ("q", "k", "v", "log_alpha", "b", "w")
     pinned = {n: t.pin_memory() for n, t in xh.items()}
@@ -266,7 +271,7 @@ def main():
             h_.copy_(t, non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e_start.elapsed_time(e_end) / args.e2e_steps
+    e2e_ms = e_start.elapsed_time(e_end) / max(1, args.e2e_steps)
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -300,7 +305,7 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "Dk": Dk, "Dv": Dv, "chunk": chunk,
+                "config": {"workload": wl.name, "B": B, "T": T, "H": H, "Dk": Dk, "Dv": Dv, "chunk": chunk,
                            "global_batch": world * B, "seq_len": T,
                            "parallelism": "dp%d (independent batches, no collective)" % world,
                            "l2": "inputs larger than L2 (%.0f MB read per step)" % (h2d / 1e6),

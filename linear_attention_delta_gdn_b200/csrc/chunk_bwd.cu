@@ -4,22 +4,24 @@
 // "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention" (arXiv
 // abstract) names a gate-aware backward that keeps training parallel; the page
 // prints no equations. The adjoint of the chunk form (see chunk_common.cuh), for
-// one chunk with start state S, next-state gradient dS' and output gradient dO:
-//   dDelta = Kh dS' + P^T dO                         (P = tril(Qt Kt^T))
-//   dS     = Diag(gC) dS' + Qt^T dO - Wm^T dDelta    -> gradient of the chunk-start state
+// one chunk with start state S, S' = Diag(gC) (S + Kt^T Delta), next-state gradient dS'
+// and output gradient dO; write dZ = Diag(gC) dS' (the gradient of S + Kt^T Delta):
+//   dDelta = Kt dZ + P^T dO                          (P = tril(Qt Kt^T))
+//   dS     = dZ + Qt^T dO - Wm^T dDelta              -> gradient of the chunk-start state
 //   dU     = T^T dDelta                              -> dv = dU*w, dw = dU*v
 //   dP     = (dO Delta^T) * incl,  dA = -(dU Delta^T) * strict
 //   dQt    = dO S^T + dP Kt,       dEt = -dU S^T + dA Kt
-//   dKt    = dP^T Qt + dA^T Et,    dKh = Delta dS'^T,  dgC = rowsum(dS' * S)
+//   dKt    = dP^T Qt + dA^T Et + Delta dZ^T
 // (dA uses T^T dT T^T = dU Delta^T, since dT = dDelta (U - Et S)^T = dDelta Delta^T (I + A)^T.)
-// Gate chain through g = exp(cumsum log_alpha):
-//   dq = g*dQt;  dE = g*dEt;  db = dE*k;  dk = dKt/g + (gC/g)*dKh + dE*b
-//   dG = Qt*dQt + Et*dEt - Kt*dKt - Kh*dKh;  dG[last] += sum_t Kh*dKh + gC*dgC
-//   dlog_alpha = reverse in-chunk cumsum of dG
+// Gate chain through g = exp(G), G = in-chunk cumsum of log_alpha:
+//   dq = g*dQt;  dE = g*dEt;  db = dE*k;  dk = dKt/g + dE*b
+//   dG_t = Qt*dQt + Et*dEt - Kt*dKt;  the last position also gets
+//   E = rowsum(dZ * S) + sum_t Kt_t * (Delta dZ^T)_t   (the dependence of S' on gC)
+//   dlog_alpha_t = sum_{tau >= t} dG_tau + E
 //
 // Two kernels:
 //   reverse_state_kernel  one CTA per (batch, head) walks the chunks backwards carrying
-//                         dS^T in TMEM (fp32) and stores each chunk's dS' as a bf16 image;
+//                         dS^T in TMEM (fp32) and stores each chunk's dZ^T as a bf16 image;
 //   chunk_grad_kernel     one CTA per (batch, head, chunk) computes every gradient of the
 //                         chunk from the saved S, dS', the inputs and dout.
 #include <cuda.h>
@@ -41,19 +43,19 @@ __device__ unsigned int g_bwd_error;
 
 namespace rs {
 constexpr uint32_t OFF_QE = 0;           // rows 0..63: b -> Et, rows 64..127: q -> Qt
-constexpr uint32_t OFF_KH = 32768;       // k -> Kh
+constexpr uint32_t OFF_KH = 32768;       // k
 constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
 constexpr uint32_t OFF_DO = 65536;       // dout
-constexpr uint32_t OFF_WW = 81920;       // Wm
-constexpr uint32_t OFF_ST = 98304;       // dS'^T (bf16)
+constexpr uint32_t OFF_WW = 81920;       // solve temporaries, then Wm
+constexpr uint32_t OFF_ST = 98304;       // dZ^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16) | fp32 A scratch
-constexpr uint32_t OFF_TF = 147456;      // fp32 T
-constexpr uint32_t OFF_TT = 163840;      // T (bf16) | solve temporaries
+constexpr uint32_t OFF_TF = 147456;      // fp32 T | prep scan scratch
+constexpr uint32_t OFF_TT = 163840;      // T (bf16)
 constexpr uint32_t OFF_PP = 172032;      // P (bf16)
 constexpr uint32_t OFF_GC = 180224;
 constexpr uint32_t OFF_BAR = 180736;
 constexpr uint32_t SMEM_BYTES = 180800 + 1024;
-constexpr uint32_t TM_S = 0, TM_AP = 128, TM_W = 192, TM_D = 256, TM_COLS = 512;
+constexpr uint32_t TM_S = 0, TM_AP = 128, TM_D = 192, TM_W = 256, TM_COLS = 512;
 constexpr uint32_t LOAD_BYTES = 5 * 64 * 128 * 2;
 }  // namespace rs
 
@@ -64,7 +66,7 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
                      float* __restrict__ dS0, unsigned char* __restrict__ dstates, int T, int H) {
     using namespace rs;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     unsigned char* QE = sm + OFF_QE;
     unsigned char* KH = sm + OFF_KH;
     unsigned char* KT = sm + OFF_KT;
@@ -74,7 +76,7 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     unsigned char* DT = sm + OFF_DT;
     float* sA = reinterpret_cast<float*>(sm + OFF_DT);
     float* sTf = reinterpret_cast<float*>(sm + OFF_TF);
-    float* sX = reinterpret_cast<float*>(sm + OFF_TT);
+    float* sX = reinterpret_cast<float*>(sm + OFF_WW);   // Wm is written after the solve
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
@@ -83,7 +85,7 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
     int* abort_flag = reinterpret_cast<int*>(sm + OFF_BAR + 20);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x % H, b = blockIdx.x / H;
     const size_t head = blockIdx.x;
     const int nc = (T + C - 1) / C;
@@ -123,21 +125,18 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] = dST ? dST[(head * D + i0 + u) * D + j] : 0.f;
             tc::tmem_st32(lane_base + TM_S + i0, v);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
         }
         tc::tmem_wait_st();
     }
-    tc::fence_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
 
-    const uint32_t sQE = tc::smem_u32(QE), sKH = tc::smem_u32(KH), sKT = tc::smem_u32(KT),
-                   sDO = tc::smem_u32(DO), sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt),
-                   sDT = tc::smem_u32(DT), sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
+    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sDO = tc::smem_u32(DO),
+                   sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
+                   sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
     constexpr uint32_t ID_M1 = tc::idesc_bf16(128, 64, false, false);
-    constexpr uint32_t ID_M2 = tc::idesc_bf16(128, 64, true, false);
+    constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
     constexpr uint32_t ID_N1a = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_N1b = tc::idesc_bf16(128, 64, true, true);
     constexpr uint32_t ID_N2a = tc::idesc_bf16(128, 128, true, true);
@@ -149,19 +148,40 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         ph_mma ^= 1;
         tc::tc_fence_after();
     };
+    auto sync_for_mma = [&]() {
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+    };
 
     for (int c = nc - 1; c >= 0; --c) {
-        // the tile holds dS_{c+1}^T: keep its image for the gradient kernel
-        if (tid == 0) {
-            tc::bulk_store(dstates + (head * nc + c) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
-            tc::bulk_commit();
-        }
         if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
         ph_load ^= 1;
 
-        gate_prep(QE, KH, KT, nullptr, nullptr, sGC, tid, true, false);
-        tc::fence_async_smem();
+        gate_prep(QE, KH, KT, nullptr, nullptr, sGC, sTf, tid, true, false);
+        // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
+        if (tid == 0) tc::bulk_wait_read();
         __syncthreads();
+        {
+            const int j = tid;
+            float v[32];
+#pragma unroll 1
+            for (int i0 = 0; i0 < D; i0 += 32) {
+                tc::tmem_ld32(lane_base + TM_S + i0, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
+                tc::tmem_st32(lane_base + TM_S + i0, v);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+            }
+            tc::tmem_wait_st();
+        }
+        sync_for_mma();
+        if (tid == 0) {     // keep the dZ^T image of this chunk for the gradient kernel
+            tc::bulk_store(dstates + (head * nc + c) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
+            tc::bulk_commit();
+        }
 
         // [A; P] = [Et; Qt] Kt^T
         if (tid == 0) {
@@ -176,42 +196,28 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         tc::tc_fence_before();
         __syncthreads();
         solve_unit_lower(sA, sTf, sX, TT, tid);
-        tc::fence_async_smem();
-        __syncthreads();
+        sync_for_mma();
 
-        // Wm^T = Et^T T^T
+        // Wm = T Et (M=64) ;  dDelta^T = dZ^T Kt^T + dO^T P
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_W, tc::desc_mn(sQE, 2 * C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M2, kk > 0);
-            tc::mma_commit(bar_mma);
-        }
-        wait_mma();
-        tmem_to_tile_transposed(lane_base + TM_W, WW, tid);
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // dDelta^T = dS'^T Kh^T + dO^T P
-        if (tid == 0) {
-            tc::tc_fence_after();
+                tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), ID_M2, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sKH, C, 0, kk), ID_N1a, kk > 0);
+                tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_N1a, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16(tmem + TM_D, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), ID_N1b, 1);
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);
-        tmem_scale_columns(lane_base + TM_S, sGC);            // dS'^T Diag(gC)
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
+        tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);    // Wm rows
+        tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);      // dDelta^T rows
+        sync_for_mma();
 
-        // dS^T = dS'^T Diag(gC) + dO^T Qt - dDelta^T Wm
+        // dS^T = dZ^T + dO^T Qt - dDelta^T Wm
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
@@ -223,10 +229,6 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         }
         wait_mma();
         if (tid == 0 && c > 0) issue_loads(c - 1);
-        if (tid == 0) tc::bulk_wait_read();
-        __syncthreads();
-        tmem_to_tile_rows<128>(lane_base + TM_S, STt, tid);
-        tc::fence_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
@@ -257,22 +259,29 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 
 namespace cg {
 constexpr uint32_t OFF_QE = 0;           // rows 0..63: b -> Et, rows 64..127: q -> Qt
-constexpr uint32_t OFF_KH = 32768;       // k -> Kh
+constexpr uint32_t OFF_KH = 32768;       // k (kept)
 constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
-constexpr uint32_t OFF_UU = 65536;       // v -> U, later dU^T [128 x 64]
-constexpr uint32_t OFF_WW = 81920;       // w -> Wm
+constexpr uint32_t OFF_UU = 65536;       // v -> U, later dU rows [t][j]
+constexpr uint32_t OFF_WW = 81920;       // w -> solve temporaries -> Wm rows, later b (reloaded)
 constexpr uint32_t OFF_DO = 98304;       // dout
 constexpr uint32_t OFF_ST = 114688;      // S^T image (chunk start)
-constexpr uint32_t OFF_DS = 147456;      // dS'^T image (chunk end)
+constexpr uint32_t OFF_DS = 147456;      // dZ^T image
 constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64] | fp32 A scratch
 constexpr uint32_t OFF_DDT = 196608;     // dDelta^T [128 x 64] | fp32 T
-constexpr uint32_t OFF_TT = 212992;      // T | solve temporaries, later dA^T [64 x 64]
+constexpr uint32_t OFF_TT = 212992;      // T, later dA^T [64 x 64]
 constexpr uint32_t OFF_PP = 221184;      // P, later dP^T [64 x 64]
 constexpr uint32_t OFF_GC = 229376;
 constexpr uint32_t OFF_BAR = 229888;
 constexpr uint32_t SMEM_BYTES = 229952 + 1024;
-constexpr uint32_t TM_AP = 0, TM_W = 64, TM_D = 128, TM_DD = 192, TM_DU = 256, TM_G1 = 320, TM_G2 = 384,
-                   TM_G3 = 448, TM_COLS = 512;
+// TMEM columns (M=64 accumulators use lanes 0-15 of each 32-lane quarter)
+constexpr uint32_t TM_AP = 0,      // [A; P], later dP^T (M=64)
+    TM_W = 64,                     // Wm (M=64, 128 columns), later dA^T (M=64, 64 columns)
+    TM_D = 192,                    // Ut^T -> Delta^T, later G4 = (Delta dZ^T)^T
+    TM_DD = 256,                   // dDelta^T, later G3 = dKt^T (P and A paths)
+    TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
+    TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,
+    TM_GV = 448,                   // G[t] per key channel (cumulative log-decay)
+    TM_COLS = 512;
 constexpr uint32_t LOAD_BYTES = 7 * 64 * 128 * 2 + 2 * (uint32_t)TC_STATE_BYTES;
 }  // namespace cg
 
@@ -280,15 +289,14 @@ __global__ void __launch_bounds__(NT, 1)
 chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mla,
                   const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
-                  const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16* __restrict__ k_g,
-                  const __nv_bfloat16* __restrict__ v_g, const __nv_bfloat16* __restrict__ la_g,
-                  const __nv_bfloat16* __restrict__ b_g, const __nv_bfloat16* __restrict__ w_g,
-                  __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                  __nv_bfloat16* __restrict__ dla, __nv_bfloat16* __restrict__ db, __nv_bfloat16* __restrict__ dw,
+                  const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16* __restrict__ v_g,
+                  const __nv_bfloat16* __restrict__ w_g, __nv_bfloat16* __restrict__ dq,
+                  __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, __nv_bfloat16* __restrict__ dla,
+                  __nv_bfloat16* __restrict__ db, __nv_bfloat16* __restrict__ dw,
                   const unsigned char* __restrict__ states, const unsigned char* __restrict__ dstates, int T, int H) {
     using namespace cg;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     unsigned char* QE = sm + OFF_QE;
     unsigned char* KH = sm + OFF_KH;
     unsigned char* KT = sm + OFF_KT;
@@ -301,13 +309,14 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     unsigned char* DDT = sm + OFF_DDT;
     float* sA = reinterpret_cast<float*>(sm + OFF_DT);
     float* sTf = reinterpret_cast<float*>(sm + OFF_DDT);
-    float* sX = reinterpret_cast<float*>(sm + OFF_TT);
+    float* sX = reinterpret_cast<float*>(sm + OFF_WW);   // w is consumed by the prep, Wm written after M2
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_load + 1;
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
+    uint64_t* bar_b = bar_load + 2;
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 24);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
@@ -320,6 +329,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     if (tid == 0) {
         tc::mbar_init(bar_load, 1);
         tc::mbar_init(bar_mma, 1);
+        tc::mbar_init(bar_b, 1);
         tc::fence_mbar_init();
         tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
         tma_tile(QE, 2 * C, 0, &mb, b, h, t0, bar_load);
@@ -348,16 +358,20 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         ph_mma ^= 1;
         tc::tc_fence_after();
     };
+    auto sync_for_mma = [&]() {
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+    };
 
-    const uint32_t sQE = tc::smem_u32(QE), sKH = tc::smem_u32(KH), sKT = tc::smem_u32(KT),
-                   sUU = tc::smem_u32(UU), sWW = tc::smem_u32(WW), sDO = tc::smem_u32(DO),
-                   sST = tc::smem_u32(STt), sDS = tc::smem_u32(DS), sDT = tc::smem_u32(DT),
-                   sDDT = tc::smem_u32(DDT), sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
+    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sUU = tc::smem_u32(UU),
+                   sWW = tc::smem_u32(WW), sDO = tc::smem_u32(DO), sST = tc::smem_u32(STt),
+                   sDS = tc::smem_u32(DS), sDT = tc::smem_u32(DT), sDDT = tc::smem_u32(DDT),
+                   sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
-    // ---- factors, [A; P], T
-    gate_prep(QE, KH, KT, UU, WW, sGC, tid, true, true);
-    tc::fence_async_smem();
-    __syncthreads();
+    // ---- factors (G kept in TMEM), [A; P], T
+    gate_prep_cols(QE, KH, KT, UU, WW, sGC, tid, true, true, lane_base + TM_GV);
+    sync_for_mma();
     if (tid == 0) {
         tc::tc_fence_after();
         constexpr uint32_t id = tc::idesc_bf16(128, 64, false, false);
@@ -371,27 +385,25 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     tc::tc_fence_before();
     __syncthreads();
     solve_unit_lower(sA, sTf, sX, TT, tid);
-    tc::fence_async_smem();
-    __syncthreads();
+    sync_for_mma();
 
-    // ---- Wm^T = Et^T T^T ; Ut^T = U^T T^T
+    // ---- Wm = T Et (M=64) ; Ut^T = U^T T^T
     if (tid == 0) {
         tc::tc_fence_after();
-        constexpr uint32_t id = tc::idesc_bf16(128, 64, true, false);
+        constexpr uint32_t id_w = tc::idesc_bf16(64, 128, false, true);
+        constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            tc::mma_bf16(tmem + TM_W, tc::desc_mn(sQE, 2 * C, 0, kk), tc::desc_k(sTT, C, 0, kk), id, kk > 0);
-            tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), id, kk > 0);
+            tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), id_w, kk > 0);
+            tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), id_u, kk > 0);
         }
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    tmem_to_tile_transposed(lane_base + TM_W, WW, tid);
-    tc::fence_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
+    tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);       // Wm rows
+    sync_for_mma();
 
-    // ---- Delta^T = Ut^T - S^T Wm^T ;  dDelta^T = dS'^T Kh^T + dO^T P
+    // ---- Delta^T = Ut^T - S^T Wm^T ;  dDelta^T = dZ^T Kt^T + dO^T P
     if (tid == 0) {
         tc::tc_fence_after();
         constexpr uint32_t id_neg = tc::idesc_bf16(128, 64, false, false, true);
@@ -400,7 +412,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWW, C, 0, kk), id_neg, 1);
-            tc::mma_bf16(tmem + TM_DD, tc::desc_k(sDS, D, 0, kk), tc::desc_k(sKH, C, 0, kk), id_kk, kk > 0);
+            tc::mma_bf16(tmem + TM_DD, tc::desc_k(sDS, D, 0, kk), tc::desc_k(sKT, C, 0, kk), id_kk, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -408,61 +420,80 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::mma_commit(bar_mma);
     }
     wait_mma();
+    if (tid == 0) {     // Wm is consumed: bring b back for the gate chain
+        tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
+        tma_tile(WW, C, 0, &mb, b, h, t0, bar_b);
+    }
     tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);      // Delta^T [j][t]
     tmem_to_tile_rows<64>(lane_base + TM_DD, DDT, tid);    // dDelta^T [j][t]
-    tc::fence_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
+    sync_for_mma();
 
-    // ---- dU^T = dDelta^T T
+    // ---- dU = T^T dDelta (M=64)
     if (tid == 0) {
         tc::tc_fence_after();
-        constexpr uint32_t id = tc::idesc_bf16(128, 64, false, true);
+        constexpr uint32_t id = tc::idesc_bf16(64, 128, true, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(tmem + TM_DU, tc::desc_k(sDDT, D, 0, kk), tc::desc_mn(sTT, C, 0, kk), id, kk > 0);
+            tc::mma_bf16(tmem + TM_DU, tc::desc_mn(sTT, C, 0, kk), tc::desc_k(sDDT, D, 0, kk), id, kk > 0);
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    {   // dv = dU*w, dw = dU*v ; keep dU^T as a bf16 row tile
-        const int j = tid;
+    {   // dv = dU*w, dw = dU*v (rows t, 16-byte accesses); keep dU as a bf16 row tile
+        const int t = m64_row(warp, lane);
+        const bool row_ok = lane < 16 && t < L;
         float v[32];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            tc::tmem_ld32(lane_base + TM_DU + 32 * h2, v);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            tc::tmem_ld32(lane_base + TM_DU + c0, v);
             tc::tmem_wait_ld();
+            if (lane < 16) {
 #pragma unroll
-            for (int g = 0; g < 4; ++g) tc::st_row8(UU, D, j, 4 * h2 + g, v + 8 * g);
-#pragma unroll 4
-            for (int u = 0; u < 32; ++u) {
-                const int t = 32 * h2 + u;
-                if (t < L) {
-                    const size_t off = tok_off(b, t0 + t, h, T, H, D) + j;
-                    dv[off] = __float2bfloat16_rn(v[u] * __bfloat162float(w_g[off]));
-                    dw[off] = __float2bfloat16_rn(v[u] * __bfloat162float(v_g[off]));
+                for (int g = 0; g < 4; ++g) tc::st_row8(UU, C, t, (c0 >> 3) + g, v + 8 * g);
+            }
+            if (row_ok) {
+                const size_t off = tok_off(b, t0 + t, h, T, H, D) + c0;
+                const uint4* wp = reinterpret_cast<const uint4*>(w_g + off);
+                const uint4* vp = reinterpret_cast<const uint4*>(v_g + off);
+                uint4 wv[4], vv[4];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) { wv[g] = wp[g]; vv[g] = vp[g]; }
+                uint4* dvp = reinterpret_cast<uint4*>(dv + off);
+                uint4* dwp = reinterpret_cast<uint4*>(dw + off);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv[g]);
+                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv[g]);
+                    uint32_t ov[4], ow[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 wf = __bfloat1622float2(w2[e]), vf = __bfloat1622float2(v2[e]);
+                        const float d0 = v[8 * g + 2 * e], d1 = v[8 * g + 2 * e + 1];
+                        ov[e] = tc::pack_bf16x2(d0 * wf.x, d1 * wf.y);
+                        ow[e] = tc::pack_bf16x2(d0 * vf.x, d1 * vf.y);
+                    }
+                    dvp[g] = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+                    dwp[g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
         }
     }
-    tc::fence_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
+    sync_for_mma();
 
     // ---- dP^T = Delta dO^T (M=64), dA^T = -Delta dU^T (M=64)
     if (tid == 0) {
         tc::tc_fence_after();
         constexpr uint32_t id_p = tc::idesc_bf16(64, 64, true, false);
-        constexpr uint32_t id_a = tc::idesc_bf16(64, 64, true, true, true);
+        constexpr uint32_t id_a = tc::idesc_bf16(64, 64, true, false, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             tc::mma_bf16(tmem + TM_AP, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sDO, C, 0, kk), id_p, kk > 0);
-            tc::mma_bf16(tmem + TM_W, tc::desc_mn(sDT, D, 0, kk), tc::desc_mn(sUU, D, 0, kk), id_a, kk > 0);
+            tc::mma_bf16(tmem + TM_W, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sUU, C, 0, kk), id_a, kk > 0);
         }
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    {   // M=64 accumulators: row s lives in lane (s % 16) + 32 (s / 16); lanes 16..31 of a warp hold nothing
-        const int s = 16 * warp + (lane & 15);
+    {   // M=64 accumulators: rows s = 16 warp + lane (lanes < 16)
+        const int s = m64_row(warp, lane);
         float v[32];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -487,21 +518,20 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
             }
         }
     }
-    tc::fence_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
+    sync_for_mma();
 
-    // ---- dQt^T = S dO^T + Kt^T dP^T ; dEt^T = -S dU^T + Kt^T dA^T ; dKt^T = Qt^T dP + Et^T dA ; dKh^T = dS' Delta^T
+    // ---- G1 = dQt^T = S dO^T + Kt^T dP^T ; G2 = dEt^T = -S dU^T + Kt^T dA^T
+    //      G3 = Qt^T dP + Et^T dA ;        G4 = dZ Delta^T          (all [key channel i][token t])
     if (tid == 0) {
         tc::tc_fence_after();
         constexpr uint32_t id_mk = tc::idesc_bf16(128, 64, true, false);
+        constexpr uint32_t id_mk_neg = tc::idesc_bf16(128, 64, true, false, true);
         constexpr uint32_t id_mm = tc::idesc_bf16(128, 64, true, true);
-        constexpr uint32_t id_mm_neg = tc::idesc_bf16(128, 64, true, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             tc::mma_bf16(tmem + TM_G1, tc::desc_mn(sST, D, 0, kk), tc::desc_k(sDO, C, 0, kk), id_mk, kk > 0);
-            tc::mma_bf16(tmem + TM_G2, tc::desc_mn(sST, D, 0, kk), tc::desc_mn(sUU, D, 0, kk), id_mm_neg, kk > 0);
-            tc::mma_bf16(tmem + TM_D, tc::desc_mn(sDS, D, 0, kk), tc::desc_mn(sDT, D, 0, kk), id_mm, kk > 0);
+            tc::mma_bf16(tmem + TM_G2, tc::desc_mn(sST, D, 0, kk), tc::desc_k(sUU, C, 0, kk), id_mk_neg, kk > 0);
+            tc::mma_bf16(tmem + TM_G4, tc::desc_mn(sDS, D, 0, kk), tc::desc_mn(sDT, D, 0, kk), id_mm, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -515,64 +545,70 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::mma_commit(bar_mma);
     }
 
-    // dgC[i] = sum_j dS'[i][j] S[i][j] (both images hold row j = value channel)
+    // rowsum(dZ * S) for key channel i (both images hold row j = value channel)
     const int i = tid;
-    float dgC = 0.f;
+    float E = 0.f;
+    {
+        float e2 = 0.f;
 #pragma unroll 8
-    for (int j = 0; j < D; ++j) {
-        const uint32_t off = tc::tile_off(D, j, i);
-        dgC += tc::ld_bf16(DS, off) * tc::ld_bf16(STt, off);
+        for (int j = 0; j < D; j += 2) {
+            E += tc::ld_bf16(DS, tc::tile_off(D, j, i)) * tc::ld_bf16(STt, tc::tile_off(D, j, i));
+            e2 += tc::ld_bf16(DS, tc::tile_off(D, j + 1, i)) * tc::ld_bf16(STt, tc::tile_off(D, j + 1, i));
+        }
+        E += e2;
     }
     wait_mma();
+    ok = tc::mbar_wait(bar_b, 0) && ok;
 
-    // ---- gate chain, thread = key channel i.
-    // dlog_alpha_t = sum_{tau >= t} dG_tau + E with the chunk-end term
-    // E = sum_tau Kh_tau dKh_tau + gC dgC (added at the last position, so every t sees it).
-    // Pass 1: G_C and E. Pass 2: tokens in reverse, suffix sums of dG.
-    const float gC = sGC[i];
-    float GC = 0.f, E = gC * dgC;
+    // ---- gate chain, thread = key channel i: E += sum_t Kt G4, then tokens in reverse
+    const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
+    const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
+    const uint32_t chk = (uint32_t)((i & 63) >> 3);
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
         float g4[16];
-        tc::tmem_ld16(lane_base + TM_D + 16 * q4, g4);
+        tc::tmem_ld16(lane_base + TM_G4 + 16 * q4, g4);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const int t = 16 * q4 + u;
-            if (t < L) GC += __bfloat162float(la_g[tok_off(b, t0 + t, h, T, H, D) + i]);
-            E += tc::ld_bf16(KH, tc::tile_off(C, t, i)) * g4[u];
+            const uint32_t t = (uint32_t)(16 * q4 + u);
+            E += tc::ld_bf16(KT, col64 + t * 128 + ((chk ^ (t & 7)) << 4)) * g4[u];
         }
     }
-    float G = GC, suffix = 0.f;
+    float suffix = 0.f;
 #pragma unroll 1
     for (int q4 = 3; q4 >= 0; --q4) {
-        float g1[16], g2[16], g3[16], g4[16];
+        float g1[16], g2[16], g3[16], g4[16], gv[16];
         tc::tmem_ld16(lane_base + TM_G1 + 16 * q4, g1);
         tc::tmem_ld16(lane_base + TM_G2 + 16 * q4, g2);
         tc::tmem_ld16(lane_base + TM_G3 + 16 * q4, g3);
-        tc::tmem_ld16(lane_base + TM_D + 16 * q4, g4);
+        tc::tmem_ld16(lane_base + TM_G4 + 16 * q4, g4);
+        tc::tmem_ld16(lane_base + TM_GV + 16 * q4, gv);
         tc::tmem_wait_ld();
+        float qt[16], et[16], kt[16], kk[16], bb[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const uint32_t t = (uint32_t)(16 * q4 + u);
+            const uint32_t sw = t * 128 + ((chk ^ (t & 7)) << 4);
+            qt[u] = tc::ld_bf16(QE, col128 + C * 128 + sw);
+            et[u] = tc::ld_bf16(QE, col128 + sw);
+            kt[u] = tc::ld_bf16(KT, col64 + sw);
+            kk[u] = tc::ld_bf16(KH, col64 + sw);
+            bb[u] = tc::ld_bf16(WW, col64 + sw);
+        }
 #pragma unroll
         for (int u = 15; u >= 0; --u) {
             const int t = 16 * q4 + u;
-            const bool valid = t < L;
-            const size_t off = tok_off(b, t0 + (valid ? t : 0), h, T, H, D) + i;
-            // here G = G_t (cumulative log-decay through token t)
-            const float g = fast_exp(G), ig = fast_exp(-G);
-            const float qt = tc::ld_bf16(QE, tc::tile_off(2 * C, C + t, i));
-            const float et = tc::ld_bf16(QE, tc::tile_off(2 * C, t, i));
-            const float kt = tc::ld_bf16(KT, tc::tile_off(C, t, i));
-            const float kh = tc::ld_bf16(KH, tc::tile_off(C, t, i));
-            suffix += qt * g1[u] + et * g2[u] - kt * g3[u] - kh * g4[u];
-            if (valid) {
+            const float g = fast_exp(gv[u]), ig = fast_exp(-gv[u]);
+            const float dKt = g3[u] + g4[u];
+            suffix += qt[u] * g1[u] + et[u] * g2[u] - kt[u] * dKt;
+            if (t < L) {
+                const size_t off = tok_off(b, t0 + t, h, T, H, D) + i;
                 const float dE = g * g2[u];
-                const float kk = __bfloat162float(k_g[off]);
-                const float bb = __bfloat162float(b_g[off]);
                 dq[off] = __float2bfloat16_rn(g * g1[u]);
-                db[off] = __float2bfloat16_rn(dE * kk);
-                dk[off] = __float2bfloat16_rn(g3[u] * ig + gC * ig * g4[u] + dE * bb);
+                db[off] = __float2bfloat16_rn(dE * kk[u]);
+                dk[off] = __float2bfloat16_rn(dKt * ig + dE * bb[u]);
                 dla[off] = __float2bfloat16_rn(suffix + E);
-                G -= __bfloat162float(la_g[off]);
             }
         }
     }
@@ -610,11 +646,10 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const dim3 grid(d.nchunks(), d.B * d.H);
     chunk_grad_kernel<<<grid, NT, cg::SMEM_BYTES, s>>>(
-        mq, mk, mv, mla, mb, mw, mdo, static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v),
-        static_cast<const __nv_bfloat16*>(a.la), static_cast<const __nv_bfloat16*>(a.b),
-        static_cast<const __nv_bfloat16*>(a.w), static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk),
-        static_cast<__nv_bfloat16*>(a.dv), static_cast<__nv_bfloat16*>(a.dla), static_cast<__nv_bfloat16*>(a.db),
-        static_cast<__nv_bfloat16*>(a.dw), a.states, a.dstates, d.T, d.H);
+        mq, mk, mv, mla, mb, mw, mdo, static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.w),
+        static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv),
+        static_cast<__nv_bfloat16*>(a.dla), static_cast<__nv_bfloat16*>(a.db), static_cast<__nv_bfloat16*>(a.dw),
+        a.states, a.dstates, d.T, d.H);
     return cudaGetLastError();
 }
 

@@ -11,6 +11,8 @@
 //   Qt = g*q,  Kh = (gC/g)*k = gC*Kt,  U = w*v
 //   A  = strictly_lower(Et Kt^T),  T = (I + A)^{-1},  Wm = T Et,  Ut = T U
 //   Delta = Ut - Wm S;   O = Qt S + tril(Qt Kt^T) Delta;   S' = Diag(gC) S + Kh^T Delta
+// The kernels apply the last step as S' = Diag(gC) (S + Kt^T Delta) (Kh = gC*Kt), scaling the
+// fp32 accumulator after the contraction, so no Kh tile is formed.
 // Rows past the end of the sequence are zero-filled by TMA: they give zero
 // factors, a flat cumulative decay and an identity block of T, so a ragged
 // last chunk needs no special case except masked stores.
@@ -65,37 +67,111 @@ __device__ __forceinline__ void tma_tile(unsigned char* dst, int R, int dst_row0
     tc::tma_load_4d(dst + R * 128 + dst_row0 * 128, map, 64, h, t0, b, bar);
 }
 
-// Gate preparation, one thread per channel i (= threadIdx.x):
-//   reads q (rows 64.. of QE), b (rows 0.. of QE), k (KH), log_alpha (KT), v (UU), w (WW)
-//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT, Kh -> KH, U -> UU,
-//   gC[i] -> gC_out. Each element is read and rewritten by the same thread.
-// With want_u = false, v/w are left untouched.
-__device__ __forceinline__ void gate_prep(unsigned char* QE, unsigned char* KH, unsigned char* KT,
+// Gate preparation, channel-major variant: one thread per key/value channel i (= threadIdx.x),
+// tokens in blocks of 8 (loads of a block are issued together, then its stores):
+//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
+//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127 (want_q),
+//          Kt = k/g -> KT, U = w*v -> UU (want_u); KH keeps k.
+//   g = exp(G), G = inclusive cumsum of log_alpha. gC[i] = g at the last row.
+//   If tmem_g != 0, G[t][i] is also stored to TMEM (lane i, columns t) for later use.
+__device__ __forceinline__ void gate_prep_cols(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
                                           unsigned char* UU, const unsigned char* WW, float* gC_out, int i,
-                                          bool want_q, bool want_u) {
+                                          bool want_q, bool want_u, uint32_t tmem_g = 0) {
+    // byte offset of (row 8*tb + u, channel i) in a 64-row tile, and in the 128-row QE tile
+    const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
+    const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
+    const uint32_t chunk = (uint32_t)((i & 63) >> 3);
     float G = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < C; ++t) G += tc::ld_bf16(KT, tc::tile_off(C, t, i));
-    const float gC = fast_exp(G);
-    gC_out[i] = gC;
-    G = 0.f;
-#pragma unroll 4
-    for (int t = 0; t < C; ++t) {
-        const uint32_t o64 = tc::tile_off(C, t, i);
-        G += tc::ld_bf16(KT, o64);
-        const float g = fast_exp(G), ig = fast_exp(-G);
-        const float kk = tc::ld_bf16(KH, o64);
-        const uint32_t oe = tc::tile_off(2 * C, t, i);
-        const float bb = tc::ld_bf16(QE, oe);
-        tc::st_bf16(QE, oe, g * bb * kk);                    // Et
-        if (want_q) {
-            const uint32_t oq = tc::tile_off(2 * C, C + t, i);
-            tc::st_bf16(QE, oq, g * tc::ld_bf16(QE, oq));     // Qt
+#pragma unroll 1
+    for (int tb2 = 0; tb2 < C / 16; ++tb2) {
+        float gvals[16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int tb = 2 * tb2 + half;
+            float la[8], kk[8], bb[8], qq[8], vv[8], ww[8];
+            uint32_t o64[8], o128[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t row = (uint32_t)(8 * tb + u);
+                const uint32_t sw = ((chunk ^ (uint32_t)u) << 4);
+                o64[u] = col64 + row * 128 + sw;
+                o128[u] = col128 + row * 128 + sw;
+                la[u] = tc::ld_bf16(KT, o64[u]);
+                kk[u] = tc::ld_bf16(KH, o64[u]);
+                bb[u] = tc::ld_bf16(QE, o128[u]);
+                if (want_q) qq[u] = tc::ld_bf16(QE, o128[u] + C * 128);
+                if (want_u) { vv[u] = tc::ld_bf16(UU, o64[u]); ww[u] = tc::ld_bf16(WW, o64[u]); }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                G += la[u];
+                gvals[half * 8 + u] = G;
+                const float g = fast_exp(G), ig = fast_exp(-G);
+                tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);                 // Et
+                if (want_q) tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);    // Qt
+                tc::st_bf16(KT, o64[u], kk[u] * ig);                          // Kt
+                if (want_u) tc::st_bf16(UU, o64[u], ww[u] * vv[u]);            // U
+            }
         }
-        const float kt = kk * ig;
-        tc::st_bf16(KT, o64, kt);                            // Kt
-        tc::st_bf16(KH, o64, gC * kt);                       // Kh
-        if (want_u) tc::st_bf16(UU, o64, tc::ld_bf16(WW, o64) * tc::ld_bf16(UU, o64));   // U = w*v
+        if (tmem_g != 0) tc::tmem_st16(tmem_g + 16 * tb2, gvals);
+    }
+    if (tmem_g != 0) tc::tmem_wait_st();
+    gC_out[i] = fast_exp(G);
+}
+
+// Gate preparation, vectorised: thread = (8-token block tb = tid / 16, 8-channel group cg = tid % 16),
+// 16-byte shared-memory accesses. Same inputs/outputs as gate_prep_cols (without the TMEM copy of G).
+// The in-chunk cumsum is a local scan over the thread's 8 rows plus the totals of the earlier
+// blocks, exchanged through `red` (fp32 [8][128], 4 KB). Contains one __syncthreads.
+__device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
+                                          unsigned char* UU, const unsigned char* WW, float* gC_out,
+                                          float* red, int tid, bool want_q, bool want_u) {
+    const int cg = tid & 15, tb = tid >> 4;
+    float G[8][8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        tc::ld_row8(KT, C, 8 * tb + u, cg, G[u]);
+        if (u > 0) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) G[u][c] += G[u - 1][c];
+        }
+    }
+    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg) = make_float4(G[7][0], G[7][1], G[7][2], G[7][3]);
+    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg + 4) = make_float4(G[7][4], G[7][5], G[7][6], G[7][7]);
+    __syncthreads();
+    float pre[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int p = 0; p < tb; ++p) {
+        const float4 x0 = *reinterpret_cast<const float4*>(red + p * 128 + 8 * cg);
+        const float4 x1 = *reinterpret_cast<const float4*>(red + p * 128 + 8 * cg + 4);
+        pre[0] += x0.x; pre[1] += x0.y; pre[2] += x0.z; pre[3] += x0.w;
+        pre[4] += x1.x; pre[5] += x1.y; pre[6] += x1.z; pre[7] += x1.w;
+    }
+    if (tb == 7) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) gC_out[8 * cg + c] = fast_exp(pre[c] + G[7][c]);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int row = 8 * tb + u;
+        float kk[8], bb[8], qq[8], vv[8], ww[8];
+        tc::ld_row8(KH, C, row, cg, kk);
+        tc::ld_row8(QE, 2 * C, row, cg, bb);
+        if (want_q) tc::ld_row8(QE, 2 * C, C + row, cg, qq);
+        if (want_u) { tc::ld_row8(UU, C, row, cg, vv); tc::ld_row8(WW, C, row, cg, ww); }
+        float e[8], kt[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float Gv = pre[c] + G[u][c];
+            const float g = fast_exp(Gv), ig = fast_exp(-Gv);
+            e[c] = g * bb[c] * kk[c];
+            kt[c] = kk[c] * ig;
+            if (want_q) qq[c] *= g;
+            if (want_u) vv[c] *= ww[c];
+        }
+        tc::st_row8(QE, 2 * C, row, cg, e);
+        tc::st_row8(KT, C, row, cg, kt);
+        if (want_q) tc::st_row8(QE, 2 * C, C + row, cg, qq);
+        if (want_u) tc::st_row8(UU, C, row, cg, vv);
     }
 }
 
@@ -135,62 +211,167 @@ __device__ __forceinline__ void extract_AP(uint32_t lane_base_ap, float* sA, uns
     }
 }
 
-// (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32 scratch sA).
-// Writes the fp32 inverse to sTf (lower triangle incl. the unit diagonal is
-// valid) and the bf16 row tile T (64 x 64, zeros above the diagonal).
-// 16 x 16 diagonal blocks by forward substitution (one warp per block), then the
-// off-diagonal blocks by diagonals: T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj.
-// sX (768 floats) may alias the T tile: it is dead before T is written.
-__device__ __forceinline__ void solve_unit_lower(const float* sA, float* sTf, float* sX, unsigned char* Ttile,
-                                                 int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    if (lane < 16) {
-        const int s = lane, base = 16 * warp;
-        float x[16];
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Row stride of the per-warp 16 x 16 fp32 temporaries (conflict-free fragment loads).
+constexpr int XS = 24;
+// acc (16 x 16, two m16n8 C fragments) += A[ar.., ac..] (16 x 16) * B (16 x 16), one warp,
+// tf32 inputs, fp32 accumulation. A comes from a 64 x 64 scratch (sq_idx layout); B from
+// the same layout (b_sq) or from a per-warp temporary with row stride XS.
+__device__ __forceinline__ void warp_mm16(float (&acc)[2][4], const float* __restrict__ A, int ar, int ac,
+                                          const float* __restrict__ Bm, int br, int bc, bool b_sq, int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = (r == s) ? 1.f : 0.f;
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = to_tf32(A[sq_idx(ar + g, ac + 8 * ks + t4)]);
+        const uint32_t a1 = to_tf32(A[sq_idx(ar + g + 8, ac + 8 * ks + t4)]);
+        const uint32_t a2 = to_tf32(A[sq_idx(ar + g, ac + 8 * ks + t4 + 4)]);
+        const uint32_t a3 = to_tf32(A[sq_idx(ar + g + 8, ac + 8 * ks + t4 + 4)]);
 #pragma unroll
-            for (int m = 0; m < r; ++m) acc -= sA[sq_idx(base + r, base + m)] * x[m];
-            x[r] = acc;
-            sTf[sq_idx(base + r, base + s)] = acc;
+        for (int nt = 0; nt < 2; ++nt) {
+            const int r0 = br + 8 * ks + t4, c0 = bc + 8 * nt + g;
+            const float x0 = b_sq ? Bm[sq_idx(r0, c0)] : Bm[r0 * XS + c0];
+            const float x1 = b_sq ? Bm[sq_idx(r0 + 4, c0)] : Bm[(r0 + 4) * XS + c0];
+            mma_tf32_16x8x8(acc[nt], a0, a1, a2, a3, to_tf32(x0), to_tf32(x1));
         }
+    }
+}
+// Store a 16 x 16 accumulator (times `scale`) to a sq_idx scratch at (rr, cc) or to a per-warp temporary.
+__device__ __forceinline__ void warp_store16(const float (&acc)[2][4], float* dst, int rr, int cc, bool sq,
+                                             float scale, int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int r = rr + g + ((e >> 1) << 3), c = cc + 8 * nt + 2 * t4 + (e & 1);
+            if (sq) dst[sq_idx(r, c)] = scale * acc[nt][e];
+            else dst[r * XS + c] = scale * acc[nt][e];
+        }
+}
+__device__ __forceinline__ void warp_load16(float (&acc)[2][4], const float* src, int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = src[(g + ((e >> 1) << 3)) * XS + 8 * nt + 2 * t4 + (e & 1)];
+}
+__device__ __forceinline__ void zero16(float (&acc)[2][4]) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+}
+
+// bf16 copy of a 16 x 16 accumulator into the T row tile (64 x 64) at block (rr, cc), times scale.
+__device__ __forceinline__ void warp_store16_tile(const float (&acc)[2][4], unsigned char* Ttile, int rr, int cc,
+                                                  float scale, int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int r = rr + g + 8 * hf, c = cc + 8 * nt + 2 * t4;
+            *reinterpret_cast<uint32_t*>(Ttile + tc::tile_off(C, r, c)) =
+                tc::pack_bf16x2(scale * acc[nt][2 * hf], scale * acc[nt][2 * hf + 1]);
+        }
+}
+
+// (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32 scratch sA, sq_idx layout).
+// Writes the inverse to sTf (lower triangle incl. the unit diagonal is valid) and the bf16
+// row tile T (64 x 64, zeros above the diagonal).
+//   1. 16 x 16 diagonal blocks T_ii by right-looking forward substitution (warp i, lane =
+//      column): once x_m is final, every later row is updated with it, so the FMAs of one
+//      step are independent.
+//   2. off-diagonal blocks T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj, by diagonals i - j = 1, 2, 3,
+//      as warp-level tf32 tensor-core products (mma.sync m16n8k8).
+// sX: 4 warps x 16 x XS floats (6 KB), must not alias the T tile.
+__device__ __forceinline__ void solve_unit_lower(const float* __restrict__ sA, float* __restrict__ sTf,
+                                                 float* __restrict__ sX, unsigned char* Ttile, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    {
+        const int s = lane & 15, base = 16 * warp;
+        float acc[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] = (r == s) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < 15; ++m) {
+            const float xm = acc[m];
+#pragma unroll
+            for (int r = m + 1; r < 16; ++r) acc[r] -= sA[sq_idx(base + r, base + m)] * xm;
+        }
+        if (lane < 16) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                sTf[sq_idx(base + r, base + s)] = acc[r];
+                tc::st_bf16(Ttile, tc::tile_off(C, base + r, base + s), acc[r]);
+            }
+        }
+        // zeros above the diagonal blocks: rows base..base+15, columns base+16..63
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const int ngrp = (C - base - 16) / 8;        // 8-column groups to clear per row
+        for (int e = lane; e < 16 * ngrp; e += 32)
+            tc::st_row8(Ttile, C, base + (e / ngrp), (base + 16) / 8 + (e % ngrp), z);
     }
     __syncthreads();
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int j = e >> 8, i = j + d, r = (e >> 4) & 15, c = e & 15;
-            float acc = 0.f;
-            for (int kb = j; kb < i; ++kb) {
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc += sA[sq_idx(16 * i + r, 16 * kb + m)] * sTf[sq_idx(16 * kb + m, 16 * j + c)];
-            }
-            sX[e] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int j = e >> 8, i = j + d, r = (e >> 4) & 15, c = e & 15;
-            float acc = 0.f;
-            for (int m = 0; m <= r; ++m) acc += sTf[sq_idx(16 * i + r, 16 * i + m)] * sX[(j << 8) + m * 16 + c];
-            sTf[sq_idx(16 * i + r, 16 * j + c)] = -acc;
-        }
-        __syncthreads();
+    float* Xw = sX + warp * 16 * XS;
+    float acc[2][4];
+    // diagonal 1: T_{j+1,j} (warps 0..2); warp 3 starts T_30's sum with A_30 T_00
+    if (warp < 3) {
+        const int j = warp, i = j + 1;
+        zero16(acc);
+        warp_mm16(acc, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j, true, lane);
+        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+        __syncwarp();
+        zero16(acc);
+        warp_mm16(acc, sTf, 16 * i, 16 * i, Xw, 0, 0, false, lane);
+        warp_store16(acc, sTf, 16 * i, 16 * j, true, -1.f, lane);
+        warp_store16_tile(acc, Ttile, 16 * i, 16 * j, -1.f, lane);
+    } else {
+        zero16(acc);
+        warp_mm16(acc, sA, 48, 0, sTf, 0, 0, true, lane);          // A_30 T_00
+        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
     }
-    if (tid < C) {
-        const int t = tid;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            float x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int s = 8 * g + u;
-                x[u] = (s <= t) ? sTf[sq_idx(t, s)] : 0.f;
-            }
-            tc::st_row8(Ttile, C, t, g, x);
-        }
+    __syncthreads();
+    // diagonal 2: T_20 (warp 0), T_31 (warp 1); warp 3 adds A_31 T_10 to its partial
+    if (warp < 2) {
+        const int j = warp, i = j + 2;
+        zero16(acc);
+        warp_mm16(acc, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j, true, lane);
+        warp_mm16(acc, sA, 16 * i, 16 * (j + 1), sTf, 16 * (j + 1), 16 * j, true, lane);
+        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+        __syncwarp();
+        zero16(acc);
+        warp_mm16(acc, sTf, 16 * i, 16 * i, Xw, 0, 0, false, lane);
+        warp_store16(acc, sTf, 16 * i, 16 * j, true, -1.f, lane);
+        warp_store16_tile(acc, Ttile, 16 * i, 16 * j, -1.f, lane);
+    } else if (warp == 3) {
+        warp_load16(acc, Xw, lane);
+        warp_mm16(acc, sA, 48, 16, sTf, 16, 0, true, lane);         // + A_31 T_10
+        __syncwarp();
+        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+    }
+    __syncthreads();
+    // diagonal 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20)   (warp 3)
+    if (warp == 3) {
+        warp_load16(acc, Xw, lane);
+        warp_mm16(acc, sA, 48, 32, sTf, 32, 0, true, lane);
+        __syncwarp();
+        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+        __syncwarp();
+        zero16(acc);
+        warp_mm16(acc, sTf, 48, 48, Xw, 0, 0, false, lane);
+        warp_store16_tile(acc, Ttile, 48, 0, -1.f, lane);
     }
 }
 
@@ -233,6 +414,25 @@ __device__ __forceinline__ void tmem_scale_columns(uint32_t lane_base_col, const
         tc::tmem_st32(lane_base_col + i0, v);
     }
     tc::tmem_wait_st();
+}
+
+// M = 64 accumulators (cta_group::1): row r of D lives in TMEM lane (r % 16) + 32 (r / 16).
+// Warp w, lanes 0..15 therefore hold rows 16w .. 16w+15. All 32 lanes must execute the loads.
+__device__ __forceinline__ int m64_row(int warp, int lane) { return 16 * warp + (lane & 15); }
+
+// Copy a [64 rows x 128 columns] M=64 accumulator into a bf16 row tile of 64 rows (optionally scaled).
+__device__ __forceinline__ void tmem_m64_to_tile(uint32_t lane_base_col, unsigned char* dst, int warp, int lane) {
+    const int r = m64_row(warp, lane);
+    float v[32];
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+        tc::tmem_ld32(lane_base_col + c0, v);
+        tc::tmem_wait_ld();
+        if (lane < 16) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) tc::st_row8(dst, C, r, (c0 >> 3) + g, v + 8 * g);
+        }
+    }
 }
 
 }  // namespace chunk

@@ -10,10 +10,11 @@
 //   TMA      q, k, v, log_alpha, b, w tiles (64 tokens x 128, bf16, 128B swizzle)
 //   prep     Et = g*b*k, Qt = g*q, Kt = k/g, Kh = gC*Kt, U = w*v       (g = exp(cumsum log_alpha))
 //   M1       [A; P] = [Et; Qt] Kt^T                                     (M=128, N=64, K=128)
-//   solve    T = (I + strict_lower(A))^{-1}                            (fp32, 16x16 blocks)
-//   M2, M3   Wm^T = Et^T T^T ,  Delta^T := U^T T^T                      (M=128, N=64, K=64)
-//   M4, M5   Delta^T -= S^T Wm^T ,  O^T = S^T Qt^T                      (M=128, N=64, K=128)
-//   M6, M7   O^T += Delta^T P^T ,   S^T <- S^T Diag(gC) + Delta^T Kh    (N=64 / N=128, K=64)
+//   solve    T = (I + strict_lower(A))^{-1}     (16x16 blocks, off-diagonal merges on mma.sync tf32)
+//   M2, M3   Wm = T Et (M=64, N=128) ,  Delta^T := U^T T^T (M=128, N=64)
+//   M4, M5   Delta^T -= S^T Wm^T (M=128) ,  O = Qt S (M=64, N=128)
+//   M6, M7   O += P Delta (M=64) ,  Z^T = S^T + Delta^T Kt (M=128, N=128)
+//   scale    S'^T = Z^T Diag(gC) on the fp32 accumulator, bf16 copy for the next chunk
 // Optionally the chunk-start states are written (bf16 tile images) for the backward.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -30,21 +31,21 @@ using namespace chunk;
 
 // shared-memory layout (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_QE = 0;           // [128 x 128] rows 0..63: b -> Et, rows 64..127: q -> Qt
-constexpr uint32_t OFF_KH = 32768;       // [64 x 128] k -> Kh
+constexpr uint32_t OFF_KH = 32768;       // [64 x 128] k
 constexpr uint32_t OFF_KT = 49152;       // [64 x 128] log_alpha -> Kt
 constexpr uint32_t OFF_UU = 65536;       // [64 x 128] v -> U
-constexpr uint32_t OFF_WW = 81920;       // [64 x 128] w -> Wm
+constexpr uint32_t OFF_WW = 81920;       // [64 x 128] w -> solve temporaries -> Wm
 constexpr uint32_t OFF_ST = 98304;       // [128 x 128] S^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // [128 x 64] Delta^T (bf16)  | fp32 A scratch [64 x 64]
-constexpr uint32_t OFF_TF = 147456;      // fp32 T [64 x 64]
-constexpr uint32_t OFF_TT = 163840;      // [64 x 64] T (bf16)  | solve temporaries (768 floats)
+constexpr uint32_t OFF_TF = 147456;      // fp32 T [64 x 64] | prep scan scratch
+constexpr uint32_t OFF_TT = 163840;      // [64 x 64] T (bf16)
 constexpr uint32_t OFF_PP = 172032;      // [64 x 64] P (bf16)
 constexpr uint32_t OFF_GC = 180224;      // fp32 gC[128]
 constexpr uint32_t OFF_BAR = 180736;     // 2 mbarriers, tmem base, abort flag
 constexpr uint32_t SMEM_BYTES = 180800 + 1024;
 
-// TMEM columns
-constexpr uint32_t TM_S = 0, TM_AP = 128, TM_W = 192, TM_D = 256, TM_O = 320, TM_COLS = 512;
+// TMEM columns: S^T (fp32 state), [A; P], Ut^T -> Delta^T, Wm (M=64), O (M=64)
+constexpr uint32_t TM_S = 0, TM_AP = 128, TM_D = 192, TM_W = 256, TM_O = 384, TM_COLS = 512;
 
 constexpr uint32_t LOAD_BYTES = 6 * 64 * 128 * 2;
 
@@ -57,7 +58,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                  const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
                  unsigned char* __restrict__ states, int T, int H) {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     unsigned char* QE = sm + OFF_QE;
     unsigned char* KH = sm + OFF_KH;
     unsigned char* KT = sm + OFF_KT;
@@ -67,7 +68,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     unsigned char* DT = sm + OFF_DT;
     float* sA = reinterpret_cast<float*>(sm + OFF_DT);
     float* sTf = reinterpret_cast<float*>(sm + OFF_TF);
-    float* sX = reinterpret_cast<float*>(sm + OFF_TT);
+    float* sX = reinterpret_cast<float*>(sm + OFF_WW);   // w is consumed by the prep, Wm written after M2
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
@@ -76,7 +77,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
     int* abort_flag = reinterpret_cast<int*>(sm + OFF_BAR + 20);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x % H, b = blockIdx.x / H;
     const size_t head = blockIdx.x;
     const int nc = (T + C - 1) / C;
@@ -100,7 +101,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     const uint32_t tmem = *tmem_base_ptr;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lanes
 
-    // issue the first chunk's loads
     auto issue_loads = [&](int c) {
         const int t0 = c * C;
         tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
@@ -136,13 +136,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         tc::bulk_commit();
     }
 
-    const uint32_t sQE = tc::smem_u32(QE), sKH = tc::smem_u32(KH), sKT = tc::smem_u32(KT),
-                   sUU = tc::smem_u32(UU), sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt),
-                   sDT = tc::smem_u32(DT), sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
+    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sUU = tc::smem_u32(UU),
+                   sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
+                   sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
     constexpr uint32_t ID_M1 = tc::idesc_bf16(128, 64, false, false);
-    constexpr uint32_t ID_M23 = tc::idesc_bf16(128, 64, true, false);
+    constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
+    constexpr uint32_t ID_M3 = tc::idesc_bf16(128, 64, true, false);
     constexpr uint32_t ID_M4 = tc::idesc_bf16(128, 64, false, false, true);
-    constexpr uint32_t ID_M56 = tc::idesc_bf16(128, 64, false, false);
+    constexpr uint32_t ID_M56 = tc::idesc_bf16(64, 128, false, false);
     constexpr uint32_t ID_M7 = tc::idesc_bf16(128, 128, false, true);
 
     uint32_t ph_load = 0, ph_mma = 0;
@@ -150,6 +151,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         if (!tc::mbar_wait(bar_mma, ph_mma)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 1u); }
         ph_mma ^= 1;
         tc::tc_fence_after();
+    };
+    auto sync_for_mma = [&]() {   // smem written by threads + TMEM accesses done -> visible to the MMA issuer
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
     };
 
     for (int c = 0; c < nc; ++c) {
@@ -159,9 +165,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         ph_load ^= 1;
 
         // ---- gate prep (thread = channel)
-        gate_prep(QE, KH, KT, UU, WW, sGC, tid, want_o, true);
-        tc::fence_async_smem();
-        __syncthreads();
+        gate_prep(QE, KH, KT, UU, WW, sGC, sTf, tid, want_o, true);
+        sync_for_mma();
 
         // ---- M1: [A; P] = [Et; Qt] Kt^T
         if (tid == 0) {
@@ -178,79 +183,87 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 
         // ---- T = (I + A)^{-1}
         solve_unit_lower(sA, sTf, sX, TT, tid);
-        tc::fence_async_smem();
-        __syncthreads();
+        sync_for_mma();
 
-        // ---- M2: Wm^T = Et^T T^T ;  M3: Delta^T := U^T T^T
+        // ---- M2: Wm = T Et ;  M3: Delta^T := U^T T^T
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                tc::mma_bf16(tmem + TM_W, tc::desc_mn(sQE, 2 * C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M23, kk > 0);
-                tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M23, kk > 0);
+                tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), ID_M2, kk > 0);
+                tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M3, kk > 0);
             }
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        tmem_to_tile_transposed(lane_base + TM_W, WW, tid);   // Wm [t][i] from Wm^T (lane i)
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
+        tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);   // Wm rows [t][i]
+        sync_for_mma();
 
-        // ---- M4: Delta^T -= S^T Wm^T ;  M5: O^T = S^T Qt^T
+        // ---- M4: Delta^T -= S^T Wm^T ;  M5: O = Qt S
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWW, C, 0, kk), ID_M4, 1);
                 if (want_o)
-                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sST, D, 0, kk), tc::desc_k(sQE, 2 * C, C, kk), ID_M56, kk > 0);
+                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sQE, 2 * C, C, kk), tc::desc_k(sST, D, 0, kk), ID_M56, kk > 0);
             }
             tc::mma_commit(bar_mma);
         }
         wait_mma();
         tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);       // Delta^T (lane j) -> bf16 rows
-        tmem_scale_columns(lane_base + TM_S, sGC);               // S^T <- S^T Diag(gC)
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
+        sync_for_mma();
 
-        // ---- M6: O^T += Delta^T P^T ;  M7: S^T += Delta^T Kh
+        // ---- M6: O += P Delta ;  M7: Z^T = S^T + Delta^T Kt
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 if (want_o)
-                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sDT, D, 0, kk), tc::desc_k(sPP, C, 0, kk), ID_M56, 1);
-                tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sKH, C, 0, kk), ID_M7, 1);
+                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sPP, C, 0, kk), tc::desc_k(sDT, D, 0, kk), ID_M56, 1);
+                tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sKT, C, 0, kk), ID_M7, 1);
             }
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        // all smem tiles of this chunk are consumed: prefetch the next chunk
+        // all smem input tiles of this chunk are consumed: prefetch the next chunk
         if (tid == 0 && c + 1 < nc) issue_loads(c + 1);
 
-        if (want_o) {   // o[t][j] for t < L from O^T (lane j)
-            const int j = tid;
+        if (want_o) {   // o rows t from the M=64 accumulator: 16-byte stores
+            const int t = m64_row(warp, lane);
             float v[32];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                tc::tmem_ld32(lane_base + TM_O + 32 * h2, v);
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                tc::tmem_ld32(lane_base + TM_O + c0, v);
                 tc::tmem_wait_ld();
+                if (lane < 16 && t < L) {
+                    uint4* dst = reinterpret_cast<uint4*>(o + tok_off(b, t0 + t, h, T, H, D) + c0);
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int t = 32 * h2 + u;
-                    if (t < L) o[tok_off(b, t0 + t, h, T, H, D) + j] = __float2bfloat16_rn(v[u]);
+                    for (int g = 0; g < 4; ++g)
+                        dst[g] = make_uint4(tc::pack_bf16x2(v[8 * g], v[8 * g + 1]), tc::pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
+                                            tc::pack_bf16x2(v[8 * g + 4], v[8 * g + 5]), tc::pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
                 }
             }
         }
-        // new state: bf16 copy for the next chunk's operands (and the saved image)
+        // S'^T = Z^T Diag(gC): scale the fp32 state, keep a bf16 copy for the next chunk
         if (states && tid == 0) tc::bulk_wait_read();
         __syncthreads();
-        tmem_to_tile_rows<128>(lane_base + TM_S, STt, tid);
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
+        {
+            const int j = tid;
+            float v[32];
+#pragma unroll 1
+            for (int i0 = 0; i0 < D; i0 += 32) {
+                tc::tmem_ld32(lane_base + TM_S + i0, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
+                tc::tmem_st32(lane_base + TM_S + i0, v);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+            }
+            tc::tmem_wait_st();
+        }
+        sync_for_mma();
         tc::tc_fence_after();
         if (states && tid == 0 && c + 1 < nc) {
             tc::bulk_store(states + (head * nc + c + 1) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
@@ -290,12 +303,8 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     CUtensorMap* maps[6] = {&mq, &mk, &mv, &mla, &mb, &mw};
     for (int i = 0; i < 6; ++i)
         if (make_token_map(maps[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     chunk_fwd_kernel<<<d.B * d.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mla, mb, mw, a.S0,
                                                        static_cast<__nv_bfloat16*>(a.o), a.ST, a.states, d.T, d.H);
     return cudaGetLastError();
