@@ -19,11 +19,11 @@
 //   E = rowsum(dZ * S) + sum_t Kt_t * (Delta dZ^T)_t   (the dependence of S' on gC)
 //   dlog_alpha_t = sum_{tau >= t} dG_tau + E
 //
-// Two kernels:
+// Two kernels, both reading the forward's per-chunk T and P tiles instead of redoing the solve:
 //   reverse_state_kernel  one CTA per (batch, head) walks the chunks backwards carrying
 //                         dS^T in TMEM (fp32) and stores each chunk's dZ^T as a bf16 image;
 //   chunk_grad_kernel     one CTA per (batch, head, chunk) computes every gradient of the
-//                         chunk from the saved S, dS', the inputs and dout.
+//                         chunk from the saved S, dZ, T, P, the inputs and dout.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -39,6 +39,8 @@ using namespace chunk;
 
 __device__ unsigned int g_bwd_error;
 
+constexpr uint32_t TILE_C = 64 * 64 * 2;   // bytes of a 64 x 64 bf16 tile
+
 // ====================================================================== reverse state pass
 
 namespace rs {
@@ -46,24 +48,25 @@ constexpr uint32_t OFF_QE = 0;           // rows 0..63: b -> Et, rows 64..127: q
 constexpr uint32_t OFF_KH = 32768;       // k
 constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
 constexpr uint32_t OFF_DO = 65536;       // dout
-constexpr uint32_t OFF_WW = 81920;       // solve temporaries, then Wm
+constexpr uint32_t OFF_WW = 81920;       // Wm
 constexpr uint32_t OFF_ST = 98304;       // dZ^T (bf16)
-constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16) | fp32 A scratch
-constexpr uint32_t OFF_TF = 147456;      // fp32 T | prep scan scratch
-constexpr uint32_t OFF_TT = 163840;      // T (bf16)
-constexpr uint32_t OFF_PP = 172032;      // P (bf16)
-constexpr uint32_t OFF_GC = 180224;
-constexpr uint32_t OFF_BAR = 180736;
-constexpr uint32_t SMEM_BYTES = 180800 + 1024;
-constexpr uint32_t TM_S = 0, TM_AP = 128, TM_D = 192, TM_W = 256, TM_COLS = 512;
-constexpr uint32_t LOAD_BYTES = 5 * 64 * 128 * 2;
+constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16)
+constexpr uint32_t OFF_TT = 147456;      // T (bf16, from the forward)
+constexpr uint32_t OFF_PP = 155648;      // P (bf16, from the forward)
+constexpr uint32_t OFF_RED = 163840;     // prep scan scratch (4 KB)
+constexpr uint32_t OFF_GC = 167936;
+constexpr uint32_t OFF_BAR = 168448;
+constexpr uint32_t SMEM_BYTES = 168512 + 1024;
+constexpr uint32_t TM_S = 0, TM_D = 128, TM_W = 192, TM_COLS = 512;
+constexpr uint32_t LOAD_BYTES = 5 * 64 * 128 * 2 + 2 * TILE_C;
 }  // namespace rs
 
 __global__ void __launch_bounds__(NT, 1)
 reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                      const __grid_constant__ CUtensorMap mla, const __grid_constant__ CUtensorMap mb,
                      const __grid_constant__ CUtensorMap mdo, const float* __restrict__ dST,
-                     float* __restrict__ dS0, unsigned char* __restrict__ dstates, int T, int H) {
+                     float* __restrict__ dS0, const unsigned char* __restrict__ tp,
+                     unsigned char* __restrict__ dstates, int T, int H) {
     using namespace rs;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
@@ -74,11 +77,9 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     unsigned char* WW = sm + OFF_WW;
     unsigned char* STt = sm + OFF_ST;
     unsigned char* DT = sm + OFF_DT;
-    float* sA = reinterpret_cast<float*>(sm + OFF_DT);
-    float* sTf = reinterpret_cast<float*>(sm + OFF_TF);
-    float* sX = reinterpret_cast<float*>(sm + OFF_WW);   // Wm is written after the solve
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
+    float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_load + 1;
@@ -114,6 +115,9 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         tma_tile(KH, C, 0, &mk, b, h, t0, bar_load);
         tma_tile(KT, C, 0, &mla, b, h, t0, bar_load);
         tma_tile(DO, C, 0, &mdo, b, h, t0, bar_load);
+        const unsigned char* src = tp + (head * nc + c) * TC_TP_BYTES;
+        tc::bulk_load(TT, src, TILE_C, bar_load);
+        tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
     };
     if (tid == 0) issue_loads(nc - 1);
 
@@ -135,7 +139,6 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sDO = tc::smem_u32(DO),
                    sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
-    constexpr uint32_t ID_M1 = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
     constexpr uint32_t ID_N1a = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_N1b = tc::idesc_bf16(128, 64, true, true);
@@ -158,7 +161,7 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
         ph_load ^= 1;
 
-        gate_prep(QE, KH, KT, nullptr, nullptr, sGC, sTf, tid, true, false);
+        gate_prep(QE, KH, KT, nullptr, nullptr, sGC, sRed, tid, true, false);
         // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
         if (tid == 0) tc::bulk_wait_read();
         __syncthreads();
@@ -178,28 +181,11 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
             tc::tmem_wait_st();
         }
         sync_for_mma();
-        if (tid == 0) {     // keep the dZ^T image of this chunk for the gradient kernel
-            tc::bulk_store(dstates + (head * nc + c) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
-            tc::bulk_commit();
-        }
-
-        // [A; P] = [Et; Qt] Kt^T
-        if (tid == 0) {
-            tc::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
-            tc::mma_commit(bar_mma);
-        }
-        wait_mma();
-        extract_AP(lane_base + TM_AP, sA, PP, true, tid);
-        tc::tc_fence_before();
-        __syncthreads();
-        solve_unit_lower(sA, sTf, sX, TT, tid);
-        sync_for_mma();
 
         // Wm = T Et (M=64) ;  dDelta^T = dZ^T Kt^T + dO^T P
         if (tid == 0) {
+            tc::bulk_store(dstates + (head * nc + c) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
+            tc::bulk_commit();
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -259,22 +245,22 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 
 namespace cg {
 constexpr uint32_t OFF_QE = 0;           // rows 0..63: b -> Et, rows 64..127: q -> Qt
-constexpr uint32_t OFF_KH = 32768;       // k (kept)
+constexpr uint32_t OFF_KH = 32768;       // k -> U, later k (reloaded)
 constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
-constexpr uint32_t OFF_UU = 65536;       // v -> U, later dU rows [t][j]
-constexpr uint32_t OFF_WW = 81920;       // w -> solve temporaries -> Wm rows, later b (reloaded)
-constexpr uint32_t OFF_DO = 98304;       // dout
+constexpr uint32_t OFF_UU = 65536;       // v, later dU rows [t][j], later staged dlog_alpha
+constexpr uint32_t OFF_WW = 81920;       // w, later b (reloaded)
+constexpr uint32_t OFF_DO = 98304;       // dout, later staged dq
 constexpr uint32_t OFF_ST = 114688;      // S^T image (chunk start)
 constexpr uint32_t OFF_DS = 147456;      // dZ^T image
-constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64] | fp32 A scratch
-constexpr uint32_t OFF_DDT = 196608;     // dDelta^T [128 x 64] | fp32 T
+constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64], later staged dk
+constexpr uint32_t OFF_DDT = 196608;     // Wm rows, then dDelta^T [128 x 64], later staged db
 constexpr uint32_t OFF_TT = 212992;      // T, later dA^T [64 x 64]
 constexpr uint32_t OFF_PP = 221184;      // P, later dP^T [64 x 64]
 constexpr uint32_t OFF_GC = 229376;
 constexpr uint32_t OFF_BAR = 229888;
 constexpr uint32_t SMEM_BYTES = 229952 + 1024;
 // TMEM columns (M=64 accumulators use lanes 0-15 of each 32-lane quarter)
-constexpr uint32_t TM_AP = 0,      // [A; P], later dP^T (M=64)
+constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_W = 64,                     // Wm (M=64, 128 columns), later dA^T (M=64, 64 columns)
     TM_D = 192,                    // Ut^T -> Delta^T, later G4 = (Delta dZ^T)^T
     TM_DD = 256,                   // dDelta^T, later G3 = dKt^T (P and A paths)
@@ -282,18 +268,18 @@ constexpr uint32_t TM_AP = 0,      // [A; P], later dP^T (M=64)
     TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,
     TM_GV = 448,                   // G[t] per key channel (cumulative log-decay)
     TM_COLS = 512;
-constexpr uint32_t LOAD_BYTES = 7 * 64 * 128 * 2 + 2 * (uint32_t)TC_STATE_BYTES;
+constexpr uint32_t LOAD_BYTES = 7 * 64 * 128 * 2 + 2 * (uint32_t)TC_STATE_BYTES + 2 * TILE_C;
 }  // namespace cg
 
 __global__ void __launch_bounds__(NT, 1)
 chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mla,
                   const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
-                  const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16* __restrict__ v_g,
-                  const __nv_bfloat16* __restrict__ w_g, __nv_bfloat16* __restrict__ dq,
-                  __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, __nv_bfloat16* __restrict__ dla,
-                  __nv_bfloat16* __restrict__ db, __nv_bfloat16* __restrict__ dw,
-                  const unsigned char* __restrict__ states, const unsigned char* __restrict__ dstates, int T, int H) {
+                  const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mdq,
+                  const __grid_constant__ CUtensorMap mdk, const __grid_constant__ CUtensorMap mdb,
+                  const __grid_constant__ CUtensorMap mdla, __nv_bfloat16* __restrict__ dv,
+                  __nv_bfloat16* __restrict__ dw, const unsigned char* __restrict__ states,
+                  const unsigned char* __restrict__ tp, const unsigned char* __restrict__ dstates, int T, int H) {
     using namespace cg;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
@@ -307,16 +293,14 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     unsigned char* DS = sm + OFF_DS;
     unsigned char* DT = sm + OFF_DT;
     unsigned char* DDT = sm + OFF_DDT;
-    float* sA = reinterpret_cast<float*>(sm + OFF_DT);
-    float* sTf = reinterpret_cast<float*>(sm + OFF_DDT);
-    float* sX = reinterpret_cast<float*>(sm + OFF_WW);   // w is consumed by the prep, Wm written after M2
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_load + 1;
-    uint64_t* bar_b = bar_load + 2;
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 24);
+    uint64_t* bar_k = bar_load + 2;
+    uint64_t* bar_b = bar_load + 3;
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 32);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
@@ -329,6 +313,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     if (tid == 0) {
         tc::mbar_init(bar_load, 1);
         tc::mbar_init(bar_mma, 1);
+        tc::mbar_init(bar_k, 1);
         tc::mbar_init(bar_b, 1);
         tc::fence_mbar_init();
         tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
@@ -341,6 +326,9 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tma_tile(DO, C, 0, &mdo, b, h, t0, bar_load);
         tc::bulk_load(STt, states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
         tc::bulk_load(DS, dstates + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
+        const unsigned char* src = tp + (head * nc + c) * TC_TP_BYTES;
+        tc::bulk_load(TT, src, TILE_C, bar_load);
+        tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_base_ptr, TM_COLS);
@@ -364,27 +352,13 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         __syncthreads();
     };
 
-    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sUU = tc::smem_u32(UU),
-                   sWW = tc::smem_u32(WW), sDO = tc::smem_u32(DO), sST = tc::smem_u32(STt),
+    const uint32_t sQE = tc::smem_u32(QE), sKH = tc::smem_u32(KH), sKT = tc::smem_u32(KT),
+                   sUU = tc::smem_u32(UU), sDO = tc::smem_u32(DO), sST = tc::smem_u32(STt),
                    sDS = tc::smem_u32(DS), sDT = tc::smem_u32(DT), sDDT = tc::smem_u32(DDT),
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
-    // ---- factors (G kept in TMEM), [A; P], T
-    gate_prep_cols(QE, KH, KT, UU, WW, sGC, tid, true, true, lane_base + TM_GV);
-    sync_for_mma();
-    if (tid == 0) {
-        tc::tc_fence_after();
-        constexpr uint32_t id = tc::idesc_bf16(128, 64, false, false);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), id, kk > 0);
-        tc::mma_commit(bar_mma);
-    }
-    wait_mma();
-    extract_AP(lane_base + TM_AP, sA, PP, true, tid);
-    tc::tc_fence_before();
-    __syncthreads();
-    solve_unit_lower(sA, sTf, sX, TT, tid);
+    // ---- factors (U over k, G kept in TMEM)
+    gate_prep_cols(QE, KH, KT, UU, WW, sGC, tid, lane_base + TM_GV);
     sync_for_mma();
 
     // ---- Wm = T Et (M=64) ; Ut^T = U^T T^T
@@ -395,12 +369,16 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), id_w, kk > 0);
-            tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), id_u, kk > 0);
+            tc::mma_bf16(tmem + TM_D, tc::desc_mn(sKH, C, 0, kk), tc::desc_k(sTT, C, 0, kk), id_u, kk > 0);
         }
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);       // Wm rows
+    if (tid == 0) {     // U is consumed: bring k back for the gate chain
+        tc::mbar_arrive_expect_tx(bar_k, 64 * 128 * 2);
+        tma_tile(KH, C, 0, &mk, b, h, t0, bar_k);
+    }
+    tmem_m64_to_tile(lane_base + TM_W, DDT, warp, lane);      // Wm rows (DDT is free until dDelta^T)
     sync_for_mma();
 
     // ---- Delta^T = Ut^T - S^T Wm^T ;  dDelta^T = dZ^T Kt^T + dO^T P
@@ -411,7 +389,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         constexpr uint32_t id_mm = tc::idesc_bf16(128, 64, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWW, C, 0, kk), id_neg, 1);
+            tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sDDT, C, 0, kk), id_neg, 1);
             tc::mma_bf16(tmem + TM_DD, tc::desc_k(sDS, D, 0, kk), tc::desc_k(sKT, C, 0, kk), id_kk, kk > 0);
         }
 #pragma unroll
@@ -420,10 +398,6 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    if (tid == 0) {     // Wm is consumed: bring b back for the gate chain
-        tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
-        tma_tile(WW, C, 0, &mb, b, h, t0, bar_b);
-    }
     tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);      // Delta^T [j][t]
     tmem_to_tile_rows<64>(lane_base + TM_DD, DDT, tid);    // dDelta^T [j][t]
     sync_for_mma();
@@ -438,46 +412,43 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    {   // dv = dU*w, dw = dU*v (rows t, 16-byte accesses); keep dU as a bf16 row tile
+    {   // dv = dU*w, dw = dU*v (rows t; v, w from shared memory); dU replaces v as a bf16 row tile
         const int t = m64_row(warp, lane);
         const bool row_ok = lane < 16 && t < L;
         float v[32];
-#pragma unroll
+#pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
             tc::tmem_ld32(lane_base + TM_DU + c0, v);
             tc::tmem_wait_ld();
             if (lane < 16) {
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(UU, C, t, (c0 >> 3) + g, v + 8 * g);
-            }
-            if (row_ok) {
-                const size_t off = tok_off(b, t0 + t, h, T, H, D) + c0;
-                const uint4* wp = reinterpret_cast<const uint4*>(w_g + off);
-                const uint4* vp = reinterpret_cast<const uint4*>(v_g + off);
-                uint4 wv[4], vv[4];
-#pragma unroll
-                for (int g = 0; g < 4; ++g) { wv[g] = wp[g]; vv[g] = vp[g]; }
-                uint4* dvp = reinterpret_cast<uint4*>(dv + off);
-                uint4* dwp = reinterpret_cast<uint4*>(dw + off);
+                uint4* dvp = reinterpret_cast<uint4*>(dv + tok_off(b, t0 + (row_ok ? t : 0), h, T, H, D) + c0);
+                uint4* dwp = reinterpret_cast<uint4*>(dw + tok_off(b, t0 + (row_ok ? t : 0), h, T, H, D) + c0);
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
-                    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv[g]);
-                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv[g]);
+                    float vv[8], ww[8];
+                    tc::ld_row8(UU, C, t, (c0 >> 3) + g, vv);
+                    tc::ld_row8(WW, C, t, (c0 >> 3) + g, ww);
                     uint32_t ov[4], ow[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 wf = __bfloat1622float2(w2[e]), vf = __bfloat1622float2(v2[e]);
                         const float d0 = v[8 * g + 2 * e], d1 = v[8 * g + 2 * e + 1];
-                        ov[e] = tc::pack_bf16x2(d0 * wf.x, d1 * wf.y);
-                        ow[e] = tc::pack_bf16x2(d0 * vf.x, d1 * vf.y);
+                        ov[e] = tc::pack_bf16x2(d0 * ww[2 * e], d1 * ww[2 * e + 1]);
+                        ow[e] = tc::pack_bf16x2(d0 * vv[2 * e], d1 * vv[2 * e + 1]);
                     }
-                    dvp[g] = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-                    dwp[g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    if (row_ok) {
+                        dvp[g] = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+                        dwp[g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                    tc::st_row8(UU, C, t, (c0 >> 3) + g, v + 8 * g);
                 }
             }
         }
     }
     sync_for_mma();
+    if (tid == 0) {     // w is consumed: bring b back for the gate chain
+        tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
+        tma_tile(WW, C, 0, &mb, b, h, t0, bar_b);
+    }
 
     // ---- dP^T = Delta dO^T (M=64), dA^T = -Delta dU^T (M=64)
     if (tid == 0) {
@@ -558,13 +529,15 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         E += e2;
     }
     wait_mma();
+    ok = tc::mbar_wait(bar_k, 0) && ok;
     ok = tc::mbar_wait(bar_b, 0) && ok;
 
-    // ---- gate chain, thread = key channel i: E += sum_t Kt G4, then tokens in reverse
+    // ---- gate chain, thread = key channel i: E += sum_t Kt G4, then tokens in reverse.
+    // Results go to bf16 row tiles (dq -> DO, dk -> DT, db -> DDT, dlog_alpha -> UU), stored by TMA.
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chk = (uint32_t)((i & 63) >> 3);
-#pragma unroll
+#pragma unroll 1
     for (int q4 = 0; q4 < 4; ++q4) {
         float g4[16];
         tc::tmem_ld16(lane_base + TM_G4 + 16 * q4, g4);
@@ -585,32 +558,37 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::tmem_ld16(lane_base + TM_G4 + 16 * q4, g4);
         tc::tmem_ld16(lane_base + TM_GV + 16 * q4, gv);
         tc::tmem_wait_ld();
-        float qt[16], et[16], kt[16], kk[16], bb[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const uint32_t t = (uint32_t)(16 * q4 + u);
-            const uint32_t sw = t * 128 + ((chk ^ (t & 7)) << 4);
-            qt[u] = tc::ld_bf16(QE, col128 + C * 128 + sw);
-            et[u] = tc::ld_bf16(QE, col128 + sw);
-            kt[u] = tc::ld_bf16(KT, col64 + sw);
-            kk[u] = tc::ld_bf16(KH, col64 + sw);
-            bb[u] = tc::ld_bf16(WW, col64 + sw);
-        }
 #pragma unroll
         for (int u = 15; u >= 0; --u) {
-            const int t = 16 * q4 + u;
+            const uint32_t t = (uint32_t)(16 * q4 + u);
+            const uint32_t sw = t * 128 + ((chk ^ (t & 7)) << 4);
+            const float qt = tc::ld_bf16(QE, col128 + C * 128 + sw);
+            const float et = tc::ld_bf16(QE, col128 + sw);
+            const float kt = tc::ld_bf16(KT, col64 + sw);
+            const float kk = tc::ld_bf16(KH, col64 + sw);
+            const float bb = tc::ld_bf16(WW, col64 + sw);
             const float g = fast_exp(gv[u]), ig = fast_exp(-gv[u]);
             const float dKt = g3[u] + g4[u];
-            suffix += qt[u] * g1[u] + et[u] * g2[u] - kt[u] * dKt;
-            if (t < L) {
-                const size_t off = tok_off(b, t0 + t, h, T, H, D) + i;
-                const float dE = g * g2[u];
-                dq[off] = __float2bfloat16_rn(g * g1[u]);
-                db[off] = __float2bfloat16_rn(dE * kk[u]);
-                dk[off] = __float2bfloat16_rn(dKt * ig + dE * bb[u]);
-                dla[off] = __float2bfloat16_rn(suffix + E);
-            }
+            suffix += qt * g1[u] + et * g2[u] - kt * dKt;
+            const float dE = g * g2[u];
+            tc::st_bf16(DO, col64 + sw, g * g1[u]);                 // dq
+            tc::st_bf16(DT, col64 + sw, dKt * ig + dE * bb);        // dk
+            tc::st_bf16(DDT, col64 + sw, dE * kk);                  // db
+            tc::st_bf16(UU, col64 + sw, suffix + E);                // dlog_alpha
         }
+    }
+    tc::fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {   // rows past the end of the sequence are skipped by the tensor store
+        const CUtensorMap* maps[4] = {&mdq, &mdk, &mdb, &mdla};
+        const unsigned char* tiles[4] = {DO, DT, DDT, UU};
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+            tc::tma_store_4d(maps[o], 0, h, t0, b, tiles[o]);
+            tc::tma_store_4d(maps[o], 64, h, t0, b, tiles[o] + C * 128);
+        }
+        tc::bulk_commit();
+        tc::bulk_wait_read();
     }
     if (!ok) atomicOr(&g_bwd_error, 4u);
 
@@ -632,24 +610,23 @@ cudaError_t set_smem(K kernel, uint32_t bytes) {
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
-    CUtensorMap mq, mk, mv, mla, mb, mw, mdo;
-    const void* ptrs[7] = {a.q, a.k, a.v, a.la, a.b, a.w, a.dout};
-    CUtensorMap* maps[7] = {&mq, &mk, &mv, &mla, &mb, &mw, &mdo};
-    for (int i = 0; i < 7; ++i)
+    CUtensorMap mq, mk, mv, mla, mb, mw, mdo, mdq, mdk, mdb, mdla;
+    const void* ptrs[11] = {a.q, a.k, a.v, a.la, a.b, a.w, a.dout, a.dq, a.dk, a.db, a.dla};
+    CUtensorMap* maps[11] = {&mq, &mk, &mv, &mla, &mb, &mw, &mdo, &mdq, &mdk, &mdb, &mdla};
+    for (int i = 0; i < 11; ++i)
         if (make_token_map(maps[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     cudaError_t e = set_smem(reverse_state_kernel, rs::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = set_smem(chunk_grad_kernel, cg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    reverse_state_kernel<<<d.B * d.H, NT, rs::SMEM_BYTES, s>>>(mq, mk, mla, mb, mdo, a.dST, a.dS0, a.dstates, d.T, d.H);
+    reverse_state_kernel<<<d.B * d.H, NT, rs::SMEM_BYTES, s>>>(mq, mk, mla, mb, mdo, a.dST, a.dS0, a.tp, a.dstates,
+                                                                d.T, d.H);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const dim3 grid(d.nchunks(), d.B * d.H);
     chunk_grad_kernel<<<grid, NT, cg::SMEM_BYTES, s>>>(
-        mq, mk, mv, mla, mb, mw, mdo, static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.w),
-        static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv),
-        static_cast<__nv_bfloat16*>(a.dla), static_cast<__nv_bfloat16*>(a.db), static_cast<__nv_bfloat16*>(a.dw),
-        a.states, a.dstates, d.T, d.H);
+        mq, mk, mv, mla, mb, mw, mdo, mdq, mdk, mdb, mdla, static_cast<__nv_bfloat16*>(a.dv),
+        static_cast<__nv_bfloat16*>(a.dw), a.states, a.tp, a.dstates, d.T, d.H);
     return cudaGetLastError();
 }
 

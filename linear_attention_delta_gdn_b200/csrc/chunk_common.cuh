@@ -70,14 +70,13 @@ __device__ __forceinline__ void tma_tile(unsigned char* dst, int R, int dst_row0
 // Gate preparation, channel-major variant: one thread per key/value channel i (= threadIdx.x),
 // tokens in blocks of 8 (loads of a block are issued together, then its stores):
 //   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
-//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127 (want_q),
-//          Kt = k/g -> KT, U = w*v -> UU (want_u); KH keeps k.
-//   g = exp(G), G = inclusive cumsum of log_alpha. gC[i] = g at the last row.
-//   If tmem_g != 0, G[t][i] is also stored to TMEM (lane i, columns t) for later use.
-__device__ __forceinline__ void gate_prep_cols(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
-                                          unsigned char* UU, const unsigned char* WW, float* gC_out, int i,
-                                          bool want_q, bool want_u, uint32_t tmem_g = 0) {
-    // byte offset of (row 8*tb + u, channel i) in a 64-row tile, and in the 128-row QE tile
+//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127, Kt = k/g -> KT,
+//          U = w*v -> KH (over k, which the thread has read); UU and WW keep v and w.
+//   g = exp(G), G = inclusive cumsum of log_alpha; gC[i] = g at the last row.
+//   G[t][i] is also stored to TMEM at tmem_g (lane i, columns t).
+__device__ __forceinline__ void gate_prep_cols(unsigned char* QE, unsigned char* KH, unsigned char* KT,
+                                               const unsigned char* UU, const unsigned char* WW, float* gC_out,
+                                               int i, uint32_t tmem_g) {
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chunk = (uint32_t)((i & 63) >> 3);
@@ -99,23 +98,24 @@ __device__ __forceinline__ void gate_prep_cols(unsigned char* QE, const unsigned
                 la[u] = tc::ld_bf16(KT, o64[u]);
                 kk[u] = tc::ld_bf16(KH, o64[u]);
                 bb[u] = tc::ld_bf16(QE, o128[u]);
-                if (want_q) qq[u] = tc::ld_bf16(QE, o128[u] + C * 128);
-                if (want_u) { vv[u] = tc::ld_bf16(UU, o64[u]); ww[u] = tc::ld_bf16(WW, o64[u]); }
+                qq[u] = tc::ld_bf16(QE, o128[u] + C * 128);
+                vv[u] = tc::ld_bf16(UU, o64[u]);
+                ww[u] = tc::ld_bf16(WW, o64[u]);
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 G += la[u];
                 gvals[half * 8 + u] = G;
                 const float g = fast_exp(G), ig = fast_exp(-G);
-                tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);                 // Et
-                if (want_q) tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);    // Qt
-                tc::st_bf16(KT, o64[u], kk[u] * ig);                          // Kt
-                if (want_u) tc::st_bf16(UU, o64[u], ww[u] * vv[u]);            // U
+                tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);          // Et
+                tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);        // Qt
+                tc::st_bf16(KT, o64[u], kk[u] * ig);                  // Kt
+                tc::st_bf16(KH, o64[u], ww[u] * vv[u]);               // U
             }
         }
-        if (tmem_g != 0) tc::tmem_st16(tmem_g + 16 * tb2, gvals);
+        tc::tmem_st16(tmem_g + 16 * tb2, gvals);
     }
-    if (tmem_g != 0) tc::tmem_wait_st();
+    tc::tmem_wait_st();
     gC_out[i] = fast_exp(G);
 }
 

@@ -15,7 +15,8 @@
 //   M4, M5   Delta^T -= S^T Wm^T (M=128) ,  O = Qt S (M=64, N=128)
 //   M6, M7   O += P Delta (M=64) ,  Z^T = S^T + Delta^T Kt (M=128, N=128)
 //   scale    S'^T = Z^T Diag(gC) on the fp32 accumulator, bf16 copy for the next chunk
-// Optionally the chunk-start states are written (bf16 tile images) for the backward.
+// For training, the chunk-start states and the T and P tiles of every chunk are written
+// (bf16 shared-memory images) for the backward.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -56,7 +57,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                  const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mla,
                  const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
                  const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
-                 unsigned char* __restrict__ states, int T, int H) {
+                 unsigned char* __restrict__ states, unsigned char* __restrict__ tp, int T, int H) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     unsigned char* QE = sm + OFF_QE;
@@ -82,6 +83,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     const size_t head = blockIdx.x;
     const int nc = (T + C - 1) / C;
     const bool want_o = (o != nullptr);
+    const bool save = (states != nullptr);          // training: keep S, T and P of every chunk
+    const bool want_qp = want_o || save;
 
     if (tid == 0) {
         tc::mbar_init(bar_load, 1);
@@ -165,7 +168,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         ph_load ^= 1;
 
         // ---- gate prep (thread = channel)
-        gate_prep(QE, KH, KT, UU, WW, sGC, sTf, tid, want_o, true);
+        gate_prep(QE, KH, KT, UU, WW, sGC, sTf, tid, want_qp, true);
         sync_for_mma();
 
         // ---- M1: [A; P] = [Et; Qt] Kt^T
@@ -177,13 +180,19 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        extract_AP(lane_base + TM_AP, sA, PP, want_o, tid);
+        extract_AP(lane_base + TM_AP, sA, PP, want_qp, tid);
         tc::tc_fence_before();
         __syncthreads();
 
         // ---- T = (I + A)^{-1}
         solve_unit_lower(sA, sTf, sX, TT, tid);
         sync_for_mma();
+        if (save && tid == 0) {   // T and P of this chunk for the backward
+            unsigned char* dst = tp + (head * nc + c) * TC_TP_BYTES;
+            tc::bulk_store(dst, TT, (uint32_t)(TC_TP_BYTES / 2));
+            tc::bulk_store(dst + TC_TP_BYTES / 2, PP, (uint32_t)(TC_TP_BYTES / 2));
+            tc::bulk_commit();
+        }
 
         // ---- M2: Wm = T Et ;  M3: Delta^T := U^T T^T
         if (tid == 0) {
@@ -306,7 +315,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     chunk_fwd_kernel<<<d.B * d.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mla, mb, mw, a.S0,
-                                                       static_cast<__nv_bfloat16*>(a.o), a.ST, a.states, d.T, d.H);
+                                                       static_cast<__nv_bfloat16*>(a.o), a.ST, a.states, a.tp, d.T, d.H);
     return cudaGetLastError();
 }
 

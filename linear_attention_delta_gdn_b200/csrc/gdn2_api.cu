@@ -53,10 +53,13 @@ gdn2_status check_dims(int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtyp
     return GDN2_OK;
 }
 
+// Forward-saved region: chunk-start states (and, on the tensor-core path, the [T | P] tiles).
 size_t states_bytes(const Dims& d, gdn2_dtype dt) {
     const size_t units = (size_t)d.B * d.H * (size_t)d.nchunks();
-    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * TC_STATE_BYTES : units * d.Dk * d.Dv * sizeof(float);
+    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * (TC_STATE_BYTES + TC_TP_BYTES)
+                                                  : units * d.Dk * d.Dv * sizeof(float);
 }
+size_t tc_tp_offset(const Dims& d) { return (size_t)d.B * d.H * (size_t)d.nchunks() * TC_STATE_BYTES; }
 
 size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
     if (tc_train_path(dt, d.Dk, d.Dv, d.chunk)) return (size_t)d.B * d.H * (size_t)d.nchunks() * TC_STATE_BYTES;
@@ -140,6 +143,7 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
         a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
         a.S0 = S0; a.o = o; a.ST = ST;
         a.states = save_states ? static_cast<unsigned char*>(ws) : nullptr;
+        a.tp = save_states ? static_cast<unsigned char*>(ws) + tc_tp_offset(d) : nullptr;
         return cuda_status(chunk_fwd_launch(a, s), "gdn2_fwd (tensor-core path)");
     }
     RecurrentArgs a{};
@@ -181,7 +185,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
             ChunkFwdArgs f{};
             f.d = d;
             f.q = q; f.k = k; f.v = v; f.la = log_alpha; f.b = b; f.w = w;
-            f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb;
+            f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.tp = wsb + tc_tp_offset(d);
             gdn2_status e = cuda_status(chunk_fwd_launch(f, s), "gdn2_bwd state recompute");
             if (e != GDN2_OK) return e;
         }
@@ -191,6 +195,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
         a.dST = dST;
         a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.db = db; a.dw = dw; a.dS0 = dS0;
         a.states = wsb;
+        a.tp = wsb + tc_tp_offset(d);
         a.dstates = extra;
         return cuda_status(chunk_bwd_launch(a, s), "gdn2_bwd (tensor-core path)");
     }
