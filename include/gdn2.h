@@ -130,6 +130,38 @@ gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const 
                              const void* b, const void* w, float* S, void* o, int B, int H,
                              int Dk, int Dv, gdn2_dtype dt, void* stream);
 
+/*
+ * Backward without a caller-supplied workspace. The paper has no counterpart:
+ * this entry point exists for callers that cannot call cudaMalloc where they
+ * need gradients -- code running inside another component's memory management
+ * (a framework's caching allocator, a plugin handed only its tensors), code
+ * that must not synchronise the device (cudaMalloc/cudaFree may), or code that
+ * must not be able to fail for lack of memory after start-up.
+ *
+ * Same arguments and results as gdn2_bwd with states_saved = 0, minus the
+ * workspace: the scratch memory lives in a fixed array of
+ * GDN2_NO_ALLOC_SCRATCH_BYTES bytes inside the library, present on every GPU
+ * that loads the library until it is unloaded. Nothing is allocated.
+ *   - Problems whose gdn2_workspace_size(GDN2_OP_BWD, ...) exceeds that size
+ *     are rejected with GDN2_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture on the device.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents (nothing in it needs to start at zero). Calls whose work overlaps
+ *     on the GPU -- other streams or host threads on the same device -- race on
+ *     it: order them.
+ */
+#define GDN2_NO_ALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+gdn2_status gdn2_bwd_no_alloc(const void* q, const void* k, const void* v, const void* log_alpha,
+                              const void* b, const void* w, const float* S0, const void* dout,
+                              const float* dST, void* dq, void* dk, void* dv, void* dlog_alpha,
+                              void* db, void* dw, float* dS0, int B, int T, int H, int Dk, int Dv,
+                              int chunk, gdn2_dtype dt, void* stream);
+
+/* Size in bytes of the fixed scratch array used by gdn2_bwd_no_alloc. */
+size_t gdn2_no_alloc_scratch_bytes(void);
+
 /* Static description of a status code. */
 const char* gdn2_status_string(gdn2_status s);
 

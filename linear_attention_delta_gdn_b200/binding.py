@@ -27,7 +27,7 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GD
 
 #: exported symbols, as declared in include/gdn2.h
 EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "gdn2_status_string",
-           "gdn2_last_error", "gdn2_version")
+           "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes")
 
 
 class Gdn2Error(RuntimeError):
@@ -60,6 +60,10 @@ def lib(path: Optional[str] = None) -> ctypes.CDLL:
     L.gdn2_last_error.restype = ctypes.c_char_p
     L.gdn2_version.argtypes = []
     L.gdn2_version.restype = I
+    L.gdn2_bwd_no_alloc.argtypes = [P] * 16 + [I] * 7 + [P]
+    L.gdn2_bwd_no_alloc.restype = I
+    L.gdn2_no_alloc_scratch_bytes.argtypes = []
+    L.gdn2_no_alloc_scratch_bytes.restype = Z
     if path is None:
         _lib = L
     return L

@@ -89,6 +89,10 @@ gdn2_status copy_or_zero_state(float* dst, const float* src, const Dims& d, cuda
 
 }  // namespace
 
+namespace gdn2 {
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace gdn2
+
 extern "C" {
 
 int gdn2_version(void) { return 100; }

@@ -56,6 +56,9 @@ struct ChunkBwdArgs {
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 
+// Sets the detail string returned by gdn2_last_error() on this host thread.
+void set_last_error(const char* msg);
+
 // Whether the tensor-core forward handles this problem.
 inline bool tc_path(gdn2_dtype dt, int Dk, int Dv, int chunk) {
     return dt == GDN2_BF16 && Dk == TC_D && Dv == TC_D && chunk == TC_C;
