@@ -30,12 +30,44 @@ sys.path.insert(0, ROOT)
 METRIC = "GDN-2 fwd+bwd tokens/s (H16 d128 T4K bf16, 1×B200); % of roofline"
 WORKLOAD = "fwdbwd-bf16-b4h16t4096d128"
 
-# Algorithmic work per token and head (C = 64, d = 128): forward reads q, k, v,
-# log_alpha, b, w and writes o (7 x 256 B); the backward re-reads the six inputs,
-# reads dout and writes six gradients (13 x 256 B). Flops: forward 180,224
-# (the chunk contractions), backward counted as twice the forward.
-BYTES_PER_TOKEN_HEAD = {"fwd": 1792, "bwd": 3328}
-FLOPS_PER_TOKEN_HEAD = {"fwd": 180224, "bwd": 2 * 180224}
+# Algorithmic work per token and head (C = 64, d = 128, bf16 tensors of 256 B per
+# token and head). The step: the forward reads q, k, v, log_alpha, b, w and writes
+# o (7 x 256 B); the backward reads the six inputs and dout and writes six
+# gradients (13 x 256 B); plus the fp32 final state and dS0 per head. Per kernel:
+#   chunk_fwd_kernel      7 x 256 B  (its inputs and o)
+#   reverse_state_kernel  5 x 256 B  (q, k, log_alpha, b, dout)
+#   chunk_grad_kernel    13 x 256 B  (all backward inputs and gradients)
+# Flops: forward 180,224 per token and head (the chunk contractions), backward
+# counted as twice the forward.
+STEP_BYTES_PER_TOKEN_HEAD = 1792 + 3328
+STEP_FLOPS_PER_TOKEN_HEAD = 3 * 180224
+KERNEL_BYTES_PER_TOKEN_HEAD = {"chunk_fwd_kernel": 1792, "reverse_state_kernel": 1280, "chunk_grad_kernel": 3328,
+                               "recurrent_fwd_kernel": 1792, "recurrent_bwd_kernel": 3328}
+KERNEL_SOURCES = {"chunk_fwd_kernel": ["chunk_fwd.cu"], "reverse_state_kernel": ["chunk_bwd.cu"],
+                  "chunk_grad_kernel": ["chunk_bwd.cu"]}
+COMMON_SOURCES = ["chunk_common.cuh", "tc.cuh", "common.cuh"]
+
+
+def kernel_source_hash(kernel):
+    """sha256 over the CUDA sources a kernel is built from (to tell whether recorded counters still apply)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []) + COMMON_SOURCES:
+        with open(os.path.join(ROOT, "linear_attention_delta_gdn_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel, token_heads):
+    """DRAM bytes per launch from profiles/kernel_traffic.json, scaled to this launch, if still valid."""
+    p = os.path.join(ROOT, "profiles", "kernel_traffic.json")
+    if not os.path.exists(p) or kernel not in KERNEL_SOURCES:
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("source_sha256") != kernel_source_hash(kernel):
+        return None
+    return rec["dram_bytes_per_token_head"] * token_heads
 
 
 def peaks():
@@ -104,7 +136,8 @@ def make_host_inputs(rank, B=None, T=None):
     wl = WORKLOADS[WORKLOAD]
     if B or T:
         wl = dataclasses.replace(wl, name="%s-B%d-T%d" % (wl.name, B or wl.B, T or wl.T), B=B or wl.B, T=T or wl.T)
-    return wl, make_inputs(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, wl.seed + 7919 * rank, wl.dtype, with_do=True)
+    from linear_attention_delta_gdn_b200.replicas import rank_seed
+    return wl, make_inputs(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, rank_seed(wl.seed, rank), wl.dtype, with_do=True)
 
 
 def cpu_baseline(wl, x, budget_s=20.0, steps=1):
@@ -220,10 +253,9 @@ def main():
     torch.cuda.synchronize(dev)
 
     # ---- device-timed region: inputs resident in HBM (470 MB per step, larger than L2)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clock_log = os.path.join(ROOT, "gpurun_out", "bench_clocks_rank%d.csv" % rank)
     os.makedirs(os.path.dirname(clock_log), exist_ok=True)
+    binding.trace_read()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -231,29 +263,21 @@ def main():
         time.sleep(0.3)
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
+        binding.trace_enable(True)
         start.record(stream)
         for i in range(args.steps):
-            e0, e1, e2 = ev[i]
-            e0.record(stream)
-            binding.gdn2_fwd(*(d[n] for n in names), None, chunk=chunk, save_states=True, ws=ws, o=o, ST=ST)
-            e1.record(stream)
-            binding.gdn2_bwd(*(d[n] for n in names), d["dout"], None, None, chunk=chunk, states_saved=True,
-                             ws=ws, grads=grads)
-            e2.record(stream)
+            step(d)
         end.record(stream)
+        binding.trace_enable(False)
         torch.cuda.synchronize(dev)
+    kernels = binding.trace_read()       # {name: (launches, summed device ms)} of the timed region
     if world > 1:
         dist.barrier()
-    total_ms = start.elapsed_time(end)
-    fwd_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in ev)
-    bwd_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in ev)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = t.item()
+    from linear_attention_delta_gdn_b200.replicas import aggregate_tokens_per_s, max_over_ranks
+    total_ms = max_over_ranks(start.elapsed_time(end), dist, dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = B * T
-    value = world * tokens_per_step / (ms_per_step / 1e3)
+    value = aggregate_tokens_per_s(world, tokens_per_step, ms_per_step)
 
     # ---- end to end through host buffers: H2D inputs, fwd + bwd, D2H o and gradients
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
@@ -271,30 +295,26 @@ def main():
             h_.copy_(t, non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e_start.elapsed_time(e_end) / max(1, args.e2e_steps)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e_value = world * tokens_per_step / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / max(1, args.e2e_steps), dist, dev)
+    e2e_value = aggregate_tokens_per_s(world, tokens_per_step, e2e_ms)
 
-    # ---- roofline of the dominant call
+    # ---- roofline of the dominant kernel (device time summed over the timed region)
     pk = peaks()
     th = B * T * H
-    calls = {"fwd": fwd_ms, "bwd": bwd_ms}
-    dom = max(calls, key=calls.get)
-    alg_bytes = th * BYTES_PER_TOKEN_HEAD[dom] + (B * H * Dk * Dv * 4 if dom == "bwd" else B * H * Dk * Dv * 4)
-    achieved = alg_bytes / (calls[dom] / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "gdn2_%s" % dom, "achieved": achieved, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                "peak_source": pk["source"], "alg_bytes_per_launch": alg_bytes,
-                "call_ms": {"fwd": fwd_ms, "bwd": bwd_ms},
-                "step_frac": (th * sum(BYTES_PER_TOKEN_HEAD.values()) + 2 * B * H * Dk * Dv * 4)
+    dom = max(kernels, key=lambda k: kernels[k][1])
+    n_launch, dom_ms = kernels[dom]
+    per_launch_s = dom_ms / n_launch / 1e3
+    alg_bytes = th * KERNEL_BYTES_PER_TOKEN_HEAD.get(dom, STEP_BYTES_PER_TOKEN_HEAD)
+    achieved = alg_bytes / per_launch_s / 1e9
+    traffic = recorded_traffic(dom, th)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_source": pk["source"],
+                "alg_bytes_per_launch": alg_bytes, "launch_ms": per_launch_s * 1e3,
+                "kernels_ms_per_step": {k: v[1] / args.steps for k, v in kernels.items()},
+                "step_alg_bytes": th * STEP_BYTES_PER_TOKEN_HEAD + 2 * B * H * Dk * Dv * 4,
+                "step_frac": (th * STEP_BYTES_PER_TOKEN_HEAD + 2 * B * H * Dk * Dv * 4)
                 / (ms_per_step / 1e3) / 1e9 / pk["hbm_gbs"]}
-
-    tc = binding.gdn2_workspace_size(binding.GDN2_OP_FWD_SAVE, B, T, H, Dk, Dv, chunk, binding.GDN2_BF16) \
-        < B * H * ((T + chunk - 1) // chunk) * Dk * Dv * 4
-    launches_per_step = (1 + 2) if tc else (1 + 1)
+    launches_in_timed_region = sum(v[0] for v in kernels.values())
 
     line = None
     if rank == 0:
@@ -309,11 +329,11 @@ def main():
                            "global_batch": world * B, "seq_len": T,
                            "parallelism": "dp%d (independent batches, no collective)" % world,
                            "l2": "inputs larger than L2 (%.0f MB read per step)" % (h2d / 1e6),
-                           "path": "tensor-core chunkwise" if tc else "fp32 recurrent"},
+                           "kernels": sorted(kernels)},
                 "roofline": roofline, "cpu_baseline": cb, "clocks": clocks.summary(),
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
-                "gpu_launches": launches_per_step * args.steps}
+                "gpu_launches": launches_in_timed_region}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

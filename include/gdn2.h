@@ -162,6 +162,18 @@ gdn2_status gdn2_bwd_no_alloc(const void* q, const void* k, const void* v, const
 /* Size in bytes of the fixed scratch array used by gdn2_bwd_no_alloc. */
 size_t gdn2_no_alloc_scratch_bytes(void);
 
+/*
+ * Per-kernel timing, for profiling. gdn2_trace_enable(1) makes every later
+ * kernel launch of the library record a CUDA event before and after it on the
+ * launch's stream (gdn2_trace_enable(0) stops it; off by default).
+ * gdn2_trace_read waits for the recorded events, writes up to max_kernels
+ * entries -- comma-separated kernel names into names (capacity names_cap),
+ * launch counts into launches, summed device milliseconds into ms -- returns
+ * the number of entries, and clears the record. Host pointers; any may be NULL.
+ */
+void gdn2_trace_enable(int on);
+int gdn2_trace_read(char* names, size_t names_cap, int* launches, double* ms, int max_kernels);
+
 /* Static description of a status code. */
 const char* gdn2_status_string(gdn2_status s);
 

@@ -27,7 +27,8 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GD
 
 #: exported symbols, as declared in include/gdn2.h
 EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "gdn2_status_string",
-           "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes")
+           "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes",
+           "gdn2_trace_enable", "gdn2_trace_read")
 
 
 class Gdn2Error(RuntimeError):
@@ -64,6 +65,10 @@ def lib(path: Optional[str] = None) -> ctypes.CDLL:
     L.gdn2_bwd_no_alloc.restype = I
     L.gdn2_no_alloc_scratch_bytes.argtypes = []
     L.gdn2_no_alloc_scratch_bytes.restype = Z
+    L.gdn2_trace_enable.argtypes = [I]
+    L.gdn2_trace_enable.restype = None
+    L.gdn2_trace_read.argtypes = [ctypes.c_char_p, Z, P, P, I]
+    L.gdn2_trace_read.restype = I
     if path is None:
         _lib = L
     return L
@@ -181,6 +186,22 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None):
                                 B, H, Dk, Dv, _dt(q), _stream(q.device))
     _check("gdn2_decode_step", rc)
     return o
+
+
+def trace_enable(on: bool = True) -> None:
+    """Start (or stop) per-kernel event timing of the library's launches."""
+    lib().gdn2_trace_enable(1 if on else 0)
+
+
+def trace_read() -> dict:
+    """{kernel name: (launches, summed device ms)} since the last read (waits for the events)."""
+    n_max = 16
+    names = ctypes.create_string_buffer(1024)
+    launches = (ctypes.c_int * n_max)()
+    ms = (ctypes.c_double * n_max)()
+    n = lib().gdn2_trace_read(names, 1024, ctypes.cast(launches, ctypes.c_void_p), ctypes.cast(ms, ctypes.c_void_p), n_max)
+    keys = names.value.decode().split(",") if n else []
+    return {k: (int(launches[i]), float(ms[i])) for i, k in enumerate(keys)}
 
 
 class GatedDeltaRule2(torch.autograd.Function):

@@ -619,11 +619,15 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     e = set_smem(chunk_grad_kernel, cg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    reverse_state_kernel<<<d.B * d.H, NT, rs::SMEM_BYTES, s>>>(mq, mk, mla, mb, mdo, a.dST, a.dS0, a.tp, a.dstates,
-                                                                d.T, d.H);
+    {
+        TraceScope trace(K_REVERSE, s);
+        reverse_state_kernel<<<d.B * d.H, NT, rs::SMEM_BYTES, s>>>(mq, mk, mla, mb, mdo, a.dST, a.dS0, a.tp,
+                                                                    a.dstates, d.T, d.H);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const dim3 grid(d.nchunks(), d.B * d.H);
+    TraceScope trace(K_GRAD, s);
     chunk_grad_kernel<<<grid, NT, cg::SMEM_BYTES, s>>>(
         mq, mk, mv, mla, mb, mw, mdo, mdq, mdk, mdb, mdla, static_cast<__nv_bfloat16*>(a.dv),
         static_cast<__nv_bfloat16*>(a.dw), a.states, a.tp, a.dstates, d.T, d.H);

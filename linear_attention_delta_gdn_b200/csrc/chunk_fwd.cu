@@ -314,6 +314,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
         if (make_token_map(maps[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    TraceScope trace(K_CHUNK_FWD, s);
     chunk_fwd_kernel<<<d.B * d.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mla, mb, mw, a.S0,
                                                        static_cast<__nv_bfloat16*>(a.o), a.ST, a.states, a.tp, d.T, d.H);
     return cudaGetLastError();

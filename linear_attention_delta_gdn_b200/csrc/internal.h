@@ -56,6 +56,24 @@ struct ChunkBwdArgs {
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 
+// Kernels of the library, for gdn2_trace_read().
+enum KernelId { K_CHUNK_FWD = 0, K_REVERSE, K_GRAD, K_REC_FWD, K_REC_BWD, K_DECODE, KERNEL_COUNT };
+
+// Brackets one kernel launch with CUDA events on its stream while tracing is on.
+class TraceScope {
+  public:
+    TraceScope(KernelId id, cudaStream_t s);
+    ~TraceScope();
+    TraceScope(const TraceScope&) = delete;
+    TraceScope& operator=(const TraceScope&) = delete;
+
+  private:
+    KernelId id_;
+    cudaStream_t stream_;
+    cudaEvent_t start_;
+    bool active_;
+};
+
 // Sets the detail string returned by gdn2_last_error() on this host thread.
 void set_last_error(const char* msg);
 

@@ -335,20 +335,26 @@ cudaError_t launch_all(const RecurrentArgs& a, cudaStream_t s) {
     const Tin* b = static_cast<const Tin*>(a.b);
     const Tin* w = static_cast<const Tin*>(a.w);
     switch (a.op) {
-    case RecurrentArgs::DECODE:
+    case RecurrentArgs::DECODE: {
+        TraceScope trace(K_DECODE, s);
         decode_kernel<Tin, DK, DV><<<grid, L::NT, 0, s>>>(q, k, v, la, b, w, a.S, static_cast<Tin*>(a.o));
         break;
-    case RecurrentArgs::FWD:
+    }
+    case RecurrentArgs::FWD: {
+        TraceScope trace(K_REC_FWD, s);
         fwd_kernel<Tin, DK, DV><<<grid, L::NT, 0, s>>>(q, k, v, la, b, w, a.S0, static_cast<Tin*>(a.o),
                                                        a.ST, a.states, d.T, d.H, d.chunk);
         break;
-    case RecurrentArgs::BWD:
+    }
+    case RecurrentArgs::BWD: {
+        TraceScope trace(K_REC_BWD, s);
         bwd_kernel<Tin, DK, DV><<<grid, L::NT, 0, s>>>(
             q, k, v, la, b, w, static_cast<const Tin*>(a.dout), a.dST, static_cast<Tin*>(a.dq),
             static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), static_cast<Tin*>(a.dla),
             static_cast<Tin*>(a.db), static_cast<Tin*>(a.dw), a.dS0, a.states, a.seg, a.segdelta,
             d.T, d.H, d.chunk);
         break;
+    }
     }
     return cudaGetLastError();
 }
