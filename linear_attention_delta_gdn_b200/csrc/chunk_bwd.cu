@@ -53,10 +53,10 @@ constexpr uint32_t OFF_ST = 98304;       // dZ^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16)
 constexpr uint32_t OFF_TT = 147456;      // T (bf16, from the forward)
 constexpr uint32_t OFF_PP = 155648;      // P (bf16, from the forward)
-constexpr uint32_t OFF_RED = 163840;     // prep scan scratch (4 KB)
-constexpr uint32_t OFF_GC = 167936;
-constexpr uint32_t OFF_BAR = 168448;
-constexpr uint32_t SMEM_BYTES = 168512 + 1024;
+constexpr uint32_t OFF_RED = 163840;     // prep scan scratch (8 KB)
+constexpr uint32_t OFF_GC = 172032;
+constexpr uint32_t OFF_BAR = 172544;
+constexpr uint32_t SMEM_BYTES = 172608 + 1024;
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_W = 192, TM_COLS = 512;
 constexpr uint32_t LOAD_BYTES = 5 * 64 * 128 * 2 + 2 * TILE_C;
 }  // namespace rs
@@ -105,7 +105,8 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_base_ptr;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
+    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
 
     auto issue_loads = [&](int c) {
         const int t0 = c * C;
@@ -122,10 +123,10 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     if (tid == 0) issue_loads(nc - 1);
 
     {   // dS_{NC}^T = dST^T (or zero): lane j holds column j of dST
-        const int j = tid;
+        const int j = jrow;
         float v[32];
 #pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 32) {
+        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] = dST ? dST[(head * D + i0 + u) * D + j] : 0.f;
             tc::tmem_st32(lane_base + TM_S + i0, v);
@@ -166,10 +167,10 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         if (tid == 0) tc::bulk_wait_read();
         __syncthreads();
         {
-            const int j = tid;
+            const int j = jrow;
             float v[32];
 #pragma unroll 1
-            for (int i0 = 0; i0 < D; i0 += 32) {
+            for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
                 tc::tmem_wait_ld();
 #pragma unroll
@@ -200,7 +201,7 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         }
         wait_mma();
         tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);    // Wm rows
-        tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);      // dDelta^T rows
+        tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
 
         // dS^T = dZ^T + dO^T Qt - dDelta^T Wm
@@ -222,10 +223,10 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     }
 
     if (dS0) {   // dS0[i][j] from dS^T (lane j)
-        const int j = tid;
+        const int j = jrow;
         float v[32];
 #pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 32) {
+        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
             tc::tmem_ld32(lane_base + TM_S + i0, v);
             tc::tmem_wait_ld();
 #pragma unroll
@@ -338,7 +339,8 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_base_ptr;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
+    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
     uint32_t ph_mma = 0;
     bool ok = tc::mbar_wait(bar_load, 0);
     auto wait_mma = [&]() {
@@ -398,8 +400,8 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);      // Delta^T [j][t]
-    tmem_to_tile_rows<64>(lane_base + TM_DD, DDT, tid);    // dDelta^T [j][t]
+    tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);     // Delta^T [j][t]
+    tmem_to_tile_rows<64>(lane_base + TM_DD, DDT, warp, lane);   // dDelta^T [j][t]
     sync_for_mma();
 
     // ---- dU = T^T dDelta (M=64)
@@ -417,7 +419,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         const bool row_ok = lane < 16 && t < L;
         float v[32];
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
             tc::tmem_ld32(lane_base + TM_DU + c0, v);
             tc::tmem_wait_ld();
             if (lane < 16) {
@@ -463,30 +465,24 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    {   // M=64 accumulators: rows s = 16 warp + lane (lanes < 16)
-        const int s = m64_row(warp, lane);
+    {   // M=64 accumulators: rows s = 16 q + lane (lanes < 16); the warps of a quarter take 32 columns each
+        const int s_ = m64_row(warp, lane), c0 = 32 * tm_part(warp);
         float v[32];
+        tc::tmem_ld32(lane_base + TM_AP + c0, v);
+        tc::tmem_wait_ld();
+        if (lane < 16) {
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            tc::tmem_ld32(lane_base + TM_AP + 32 * h2, v);
-            tc::tmem_wait_ld();
-            if (lane < 16) {
+            for (int u = 0; u < 32; ++u) v[u] = (s_ <= c0 + u) ? v[u] : 0.f;   // dP[t][s], t >= s
 #pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] = (s <= 32 * h2 + u) ? v[u] : 0.f;   // dP[t][s], t >= s
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, s, 4 * h2 + g, v + 8 * g);
-            }
+            for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, s_, (c0 >> 3) + g, v + 8 * g);
         }
+        tc::tmem_ld32(lane_base + TM_W + c0, v);
+        tc::tmem_wait_ld();
+        if (lane < 16) {
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            tc::tmem_ld32(lane_base + TM_W + 32 * h2, v);
-            tc::tmem_wait_ld();
-            if (lane < 16) {
+            for (int u = 0; u < 32; ++u) v[u] = (s_ < c0 + u) ? v[u] : 0.f;    // dA[t][s], t > s
 #pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] = (s < 32 * h2 + u) ? v[u] : 0.f;    // dA[t][s], t > s
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(TT, C, s, 4 * h2 + g, v + 8 * g);
-            }
+            for (int g = 0; g < 4; ++g) tc::st_row8(TT, C, s_, (c0 >> 3) + g, v + 8 * g);
         }
     }
     sync_for_mma();
@@ -516,41 +512,34 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::mma_commit(bar_mma);
     }
 
-    // rowsum(dZ * S) for key channel i (both images hold row j = value channel)
-    const int i = tid;
-    float E = 0.f;
+    // rowsum(dZ * S) for key channel i, this half's value channels (both images hold row j = value channel)
+    const int i = tid & 127, hf = tid >> 7;
+    float Epart = 0.f;
     {
         float e2 = 0.f;
 #pragma unroll 8
-        for (int j = 0; j < D; j += 2) {
-            E += tc::ld_bf16(DS, tc::tile_off(D, j, i)) * tc::ld_bf16(STt, tc::tile_off(D, j, i));
+        for (int j = 64 * hf; j < 64 * hf + 64; j += 2) {
+            Epart += tc::ld_bf16(DS, tc::tile_off(D, j, i)) * tc::ld_bf16(STt, tc::tile_off(D, j, i));
             e2 += tc::ld_bf16(DS, tc::tile_off(D, j + 1, i)) * tc::ld_bf16(STt, tc::tile_off(D, j + 1, i));
         }
-        E += e2;
+        Epart += e2;
     }
     wait_mma();
     ok = tc::mbar_wait(bar_k, 0) && ok;
     ok = tc::mbar_wait(bar_b, 0) && ok;
 
-    // ---- gate chain, thread = key channel i: E += sum_t Kt G4, then tokens in reverse.
+    // ---- gate chain, thread = (key channel i, token half hf). Pass 1 over the half's 32 tokens: dq, dk,
+    // db and dG_t; partial sums of Kt*G4 and dG are exchanged between the halves (in the consumed dP^T
+    // tile). Pass 2: dlog_alpha_t = sum_{tau >= t} dG_tau + E, E = rowsum(dZ*S) + sum_t Kt*G4.
     // Results go to bf16 row tiles (dq -> DO, dk -> DT, db -> DDT, dlog_alpha -> UU), stored by TMA.
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chk = (uint32_t)((i & 63) >> 3);
-#pragma unroll 1
-    for (int q4 = 0; q4 < 4; ++q4) {
-        float g4[16];
-        tc::tmem_ld16(lane_base + TM_G4 + 16 * q4, g4);
-        tc::tmem_wait_ld();
+    float dG[32];
+    float dGsum = 0.f;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const uint32_t t = (uint32_t)(16 * q4 + u);
-            E += tc::ld_bf16(KT, col64 + t * 128 + ((chk ^ (t & 7)) << 4)) * g4[u];
-        }
-    }
-    float suffix = 0.f;
-#pragma unroll 1
-    for (int q4 = 3; q4 >= 0; --q4) {
+    for (int qq = 0; qq < 2; ++qq) {
+        const int q4 = 2 * hf + qq;
         float g1[16], g2[16], g3[16], g4[16], gv[16];
         tc::tmem_ld16(lane_base + TM_G1 + 16 * q4, g1);
         tc::tmem_ld16(lane_base + TM_G2 + 16 * q4, g2);
@@ -559,7 +548,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::tmem_ld16(lane_base + TM_GV + 16 * q4, gv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int u = 15; u >= 0; --u) {
+        for (int u = 0; u < 16; ++u) {
             const uint32_t t = (uint32_t)(16 * q4 + u);
             const uint32_t sw = t * 128 + ((chk ^ (t & 7)) << 4);
             const float qt = tc::ld_bf16(QE, col128 + C * 128 + sw);
@@ -569,13 +558,27 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
             const float bb = tc::ld_bf16(WW, col64 + sw);
             const float g = fast_exp(gv[u]), ig = fast_exp(-gv[u]);
             const float dKt = g3[u] + g4[u];
-            suffix += qt * g1[u] + et * g2[u] - kt * dKt;
+            const float dGt = qt * g1[u] + et * g2[u] - kt * dKt;
+            dG[16 * qq + u] = dGt;
+            dGsum += dGt;
+            Epart += kt * g4[u];
             const float dE = g * g2[u];
             tc::st_bf16(DO, col64 + sw, g * g1[u]);                 // dq
             tc::st_bf16(DT, col64 + sw, dKt * ig + dE * bb);        // dk
             tc::st_bf16(DDT, col64 + sw, dE * kk);                  // db
-            tc::st_bf16(UU, col64 + sw, suffix + E);                // dlog_alpha
         }
+    }
+    float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][2 halves][128]
+    xch[(0 * 2 + hf) * 128 + i] = Epart;
+    xch[(1 * 2 + hf) * 128 + i] = dGsum;
+    __syncthreads();
+    const float E = xch[(0 * 2 + 0) * 128 + i] + xch[(0 * 2 + 1) * 128 + i];
+    float suffix = hf == 0 ? xch[(1 * 2 + 1) * 128 + i] : 0.f;      // dG of the later half
+#pragma unroll
+    for (int u = 31; u >= 0; --u) {
+        const uint32_t t = (uint32_t)(32 * hf + u);
+        suffix += dG[u];
+        tc::st_bf16(UU, col64 + t * 128 + ((chk ^ (t & 7)) << 4), suffix + E);    // dlog_alpha
     }
     tc::fence_async_smem();
     __syncthreads();

@@ -31,7 +31,11 @@ namespace chunk {
 
 constexpr int D = 128;        // d_k = d_v
 constexpr int C = 64;         // chunk length
-constexpr int NT = 128;       // threads per CTA (one warpgroup; thread i <-> TMEM lane i)
+constexpr int NT = 256;       // threads per CTA (two warpgroups)
+// TMEM access: warp w reads lane quarter (w % 4), i.e. lanes 32 (w % 4) .. +31; the two warps of a
+// quarter (w and w + 4) split the columns of each read-out between them (part = w / 4).
+__device__ __forceinline__ int tm_quarter(int warp) { return warp & 3; }
+__device__ __forceinline__ int tm_part(int warp) { return warp >> 2; }
 constexpr uint32_t TILE_64x128 = 64 * 128 * 2;    // bytes of a [64 x 128] bf16 row tile
 
 // ------------------------------------------------------------ host: TMA maps
@@ -67,26 +71,37 @@ __device__ __forceinline__ void tma_tile(unsigned char* dst, int R, int dst_row0
     tc::tma_load_4d(dst + R * 128 + dst_row0 * 128, map, 64, h, t0, b, bar);
 }
 
-// Gate preparation, channel-major variant: one thread per key/value channel i (= threadIdx.x),
-// tokens in blocks of 8 (loads of a block are issued together, then its stores):
+// Gate preparation, channel-major variant: thread = (key/value channel i = tid % 128,
+// token half hf = tid / 128: tokens 32 hf .. 32 hf + 31), tokens in blocks of 8:
 //   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
 //   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127, Kt = k/g -> KT,
 //          U = w*v -> KH (over k, which the thread has read); UU and WW keep v and w.
 //   g = exp(G), G = inclusive cumsum of log_alpha; gC[i] = g at the last row.
-//   G[t][i] is also stored to TMEM at tmem_g (lane i, columns t).
+//   G[t][i] is also stored to TMEM at tmem_g (lane i, column t); tmem_g is the thread's lane base.
 __device__ __forceinline__ void gate_prep_cols(unsigned char* QE, unsigned char* KH, unsigned char* KT,
                                                const unsigned char* UU, const unsigned char* WW, float* gC_out,
-                                               int i, uint32_t tmem_g) {
+                                               int tid, uint32_t tmem_g) {
+    const int i = tid & 127, hf = tid >> 7;
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chunk = (uint32_t)((i & 63) >> 3);
     float G = 0.f;
+    if (hf) {   // the second half starts from the sum over the first 32 tokens
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+        for (int t = 0; t < 32; t += 2) {
+            s0 += tc::ld_bf16(KT, col64 + (uint32_t)t * 128 + ((chunk ^ (uint32_t)(t & 7)) << 4));
+            s1 += tc::ld_bf16(KT, col64 + (uint32_t)(t + 1) * 128 + ((chunk ^ (uint32_t)((t + 1) & 7)) << 4));
+        }
+        G = s0 + s1;
+    }
+    __syncthreads();   // every thread has read the log_alpha it needs before Kt overwrites it
 #pragma unroll 1
-    for (int tb2 = 0; tb2 < C / 16; ++tb2) {
+    for (int tb2 = 0; tb2 < 2; ++tb2) {
         float gvals[16];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-            const int tb = 2 * tb2 + half;
+            const int tb = 4 * hf + 2 * tb2 + half;
             float la[8], kk[8], bb[8], qq[8], vv[8], ww[8];
             uint32_t o64[8], o128[8];
 #pragma unroll
@@ -113,46 +128,52 @@ __device__ __forceinline__ void gate_prep_cols(unsigned char* QE, unsigned char*
                 tc::st_bf16(KH, o64[u], ww[u] * vv[u]);               // U
             }
         }
-        tc::tmem_st16(tmem_g + 16 * tb2, gvals);
+        tc::tmem_st16(tmem_g + 32 * hf + 16 * tb2, gvals);
     }
     tc::tmem_wait_st();
-    gC_out[i] = fast_exp(G);
+    if (hf) gC_out[i] = fast_exp(G);
 }
 
-// Gate preparation, vectorised: thread = (8-token block tb = tid / 16, 8-channel group cg = tid % 16),
-// 16-byte shared-memory accesses. Same inputs/outputs as gate_prep_cols (without the TMEM copy of G).
-// The in-chunk cumsum is a local scan over the thread's 8 rows plus the totals of the earlier
-// blocks, exchanged through `red` (fp32 [8][128], 4 KB). Contains one __syncthreads.
+// Gate preparation, vectorised: thread = (4-token block tb = tid / 16, 8-channel group cg = tid % 16),
+// 16-byte shared-memory accesses:
+//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
+//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127 (want_q),
+//          Kt = k/g -> KT, U = w*v -> UU (want_u); KH keeps k.
+//   g = exp(G), G = inclusive cumsum of log_alpha over the chunk; gC[i] = g at the last row.
+// The cumsum is a local scan over the thread's 4 rows plus the totals of the earlier blocks,
+// exchanged through `red` (fp32 [16][128], 8 KB). Contains one __syncthreads.
 __device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
                                           unsigned char* UU, const unsigned char* WW, float* gC_out,
                                           float* red, int tid, bool want_q, bool want_u) {
+    constexpr int RB = 4;                       // rows per thread
     const int cg = tid & 15, tb = tid >> 4;
-    float G[8][8];
+    float G[RB][8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        tc::ld_row8(KT, C, 8 * tb + u, cg, G[u]);
+    for (int u = 0; u < RB; ++u) {
+        tc::ld_row8(KT, C, RB * tb + u, cg, G[u]);
         if (u > 0) {
 #pragma unroll
             for (int c = 0; c < 8; ++c) G[u][c] += G[u - 1][c];
         }
     }
-    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg) = make_float4(G[7][0], G[7][1], G[7][2], G[7][3]);
-    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg + 4) = make_float4(G[7][4], G[7][5], G[7][6], G[7][7]);
+    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg) = make_float4(G[RB - 1][0], G[RB - 1][1], G[RB - 1][2], G[RB - 1][3]);
+    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg + 4) = make_float4(G[RB - 1][4], G[RB - 1][5], G[RB - 1][6], G[RB - 1][7]);
     __syncthreads();
     float pre[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
     for (int p = 0; p < tb; ++p) {
         const float4 x0 = *reinterpret_cast<const float4*>(red + p * 128 + 8 * cg);
         const float4 x1 = *reinterpret_cast<const float4*>(red + p * 128 + 8 * cg + 4);
         pre[0] += x0.x; pre[1] += x0.y; pre[2] += x0.z; pre[3] += x0.w;
         pre[4] += x1.x; pre[5] += x1.y; pre[6] += x1.z; pre[7] += x1.w;
     }
-    if (tb == 7) {
+    if (tb == C / RB - 1) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) gC_out[8 * cg + c] = fast_exp(pre[c] + G[7][c]);
+        for (int c = 0; c < 8; ++c) gC_out[8 * cg + c] = fast_exp(pre[c] + G[RB - 1][c]);
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const int row = 8 * tb + u;
+    for (int u = 0; u < RB; ++u) {
+        const int row = RB * tb + u;
         float kk[8], bb[8], qq[8], vv[8], ww[8];
         tc::ld_row8(KH, C, row, cg, kk);
         tc::ld_row8(QE, 2 * C, row, cg, bb);
@@ -181,33 +202,24 @@ __device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char
 __device__ __forceinline__ int sq_idx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
 
 // Copy the strictly lower part of [A; P] from TMEM (lanes 0..63 = A, 64..127 = P,
-// 64 columns at tm_ap) into the fp32 scratch sA (warps 0, 1) and, if want_p,
-// the causal part of P into the bf16 row tile PP (warps 2, 3).
+// 64 columns at the warp's lane base + column 0) into the fp32 scratch sA and, if want_p,
+// the causal part of P into the bf16 row tile PP. Each warp handles 32 of the 64 columns.
 __device__ __forceinline__ void extract_AP(uint32_t lane_base_ap, float* sA, unsigned char* PP, bool want_p,
-                                           int tid) {
+                                           int warp, int lane) {
+    const int q = tm_quarter(warp), c0 = 32 * tm_part(warp);
     float v[32];
-    if (tid < 64) {
-        const int t = tid;
+    tc::tmem_ld32(lane_base_ap + c0, v);
+    tc::tmem_wait_ld();
+    if (q < 2) {
+        const int t = 32 * q + lane;
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            tc::tmem_ld32(lane_base_ap + 32 * h2, v);
-            tc::tmem_wait_ld();
+        for (int u = 0; u < 32; ++u) sA[sq_idx(t, c0 + u)] = v[u];
+    } else if (want_p) {
+        const int t = 32 * (q - 2) + lane;
 #pragma unroll
-            for (int u = 0; u < 32; ++u) sA[sq_idx(t, 32 * h2 + u)] = v[u];
-        }
-    } else {
-        const int t = tid - 64;
+        for (int u = 0; u < 32; ++u) v[u] = (c0 + u <= t) ? v[u] : 0.f;
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            tc::tmem_ld32(lane_base_ap + 32 * h2, v);
-            tc::tmem_wait_ld();
-            if (want_p) {
-#pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] = (32 * h2 + u <= t) ? v[u] : 0.f;
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, t, 4 * h2 + g, v + 8 * g);
-            }
-        }
+        for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, t, (c0 >> 3) + g, v + 8 * g);
     }
 }
 
@@ -223,13 +235,13 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], uint32_t a0, uint
                  : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// Row stride of the per-warp 16 x 16 fp32 temporaries (conflict-free fragment loads).
+// Row stride of the per-warp 16 x 8 fp32 temporaries (conflict-free fragment loads).
 constexpr int XS = 24;
-// acc (16 x 16, two m16n8 C fragments) += A[ar.., ac..] (16 x 16) * B (16 x 16), one warp,
-// tf32 inputs, fp32 accumulation. A comes from a 64 x 64 scratch (sq_idx layout); B from
-// the same layout (b_sq) or from a per-warp temporary with row stride XS.
-__device__ __forceinline__ void warp_mm16(float (&acc)[2][4], const float* __restrict__ A, int ar, int ac,
-                                          const float* __restrict__ Bm, int br, int bc, bool b_sq, int lane) {
+// acc (16 x 8, one m16n8 C fragment) += A[ar.., ac..] (16 x 16) * B[br.., bc..] (16 x 8), one warp,
+// tf32 inputs, fp32 accumulation. A comes from a 64 x 64 scratch (sq_idx layout); B from the same
+// layout (b_sq) or from a per-warp 16 x 8 temporary with row stride XS.
+__device__ __forceinline__ void warp_mm16x8(float (&acc)[4], const float* __restrict__ A, int ar, int ac,
+                                            const float* __restrict__ Bm, int br, int bc, bool b_sq, int lane) {
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
@@ -237,69 +249,53 @@ __device__ __forceinline__ void warp_mm16(float (&acc)[2][4], const float* __res
         const uint32_t a1 = to_tf32(A[sq_idx(ar + g + 8, ac + 8 * ks + t4)]);
         const uint32_t a2 = to_tf32(A[sq_idx(ar + g, ac + 8 * ks + t4 + 4)]);
         const uint32_t a3 = to_tf32(A[sq_idx(ar + g + 8, ac + 8 * ks + t4 + 4)]);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int r0 = br + 8 * ks + t4, c0 = bc + 8 * nt + g;
-            const float x0 = b_sq ? Bm[sq_idx(r0, c0)] : Bm[r0 * XS + c0];
-            const float x1 = b_sq ? Bm[sq_idx(r0 + 4, c0)] : Bm[(r0 + 4) * XS + c0];
-            mma_tf32_16x8x8(acc[nt], a0, a1, a2, a3, to_tf32(x0), to_tf32(x1));
-        }
+        const int r0 = br + 8 * ks + t4, c0 = bc + g;
+        const float x0 = b_sq ? Bm[sq_idx(r0, c0)] : Bm[r0 * XS + c0];
+        const float x1 = b_sq ? Bm[sq_idx(r0 + 4, c0)] : Bm[(r0 + 4) * XS + c0];
+        mma_tf32_16x8x8(acc, a0, a1, a2, a3, to_tf32(x0), to_tf32(x1));
     }
 }
-// Store a 16 x 16 accumulator (times `scale`) to a sq_idx scratch at (rr, cc) or to a per-warp temporary.
-__device__ __forceinline__ void warp_store16(const float (&acc)[2][4], float* dst, int rr, int cc, bool sq,
-                                             float scale, int lane) {
+// Store a 16 x 8 accumulator (times scale) to a sq_idx scratch at (rr, cc) or to a per-warp temporary.
+__device__ __forceinline__ void warp_store16x8(const float (&acc)[4], float* dst, int rr, int cc, bool sq, float scale,
+                                               int lane) {
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int r = rr + g + ((e >> 1) << 3), c = cc + 8 * nt + 2 * t4 + (e & 1);
-            if (sq) dst[sq_idx(r, c)] = scale * acc[nt][e];
-            else dst[r * XS + c] = scale * acc[nt][e];
-        }
+    for (int e = 0; e < 4; ++e) {
+        const int r = rr + g + ((e >> 1) << 3), c = cc + 2 * t4 + (e & 1);
+        if (sq) dst[sq_idx(r, c)] = scale * acc[e];
+        else dst[r * XS + c] = scale * acc[e];
+    }
 }
-__device__ __forceinline__ void warp_load16(float (&acc)[2][4], const float* src, int lane) {
+__device__ __forceinline__ void warp_load16x8(float (&acc)[4], const float* src, int lane) {
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] = src[(g + ((e >> 1) << 3)) * XS + 8 * nt + 2 * t4 + (e & 1)];
+    for (int e = 0; e < 4; ++e) acc[e] = src[(g + ((e >> 1) << 3)) * XS + 2 * t4 + (e & 1)];
 }
-__device__ __forceinline__ void zero16(float (&acc)[2][4]) {
+// bf16 copy of a 16 x 8 accumulator (times scale) into the T row tile (64 x 64) at (rr, cc).
+__device__ __forceinline__ void warp_store16x8_tile(const float (&acc)[4], unsigned char* Ttile, int rr, int cc,
+                                                    float scale, int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    for (int hf = 0; hf < 2; ++hf) {
+        const int r = rr + g + 8 * hf, c = cc + 2 * t4;
+        *reinterpret_cast<uint32_t*>(Ttile + tc::tile_off(C, r, c)) =
+            tc::pack_bf16x2(scale * acc[2 * hf], scale * acc[2 * hf + 1]);
+    }
 }
 
-// bf16 copy of a 16 x 16 accumulator into the T row tile (64 x 64) at block (rr, cc), times scale.
-__device__ __forceinline__ void warp_store16_tile(const float (&acc)[2][4], unsigned char* Ttile, int rr, int cc,
-                                                  float scale, int lane) {
-    const int g = lane >> 2, t4 = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int r = rr + g + 8 * hf, c = cc + 8 * nt + 2 * t4;
-            *reinterpret_cast<uint32_t*>(Ttile + tc::tile_off(C, r, c)) =
-                tc::pack_bf16x2(scale * acc[nt][2 * hf], scale * acc[nt][2 * hf + 1]);
-        }
-}
-
-// (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32 scratch sA, sq_idx layout).
-// Writes the inverse to sTf (lower triangle incl. the unit diagonal is valid) and the bf16
-// row tile T (64 x 64, zeros above the diagonal).
-//   1. 16 x 16 diagonal blocks T_ii by right-looking forward substitution (warp i, lane =
-//      column): once x_m is final, every later row is updated with it, so the FMAs of one
-//      step are independent.
+// (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32 scratch sA, sq_idx layout), 8 warps.
+// Writes the inverse to sTf (lower triangle incl. the unit diagonal is valid) and the bf16 row
+// tile T (64 x 64, zeros above the diagonal).
+//   1. 16 x 16 diagonal blocks T_ii by right-looking forward substitution (warp i < 4, lane =
+//      column); warps 4..7 clear T above the diagonal blocks meanwhile.
 //   2. off-diagonal blocks T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj, by diagonals i - j = 1, 2, 3,
-//      as warp-level tf32 tensor-core products (mma.sync m16n8k8).
-// sX: 4 warps x 16 x XS floats (6 KB), must not alias the T tile.
+//      as warp-level tf32 tensor-core products (mma.sync m16n8k8); the warps w and w + 4 take the
+//      left and right 8 columns of a block.
+// sX: 8 warps x 16 x XS floats (12 KB), must not alias the T tile.
 __device__ __forceinline__ void solve_unit_lower(const float* __restrict__ sA, float* __restrict__ sTf,
                                                  float* __restrict__ sX, unsigned char* Ttile, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
-    {
+    if (warp < 4) {
         const int s = lane & 15, base = 16 * warp;
         float acc[16];
 #pragma unroll
@@ -317,120 +313,98 @@ __device__ __forceinline__ void solve_unit_lower(const float* __restrict__ sA, f
                 tc::st_bf16(Ttile, tc::tile_off(C, base + r, base + s), acc[r]);
             }
         }
-        // zeros above the diagonal blocks: rows base..base+15, columns base+16..63
+    } else {
+        // zeros above the diagonal blocks: block row br = warp - 4, columns 16 br + 16 .. 63
+        const int br = warp - 4, base = 16 * br;
         const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const int ngrp = (C - base - 16) / 8;        // 8-column groups to clear per row
+        const int ngrp = (C - base - 16) / 8;
         for (int e = lane; e < 16 * ngrp; e += 32)
             tc::st_row8(Ttile, C, base + (e / ngrp), (base + 16) / 8 + (e % ngrp), z);
     }
     __syncthreads();
+    const int blk = warp & 3, nt = warp >> 2, nc = 8 * nt;     // warp pair blk, column half nt
     float* Xw = sX + warp * 16 * XS;
-    float acc[2][4];
-    // diagonal 1: T_{j+1,j} (warps 0..2); warp 3 starts T_30's sum with A_30 T_00
-    if (warp < 3) {
-        const int j = warp, i = j + 1;
-        zero16(acc);
-        warp_mm16(acc, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j, true, lane);
-        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+    float acc[4];
+    // diagonal 1: T_{j+1,j} (pairs 0..2); pair 3 starts T_30's sum with A_30 T_00
+    if (blk < 3) {
+        const int j = blk, i = j + 1;
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        warp_mm16x8(acc, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j + nc, true, lane);
+        warp_store16x8(acc, Xw, 0, 0, false, 1.f, lane);
         __syncwarp();
-        zero16(acc);
-        warp_mm16(acc, sTf, 16 * i, 16 * i, Xw, 0, 0, false, lane);
-        warp_store16(acc, sTf, 16 * i, 16 * j, true, -1.f, lane);
-        warp_store16_tile(acc, Ttile, 16 * i, 16 * j, -1.f, lane);
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        warp_mm16x8(acc, sTf, 16 * i, 16 * i, Xw, 0, 0, false, lane);
+        warp_store16x8(acc, sTf, 16 * i, 16 * j + nc, true, -1.f, lane);
+        warp_store16x8_tile(acc, Ttile, 16 * i, 16 * j + nc, -1.f, lane);
     } else {
-        zero16(acc);
-        warp_mm16(acc, sA, 48, 0, sTf, 0, 0, true, lane);          // A_30 T_00
-        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        warp_mm16x8(acc, sA, 48, 0, sTf, 0, nc, true, lane);          // A_30 T_00
+        warp_store16x8(acc, Xw, 0, 0, false, 1.f, lane);
     }
     __syncthreads();
-    // diagonal 2: T_20 (warp 0), T_31 (warp 1); warp 3 adds A_31 T_10 to its partial
-    if (warp < 2) {
-        const int j = warp, i = j + 2;
-        zero16(acc);
-        warp_mm16(acc, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j, true, lane);
-        warp_mm16(acc, sA, 16 * i, 16 * (j + 1), sTf, 16 * (j + 1), 16 * j, true, lane);
-        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+    // diagonal 2: T_20 (pair 0), T_31 (pair 1); pair 3 adds A_31 T_10 to its partial
+    if (blk < 2) {
+        const int j = blk, i = j + 2;
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        warp_mm16x8(acc, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j + nc, true, lane);
+        warp_mm16x8(acc, sA, 16 * i, 16 * (j + 1), sTf, 16 * (j + 1), 16 * j + nc, true, lane);
+        warp_store16x8(acc, Xw, 0, 0, false, 1.f, lane);
         __syncwarp();
-        zero16(acc);
-        warp_mm16(acc, sTf, 16 * i, 16 * i, Xw, 0, 0, false, lane);
-        warp_store16(acc, sTf, 16 * i, 16 * j, true, -1.f, lane);
-        warp_store16_tile(acc, Ttile, 16 * i, 16 * j, -1.f, lane);
-    } else if (warp == 3) {
-        warp_load16(acc, Xw, lane);
-        warp_mm16(acc, sA, 48, 16, sTf, 16, 0, true, lane);         // + A_31 T_10
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        warp_mm16x8(acc, sTf, 16 * i, 16 * i, Xw, 0, 0, false, lane);
+        warp_store16x8(acc, sTf, 16 * i, 16 * j + nc, true, -1.f, lane);
+        warp_store16x8_tile(acc, Ttile, 16 * i, 16 * j + nc, -1.f, lane);
+    } else if (blk == 3) {
+        warp_load16x8(acc, Xw, lane);
+        warp_mm16x8(acc, sA, 48, 16, sTf, 16, nc, true, lane);         // + A_31 T_10
         __syncwarp();
-        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+        warp_store16x8(acc, Xw, 0, 0, false, 1.f, lane);
     }
     __syncthreads();
-    // diagonal 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20)   (warp 3)
-    if (warp == 3) {
-        warp_load16(acc, Xw, lane);
-        warp_mm16(acc, sA, 48, 32, sTf, 32, 0, true, lane);
+    // diagonal 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20)   (pair 3)
+    if (blk == 3) {
+        warp_load16x8(acc, Xw, lane);
+        warp_mm16x8(acc, sA, 48, 32, sTf, 32, nc, true, lane);
         __syncwarp();
-        warp_store16(acc, Xw, 0, 0, false, 1.f, lane);
+        warp_store16x8(acc, Xw, 0, 0, false, 1.f, lane);
         __syncwarp();
-        zero16(acc);
-        warp_mm16(acc, sTf, 48, 48, Xw, 0, 0, false, lane);
-        warp_store16_tile(acc, Ttile, 48, 0, -1.f, lane);
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        warp_mm16x8(acc, sTf, 48, 48, Xw, 0, 0, false, lane);
+        warp_store16x8_tile(acc, Ttile, 48, nc, -1.f, lane);
     }
 }
 
-// Transpose a [128 lanes x 64 columns] fp32 TMEM accumulator (lane = channel,
-// column = token) into the bf16 row tile dst [64 tokens x 128 channels].
-__device__ __forceinline__ void tmem_to_tile_transposed(uint32_t lane_base_col, unsigned char* dst, int tid) {
-    float v[32];
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        tc::tmem_ld32(lane_base_col + 32 * h2, v);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 32; ++u) tc::st_bf16(dst, tc::tile_off(C, 32 * h2 + u, tid), v[u]);
-    }
-}
-
-// Copy a [128 lanes x ncol] fp32 TMEM accumulator into a bf16 row tile of 128
-// rows (row = lane), ncol in {64, 128}.
+// Copy a [128 lanes x NCOL] fp32 TMEM accumulator into a bf16 row tile of 128 rows (row = lane);
+// the two warps of a lane quarter take half of the columns each.
 template <int NCOL>
-__device__ __forceinline__ void tmem_to_tile_rows(uint32_t lane_base_col, unsigned char* dst, int tid) {
+__device__ __forceinline__ void tmem_to_tile_rows(uint32_t lane_base_col, unsigned char* dst, int warp, int lane) {
+    const int row = 32 * tm_quarter(warp) + lane, c0 = (NCOL / 2) * tm_part(warp);
     float v[32];
 #pragma unroll
-    for (int c0 = 0; c0 < NCOL; c0 += 32) {
-        tc::tmem_ld32(lane_base_col + c0, v);
+    for (int cc = 0; cc < NCOL / 2; cc += 32) {
+        tc::tmem_ld32(lane_base_col + c0 + cc, v);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < 4; ++g) tc::st_row8(dst, 128, tid, (c0 >> 3) + g, v + 8 * g);
+        for (int g = 0; g < 4; ++g) tc::st_row8(dst, 128, row, ((c0 + cc) >> 3) + g, v + 8 * g);
     }
-}
-
-// Multiply a [128 lanes x 128 columns] fp32 TMEM state by gC[column] in place.
-__device__ __forceinline__ void tmem_scale_columns(uint32_t lane_base_col, const float* gC) {
-    float v[32];
-#pragma unroll 1
-    for (int i0 = 0; i0 < D; i0 += 32) {
-        tc::tmem_ld32(lane_base_col + i0, v);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 32; ++u) v[u] *= gC[i0 + u];
-        tc::tmem_st32(lane_base_col + i0, v);
-    }
-    tc::tmem_wait_st();
 }
 
 // M = 64 accumulators (cta_group::1): row r of D lives in TMEM lane (r % 16) + 32 (r / 16).
-// Warp w, lanes 0..15 therefore hold rows 16w .. 16w+15. All 32 lanes must execute the loads.
-__device__ __forceinline__ int m64_row(int warp, int lane) { return 16 * warp + (lane & 15); }
+// In lane quarter q, lanes 0..15 hold rows 16 q .. 16 q + 15. All 32 lanes must execute the loads.
+__device__ __forceinline__ int m64_row(int warp, int lane) { return 16 * tm_quarter(warp) + (lane & 15); }
 
-// Copy a [64 rows x 128 columns] M=64 accumulator into a bf16 row tile of 64 rows (optionally scaled).
+// Copy a [64 rows x 128 columns] M=64 accumulator into a bf16 row tile of 64 rows; the two warps of
+// a lane quarter take 64 columns each.
 __device__ __forceinline__ void tmem_m64_to_tile(uint32_t lane_base_col, unsigned char* dst, int warp, int lane) {
-    const int r = m64_row(warp, lane);
+    const int r = m64_row(warp, lane), c0 = 64 * tm_part(warp);
     float v[32];
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-        tc::tmem_ld32(lane_base_col + c0, v);
+    for (int cc = 0; cc < 64; cc += 32) {
+        tc::tmem_ld32(lane_base_col + c0 + cc, v);
         tc::tmem_wait_ld();
         if (lane < 16) {
 #pragma unroll
-            for (int g = 0; g < 4; ++g) tc::st_row8(dst, C, r, (c0 >> 3) + g, v + 8 * g);
+            for (int g = 0; g < 4; ++g) tc::st_row8(dst, C, r, ((c0 + cc) >> 3) + g, v + 8 * g);
         }
     }
 }

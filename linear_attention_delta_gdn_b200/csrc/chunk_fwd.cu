@@ -1,7 +1,7 @@
 // chunk_fwd.cu -- chunkwise WY forward of the Gated Delta Rule-2 operator on
 // tcgen05 tensor cores (bf16 operands, fp32 TMEM accumulators, fp32 state).
 //
-// One CTA (128 threads) per (batch, head) walks the chunks in order; the state
+// One CTA (256 threads) per (batch, head) walks the chunks in order; the state
 // is carried across chunks in TMEM as S^T (lane j = value channel, column i =
 // key channel) in fp32, with a bf16 copy in shared memory as the UMMA operand.
 // Per chunk ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
@@ -102,7 +102,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_base_ptr;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lanes
+    const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);   // this warp's TMEM lanes
+    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
 
     auto issue_loads = [&](int c) {
         const int t0 = c * C;
@@ -118,10 +119,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 
     // initial state: S^T row j = column j of S0
     {
-        const int j = tid;
+        const int j = jrow;
         float v[32];
 #pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 32) {
+        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] = S0 ? S0[(head * D + i0 + u) * D + j] : 0.f;
             tc::tmem_st32(lane_base + TM_S + i0, v);
@@ -180,7 +181,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        extract_AP(lane_base + TM_AP, sA, PP, want_qp, tid);
+        extract_AP(lane_base + TM_AP, sA, PP, want_qp, warp, lane);
         tc::tc_fence_before();
         __syncthreads();
 
@@ -220,7 +221,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        tmem_to_tile_rows<64>(lane_base + TM_D, DT, tid);       // Delta^T (lane j) -> bf16 rows
+        tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
         sync_for_mma();
 
         // ---- M6: O += P Delta ;  M7: Z^T = S^T + Delta^T Kt
@@ -242,7 +243,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             const int t = m64_row(warp, lane);
             float v[32];
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
                 tc::tmem_ld32(lane_base + TM_O + c0, v);
                 tc::tmem_wait_ld();
                 if (lane < 16 && t < L) {
@@ -258,10 +259,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         if (states && tid == 0) tc::bulk_wait_read();
         __syncthreads();
         {
-            const int j = tid;
+            const int j = jrow;
             float v[32];
 #pragma unroll 1
-            for (int i0 = 0; i0 < D; i0 += 32) {
+            for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
                 tc::tmem_wait_ld();
 #pragma unroll
@@ -283,10 +284,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 
     // final state (fp32): ST[i][j] from S^T (lane j)
     if (ST) {
-        const int j = tid;
+        const int j = jrow;
         float v[32];
 #pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 32) {
+        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
             tc::tmem_ld32(lane_base + TM_S + i0, v);
             tc::tmem_wait_ld();
 #pragma unroll
