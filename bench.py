@@ -176,6 +176,45 @@ def cpu_baseline(wl, x, budget_s=20.0, steps=1):
             "seconds": dt}
 
 
+def bench_decode(binding, dev, steps=1024, pool=64):
+    """Time the decode workload: 1024 consecutive single-token steps, batch 256, 16 heads, d = 128,
+    fp32 state updated in place, bf16 inputs. Step inputs cycle through a pool of `pool` distinct draws
+    (the state traffic, not the input values, sets the time). Returns per-step time and HBM figures."""
+    import torch
+    from linear_attention_delta_gdn_b200.inputs import WORKLOADS, make_decode_stream
+    wl = WORKLOADS["decode-bf16-b256h16d128x1024"]
+    xs = make_decode_stream(pool, wl.B, wl.H, wl.Dk, wl.Dv, wl.seed, wl.dtype, device=dev)
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    S = xs["S0"].clone()
+    o = torch.empty((wl.B, wl.H, wl.Dv), dtype=torch.bfloat16, device=dev)
+    step_in = [[xs[n][i] for n in names] for i in range(pool)]
+    for i in range(8):
+        binding.gdn2_decode_step(*step_in[i % pool], S, o=o)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    binding.trace_read()
+    binding.trace_enable(True)
+    a.record()
+    for i in range(steps):
+        binding.gdn2_decode_step(*step_in[i % pool], S, o=o)
+    b.record()
+    binding.trace_enable(False)
+    torch.cuda.synchronize(dev)
+    kern = binding.trace_read().get("decode_kernel", (steps, 0.0))
+    ms = a.elapsed_time(b) / steps
+    kern_ms = kern[1] / max(1, kern[0])
+    heads = wl.B * wl.H
+    state_bytes = heads * wl.Dk * wl.Dv * 4
+    io_bytes = heads * (4 * wl.Dk + 3 * wl.Dv) * 2       # q, k, log_alpha, b, v, w in; o out
+    alg = 2 * state_bytes + io_bytes
+    pk = peaks()
+    return {"workload": wl.name, "steps": steps, "ms_per_step": ms, "kernel_ms": kern_ms,
+            "alg_bytes_per_step": alg, "achieved_gbs": alg / (kern_ms / 1e3) / 1e9,
+            "frac_of_hbm": alg / (kern_ms / 1e3) / 1e9 / pk["hbm_gbs"], "peak_gbs": pk["hbm_gbs"],
+            "inputs": "%d-step input pool cycled; state evolves over all %d steps" % (pool, steps),
+            "launches": kern[0]}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -205,6 +244,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
     ap.add_argument("--B", type=int, default=None, help="override the batch size (small profiling cases)")
     ap.add_argument("--T", type=int, default=None, help="override the sequence length (small profiling cases)")
     args = ap.parse_args()
@@ -316,6 +356,10 @@ def main():
                 / (ms_per_step / 1e3) / 1e9 / pk["hbm_gbs"]}
     launches_in_timed_region = sum(v[0] for v in kernels.values())
 
+    decode = None
+    if not args.no_decode and args.B is None and args.T is None:
+        decode = bench_decode(binding, dev)
+
     line = None
     if rank == 0:
         cb = None
@@ -333,7 +377,8 @@ def main():
                 "roofline": roofline, "cpu_baseline": cb, "clocks": clocks.summary(),
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
-                "gpu_launches": launches_in_timed_region}
+                "gpu_launches": launches_in_timed_region,
+                "decode": decode}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
