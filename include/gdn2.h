@@ -74,8 +74,13 @@ typedef enum gdn2_op {
  * The workspace of GDN2_OP_BWD starts with the region that GDN2_OP_FWD_SAVE
  * fills, so one buffer of gdn2_workspace_size(GDN2_OP_BWD, ...) bytes serves a
  * gdn2_fwd(save_states = 1) followed by a gdn2_bwd(states_saved = 1).
- * Returns 0 for an invalid or unsupported problem (and for GDN2_OP_FWD, which
- * needs none). The workspace must be 256-byte aligned.
+ * GDN2_OP_FWD needs a workspace only on the tensor-core path (dt = GDN2_BF16,
+ * Dk = Dv = 128, chunk = 64): there the forward keeps, per chunk, the
+ * T | P | Wm tiles of the WY step and a ready flag that hands them from the CTAs
+ * that compute them to the CTAs that walk the chunks of a head.
+ * Returns 0 for an invalid or unsupported problem and for a forward that needs
+ * no workspace. The workspace must be 256-byte aligned; its contents on entry
+ * do not matter.
  */
 size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk,
                            gdn2_dtype dt);
@@ -90,8 +95,9 @@ size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int 
  *   chunk              : chunk length of the WY algorithm (16, 32 or 64)
  *   save_states        : nonzero -> keep the chunk-start states in ws for a
  *                        later gdn2_bwd(states_saved = 1) on the same inputs
- *   ws, ws_bytes       : workspace of >= gdn2_workspace_size(GDN2_OP_FWD[_SAVE])
- *                        bytes (may be NULL when that size is 0)
+ *   ws, ws_bytes       : workspace of >= gdn2_workspace_size(GDN2_OP_FWD, or
+ *                        GDN2_OP_FWD_SAVE when save_states) bytes; may be NULL
+ *                        when that size is 0
  * S0 and ST may alias (the state is updated in place).
  */
 gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* log_alpha,

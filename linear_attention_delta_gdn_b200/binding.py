@@ -117,10 +117,10 @@ def gdn2_fwd(q, k, v, log_alpha, b, w, S0=None, chunk: int = 64, want_state: boo
              save_states: bool = False, ws: Optional[torch.Tensor] = None, o=None, ST=None):
     """Forward. Tensors [B, T, H, D] (bf16 or fp32), S0 [B, H, Dk, Dv] fp32 or None.
 
-    Returns ``(o, ST)`` (``ST`` is None unless ``want_state``). With
-    ``save_states`` the chunk-start states are kept in ``ws`` (a uint8 CUDA tensor
-    of at least ``gdn2_workspace_size(GDN2_OP_FWD_SAVE, ...)`` bytes; allocated
-    if not given) for a later :func:`gdn2_bwd` with ``states_saved=True``.
+    Returns ``(o, ST)`` (``ST`` is None unless ``want_state``). ``ws`` is a uint8
+    CUDA tensor of at least ``gdn2_workspace_size(GDN2_OP_FWD[_SAVE], ...)`` bytes,
+    allocated if not given. With ``save_states`` the chunk-start states are kept in
+    it for a later :func:`gdn2_bwd` with ``states_saved=True``.
     """
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
@@ -134,10 +134,10 @@ def gdn2_fwd(q, k, v, log_alpha, b, w, S0=None, chunk: int = 64, want_state: boo
     if ST is None and want_state:
         ST = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
     ws_bytes = 0
-    if save_states:
-        need = gdn2_workspace_size(GDN2_OP_FWD_SAVE, B, T, H, Dk, Dv, chunk, dt)
-        if ws is None:
-            ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    need = gdn2_workspace_size(GDN2_OP_FWD_SAVE if save_states else GDN2_OP_FWD, B, T, H, Dk, Dv, chunk, dt)
+    if need and ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if ws is not None:
         ws_bytes = ws.numel()
     rc = lib().gdn2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
                         _ptr(ST), B, T, H, Dk, Dv, chunk, dt, int(save_states), _ptr(ws), ws_bytes,

@@ -116,7 +116,7 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         tma_tile(KH, C, 0, &mk, b, h, t0, bar_load);
         tma_tile(KT, C, 0, &mla, b, h, t0, bar_load);
         tma_tile(DO, C, 0, &mdo, b, h, t0, bar_load);
-        const unsigned char* src = tp + (head * nc + c) * TC_TP_BYTES;
+        const unsigned char* src = tp + (head * nc + c) * TC_WY_BYTES;
         tc::bulk_load(TT, src, TILE_C, bar_load);
         tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
     };
@@ -327,7 +327,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tma_tile(DO, C, 0, &mdo, b, h, t0, bar_load);
         tc::bulk_load(STt, states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
         tc::bulk_load(DS, dstates + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
-        const unsigned char* src = tp + (head * nc + c) * TC_TP_BYTES;
+        const unsigned char* src = tp + (head * nc + c) * TC_WY_BYTES;
         tc::bulk_load(TT, src, TILE_C, bar_load);
         tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
     }

@@ -134,20 +134,15 @@ __device__ __forceinline__ void gate_prep_cols(unsigned char* QE, unsigned char*
     if (hf) gC_out[i] = fast_exp(G);
 }
 
-// Gate preparation, vectorised: thread = (4-token block tb = tid / 16, 8-channel group cg = tid % 16),
-// 16-byte shared-memory accesses:
-//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
-//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127 (want_q),
-//          Kt = k/g -> KT, U = w*v -> UU (want_u); KH keeps k.
-//   g = exp(G), G = inclusive cumsum of log_alpha over the chunk; gC[i] = g at the last row.
-// The cumsum is a local scan over the thread's 4 rows plus the totals of the earlier blocks,
-// exchanged through `red` (fp32 [16][128], 8 KB). Contains one __syncthreads.
-__device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
-                                          unsigned char* UU, const unsigned char* WW, float* gC_out,
-                                          float* red, int tid, bool want_q, bool want_u) {
-    constexpr int RB = 4;                       // rows per thread
+// Inclusive cumulative log-decay of the chunk for one thread = (4-token block tb = tid / 16,
+// 8-channel group cg = tid % 16): on return G[u][c] + pre[c] is G at row 4 tb + u, channel 8 cg + c.
+// The thread's log_alpha rows are read from KT (row tile of 64 rows); block totals are exchanged
+// through `red` (fp32 [16][128], 8 KB). gC[i] = exp(G) at the last row when gC_out is not null.
+// Contains one __syncthreads; afterwards the thread may overwrite its own rows and channels of KT.
+__device__ __forceinline__ void chunk_cumsum(const unsigned char* KT, float* red, float* gC_out, int tid,
+                                             float (&G)[4][8], float (&pre)[8]) {
+    constexpr int RB = 4;
     const int cg = tid & 15, tb = tid >> 4;
-    float G[RB][8];
 #pragma unroll
     for (int u = 0; u < RB; ++u) {
         tc::ld_row8(KT, C, RB * tb + u, cg, G[u]);
@@ -159,7 +154,8 @@ __device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char
     *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg) = make_float4(G[RB - 1][0], G[RB - 1][1], G[RB - 1][2], G[RB - 1][3]);
     *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg + 4) = make_float4(G[RB - 1][4], G[RB - 1][5], G[RB - 1][6], G[RB - 1][7]);
     __syncthreads();
-    float pre[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) pre[c] = 0.f;
 #pragma unroll 1
     for (int p = 0; p < tb; ++p) {
         const float4 x0 = *reinterpret_cast<const float4*>(red + p * 128 + 8 * cg);
@@ -167,10 +163,26 @@ __device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char
         pre[0] += x0.x; pre[1] += x0.y; pre[2] += x0.z; pre[3] += x0.w;
         pre[4] += x1.x; pre[5] += x1.y; pre[6] += x1.z; pre[7] += x1.w;
     }
-    if (tb == C / RB - 1) {
+    if (gC_out && tb == C / RB - 1) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) gC_out[8 * cg + c] = fast_exp(pre[c] + G[RB - 1][c]);
     }
+}
+
+// Gate preparation, vectorised: thread = (4-token block tb = tid / 16, 8-channel group cg = tid % 16),
+// 16-byte shared-memory accesses:
+//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
+//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127 (want_q),
+//          Kt = k/g -> KT, U = w*v -> UU (want_u); KH keeps k.
+//   g = exp(G), G = inclusive cumsum of log_alpha over the chunk; gC[i] = g at the last row.
+// Contains one __syncthreads.
+__device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
+                                          unsigned char* UU, const unsigned char* WW, float* gC_out,
+                                          float* red, int tid, bool want_q, bool want_u) {
+    constexpr int RB = 4;
+    const int cg = tid & 15, tb = tid >> 4;
+    float G[RB][8], pre[8];
+    chunk_cumsum(KT, red, gC_out, tid, G, pre);
 #pragma unroll
     for (int u = 0; u < RB; ++u) {
         const int row = RB * tb + u;
@@ -193,6 +205,39 @@ __device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char
         tc::st_row8(KT, C, row, cg, kt);
         if (want_q) tc::st_row8(QE, 2 * C, C + row, cg, qq);
         if (want_u) tc::st_row8(UU, C, row, cg, vv);
+    }
+}
+
+// Gate preparation of the state pass (no erase factor): same thread layout as gate_prep;
+//   reads  log_alpha (KT), k (KH), q (QQ, 64 rows), v (UU), w (WW)
+//   writes Qt = g*q -> QQ, Kt = k/g -> KT, U = w*v -> UU, gC.
+// Contains one __syncthreads.
+__device__ __forceinline__ void gate_prep_state(unsigned char* QQ, const unsigned char* KH, unsigned char* KT,
+                                                unsigned char* UU, const unsigned char* WW, float* gC_out,
+                                                float* red, int tid) {
+    constexpr int RB = 4;
+    const int cg = tid & 15, tb = tid >> 4;
+    float G[RB][8], pre[8];
+    chunk_cumsum(KT, red, gC_out, tid, G, pre);
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+        const int row = RB * tb + u;
+        float kk[8], qq[8], vv[8], ww[8];
+        tc::ld_row8(KH, C, row, cg, kk);
+        tc::ld_row8(QQ, C, row, cg, qq);
+        tc::ld_row8(UU, C, row, cg, vv);
+        tc::ld_row8(WW, C, row, cg, ww);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float Gv = pre[c] + G[u][c];
+            const float g = fast_exp(Gv), ig = fast_exp(-Gv);
+            kk[c] *= ig;
+            qq[c] *= g;
+            vv[c] *= ww[c];
+        }
+        tc::st_row8(KT, C, row, cg, kk);
+        tc::st_row8(QQ, C, row, cg, qq);
+        tc::st_row8(UU, C, row, cg, vv);
     }
 }
 

@@ -1,22 +1,27 @@
 // chunk_fwd.cu -- chunkwise WY forward of the Gated Delta Rule-2 operator on
 // tcgen05 tensor cores (bf16 operands, fp32 TMEM accumulators, fp32 state).
 //
-// One CTA (256 threads) per (batch, head) walks the chunks in order; the state
-// is carried across chunks in TMEM as S^T (lane j = value channel, column i =
-// key channel) in fp32, with a bf16 copy in shared memory as the UMMA operand.
-// Per chunk ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
+// Chunk algebra ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
 // Attention", arXiv abstract: chunkwise WY algorithm, decay absorbed into
-// asymmetric erase factors):
-//   TMA      q, k, v, log_alpha, b, w tiles (64 tokens x 128, bf16, 128B swizzle)
-//   prep     Et = g*b*k, Qt = g*q, Kt = k/g, Kh = gC*Kt, U = w*v       (g = exp(cumsum log_alpha))
-//   M1       [A; P] = [Et; Qt] Kt^T                                     (M=128, N=64, K=128)
-//   solve    T = (I + strict_lower(A))^{-1}     (16x16 blocks, off-diagonal merges on mma.sync tf32)
-//   M2, M3   Wm = T Et (M=64, N=128) ,  Delta^T := U^T T^T (M=128, N=64)
-//   M4, M5   Delta^T -= S^T Wm^T (M=128) ,  O = Qt S (M=64, N=128)
-//   M6, M7   O += P Delta (M=64) ,  Z^T = S^T + Delta^T Kt (M=128, N=128)
-//   scale    S'^T = Z^T Diag(gC) on the fp32 accumulator, bf16 copy for the next chunk
-// For training, the chunk-start states and the T and P tiles of every chunk are written
-// (bf16 shared-memory images) for the backward.
+// asymmetric erase factors), per head and chunk of 64 tokens starting from S:
+//   prep     Et = g*b*k, Qt = g*q, Kt = k/g, U = w*v          (g = exp(cumsum log_alpha))
+//   WY       [A; P] = [Et; Qt] Kt^T,  T = (I + strict_lower(A))^{-1},  Wm = T Et
+//   state    Delta^T = U^T T^T - S^T Wm^T,  O = Qt S + P Delta,  S'^T = (S^T + Delta^T Kt) Diag(gC)
+// The WY step does not depend on S; the state step is a chain over the chunks of a head.
+//
+// One launch, two kinds of CTA (256 threads each, one CTA per SM):
+//   * producers walk the chunks of all heads in chunk-major order and compute the WY step; each
+//     writes T, P and Wm of its chunk ("WY image", 32 KB) to the workspace and then sets the
+//     chunk's ready flag (release);
+//   * consumers (one per head, or several heads each when heads outnumber them) walk their head's
+//     chunks in order: they wait for the chunk's flag (acquire), copy its WY image into shared
+//     memory and run the state step. The state S^T lives in TMEM (lane j = value channel, column
+//     i = key channel) in fp32 with a bf16 copy in shared memory as the UMMA operand.
+// With few heads the producers run on the SMs that the consumers leave idle, in the same
+// cooperative launch (all CTAs resident, so every wait ends; each wait is also bounded in time).
+// Otherwise the producers run as one launch and the consumers as a second one.
+// For training, the chunk-start states are written as bf16 images; the WY images stay in the
+// workspace for the backward.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,121 +35,180 @@ namespace {
 
 using namespace chunk;
 
-// shared-memory layout (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_QE = 0;           // [128 x 128] rows 0..63: b -> Et, rows 64..127: q -> Qt
-constexpr uint32_t OFF_KH = 32768;       // [64 x 128] k
-constexpr uint32_t OFF_KT = 49152;       // [64 x 128] log_alpha -> Kt
-constexpr uint32_t OFF_UU = 65536;       // [64 x 128] v -> U
-constexpr uint32_t OFF_WW = 81920;       // [64 x 128] w -> solve temporaries -> Wm
-constexpr uint32_t OFF_ST = 98304;       // [128 x 128] S^T (bf16)
-constexpr uint32_t OFF_DT = 131072;      // [128 x 64] Delta^T (bf16)  | fp32 A scratch [64 x 64]
-constexpr uint32_t OFF_TF = 147456;      // fp32 T [64 x 64] | prep scan scratch
-constexpr uint32_t OFF_TT = 163840;      // [64 x 64] T (bf16)
-constexpr uint32_t OFF_PP = 172032;      // [64 x 64] P (bf16)
-constexpr uint32_t OFF_GC = 180224;      // fp32 gC[128]
-constexpr uint32_t OFF_BAR = 180736;     // 2 mbarriers, tmem base, abort flag
-constexpr uint32_t SMEM_BYTES = 180800 + 1024;
+// ---- consumer (state pass) shared memory, bytes from a 1024-aligned base
+namespace sp {
+constexpr uint32_t QQ = 0;          // [64 x 128] q -> Qt
+constexpr uint32_t KH = 16384;      // [64 x 128] k
+constexpr uint32_t KT = 32768;      // [64 x 128] log_alpha -> Kt
+constexpr uint32_t UU = 49152;      // [64 x 128] v -> U
+constexpr uint32_t WW = 65536;      // [64 x 128] w
+constexpr uint32_t WY = 81920;      // WY image: T [64 x 64] | P [64 x 64] | Wm [64 x 128]
+constexpr uint32_t TT = WY, PP = WY + 8192, WM = WY + 16384;
+constexpr uint32_t ST = 114688;     // [128 x 128] S^T (bf16)
+constexpr uint32_t DT = 147456;     // [128 x 64] Delta^T (bf16)
+constexpr uint32_t RED = 163840;    // fp32 [16][128] prep scan scratch
+constexpr uint32_t GC = 172032;     // fp32 gC[128]
+constexpr uint32_t BAR = 172544;    // 3 mbarriers (load, mma, unused), tmem base, abort flag
+}  // namespace sp
+// ---- producer (WY) shared memory: two input stages, then the solve scratch and the WY image
+namespace wy {
+constexpr uint32_t STAGE = 65536;   // per stage: [b; q] rows (32 KB) at 0, k at 32768, log_alpha at 49152
+constexpr uint32_t QE = 0, KH = 32768, KT = 49152;
+constexpr uint32_t SA = 131072;     // fp32 A [64 x 64] (sq_idx) | prep scan scratch
+constexpr uint32_t TF = 147456;     // fp32 T [64 x 64]
+constexpr uint32_t SX = 163840;     // solve temporaries, 12 KB
+constexpr uint32_t IMG = 176128;    // WY image: T | P | Wm (32 KB)
+constexpr uint32_t TT = IMG, PP = IMG + 8192, WM = IMG + 16384;
+constexpr uint32_t BAR = 208896;    // 3 mbarriers (2 stages, mma), tmem base, abort flag
+}  // namespace wy
+constexpr uint32_t SMEM_BYTES = 208960 + 1024;
+static_assert(sp::BAR + 64 <= wy::BAR + 64, "consumer layout fits");
+static_assert(TC_WY_BYTES == 32768, "WY image = T | P | Wm");
 
-// TMEM columns: S^T (fp32 state), [A; P], Ut^T -> Delta^T, Wm (M=64), O (M=64)
-constexpr uint32_t TM_S = 0, TM_AP = 128, TM_D = 192, TM_W = 256, TM_O = 384, TM_COLS = 512;
+// TMEM columns. Consumer: S^T (fp32 state), Ut^T -> Delta^T, O (M=64). Producer: [A; P], Wm (M=64).
+constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 256;
+constexpr uint32_t TM_AP = 0, TM_W = 128;
+constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t LOAD_BYTES = 6 * 64 * 128 * 2;
+constexpr uint32_t CONS_LOAD_BYTES = 5 * 64 * 128 * 2;
+constexpr uint32_t PROD_LOAD_BYTES = 4 * 64 * 128 * 2;
 
 __device__ unsigned int g_fwd_error;
 
-__global__ void __launch_bounds__(NT, 1)
-chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                 const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mla,
-                 const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
-                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
-                 unsigned char* __restrict__ states, unsigned char* __restrict__ tp, int T, int H) {
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
-    unsigned char* QE = sm + OFF_QE;
-    unsigned char* KH = sm + OFF_KH;
-    unsigned char* KT = sm + OFF_KT;
-    unsigned char* UU = sm + OFF_UU;
-    unsigned char* WW = sm + OFF_WW;
-    unsigned char* STt = sm + OFF_ST;
-    unsigned char* DT = sm + OFF_DT;
-    float* sA = reinterpret_cast<float*>(sm + OFF_DT);
-    float* sTf = reinterpret_cast<float*>(sm + OFF_TF);
-    float* sX = reinterpret_cast<float*>(sm + OFF_WW);   // w is consumed by the prep, Wm written after M2
-    unsigned char* TT = sm + OFF_TT;
-    unsigned char* PP = sm + OFF_PP;
-    float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    uint64_t* bar_mma = bar_load + 1;
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
-    int* abort_flag = reinterpret_cast<int*>(sm + OFF_BAR + 20);
+struct FwdParams {
+    int T, H, BH, nc;
+    int ncons, nprod;              // CTAs [0, ncons) are consumers, the next nprod are producers
+    const float* S0;
+    __nv_bfloat16* o;              // may be null (states only)
+    float* ST;
+    unsigned char* states;         // [BH, nc] chunk-start state images, or null
+    unsigned char* wyimg;          // [BH, nc] WY images
+    unsigned int* flags;           // [BH, nc] ready flags (zero at launch)
+};
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x % H, b = blockIdx.x / H;
-    const size_t head = blockIdx.x;
-    const int nc = (T + C - 1) / C;
-    const bool want_o = (o != nullptr);
-    const bool save = (states != nullptr);          // training: keep S, T and P of every chunk
-    const bool want_qp = want_o || save;
+struct Maps {
+    CUtensorMap q, k, v, la, b, w;
+};
 
-    if (tid == 0) {
-        tc::mbar_init(bar_load, 1);
-        tc::mbar_init(bar_mma, 1);
-        *abort_flag = 0;
-        tc::fence_mbar_init();
-        tc::tma_prefetch_desc(&mq); tc::tma_prefetch_desc(&mk); tc::tma_prefetch_desc(&mv);
-        tc::tma_prefetch_desc(&mla); tc::tma_prefetch_desc(&mb); tc::tma_prefetch_desc(&mw);
-    }
-    if (warp == 0) {
-        tc::tmem_alloc(tmem_base_ptr, TM_COLS);
-        tc::tmem_relinquish();
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = *tmem_base_ptr;
-    const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);   // this warp's TMEM lanes
-    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
-
-    auto issue_loads = [&](int c) {
-        const int t0 = c * C;
-        tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-        tma_tile(QE, 2 * C, 0, &mb, b, h, t0, bar_load);
-        tma_tile(QE, 2 * C, C, &mq, b, h, t0, bar_load);
-        tma_tile(KH, C, 0, &mk, b, h, t0, bar_load);
-        tma_tile(KT, C, 0, &mla, b, h, t0, bar_load);
-        tma_tile(UU, C, 0, &mv, b, h, t0, bar_load);
-        tma_tile(WW, C, 0, &mw, b, h, t0, bar_load);
-    };
-    if (tid == 0 && nc > 0) issue_loads(0);
-
-    // initial state: S^T row j = column j of S0
-    {
-        const int j = jrow;
-        float v[32];
-#pragma unroll 1
-        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
-#pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] = S0 ? S0[(head * D + i0 + u) * D + j] : 0.f;
-            tc::tmem_st32(lane_base + TM_S + i0, v);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
-        }
-        tc::tmem_wait_st();
-    }
+__device__ __forceinline__ void sync_for_mma() {   // smem written by threads + TMEM accesses done -> MMA issuer
     tc::fence_async_smem();
     tc::tc_fence_before();
     __syncthreads();
-    tc::tc_fence_after();
-    if (states && tid == 0) {
-        tc::bulk_store(states + (head * nc + 0) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
-        tc::bulk_commit();
-    }
+}
 
-    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sUU = tc::smem_u32(UU),
-                   sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
-                   sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
+// ------------------------------------------------------------------ producer
+__device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int pid) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + wy::BAR);   // [2]
+    uint64_t* bar_mma = bar_in + 2;
+    int* abort_flag = reinterpret_cast<int*>(sm + wy::BAR + 28);
+    float* sA = reinterpret_cast<float*>(sm + wy::SA);
+    float* sTf = reinterpret_cast<float*>(sm + wy::TF);
+    float* sX = reinterpret_cast<float*>(sm + wy::SX);
+    unsigned char* TT = sm + wy::TT;
+    unsigned char* PP = sm + wy::PP;
+    unsigned char* WM = sm + wy::WM;
+    const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
+    const uint32_t sTT = tc::smem_u32(TT);
     constexpr uint32_t ID_M1 = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
+    const int units = p.BH * p.nc;
+
+    auto issue_loads = [&](int stage, int u) {
+        const int c = u / p.BH, head = u % p.BH;
+        const int b = head / p.H, h = head % p.H, t0 = c * C;
+        unsigned char* base = sm + stage * wy::STAGE;
+        tc::mbar_arrive_expect_tx(&bar_in[stage], PROD_LOAD_BYTES);
+        tma_tile(base + wy::QE, 2 * C, 0, &m.b, b, h, t0, &bar_in[stage]);
+        tma_tile(base + wy::QE, 2 * C, C, &m.q, b, h, t0, &bar_in[stage]);
+        tma_tile(base + wy::KH, C, 0, &m.k, b, h, t0, &bar_in[stage]);
+        tma_tile(base + wy::KT, C, 0, &m.la, b, h, t0, &bar_in[stage]);
+    };
+    if (tid == 0 && pid < units) issue_loads(0, pid);
+
+    uint32_t ph_in = 0, ph_mma = 0;   // ph_in: bit s = phase parity of input stage s
+    auto wait_mma = [&]() {
+        if (!tc::mbar_wait(bar_mma, ph_mma)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 1u); }
+        ph_mma ^= 1;
+        tc::tc_fence_after();
+    };
+    int stage = 0;
+    bool pending = false;   // a prefetch into the other stage is in flight (thread 0's view)
+    for (int u = pid; u < units; u += p.nprod, stage ^= 1) {
+        const int c = u / p.BH, head = u % p.BH;
+        unsigned char* base = sm + stage * wy::STAGE;
+        unsigned char* QE = base + wy::QE;
+        if (!tc::mbar_wait(&bar_in[stage], (ph_in >> stage) & 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
+        ph_in ^= 1u << stage;
+        // the other stage was last read by the previous unit's MMAs, which have completed
+        pending = u + p.nprod < units;
+        if (tid == 0 && pending) issue_loads(stage ^ 1, u + p.nprod);
+
+        gate_prep(QE, base + wy::KH, base + wy::KT, nullptr, nullptr, nullptr, sA, tid, true, false);
+        sync_for_mma();
+        const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(base + wy::KT);
+        if (tid == 0) {   // [A; P] = [Et; Qt] Kt^T
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
+            tc::mma_commit(bar_mma);
+        }
+        wait_mma();
+        extract_AP(lane_base + TM_AP, sA, PP, true, warp, lane);
+        tc::tc_fence_before();
+        __syncthreads();
+        solve_unit_lower(sA, sTf, sX, TT, tid);   // T = (I + A)^{-1}
+        sync_for_mma();
+        if (tid == 0) {   // Wm = T Et
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), ID_M2, kk > 0);
+            tc::mma_commit(bar_mma);
+        }
+        wait_mma();
+        tmem_m64_to_tile(lane_base + TM_W, WM, warp, lane);
+        tc::tc_fence_before();
+        __syncthreads();
+        // publish the WY image of (head, c)
+        const size_t unit = (size_t)head * p.nc + c;
+        uint4* dst = reinterpret_cast<uint4*>(p.wyimg + unit * TC_WY_BYTES);
+        const uint4* src = reinterpret_cast<const uint4*>(sm + wy::IMG);
+#pragma unroll
+        for (int i = 0; i < (int)(TC_WY_BYTES / 16 / NT); ++i) dst[tid + NT * i] = src[tid + NT * i];
+        __syncthreads();
+        if (tid == 0 && !*abort_flag) tc::flag_release(p.flags + unit, 1u);
+        if (*abort_flag) break;
+        pending = false;
+    }
+    // after an abort: let the prefetch in flight land before the CTA's shared memory is released
+    if (tid == 0 && pending) (void)tc::mbar_wait(&bar_in[stage ^ 1], (ph_in >> (stage ^ 1)) & 1u);
+}
+
+// ------------------------------------------------------------------ consumer
+__device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int cid) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    unsigned char* QQ = sm + sp::QQ;
+    unsigned char* KH = sm + sp::KH;
+    unsigned char* KT = sm + sp::KT;
+    unsigned char* UU = sm + sp::UU;
+    unsigned char* WW = sm + sp::WW;
+    unsigned char* STt = sm + sp::ST;
+    unsigned char* DT = sm + sp::DT;
+    float* sRed = reinterpret_cast<float*>(sm + sp::RED);
+    float* sGC = reinterpret_cast<float*>(sm + sp::GC);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + sp::BAR);
+    uint64_t* bar_mma = bar_load + 1;
+    int* abort_flag = reinterpret_cast<int*>(sm + sp::BAR + 28);
+    const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);   // this warp's TMEM lanes
+    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
+    const int T = p.T, H = p.H, nc = p.nc;
+    const bool want_o = (p.o != nullptr);
+
+    const uint32_t sQQ = tc::smem_u32(QQ), sKT = tc::smem_u32(KT), sUU = tc::smem_u32(UU),
+                   sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT), sTT = tc::smem_u32(sm + sp::TT),
+                   sPP = tc::smem_u32(sm + sp::PP), sWM = tc::smem_u32(sm + sp::WM);
     constexpr uint32_t ID_M3 = tc::idesc_bf16(128, 64, true, false);
     constexpr uint32_t ID_M4 = tc::idesc_bf16(128, 64, false, false, true);
     constexpr uint32_t ID_M56 = tc::idesc_bf16(64, 128, false, false);
@@ -156,109 +220,152 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         ph_mma ^= 1;
         tc::tc_fence_after();
     };
-    auto sync_for_mma = [&]() {   // smem written by threads + TMEM accesses done -> visible to the MMA issuer
+    // thread 0 waits for the WY image of (head, c); the caller synchronises the CTA afterwards
+    auto wait_wy = [&](size_t head, int c) {
+        if (!tc::flag_wait(p.flags + head * nc + c, 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 4u); }
+    };
+    auto copy_wy = [&](size_t head, int c) {   // every thread: 8 x 16 bytes of the 32 KB image
+        const unsigned char* src = p.wyimg + (head * nc + c) * TC_WY_BYTES;
+#pragma unroll
+        for (int i = 0; i < (int)(TC_WY_BYTES / 16 / NT); ++i)
+            tc::cp_async16_cg(sm + sp::WY + 16 * (tid + NT * i), src + 16 * (tid + NT * i));
+        tc::cp_async_commit();
+    };
+
+    for (int headi = cid; headi < p.BH; headi += p.ncons) {
+        const size_t head = (size_t)headi;
+        const int h = headi % H, b = headi / H;
+        auto issue_loads = [&](int c) {
+            const int t0 = c * C;
+            tc::mbar_arrive_expect_tx(bar_load, CONS_LOAD_BYTES);
+            tma_tile(QQ, C, 0, &m.q, b, h, t0, bar_load);
+            tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load);
+            tma_tile(KT, C, 0, &m.la, b, h, t0, bar_load);
+            tma_tile(UU, C, 0, &m.v, b, h, t0, bar_load);
+            tma_tile(WW, C, 0, &m.w, b, h, t0, bar_load);
+        };
+        if (tid == 0) {
+            issue_loads(0);
+            wait_wy(head, 0);
+        }
+        // initial state: S^T row j = column j of S0
+        {
+            const int j = jrow;
+            float v[32];
+#pragma unroll 1
+            for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] = p.S0 ? p.S0[(head * D + i0 + u) * D + j] : 0.f;
+                tc::tmem_st32(lane_base + TM_S + i0, v);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+            }
+            tc::tmem_wait_st();
+        }
         tc::fence_async_smem();
         tc::tc_fence_before();
         __syncthreads();
-    };
-
-    for (int c = 0; c < nc; ++c) {
-        const int t0 = c * C;
-        const int L = min(C, T - t0);
-        if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
-        ph_load ^= 1;
-
-        // ---- gate prep (thread = channel)
-        gate_prep(QE, KH, KT, UU, WW, sGC, sTf, tid, want_qp, true);
-        sync_for_mma();
-
-        // ---- M1: [A; P] = [Et; Qt] Kt^T
-        if (tid == 0) {
-            tc::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
-            tc::mma_commit(bar_mma);
-        }
-        wait_mma();
-        extract_AP(lane_base + TM_AP, sA, PP, want_qp, warp, lane);
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // ---- T = (I + A)^{-1}
-        solve_unit_lower(sA, sTf, sX, TT, tid);
-        sync_for_mma();
-        if (save && tid == 0) {   // T and P of this chunk for the backward
-            unsigned char* dst = tp + (head * nc + c) * TC_TP_BYTES;
-            tc::bulk_store(dst, TT, (uint32_t)(TC_TP_BYTES / 2));
-            tc::bulk_store(dst + TC_TP_BYTES / 2, PP, (uint32_t)(TC_TP_BYTES / 2));
+        tc::tc_fence_after();
+        copy_wy(head, 0);
+        if (p.states && tid == 0) {
+            tc::bulk_store(p.states + (head * nc + 0) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
             tc::bulk_commit();
         }
 
-        // ---- M2: Wm = T Et ;  M3: Delta^T := U^T T^T
-        if (tid == 0) {
-            tc::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), ID_M2, kk > 0);
-                tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M3, kk > 0);
-            }
-            tc::mma_commit(bar_mma);
-        }
-        wait_mma();
-        tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);   // Wm rows [t][i]
-        sync_for_mma();
+        for (int c = 0; c < nc; ++c) {
+            const int t0 = c * C;
+            const int L = min(C, T - t0);
+            if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
+            ph_load ^= 1;
 
-        // ---- M4: Delta^T -= S^T Wm^T ;  M5: O = Qt S
-        if (tid == 0) {
-            tc::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWW, C, 0, kk), ID_M4, 1);
-                if (want_o)
-                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sQE, 2 * C, C, kk), tc::desc_k(sST, D, 0, kk), ID_M56, kk > 0);
-            }
-            tc::mma_commit(bar_mma);
-        }
-        wait_mma();
-        tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
-        sync_for_mma();
+            // ---- gate prep: Qt, Kt, U, gC
+            gate_prep_state(QQ, KH, KT, UU, WW, sGC, sRed, tid);
+            tc::cp_async_wait_all();   // this chunk's WY image
+            sync_for_mma();
 
-        // ---- M6: O += P Delta ;  M7: Z^T = S^T + Delta^T Kt
-        if (tid == 0) {
-            tc::tc_fence_after();
+            // ---- M3: Delta^T := U^T T^T ;  M4: Delta^T -= S^T Wm^T ;  M5: O = Qt S
+            if (tid == 0) {
+                tc::tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                if (want_o)
-                    tc::mma_bf16(tmem + TM_O, tc::desc_k(sPP, C, 0, kk), tc::desc_k(sDT, D, 0, kk), ID_M56, 1);
-                tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sKT, C, 0, kk), ID_M7, 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M3, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWM, C, 0, kk), ID_M4, 1);
+                    if (want_o)
+                        tc::mma_bf16(tmem + TM_O, tc::desc_k(sQQ, C, 0, kk), tc::desc_k(sST, D, 0, kk), ID_M56, kk > 0);
+                }
+                tc::mma_commit(bar_mma);
             }
-            tc::mma_commit(bar_mma);
-        }
-        wait_mma();
-        // all smem input tiles of this chunk are consumed: prefetch the next chunk
-        if (tid == 0 && c + 1 < nc) issue_loads(c + 1);
+            wait_mma();
+            tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
+            sync_for_mma();
 
-        if (want_o) {   // o rows t from the M=64 accumulator: 16-byte stores
-            const int t = m64_row(warp, lane);
-            float v[32];
+            // ---- M6: O += P Delta ;  M7: Z^T = S^T + Delta^T Kt
+            if (tid == 0) {
+                tc::tc_fence_after();
 #pragma unroll
-            for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
-                tc::tmem_ld32(lane_base + TM_O + c0, v);
-                tc::tmem_wait_ld();
-                if (lane < 16 && t < L) {
-                    uint4* dst = reinterpret_cast<uint4*>(o + tok_off(b, t0 + t, h, T, H, D) + c0);
+                for (int kk = 0; kk < 4; ++kk) {
+                    if (want_o)
+                        tc::mma_bf16(tmem + TM_O, tc::desc_k(sPP, C, 0, kk), tc::desc_k(sDT, D, 0, kk), ID_M56, 1);
+                    tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sKT, C, 0, kk), ID_M7, 1);
+                }
+                tc::mma_commit(bar_mma);
+                if (c + 1 < nc) wait_wy(head, c + 1);   // overlaps the MMAs
+            }
+            wait_mma();
+            // every shared-memory input of this chunk is consumed: prefetch the next chunk
+            if (tid == 0 && c + 1 < nc) issue_loads(c + 1);
+
+            if (want_o) {   // o rows t from the M=64 accumulator: 16-byte stores
+                const int t = m64_row(warp, lane);
+                float v[32];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        dst[g] = make_uint4(tc::pack_bf16x2(v[8 * g], v[8 * g + 1]), tc::pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
-                                            tc::pack_bf16x2(v[8 * g + 4], v[8 * g + 5]), tc::pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
+                for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
+                    tc::tmem_ld32(lane_base + TM_O + c0, v);
+                    tc::tmem_wait_ld();
+                    if (lane < 16 && t < L) {
+                        uint4* dst = reinterpret_cast<uint4*>(p.o + tok_off(b, t0 + t, h, T, H, D) + c0);
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            dst[g] = make_uint4(tc::pack_bf16x2(v[8 * g], v[8 * g + 1]), tc::pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
+                                                tc::pack_bf16x2(v[8 * g + 4], v[8 * g + 5]), tc::pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
+                    }
                 }
             }
+            // S'^T = Z^T Diag(gC): scale the fp32 state, keep a bf16 copy for the next chunk
+            if (p.states && tid == 0) tc::bulk_wait_read();
+            __syncthreads();   // also orders thread 0's flag acquire before the image copy
+            if (c + 1 < nc) copy_wy(head, c + 1);
+            {
+                const int j = jrow;
+                float v[32];
+#pragma unroll 1
+                for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
+                    tc::tmem_ld32(lane_base + TM_S + i0, v);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
+                    tc::tmem_st32(lane_base + TM_S + i0, v);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+                }
+                tc::tmem_wait_st();
+            }
+            sync_for_mma();
+            tc::tc_fence_after();
+            if (p.states && tid == 0 && c + 1 < nc) {
+                tc::bulk_store(p.states + (head * nc + c + 1) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
+                tc::bulk_commit();
+            }
+            if (*abort_flag) {   // let the next chunk's loads land before leaving
+                if (tid == 0 && c + 1 < nc) (void)tc::mbar_wait(bar_load, ph_load);
+                break;
+            }
         }
-        // S'^T = Z^T Diag(gC): scale the fp32 state, keep a bf16 copy for the next chunk
-        if (states && tid == 0) tc::bulk_wait_read();
-        __syncthreads();
-        {
+
+        // final state (fp32): ST[i][j] from S^T (lane j)
+        if (p.ST) {
             const int j = jrow;
             float v[32];
 #pragma unroll 1
@@ -266,35 +373,45 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
-                tc::tmem_st32(lane_base + TM_S + i0, v);
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+                for (int u = 0; u < 32; ++u) p.ST[(head * D + i0 + u) * D + j] = v[u];
             }
-            tc::tmem_wait_st();
         }
-        sync_for_mma();
+        tc::cp_async_wait_all();
+        if (p.states && tid == 0) tc::bulk_wait_all();
+        tc::tc_fence_before();
+        __syncthreads();
         tc::tc_fence_after();
-        if (states && tid == 0 && c + 1 < nc) {
-            tc::bulk_store(states + (head * nc + c + 1) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
-            tc::bulk_commit();
-        }
         if (*abort_flag) break;
     }
+}
 
-    // final state (fp32): ST[i][j] from S^T (lane j)
-    if (ST) {
-        const int j = jrow;
-        float v[32];
-#pragma unroll 1
-        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
-            tc::tmem_ld32(lane_base + TM_S + i0, v);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < 32; ++u) ST[(head * D + i0 + u) * D + j] = v[u];
-        }
+__global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant__ Maps maps, const FwdParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const bool consumer = (int)blockIdx.x < p.ncons;
+    const uint32_t bar_off = consumer ? sp::BAR : wy::BAR;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + bar_off);
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + bar_off + 24);
+    int* abort_flag = reinterpret_cast<int*>(sm + bar_off + 28);
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) tc::mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&maps.q); tc::tma_prefetch_desc(&maps.k); tc::tma_prefetch_desc(&maps.la);
+        if (consumer) { tc::tma_prefetch_desc(&maps.v); tc::tma_prefetch_desc(&maps.w); }
+        else tc::tma_prefetch_desc(&maps.b);
     }
-    if (states && tid == 0) tc::bulk_wait_all();
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_base_ptr, TM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_base_ptr;
+    if (consumer) run_consumer(maps, p, sm, tmem, blockIdx.x);
+    else run_producer(maps, p, sm, tmem, blockIdx.x - p.ncons);
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -308,16 +425,50 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
-    CUtensorMap mq, mk, mv, mla, mb, mw;
+    Maps maps;
     const void* ptrs[6] = {a.q, a.k, a.v, a.la, a.b, a.w};
-    CUtensorMap* maps[6] = {&mq, &mk, &mv, &mla, &mb, &mw};
+    CUtensorMap* mp[6] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w};
     for (int i = 0; i < 6; ++i)
-        if (make_token_map(maps[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 0, coop = 0, occ = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, chunk_fwd_kernel, NT, SMEM_BYTES)) != cudaSuccess)
+        return e;
+    const int BH = d.B * d.H, nc = d.nchunks();
+    const int units = BH * nc;
+    const int slots = nsm * occ;
+
+    FwdParams p{};
+    p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
+    p.S0 = a.S0; p.o = static_cast<__nv_bfloat16*>(a.o); p.ST = a.ST;
+    p.states = a.states; p.wyimg = a.wy; p.flags = a.flags;
+    if ((e = cudaMemsetAsync(a.flags, 0, (size_t)units * sizeof(unsigned int), s)) != cudaSuccess) return e;
+
     TraceScope trace(K_CHUNK_FWD, s);
-    chunk_fwd_kernel<<<d.B * d.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mla, mb, mw, a.S0,
-                                                       static_cast<__nv_bfloat16*>(a.o), a.ST, a.states, a.tp, d.T, d.H);
+    // Heads share the launch with the producers while the producers keep pace: per chunk step the
+    // BH consumer chunks take about as long as BH WY units spread over the remaining CTAs.
+    if (coop && slots >= 2 && 16 * BH <= 9 * slots) {
+        p.ncons = BH;
+        p.nprod = slots - BH < units ? slots - BH : units;
+        void* args[2] = {&maps, &p};
+        e = cudaLaunchCooperativeKernel((const void*)chunk_fwd_kernel, dim3(p.ncons + p.nprod), dim3(NT), args,
+                                        SMEM_BYTES, s);
+        if (e == cudaSuccess) return cudaSuccess;
+        (void)cudaGetLastError();   // not launched: fall back to two launches
+    }
+    FwdParams pp = p;   // producers only
+    pp.ncons = 0;
+    pp.nprod = units < slots ? units : slots;
+    chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    FwdParams pc = p;   // consumers only; every flag is set when they start
+    pc.ncons = BH;
+    pc.nprod = 0;
+    chunk_fwd_kernel<<<BH, NT, SMEM_BYTES, s>>>(maps, pc);
     return cudaGetLastError();
 }
 

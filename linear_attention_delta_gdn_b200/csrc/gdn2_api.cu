@@ -53,16 +53,25 @@ gdn2_status check_dims(int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtyp
     return GDN2_OK;
 }
 
-// Forward-saved region: chunk-start states (and, on the tensor-core path, the [T | P] tiles).
+// Tensor-core workspace (units = B*H*NC chunks), each region 256-byte aligned:
+//   [states: units x TC_STATE_BYTES, training only][WY images: units x TC_WY_BYTES][ready flags]
+//   then, for the backward, [dstates: units x TC_STATE_BYTES].
+size_t tc_units(const Dims& d) { return (size_t)d.B * d.H * (size_t)d.nchunks(); }
+size_t tc_wy_bytes(const Dims& d) { return tc_units(d) * TC_WY_BYTES + align256(tc_units(d) * sizeof(unsigned int)); }
+
+// Forward-saved region: chunk-start states (and, on the tensor-core path, the WY images and flags).
 size_t states_bytes(const Dims& d, gdn2_dtype dt) {
-    const size_t units = (size_t)d.B * d.H * (size_t)d.nchunks();
-    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * (TC_STATE_BYTES + TC_TP_BYTES)
+    const size_t units = tc_units(d);
+    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * TC_STATE_BYTES + tc_wy_bytes(d)
                                                   : units * d.Dk * d.Dv * sizeof(float);
 }
-size_t tc_tp_offset(const Dims& d) { return (size_t)d.B * d.H * (size_t)d.nchunks() * TC_STATE_BYTES; }
+size_t tc_tp_offset(const Dims& d) { return tc_units(d) * TC_STATE_BYTES; }
+size_t tc_flags_offset(const Dims& d, bool with_states) {
+    return (with_states ? tc_tp_offset(d) : 0) + tc_units(d) * TC_WY_BYTES;
+}
 
 size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
-    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk)) return (size_t)d.B * d.H * (size_t)d.nchunks() * TC_STATE_BYTES;
+    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk)) return tc_units(d) * TC_STATE_BYTES;
     const size_t seg = (size_t)d.B * d.H * d.chunk * d.Dk * d.Dv * sizeof(float);
     const size_t del = (size_t)d.B * d.H * d.chunk * d.Dv * sizeof(float);
     return align256(seg) + align256(del);
@@ -115,7 +124,7 @@ size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int 
     if (check_dims(B, T, H, Dk, Dv, chunk, dt, true) != GDN2_OK) return 0;
     const Dims d{B, T, H, Dk, Dv, chunk};
     switch (op) {
-    case GDN2_OP_FWD: return 0;
+    case GDN2_OP_FWD: return tc_path(dt, Dk, Dv, chunk) ? align256(tc_wy_bytes(d)) : 0;
     case GDN2_OP_FWD_SAVE: return align256(states_bytes(d, dt));
     case GDN2_OP_BWD: return align256(states_bytes(d, dt)) + align256(bwd_extra_bytes(d, dt));
     }
@@ -135,19 +144,23 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
     if (T == 0) return copy_or_zero_state(ST, S0, d, s);
     REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(log_alpha);
     REQUIRE_PTR(b); REQUIRE_PTR(w); REQUIRE_PTR(o);
-    if (save_states) {
-        const size_t need = gdn2_workspace_size(GDN2_OP_FWD_SAVE, B, T, H, Dk, Dv, chunk, dt);
-        if (!ws || ws_bytes < need)
-            return fail(GDN2_ERR_WORKSPACE, "save_states needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
-        if (!aligned(ws, 256)) return fail(GDN2_ERR_INVALID, "ws must be 256-byte aligned");
+    {
+        const size_t need = gdn2_workspace_size(save_states ? GDN2_OP_FWD_SAVE : GDN2_OP_FWD, B, T, H, Dk, Dv, chunk, dt);
+        if (need && (!ws || ws_bytes < need))
+            return fail(GDN2_ERR_WORKSPACE, "gdn2_fwd%s needs %zu workspace bytes, got %zu",
+                        save_states ? " with save_states" : "", need, ws ? ws_bytes : 0);
+        if (need && !aligned(ws, 256)) return fail(GDN2_ERR_INVALID, "ws must be 256-byte aligned");
     }
     if (save_states ? tc_train_path(dt, Dk, Dv, chunk) : tc_path(dt, Dk, Dv, chunk)) {
         ChunkFwdArgs a{};
         a.d = d;
         a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
         a.S0 = S0; a.o = o; a.ST = ST;
-        a.states = save_states ? static_cast<unsigned char*>(ws) : nullptr;
-        a.tp = save_states ? static_cast<unsigned char*>(ws) + tc_tp_offset(d) : nullptr;
+        unsigned char* wsb = static_cast<unsigned char*>(ws);
+        const bool keep = save_states != 0;
+        a.states = keep ? wsb : nullptr;
+        a.wy = wsb + (keep ? tc_tp_offset(d) : 0);
+        a.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, keep));
         return cuda_status(chunk_fwd_launch(a, s), "gdn2_fwd (tensor-core path)");
     }
     RecurrentArgs a{};
@@ -189,7 +202,8 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
             ChunkFwdArgs f{};
             f.d = d;
             f.q = q; f.k = k; f.v = v; f.la = log_alpha; f.b = b; f.w = w;
-            f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.tp = wsb + tc_tp_offset(d);
+            f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.wy = wsb + tc_tp_offset(d);
+            f.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, true));
             gdn2_status e = cuda_status(chunk_fwd_launch(f, s), "gdn2_bwd state recompute");
             if (e != GDN2_OK) return e;
         }

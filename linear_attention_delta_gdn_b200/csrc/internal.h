@@ -30,8 +30,9 @@ constexpr int TC_D = 128;
 constexpr int TC_C = 64;
 // bytes of one saved state image (bf16 128 x 128, 128B-swizzled panels)
 constexpr size_t TC_STATE_BYTES = (size_t)TC_D * TC_D * 2;
-// bytes of one saved [T | P] image per chunk (two bf16 64 x 64 tiles)
+// bytes of one WY image per chunk: T and P (bf16 64 x 64 tiles), then Wm (bf16 64 x 128 tile)
 constexpr size_t TC_TP_BYTES = (size_t)2 * TC_C * TC_C * 2;
+constexpr size_t TC_WY_BYTES = TC_TP_BYTES + (size_t)TC_C * TC_D * 2;
 
 struct ChunkFwdArgs {
     Dims d;
@@ -40,7 +41,8 @@ struct ChunkFwdArgs {
     void* o;               // may be null: states only
     float* ST;
     unsigned char* states; // [B,H,NC] chunk-start state images, or null
-    unsigned char* tp;     // [B,H,NC] [T | P] images (written when states != null)
+    unsigned char* wy;     // [B,H,NC] WY images (T | P | Wm), always written
+    unsigned int* flags;   // [B,H,NC] ready flags (scratch)
 };
 cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s);
 
@@ -51,7 +53,7 @@ struct ChunkBwdArgs {
     void *dq, *dk, *dv, *dla, *db, *dw;
     float* dS0;
     const unsigned char* states;  // [B,H,NC] chunk-start state images
-    const unsigned char* tp;      // [B,H,NC] [T | P] images of every chunk
+    const unsigned char* tp;      // [B,H,NC] WY images (T | P | Wm) of every chunk
     unsigned char* dstates;       // [B,H,NC] images of Diag(gC) dL/dS' per chunk (scratch)
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);

@@ -254,5 +254,35 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 // wait until all committed bulk stores are complete
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// 16-byte global -> shared copy through L2 only (not L1), completed by cp_async_wait_all().
+__device__ __forceinline__ void cp_async16_cg(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// ------------------------------------------------------------ flags between CTAs of one launch
+// Publishing: every thread writes its data, __syncthreads(), then one thread calls flag_release
+// (a gpu-scope acq_rel fence orders the whole CTA's earlier writes before the flag store).
+__device__ __forceinline__ void flag_release(unsigned int* flag, unsigned int value) {
+    asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(value) : "memory");
+}
+__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* flag) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    return v;
+}
+// One thread waits until *flag == value (acquire), then the CTA synchronises before reading the
+// published data. Gives up after ~2 s and returns false.
+__device__ __forceinline__ bool flag_wait(const unsigned int* flag, unsigned int value) {
+    if (ld_acquire(flag) == value) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire(flag) == value) return true;
+        if (global_timer_ns() - t0 > 2000000000ull) return false;
+    }
+}
+
 }  // namespace tc
 }  // namespace gdn2

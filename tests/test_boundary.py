@@ -52,10 +52,15 @@ def test_workspace_sizes(L):
     fs = ws(1, 1, 256, 2, 64, 64, 64, 0)
     assert fs >= 1 * 2 * 4 * 64 * 64 * 4 and fs % 256 == 0
     assert ws(2, 1, 256, 2, 64, 64, 64, 0) > fs
-    # bf16 shape of the 1.3B training layer
+    # bf16 shape of the 1.3B training layer: the inference forward keeps a WY image
+    # (T | P | Wm, 32 KB) and a ready flag per chunk; training adds the state images
+    units = 4 * 16 * 64
+    i = ws(0, 4, 4096, 16, 128, 128, 64, 1)
+    assert i == units * 32768 + units * 4
     f = ws(1, 4, 4096, 16, 128, 128, 64, 1)
     b = ws(2, 4, 4096, 16, 128, 128, 64, 1)
-    assert 0 < f < b
+    assert f == units * 32768 + i
+    assert b == f + units * 32768
     # ragged T rounds the chunk count up
     assert ws(1, 1, 65, 1, 128, 128, 64, 1) == ws(1, 1, 128, 1, 128, 128, 64, 1)
     # invalid problems report zero
@@ -87,6 +92,10 @@ def test_fwd_rejects_bad_arguments(L):
     assert _fwd(L, save=1) == 3                            # no workspace
     assert _fwd(L, save=1, ws=1 << 20, wsb=16) == 3        # too small
     assert b"workspace" in L.gdn2_last_error()
+    # the tensor-core forward needs its WY workspace even without save_states
+    assert _fwd(L, Dk=128, Dv=128) == 3
+    assert _fwd(L, Dk=128, Dv=128, ws=(1 << 20) + 16, wsb=1 << 30) == 1   # misaligned workspace
+    assert b"256-byte" in L.gdn2_last_error()
 
 
 def test_bwd_and_decode_reject_bad_arguments(L):
