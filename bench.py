@@ -35,16 +35,15 @@ WORKLOAD = "fwdbwd-bf16-b4h16t4096d128"
 # o (7 x 256 B); the backward reads the six inputs and dout and writes six
 # gradients (13 x 256 B); plus the fp32 final state and dS0 per head. Per kernel:
 #   chunk_fwd_kernel      7 x 256 B  (its inputs and o)
-#   reverse_state_kernel  5 x 256 B  (q, k, log_alpha, b, dout)
-#   chunk_grad_kernel    13 x 256 B  (all backward inputs and gradients)
+#   chunk_bwd_kernel     13 x 256 B  (all backward inputs and gradients: reverse pass and
+#                                     per-chunk gradients run in the same launch)
 # Flops: forward 180,224 per token and head (the chunk contractions), backward
 # counted as twice the forward.
 STEP_BYTES_PER_TOKEN_HEAD = 1792 + 3328
 STEP_FLOPS_PER_TOKEN_HEAD = 3 * 180224
-KERNEL_BYTES_PER_TOKEN_HEAD = {"chunk_fwd_kernel": 1792, "reverse_state_kernel": 1280, "chunk_grad_kernel": 3328,
+KERNEL_BYTES_PER_TOKEN_HEAD = {"chunk_fwd_kernel": 1792, "chunk_bwd_kernel": 3328,
                                "recurrent_fwd_kernel": 1792, "recurrent_bwd_kernel": 3328}
-KERNEL_SOURCES = {"chunk_fwd_kernel": ["chunk_fwd.cu"], "reverse_state_kernel": ["chunk_bwd.cu"],
-                  "chunk_grad_kernel": ["chunk_bwd.cu"]}
+KERNEL_SOURCES = {"chunk_fwd_kernel": ["chunk_fwd.cu"], "chunk_bwd_kernel": ["chunk_bwd.cu"]}
 COMMON_SOURCES = ["chunk_common.cuh", "tc.cuh", "common.cuh"]
 
 

@@ -19,11 +19,17 @@
 //   E = rowsum(dZ * S) + sum_t Kt_t * (Delta dZ^T)_t   (the dependence of S' on gC)
 //   dlog_alpha_t = sum_{tau >= t} dG_tau + E
 //
-// Two kernels, both reading the forward's per-chunk T and P tiles instead of redoing the solve:
-//   reverse_state_kernel  one CTA per (batch, head) walks the chunks backwards carrying
-//                         dS^T in TMEM (fp32) and stores each chunk's dZ^T as a bf16 image;
-//   chunk_grad_kernel     one CTA per (batch, head, chunk) computes every gradient of the
-//                         chunk from the saved S, dZ, T, P, the inputs and dout.
+// One launch, two kinds of work, both reading the forward's per-chunk T and P tiles instead of
+// redoing the solve:
+//   reverse pass    one CTA per (batch, head) walks the chunks backwards carrying dS^T in TMEM
+//                   (fp32); per chunk it writes dZ^T as a bf16 image and then sets the chunk's
+//                   ready flag (release);
+//   chunk gradients every other CTA takes (head, chunk) units from a shared counter, in the
+//                   order the reverse pass produces them, waits for the unit's flag (acquire) and
+//                   computes every gradient of the chunk from the saved S, dZ, T, P, the inputs and
+//                   dout. Reverse-pass CTAs join them once their head is done.
+// With few heads this is one cooperative launch (all CTAs resident, so every wait ends; each wait is
+// also bounded in time); otherwise the reverse pass and the gradients run as two launches.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -41,6 +47,33 @@ __device__ unsigned int g_bwd_error;
 
 constexpr uint32_t TILE_C = 64 * 64 * 2;   // bytes of a 64 x 64 bf16 tile
 
+// Barrier block shared by both kinds of work (above every tile of either layout):
+// 4 mbarriers (load, mma, k, b), TMEM base, abort flag, broadcast unit index.
+constexpr uint32_t OFF_BARS = 229888;
+constexpr uint32_t SMEM_BYTES_ALL = 229952 + 1024;
+
+struct BwdMaps {
+    CUtensorMap q, k, v, la, b, w, dout, dq, dk, db, dla;
+};
+struct BwdParams {
+    int T, H, BH, nc;
+    int nrev;                        // CTAs [0, nrev) run the reverse pass of head blockIdx.x
+    int join;                        // reverse-pass CTAs take gradient units afterwards
+    int grad;                        // this launch computes gradient units
+    const float* dST;
+    float* dS0;
+    __nv_bfloat16 *dv, *dw;
+    const unsigned char* states;     // chunk-start state images
+    const unsigned char* tp;         // WY images (T | P | Wm)
+    unsigned char* dstates;          // dZ^T images
+    unsigned int* flags;             // [BH, nc] dZ ready flags (zero at launch)
+    unsigned int* counter;           // [0]: next gradient unit, [1]: abort word (zero at launch)
+};
+// mbarrier parities carried across the units a CTA works on
+struct Phases {
+    uint32_t load = 0, mma = 0, k = 0, b = 0;
+};
+
 // ====================================================================== reverse state pass
 
 namespace rs {
@@ -55,21 +88,13 @@ constexpr uint32_t OFF_TT = 147456;      // T (bf16, from the forward)
 constexpr uint32_t OFF_PP = 155648;      // P (bf16, from the forward)
 constexpr uint32_t OFF_RED = 163840;     // prep scan scratch (8 KB)
 constexpr uint32_t OFF_GC = 172032;
-constexpr uint32_t OFF_BAR = 172544;
-constexpr uint32_t SMEM_BYTES = 172608 + 1024;
-constexpr uint32_t TM_S = 0, TM_D = 128, TM_W = 192, TM_COLS = 512;
+constexpr uint32_t TM_S = 0, TM_D = 128, TM_W = 192;
 constexpr uint32_t LOAD_BYTES = 5 * 64 * 128 * 2 + 2 * TILE_C;
 }  // namespace rs
 
-__global__ void __launch_bounds__(NT, 1)
-reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                     const __grid_constant__ CUtensorMap mla, const __grid_constant__ CUtensorMap mb,
-                     const __grid_constant__ CUtensorMap mdo, const float* __restrict__ dST,
-                     float* __restrict__ dS0, const unsigned char* __restrict__ tp,
-                     unsigned char* __restrict__ dstates, int T, int H) {
+__device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi,
+                            Phases& ph) {
     using namespace rs;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     unsigned char* QE = sm + OFF_QE;
     unsigned char* KH = sm + OFF_KH;
     unsigned char* KT = sm + OFF_KT;
@@ -81,42 +106,26 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     unsigned char* PP = sm + OFF_PP;
     float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_load + 1;
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
-    int* abort_flag = reinterpret_cast<int*>(sm + OFF_BAR + 20);
+    int* abort_flag = reinterpret_cast<int*>(sm + OFF_BARS + 36);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x % H, b = blockIdx.x / H;
-    const size_t head = blockIdx.x;
-    const int nc = (T + C - 1) / C;
-
-    if (tid == 0) {
-        tc::mbar_init(bar_load, 1);
-        tc::mbar_init(bar_mma, 1);
-        *abort_flag = 0;
-        tc::fence_mbar_init();
-    }
-    if (warp == 0) {
-        tc::tmem_alloc(tmem_base_ptr, TM_COLS);
-        tc::tmem_relinquish();
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = *tmem_base_ptr;
+    const int h = headi % p.H, b = headi / p.H;
+    const size_t head = (size_t)headi;
+    const int nc = p.nc;
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
 
     auto issue_loads = [&](int c) {
         const int t0 = c * C;
         tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-        tma_tile(QE, 2 * C, 0, &mb, b, h, t0, bar_load);
-        tma_tile(QE, 2 * C, C, &mq, b, h, t0, bar_load);
-        tma_tile(KH, C, 0, &mk, b, h, t0, bar_load);
-        tma_tile(KT, C, 0, &mla, b, h, t0, bar_load);
-        tma_tile(DO, C, 0, &mdo, b, h, t0, bar_load);
-        const unsigned char* src = tp + (head * nc + c) * TC_WY_BYTES;
+        tma_tile(QE, 2 * C, 0, &m.b, b, h, t0, bar_load);
+        tma_tile(QE, 2 * C, C, &m.q, b, h, t0, bar_load);
+        tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load);
+        tma_tile(KT, C, 0, &m.la, b, h, t0, bar_load);
+        tma_tile(DO, C, 0, &m.dout, b, h, t0, bar_load);
+        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;
         tc::bulk_load(TT, src, TILE_C, bar_load);
         tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
     };
@@ -128,7 +137,7 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 #pragma unroll 1
         for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] = dST ? dST[(head * D + i0 + u) * D + j] : 0.f;
+            for (int u = 0; u < 32; ++u) v[u] = p.dST ? p.dST[(head * D + i0 + u) * D + j] : 0.f;
             tc::tmem_st32(lane_base + TM_S + i0, v);
         }
         tc::tmem_wait_st();
@@ -146,10 +155,9 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     constexpr uint32_t ID_N2a = tc::idesc_bf16(128, 128, true, true);
     constexpr uint32_t ID_N2b = tc::idesc_bf16(128, 128, false, true, true);
 
-    uint32_t ph_load = 0, ph_mma = 0;
     auto wait_mma = [&]() {
-        if (!tc::mbar_wait(bar_mma, ph_mma)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 1u); }
-        ph_mma ^= 1;
+        if (!tc::mbar_wait(bar_mma, ph.mma)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 1u); }
+        ph.mma ^= 1;
         tc::tc_fence_after();
     };
     auto sync_for_mma = [&]() {
@@ -158,14 +166,14 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         __syncthreads();
     };
 
+    int unreleased = -1;   // chunk whose dZ image is written but whose flag is not yet set
     for (int c = nc - 1; c >= 0; --c) {
-        if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
-        ph_load ^= 1;
+        if (!tc::mbar_wait(bar_load, ph.load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
+        ph.load ^= 1;
 
         gate_prep(QE, KH, KT, nullptr, nullptr, sGC, sRed, tid, true, false);
-        // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
-        if (tid == 0) tc::bulk_wait_read();
         __syncthreads();
+        // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
         {
             const int j = jrow;
             float v[32];
@@ -185,8 +193,6 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 
         // Wm = T Et (M=64) ;  dDelta^T = dZ^T Kt^T + dO^T P
         if (tid == 0) {
-            tc::bulk_store(dstates + (head * nc + c) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
-            tc::bulk_commit();
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -199,6 +205,16 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
                 tc::mma_bf16(tmem + TM_D, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), ID_N1b, 1);
             tc::mma_commit(bar_mma);
         }
+        // the previous chunk's dZ image stores have drained: publish it while the MMAs run
+        if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
+        // this chunk's dZ^T image for the gradient units (plain stores, published one chunk later)
+        {
+            uint4* dst = reinterpret_cast<uint4*>(p.dstates + (head * nc + c) * TC_STATE_BYTES);
+            const uint4* src = reinterpret_cast<const uint4*>(STt);
+#pragma unroll
+            for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / NT); ++i) dst[tid + NT * i] = src[tid + NT * i];
+        }
+        unreleased = c;
         wait_mma();
         tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);    // Wm rows
         tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
@@ -219,10 +235,17 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
-        if (*abort_flag) break;
+        if (*abort_flag) {   // let the next chunk's loads land before leaving
+            if (tid == 0) {
+                atomicExch(p.counter + 1, 1u);   // gradient units of this head will never be ready
+                if (c > 0) (void)tc::mbar_wait(bar_load, ph.load);
+            }
+            break;
+        }
     }
+    if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
 
-    if (dS0) {   // dS0[i][j] from dS^T (lane j)
+    if (p.dS0) {   // dS0[i][j] from dS^T (lane j)
         const int j = jrow;
         float v[32];
 #pragma unroll 1
@@ -230,16 +253,12 @@ reverse_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
             tc::tmem_ld32(lane_base + TM_S + i0, v);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 32; ++u) dS0[(head * D + i0 + u) * D + j] = v[u];
+            for (int u = 0; u < 32; ++u) p.dS0[(head * D + i0 + u) * D + j] = v[u];
         }
     }
-    if (tid == 0) tc::bulk_wait_all();
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
-        tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, TM_COLS);
-    }
+    tc::tc_fence_after();
 }
 
 // ====================================================================== per-chunk gradients
@@ -258,8 +277,6 @@ constexpr uint32_t OFF_DDT = 196608;     // Wm rows, then dDelta^T [128 x 64], l
 constexpr uint32_t OFF_TT = 212992;      // T, later dA^T [64 x 64]
 constexpr uint32_t OFF_PP = 221184;      // P, later dP^T [64 x 64]
 constexpr uint32_t OFF_GC = 229376;
-constexpr uint32_t OFF_BAR = 229888;
-constexpr uint32_t SMEM_BYTES = 229952 + 1024;
 // TMEM columns (M=64 accumulators use lanes 0-15 of each 32-lane quarter)
 constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_W = 64,                     // Wm (M=64, 128 columns), later dA^T (M=64, 64 columns)
@@ -267,23 +284,14 @@ constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_DD = 256,                   // dDelta^T, later G3 = dKt^T (P and A paths)
     TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
     TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,
-    TM_GV = 448,                   // G[t] per key channel (cumulative log-decay)
-    TM_COLS = 512;
-constexpr uint32_t LOAD_BYTES = 7 * 64 * 128 * 2 + 2 * (uint32_t)TC_STATE_BYTES + 2 * TILE_C;
+    TM_GV = 448;                   // G[t] per key channel (cumulative log-decay)
+constexpr uint32_t LOAD_BYTES = 7 * 64 * 128 * 2 + (uint32_t)TC_STATE_BYTES + 2 * TILE_C;   // dZ^T: cp.async
 }  // namespace cg
 
-__global__ void __launch_bounds__(NT, 1)
-chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                  const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mla,
-                  const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
-                  const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mdq,
-                  const __grid_constant__ CUtensorMap mdk, const __grid_constant__ CUtensorMap mdb,
-                  const __grid_constant__ CUtensorMap mdla, __nv_bfloat16* __restrict__ dv,
-                  __nv_bfloat16* __restrict__ dw, const unsigned char* __restrict__ states,
-                  const unsigned char* __restrict__ tp, const unsigned char* __restrict__ dstates, int T, int H) {
+// Gradients of chunk c of head `headi`; returns false if a bounded wait gave up.
+__device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi, int c,
+                          Phases& ph) {
     using namespace cg;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     unsigned char* QE = sm + OFF_QE;
     unsigned char* KH = sm + OFF_KH;
     unsigned char* KT = sm + OFF_KT;
@@ -297,55 +305,60 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_load + 1;
     uint64_t* bar_k = bar_load + 2;
     uint64_t* bar_b = bar_load + 3;
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 32);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x;
-    const int h = blockIdx.y % H, b = blockIdx.y / H;
-    const size_t head = blockIdx.y;
-    const int nc = gridDim.x;
+    const int T = p.T, H = p.H, nc = p.nc;
+    const int h = headi % H, b = headi / H;
+    const size_t head = (size_t)headi;
     const int t0 = c * C;
     const int L = min(C, T - t0);
+    const CUtensorMap *mq = &m.q, *mk = &m.k, *mv = &m.v, *mla = &m.la, *mb = &m.b, *mw = &m.w, *mdo = &m.dout;
+    const CUtensorMap *mdq = &m.dq, *mdk = &m.dk, *mdb = &m.db, *mdla = &m.dla;
+    __nv_bfloat16* __restrict__ dv = p.dv;
+    __nv_bfloat16* __restrict__ dw = p.dw;
 
+    bool ok = true;
     if (tid == 0) {
-        tc::mbar_init(bar_load, 1);
-        tc::mbar_init(bar_mma, 1);
-        tc::mbar_init(bar_k, 1);
-        tc::mbar_init(bar_b, 1);
-        tc::fence_mbar_init();
         tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-        tma_tile(QE, 2 * C, 0, &mb, b, h, t0, bar_load);
-        tma_tile(QE, 2 * C, C, &mq, b, h, t0, bar_load);
-        tma_tile(KH, C, 0, &mk, b, h, t0, bar_load);
-        tma_tile(KT, C, 0, &mla, b, h, t0, bar_load);
-        tma_tile(UU, C, 0, &mv, b, h, t0, bar_load);
-        tma_tile(WW, C, 0, &mw, b, h, t0, bar_load);
-        tma_tile(DO, C, 0, &mdo, b, h, t0, bar_load);
-        tc::bulk_load(STt, states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
-        tc::bulk_load(DS, dstates + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
-        const unsigned char* src = tp + (head * nc + c) * TC_WY_BYTES;
+        tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
+        tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load);
+        tma_tile(KH, C, 0, mk, b, h, t0, bar_load);
+        tma_tile(KT, C, 0, mla, b, h, t0, bar_load);
+        tma_tile(UU, C, 0, mv, b, h, t0, bar_load);
+        tma_tile(WW, C, 0, mw, b, h, t0, bar_load);
+        tma_tile(DO, C, 0, mdo, b, h, t0, bar_load);
+        tc::bulk_load(STt, p.states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
+        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;
         tc::bulk_load(TT, src, TILE_C, bar_load);
         tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
+        // dZ^T of this chunk comes from the reverse pass: wait for its flag
+        if (!tc::flag_wait(p.flags + head * nc + c, 1u)) {
+            ok = false;
+            atomicOr(&g_bwd_error, 8u);
+            atomicExch(p.counter + 1, 1u);
+        }
     }
-    if (warp == 0) {
-        tc::tmem_alloc(tmem_base_ptr, TM_COLS);
-        tc::tmem_relinquish();
+    __syncthreads();   // orders thread 0's acquire before every thread's copy of the dZ^T image
+    {
+        const unsigned char* src = p.dstates + (head * nc + c) * TC_STATE_BYTES;
+#pragma unroll
+        for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / NT); ++i)
+            tc::cp_async16_cg(DS + 16 * (tid + NT * i), src + 16 * (tid + NT * i));
+        tc::cp_async_commit();
     }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = *tmem_base_ptr;
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
-    uint32_t ph_mma = 0;
-    bool ok = tc::mbar_wait(bar_load, 0);
+    (void)jrow;
+    ok = tc::mbar_wait(bar_load, ph.load) && ok;
+    ph.load ^= 1;
+    tc::cp_async_wait_all();
     auto wait_mma = [&]() {
-        ok = tc::mbar_wait(bar_mma, ph_mma) && ok;
-        ph_mma ^= 1;
+        ok = tc::mbar_wait(bar_mma, ph.mma) && ok;
+        ph.mma ^= 1;
         tc::tc_fence_after();
     };
     auto sync_for_mma = [&]() {
@@ -378,7 +391,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     wait_mma();
     if (tid == 0) {     // U is consumed: bring k back for the gate chain
         tc::mbar_arrive_expect_tx(bar_k, 64 * 128 * 2);
-        tma_tile(KH, C, 0, &mk, b, h, t0, bar_k);
+        tma_tile(KH, C, 0, mk, b, h, t0, bar_k);
     }
     tmem_m64_to_tile(lane_base + TM_W, DDT, warp, lane);      // Wm rows (DDT is free until dDelta^T)
     sync_for_mma();
@@ -449,7 +462,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     sync_for_mma();
     if (tid == 0) {     // w is consumed: bring b back for the gate chain
         tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
-        tma_tile(WW, C, 0, &mb, b, h, t0, bar_b);
+        tma_tile(WW, C, 0, mb, b, h, t0, bar_b);
     }
 
     // ---- dP^T = Delta dO^T (M=64), dA^T = -Delta dU^T (M=64)
@@ -525,8 +538,10 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         Epart += e2;
     }
     wait_mma();
-    ok = tc::mbar_wait(bar_k, 0) && ok;
-    ok = tc::mbar_wait(bar_b, 0) && ok;
+    ok = tc::mbar_wait(bar_k, ph.k) && ok;
+    ph.k ^= 1;
+    ok = tc::mbar_wait(bar_b, ph.b) && ok;
+    ph.b ^= 1;
 
     // ---- gate chain, thread = (key channel i, token half hf). Pass 1 over the half's 32 tokens: dq, dk,
     // db and dG_t; partial sums of Kt*G4 and dG are exchanged between the halves (in the consumed dP^T
@@ -583,7 +598,7 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     tc::fence_async_smem();
     __syncthreads();
     if (tid == 0) {   // rows past the end of the sequence are skipped by the tensor store
-        const CUtensorMap* maps[4] = {&mdq, &mdk, &mdb, &mdla};
+        const CUtensorMap* maps[4] = {mdq, mdk, mdb, mdla};
         const unsigned char* tiles[4] = {DO, DT, DDT, UU};
 #pragma unroll
         for (int o = 0; o < 4; ++o) {
@@ -594,12 +609,56 @@ chunk_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tc::bulk_wait_read();
     }
     if (!ok) atomicOr(&g_bwd_error, 4u);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    return ok;
+}
 
+__global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
+    const int tid = threadIdx.x, warp = tid >> 5;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 32);
+    int* abort_flag = reinterpret_cast<int*>(sm + OFF_BARS + 36);
+    int* unit_bcast = reinterpret_cast<int*>(sm + OFF_BARS + 40);
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_base_ptr, 512);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_base_ptr;
+    Phases ph;
+    const bool reverse = (int)blockIdx.x < p.nrev;
+    if (reverse) run_reverse(maps, p, sm, tmem, blockIdx.x, ph);
+    if (p.grad && (!reverse || p.join) && !*abort_flag) {
+        const int units = p.BH * p.nc;
+        while (true) {
+            if (tid == 0)   // stop taking units once any CTA of the launch has given up
+                *unit_bcast = *reinterpret_cast<volatile unsigned int*>(p.counter + 1) ? units
+                                                                                       : (int)atomicAdd(p.counter, 1u);
+            __syncthreads();
+            const int u = *unit_bcast;
+            __syncthreads();
+            if (u >= units) break;
+            // units in the order the reverse pass produces them: chunks from the last, heads inside
+            const int c = p.nc - 1 - u / p.BH, headi = u % p.BH;
+            if (!grad_unit(maps, p, sm, tmem, headi, c, ph)) break;
+        }
+    }
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, TM_COLS);
+        tc::tmem_dealloc(tmem, 512);
     }
 }
 
@@ -613,27 +672,48 @@ cudaError_t set_smem(K kernel, uint32_t bytes) {
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
-    CUtensorMap mq, mk, mv, mla, mb, mw, mdo, mdq, mdk, mdb, mdla;
+    BwdMaps maps;
     const void* ptrs[11] = {a.q, a.k, a.v, a.la, a.b, a.w, a.dout, a.dq, a.dk, a.db, a.dla};
-    CUtensorMap* maps[11] = {&mq, &mk, &mv, &mla, &mb, &mw, &mdo, &mdq, &mdk, &mdb, &mdla};
+    CUtensorMap* mp[11] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w, &maps.dout,
+                           &maps.dq, &maps.dk, &maps.db, &maps.dla};
     for (int i = 0; i < 11; ++i)
-        if (make_token_map(maps[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    cudaError_t e = set_smem(reverse_state_kernel, rs::SMEM_BYTES);
+        if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    cudaError_t e = set_smem(chunk_bwd_kernel, SMEM_BYTES_ALL);
     if (e != cudaSuccess) return e;
-    e = set_smem(chunk_grad_kernel, cg::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    {
-        TraceScope trace(K_REVERSE, s);
-        reverse_state_kernel<<<d.B * d.H, NT, rs::SMEM_BYTES, s>>>(mq, mk, mla, mb, mdo, a.dST, a.dS0, a.tp,
-                                                                    a.dstates, d.T, d.H);
+    int dev = 0, nsm = 0, coop = 0, occ = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, chunk_bwd_kernel, NT, SMEM_BYTES_ALL)) != cudaSuccess)
+        return e;
+    const int BH = d.B * d.H, nc = d.nchunks();
+    const int units = BH * nc;
+    const int slots = nsm * occ;
+
+    BwdParams p{};
+    p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
+    p.dST = a.dST; p.dS0 = a.dS0;
+    p.dv = static_cast<__nv_bfloat16*>(a.dv); p.dw = static_cast<__nv_bfloat16*>(a.dw);
+    p.states = a.states; p.tp = a.tp; p.dstates = a.dstates;
+    p.flags = a.flags; p.counter = a.flags + units;
+    if ((e = cudaMemsetAsync(a.flags, 0, ((size_t)units + 2) * sizeof(unsigned int), s)) != cudaSuccess) return e;
+
+    TraceScope trace(K_CHUNK_BWD, s);
+    // Every head's reverse pass plus at least one gradient worker resident at once: one launch.
+    if (coop && BH < slots) {
+        p.nrev = BH; p.join = 1; p.grad = 1;
+        void* args[2] = {&maps, &p};
+        e = cudaLaunchCooperativeKernel((const void*)chunk_bwd_kernel, dim3(slots), dim3(NT), args, SMEM_BYTES_ALL, s);
+        if (e == cudaSuccess) return cudaSuccess;
+        (void)cudaGetLastError();   // not launched: fall back to two launches
     }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const dim3 grid(d.nchunks(), d.B * d.H);
-    TraceScope trace(K_GRAD, s);
-    chunk_grad_kernel<<<grid, NT, cg::SMEM_BYTES, s>>>(
-        mq, mk, mv, mla, mb, mw, mdo, mdq, mdk, mdb, mdla, static_cast<__nv_bfloat16*>(a.dv),
-        static_cast<__nv_bfloat16*>(a.dw), a.states, a.tp, a.dstates, d.T, d.H);
+    BwdParams pr = p;   // reverse pass only
+    pr.nrev = BH; pr.join = 0; pr.grad = 0;
+    chunk_bwd_kernel<<<BH, NT, SMEM_BYTES_ALL, s>>>(maps, pr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    BwdParams pg = p;   // gradient units only; every flag is set when they start
+    pg.nrev = 0; pg.join = 0; pg.grad = 1;
+    chunk_bwd_kernel<<<units < slots ? units : slots, NT, SMEM_BYTES_ALL, s>>>(maps, pg);
     return cudaGetLastError();
 }
 

@@ -37,18 +37,18 @@ using namespace chunk;
 
 // ---- consumer (state pass) shared memory, bytes from a 1024-aligned base
 namespace sp {
-constexpr uint32_t QQ = 0;          // [64 x 128] q -> Qt
-constexpr uint32_t KH = 16384;      // [64 x 128] k
-constexpr uint32_t KT = 32768;      // [64 x 128] log_alpha -> Kt
-constexpr uint32_t UU = 49152;      // [64 x 128] v -> U
-constexpr uint32_t WW = 65536;      // [64 x 128] w
-constexpr uint32_t WY = 81920;      // WY image: T [64 x 64] | P [64 x 64] | Wm [64 x 128]
+constexpr uint32_t QQ = 0;          // 2 x [64 x 128] q -> Qt (by chunk parity)
+constexpr uint32_t KT = 32768;      // 2 x [64 x 128] log_alpha -> Kt (by chunk parity)
+constexpr uint32_t KH = 65536;      // [64 x 128] k
+constexpr uint32_t UU = 81920;      // [64 x 128] v -> U
+constexpr uint32_t WW = 98304;      // [64 x 128] w
+constexpr uint32_t WY = 114688;     // WY image: T [64 x 64] | P [64 x 64] | Wm [64 x 128]
 constexpr uint32_t TT = WY, PP = WY + 8192, WM = WY + 16384;
-constexpr uint32_t ST = 114688;     // [128 x 128] S^T (bf16)
-constexpr uint32_t DT = 147456;     // [128 x 64] Delta^T (bf16)
-constexpr uint32_t RED = 163840;    // fp32 [16][128] prep scan scratch
-constexpr uint32_t GC = 172032;     // fp32 gC[128]
-constexpr uint32_t BAR = 172544;    // 3 mbarriers (load, mma, unused), tmem base, abort flag
+constexpr uint32_t ST = 147456;     // [128 x 128] S^T (bf16)
+constexpr uint32_t DT = 180224;     // [128 x 64] Delta^T (bf16)
+constexpr uint32_t RED = 196608;    // fp32 [16][128] prep scan scratch
+constexpr uint32_t GC = 204800;     // fp32 gC[128]
+constexpr uint32_t BAR = 205312;    // 3 mbarriers (load, mma, unused), tmem base, abort flag
 }  // namespace sp
 // ---- producer (WY) shared memory: two input stages, then the solve scratch and the WY image
 namespace wy {
@@ -65,8 +65,8 @@ constexpr uint32_t SMEM_BYTES = 208960 + 1024;
 static_assert(sp::BAR + 64 <= wy::BAR + 64, "consumer layout fits");
 static_assert(TC_WY_BYTES == 32768, "WY image = T | P | Wm");
 
-// TMEM columns. Consumer: S^T (fp32 state), Ut^T -> Delta^T, O (M=64). Producer: [A; P], Wm (M=64).
-constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 256;
+// TMEM columns. Consumer: S^T (fp32 state), Ut^T -> Delta^T, O x 2 (M=64). Producer: [A; P], Wm (M=64).
+constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 256;   // O: two buffers of 128 columns (chunk parity)
 constexpr uint32_t TM_AP = 0, TM_W = 128;
 constexpr uint32_t TM_COLS = 512;
 
@@ -134,6 +134,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     };
     int stage = 0;
     bool pending = false;   // a prefetch into the other stage is in flight (thread 0's view)
+    long long unreleased = -1;   // unit whose WY image is written but whose flag is not yet set
     for (int u = pid; u < units; u += p.nprod, stage ^= 1) {
         const int c = u / p.BH, head = u % p.BH;
         unsigned char* base = sm + stage * wy::STAGE;
@@ -153,7 +154,10 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
             tc::mma_commit(bar_mma);
+            // the previous unit's image stores have drained during this unit's prep: set its flag now
+            if (unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
         }
+        unreleased = -1;
         wait_mma();
         extract_AP(lane_base + TM_AP, sA, PP, true, warp, lane);
         tc::tc_fence_before();
@@ -178,10 +182,11 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
 #pragma unroll
         for (int i = 0; i < (int)(TC_WY_BYTES / 16 / NT); ++i) dst[tid + NT * i] = src[tid + NT * i];
         __syncthreads();
-        if (tid == 0 && !*abort_flag) tc::flag_release(p.flags + unit, 1u);
+        unreleased = (long long)unit;
         if (*abort_flag) break;
         pending = false;
     }
+    if (tid == 0 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
     // after an abort: let the prefetch in flight land before the CTA's shared memory is released
     if (tid == 0 && pending) (void)tc::mbar_wait(&bar_in[stage ^ 1], (ph_in >> (stage ^ 1)) & 1u);
 }
@@ -189,9 +194,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
 // ------------------------------------------------------------------ consumer
 __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int cid) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    unsigned char* QQ = sm + sp::QQ;
     unsigned char* KH = sm + sp::KH;
-    unsigned char* KT = sm + sp::KT;
     unsigned char* UU = sm + sp::UU;
     unsigned char* WW = sm + sp::WW;
     unsigned char* STt = sm + sp::ST;
@@ -206,9 +209,8 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     const int T = p.T, H = p.H, nc = p.nc;
     const bool want_o = (p.o != nullptr);
 
-    const uint32_t sQQ = tc::smem_u32(QQ), sKT = tc::smem_u32(KT), sUU = tc::smem_u32(UU),
-                   sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT), sTT = tc::smem_u32(sm + sp::TT),
-                   sPP = tc::smem_u32(sm + sp::PP), sWM = tc::smem_u32(sm + sp::WM);
+    const uint32_t sUU = tc::smem_u32(UU), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
+                   sTT = tc::smem_u32(sm + sp::TT), sPP = tc::smem_u32(sm + sp::PP), sWM = tc::smem_u32(sm + sp::WM);
     constexpr uint32_t ID_M3 = tc::idesc_bf16(128, 64, true, false);
     constexpr uint32_t ID_M4 = tc::idesc_bf16(128, 64, false, false, true);
     constexpr uint32_t ID_M56 = tc::idesc_bf16(64, 128, false, false);
@@ -235,14 +237,35 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     for (int headi = cid; headi < p.BH; headi += p.ncons) {
         const size_t head = (size_t)headi;
         const int h = headi % H, b = headi / H;
+        // q and log_alpha tiles alternate between two buffers by chunk parity (read by the MMAs of
+        // chunk c while the tiles of chunk c + 1 arrive); k, v and w have one buffer each
         auto issue_loads = [&](int c) {
-            const int t0 = c * C;
+            const int t0 = c * C, par = c & 1;
             tc::mbar_arrive_expect_tx(bar_load, CONS_LOAD_BYTES);
-            tma_tile(QQ, C, 0, &m.q, b, h, t0, bar_load);
+            tma_tile(sm + sp::QQ + par * TILE_64x128, C, 0, &m.q, b, h, t0, bar_load);
+            tma_tile(sm + sp::KT + par * TILE_64x128, C, 0, &m.la, b, h, t0, bar_load);
             tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load);
-            tma_tile(KT, C, 0, &m.la, b, h, t0, bar_load);
             tma_tile(UU, C, 0, &m.v, b, h, t0, bar_load);
             tma_tile(WW, C, 0, &m.w, b, h, t0, bar_load);
+        };
+        // o rows of chunk c from its M=64 accumulator (16-byte stores)
+        auto store_o = [&](int c) {
+            const int t0 = c * C, L = min(C, T - t0);
+            const int t = m64_row(warp, lane);
+            const uint32_t ob = lane_base + TM_O + 128 * (c & 1);
+            float v[32];
+#pragma unroll
+            for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
+                tc::tmem_ld32(ob + c0, v);
+                tc::tmem_wait_ld();
+                if (lane < 16 && t < L) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + tok_off(b, t0 + t, h, T, H, D) + c0);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        dst[g] = make_uint4(tc::pack_bf16x2(v[8 * g], v[8 * g + 1]), tc::pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
+                                            tc::pack_bf16x2(v[8 * g + 4], v[8 * g + 5]), tc::pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
+                }
+            }
         };
         if (tid == 0) {
             issue_loads(0);
@@ -272,9 +295,13 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             tc::bulk_commit();
         }
 
-        for (int c = 0; c < nc; ++c) {
-            const int t0 = c * C;
-            const int L = min(C, T - t0);
+        int c = 0;
+        for (; c < nc; ++c) {
+            const int par = c & 1;
+            unsigned char* QQ = sm + sp::QQ + par * TILE_64x128;
+            unsigned char* KT = sm + sp::KT + par * TILE_64x128;
+            const uint32_t sQQ = tc::smem_u32(QQ), sKT = tc::smem_u32(KT);
+            const uint32_t tm_o = tmem + TM_O + 128 * par;
             if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
             ph_load ^= 1;
 
@@ -283,21 +310,27 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             tc::cp_async_wait_all();   // this chunk's WY image
             sync_for_mma();
 
-            // ---- M3: Delta^T := U^T T^T ;  M4: Delta^T -= S^T Wm^T ;  M5: O = Qt S
+            // ---- M3: Delta^T := U^T T^T ;  M4: Delta^T -= S^T Wm^T  (commit) ;  M5: O = Qt S
             if (tid == 0) {
                 tc::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M3, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWM, C, 0, kk), ID_M4, 1);
-                    if (want_o)
-                        tc::mma_bf16(tmem + TM_O, tc::desc_k(sQQ, C, 0, kk), tc::desc_k(sST, D, 0, kk), ID_M56, kk > 0);
-                }
                 tc::mma_commit(bar_mma);
+                if (want_o) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_bf16(tm_o, tc::desc_k(sQQ, C, 0, kk), tc::desc_k(sST, D, 0, kk), ID_M56, kk > 0);
+                }
+                if (c + 1 < nc) wait_wy(head, c + 1);   // overlaps the MMAs
             }
+            if (want_o && c > 0) store_o(c - 1);      // previous chunk's output, in the MMAs' shadow
             wait_mma();
+            // k, v, w and the other parity's q, log_alpha tiles are free: prefetch the next chunk
+            if (tid == 0 && c + 1 < nc) issue_loads(c + 1);
             tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
             sync_for_mma();
 
@@ -307,32 +340,12 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     if (want_o)
-                        tc::mma_bf16(tmem + TM_O, tc::desc_k(sPP, C, 0, kk), tc::desc_k(sDT, D, 0, kk), ID_M56, 1);
+                        tc::mma_bf16(tm_o, tc::desc_k(sPP, C, 0, kk), tc::desc_k(sDT, D, 0, kk), ID_M56, 1);
                     tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sKT, C, 0, kk), ID_M7, 1);
                 }
                 tc::mma_commit(bar_mma);
-                if (c + 1 < nc) wait_wy(head, c + 1);   // overlaps the MMAs
             }
             wait_mma();
-            // every shared-memory input of this chunk is consumed: prefetch the next chunk
-            if (tid == 0 && c + 1 < nc) issue_loads(c + 1);
-
-            if (want_o) {   // o rows t from the M=64 accumulator: 16-byte stores
-                const int t = m64_row(warp, lane);
-                float v[32];
-#pragma unroll
-                for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
-                    tc::tmem_ld32(lane_base + TM_O + c0, v);
-                    tc::tmem_wait_ld();
-                    if (lane < 16 && t < L) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.o + tok_off(b, t0 + t, h, T, H, D) + c0);
-#pragma unroll
-                        for (int g = 0; g < 4; ++g)
-                            dst[g] = make_uint4(tc::pack_bf16x2(v[8 * g], v[8 * g + 1]), tc::pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
-                                                tc::pack_bf16x2(v[8 * g + 4], v[8 * g + 5]), tc::pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
-                    }
-                }
-            }
             // S'^T = Z^T Diag(gC): scale the fp32 state, keep a bf16 copy for the next chunk
             if (p.states && tid == 0) tc::bulk_wait_read();
             __syncthreads();   // also orders thread 0's flag acquire before the image copy
@@ -363,6 +376,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 break;
             }
         }
+        if (want_o && c == nc) store_o(nc - 1);
 
         // final state (fp32): ST[i][j] from S^T (lane j)
         if (p.ST) {

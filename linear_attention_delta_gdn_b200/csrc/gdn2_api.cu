@@ -71,7 +71,8 @@ size_t tc_flags_offset(const Dims& d, bool with_states) {
 }
 
 size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
-    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk)) return tc_units(d) * TC_STATE_BYTES;
+    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk))   // dZ images, then ready flags, work counter, abort word
+        return tc_units(d) * TC_STATE_BYTES + align256((tc_units(d) + 2) * sizeof(unsigned int));
     const size_t seg = (size_t)d.B * d.H * d.chunk * d.Dk * d.Dv * sizeof(float);
     const size_t del = (size_t)d.B * d.H * d.chunk * d.Dv * sizeof(float);
     return align256(seg) + align256(del);
@@ -215,6 +216,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
         a.states = wsb;
         a.tp = wsb + tc_tp_offset(d);
         a.dstates = extra;
+        a.flags = reinterpret_cast<unsigned int*>(extra + tc_units(d) * TC_STATE_BYTES);
         return cuda_status(chunk_bwd_launch(a, s), "gdn2_bwd (tensor-core path)");
     }
 

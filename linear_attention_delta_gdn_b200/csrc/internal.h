@@ -55,11 +55,12 @@ struct ChunkBwdArgs {
     const unsigned char* states;  // [B,H,NC] chunk-start state images
     const unsigned char* tp;      // [B,H,NC] WY images (T | P | Wm) of every chunk
     unsigned char* dstates;       // [B,H,NC] images of Diag(gC) dL/dS' per chunk (scratch)
+    unsigned int* flags;          // [B,H,NC] ready flags, then work counter and abort word (scratch)
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 
 // Kernels of the library, for gdn2_trace_read().
-enum KernelId { K_CHUNK_FWD = 0, K_REVERSE, K_GRAD, K_REC_FWD, K_REC_BWD, K_DECODE, KERNEL_COUNT };
+enum KernelId { K_CHUNK_FWD = 0, K_CHUNK_BWD, K_REC_FWD, K_REC_BWD, K_DECODE, KERNEL_COUNT };
 
 // Brackets one kernel launch with CUDA events on its stream while tracing is on.
 class TraceScope {
