@@ -77,32 +77,30 @@ struct Phases {
 // ====================================================================== reverse state pass
 
 namespace rs {
-constexpr uint32_t OFF_QE = 0;           // rows 0..63: b -> Et, rows 64..127: q -> Qt
+constexpr uint32_t OFF_QQ = 0;           // q -> Qt (64 rows)
 constexpr uint32_t OFF_KH = 32768;       // k
 constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
 constexpr uint32_t OFF_DO = 65536;       // dout
-constexpr uint32_t OFF_WW = 81920;       // Wm
+constexpr uint32_t OFF_WW = 81920;       // Wm (from the forward's WY image)
 constexpr uint32_t OFF_ST = 98304;       // dZ^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16)
-constexpr uint32_t OFF_TT = 147456;      // T (bf16, from the forward)
-constexpr uint32_t OFF_PP = 155648;      // P (bf16, from the forward)
+constexpr uint32_t OFF_PP = 155648;      // P (bf16, from the forward's WY image)
 constexpr uint32_t OFF_RED = 163840;     // prep scan scratch (8 KB)
 constexpr uint32_t OFF_GC = 172032;
-constexpr uint32_t TM_S = 0, TM_D = 128, TM_W = 192;
-constexpr uint32_t LOAD_BYTES = 5 * 64 * 128 * 2 + 2 * TILE_C;
+constexpr uint32_t TM_S = 0, TM_D = 128;
+constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 64 * 128 * 2;
 }  // namespace rs
 
 __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi,
                             Phases& ph) {
     using namespace rs;
-    unsigned char* QE = sm + OFF_QE;
+    unsigned char* QQ = sm + OFF_QQ;
     unsigned char* KH = sm + OFF_KH;
     unsigned char* KT = sm + OFF_KT;
     unsigned char* DO = sm + OFF_DO;
     unsigned char* WW = sm + OFF_WW;
     unsigned char* STt = sm + OFF_ST;
     unsigned char* DT = sm + OFF_DT;
-    unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
     float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
     float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
@@ -120,14 +118,13 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     auto issue_loads = [&](int c) {
         const int t0 = c * C;
         tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-        tma_tile(QE, 2 * C, 0, &m.b, b, h, t0, bar_load);
-        tma_tile(QE, 2 * C, C, &m.q, b, h, t0, bar_load);
+        tma_tile(QQ, C, 0, &m.q, b, h, t0, bar_load);
         tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load);
         tma_tile(KT, C, 0, &m.la, b, h, t0, bar_load);
         tma_tile(DO, C, 0, &m.dout, b, h, t0, bar_load);
-        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;
-        tc::bulk_load(TT, src, TILE_C, bar_load);
+        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
         tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
+        tc::bulk_load(WW, src + 2 * TILE_C, 64 * 128 * 2, bar_load);
     };
     if (tid == 0) issue_loads(nc - 1);
 
@@ -146,10 +143,8 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     __syncthreads();
     tc::tc_fence_after();
 
-    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sDO = tc::smem_u32(DO),
-                   sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
-                   sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
-    constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
+    const uint32_t sQQ = tc::smem_u32(QQ), sKT = tc::smem_u32(KT), sDO = tc::smem_u32(DO),
+                   sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT), sPP = tc::smem_u32(PP);
     constexpr uint32_t ID_N1a = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_N1b = tc::idesc_bf16(128, 64, true, true);
     constexpr uint32_t ID_N2a = tc::idesc_bf16(128, 128, true, true);
@@ -171,7 +166,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         if (!tc::mbar_wait(bar_load, ph.load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
         ph.load ^= 1;
 
-        gate_prep(QE, KH, KT, nullptr, nullptr, sGC, sRed, tid, true, false);
+        gate_prep_state<false>(QQ, KH, KT, nullptr, nullptr, sGC, sRed, tid);   // Qt, Kt, gC
         __syncthreads();
         // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
         {
@@ -191,12 +186,9 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         }
         sync_for_mma();
 
-        // Wm = T Et (M=64) ;  dDelta^T = dZ^T Kt^T + dO^T P
+        // dDelta^T = dZ^T Kt^T + dO^T P
         if (tid == 0) {
             tc::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), ID_M2, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_N1a, kk > 0);
@@ -216,7 +208,6 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         }
         unreleased = c;
         wait_mma();
-        tmem_m64_to_tile(lane_base + TM_W, WW, warp, lane);    // Wm rows
         tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
 
@@ -225,7 +216,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQE, 2 * C, C, kk), ID_N2a, 1);
+                tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQQ, C, 0, kk), ID_N2a, 1);
                 tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sWW, C, 0, kk), ID_N2b, 1);
             }
             tc::mma_commit(bar_mma);
@@ -285,7 +276,7 @@ constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
     TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,
     TM_GV = 448;                   // G[t] per key channel (cumulative log-decay)
-constexpr uint32_t LOAD_BYTES = 7 * 64 * 128 * 2 + (uint32_t)TC_STATE_BYTES + 2 * TILE_C;   // dZ^T: cp.async
+constexpr uint32_t LOAD_BYTES = 8 * 64 * 128 * 2 + (uint32_t)TC_STATE_BYTES + 2 * TILE_C;   // dZ^T: cp.async
 }  // namespace cg
 
 // Gradients of chunk c of head `headi`; returns false if a bounded wait gave up.
@@ -332,9 +323,10 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tma_tile(WW, C, 0, mw, b, h, t0, bar_load);
         tma_tile(DO, C, 0, mdo, b, h, t0, bar_load);
         tc::bulk_load(STt, p.states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
-        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;
+        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
         tc::bulk_load(TT, src, TILE_C, bar_load);
         tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
+        tc::bulk_load(DDT, src + 2 * TILE_C, 64 * 128 * 2, bar_load);   // Wm rows (DDT is free until dDelta^T)
         // dZ^T of this chunk comes from the reverse pass: wait for its flag
         if (!tc::flag_wait(p.flags + head * nc + c, 1u)) {
             ok = false;
@@ -376,16 +368,13 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     gate_prep_cols(QE, KH, KT, UU, WW, sGC, tid, lane_base + TM_GV);
     sync_for_mma();
 
-    // ---- Wm = T Et (M=64) ; Ut^T = U^T T^T
+    // ---- Ut^T = U^T T^T
     if (tid == 0) {
         tc::tc_fence_after();
-        constexpr uint32_t id_w = tc::idesc_bf16(64, 128, false, true);
         constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), id_w, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)
             tc::mma_bf16(tmem + TM_D, tc::desc_mn(sKH, C, 0, kk), tc::desc_k(sTT, C, 0, kk), id_u, kk > 0);
-        }
         tc::mma_commit(bar_mma);
     }
     wait_mma();
@@ -393,8 +382,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mbar_arrive_expect_tx(bar_k, 64 * 128 * 2);
         tma_tile(KH, C, 0, mk, b, h, t0, bar_k);
     }
-    tmem_m64_to_tile(lane_base + TM_W, DDT, warp, lane);      // Wm rows (DDT is free until dDelta^T)
-    sync_for_mma();
+    tc::tc_fence_before();
+    __syncthreads();
 
     // ---- Delta^T = Ut^T - S^T Wm^T ;  dDelta^T = dZ^T Kt^T + dO^T P
     if (tid == 0) {

@@ -208,10 +208,11 @@ __device__ __forceinline__ void gate_prep(unsigned char* QE, const unsigned char
     }
 }
 
-// Gate preparation of the state pass (no erase factor): same thread layout as gate_prep;
+// Gate preparation of the state passes (no erase factor): same thread layout as gate_prep;
 //   reads  log_alpha (KT), k (KH), q (QQ, 64 rows), v (UU), w (WW)
-//   writes Qt = g*q -> QQ, Kt = k/g -> KT, U = w*v -> UU, gC.
+//   writes Qt = g*q -> QQ, Kt = k/g -> KT, U = w*v -> UU (kU), gC.
 // Contains one __syncthreads.
+template <bool kU = true>
 __device__ __forceinline__ void gate_prep_state(unsigned char* QQ, const unsigned char* KH, unsigned char* KT,
                                                 unsigned char* UU, const unsigned char* WW, float* gC_out,
                                                 float* red, int tid) {
@@ -225,19 +226,21 @@ __device__ __forceinline__ void gate_prep_state(unsigned char* QQ, const unsigne
         float kk[8], qq[8], vv[8], ww[8];
         tc::ld_row8(KH, C, row, cg, kk);
         tc::ld_row8(QQ, C, row, cg, qq);
-        tc::ld_row8(UU, C, row, cg, vv);
-        tc::ld_row8(WW, C, row, cg, ww);
+        if (kU) {
+            tc::ld_row8(UU, C, row, cg, vv);
+            tc::ld_row8(WW, C, row, cg, ww);
+        }
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float Gv = pre[c] + G[u][c];
             const float g = fast_exp(Gv), ig = fast_exp(-Gv);
             kk[c] *= ig;
             qq[c] *= g;
-            vv[c] *= ww[c];
+            if (kU) vv[c] *= ww[c];
         }
         tc::st_row8(KT, C, row, cg, kk);
         tc::st_row8(QQ, C, row, cg, qq);
-        tc::st_row8(UU, C, row, cg, vv);
+        if (kU) tc::st_row8(UU, C, row, cg, vv);
     }
 }
 

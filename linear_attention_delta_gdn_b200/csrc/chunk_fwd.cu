@@ -154,9 +154,10 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
             tc::mma_commit(bar_mma);
-            // the previous unit's image stores have drained during this unit's prep: set its flag now
-            if (unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
         }
+        // the previous unit's image stores have drained during this unit's prep: set its flag now,
+        // from a thread outside the MMA-issuing warp, while M1 runs
+        if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
         unreleased = -1;
         wait_mma();
         extract_AP(lane_base + TM_AP, sA, PP, true, warp, lane);
@@ -186,7 +187,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         if (*abort_flag) break;
         pending = false;
     }
-    if (tid == 0 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
+    if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
     // after an abort: let the prefetch in flight land before the CTA's shared memory is released
     if (tid == 0 && pending) (void)tc::mbar_wait(&bar_in[stage ^ 1], (ph_in >> (stage ^ 1)) & 1u);
 }
