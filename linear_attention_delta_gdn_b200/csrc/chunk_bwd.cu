@@ -77,28 +77,30 @@ struct Phases {
 // ====================================================================== reverse state pass
 
 namespace rs {
-constexpr uint32_t OFF_QQ = 0;           // q -> Qt (64 rows)
+// q, log_alpha, dout and Wm alternate between two buffers by chunk parity, so the next chunk's
+// tiles can land while this chunk's MMAs read the current ones; k and P have one buffer each.
+constexpr uint32_t OFF_QQ = 0;           // 2 x q -> Qt (64 rows), at +0 / +16384
 constexpr uint32_t OFF_KH = 32768;       // k
-constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
-constexpr uint32_t OFF_DO = 65536;       // dout
-constexpr uint32_t OFF_WW = 81920;       // Wm (from the forward's WY image)
+constexpr uint32_t OFF_KT0 = 49152;      // log_alpha -> Kt (even chunks)
+constexpr uint32_t OFF_DO0 = 65536;      // dout (even chunks)
+constexpr uint32_t OFF_WW0 = 81920;      // Wm from the forward's WY image (even chunks)
 constexpr uint32_t OFF_ST = 98304;       // dZ^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16)
-constexpr uint32_t OFF_PP = 155648;      // P (bf16, from the forward's WY image)
-constexpr uint32_t OFF_RED = 163840;     // prep scan scratch (8 KB)
-constexpr uint32_t OFF_GC = 172032;
+constexpr uint32_t OFF_PP = 147456;      // P from the forward's WY image
+constexpr uint32_t OFF_RED = 155648;     // prep scan scratch (8 KB)
+constexpr uint32_t OFF_DO1 = 163840;     // dout (odd chunks)
+constexpr uint32_t OFF_WW1 = 180224;     // Wm (odd chunks)
+constexpr uint32_t OFF_KT1 = 196608;     // log_alpha -> Kt (odd chunks)
+constexpr uint32_t OFF_GC = 212992;
 constexpr uint32_t TM_S = 0, TM_D = 128;
-constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 64 * 128 * 2;
+constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 64 * 128 * 2;   // q, log_alpha, dout, k, P, Wm
 }  // namespace rs
+static_assert(rs::OFF_GC + 512 <= OFF_BARS, "reverse-pass layout lies below the barrier block");
 
 __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi,
                             Phases& ph) {
     using namespace rs;
-    unsigned char* QQ = sm + OFF_QQ;
     unsigned char* KH = sm + OFF_KH;
-    unsigned char* KT = sm + OFF_KT;
-    unsigned char* DO = sm + OFF_DO;
-    unsigned char* WW = sm + OFF_WW;
     unsigned char* STt = sm + OFF_ST;
     unsigned char* DT = sm + OFF_DT;
     unsigned char* PP = sm + OFF_PP;
@@ -107,6 +109,10 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_load + 1;
     int* abort_flag = reinterpret_cast<int*>(sm + OFF_BARS + 36);
+    auto QQ = [&](int c) { return sm + OFF_QQ + (c & 1) * TILE_64x128; };
+    auto KT = [&](int c) { return sm + ((c & 1) ? OFF_KT1 : OFF_KT0); };
+    auto DO = [&](int c) { return sm + ((c & 1) ? OFF_DO1 : OFF_DO0); };
+    auto WW = [&](int c) { return sm + ((c & 1) ? OFF_WW1 : OFF_WW0); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = headi % p.H, b = headi / p.H;
@@ -115,18 +121,24 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
 
-    auto issue_loads = [&](int c) {
+    // chunk c's tiles arrive on one barrier phase, issued in three groups as their buffers free up
+    auto issue_first = [&](int c) {   // q, log_alpha, dout, Wm: buffers of this parity are free
         const int t0 = c * C;
         tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-        tma_tile(QQ, C, 0, &m.q, b, h, t0, bar_load);
-        tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load);
-        tma_tile(KT, C, 0, &m.la, b, h, t0, bar_load);
-        tma_tile(DO, C, 0, &m.dout, b, h, t0, bar_load);
-        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
-        tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
-        tc::bulk_load(WW, src + 2 * TILE_C, 64 * 128 * 2, bar_load);
+        tma_tile(QQ(c), C, 0, &m.q, b, h, t0, bar_load);
+        tma_tile(KT(c), C, 0, &m.la, b, h, t0, bar_load);
+        tma_tile(DO(c), C, 0, &m.dout, b, h, t0, bar_load);
+        tc::bulk_load(WW(c), p.tp + (head * nc + c) * TC_WY_BYTES + 2 * TILE_C, 64 * 128 * 2, bar_load);
     };
-    if (tid == 0) issue_loads(nc - 1);
+    auto issue_k = [&](int c) { tma_tile(KH, C, 0, &m.k, b, h, c * C, bar_load); };   // after the prep
+    auto issue_p = [&](int c) {   // after the MMAs that read P
+        tc::bulk_load(PP, p.tp + (head * nc + c) * TC_WY_BYTES + TILE_C, TILE_C, bar_load);
+    };
+    if (tid == 0) {
+        issue_first(nc - 1);
+        issue_k(nc - 1);
+        issue_p(nc - 1);
+    }
 
     {   // dS_{NC}^T = dST^T (or zero): lane j holds column j of dST
         const int j = jrow;
@@ -143,8 +155,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     __syncthreads();
     tc::tc_fence_after();
 
-    const uint32_t sQQ = tc::smem_u32(QQ), sKT = tc::smem_u32(KT), sDO = tc::smem_u32(DO),
-                   sWW = tc::smem_u32(WW), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT), sPP = tc::smem_u32(PP);
+    const uint32_t sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT), sPP = tc::smem_u32(PP);
     constexpr uint32_t ID_N1a = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_N1b = tc::idesc_bf16(128, 64, true, true);
     constexpr uint32_t ID_N2a = tc::idesc_bf16(128, 128, true, true);
@@ -163,11 +174,17 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
 
     int unreleased = -1;   // chunk whose dZ image is written but whose flag is not yet set
     for (int c = nc - 1; c >= 0; --c) {
+        const uint32_t sQQ = tc::smem_u32(QQ(c)), sKT = tc::smem_u32(KT(c)), sDO = tc::smem_u32(DO(c)),
+                       sWW = tc::smem_u32(WW(c));
         if (!tc::mbar_wait(bar_load, ph.load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
         ph.load ^= 1;
+        // the other parity's buffers were last read by chunk c + 1, whose MMAs are complete
+        if (tid == 0 && c > 0) issue_first(c - 1);
 
-        gate_prep_state<false>(QQ, KH, KT, nullptr, nullptr, sGC, sRed, tid);   // Qt, Kt, gC
+        gate_prep_state<false>(QQ(c), KH, KT(c), nullptr, nullptr, sGC, sRed, tid);   // Qt, Kt, gC
+        tc::fence_async_smem();   // the prep's reads of k precede the TMA that overwrites it
         __syncthreads();
+        if (tid == 0 && c > 0) issue_k(c - 1);
         // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
         {
             const int j = jrow;
@@ -186,7 +203,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         }
         sync_for_mma();
 
-        // dDelta^T = dZ^T Kt^T + dO^T P
+        // dDelta^T = dZ^T Kt^T + dO^T P (commit) ;  dS^T = dZ^T + dO^T Qt (continues below)
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
@@ -196,6 +213,9 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16(tmem + TM_D, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), ID_N1b, 1);
             tc::mma_commit(bar_mma);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQQ, C, 0, kk), ID_N2a, 1);
         }
         // the previous chunk's dZ image stores have drained: publish it while the MMAs run
         if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
@@ -208,21 +228,19 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         }
         unreleased = c;
         wait_mma();
+        if (tid == 0 && c > 0) issue_p(c - 1);
         tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
 
-        // dS^T = dZ^T + dO^T Qt - dDelta^T Wm
+        // dS^T -= dDelta^T Wm
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQQ, C, 0, kk), ID_N2a, 1);
+            for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16(tmem + TM_S, tc::desc_k(sDT, D, 0, kk), tc::desc_mn(sWW, C, 0, kk), ID_N2b, 1);
-            }
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        if (tid == 0 && c > 0) issue_loads(c - 1);
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
