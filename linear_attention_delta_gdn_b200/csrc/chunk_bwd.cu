@@ -45,6 +45,127 @@ using namespace chunk;
 
 __device__ unsigned int g_bwd_error;
 
+// The backward runs 512 threads per CTA: 16 warps, four per TMEM lane quarter (warp w reads lanes
+// 32 (w % 4) .. + 31; the four warps of a quarter, part = w / 4, split the columns of a read-out).
+constexpr int BT = 512;
+constexpr int BPARTS = BT / 128;
+
+// Copy a [128 lanes x NCOL] fp32 accumulator into a bf16 row tile of 128 rows (row = lane); each of
+// the four warps of a lane quarter takes NCOL / 4 columns.
+template <int NCOL>
+__device__ __forceinline__ void tmem_rows_to_tile(uint32_t lane_base_col, unsigned char* dst, int warp, int lane) {
+    static_assert(NCOL == 64, "16 columns per warp");
+    const int row = 32 * tm_quarter(warp) + lane, c0 = (NCOL / BPARTS) * tm_part(warp);
+    float v[16];
+    tc::tmem_ld16(lane_base_col + c0, v);
+    tc::tmem_wait_ld();
+    tc::st_row8(dst, 128, row, (c0 >> 3), v);
+    tc::st_row8(dst, 128, row, (c0 >> 3) + 1, v + 8);
+}
+
+// Reverse-pass prep: Qt = g*q (QQ), Kt = k/g (KT over log_alpha), gC, with g = exp(G) and G the
+// inclusive in-chunk cumsum of log_alpha. Thread = (4-token block tb = tid / 32, 4-channel group
+// cg = tid % 32), 8-byte shared-memory accesses; block totals are exchanged through red
+// (fp32 [16][128]). Contains one __syncthreads.
+__device__ __forceinline__ void prep_qk4(unsigned char* QQ, const unsigned char* KH, unsigned char* KT,
+                                         float* gC_out, float* red, int tid) {
+    const int cg = tid & 31, tb = tid >> 5;
+    float G[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        tc::ld_row4(KT, C, 4 * tb + u, cg, G[u]);
+        if (u > 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) G[u][c] += G[u - 1][c];
+        }
+    }
+    *reinterpret_cast<float4*>(red + tb * 128 + 4 * cg) = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+    __syncthreads();
+    float pre[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int q = 0; q < tb; ++q) {
+        const float4 x = *reinterpret_cast<const float4*>(red + q * 128 + 4 * cg);
+        pre[0] += x.x; pre[1] += x.y; pre[2] += x.z; pre[3] += x.w;
+    }
+    if (tb == C / 4 - 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) gC_out[4 * cg + c] = fast_exp(pre[c] + G[3][c]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int row = 4 * tb + u;
+        float kk[4], qq[4];
+        tc::ld_row4(KH, C, row, cg, kk);
+        tc::ld_row4(QQ, C, row, cg, qq);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float Gv = pre[c] + G[u][c];
+            kk[c] *= fast_exp(-Gv);
+            qq[c] *= fast_exp(Gv);
+        }
+        tc::st_row4(KT, C, row, cg, kk);
+        tc::st_row4(QQ, C, row, cg, qq);
+    }
+}
+
+// Gradient-unit prep, thread = (key/value channel i = tid % 128, token quarter qt = tid / 128: tokens
+// 16 qt .. 16 qt + 15):
+//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
+//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT, U = w*v -> KH (over k);
+//   G[t][i] goes to TMEM at tmem_g (lane i, column t). Quarter sums of log_alpha are exchanged
+//   through qsum (fp32 [4][128]). Contains one __syncthreads.
+__device__ __forceinline__ void grad_prep(unsigned char* QE, unsigned char* KH, unsigned char* KT,
+                                          const unsigned char* UU, const unsigned char* WW, float* qsum,
+                                          int tid, uint32_t tmem_g) {
+    const int i = tid & 127, qt = tid >> 7;
+    const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
+    const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
+    const uint32_t chunk = (uint32_t)((i & 63) >> 3);
+    float la[16];
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const uint32_t t = (uint32_t)(16 * qt + u);
+        la[u] = tc::ld_bf16(KT, col64 + t * 128 + ((chunk ^ (t & 7)) << 4));
+        if (u & 1) s1 += la[u]; else s0 += la[u];
+    }
+    qsum[qt * 128 + i] = s0 + s1;
+    __syncthreads();   // also: every log_alpha is read before Kt overwrites it
+    float G = 0.f;
+#pragma unroll 1
+    for (int q = 0; q < qt; ++q) G += qsum[q * 128 + i];
+    float gvals[16];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float kk[8], bb[8], qq[8], vv[8], ww[8];
+        uint32_t o64[8], o128[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t t = (uint32_t)(16 * qt + 8 * half + u);
+            const uint32_t sw = t * 128 + ((chunk ^ (t & 7)) << 4);
+            o64[u] = col64 + sw;
+            o128[u] = col128 + sw;
+            kk[u] = tc::ld_bf16(KH, o64[u]);
+            bb[u] = tc::ld_bf16(QE, o128[u]);
+            qq[u] = tc::ld_bf16(QE, o128[u] + C * 128);
+            vv[u] = tc::ld_bf16(UU, o64[u]);
+            ww[u] = tc::ld_bf16(WW, o64[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            G += la[8 * half + u];
+            gvals[8 * half + u] = G;
+            const float g = fast_exp(G), ig = fast_exp(-G);
+            tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);          // Et
+            tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);        // Qt
+            tc::st_bf16(KT, o64[u], kk[u] * ig);                  // Kt
+            tc::st_bf16(KH, o64[u], ww[u] * vv[u]);               // U
+        }
+    }
+    tc::tmem_st16(tmem_g + 16 * qt, gvals);
+    tc::tmem_wait_st();
+}
+
 constexpr uint32_t TILE_C = 64 * 64 * 2;   // bytes of a 64 x 64 bf16 tile
 
 // Barrier block shared by both kinds of work (above every tile of either layout):
@@ -119,7 +240,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     const size_t head = (size_t)headi;
     const int nc = p.nc;
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
-    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
+    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 32 * tm_part(warp);      // lane row, column quarter
 
     // chunk c's tiles arrive on one barrier phase, issued in three groups as their buffers free up
     auto issue_first = [&](int c) {   // q, log_alpha, dout, Wm: buffers of this parity are free
@@ -144,7 +265,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         const int j = jrow;
         float v[32];
 #pragma unroll 1
-        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
+        for (int i0 = cpart; i0 < cpart + 32; i0 += 32) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] = p.dST ? p.dST[(head * D + i0 + u) * D + j] : 0.f;
             tc::tmem_st32(lane_base + TM_S + i0, v);
@@ -181,7 +302,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         // the other parity's buffers were last read by chunk c + 1, whose MMAs are complete
         if (tid == 0 && c > 0) issue_first(c - 1);
 
-        gate_prep_state<false>(QQ(c), KH, KT(c), nullptr, nullptr, sGC, sRed, tid);   // Qt, Kt, gC
+        prep_qk4(QQ(c), KH, KT(c), sGC, sRed, tid);   // Qt, Kt, gC
         tc::fence_async_smem();   // the prep's reads of k precede the TMA that overwrites it
         __syncthreads();
         if (tid == 0 && c > 0) issue_k(c - 1);
@@ -190,7 +311,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             const int j = jrow;
             float v[32];
 #pragma unroll 1
-            for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
+            for (int i0 = cpart; i0 < cpart + 32; i0 += 32) {
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
                 tc::tmem_wait_ld();
 #pragma unroll
@@ -224,12 +345,12 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             uint4* dst = reinterpret_cast<uint4*>(p.dstates + (head * nc + c) * TC_STATE_BYTES);
             const uint4* src = reinterpret_cast<const uint4*>(STt);
 #pragma unroll
-            for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / NT); ++i) dst[tid + NT * i] = src[tid + NT * i];
+            for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i) dst[tid + BT * i] = src[tid + BT * i];
         }
         unreleased = c;
         wait_mma();
         if (tid == 0 && c > 0) issue_p(c - 1);
-        tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
+        tmem_rows_to_tile<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
 
         // dS^T -= dDelta^T Wm
@@ -258,7 +379,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         const int j = jrow;
         float v[32];
 #pragma unroll 1
-        for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
+        for (int i0 = cpart; i0 < cpart + 32; i0 += 32) {
             tc::tmem_ld32(lane_base + TM_S + i0, v);
             tc::tmem_wait_ld();
 #pragma unroll
@@ -285,7 +406,6 @@ constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64], later staged dk
 constexpr uint32_t OFF_DDT = 196608;     // Wm rows, then dDelta^T [128 x 64], later staged db
 constexpr uint32_t OFF_TT = 212992;      // T, later dA^T [64 x 64]
 constexpr uint32_t OFF_PP = 221184;      // P, later dP^T [64 x 64]
-constexpr uint32_t OFF_GC = 229376;
 // TMEM columns (M=64 accumulators use lanes 0-15 of each 32-lane quarter)
 constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_W = 64,                     // Wm (M=64, 128 columns), later dA^T (M=64, 64 columns)
@@ -313,7 +433,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     unsigned char* DDT = sm + OFF_DDT;
     unsigned char* TT = sm + OFF_TT;
     unsigned char* PP = sm + OFF_PP;
-    float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_load + 1;
     uint64_t* bar_k = bar_load + 2;
@@ -356,12 +475,12 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     {
         const unsigned char* src = p.dstates + (head * nc + c) * TC_STATE_BYTES;
 #pragma unroll
-        for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / NT); ++i)
-            tc::cp_async16_cg(DS + 16 * (tid + NT * i), src + 16 * (tid + NT * i));
+        for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i)
+            tc::cp_async16_cg(DS + 16 * (tid + BT * i), src + 16 * (tid + BT * i));
         tc::cp_async_commit();
     }
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
-    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
+    const int jrow = 32 * tm_quarter(warp) + lane, cpart = 32 * tm_part(warp);      // lane row, column quarter
     (void)jrow;
     ok = tc::mbar_wait(bar_load, ph.load) && ok;
     ph.load ^= 1;
@@ -383,7 +502,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
     // ---- factors (U over k, G kept in TMEM)
-    gate_prep_cols(QE, KH, KT, UU, WW, sGC, tid, lane_base + TM_GV);
+    grad_prep(QE, KH, KT, UU, WW, reinterpret_cast<float*>(DT), tid, lane_base + TM_GV);   // DT: scratch
     sync_for_mma();
 
     // ---- Ut^T = U^T T^T
@@ -420,8 +539,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);     // Delta^T [j][t]
-    tmem_to_tile_rows<64>(lane_base + TM_DD, DDT, warp, lane);   // dDelta^T [j][t]
+    tmem_rows_to_tile<64>(lane_base + TM_D, DT, warp, lane);     // Delta^T [j][t]
+    tmem_rows_to_tile<64>(lane_base + TM_DD, DDT, warp, lane);   // dDelta^T [j][t]
     sync_for_mma();
 
     // ---- dU = T^T dDelta (M=64)
@@ -439,7 +558,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         const bool row_ok = lane < 16 && t < L;
         float v[32];
 #pragma unroll 1
-        for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
+        for (int c0 = cpart; c0 < cpart + 32; c0 += 32) {
             tc::tmem_ld32(lane_base + TM_DU + c0, v);
             tc::tmem_wait_ld();
             if (lane < 16) {
@@ -485,24 +604,24 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    {   // M=64 accumulators: rows s = 16 q + lane (lanes < 16); the warps of a quarter take 32 columns each
-        const int s_ = m64_row(warp, lane), c0 = 32 * tm_part(warp);
-        float v[32];
-        tc::tmem_ld32(lane_base + TM_AP + c0, v);
+    {   // M=64 accumulators: rows s = 16 q + lane (lanes < 16); the warps of a quarter take 16 columns each
+        const int s_ = m64_row(warp, lane), c0 = 16 * tm_part(warp);
+        float v[16];
+        tc::tmem_ld16(lane_base + TM_AP + c0, v);
         tc::tmem_wait_ld();
         if (lane < 16) {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] = (s_ <= c0 + u) ? v[u] : 0.f;   // dP[t][s], t >= s
+            for (int u = 0; u < 16; ++u) v[u] = (s_ <= c0 + u) ? v[u] : 0.f;   // dP[t][s], t >= s
 #pragma unroll
-            for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, s_, (c0 >> 3) + g, v + 8 * g);
+            for (int g = 0; g < 2; ++g) tc::st_row8(PP, C, s_, (c0 >> 3) + g, v + 8 * g);
         }
-        tc::tmem_ld32(lane_base + TM_W + c0, v);
+        tc::tmem_ld16(lane_base + TM_W + c0, v);
         tc::tmem_wait_ld();
         if (lane < 16) {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] = (s_ < c0 + u) ? v[u] : 0.f;    // dA[t][s], t > s
+            for (int u = 0; u < 16; ++u) v[u] = (s_ < c0 + u) ? v[u] : 0.f;    // dA[t][s], t > s
 #pragma unroll
-            for (int g = 0; g < 4; ++g) tc::st_row8(TT, C, s_, (c0 >> 3) + g, v + 8 * g);
+            for (int g = 0; g < 2; ++g) tc::st_row8(TT, C, s_, (c0 >> 3) + g, v + 8 * g);
         }
     }
     sync_for_mma();
@@ -532,13 +651,14 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mma_commit(bar_mma);
     }
 
-    // rowsum(dZ * S) for key channel i, this half's value channels (both images hold row j = value channel)
-    const int i = tid & 127, hf = tid >> 7;
+    // rowsum(dZ * S) for key channel i over this quarter's value channels (both images hold row j =
+    // value channel)
+    const int i = tid & 127, qt = tid >> 7;
     float Epart = 0.f;
     {
         float e2 = 0.f;
 #pragma unroll 8
-        for (int j = 64 * hf; j < 64 * hf + 64; j += 2) {
+        for (int j = 32 * qt; j < 32 * qt + 32; j += 2) {
             Epart += tc::ld_bf16(DS, tc::tile_off(D, j, i)) * tc::ld_bf16(STt, tc::tile_off(D, j, i));
             e2 += tc::ld_bf16(DS, tc::tile_off(D, j + 1, i)) * tc::ld_bf16(STt, tc::tile_off(D, j + 1, i));
         }
@@ -550,38 +670,36 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     ok = tc::mbar_wait(bar_b, ph.b) && ok;
     ph.b ^= 1;
 
-    // ---- gate chain, thread = (key channel i, token half hf). Pass 1 over the half's 32 tokens: dq, dk,
-    // db and dG_t; partial sums of Kt*G4 and dG are exchanged between the halves (in the consumed dP^T
-    // tile). Pass 2: dlog_alpha_t = sum_{tau >= t} dG_tau + E, E = rowsum(dZ*S) + sum_t Kt*G4.
+    // ---- gate chain, thread = (key channel i, token quarter qt: tokens 16 qt .. 16 qt + 15). Pass 1: dq,
+    // dk, db and dG_t; partial sums of Kt*G4 and dG are exchanged between the quarters (in the consumed
+    // dP^T tile). Pass 2: dlog_alpha_t = sum_{tau >= t} dG_tau + E, E = rowsum(dZ*S) + sum_t Kt*G4.
     // Results go to bf16 row tiles (dq -> DO, dk -> DT, db -> DDT, dlog_alpha -> UU), stored by TMA.
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chk = (uint32_t)((i & 63) >> 3);
-    float dG[32];
+    float dG[16];
     float dGsum = 0.f;
-#pragma unroll
-    for (int qq = 0; qq < 2; ++qq) {
-        const int q4 = 2 * hf + qq;
+    {
         float g1[16], g2[16], g3[16], g4[16], gv[16];
-        tc::tmem_ld16(lane_base + TM_G1 + 16 * q4, g1);
-        tc::tmem_ld16(lane_base + TM_G2 + 16 * q4, g2);
-        tc::tmem_ld16(lane_base + TM_G3 + 16 * q4, g3);
-        tc::tmem_ld16(lane_base + TM_G4 + 16 * q4, g4);
-        tc::tmem_ld16(lane_base + TM_GV + 16 * q4, gv);
+        tc::tmem_ld16(lane_base + TM_G1 + 16 * qt, g1);
+        tc::tmem_ld16(lane_base + TM_G2 + 16 * qt, g2);
+        tc::tmem_ld16(lane_base + TM_G3 + 16 * qt, g3);
+        tc::tmem_ld16(lane_base + TM_G4 + 16 * qt, g4);
+        tc::tmem_ld16(lane_base + TM_GV + 16 * qt, gv);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const uint32_t t = (uint32_t)(16 * q4 + u);
+            const uint32_t t = (uint32_t)(16 * qt + u);
             const uint32_t sw = t * 128 + ((chk ^ (t & 7)) << 4);
-            const float qt = tc::ld_bf16(QE, col128 + C * 128 + sw);
+            const float qv = tc::ld_bf16(QE, col128 + C * 128 + sw);
             const float et = tc::ld_bf16(QE, col128 + sw);
             const float kt = tc::ld_bf16(KT, col64 + sw);
             const float kk = tc::ld_bf16(KH, col64 + sw);
             const float bb = tc::ld_bf16(WW, col64 + sw);
             const float g = fast_exp(gv[u]), ig = fast_exp(-gv[u]);
             const float dKt = g3[u] + g4[u];
-            const float dGt = qt * g1[u] + et * g2[u] - kt * dKt;
-            dG[16 * qq + u] = dGt;
+            const float dGt = qv * g1[u] + et * g2[u] - kt * dKt;
+            dG[u] = dGt;
             dGsum += dGt;
             Epart += kt * g4[u];
             const float dE = g * g2[u];
@@ -590,15 +708,19 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             tc::st_bf16(DDT, col64 + sw, dE * kk);                  // db
         }
     }
-    float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][2 halves][128]
-    xch[(0 * 2 + hf) * 128 + i] = Epart;
-    xch[(1 * 2 + hf) * 128 + i] = dGsum;
+    float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][4 quarters][128]
+    xch[(0 * BPARTS + qt) * 128 + i] = Epart;
+    xch[(1 * BPARTS + qt) * 128 + i] = dGsum;
     __syncthreads();
-    const float E = xch[(0 * 2 + 0) * 128 + i] + xch[(0 * 2 + 1) * 128 + i];
-    float suffix = hf == 0 ? xch[(1 * 2 + 1) * 128 + i] : 0.f;      // dG of the later half
+    float E = 0.f, suffix = 0.f;                                    // suffix: dG of the later quarters
 #pragma unroll
-    for (int u = 31; u >= 0; --u) {
-        const uint32_t t = (uint32_t)(32 * hf + u);
+    for (int q = 0; q < BPARTS; ++q) {
+        E += xch[(0 * BPARTS + q) * 128 + i];
+        if (q > qt) suffix += xch[(1 * BPARTS + q) * 128 + i];
+    }
+#pragma unroll
+    for (int u = 15; u >= 0; --u) {
+        const uint32_t t = (uint32_t)(16 * qt + u);
         suffix += dG[u];
         tc::st_bf16(UU, col64 + t * 128 + ((chk ^ (t & 7)) << 4), suffix + E);    // dlog_alpha
     }
@@ -622,7 +744,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     return ok;
 }
 
-__global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
+__global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -691,7 +813,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, chunk_bwd_kernel, NT, SMEM_BYTES_ALL)) != cudaSuccess)
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, chunk_bwd_kernel, BT, SMEM_BYTES_ALL)) != cudaSuccess)
         return e;
     const int BH = d.B * d.H, nc = d.nchunks();
     const int units = BH * nc;
@@ -710,17 +832,17 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     if (coop && BH < slots) {
         p.nrev = BH; p.join = 1; p.grad = 1;
         void* args[2] = {&maps, &p};
-        e = cudaLaunchCooperativeKernel((const void*)chunk_bwd_kernel, dim3(slots), dim3(NT), args, SMEM_BYTES_ALL, s);
+        e = cudaLaunchCooperativeKernel((const void*)chunk_bwd_kernel, dim3(slots), dim3(BT), args, SMEM_BYTES_ALL, s);
         if (e == cudaSuccess) return cudaSuccess;
         (void)cudaGetLastError();   // not launched: fall back to two launches
     }
     BwdParams pr = p;   // reverse pass only
     pr.nrev = BH; pr.join = 0; pr.grad = 0;
-    chunk_bwd_kernel<<<BH, NT, SMEM_BYTES_ALL, s>>>(maps, pr);
+    chunk_bwd_kernel<<<BH, BT, SMEM_BYTES_ALL, s>>>(maps, pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     BwdParams pg = p;   // gradient units only; every flag is set when they start
     pg.nrev = 0; pg.join = 0; pg.grad = 1;
-    chunk_bwd_kernel<<<units < slots ? units : slots, NT, SMEM_BYTES_ALL, s>>>(maps, pg);
+    chunk_bwd_kernel<<<units < slots ? units : slots, BT, SMEM_BYTES_ALL, s>>>(maps, pg);
     return cudaGetLastError();
 }
 

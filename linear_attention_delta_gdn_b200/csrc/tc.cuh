@@ -55,6 +55,23 @@ __device__ __forceinline__ void st_row8(unsigned char* tile, int R, int r, int g
     v.w = pack_bf16x2(x[6], x[7]);
     *reinterpret_cast<uint4*>(tile + tile_chunk_off(R, r, g)) = v;
 }
+// store / load 4 consecutive columns [4g, 4g+4) of row r (8 bytes, half of a 16-byte chunk)
+__device__ __forceinline__ void st_row4(unsigned char* tile, int R, int r, int g, const float* x) {
+    uint2 v;
+    v.x = pack_bf16x2(x[0], x[1]);
+    v.y = pack_bf16x2(x[2], x[3]);
+    *reinterpret_cast<uint2*>(tile + tile_chunk_off(R, r, g >> 1) + ((g & 1) << 3)) = v;
+}
+__device__ __forceinline__ void ld_row4(const unsigned char* tile, int R, int r, int g, float* x) {
+    uint2 v = *reinterpret_cast<const uint2*>(tile + tile_chunk_off(R, r, g >> 1) + ((g & 1) << 3));
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        float2 f = __bfloat1622float2(p[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
 __device__ __forceinline__ void ld_row8(const unsigned char* tile, int R, int r, int g, float* x) {
     uint4 v = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(R, r, g));
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
