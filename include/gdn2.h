@@ -39,6 +39,13 @@
  *     every other supported combination runs on the fp32 recurrent kernels.
  *   - Thread safety: calls may be made from several host threads; error
  *     detail strings are per thread.
+ *   - Launches: on the tensor-core path the forward and the backward each run
+ *     as one cooperative launch when the device allows it (the per-head chain
+ *     and the per-chunk work share the SMs and hand chunks over through ready
+ *     flags in the workspace), else as two ordinary launches with the same
+ *     results. Setting the environment variable GDN2_NO_COOPERATIVE (to any
+ *     value but "0") selects the two-launch form, e.g. for tools that do not
+ *     support cooperative launches.
  */
 #ifndef GDN2_H
 #define GDN2_H

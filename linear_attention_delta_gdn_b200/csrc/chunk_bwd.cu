@@ -829,7 +829,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
 
     TraceScope trace(K_CHUNK_BWD, s);
     // Every head's reverse pass plus at least one gradient worker resident at once: one launch.
-    if (coop && BH < slots) {
+    if (coop && !cooperative_disabled() && BH < slots) {
         p.nrev = BH; p.join = 1; p.grad = 1;
         void* args[2] = {&maps, &p};
         e = cudaLaunchCooperativeKernel((const void*)chunk_bwd_kernel, dim3(slots), dim3(BT), args, SMEM_BYTES_ALL, s);

@@ -466,7 +466,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     TraceScope trace(K_CHUNK_FWD, s);
     // Heads share the launch with the producers while the producers keep pace: per chunk step the
     // BH consumer chunks take about as long as BH WY units spread over the remaining CTAs.
-    if (coop && slots >= 2 && 16 * BH <= 9 * slots) {
+    if (coop && !cooperative_disabled() && slots >= 2 && 16 * BH <= 9 * slots) {
         p.ncons = BH;
         p.nprod = slots - BH < units ? slots - BH : units;
         void* args[2] = {&maps, &p};

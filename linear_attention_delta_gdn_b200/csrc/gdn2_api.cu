@@ -8,6 +8,7 @@
 #include <stdarg.h>
 #include <stdint.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "gdn2.h"
@@ -101,6 +102,10 @@ gdn2_status copy_or_zero_state(float* dst, const float* src, const Dims& d, cuda
 
 namespace gdn2 {
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+bool cooperative_disabled() {
+    const char* v = getenv("GDN2_NO_COOPERATIVE");
+    return v && v[0] && !(v[0] == '0' && v[1] == 0);
+}
 }  // namespace gdn2
 
 extern "C" {

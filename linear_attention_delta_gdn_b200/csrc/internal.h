@@ -77,6 +77,10 @@ class TraceScope {
     bool active_;
 };
 
+// True when the environment variable GDN2_NO_COOPERATIVE is set: the chunkwise kernels then run
+// their producer and consumer work as two ordinary launches instead of one cooperative launch.
+bool cooperative_disabled();
+
 // Sets the detail string returned by gdn2_last_error() on this host thread.
 void set_last_error(const char* msg);
 
