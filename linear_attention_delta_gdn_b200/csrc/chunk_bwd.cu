@@ -169,7 +169,7 @@ __device__ __forceinline__ void grad_prep(unsigned char* QE, unsigned char* KH, 
 constexpr uint32_t TILE_C = 64 * 64 * 2;   // bytes of a 64 x 64 bf16 tile
 
 // Barrier block shared by both kinds of work (above every tile of either layout):
-// 4 mbarriers (load, mma, k, b), TMEM base, abort flag, broadcast unit index.
+// 4 mbarriers (load, mma, k, b), TMEM base, abort flag, next unit (2 ints), prefetch mbarrier at +48.
 constexpr uint32_t OFF_BARS = 229888;
 constexpr uint32_t SMEM_BYTES_ALL = 229952 + 1024;
 
@@ -192,7 +192,12 @@ struct BwdParams {
 };
 // mbarrier parities carried across the units a CTA works on
 struct Phases {
-    uint32_t load = 0, mma = 0, k = 0, b = 0;
+    uint32_t load = 0, mma = 0, k = 0, b = 0, pre = 0;
+};
+// The next gradient unit of a CTA, handed between units through shared memory (OFF_BARS + 40):
+// [0] unit index, [1] nonzero once its S, T and dZ^T images are being prefetched (flag acquired).
+struct NextUnit {
+    int unit, prefetched;
 };
 
 // ====================================================================== reverse state pass
@@ -243,20 +248,27 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 32 * tm_part(warp);      // lane row, column quarter
 
     // chunk c's tiles arrive on one barrier phase, issued in three groups as their buffers free up
-    auto issue_first = [&](int c) {   // q, log_alpha, dout, Wm: buffers of this parity are free
+    // q, log_alpha, dout, Wm (buffers of this parity are free): issued by lane 0 of warps 0-3 at once
+    auto issue_first = [&](int c) {
+        if (lane != 0 || warp > 3) return;
         const int t0 = c * C;
-        tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-        tma_tile(QQ(c), C, 0, &m.q, b, h, t0, bar_load);
-        tma_tile(KT(c), C, 0, &m.la, b, h, t0, bar_load);
-        tma_tile(DO(c), C, 0, &m.dout, b, h, t0, bar_load);
-        tc::bulk_load(WW(c), p.tp + (head * nc + c) * TC_WY_BYTES + 2 * TILE_C, 64 * 128 * 2, bar_load);
+        if (warp == 0) {
+            tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
+            tma_tile(QQ(c), C, 0, &m.q, b, h, t0, bar_load);
+        } else if (warp == 1) {
+            tma_tile(KT(c), C, 0, &m.la, b, h, t0, bar_load);
+        } else if (warp == 2) {
+            tma_tile(DO(c), C, 0, &m.dout, b, h, t0, bar_load);
+        } else {
+            tc::bulk_load(WW(c), p.tp + (head * nc + c) * TC_WY_BYTES + 2 * TILE_C, 64 * 128 * 2, bar_load);
+        }
     };
     auto issue_k = [&](int c) { tma_tile(KH, C, 0, &m.k, b, h, c * C, bar_load); };   // after the prep
     auto issue_p = [&](int c) {   // after the MMAs that read P
         tc::bulk_load(PP, p.tp + (head * nc + c) * TC_WY_BYTES + TILE_C, TILE_C, bar_load);
     };
+    issue_first(nc - 1);
     if (tid == 0) {
-        issue_first(nc - 1);
         issue_k(nc - 1);
         issue_p(nc - 1);
     }
@@ -300,7 +312,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         if (!tc::mbar_wait(bar_load, ph.load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
         ph.load ^= 1;
         // the other parity's buffers were last read by chunk c + 1, whose MMAs are complete
-        if (tid == 0 && c > 0) issue_first(c - 1);
+        if (c > 0) issue_first(c - 1);
 
         prep_qk4(QQ(c), KH, KT(c), sGC, sRed, tid);   // Qt, Kt, gC
         tc::fence_async_smem();   // the prep's reads of k precede the TMA that overwrites it
@@ -414,12 +426,17 @@ constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
     TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,
     TM_GV = 448;                   // G[t] per key channel (cumulative log-decay)
-constexpr uint32_t LOAD_BYTES = 8 * 64 * 128 * 2 + (uint32_t)TC_STATE_BYTES + 2 * TILE_C;   // dZ^T: cp.async
+constexpr uint32_t LOAD_TOK = 8 * 64 * 128 * 2 + TILE_C;          // 7 token tiles, Wm, P
+constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dZ^T: cp.async)
 }  // namespace cg
 
-// Gradients of chunk c of head `headi`; returns false if a bounded wait gave up.
+// Gradients of chunk c of head `headi`; returns false if a bounded wait gave up. `prefetched`: the S, T
+// and dZ^T images of this unit were requested by the previous unit (S, T on the prefetch barrier).
+// Thread 0 takes the CTA's next unit from the counter while this one runs and, once that unit's flag
+// is acquired, requests its S, T and dZ^T images into the tiles this unit has finished with; the
+// next unit is published in *nxt before the unit's last barrier.
 __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi, int c,
-                          Phases& ph) {
+                          Phases& ph, bool prefetched, NextUnit* nxt) {
     using namespace cg;
     unsigned char* QE = sm + OFF_QE;
     unsigned char* KH = sm + OFF_KH;
@@ -437,9 +454,11 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     uint64_t* bar_mma = bar_load + 1;
     uint64_t* bar_k = bar_load + 2;
     uint64_t* bar_b = bar_load + 3;
+    uint64_t* bar_pre = reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T, H = p.H, nc = p.nc;
+    const int units = p.BH * nc;
     const int h = headi % H, b = headi / H;
     const size_t head = (size_t)headi;
     const int t0 = c * C;
@@ -450,21 +469,39 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     __nv_bfloat16* __restrict__ dw = p.dw;
 
     bool ok = true;
-    if (tid == 0) {
-        tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-        tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
-        tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load);
-        tma_tile(KH, C, 0, mk, b, h, t0, bar_load);
-        tma_tile(KT, C, 0, mla, b, h, t0, bar_load);
-        tma_tile(UU, C, 0, mv, b, h, t0, bar_load);
-        tma_tile(WW, C, 0, mw, b, h, t0, bar_load);
-        tma_tile(DO, C, 0, mdo, b, h, t0, bar_load);
-        tc::bulk_load(STt, p.states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
+    int next_unit = units;    // thread 0: the CTA's next unit (its atomic returns while this unit runs)
+    bool next_ready = false;  // thread 0: the next unit's dZ^T flag has been acquired
+    // The loads are issued by lane 0 of several warps at once (a TMA issue takes ~100 cycles); the
+    // barrier phase cannot complete before thread 0's arrival, which carries the expected bytes.
+    // (*nxt is rewritten only after the next barriers: every thread has read it by then.)
+    if (lane == 0) {
         const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
-        tc::bulk_load(TT, src, TILE_C, bar_load);
-        tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
-        tc::bulk_load(DDT, src + 2 * TILE_C, 64 * 128 * 2, bar_load);   // Wm rows (DDT is free until dDelta^T)
-        // dZ^T of this chunk comes from the reverse pass: wait for its flag
+        switch (warp) {
+        case 0:
+            tc::mbar_arrive_expect_tx(bar_load, prefetched ? LOAD_TOK : LOAD_TOK + LOAD_PRE);
+            tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
+            next_unit = (int)atomicAdd(p.counter, 1u);   // the value is first needed after the G MMAs
+            break;
+        case 1: tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load); break;
+        case 2: tma_tile(KH, C, 0, mk, b, h, t0, bar_load); break;
+        case 3: tma_tile(KT, C, 0, mla, b, h, t0, bar_load); break;
+        case 4: tma_tile(UU, C, 0, mv, b, h, t0, bar_load); break;
+        case 5: tma_tile(WW, C, 0, mw, b, h, t0, bar_load); break;
+        case 6: tma_tile(DO, C, 0, mdo, b, h, t0, bar_load); break;
+        case 7:
+            tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
+            tc::bulk_load(DDT, src + 2 * TILE_C, 64 * 128 * 2, bar_load);   // Wm rows (DDT is free until dDelta^T)
+            break;
+        case 8:
+            if (!prefetched) {
+                tc::bulk_load(STt, p.states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
+                tc::bulk_load(TT, src, TILE_C, bar_load);
+            }
+            break;
+        default: break;
+        }
+    }
+    if (tid == 0 && !prefetched) {   // dZ^T of this chunk comes from the reverse pass: wait for its flag
         if (!tc::flag_wait(p.flags + head * nc + c, 1u)) {
             ok = false;
             atomicOr(&g_bwd_error, 8u);
@@ -472,7 +509,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         }
     }
     __syncthreads();   // orders thread 0's acquire before every thread's copy of the dZ^T image
-    {
+    if (!prefetched) {
         const unsigned char* src = p.dstates + (head * nc + c) * TC_STATE_BYTES;
 #pragma unroll
         for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i)
@@ -484,6 +521,10 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     (void)jrow;
     ok = tc::mbar_wait(bar_load, ph.load) && ok;
     ph.load ^= 1;
+    if (prefetched) {
+        ok = tc::mbar_wait(bar_pre, ph.pre) && ok;
+        ph.pre ^= 1;
+    }
     tc::cp_async_wait_all();
     auto wait_mma = [&]() {
         ok = tc::mbar_wait(bar_mma, ph.mma) && ok;
@@ -649,6 +690,13 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         for (int kk = 0; kk < 4; ++kk)
             tc::mma_bf16(tmem + TM_G3, tc::desc_mn(sQE, 2 * C, 0, kk), tc::desc_k(sTT, C, 0, kk), id_mk, 1);
         tc::mma_commit(bar_mma);
+        // while these run: stop if any CTA of the launch gave up; else is the next unit's dZ^T ready?
+        // (acquire; usually it has been for long)
+        if (*reinterpret_cast<volatile unsigned int*>(p.counter + 1)) next_unit = units;
+        if (next_unit < units) {
+            const int nc_ = nc - 1 - next_unit / p.BH, nh = next_unit % p.BH;
+            next_ready = tc::ld_acquire(p.flags + (size_t)nh * nc + nc_) == 1u;
+        }
     }
 
     // rowsum(dZ * S) for key channel i over this quarter's value channels (both images hold row j =
@@ -711,7 +759,28 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][4 quarters][128]
     xch[(0 * BPARTS + qt) * 128 + i] = Epart;
     xch[(1 * BPARTS + qt) * 128 + i] = dGsum;
-    __syncthreads();
+    if (tid == 0) {
+        nxt->unit = next_unit;
+        nxt->prefetched = next_ready;
+    }
+    tc::fence_async_smem();   // every read of S^T and dZ^T (G MMAs, rowsum) precedes the prefetch below
+    __syncthreads();          // also orders thread 0's acquire before every thread's copy of the next dZ^T
+    if (tid == 0 && next_ready) {   // S^T and T of the next unit into the tiles this unit has finished with
+        const int nc_ = nc - 1 - next_unit / p.BH, nh = next_unit % p.BH;
+        const size_t nu = (size_t)nh * nc + nc_;
+        tc::mbar_arrive_expect_tx(bar_pre, LOAD_PRE);
+        tc::bulk_load(STt, p.states + nu * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_pre);
+        tc::bulk_load(TT, p.tp + nu * TC_WY_BYTES, TILE_C, bar_pre);
+    }
+    if (nxt->prefetched) {
+        const int nu_ = nxt->unit;
+        const size_t nu = (size_t)(nu_ % p.BH) * nc + (nc - 1 - nu_ / p.BH);
+        const unsigned char* src = p.dstates + nu * TC_STATE_BYTES;
+#pragma unroll
+        for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i)
+            tc::cp_async16_cg(DS + 16 * (tid + BT * i), src + 16 * (tid + BT * i));
+        tc::cp_async_commit();
+    }
     float E = 0.f, suffix = 0.f;                                    // suffix: dG of the later quarters
 #pragma unroll
     for (int q = 0; q < BPARTS; ++q) {
@@ -751,9 +820,10 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 32);
     int* abort_flag = reinterpret_cast<int*>(sm + OFF_BARS + 36);
-    int* unit_bcast = reinterpret_cast<int*>(sm + OFF_BARS + 40);
+    NextUnit* nxt = reinterpret_cast<NextUnit*>(sm + OFF_BARS + 40);
     if (tid == 0) {
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
+        tc::mbar_init(reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -770,17 +840,24 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
     if (reverse) run_reverse(maps, p, sm, tmem, blockIdx.x, ph);
     if (p.grad && (!reverse || p.join) && !*abort_flag) {
         const int units = p.BH * p.nc;
-        while (true) {
-            if (tid == 0)   // stop taking units once any CTA of the launch has given up
-                *unit_bcast = *reinterpret_cast<volatile unsigned int*>(p.counter + 1) ? units
-                                                                                       : (int)atomicAdd(p.counter, 1u);
-            __syncthreads();
-            const int u = *unit_bcast;
-            __syncthreads();
-            if (u >= units) break;
+        if (tid == 0) {   // stop taking units once any CTA of the launch has given up
+            nxt->unit = *reinterpret_cast<volatile unsigned int*>(p.counter + 1) ? units : (int)atomicAdd(p.counter, 1u);
+            nxt->prefetched = 0;
+        }
+        __syncthreads();
+        int u = nxt->unit;
+        bool pre = false;
+        while (u < units) {
             // units in the order the reverse pass produces them: chunks from the last, heads inside
             const int c = p.nc - 1 - u / p.BH, headi = u % p.BH;
-            if (!grad_unit(maps, p, sm, tmem, headi, c, ph)) break;
+            if (!grad_unit(maps, p, sm, tmem, headi, c, ph, pre, nxt)) {
+                // a bounded wait gave up: let a prefetch in flight land before leaving
+                if (tid == 0 && nxt->prefetched) (void)tc::mbar_wait(reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48), ph.pre);
+                tc::cp_async_wait_all();
+                break;
+            }
+            u = nxt->unit;   // written by thread 0 before the unit's last barrier
+            pre = nxt->prefetched != 0;
         }
     }
     tc::tc_fence_before();

@@ -114,17 +114,24 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
     const int units = p.BH * p.nc;
 
+    // the four tiles of unit u, issued by lane 0 of warps 0-3 at once (a TMA issue takes ~100 cycles)
     auto issue_loads = [&](int stage, int u) {
+        if (lane != 0 || warp > 3) return;
         const int c = u / p.BH, head = u % p.BH;
         const int b = head / p.H, h = head % p.H, t0 = c * C;
         unsigned char* base = sm + stage * wy::STAGE;
-        tc::mbar_arrive_expect_tx(&bar_in[stage], PROD_LOAD_BYTES);
-        tma_tile(base + wy::QE, 2 * C, 0, &m.b, b, h, t0, &bar_in[stage]);
-        tma_tile(base + wy::QE, 2 * C, C, &m.q, b, h, t0, &bar_in[stage]);
-        tma_tile(base + wy::KH, C, 0, &m.k, b, h, t0, &bar_in[stage]);
-        tma_tile(base + wy::KT, C, 0, &m.la, b, h, t0, &bar_in[stage]);
+        if (warp == 0) {
+            tc::mbar_arrive_expect_tx(&bar_in[stage], PROD_LOAD_BYTES);
+            tma_tile(base + wy::QE, 2 * C, 0, &m.b, b, h, t0, &bar_in[stage]);
+        } else if (warp == 1) {
+            tma_tile(base + wy::QE, 2 * C, C, &m.q, b, h, t0, &bar_in[stage]);
+        } else if (warp == 2) {
+            tma_tile(base + wy::KH, C, 0, &m.k, b, h, t0, &bar_in[stage]);
+        } else {
+            tma_tile(base + wy::KT, C, 0, &m.la, b, h, t0, &bar_in[stage]);
+        }
     };
-    if (tid == 0 && pid < units) issue_loads(0, pid);
+    if (pid < units) issue_loads(0, pid);
 
     uint32_t ph_in = 0, ph_mma = 0;   // ph_in: bit s = phase parity of input stage s
     auto wait_mma = [&]() {
@@ -143,7 +150,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         ph_in ^= 1u << stage;
         // the other stage was last read by the previous unit's MMAs, which have completed
         pending = u + p.nprod < units;
-        if (tid == 0 && pending) issue_loads(stage ^ 1, u + p.nprod);
+        if (pending) issue_loads(stage ^ 1, u + p.nprod);
 
         gate_prep(QE, base + wy::KH, base + wy::KT, nullptr, nullptr, nullptr, sA, tid, true, false);
         sync_for_mma();
@@ -240,14 +247,20 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
         const int h = headi % H, b = headi / H;
         // q and log_alpha tiles alternate between two buffers by chunk parity (read by the MMAs of
         // chunk c while the tiles of chunk c + 1 arrive); k, v and w have one buffer each
+        // issued by lane 0 of warps 0-4 at once (a TMA issue takes ~100 cycles)
         auto issue_loads = [&](int c) {
+            if (lane != 0 || warp > 4) return;
             const int t0 = c * C, par = c & 1;
-            tc::mbar_arrive_expect_tx(bar_load, CONS_LOAD_BYTES);
-            tma_tile(sm + sp::QQ + par * TILE_64x128, C, 0, &m.q, b, h, t0, bar_load);
-            tma_tile(sm + sp::KT + par * TILE_64x128, C, 0, &m.la, b, h, t0, bar_load);
-            tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load);
-            tma_tile(UU, C, 0, &m.v, b, h, t0, bar_load);
-            tma_tile(WW, C, 0, &m.w, b, h, t0, bar_load);
+            switch (warp) {
+            case 0:
+                tc::mbar_arrive_expect_tx(bar_load, CONS_LOAD_BYTES);
+                tma_tile(sm + sp::QQ + par * TILE_64x128, C, 0, &m.q, b, h, t0, bar_load);
+                break;
+            case 1: tma_tile(sm + sp::KT + par * TILE_64x128, C, 0, &m.la, b, h, t0, bar_load); break;
+            case 2: tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load); break;
+            case 3: tma_tile(UU, C, 0, &m.v, b, h, t0, bar_load); break;
+            default: tma_tile(WW, C, 0, &m.w, b, h, t0, bar_load); break;
+            }
         };
         // o rows of chunk c from its M=64 accumulator (16-byte stores)
         auto store_o = [&](int c) {
@@ -268,10 +281,8 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 }
             }
         };
-        if (tid == 0) {
-            issue_loads(0);
-            wait_wy(head, 0);
-        }
+        issue_loads(0);
+        if (tid == 0) wait_wy(head, 0);
         // initial state: S^T row j = column j of S0
         {
             const int j = jrow;
@@ -331,7 +342,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             if (want_o && c > 0) store_o(c - 1);      // previous chunk's output, in the MMAs' shadow
             wait_mma();
             // k, v, w and the other parity's q, log_alpha tiles are free: prefetch the next chunk
-            if (tid == 0 && c + 1 < nc) issue_loads(c + 1);
+            if (c + 1 < nc) issue_loads(c + 1);
             tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
             sync_for_mma();
 
