@@ -26,8 +26,9 @@
 //                   ready flag (release);
 //   chunk gradients every other CTA takes (head, chunk) units from a shared counter, in the
 //                   order the reverse pass produces them, waits for the unit's flag (acquire) and
-//                   computes every gradient of the chunk from the saved S, dZ, T, P, the inputs and
-//                   dout. Reverse-pass CTAs join them once their head is done.
+//                   computes every gradient of the chunk from the saved S, Delta (forward), dZ,
+//                   dDelta (reverse pass), T, P, the inputs and dout. Reverse-pass CTAs join them
+//                   once their head is done.
 // With few heads this is one cooperative launch (all CTAs resident, so every wait ends; each wait is
 // also bounded in time); otherwise the reverse pass and the gradients run as two launches.
 #include <cuda.h>
@@ -108,15 +109,14 @@ __device__ __forceinline__ void prep_qk4(unsigned char* QQ, const unsigned char*
     }
 }
 
-// Gradient-unit prep, thread = (key/value channel i = tid % 128, token quarter qt = tid / 128: tokens
+// Gradient-unit prep, thread = (key channel i = tid % 128, token quarter qt = tid / 128: tokens
 // 16 qt .. 16 qt + 15):
-//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127), v (UU), w (WW)
-//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT, U = w*v -> KH (over k);
+//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127)
+//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT (k stays in KH);
 //   G[t][i] goes to TMEM at tmem_g (lane i, column t). Quarter sums of log_alpha are exchanged
 //   through qsum (fp32 [4][128]). Contains one __syncthreads.
-__device__ __forceinline__ void grad_prep(unsigned char* QE, unsigned char* KH, unsigned char* KT,
-                                          const unsigned char* UU, const unsigned char* WW, float* qsum,
-                                          int tid, uint32_t tmem_g) {
+__device__ __forceinline__ void grad_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
+                                          float* qsum, int tid, uint32_t tmem_g) {
     const int i = tid & 127, qt = tid >> 7;
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
@@ -137,7 +137,7 @@ __device__ __forceinline__ void grad_prep(unsigned char* QE, unsigned char* KH, 
     float gvals[16];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        float kk[8], bb[8], qq[8], vv[8], ww[8];
+        float kk[8], bb[8], qq[8];
         uint32_t o64[8], o128[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -148,8 +148,6 @@ __device__ __forceinline__ void grad_prep(unsigned char* QE, unsigned char* KH, 
             kk[u] = tc::ld_bf16(KH, o64[u]);
             bb[u] = tc::ld_bf16(QE, o128[u]);
             qq[u] = tc::ld_bf16(QE, o128[u] + C * 128);
-            vv[u] = tc::ld_bf16(UU, o64[u]);
-            ww[u] = tc::ld_bf16(WW, o64[u]);
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -159,7 +157,6 @@ __device__ __forceinline__ void grad_prep(unsigned char* QE, unsigned char* KH, 
             tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);          // Et
             tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);        // Qt
             tc::st_bf16(KT, o64[u], kk[u] * ig);                  // Kt
-            tc::st_bf16(KH, o64[u], ww[u] * vv[u]);               // U
         }
     }
     tc::tmem_st16(tmem_g + 16 * qt, gvals);
@@ -185,8 +182,10 @@ struct BwdParams {
     float* dS0;
     __nv_bfloat16 *dv, *dw;
     const unsigned char* states;     // chunk-start state images
+    const unsigned char* deltas;     // Delta^T images of the forward
     const unsigned char* tp;         // WY images (T | P | Wm)
     unsigned char* dstates;          // dZ^T images
+    unsigned char* ddeltas;          // dDelta^T images
     unsigned int* flags;             // [BH, nc] dZ ready flags (zero at launch)
     unsigned int* counter;           // [0]: next gradient unit, [1]: abort word (zero at launch)
 };
@@ -364,6 +363,12 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         if (tid == 0 && c > 0) issue_p(c - 1);
         tmem_rows_to_tile<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
+        {   // dDelta^T image for the gradient units (published with the dZ^T image)
+            uint4* dst = reinterpret_cast<uint4*>(p.ddeltas + (head * nc + c) * TC_DELTA_BYTES);
+            const uint4* src = reinterpret_cast<const uint4*>(DT);
+#pragma unroll
+            for (int i = 0; i < (int)(TC_DELTA_BYTES / 16 / BT); ++i) dst[tid + BT * i] = src[tid + BT * i];
+        }
 
         // dS^T -= dDelta^T Wm
         if (tid == 0) {
@@ -407,26 +412,24 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
 
 namespace cg {
 constexpr uint32_t OFF_QE = 0;           // rows 0..63: b -> Et, rows 64..127: q -> Qt
-constexpr uint32_t OFF_KH = 32768;       // k -> U, later k (reloaded)
+constexpr uint32_t OFF_KH = 32768;       // k
 constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
 constexpr uint32_t OFF_UU = 65536;       // v, later dU rows [t][j], later staged dlog_alpha
 constexpr uint32_t OFF_WW = 81920;       // w, later b (reloaded)
 constexpr uint32_t OFF_DO = 98304;       // dout, later staged dq
 constexpr uint32_t OFF_ST = 114688;      // S^T image (chunk start)
 constexpr uint32_t OFF_DS = 147456;      // dZ^T image
-constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64], later staged dk
-constexpr uint32_t OFF_DDT = 196608;     // Wm rows, then dDelta^T [128 x 64], later staged db
+constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64] (forward image), later staged dk
+constexpr uint32_t OFF_DDT = 196608;     // dDelta^T [128 x 64] (reverse-pass image), later staged db
 constexpr uint32_t OFF_TT = 212992;      // T, later dA^T [64 x 64]
-constexpr uint32_t OFF_PP = 221184;      // P, later dP^T [64 x 64]
+constexpr uint32_t OFF_PP = 221184;      // prep scratch, then dP^T [64 x 64]
 // TMEM columns (M=64 accumulators use lanes 0-15 of each 32-lane quarter)
 constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
-    TM_W = 64,                     // Wm (M=64, 128 columns), later dA^T (M=64, 64 columns)
-    TM_D = 192,                    // Ut^T -> Delta^T, later G4 = (Delta dZ^T)^T
-    TM_DD = 256,                   // dDelta^T, later G3 = dKt^T (P and A paths)
+    TM_W = 64,                     // dA^T (M=64, 64 columns)
     TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
-    TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,
+    TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,   // G3 = dKt^T (P and A paths), G4 = (Delta dZ^T)^T
     TM_GV = 448;                   // G[t] per key channel (cumulative log-decay)
-constexpr uint32_t LOAD_TOK = 8 * 64 * 128 * 2 + TILE_C;          // 7 token tiles, Wm, P
+constexpr uint32_t LOAD_TOK = 7 * 64 * 128 * 2 + (uint32_t)TC_DELTA_BYTES;   // 7 token tiles, Delta^T
 constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dZ^T: cp.async)
 }  // namespace cg
 
@@ -452,7 +455,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     unsigned char* PP = sm + OFF_PP;
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_load + 1;
-    uint64_t* bar_k = bar_load + 2;
     uint64_t* bar_b = bar_load + 3;
     uint64_t* bar_pre = reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48);
 
@@ -489,8 +491,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         case 5: tma_tile(WW, C, 0, mw, b, h, t0, bar_load); break;
         case 6: tma_tile(DO, C, 0, mdo, b, h, t0, bar_load); break;
         case 7:
-            tc::bulk_load(PP, src + TILE_C, TILE_C, bar_load);
-            tc::bulk_load(DDT, src + 2 * TILE_C, 64 * 128 * 2, bar_load);   // Wm rows (DDT is free until dDelta^T)
+            tc::bulk_load(DT, p.deltas + (head * nc + c) * TC_DELTA_BYTES, (uint32_t)TC_DELTA_BYTES, bar_load);
             break;
         case 8:
             if (!prefetched) {
@@ -509,11 +510,17 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         }
     }
     __syncthreads();   // orders thread 0's acquire before every thread's copy of the dZ^T image
-    if (!prefetched) {
-        const unsigned char* src = p.dstates + (head * nc + c) * TC_STATE_BYTES;
+    {   // the reverse pass's images of this chunk: dZ^T (unless prefetched) and dDelta^T
+        if (!prefetched) {
+            const unsigned char* src = p.dstates + (head * nc + c) * TC_STATE_BYTES;
 #pragma unroll
-        for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i)
-            tc::cp_async16_cg(DS + 16 * (tid + BT * i), src + 16 * (tid + BT * i));
+            for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i)
+                tc::cp_async16_cg(DS + 16 * (tid + BT * i), src + 16 * (tid + BT * i));
+        }
+        const unsigned char* src = p.ddeltas + (head * nc + c) * TC_DELTA_BYTES;
+#pragma unroll
+        for (int i = 0; i < (int)(TC_DELTA_BYTES / 16 / BT); ++i)
+            tc::cp_async16_cg(DDT + 16 * (tid + BT * i), src + 16 * (tid + BT * i));
         tc::cp_async_commit();
     }
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
@@ -537,51 +544,13 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         __syncthreads();
     };
 
-    const uint32_t sQE = tc::smem_u32(QE), sKH = tc::smem_u32(KH), sKT = tc::smem_u32(KT),
+    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT),
                    sUU = tc::smem_u32(UU), sDO = tc::smem_u32(DO), sST = tc::smem_u32(STt),
                    sDS = tc::smem_u32(DS), sDT = tc::smem_u32(DT), sDDT = tc::smem_u32(DDT),
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
-    // ---- factors (U over k, G kept in TMEM)
-    grad_prep(QE, KH, KT, UU, WW, reinterpret_cast<float*>(DT), tid, lane_base + TM_GV);   // DT: scratch
-    sync_for_mma();
-
-    // ---- Ut^T = U^T T^T
-    if (tid == 0) {
-        tc::tc_fence_after();
-        constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(tmem + TM_D, tc::desc_mn(sKH, C, 0, kk), tc::desc_k(sTT, C, 0, kk), id_u, kk > 0);
-        tc::mma_commit(bar_mma);
-    }
-    wait_mma();
-    if (tid == 0) {     // U is consumed: bring k back for the gate chain
-        tc::mbar_arrive_expect_tx(bar_k, 64 * 128 * 2);
-        tma_tile(KH, C, 0, mk, b, h, t0, bar_k);
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-
-    // ---- Delta^T = Ut^T - S^T Wm^T ;  dDelta^T = dZ^T Kt^T + dO^T P
-    if (tid == 0) {
-        tc::tc_fence_after();
-        constexpr uint32_t id_neg = tc::idesc_bf16(128, 64, false, false, true);
-        constexpr uint32_t id_kk = tc::idesc_bf16(128, 64, false, false);
-        constexpr uint32_t id_mm = tc::idesc_bf16(128, 64, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sDDT, C, 0, kk), id_neg, 1);
-            tc::mma_bf16(tmem + TM_DD, tc::desc_k(sDS, D, 0, kk), tc::desc_k(sKT, C, 0, kk), id_kk, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(tmem + TM_DD, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), id_mm, 1);
-        tc::mma_commit(bar_mma);
-    }
-    wait_mma();
-    tmem_rows_to_tile<64>(lane_base + TM_D, DT, warp, lane);     // Delta^T [j][t]
-    tmem_rows_to_tile<64>(lane_base + TM_DD, DDT, warp, lane);   // dDelta^T [j][t]
+    // ---- factors (G kept in TMEM)
+    grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV);   // PP: scratch until dP^T
     sync_for_mma();
 
     // ---- dU = T^T dDelta (M=64)
@@ -713,8 +682,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         Epart += e2;
     }
     wait_mma();
-    ok = tc::mbar_wait(bar_k, ph.k) && ok;
-    ph.k ^= 1;
     ok = tc::mbar_wait(bar_b, ph.b) && ok;
     ph.b ^= 1;
 
@@ -900,7 +867,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
     p.dST = a.dST; p.dS0 = a.dS0;
     p.dv = static_cast<__nv_bfloat16*>(a.dv); p.dw = static_cast<__nv_bfloat16*>(a.dw);
-    p.states = a.states; p.tp = a.tp; p.dstates = a.dstates;
+    p.states = a.states; p.deltas = a.deltas; p.tp = a.tp; p.dstates = a.dstates; p.ddeltas = a.ddeltas;
     p.flags = a.flags; p.counter = a.flags + units;
     if ((e = cudaMemsetAsync(a.flags, 0, ((size_t)units + 2) * sizeof(unsigned int), s)) != cudaSuccess) return e;
 

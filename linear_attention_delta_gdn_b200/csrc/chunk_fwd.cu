@@ -82,6 +82,7 @@ struct FwdParams {
     __nv_bfloat16* o;              // may be null (states only)
     float* ST;
     unsigned char* states;         // [BH, nc] chunk-start state images, or null
+    unsigned char* deltas;         // [BH, nc] Delta^T images, or null
     unsigned char* wyimg;          // [BH, nc] WY images
     unsigned int* flags;           // [BH, nc] ready flags (zero at launch)
 };
@@ -345,6 +346,10 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             if (c + 1 < nc) issue_loads(c + 1);
             tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
             sync_for_mma();
+            if (p.deltas && tid == 0) {   // Delta^T of this chunk for the backward
+                tc::bulk_store(p.deltas + (head * nc + c) * TC_DELTA_BYTES, DT, (uint32_t)TC_DELTA_BYTES);
+                tc::bulk_commit();
+            }
 
             // ---- M6: O += P Delta ;  M7: Z^T = S^T + Delta^T Kt
             if (tid == 0) {
@@ -358,7 +363,8 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 tc::mma_commit(bar_mma);
             }
             wait_mma();
-            // S'^T = Z^T Diag(gC): scale the fp32 state, keep a bf16 copy for the next chunk
+            // S'^T = Z^T Diag(gC): scale the fp32 state, keep a bf16 copy for the next chunk (the bulk
+            // stores of the previous state image and of this chunk's Delta^T must have read their tiles)
             if (p.states && tid == 0) tc::bulk_wait_read();
             __syncthreads();   // also orders thread 0's flag acquire before the image copy
             if (c + 1 < nc) copy_wy(head, c + 1);
@@ -471,7 +477,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     FwdParams p{};
     p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
     p.S0 = a.S0; p.o = static_cast<__nv_bfloat16*>(a.o); p.ST = a.ST;
-    p.states = a.states; p.wyimg = a.wy; p.flags = a.flags;
+    p.states = a.states; p.deltas = a.deltas; p.wyimg = a.wy; p.flags = a.flags;
     if ((e = cudaMemsetAsync(a.flags, 0, (size_t)units * sizeof(unsigned int), s)) != cudaSuccess) return e;
 
     TraceScope trace(K_CHUNK_FWD, s);

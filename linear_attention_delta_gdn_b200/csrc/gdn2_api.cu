@@ -55,25 +55,27 @@ gdn2_status check_dims(int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtyp
 }
 
 // Tensor-core workspace (units = B*H*NC chunks), each region 256-byte aligned:
-//   [states: units x TC_STATE_BYTES, training only][WY images: units x TC_WY_BYTES][ready flags]
-//   then, for the backward, [dstates: units x TC_STATE_BYTES].
+//   [states: units x TC_STATE_BYTES][Delta^T: units x TC_DELTA_BYTES]  (training only)
+//   [WY images: units x TC_WY_BYTES][ready flags]
+//   then, for the backward, [dZ^T: units x TC_STATE_BYTES][dDelta^T: units x TC_DELTA_BYTES][flags].
 size_t tc_units(const Dims& d) { return (size_t)d.B * d.H * (size_t)d.nchunks(); }
 size_t tc_wy_bytes(const Dims& d) { return tc_units(d) * TC_WY_BYTES + align256(tc_units(d) * sizeof(unsigned int)); }
 
-// Forward-saved region: chunk-start states (and, on the tensor-core path, the WY images and flags).
+// Forward-saved region: chunk-start states (and, on the tensor-core path, Delta^T, the WY images and flags).
 size_t states_bytes(const Dims& d, gdn2_dtype dt) {
     const size_t units = tc_units(d);
-    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * TC_STATE_BYTES + tc_wy_bytes(d)
+    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * (TC_STATE_BYTES + TC_DELTA_BYTES) + tc_wy_bytes(d)
                                                   : units * d.Dk * d.Dv * sizeof(float);
 }
-size_t tc_tp_offset(const Dims& d) { return tc_units(d) * TC_STATE_BYTES; }
+size_t tc_delta_offset(const Dims& d) { return tc_units(d) * TC_STATE_BYTES; }
+size_t tc_tp_offset(const Dims& d) { return tc_units(d) * (TC_STATE_BYTES + TC_DELTA_BYTES); }
 size_t tc_flags_offset(const Dims& d, bool with_states) {
     return (with_states ? tc_tp_offset(d) : 0) + tc_units(d) * TC_WY_BYTES;
 }
 
 size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
-    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk))   // dZ images, then ready flags, work counter, abort word
-        return tc_units(d) * TC_STATE_BYTES + align256((tc_units(d) + 2) * sizeof(unsigned int));
+    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk))   // dZ and dDelta images, ready flags, work counter, abort word
+        return tc_units(d) * (TC_STATE_BYTES + TC_DELTA_BYTES) + align256((tc_units(d) + 2) * sizeof(unsigned int));
     const size_t seg = (size_t)d.B * d.H * d.chunk * d.Dk * d.Dv * sizeof(float);
     const size_t del = (size_t)d.B * d.H * d.chunk * d.Dv * sizeof(float);
     return align256(seg) + align256(del);
@@ -165,6 +167,7 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
         unsigned char* wsb = static_cast<unsigned char*>(ws);
         const bool keep = save_states != 0;
         a.states = keep ? wsb : nullptr;
+        a.deltas = keep ? wsb + tc_delta_offset(d) : nullptr;
         a.wy = wsb + (keep ? tc_tp_offset(d) : 0);
         a.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, keep));
         return cuda_status(chunk_fwd_launch(a, s), "gdn2_fwd (tensor-core path)");
@@ -208,7 +211,8 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
             ChunkFwdArgs f{};
             f.d = d;
             f.q = q; f.k = k; f.v = v; f.la = log_alpha; f.b = b; f.w = w;
-            f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.wy = wsb + tc_tp_offset(d);
+            f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.deltas = wsb + tc_delta_offset(d);
+            f.wy = wsb + tc_tp_offset(d);
             f.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, true));
             gdn2_status e = cuda_status(chunk_fwd_launch(f, s), "gdn2_bwd state recompute");
             if (e != GDN2_OK) return e;
@@ -220,8 +224,10 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
         a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.db = db; a.dw = dw; a.dS0 = dS0;
         a.states = wsb;
         a.tp = wsb + tc_tp_offset(d);
+        a.deltas = wsb + tc_delta_offset(d);
         a.dstates = extra;
-        a.flags = reinterpret_cast<unsigned int*>(extra + tc_units(d) * TC_STATE_BYTES);
+        a.ddeltas = extra + tc_units(d) * TC_STATE_BYTES;
+        a.flags = reinterpret_cast<unsigned int*>(extra + tc_units(d) * (TC_STATE_BYTES + TC_DELTA_BYTES));
         return cuda_status(chunk_bwd_launch(a, s), "gdn2_bwd (tensor-core path)");
     }
 

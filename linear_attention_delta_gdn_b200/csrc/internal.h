@@ -33,6 +33,8 @@ constexpr size_t TC_STATE_BYTES = (size_t)TC_D * TC_D * 2;
 // bytes of one WY image per chunk: T and P (bf16 64 x 64 tiles), then Wm (bf16 64 x 128 tile)
 constexpr size_t TC_TP_BYTES = (size_t)2 * TC_C * TC_C * 2;
 constexpr size_t TC_WY_BYTES = TC_TP_BYTES + (size_t)TC_C * TC_D * 2;
+// bytes of one saved Delta^T (forward) or dDelta^T (backward) image: bf16 128 x 64 row tile
+constexpr size_t TC_DELTA_BYTES = (size_t)TC_D * TC_C * 2;
 
 struct ChunkFwdArgs {
     Dims d;
@@ -41,6 +43,7 @@ struct ChunkFwdArgs {
     void* o;               // may be null: states only
     float* ST;
     unsigned char* states; // [B,H,NC] chunk-start state images, or null
+    unsigned char* deltas; // [B,H,NC] Delta^T images (with states), or null
     unsigned char* wy;     // [B,H,NC] WY images (T | P | Wm), always written
     unsigned int* flags;   // [B,H,NC] ready flags (scratch)
 };
@@ -53,8 +56,10 @@ struct ChunkBwdArgs {
     void *dq, *dk, *dv, *dla, *db, *dw;
     float* dS0;
     const unsigned char* states;  // [B,H,NC] chunk-start state images
+    const unsigned char* deltas;  // [B,H,NC] Delta^T images saved by the forward
     const unsigned char* tp;      // [B,H,NC] WY images (T | P | Wm) of every chunk
     unsigned char* dstates;       // [B,H,NC] images of Diag(gC) dL/dS' per chunk (scratch)
+    unsigned char* ddeltas;       // [B,H,NC] dDelta^T images (scratch)
     unsigned int* flags;          // [B,H,NC] ready flags, then work counter and abort word (scratch)
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);

@@ -53,15 +53,16 @@ def test_workspace_sizes(L):
     assert fs >= 1 * 2 * 4 * 64 * 64 * 4 and fs % 256 == 0
     assert ws(2, 1, 256, 2, 64, 64, 64, 0) > fs
     # bf16 shape of the 1.3B training layer: the inference forward keeps a WY image
-    # (T | P | Wm, 32 KB) and a ready flag per chunk; training adds the state images;
-    # the backward adds the dZ images, its ready flags and one work counter
+    # (T | P | Wm, 32 KB) and a ready flag per chunk; training adds the state (32 KB) and
+    # Delta (16 KB) images; the backward adds the dZ (32 KB) and dDelta (16 KB) images, its
+    # ready flags, a work counter and an abort word
     units = 4 * 16 * 64
     i = ws(0, 4, 4096, 16, 128, 128, 64, 1)
     assert i == units * 32768 + units * 4
     f = ws(1, 4, 4096, 16, 128, 128, 64, 1)
     b = ws(2, 4, 4096, 16, 128, 128, 64, 1)
-    assert f == units * 32768 + i
-    assert b == f + units * 32768 + (units * 4 + 256)
+    assert f == units * (32768 + 16384) + i
+    assert b == f + units * (32768 + 16384) + (units * 4 + 256)
     # ragged T rounds the chunk count up
     assert ws(1, 1, 65, 1, 128, 128, 64, 1) == ws(1, 1, 128, 1, 128, 128, 64, 1)
     # invalid problems report zero
