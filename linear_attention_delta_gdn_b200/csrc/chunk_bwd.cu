@@ -113,10 +113,10 @@ __device__ __forceinline__ void prep_qk4(unsigned char* QQ, const unsigned char*
 // 16 qt .. 16 qt + 15):
 //   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127)
 //   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT (k stays in KH);
-//   G[t][i] goes to TMEM at tmem_g (lane i, column t). Quarter sums of log_alpha are exchanged
-//   through qsum (fp32 [4][128]). Contains one __syncthreads.
+//   g[t][i] = exp(G) and 1/g go to TMEM at tmem_g and tmem_ig (lane i, column t) for the gate chain.
+//   Quarter sums of log_alpha are exchanged through qsum (fp32 [4][128]). Contains one __syncthreads.
 __device__ __forceinline__ void grad_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
-                                          float* qsum, int tid, uint32_t tmem_g) {
+                                          float* qsum, int tid, uint32_t tmem_g, uint32_t tmem_ig) {
     const int i = tid & 127, qt = tid >> 7;
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
@@ -134,7 +134,7 @@ __device__ __forceinline__ void grad_prep(unsigned char* QE, const unsigned char
     float G = 0.f;
 #pragma unroll 1
     for (int q = 0; q < qt; ++q) G += qsum[q * 128 + i];
-    float gvals[16];
+    float gvals[16], igvals[16];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         float kk[8], bb[8], qq[8];
@@ -152,14 +152,16 @@ __device__ __forceinline__ void grad_prep(unsigned char* QE, const unsigned char
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             G += la[8 * half + u];
-            gvals[8 * half + u] = G;
             const float g = fast_exp(G), ig = fast_exp(-G);
+            gvals[8 * half + u] = g;
+            igvals[8 * half + u] = ig;
             tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);          // Et
             tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);        // Qt
             tc::st_bf16(KT, o64[u], kk[u] * ig);                  // Kt
         }
     }
     tc::tmem_st16(tmem_g + 16 * qt, gvals);
+    tc::tmem_st16(tmem_ig + 16 * qt, igvals);
     tc::tmem_wait_st();
 }
 
@@ -171,7 +173,7 @@ constexpr uint32_t OFF_BARS = 229888;
 constexpr uint32_t SMEM_BYTES_ALL = 229952 + 1024;
 
 struct BwdMaps {
-    CUtensorMap q, k, v, la, b, w, dout, dq, dk, db, dla;
+    CUtensorMap q, k, v, la, b, w, dout, dq, dk, db, dla, dv, dw;
 };
 struct BwdParams {
     int T, H, BH, nc;
@@ -428,7 +430,8 @@ constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_W = 64,                     // dA^T (M=64, 64 columns)
     TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
     TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,   // G3 = dKt^T (P and A paths), G4 = (Delta dZ^T)^T
-    TM_GV = 448;                   // G[t] per key channel (cumulative log-decay)
+    TM_GV = 448,                   // g[t] = exp(G) per key channel
+    TM_IGV = 128;                  // 1/g[t]
 constexpr uint32_t LOAD_TOK = 7 * 64 * 128 * 2 + (uint32_t)TC_DELTA_BYTES;   // 7 token tiles, Delta^T
 constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dZ^T: cp.async)
 }  // namespace cg
@@ -467,8 +470,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const int L = min(C, T - t0);
     const CUtensorMap *mq = &m.q, *mk = &m.k, *mv = &m.v, *mla = &m.la, *mb = &m.b, *mw = &m.w, *mdo = &m.dout;
     const CUtensorMap *mdq = &m.dq, *mdk = &m.dk, *mdb = &m.db, *mdla = &m.dla;
-    __nv_bfloat16* __restrict__ dv = p.dv;
-    __nv_bfloat16* __restrict__ dw = p.dw;
 
     bool ok = true;
     int next_unit = units;    // thread 0: the CTA's next unit (its atomic returns while this unit runs)
@@ -550,7 +551,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
     // ---- factors (G kept in TMEM)
-    grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV);   // PP: scratch until dP^T
+    grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV, lane_base + TM_IGV);   // PP: scratch
     sync_for_mma();
 
     // ---- dU = T^T dDelta (M=64)
@@ -563,40 +564,38 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    {   // dv = dU*w, dw = dU*v (rows t; v, w from shared memory); dU replaces v as a bf16 row tile
+    {   // dv = dU*w -> DDT, dw = dU*v -> TT|PP (bf16 row tiles for TMA stores; the dU MMA has read T
+        // and dDelta^T, the prep its scratch); dU replaces v as a bf16 row tile
         const int t = m64_row(warp, lane);
-        const bool row_ok = lane < 16 && t < L;
         float v[32];
-#pragma unroll 1
-        for (int c0 = cpart; c0 < cpart + 32; c0 += 32) {
-            tc::tmem_ld32(lane_base + TM_DU + c0, v);
-            tc::tmem_wait_ld();
-            if (lane < 16) {
-                uint4* dvp = reinterpret_cast<uint4*>(dv + tok_off(b, t0 + (row_ok ? t : 0), h, T, H, D) + c0);
-                uint4* dwp = reinterpret_cast<uint4*>(dw + tok_off(b, t0 + (row_ok ? t : 0), h, T, H, D) + c0);
+        const int c0 = cpart;
+        tc::tmem_ld32(lane_base + TM_DU + c0, v);
+        tc::tmem_wait_ld();
+        if (lane < 16) {
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float vv[8], ww[8];
-                    tc::ld_row8(UU, C, t, (c0 >> 3) + g, vv);
-                    tc::ld_row8(WW, C, t, (c0 >> 3) + g, ww);
-                    uint32_t ov[4], ow[4];
+            for (int g = 0; g < 4; ++g) {
+                float vv[8], ww[8], ov[8], ow[8];
+                tc::ld_row8(UU, C, t, (c0 >> 3) + g, vv);
+                tc::ld_row8(WW, C, t, (c0 >> 3) + g, ww);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float d0 = v[8 * g + 2 * e], d1 = v[8 * g + 2 * e + 1];
-                        ov[e] = tc::pack_bf16x2(d0 * ww[2 * e], d1 * ww[2 * e + 1]);
-                        ow[e] = tc::pack_bf16x2(d0 * vv[2 * e], d1 * vv[2 * e + 1]);
-                    }
-                    if (row_ok) {
-                        dvp[g] = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-                        dwp[g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    }
-                    tc::st_row8(UU, C, t, (c0 >> 3) + g, v + 8 * g);
+                for (int e = 0; e < 8; ++e) {
+                    ov[e] = v[8 * g + e] * ww[e];
+                    ow[e] = v[8 * g + e] * vv[e];
                 }
+                tc::st_row8(DDT, C, t, (c0 >> 3) + g, ov);
+                tc::st_row8(TT, C, t, (c0 >> 3) + g, ow);     // TT and PP form one 64 x 128 tile
+                tc::st_row8(UU, C, t, (c0 >> 3) + g, v + 8 * g);
             }
         }
     }
     sync_for_mma();
-    if (tid == 0) {     // w is consumed: bring b back for the gate chain
+    if (tid == 0) {     // store dv, dw (rows past the end of the sequence are skipped); bring b back for
+                        // the gate chain (w is consumed)
+        tc::tma_store_4d(&m.dv, 0, h, t0, b, DDT);
+        tc::tma_store_4d(&m.dv, 64, h, t0, b, DDT + C * 128);
+        tc::tma_store_4d(&m.dw, 0, h, t0, b, TT);
+        tc::tma_store_4d(&m.dw, 64, h, t0, b, TT + C * 128);
+        tc::bulk_commit();
         tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
         tma_tile(WW, C, 0, mb, b, h, t0, bar_b);
     }
@@ -612,8 +611,12 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             tc::mma_bf16(tmem + TM_W, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sUU, C, 0, kk), id_a, kk > 0);
         }
         tc::mma_commit(bar_mma);
+        tc::bulk_wait_read();   // the dv, dw stores have read their tiles (TT, PP are overwritten below)
     }
     wait_mma();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
     {   // M=64 accumulators: rows s = 16 q + lane (lanes < 16); the warps of a quarter take 16 columns each
         const int s_ = m64_row(warp, lane), c0 = 16 * tm_part(warp);
         float v[16];
@@ -695,12 +698,13 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     float dG[16];
     float dGsum = 0.f;
     {
-        float g1[16], g2[16], g3[16], g4[16], gv[16];
+        float g1[16], g2[16], g3[16], g4[16], gv[16], igv[16];
         tc::tmem_ld16(lane_base + TM_G1 + 16 * qt, g1);
         tc::tmem_ld16(lane_base + TM_G2 + 16 * qt, g2);
         tc::tmem_ld16(lane_base + TM_G3 + 16 * qt, g3);
         tc::tmem_ld16(lane_base + TM_G4 + 16 * qt, g4);
         tc::tmem_ld16(lane_base + TM_GV + 16 * qt, gv);
+        tc::tmem_ld16(lane_base + TM_IGV + 16 * qt, igv);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
@@ -711,7 +715,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             const float kt = tc::ld_bf16(KT, col64 + sw);
             const float kk = tc::ld_bf16(KH, col64 + sw);
             const float bb = tc::ld_bf16(WW, col64 + sw);
-            const float g = fast_exp(gv[u]), ig = fast_exp(-gv[u]);
+            const float g = gv[u], ig = igv[u];
             const float dKt = g3[u] + g4[u];
             const float dGt = qv * g1[u] + et * g2[u] - kt * dKt;
             dG[u] = dGt;
@@ -846,10 +850,10 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
     BwdMaps maps;
-    const void* ptrs[11] = {a.q, a.k, a.v, a.la, a.b, a.w, a.dout, a.dq, a.dk, a.db, a.dla};
-    CUtensorMap* mp[11] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w, &maps.dout,
-                           &maps.dq, &maps.dk, &maps.db, &maps.dla};
-    for (int i = 0; i < 11; ++i)
+    const void* ptrs[13] = {a.q, a.k, a.v, a.la, a.b, a.w, a.dout, a.dq, a.dk, a.db, a.dla, a.dv, a.dw};
+    CUtensorMap* mp[13] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w, &maps.dout,
+                           &maps.dq, &maps.dk, &maps.db, &maps.dla, &maps.dv, &maps.dw};
+    for (int i = 0; i < 13; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     cudaError_t e = set_smem(chunk_bwd_kernel, SMEM_BYTES_ALL);
     if (e != cudaSuccess) return e;
