@@ -416,15 +416,15 @@ namespace cg {
 constexpr uint32_t OFF_QE = 0;           // rows 0..63: b -> Et, rows 64..127: q -> Qt
 constexpr uint32_t OFF_KH = 32768;       // k
 constexpr uint32_t OFF_KT = 49152;       // log_alpha -> Kt
-constexpr uint32_t OFF_UU = 65536;       // v, later dU rows [t][j], later staged dlog_alpha
-constexpr uint32_t OFF_WW = 81920;       // w, later b (reloaded)
-constexpr uint32_t OFF_DO = 98304;       // dout, later staged dq
+constexpr uint32_t OFF_DU = 65536;       // [128 x 128]: rows 0..63 dout (later staged dq), rows 64..127
+                                         // v -> -dU (later staged dlog_alpha): one N = 128 operand
+constexpr uint32_t OFF_WW = 98304;       // w, later b (reloaded)
 constexpr uint32_t OFF_ST = 114688;      // S^T image (chunk start)
 constexpr uint32_t OFF_DS = 147456;      // dZ^T image
 constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64] (forward image), later staged dk
 constexpr uint32_t OFF_DDT = 196608;     // dDelta^T [128 x 64] (reverse-pass image), later staged db
-constexpr uint32_t OFF_TT = 212992;      // T, later dA^T [64 x 64]
-constexpr uint32_t OFF_PP = 221184;      // prep scratch, then dP^T [64 x 64]
+constexpr uint32_t OFF_PP = 212992;      // prep scratch, then dP^T [64 x 64]; with TT: dw staging, and
+constexpr uint32_t OFF_TT = 221184;      // T, later dA^T   [dP^T | dA^T] as one N = 128 operand
 // TMEM columns (M=64 accumulators use lanes 0-15 of each 32-lane quarter)
 constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_W = 64,                     // dA^T (M=64, 64 columns)
@@ -447,9 +447,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     unsigned char* QE = sm + OFF_QE;
     unsigned char* KH = sm + OFF_KH;
     unsigned char* KT = sm + OFF_KT;
-    unsigned char* UU = sm + OFF_UU;
+    unsigned char* DU = sm + OFF_DU;
     unsigned char* WW = sm + OFF_WW;
-    unsigned char* DO = sm + OFF_DO;
     unsigned char* STt = sm + OFF_ST;
     unsigned char* DS = sm + OFF_DS;
     unsigned char* DT = sm + OFF_DT;
@@ -488,9 +487,9 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         case 1: tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load); break;
         case 2: tma_tile(KH, C, 0, mk, b, h, t0, bar_load); break;
         case 3: tma_tile(KT, C, 0, mla, b, h, t0, bar_load); break;
-        case 4: tma_tile(UU, C, 0, mv, b, h, t0, bar_load); break;
+        case 4: tma_tile(DU, 2 * C, C, mv, b, h, t0, bar_load); break;
         case 5: tma_tile(WW, C, 0, mw, b, h, t0, bar_load); break;
-        case 6: tma_tile(DO, C, 0, mdo, b, h, t0, bar_load); break;
+        case 6: tma_tile(DU, 2 * C, 0, mdo, b, h, t0, bar_load); break;
         case 7:
             tc::bulk_load(DT, p.deltas + (head * nc + c) * TC_DELTA_BYTES, (uint32_t)TC_DELTA_BYTES, bar_load);
             break;
@@ -546,7 +545,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     };
 
     const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT),
-                   sUU = tc::smem_u32(UU), sDO = tc::smem_u32(DO), sST = tc::smem_u32(STt),
+                   sDU = tc::smem_u32(DU), sST = tc::smem_u32(STt),
                    sDS = tc::smem_u32(DS), sDT = tc::smem_u32(DT), sDDT = tc::smem_u32(DDT),
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
@@ -564,8 +563,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mma_commit(bar_mma);
     }
     wait_mma();
-    {   // dv = dU*w -> DDT, dw = dU*v -> TT|PP (bf16 row tiles for TMA stores; the dU MMA has read T
-        // and dDelta^T, the prep its scratch); dU replaces v as a bf16 row tile
+    {   // dv = dU*w -> DDT, dw = dU*v -> PP|TT (bf16 row tiles for TMA stores; the dU MMA has read T
+        // and dDelta^T, the prep its scratch); -dU replaces v
         const int t = m64_row(warp, lane);
         float v[32];
         const int c0 = cpart;
@@ -574,17 +573,19 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         if (lane < 16) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-                float vv[8], ww[8], ov[8], ow[8];
-                tc::ld_row8(UU, C, t, (c0 >> 3) + g, vv);
-                tc::ld_row8(WW, C, t, (c0 >> 3) + g, ww);
+                float x[8], y[8];
+                const float* d = v + 8 * g;
+                tc::ld_row8(WW, C, t, (c0 >> 3) + g, x);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    ov[e] = v[8 * g + e] * ww[e];
-                    ow[e] = v[8 * g + e] * vv[e];
-                }
-                tc::st_row8(DDT, C, t, (c0 >> 3) + g, ov);
-                tc::st_row8(TT, C, t, (c0 >> 3) + g, ow);     // TT and PP form one 64 x 128 tile
-                tc::st_row8(UU, C, t, (c0 >> 3) + g, v + 8 * g);
+                for (int e = 0; e < 8; ++e) y[e] = d[e] * x[e];
+                tc::st_row8(DDT, C, t, (c0 >> 3) + g, y);            // dv
+                tc::ld_row8(DU, 2 * C, C + t, (c0 >> 3) + g, x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = d[e] * x[e];
+                tc::st_row8(PP, C, t, (c0 >> 3) + g, y);             // dw (PP and TT form one 64 x 128 tile)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = -d[e];
+                tc::st_row8(DU, 2 * C, C + t, (c0 >> 3) + g, y);     // -dU over v
             }
         }
     }
@@ -593,8 +594,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
                         // the gate chain (w is consumed)
         tc::tma_store_4d(&m.dv, 0, h, t0, b, DDT);
         tc::tma_store_4d(&m.dv, 64, h, t0, b, DDT + C * 128);
-        tc::tma_store_4d(&m.dw, 0, h, t0, b, TT);
-        tc::tma_store_4d(&m.dw, 64, h, t0, b, TT + C * 128);
+        tc::tma_store_4d(&m.dw, 0, h, t0, b, PP);
+        tc::tma_store_4d(&m.dw, 64, h, t0, b, PP + C * 128);
         tc::bulk_commit();
         tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
         tma_tile(WW, C, 0, mb, b, h, t0, bar_b);
@@ -603,12 +604,11 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     // ---- dP^T = Delta dO^T (M=64), dA^T = -Delta dU^T (M=64)
     if (tid == 0) {
         tc::tc_fence_after();
-        constexpr uint32_t id_p = tc::idesc_bf16(64, 64, true, false);
-        constexpr uint32_t id_a = tc::idesc_bf16(64, 64, true, false, true);
+        constexpr uint32_t id_pa = tc::idesc_bf16(64, 64, true, false);   // the tile holds -dU: no negation
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_bf16(tmem + TM_AP, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sDO, C, 0, kk), id_p, kk > 0);
-            tc::mma_bf16(tmem + TM_W, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sUU, C, 0, kk), id_a, kk > 0);
+            tc::mma_bf16(tmem + TM_AP, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sDU, 2 * C, 0, kk), id_pa, kk > 0);
+            tc::mma_bf16(tmem + TM_W, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sDU, 2 * C, C, kk), id_pa, kk > 0);
         }
         tc::mma_commit(bar_mma);
         tc::bulk_wait_read();   // the dv, dw stores have read their tiles (TT, PP are overwritten below)
@@ -641,21 +641,22 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
 
     // ---- G1 = dQt^T = S dO^T + Kt^T dP^T ; G2 = dEt^T = -S dU^T + Kt^T dA^T
     //      G3 = Qt^T dP + Et^T dA ;        G4 = dZ Delta^T          (all [key channel i][token t])
+    // G1 and G2 (adjacent in TMEM) share their A operands: [G1 | G2] = S [dO; -dU]^T + Kt^T [dP^T | dA^T]
+    // as N = 128 products (DU rows; PP and TT panels).
     if (tid == 0) {
         tc::tc_fence_after();
         constexpr uint32_t id_mk = tc::idesc_bf16(128, 64, true, false);
-        constexpr uint32_t id_mk_neg = tc::idesc_bf16(128, 64, true, false, true);
+        constexpr uint32_t id_mk2 = tc::idesc_bf16(128, 128, true, false);
         constexpr uint32_t id_mm = tc::idesc_bf16(128, 64, true, true);
+        constexpr uint32_t id_mm2 = tc::idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_bf16(tmem + TM_G1, tc::desc_mn(sST, D, 0, kk), tc::desc_k(sDO, C, 0, kk), id_mk, kk > 0);
-            tc::mma_bf16(tmem + TM_G2, tc::desc_mn(sST, D, 0, kk), tc::desc_k(sUU, C, 0, kk), id_mk_neg, kk > 0);
+            tc::mma_bf16(tmem + TM_G1, tc::desc_mn(sST, D, 0, kk), tc::desc_k(sDU, 2 * C, 0, kk), id_mk2, kk > 0);
             tc::mma_bf16(tmem + TM_G4, tc::desc_mn(sDS, D, 0, kk), tc::desc_mn(sDT, D, 0, kk), id_mm, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            tc::mma_bf16(tmem + TM_G1, tc::desc_mn(sKT, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), id_mm, 1);
-            tc::mma_bf16(tmem + TM_G2, tc::desc_mn(sKT, C, 0, kk), tc::desc_mn(sTT, C, 0, kk), id_mm, 1);
+            tc::mma_bf16(tmem + TM_G1, tc::desc_mn(sKT, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), id_mm2, 1);
             tc::mma_bf16(tmem + TM_G3, tc::desc_mn(sQE, 2 * C, C, kk), tc::desc_k(sPP, C, 0, kk), id_mk, kk > 0);
         }
 #pragma unroll
@@ -691,24 +692,27 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     // ---- gate chain, thread = (key channel i, token quarter qt: tokens 16 qt .. 16 qt + 15). Pass 1: dq,
     // dk, db and dG_t; partial sums of Kt*G4 and dG are exchanged between the quarters (in the consumed
     // dP^T tile). Pass 2: dlog_alpha_t = sum_{tau >= t} dG_tau + E, E = rowsum(dZ*S) + sum_t Kt*G4.
-    // Results go to bf16 row tiles (dq -> DO, dk -> DT, db -> DDT, dlog_alpha -> UU), stored by TMA.
+    // Results go to bf16 row tiles (dq -> DU rows 0..63, dk -> DT, db -> DDT, dlog_alpha -> DU rows
+    // 64..127), stored by TMA.
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chk = (uint32_t)((i & 63) >> 3);
     float dG[16];
     float dGsum = 0.f;
-    {
-        float g1[16], g2[16], g3[16], g4[16], gv[16], igv[16];
-        tc::tmem_ld16(lane_base + TM_G1 + 16 * qt, g1);
-        tc::tmem_ld16(lane_base + TM_G2 + 16 * qt, g2);
-        tc::tmem_ld16(lane_base + TM_G3 + 16 * qt, g3);
-        tc::tmem_ld16(lane_base + TM_G4 + 16 * qt, g4);
-        tc::tmem_ld16(lane_base + TM_GV + 16 * qt, gv);
-        tc::tmem_ld16(lane_base + TM_IGV + 16 * qt, igv);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {   // two halves of 8 tokens (keeps the TMEM read-outs in registers)
+        const int tq = 16 * qt + 8 * hh;
+        float g1[8], g2[8], g3[8], g4[8], gv[8], igv[8];
+        tc::tmem_ld8(lane_base + TM_G1 + tq, g1);
+        tc::tmem_ld8(lane_base + TM_G2 + tq, g2);
+        tc::tmem_ld8(lane_base + TM_G3 + tq, g3);
+        tc::tmem_ld8(lane_base + TM_G4 + tq, g4);
+        tc::tmem_ld8(lane_base + TM_GV + tq, gv);
+        tc::tmem_ld8(lane_base + TM_IGV + tq, igv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const uint32_t t = (uint32_t)(16 * qt + u);
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t t = (uint32_t)(tq + u);
             const uint32_t sw = t * 128 + ((chk ^ (t & 7)) << 4);
             const float qv = tc::ld_bf16(QE, col128 + C * 128 + sw);
             const float et = tc::ld_bf16(QE, col128 + sw);
@@ -718,11 +722,11 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             const float g = gv[u], ig = igv[u];
             const float dKt = g3[u] + g4[u];
             const float dGt = qv * g1[u] + et * g2[u] - kt * dKt;
-            dG[u] = dGt;
+            dG[8 * hh + u] = dGt;
             dGsum += dGt;
             Epart += kt * g4[u];
             const float dE = g * g2[u];
-            tc::st_bf16(DO, col64 + sw, g * g1[u]);                 // dq
+            tc::st_bf16(DU, col128 + sw, g * g1[u]);                // dq
             tc::st_bf16(DT, col64 + sw, dKt * ig + dE * bb);        // dk
             tc::st_bf16(DDT, col64 + sw, dE * kk);                  // db
         }
@@ -762,17 +766,18 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     for (int u = 15; u >= 0; --u) {
         const uint32_t t = (uint32_t)(16 * qt + u);
         suffix += dG[u];
-        tc::st_bf16(UU, col64 + t * 128 + ((chk ^ (t & 7)) << 4), suffix + E);    // dlog_alpha
+        tc::st_bf16(DU, col128 + C * 128 + t * 128 + ((chk ^ (t & 7)) << 4), suffix + E);   // dlog_alpha
     }
     tc::fence_async_smem();
     __syncthreads();
     if (tid == 0) {   // rows past the end of the sequence are skipped by the tensor store
         const CUtensorMap* maps[4] = {mdq, mdk, mdb, mdla};
-        const unsigned char* tiles[4] = {DO, DT, DDT, UU};
+        const unsigned char* tiles[4] = {DU, DT, DDT, DU + C * 128};
+        const uint32_t panel[4] = {2 * C * 128, C * 128, C * 128, 2 * C * 128};   // second 64 channels
 #pragma unroll
         for (int o = 0; o < 4; ++o) {
             tc::tma_store_4d(maps[o], 0, h, t0, b, tiles[o]);
-            tc::tma_store_4d(maps[o], 64, h, t0, b, tiles[o] + C * 128);
+            tc::tma_store_4d(maps[o], 64, h, t0, b, tiles[o] + panel[o]);
         }
         tc::bulk_commit();
         tc::bulk_wait_read();
