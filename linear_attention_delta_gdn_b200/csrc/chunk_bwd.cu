@@ -64,51 +64,6 @@ __device__ __forceinline__ void tmem_rows_to_tile(uint32_t lane_base_col, unsign
     tc::st_row8(dst, 128, row, (c0 >> 3) + 1, v + 8);
 }
 
-// Reverse-pass prep: Qt = g*q (QQ), Kt = k/g (KT over log_alpha), gC, with g = exp(G) and G the
-// inclusive in-chunk cumsum of log_alpha. Thread = (4-token block tb = tid / 32, 4-channel group
-// cg = tid % 32), 8-byte shared-memory accesses; block totals are exchanged through red
-// (fp32 [16][128]). Contains one __syncthreads.
-__device__ __forceinline__ void prep_qk4(unsigned char* QQ, const unsigned char* KH, unsigned char* KT,
-                                         float* gC_out, float* red, int tid) {
-    const int cg = tid & 31, tb = tid >> 5;
-    float G[4][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        tc::ld_row4(KT, C, 4 * tb + u, cg, G[u]);
-        if (u > 0) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) G[u][c] += G[u - 1][c];
-        }
-    }
-    *reinterpret_cast<float4*>(red + tb * 128 + 4 * cg) = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
-    __syncthreads();
-    float pre[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-    for (int q = 0; q < tb; ++q) {
-        const float4 x = *reinterpret_cast<const float4*>(red + q * 128 + 4 * cg);
-        pre[0] += x.x; pre[1] += x.y; pre[2] += x.z; pre[3] += x.w;
-    }
-    if (tb == C / 4 - 1) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) gC_out[4 * cg + c] = fast_exp(pre[c] + G[3][c]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int row = 4 * tb + u;
-        float kk[4], qq[4];
-        tc::ld_row4(KH, C, row, cg, kk);
-        tc::ld_row4(QQ, C, row, cg, qq);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const float Gv = pre[c] + G[u][c];
-            kk[c] *= fast_exp(-Gv);
-            qq[c] *= fast_exp(Gv);
-        }
-        tc::st_row4(KT, C, row, cg, kk);
-        tc::st_row4(QQ, C, row, cg, qq);
-    }
-}
-
 // Gradient-unit prep, thread = (key channel i = tid % 128, token quarter qt = tid / 128: tokens
 // 16 qt .. 16 qt + 15):
 //   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127)
@@ -204,35 +159,31 @@ struct NextUnit {
 // ====================================================================== reverse state pass
 
 namespace rs {
-// q, log_alpha, dout and Wm alternate between two buffers by chunk parity, so the next chunk's
-// tiles can land while this chunk's MMAs read the current ones; k and P have one buffer each.
-constexpr uint32_t OFF_QQ = 0;           // 2 x q -> Qt (64 rows), at +0 / +16384
-constexpr uint32_t OFF_KH = 32768;       // k
-constexpr uint32_t OFF_KT0 = 49152;      // log_alpha -> Kt (even chunks)
+// Qt, Kt, dout, Wm and gC alternate between two buffers by chunk parity, so the next chunk's tiles
+// can land while this chunk's MMAs read the current ones; P has one buffer. Qt, Kt, Wm, P and gC come
+// from the forward's WY image.
+constexpr uint32_t OFF_QQ = 0;           // 2 x Qt (64 rows), at +0 / +16384
+constexpr uint32_t OFF_KT0 = 49152;      // Kt (even chunks)
 constexpr uint32_t OFF_DO0 = 65536;      // dout (even chunks)
-constexpr uint32_t OFF_WW0 = 81920;      // Wm from the forward's WY image (even chunks)
+constexpr uint32_t OFF_WW0 = 81920;      // Wm (even chunks)
 constexpr uint32_t OFF_ST = 98304;       // dZ^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16)
-constexpr uint32_t OFF_PP = 147456;      // P from the forward's WY image
-constexpr uint32_t OFF_RED = 155648;     // prep scan scratch (8 KB)
+constexpr uint32_t OFF_PP = 147456;      // P
 constexpr uint32_t OFF_DO1 = 163840;     // dout (odd chunks)
 constexpr uint32_t OFF_WW1 = 180224;     // Wm (odd chunks)
-constexpr uint32_t OFF_KT1 = 196608;     // log_alpha -> Kt (odd chunks)
-constexpr uint32_t OFF_GC = 212992;
+constexpr uint32_t OFF_KT1 = 196608;     // Kt (odd chunks)
+constexpr uint32_t OFF_GC = 212992;      // 2 x fp32 gC[128] (by parity)
 constexpr uint32_t TM_S = 0, TM_D = 128;
-constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 64 * 128 * 2;   // q, log_alpha, dout, k, P, Wm
+constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 512;   // Qt, Kt, dout, Wm, P, gC
 }  // namespace rs
-static_assert(rs::OFF_GC + 512 <= OFF_BARS, "reverse-pass layout lies below the barrier block");
+static_assert(rs::OFF_GC + 1024 <= OFF_BARS, "reverse-pass layout lies below the barrier block");
 
 __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi,
                             Phases& ph) {
     using namespace rs;
-    unsigned char* KH = sm + OFF_KH;
     unsigned char* STt = sm + OFF_ST;
     unsigned char* DT = sm + OFF_DT;
     unsigned char* PP = sm + OFF_PP;
-    float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
-    float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_load + 1;
     int* abort_flag = reinterpret_cast<int*>(sm + OFF_BARS + 36);
@@ -240,6 +191,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     auto KT = [&](int c) { return sm + ((c & 1) ? OFF_KT1 : OFF_KT0); };
     auto DO = [&](int c) { return sm + ((c & 1) ? OFF_DO1 : OFF_DO0); };
     auto WW = [&](int c) { return sm + ((c & 1) ? OFF_WW1 : OFF_WW0); };
+    auto GC = [&](int c) { return reinterpret_cast<float*>(sm + OFF_GC + (c & 1) * 512); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = headi % p.H, b = headi / p.H;
@@ -249,30 +201,26 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 32 * tm_part(warp);      // lane row, column quarter
 
     // chunk c's tiles arrive on one barrier phase, issued in three groups as their buffers free up
-    // q, log_alpha, dout, Wm (buffers of this parity are free): issued by lane 0 of warps 0-3 at once
+    // dout, Qt, Kt, Wm, gC (buffers of this parity are free): issued by lane 0 of warps 0-4 at once
     auto issue_first = [&](int c) {
-        if (lane != 0 || warp > 3) return;
-        const int t0 = c * C;
-        if (warp == 0) {
+        if (lane != 0 || warp > 4) return;
+        const unsigned char* img = p.tp + (head * nc + c) * TC_WY_BYTES;
+        switch (warp) {
+        case 0:
             tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-            tma_tile(QQ(c), C, 0, &m.q, b, h, t0, bar_load);
-        } else if (warp == 1) {
-            tma_tile(KT(c), C, 0, &m.la, b, h, t0, bar_load);
-        } else if (warp == 2) {
-            tma_tile(DO(c), C, 0, &m.dout, b, h, t0, bar_load);
-        } else {
-            tc::bulk_load(WW(c), p.tp + (head * nc + c) * TC_WY_BYTES + 2 * TILE_C, 64 * 128 * 2, bar_load);
+            tma_tile(DO(c), C, 0, &m.dout, b, h, c * C, bar_load);
+            break;
+        case 1: tc::bulk_load(QQ(c), img + TC_WY_QT, 64 * 128 * 2, bar_load); break;
+        case 2: tc::bulk_load(KT(c), img + TC_WY_KT, 64 * 128 * 2, bar_load); break;
+        case 3: tc::bulk_load(WW(c), img + TC_WY_WM, 64 * 128 * 2, bar_load); break;
+        default: tc::bulk_load(GC(c), img + TC_WY_GC, 512, bar_load); break;
         }
     };
-    auto issue_k = [&](int c) { tma_tile(KH, C, 0, &m.k, b, h, c * C, bar_load); };   // after the prep
     auto issue_p = [&](int c) {   // after the MMAs that read P
         tc::bulk_load(PP, p.tp + (head * nc + c) * TC_WY_BYTES + TILE_C, TILE_C, bar_load);
     };
     issue_first(nc - 1);
-    if (tid == 0) {
-        issue_k(nc - 1);
-        issue_p(nc - 1);
-    }
+    if (tid == 0) issue_p(nc - 1);
 
     {   // dS_{NC}^T = dST^T (or zero): lane j holds column j of dST
         const int j = jrow;
@@ -315,10 +263,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         // the other parity's buffers were last read by chunk c + 1, whose MMAs are complete
         if (c > 0) issue_first(c - 1);
 
-        prep_qk4(QQ(c), KH, KT(c), sGC, sRed, tid);   // Qt, Kt, gC
-        tc::fence_async_smem();   // the prep's reads of k precede the TMA that overwrites it
-        __syncthreads();
-        if (tid == 0 && c > 0) issue_k(c - 1);
+        const float* sGC = GC(c);   // Qt, Kt, gC came with the forward's WY image
         // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
         {
             const int j = jrow;

@@ -37,18 +37,16 @@ using namespace chunk;
 
 // ---- consumer (state pass) shared memory, bytes from a 1024-aligned base
 namespace sp {
-constexpr uint32_t QQ = 0;          // 2 x [64 x 128] q -> Qt (by chunk parity)
-constexpr uint32_t KT = 32768;      // 2 x [64 x 128] log_alpha -> Kt (by chunk parity)
-constexpr uint32_t KH = 65536;      // [64 x 128] k
-constexpr uint32_t UU = 81920;      // [64 x 128] v -> U
-constexpr uint32_t WW = 98304;      // [64 x 128] w
-constexpr uint32_t WY = 114688;     // WY image: T [64 x 64] | P [64 x 64] | Wm [64 x 128]
+constexpr uint32_t QQ = 0;          // 2 x [64 x 128] Qt from the WY image (by chunk parity)
+constexpr uint32_t KT = 32768;      // 2 x [64 x 128] Kt from the WY image (by chunk parity)
+constexpr uint32_t UU = 65536;      // [64 x 128] v -> U
+constexpr uint32_t WW = 81920;      // [64 x 128] w
+constexpr uint32_t WY = 98304;      // WY image head: T [64 x 64] | P [64 x 64] | Wm [64 x 128]
 constexpr uint32_t TT = WY, PP = WY + 8192, WM = WY + 16384;
-constexpr uint32_t ST = 147456;     // [128 x 128] S^T (bf16)
-constexpr uint32_t DT = 180224;     // [128 x 64] Delta^T (bf16)
-constexpr uint32_t RED = 196608;    // fp32 [16][128] prep scan scratch
-constexpr uint32_t GC = 204800;     // fp32 gC[128]
-constexpr uint32_t BAR = 205312;    // 3 mbarriers (load, mma, unused), tmem base, abort flag
+constexpr uint32_t ST = 131072;     // [128 x 128] S^T (bf16)
+constexpr uint32_t DT = 163840;     // [128 x 64] Delta^T (bf16)
+constexpr uint32_t GC = 180224;     // 2 x fp32 gC[128] from the WY image (by chunk parity)
+constexpr uint32_t BAR = 181248;    // 3 mbarriers (load, mma, unused), tmem base, abort flag
 }  // namespace sp
 // ---- producer (WY) shared memory: two input stages, then the solve scratch and the WY image
 namespace wy {
@@ -60,17 +58,18 @@ constexpr uint32_t SX = 163840;     // solve temporaries, 12 KB
 constexpr uint32_t IMG = 176128;    // WY image: T | P | Wm (32 KB)
 constexpr uint32_t TT = IMG, PP = IMG + 8192, WM = IMG + 16384;
 constexpr uint32_t BAR = 208896;    // 3 mbarriers (2 stages, mma), tmem base, abort flag
+constexpr uint32_t GC = 208960;     // 2 x fp32 gC[128] (by stage)
 }  // namespace wy
-constexpr uint32_t SMEM_BYTES = 208960 + 1024;
+constexpr uint32_t SMEM_BYTES = 209984 + 1024;
 static_assert(sp::BAR + 64 <= wy::BAR + 64, "consumer layout fits");
-static_assert(TC_WY_BYTES == 32768, "WY image = T | P | Wm");
+static_assert(TC_WY_QT == 32768 && TC_WY_KT == 49152 && TC_WY_GC == 65536, "WY image: T | P | Wm | Qt | Kt | gC");
 
 // TMEM columns. Consumer: S^T (fp32 state), Ut^T -> Delta^T, O x 2 (M=64). Producer: [A; P], Wm (M=64).
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 256;   // O: two buffers of 128 columns (chunk parity)
 constexpr uint32_t TM_AP = 0, TM_W = 128;
 constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t CONS_LOAD_BYTES = 5 * 64 * 128 * 2;
+constexpr uint32_t CONS_LOAD_BYTES = 2 * 64 * 128 * 2;   // v, w
 constexpr uint32_t PROD_LOAD_BYTES = 4 * 64 * 128 * 2;
 
 __device__ unsigned int g_fwd_error;
@@ -115,24 +114,37 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
     const int units = p.BH * p.nc;
 
-    // the four tiles of unit u, issued by lane 0 of warps 0-3 at once (a TMA issue takes ~100 cycles)
-    auto issue_loads = [&](int stage, int u) {
-        if (lane != 0 || warp > 3) return;
+    // The four tiles of unit u, issued by lane 0 of warps 0-2 (a TMA issue takes ~100 cycles). q and
+    // log_alpha land on Qt and Kt of the stage, which the previous image stores read: thread 32 issues
+    // them (part 2) only after waiting for those reads.
+    auto tile_coords = [&](int u, int& b, int& h, int& t0) {
         const int c = u / p.BH, head = u % p.BH;
-        const int b = head / p.H, h = head % p.H, t0 = c * C;
+        b = head / p.H; h = head % p.H; t0 = c * C;
+    };
+    auto issue_loads_1 = [&](int stage, int u) {
+        if (lane != 0 || (warp != 0 && warp != 2)) return;
+        int b, h, t0;
+        tile_coords(u, b, h, t0);
         unsigned char* base = sm + stage * wy::STAGE;
         if (warp == 0) {
             tc::mbar_arrive_expect_tx(&bar_in[stage], PROD_LOAD_BYTES);
             tma_tile(base + wy::QE, 2 * C, 0, &m.b, b, h, t0, &bar_in[stage]);
-        } else if (warp == 1) {
-            tma_tile(base + wy::QE, 2 * C, C, &m.q, b, h, t0, &bar_in[stage]);
-        } else if (warp == 2) {
-            tma_tile(base + wy::KH, C, 0, &m.k, b, h, t0, &bar_in[stage]);
         } else {
-            tma_tile(base + wy::KT, C, 0, &m.la, b, h, t0, &bar_in[stage]);
+            tma_tile(base + wy::KH, C, 0, &m.k, b, h, t0, &bar_in[stage]);
         }
     };
-    if (pid < units) issue_loads(0, pid);
+    auto issue_loads_2 = [&](int stage, int u) {   // lane 0 of warps 1 and 2
+        if (lane != 0 || (warp != 1 && warp != 2)) return;
+        int b, h, t0;
+        tile_coords(u, b, h, t0);
+        unsigned char* base = sm + stage * wy::STAGE;
+        if (warp == 1) tma_tile(base + wy::QE, 2 * C, C, &m.q, b, h, t0, &bar_in[stage]);
+        else tma_tile(base + wy::KT, C, 0, &m.la, b, h, t0, &bar_in[stage]);
+    };
+    if (pid < units) {
+        issue_loads_1(0, pid);
+        issue_loads_2(0, pid);
+    }
 
     uint32_t ph_in = 0, ph_mma = 0;   // ph_in: bit s = phase parity of input stage s
     auto wait_mma = [&]() {
@@ -142,18 +154,26 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     };
     int stage = 0;
     bool pending = false;   // a prefetch into the other stage is in flight (thread 0's view)
-    long long unreleased = -1;   // unit whose WY image is written but whose flag is not yet set
+    // The WY image of a unit is written by bulk stores that thread 32 issues at the end of the unit; the
+    // same thread sets the unit's flag one unit later (once the stores are complete) and, before any
+    // tile they read is overwritten, waits until they have read it.
+    long long unreleased = -1;   // unit whose WY image is being written but whose flag is not yet set
     for (int u = pid; u < units; u += p.nprod, stage ^= 1) {
         const int c = u / p.BH, head = u % p.BH;
         unsigned char* base = sm + stage * wy::STAGE;
         unsigned char* QE = base + wy::QE;
         if (!tc::mbar_wait(&bar_in[stage], (ph_in >> stage) & 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
         ph_in ^= 1u << stage;
-        // the other stage was last read by the previous unit's MMAs, which have completed
+        // the other stage was last read by the previous unit's MMAs, which have completed, and by its image
+        // stores: b and k do not overlap what those read; q and log_alpha follow below
         pending = u + p.nprod < units;
-        if (pending) issue_loads(stage ^ 1, u + p.nprod);
+        if (pending) issue_loads_1(stage ^ 1, u + p.nprod);
 
-        gate_prep(QE, base + wy::KH, base + wy::KT, nullptr, nullptr, nullptr, sA, tid, true, false);
+        gate_prep(QE, base + wy::KH, base + wy::KT, nullptr, nullptr, reinterpret_cast<float*>(sm + wy::GC + stage * 512),
+                  sA, tid, true, false);
+        // the previous image stores have read T | P | Wm (rewritten after this barrier) and the other
+        // stage's Qt, Kt (reloaded below)
+        if (tid == 32) tc::bulk_wait_read();
         sync_for_mma();
         const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(base + wy::KT);
         if (tid == 0) {   // [A; P] = [Et; Qt] Kt^T
@@ -163,9 +183,11 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
                 tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
             tc::mma_commit(bar_mma);
         }
-        // the previous unit's image stores have drained during this unit's prep: set its flag now,
-        // from a thread outside the MMA-issuing warp, while M1 runs
-        if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
+        // while M1 runs, warps 1 and 2 (outside the MMA-issuing warp) issue the prefetch's q and log_alpha
+        // (the image stores have read the tiles they overwrite: thread 32 waited before the barrier), and
+        // thread 32 sets the previous unit's flag (its image stores have completed during this unit's prep)
+        if (pending) issue_loads_2(stage ^ 1, u + p.nprod);
+        if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk(p.flags + unreleased, 1u);
         unreleased = -1;
         wait_mma();
         extract_AP(lane_base + TM_AP, sA, PP, true, warp, lane);
@@ -182,20 +204,29 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         }
         wait_mma();
         tmem_m64_to_tile(lane_base + TM_W, WM, warp, lane);
+        tc::fence_async_smem();   // the tiles written by threads are read by the image's bulk stores
         tc::tc_fence_before();
         __syncthreads();
-        // publish the WY image of (head, c)
+        // the WY image of (head, c): T | P | Wm, then Qt (rows 64..127 of the [b; q] tile, whose two 64-channel
+        // panels are 16 KB apart), Kt and gC, by bulk stores
         const size_t unit = (size_t)head * p.nc + c;
-        uint4* dst = reinterpret_cast<uint4*>(p.wyimg + unit * TC_WY_BYTES);
-        const uint4* src = reinterpret_cast<const uint4*>(sm + wy::IMG);
-#pragma unroll
-        for (int i = 0; i < (int)(TC_WY_BYTES / 16 / NT); ++i) dst[tid + NT * i] = src[tid + NT * i];
-        __syncthreads();
+        if (tid == 32) {
+            unsigned char* img = p.wyimg + unit * TC_WY_BYTES;
+            tc::bulk_store(img, sm + wy::IMG, 32768u);
+            tc::bulk_store(img + TC_WY_QT, QE + 8192, 8192u);
+            tc::bulk_store(img + TC_WY_QT + 8192, QE + 16384 + 8192, 8192u);
+            tc::bulk_store(img + TC_WY_KT, base + wy::KT, 16384u);
+            tc::bulk_store(img + TC_WY_GC, sm + wy::GC + stage * 512, 512u);
+            tc::bulk_commit();
+        }
         unreleased = (long long)unit;
         if (*abort_flag) break;
         pending = false;
     }
-    if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + unreleased, 1u);
+    if (tid == 32) {   // the last unit's flag; every image store completes before the CTA leaves
+        if (unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk(p.flags + unreleased, 1u);
+        tc::bulk_wait_all();
+    }
     // after an abort: let the prefetch in flight land before the CTA's shared memory is released
     if (tid == 0 && pending) (void)tc::mbar_wait(&bar_in[stage ^ 1], (ph_in >> (stage ^ 1)) & 1u);
 }
@@ -203,13 +234,10 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
 // ------------------------------------------------------------------ consumer
 __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int cid) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    unsigned char* KH = sm + sp::KH;
     unsigned char* UU = sm + sp::UU;
     unsigned char* WW = sm + sp::WW;
     unsigned char* STt = sm + sp::ST;
     unsigned char* DT = sm + sp::DT;
-    float* sRed = reinterpret_cast<float*>(sm + sp::RED);
-    float* sGC = reinterpret_cast<float*>(sm + sp::GC);
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + sp::BAR);
     uint64_t* bar_mma = bar_load + 1;
     int* abort_flag = reinterpret_cast<int*>(sm + sp::BAR + 28);
@@ -235,32 +263,37 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     auto wait_wy = [&](size_t head, int c) {
         if (!tc::flag_wait(p.flags + head * nc + c, 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 4u); }
     };
-    auto copy_wy = [&](size_t head, int c) {   // every thread: 8 x 16 bytes of the 32 KB image
+    // the WY image of (head, c): T | P | Wm to WY, Qt and Kt to this chunk's parity buffers, gC
+    auto copy_wy = [&](size_t head, int c) {
         const unsigned char* src = p.wyimg + (head * nc + c) * TC_WY_BYTES;
+        const int par = c & 1;
 #pragma unroll
-        for (int i = 0; i < (int)(TC_WY_BYTES / 16 / NT); ++i)
-            tc::cp_async16_cg(sm + sp::WY + 16 * (tid + NT * i), src + 16 * (tid + NT * i));
+        for (int i = 0; i < 8; ++i) {
+            const int o = 16 * (tid + NT * i);
+            tc::cp_async16_cg(sm + sp::WY + o, src + o);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int o = 16 * (tid + NT * i);
+            tc::cp_async16_cg(sm + sp::QQ + par * TILE_64x128 + o, src + TC_WY_QT + o);
+            tc::cp_async16_cg(sm + sp::KT + par * TILE_64x128 + o, src + TC_WY_KT + o);
+        }
+        if (tid < 32) tc::cp_async16_cg(sm + sp::GC + par * 512 + 16 * tid, src + TC_WY_GC + 16 * tid);
         tc::cp_async_commit();
     };
 
     for (int headi = cid; headi < p.BH; headi += p.ncons) {
         const size_t head = (size_t)headi;
         const int h = headi % H, b = headi / H;
-        // q and log_alpha tiles alternate between two buffers by chunk parity (read by the MMAs of
-        // chunk c while the tiles of chunk c + 1 arrive); k, v and w have one buffer each
-        // issued by lane 0 of warps 0-4 at once (a TMA issue takes ~100 cycles)
+        // v and w of chunk c (issued by lane 0 of warps 0 and 1 at once; a TMA issue takes ~100 cycles)
         auto issue_loads = [&](int c) {
-            if (lane != 0 || warp > 4) return;
-            const int t0 = c * C, par = c & 1;
-            switch (warp) {
-            case 0:
+            if (lane != 0 || warp > 1) return;
+            const int t0 = c * C;
+            if (warp == 0) {
                 tc::mbar_arrive_expect_tx(bar_load, CONS_LOAD_BYTES);
-                tma_tile(sm + sp::QQ + par * TILE_64x128, C, 0, &m.q, b, h, t0, bar_load);
-                break;
-            case 1: tma_tile(sm + sp::KT + par * TILE_64x128, C, 0, &m.la, b, h, t0, bar_load); break;
-            case 2: tma_tile(KH, C, 0, &m.k, b, h, t0, bar_load); break;
-            case 3: tma_tile(UU, C, 0, &m.v, b, h, t0, bar_load); break;
-            default: tma_tile(WW, C, 0, &m.w, b, h, t0, bar_load); break;
+                tma_tile(UU, C, 0, &m.v, b, h, t0, bar_load);
+            } else {
+                tma_tile(WW, C, 0, &m.w, b, h, t0, bar_load);
             }
         };
         // o rows of chunk c from its M=64 accumulator (16-byte stores)
@@ -311,15 +344,24 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
         int c = 0;
         for (; c < nc; ++c) {
             const int par = c & 1;
-            unsigned char* QQ = sm + sp::QQ + par * TILE_64x128;
-            unsigned char* KT = sm + sp::KT + par * TILE_64x128;
-            const uint32_t sQQ = tc::smem_u32(QQ), sKT = tc::smem_u32(KT);
+            const uint32_t sQQ = tc::smem_u32(sm + sp::QQ + par * TILE_64x128),
+                           sKT = tc::smem_u32(sm + sp::KT + par * TILE_64x128);
+            const float* sGC = reinterpret_cast<const float*>(sm + sp::GC + par * 512);
             const uint32_t tm_o = tmem + TM_O + 128 * par;
             if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
             ph_load ^= 1;
 
-            // ---- gate prep: Qt, Kt, U, gC
-            gate_prep_state(QQ, KH, KT, UU, WW, sGC, sRed, tid);
+            // ---- U = w * v (Qt, Kt and gC come with the WY image): 4 row chunks of 8 values per thread
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int idx = tid + NT * e, row = idx >> 4, g = idx & 15;
+                float vv[8], ww[8];
+                tc::ld_row8(UU, C, row, g, vv);
+                tc::ld_row8(WW, C, row, g, ww);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) vv[x] *= ww[x];
+                tc::st_row8(UU, C, row, g, vv);
+            }
             tc::cp_async_wait_all();   // this chunk's WY image
             sync_for_mma();
 
@@ -342,7 +384,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             }
             if (want_o && c > 0) store_o(c - 1);      // previous chunk's output, in the MMAs' shadow
             wait_mma();
-            // k, v, w and the other parity's q, log_alpha tiles are free: prefetch the next chunk
+            // v (read by M3) and w are free: prefetch the next chunk's
             if (c + 1 < nc) issue_loads(c + 1);
             tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
             sync_for_mma();

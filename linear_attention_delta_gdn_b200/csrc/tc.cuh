@@ -293,6 +293,12 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void flag_release(unsigned int* flag, unsigned int value) {
     asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(value) : "memory");
 }
+// Same, for data this thread wrote with bulk (async-proxy) stores: wait until they are complete, order
+// them before the thread's generic accesses (proxy fence), then release the flag.
+__device__ __forceinline__ void flag_release_after_bulk(unsigned int* flag, unsigned int value) {
+    asm volatile("cp.async.bulk.wait_group 0;\n\tfence.proxy.async.global;\n\tfence.acq_rel.gpu;\n\t"
+                 "st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(value) : "memory");
+}
 __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* flag) {
     unsigned int v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
