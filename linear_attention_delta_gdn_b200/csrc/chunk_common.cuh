@@ -331,6 +331,37 @@ __device__ __forceinline__ void warp_store16x8_tile(const float (&acc)[4], unsig
     }
 }
 
+// Inverse of the unit lower 16 x 16 diagonal block at (BASE, BASE) of I + A by right-looking forward
+// substitution, one warp, lane = column (lanes 16..31 repeat lanes 0..15). The block's 120 strictly lower
+// entries are read into registers first (compile-time addresses), so the 15 dependent steps run on
+// registers. Writes the block to sTf (fp32, sq_idx layout) and to the bf16 T tile.
+template <int BASE>
+__device__ __forceinline__ void diag_inverse16(const float* __restrict__ sA, float* __restrict__ sTf,
+                                               unsigned char* Ttile, int lane) {
+    const int s = lane & 15;
+    float a[120];
+#pragma unroll
+    for (int m = 0, idx = 0; m < 15; ++m)
+#pragma unroll
+        for (int r = m + 1; r < 16; ++r, ++idx) a[idx] = sA[sq_idx(BASE + r, BASE + m)];
+    float acc[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) acc[r] = (r == s) ? 1.f : 0.f;
+#pragma unroll
+    for (int m = 0, idx = 0; m < 15; ++m) {
+        const float xm = acc[m];
+#pragma unroll
+        for (int r = m + 1; r < 16; ++r, ++idx) acc[r] -= a[idx] * xm;
+    }
+    if (lane < 16) {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            sTf[sq_idx(BASE + r, BASE + s)] = acc[r];
+            tc::st_bf16(Ttile, tc::tile_off(C, BASE + r, BASE + s), acc[r]);
+        }
+    }
+}
+
 // (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32 scratch sA, sq_idx layout), 8 warps.
 // Writes the inverse to sTf (lower triangle incl. the unit diagonal is valid) and the bf16 row
 // tile T (64 x 64, zeros above the diagonal).
@@ -344,22 +375,11 @@ __device__ __forceinline__ void solve_unit_lower(const float* __restrict__ sA, f
                                                  float* __restrict__ sX, unsigned char* Ttile, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
     if (warp < 4) {
-        const int s = lane & 15, base = 16 * warp;
-        float acc[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = (r == s) ? 1.f : 0.f;
-#pragma unroll
-        for (int m = 0; m < 15; ++m) {
-            const float xm = acc[m];
-#pragma unroll
-            for (int r = m + 1; r < 16; ++r) acc[r] -= sA[sq_idx(base + r, base + m)] * xm;
-        }
-        if (lane < 16) {
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                sTf[sq_idx(base + r, base + s)] = acc[r];
-                tc::st_bf16(Ttile, tc::tile_off(C, base + r, base + s), acc[r]);
-            }
+        switch (warp) {
+        case 0: diag_inverse16<0>(sA, sTf, Ttile, lane); break;
+        case 1: diag_inverse16<16>(sA, sTf, Ttile, lane); break;
+        case 2: diag_inverse16<32>(sA, sTf, Ttile, lane); break;
+        default: diag_inverse16<48>(sA, sTf, Ttile, lane); break;
         }
     } else {
         // zeros above the diagonal blocks: block row br = warp - 4, columns 16 br + 16 .. 63
