@@ -383,9 +383,9 @@ constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image,
 
 // Gradients of chunk c of head `headi`; returns false if a bounded wait gave up. `prefetched`: the S, T
 // and dZ^T images of this unit were requested by the previous unit (S, T on the prefetch barrier).
-// Thread 0 takes the CTA's next unit from the counter while this one runs and, once that unit's flag
-// is acquired, requests its S, T and dZ^T images into the tiles this unit has finished with; the
-// next unit is published in *nxt before the unit's last barrier.
+// Lane 0 of warp 9 takes the CTA's next unit from the counter while this one runs and acquires its flag
+// while the G MMAs run; once this unit has finished with the S^T, T and dZ^T tiles, the next unit's
+// images are requested into them. The next unit is published in *nxt.
 __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi, int c,
                           Phases& ph, bool prefetched, NextUnit* nxt) {
     using namespace cg;
@@ -416,8 +416,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const CUtensorMap *mdq = &m.dq, *mdk = &m.dk, *mdb = &m.db, *mdla = &m.dla;
 
     bool ok = true;
-    int next_unit = units;    // thread 0: the CTA's next unit (its atomic returns while this unit runs)
-    bool next_ready = false;  // thread 0: the next unit's dZ^T flag has been acquired
+    int next_unit = units;    // lane 0 of warp 9: the CTA's next unit (its atomic returns while this unit runs)
     // The loads are issued by lane 0 of several warps at once (a TMA issue takes ~100 cycles); the
     // barrier phase cannot complete before thread 0's arrival, which carries the expected bytes.
     // (*nxt is rewritten only after the next barriers: every thread has read it by then.)
@@ -427,7 +426,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         case 0:
             tc::mbar_arrive_expect_tx(bar_load, prefetched ? LOAD_TOK : LOAD_TOK + LOAD_PRE);
             tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
-            next_unit = (int)atomicAdd(p.counter, 1u);   // the value is first needed after the G MMAs
             break;
         case 1: tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load); break;
         case 2: tma_tile(KH, C, 0, mk, b, h, t0, bar_load); break;
@@ -438,6 +436,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         case 7:
             tc::bulk_load(DT, p.deltas + (head * nc + c) * TC_DELTA_BYTES, (uint32_t)TC_DELTA_BYTES, bar_load);
             break;
+        case 9: next_unit = (int)atomicAdd(p.counter, 1u); break;   // first needed at the G MMAs
         case 8:
             if (!prefetched) {
                 tc::bulk_load(STt, p.states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
@@ -608,13 +607,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         for (int kk = 0; kk < 4; ++kk)
             tc::mma_bf16(tmem + TM_G3, tc::desc_mn(sQE, 2 * C, 0, kk), tc::desc_k(sTT, C, 0, kk), id_mk, 1);
         tc::mma_commit(bar_mma);
-        // while these run: stop if any CTA of the launch gave up; else is the next unit's dZ^T ready?
-        // (acquire; usually it has been for long)
-        if (*reinterpret_cast<volatile unsigned int*>(p.counter + 1)) next_unit = units;
-        if (next_unit < units) {
-            const int nc_ = nc - 1 - next_unit / p.BH, nh = next_unit % p.BH;
-            next_ready = tc::ld_acquire(p.flags + (size_t)nh * nc + nc_) == 1u;
-        }
     }
 
     // rowsum(dZ * S) for key channel i over this quarter's value channels (both images hold row j =
@@ -629,6 +621,16 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             e2 += tc::ld_bf16(DS, tc::tile_off(D, j + 1, i)) * tc::ld_bf16(STt, tc::tile_off(D, j + 1, i));
         }
         Epart += e2;
+    }
+    if (warp == 9 && lane == 0) {   // while the G MMAs run: the CTA's next unit, published at the next barrier
+        if (*reinterpret_cast<volatile unsigned int*>(p.counter + 1)) next_unit = units;   // a CTA gave up
+        int ready = 0;
+        if (next_unit < units) {   // acquire: usually the flag has been set for long
+            const int nc_ = nc - 1 - next_unit / p.BH, nh = next_unit % p.BH;
+            ready = tc::ld_acquire(p.flags + (size_t)nh * nc + nc_) == 1u;
+        }
+        nxt->unit = next_unit;
+        nxt->prefetched = ready;
     }
     wait_mma();
     ok = tc::mbar_wait(bar_b, ph.b) && ok;
@@ -679,15 +681,11 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][4 quarters][128]
     xch[(0 * BPARTS + qt) * 128 + i] = Epart;
     xch[(1 * BPARTS + qt) * 128 + i] = dGsum;
-    if (tid == 0) {
-        nxt->unit = next_unit;
-        nxt->prefetched = next_ready;
-    }
     tc::fence_async_smem();   // every read of S^T and dZ^T (G MMAs, rowsum) precedes the prefetch below
-    __syncthreads();          // also orders thread 0's acquire before every thread's copy of the next dZ^T
-    if (tid == 0 && next_ready) {   // S^T and T of the next unit into the tiles this unit has finished with
-        const int nc_ = nc - 1 - next_unit / p.BH, nh = next_unit % p.BH;
-        const size_t nu = (size_t)nh * nc + nc_;
+    __syncthreads();          // also orders warp 9's acquire before every thread's copy of the next dZ^T
+    if (tid == 0 && nxt->prefetched) {   // S^T and T of the next unit into the tiles this unit has finished with
+        const int nu_ = nxt->unit;
+        const size_t nu = (size_t)(nu_ % p.BH) * nc + (nc - 1 - nu_ / p.BH);
         tc::mbar_arrive_expect_tx(bar_pre, LOAD_PRE);
         tc::bulk_load(STt, p.states + nu * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_pre);
         tc::bulk_load(TT, p.tp + nu * TC_WY_BYTES, TILE_C, bar_pre);
