@@ -46,27 +46,31 @@ constexpr uint32_t TT = WY, PP = WY + 8192, WM = WY + 16384;
 constexpr uint32_t ST = 131072;     // [128 x 128] S^T (bf16)
 constexpr uint32_t DT = 163840;     // [128 x 64] Delta^T (bf16)
 constexpr uint32_t GC = 180224;     // 2 x fp32 gC[128] from the WY image (by chunk parity)
-constexpr uint32_t BAR = 181248;    // 3 mbarriers (load, mma, unused), tmem base, abort flag
+constexpr uint32_t BAR = 181248;    // 4 mbarriers (load, mma, 2 unused), tmem base, abort flag
 }  // namespace sp
-// ---- producer (WY) shared memory: two input stages, then the solve scratch and the WY image
+// ---- producer (WY) shared memory: two independent pipelines of one warpgroup (4 warps) each, so that one
+// unit's tensor-core round trips and barriers overlap the other unit's work
 namespace wy {
-constexpr uint32_t STAGE = 65536;   // per stage: [b; q] rows (32 KB) at 0, k at 32768, log_alpha at 49152
-constexpr uint32_t QE = 0, KH = 32768, KT = 49152;
-constexpr uint32_t SA = 131072;     // fp32 A [64 x 64] (sq_idx) | prep scan scratch
-constexpr uint32_t TF = 147456;     // fp32 T [64 x 64]
-constexpr uint32_t SX = 163840;     // solve temporaries, 12 KB
-constexpr uint32_t IMG = 176128;    // WY image: T | P | Wm (32 KB)
-constexpr uint32_t TT = IMG, PP = IMG + 8192, WM = IMG + 16384;
-constexpr uint32_t BAR = 208896;    // 3 mbarriers (2 stages, mma), tmem base, abort flag
-constexpr uint32_t GC = 208960;     // 2 x fp32 gC[128] (by stage)
+constexpr uint32_t PIPE = 105472;   // bytes per pipeline
+constexpr uint32_t QE = 0;          // [128 x 128]: rows 0..63 b -> Et, rows 64..127 q -> Qt
+constexpr uint32_t KH = 32768;      // k, then fp32 A [64 x 64] (sq_idx) once the prep has read k
+constexpr uint32_t KT = 49152;      // log_alpha -> Kt
+constexpr uint32_t IMG = 65536;     // T | P (bf16 64 x 64 each), then Wm (bf16 64 x 128): the image's first 48 KB
+constexpr uint32_t TT = IMG, PP = IMG + 8192;
+constexpr uint32_t TF = 81920;      // fp32 T [64 x 64] (sq_idx), then Wm once the solve is done
+constexpr uint32_t SX = 98304;      // solve temporaries (4 warps x 16 x XS fp32) | prep scan scratch (fp32 [8][128])
+constexpr uint32_t GC = 104448;     // 2 x fp32 gC[128] (by unit parity)
+constexpr uint32_t BAR = 2 * PIPE;  // 4 mbarriers (inputs, mma per pipeline), tmem base, abort flag
 }  // namespace wy
-constexpr uint32_t SMEM_BYTES = 209984 + 1024;
+constexpr uint32_t SMEM_BYTES = wy::BAR + 64 + 1024;
 static_assert(sp::BAR + 64 <= wy::BAR + 64, "consumer layout fits");
+static_assert(4 * 16 * XS * 4 <= wy::GC - wy::SX && 8 * 128 * 4 <= wy::GC - wy::SX, "producer scratch fits");
 static_assert(TC_WY_QT == 32768 && TC_WY_KT == 49152 && TC_WY_GC == 65536, "WY image: T | P | Wm | Qt | Kt | gC");
+static_assert(wy::TF == wy::IMG + TC_WY_WM, "T | P | Wm contiguous in shared memory as in the image");
 
-// TMEM columns. Consumer: S^T (fp32 state), Ut^T -> Delta^T, O x 2 (M=64). Producer: [A; P], Wm (M=64).
+// TMEM columns. Consumer: S^T (fp32 state), Ut^T -> Delta^T, O x 2 (M=64). Producer pipeline g: [A; P] at
+// 256 g, Wm (M=64) at 256 g + 64.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 256;   // O: two buffers of 128 columns (chunk parity)
-constexpr uint32_t TM_AP = 0, TM_W = 128;
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t CONS_LOAD_BYTES = 2 * 64 * 128 * 2;   // v, w
@@ -97,138 +101,298 @@ __device__ __forceinline__ void sync_for_mma() {   // smem written by threads + 
 }
 
 // ------------------------------------------------------------------ producer
+// The helpers below run on one warpgroup (wt = thread in the group, wq = warp in the group, which is
+// also the TMEM lane quarter it may read) and synchronise it with wg_sync() (a named barrier).
+
+// Gate prep of one chunk: thread = (8-token block tb = wt / 16, 8-channel group cg = wt % 16);
+//   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127)
+//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127, Kt = k/g -> KT, gC;
+//   block totals of the cumsum go through red (fp32 [8][128]).
+template <typename Sync>
+__device__ __forceinline__ void gate_prep_wg(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
+                                             float* gC_out, float* red, int wt, Sync&& wg_sync) {
+    constexpr int RB = 8;
+    const int cg = wt & 15, tb = wt >> 4;
+    float G[RB][8];
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+        tc::ld_row8(KT, C, RB * tb + u, cg, G[u]);
+        if (u > 0) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) G[u][c] += G[u - 1][c];
+        }
+    }
+    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg) = make_float4(G[RB - 1][0], G[RB - 1][1], G[RB - 1][2], G[RB - 1][3]);
+    *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg + 4) = make_float4(G[RB - 1][4], G[RB - 1][5], G[RB - 1][6], G[RB - 1][7]);
+    wg_sync();
+    float pre[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int q = 0; q < tb; ++q) {
+        const float4 x0 = *reinterpret_cast<const float4*>(red + q * 128 + 8 * cg);
+        const float4 x1 = *reinterpret_cast<const float4*>(red + q * 128 + 8 * cg + 4);
+        pre[0] += x0.x; pre[1] += x0.y; pre[2] += x0.z; pre[3] += x0.w;
+        pre[4] += x1.x; pre[5] += x1.y; pre[6] += x1.z; pre[7] += x1.w;
+    }
+    if (tb == C / RB - 1) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) gC_out[8 * cg + c] = fast_exp(pre[c] + G[RB - 1][c]);
+    }
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+        const int row = RB * tb + u;
+        float kk[8], bb[8], qq[8], e[8], kt[8];
+        tc::ld_row8(KH, C, row, cg, kk);
+        tc::ld_row8(QE, 2 * C, row, cg, bb);
+        tc::ld_row8(QE, 2 * C, C + row, cg, qq);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float Gv = pre[c] + G[u][c];
+            const float g = fast_exp(Gv), ig = fast_exp(-Gv);
+            e[c] = g * bb[c] * kk[c];
+            kt[c] = kk[c] * ig;
+            qq[c] *= g;
+        }
+        tc::st_row8(QE, 2 * C, row, cg, e);
+        tc::st_row8(KT, C, row, cg, kt);
+        tc::st_row8(QE, 2 * C, C + row, cg, qq);
+    }
+}
+
+// [A; P] from TMEM (lanes 0..63 A, 64..127 P; 64 columns): warp wq reads its lane quarter; the strictly
+// lower part of A goes to the fp32 scratch sA, the causal part of P to the bf16 tile PP.
+__device__ __forceinline__ void extract_AP_wg(uint32_t lane_base_ap, float* sA, unsigned char* PP, int wq, int lane) {
+    float v[32];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const int c0 = 32 * hf;
+        tc::tmem_ld32(lane_base_ap + c0, v);
+        tc::tmem_wait_ld();
+        if (wq < 2) {
+            const int t = 32 * wq + lane;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) sA[sq_idx(t, c0 + u)] = v[u];
+        } else {
+            const int t = 32 * (wq - 2) + lane;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] = (c0 + u <= t) ? v[u] : 0.f;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) tc::st_row8(PP, C, t, (c0 >> 3) + g, v + 8 * g);
+        }
+    }
+}
+
+// (I + A)^{-1} on one warpgroup: the diagonal 16 x 16 blocks by substitution (warp wq: block wq, which
+// also clears its block row above the diagonal), then the off-diagonal blocks by diagonals, each warp
+// taking both 8-column halves of its block in turn (warp-level tf32 products, mma.sync m16n8k8).
+template <typename Sync>
+__device__ __forceinline__ void solve_unit_lower_wg(const float* __restrict__ sA, float* __restrict__ sTf,
+                                                    float* __restrict__ sX, unsigned char* Ttile, int wq, int lane,
+                                                    Sync&& wg_sync) {
+    switch (wq) {
+    case 0: diag_inverse16<0>(sA, sTf, Ttile, lane); break;
+    case 1: diag_inverse16<16>(sA, sTf, Ttile, lane); break;
+    case 2: diag_inverse16<32>(sA, sTf, Ttile, lane); break;
+    default: diag_inverse16<48>(sA, sTf, Ttile, lane); break;
+    }
+    {   // zeros above the diagonal block: block row wq, columns 16 wq + 16 .. 63
+        const int base = 16 * wq, ngrp = (C - base - 16) / 8;
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int e = lane; e < 16 * ngrp; e += 32) tc::st_row8(Ttile, C, base + (e / ngrp), (base + 16) / 8 + (e % ngrp), z);
+    }
+    wg_sync();
+    float* Xw = sX + wq * 16 * XS;
+    float acc[4], p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};   // p0, p1: T_30's sums (warp 3)
+    // X (16 x 8) -> per-warp temporary -> T_ij[:, nc..] = -T_ii X
+    auto finish = [&](float (&x)[4], int i, int j, int nc, bool keep) {
+        warp_store16x8(x, Xw, 0, 0, false, 1.f, lane);
+        __syncwarp();
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        warp_mm16x8(acc, sTf, 16 * i, 16 * i, Xw, 0, 0, false, lane);
+        if (keep) warp_store16x8(acc, sTf, 16 * i, 16 * j + nc, true, -1.f, lane);
+        warp_store16x8_tile(acc, Ttile, 16 * i, 16 * j + nc, -1.f, lane);
+        __syncwarp();
+    };
+    // diagonal 1: T_{j+1,j} (warps 0..2); warp 3 starts T_30's sums with A_30 T_00
+    if (wq < 3) {
+        const int j = wq, i = j + 1;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_mm16x8(x, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j + 8 * nt, true, lane);
+            finish(x, i, j, 8 * nt, true);
+        }
+    } else {
+        warp_mm16x8(p0, sA, 48, 0, sTf, 0, 0, true, lane);
+        warp_mm16x8(p1, sA, 48, 0, sTf, 0, 8, true, lane);
+    }
+    wg_sync();
+    // diagonal 2: T_20 (warp 0), T_31 (warp 1); warp 3 adds A_31 T_10
+    if (wq < 2) {
+        const int j = wq, i = j + 2;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_mm16x8(x, sA, 16 * i, 16 * j, sTf, 16 * j, 16 * j + 8 * nt, true, lane);
+            warp_mm16x8(x, sA, 16 * i, 16 * (j + 1), sTf, 16 * (j + 1), 16 * j + 8 * nt, true, lane);
+            finish(x, i, j, 8 * nt, true);
+        }
+    } else if (wq == 3) {
+        warp_mm16x8(p0, sA, 48, 16, sTf, 16, 0, true, lane);
+        warp_mm16x8(p1, sA, 48, 16, sTf, 16, 8, true, lane);
+    }
+    wg_sync();
+    // diagonal 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20)   (warp 3)
+    if (wq == 3) {
+        warp_mm16x8(p0, sA, 48, 32, sTf, 32, 0, true, lane);
+        finish(p0, 3, 0, 0, false);
+        warp_mm16x8(p1, sA, 48, 32, sTf, 32, 8, true, lane);
+        finish(p1, 3, 0, 8, false);
+    }
+}
+
+// Wm (M=64 accumulator, 128 columns) into rows 0..63 of a bf16 row tile with R rows: warp wq takes rows
+// 16 wq .. 16 wq + 15 (its lane quarter's lanes 0..15).
+__device__ __forceinline__ void tmem_m64_to_tile_wg(uint32_t lane_base_col, unsigned char* dst, int R, int wq, int lane) {
+    const int r = 16 * wq + (lane & 15);
+    float v[32];
+#pragma unroll
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+        tc::tmem_ld32(lane_base_col + c0, v);
+        tc::tmem_wait_ld();
+        if (lane < 16) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) tc::st_row8(dst, R, r, (c0 >> 3) + g, v + 8 * g);
+        }
+    }
+}
+
 __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int pid) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + wy::BAR);   // [2]
-    uint64_t* bar_mma = bar_in + 2;
-    int* abort_flag = reinterpret_cast<int*>(sm + wy::BAR + 28);
-    float* sA = reinterpret_cast<float*>(sm + wy::SA);
-    float* sTf = reinterpret_cast<float*>(sm + wy::TF);
-    float* sX = reinterpret_cast<float*>(sm + wy::SX);
-    unsigned char* TT = sm + wy::TT;
-    unsigned char* PP = sm + wy::PP;
-    unsigned char* WM = sm + wy::WM;
-    const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
-    const uint32_t sTT = tc::smem_u32(TT);
+    const int wg = warp >> 2, wq = warp & 3, wt = tid & 127;   // pipeline, warp and thread in it
+    unsigned char* pb = sm + wg * wy::PIPE;
+    unsigned char* QE = pb + wy::QE;
+    unsigned char* KH = pb + wy::KH;
+    unsigned char* KT = pb + wy::KT;
+    unsigned char* TT = pb + wy::TT;
+    unsigned char* PP = pb + wy::PP;
+    float* sA = reinterpret_cast<float*>(pb + wy::KH);
+    float* sTf = reinterpret_cast<float*>(pb + wy::TF);
+    float* sX = reinterpret_cast<float*>(pb + wy::SX);
+    uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + wy::BAR) + 2 * wg;
+    uint64_t* bar_mma = bar_in + 1;
+    int* abort_flag = reinterpret_cast<int*>(sm + wy::BAR + 36);
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * wq) << 16);
+    const uint32_t tm_ap = tmem + 256 * wg, tm_w = tmem + 256 * wg + 64;
+    const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sTT = tc::smem_u32(TT);
     constexpr uint32_t ID_M1 = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
-    const int units = p.BH * p.nc;
-
-    // The four tiles of unit u, issued by lane 0 of warps 0-2 (a TMA issue takes ~100 cycles). q and
-    // log_alpha land on Qt and Kt of the stage, which the previous image stores read: thread 32 issues
-    // them (part 2) only after waiting for those reads.
-    auto tile_coords = [&](int u, int& b, int& h, int& t0) {
-        const int c = u / p.BH, head = u % p.BH;
-        b = head / p.H; h = head % p.H; t0 = c * C;
+    auto wg_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); };
+    auto sync_for_mma_wg = [&]() {
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        wg_sync();
     };
-    auto issue_loads_1 = [&](int stage, int u) {
-        if (lane != 0 || (warp != 0 && warp != 2)) return;
-        int b, h, t0;
-        tile_coords(u, b, h, t0);
-        unsigned char* base = sm + stage * wy::STAGE;
-        if (warp == 0) {
-            tc::mbar_arrive_expect_tx(&bar_in[stage], PROD_LOAD_BYTES);
-            tma_tile(base + wy::QE, 2 * C, 0, &m.b, b, h, t0, &bar_in[stage]);
-        } else {
-            tma_tile(base + wy::KH, C, 0, &m.k, b, h, t0, &bar_in[stage]);
-        }
-    };
-    auto issue_loads_2 = [&](int stage, int u) {   // lane 0 of warps 1 and 2
-        if (lane != 0 || (warp != 1 && warp != 2)) return;
-        int b, h, t0;
-        tile_coords(u, b, h, t0);
-        unsigned char* base = sm + stage * wy::STAGE;
-        if (warp == 1) tma_tile(base + wy::QE, 2 * C, C, &m.q, b, h, t0, &bar_in[stage]);
-        else tma_tile(base + wy::KT, C, 0, &m.la, b, h, t0, &bar_in[stage]);
-    };
-    if (pid < units) {
-        issue_loads_1(0, pid);
-        issue_loads_2(0, pid);
-    }
-
-    uint32_t ph_in = 0, ph_mma = 0;   // ph_in: bit s = phase parity of input stage s
+    uint32_t ph_in = 0, ph_mma = 0;
     auto wait_mma = [&]() {
         if (!tc::mbar_wait(bar_mma, ph_mma)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 1u); }
         ph_mma ^= 1;
         tc::tc_fence_after();
     };
-    int stage = 0;
-    bool pending = false;   // a prefetch into the other stage is in flight (thread 0's view)
-    // The WY image of a unit is written by bulk stores that thread 32 issues at the end of the unit; the
-    // same thread sets the unit's flag one unit later (once the stores are complete) and, before any
-    // tile they read is overwritten, waits until they have read it.
-    long long unreleased = -1;   // unit whose WY image is being written but whose flag is not yet set
-    for (int u = pid; u < units; u += p.nprod, stage ^= 1) {
+    const int units = p.BH * p.nc, npipe = 2 * p.nprod;
+    // The WY image of a unit is written by bulk stores of the pipeline's thread 0 in two groups: Qt, Kt and
+    // gC right after the prep, T | P | Wm at the end of the unit. The same thread sets the unit's flag one
+    // unit later (once the stores are complete). The next unit's tiles are loaded as soon as their
+    // buffers are free: q and log_alpha (over Qt, Kt) once M1 and the first group have read them, k (over
+    // A) after the solve, b (over Et) once M2 has read it. Before the solve writes T | P | Wm, the previous
+    // unit's second group has read them (thread 0 waits for that before issuing M1, whose completion the
+    // other threads wait for).
+    long long unreleased = -1;
+    int kunit = 0;
+    bool inflight = false;   // the next unit's loads are issued
+    auto coords = [&](int u, int& b, int& h, int& t0) {
         const int c = u / p.BH, head = u % p.BH;
-        unsigned char* base = sm + stage * wy::STAGE;
-        unsigned char* QE = base + wy::QE;
-        if (!tc::mbar_wait(&bar_in[stage], (ph_in >> stage) & 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
-        ph_in ^= 1u << stage;
-        // the other stage was last read by the previous unit's MMAs, which have completed, and by its image
-        // stores: b and k do not overlap what those read; q and log_alpha follow below
-        pending = u + p.nprod < units;
-        if (pending) issue_loads_1(stage ^ 1, u + p.nprod);
+        b = head / p.H; h = head % p.H; t0 = c * C;
+    };
+    const int u0 = 2 * pid + wg;
+    if (u0 < units && wt == 0) {   // the first unit's tiles
+        int b, h, t0;
+        coords(u0, b, h, t0);
+        tc::mbar_arrive_expect_tx(bar_in, PROD_LOAD_BYTES);
+        tma_tile(QE, 2 * C, C, &m.q, b, h, t0, bar_in);
+        tma_tile(KT, C, 0, &m.la, b, h, t0, bar_in);
+        tma_tile(KH, C, 0, &m.k, b, h, t0, bar_in);
+        tma_tile(QE, 2 * C, 0, &m.b, b, h, t0, bar_in);
+    }
+    for (int u = u0; u < units; u += npipe, ++kunit) {
+        const int c = u / p.BH, head = u % p.BH;
+        const bool next = u + npipe < units;
+        int nb = 0, nh = 0, nt0 = 0;
+        if (next) coords(u + npipe, nb, nh, nt0);
+        float* gC = reinterpret_cast<float*>(pb + wy::GC + (kunit & 1) * 512);
+        if (!tc::mbar_wait(bar_in, ph_in)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
+        ph_in ^= 1;
+        inflight = false;
 
-        gate_prep(QE, base + wy::KH, base + wy::KT, nullptr, nullptr, reinterpret_cast<float*>(sm + wy::GC + stage * 512),
-                  sA, tid, true, false);
-        // the previous image stores have read T | P | Wm (rewritten after this barrier) and the other
-        // stage's Qt, Kt (reloaded below)
-        if (tid == 32) tc::bulk_wait_read();
-        sync_for_mma();
-        const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(base + wy::KT);
-        if (tid == 0) {   // [A; P] = [Et; Qt] Kt^T
+        gate_prep_wg(QE, KH, KT, gC, sX, wt, wg_sync);
+        sync_for_mma_wg();
+        if (wt == 0) {   // first image group: Qt, Kt, gC (final after the prep)
+            const size_t unit = (size_t)head * p.nc + c;
+            unsigned char* img = p.wyimg + unit * TC_WY_BYTES;
+            tc::bulk_store(img + TC_WY_QT, QE + 8192, 8192u);               // Qt (two 64-row halves of the
+            tc::bulk_store(img + TC_WY_QT + 8192, QE + 24576, 8192u);       //  128-row tile, 16 KB apart)
+            tc::bulk_store(img + TC_WY_KT, KT, 16384u);                     // Kt
+            tc::bulk_store(img + TC_WY_GC, gC, 512u);                       // gC
+            tc::bulk_commit();
+        }
+        if (wt == 0) {   // [A; P] = [Et; Qt] Kt^T ; then the previous unit's flag (its stores have completed)
+            tc::bulk_wait_read_but1();   // the previous unit's T | P | Wm may be overwritten
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_AP, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
+                tc::mma_bf16(tm_ap, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
             tc::mma_commit(bar_mma);
+            if (unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk_but1(p.flags + unreleased, 1u);
+            unreleased = -1;
         }
-        // while M1 runs, warps 1 and 2 (outside the MMA-issuing warp) issue the prefetch's q and log_alpha
-        // (the image stores have read the tiles they overwrite: thread 32 waited before the barrier), and
-        // thread 32 sets the previous unit's flag (its image stores have completed during this unit's prep)
-        if (pending) issue_loads_2(stage ^ 1, u + p.nprod);
-        if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk(p.flags + unreleased, 1u);
-        unreleased = -1;
         wait_mma();
-        extract_AP(lane_base + TM_AP, sA, PP, true, warp, lane);
+        if (wt == 0 && next) {   // the next unit's q and log_alpha over Qt, Kt
+            tc::bulk_wait_read();
+            tc::mbar_arrive_expect_tx(bar_in, PROD_LOAD_BYTES);
+            tma_tile(QE, 2 * C, C, &m.q, nb, nh, nt0, bar_in);
+            tma_tile(KT, C, 0, &m.la, nb, nh, nt0, bar_in);
+            inflight = true;
+        }
+        extract_AP_wg(lane_base + (tm_ap - tmem), sA, PP, wq, lane);   // A over k: the prep has read k
         tc::tc_fence_before();
-        __syncthreads();
-        solve_unit_lower(sA, sTf, sX, TT, tid);   // T = (I + A)^{-1}
-        sync_for_mma();
-        if (tid == 0) {   // Wm = T Et
+        wg_sync();
+        solve_unit_lower_wg(sA, sTf, sX, TT, wq, lane, wg_sync);   // T = (I + A)^{-1}
+        sync_for_mma_wg();
+        if (wt == 0) {   // Wm = T Et ; the next unit's k over A (which the solve has finished with)
+            if (next) tma_tile(KH, C, 0, &m.k, nb, nh, nt0, bar_in);
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_W, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), ID_M2, kk > 0);
+                tc::mma_bf16(tm_w, tc::desc_k(sTT, C, 0, kk), tc::desc_mn(sQE, 2 * C, 0, kk), ID_M2, kk > 0);
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        tmem_m64_to_tile(lane_base + TM_W, WM, warp, lane);
-        tc::fence_async_smem();   // the tiles written by threads are read by the image's bulk stores
-        tc::tc_fence_before();
-        __syncthreads();
-        // the WY image of (head, c): T | P | Wm, then Qt (rows 64..127 of the [b; q] tile, whose two 64-channel
-        // panels are 16 KB apart), Kt and gC, by bulk stores
-        const size_t unit = (size_t)head * p.nc + c;
-        if (tid == 32) {
-            unsigned char* img = p.wyimg + unit * TC_WY_BYTES;
-            tc::bulk_store(img, sm + wy::IMG, 32768u);
-            tc::bulk_store(img + TC_WY_QT, QE + 8192, 8192u);
-            tc::bulk_store(img + TC_WY_QT + 8192, QE + 16384 + 8192, 8192u);
-            tc::bulk_store(img + TC_WY_KT, base + wy::KT, 16384u);
-            tc::bulk_store(img + TC_WY_GC, sm + wy::GC + stage * 512, 512u);
+        if (wt == 0 && next) tma_tile(QE, 2 * C, 0, &m.b, nb, nh, nt0, bar_in);   // the next unit's b over Et
+        tmem_m64_to_tile_wg(lane_base + (tm_w - tmem), pb + wy::TF, C, wq, lane);   // Wm over the fp32 T
+        sync_for_mma_wg();
+        if (wt == 0) {   // second image group: T | P | Wm
+            const size_t unit = (size_t)head * p.nc + c;
+            tc::bulk_store(p.wyimg + unit * TC_WY_BYTES + TC_WY_T, TT, 32768u);
             tc::bulk_commit();
+            unreleased = (long long)unit;
         }
-        unreleased = (long long)unit;
         if (*abort_flag) break;
-        pending = false;
     }
-    if (tid == 32) {   // the last unit's flag; every image store completes before the CTA leaves
+    if (wt == 0) {   // the last unit's flag; every image store completes before the CTA leaves
         if (unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk(p.flags + unreleased, 1u);
         tc::bulk_wait_all();
     }
-    // after an abort: let the prefetch in flight land before the CTA's shared memory is released
-    if (tid == 0 && pending) (void)tc::mbar_wait(&bar_in[stage ^ 1], (ph_in >> (stage ^ 1)) & 1u);
+    // after an abort: the next unit's loads land before the CTA's shared memory is released
+    if (wt == 0 && inflight) (void)tc::mbar_wait(bar_in, ph_in);
 }
 
 // ------------------------------------------------------------------ consumer
@@ -240,7 +404,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     unsigned char* DT = sm + sp::DT;
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + sp::BAR);
     uint64_t* bar_mma = bar_load + 1;
-    int* abort_flag = reinterpret_cast<int*>(sm + sp::BAR + 28);
+    int* abort_flag = reinterpret_cast<int*>(sm + sp::BAR + 36);
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);   // this warp's TMEM lanes
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
     const int T = p.T, H = p.H, nc = p.nc;
@@ -466,10 +630,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     const bool consumer = (int)blockIdx.x < p.ncons;
     const uint32_t bar_off = consumer ? sp::BAR : wy::BAR;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + bar_off);
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + bar_off + 24);
-    int* abort_flag = reinterpret_cast<int*>(sm + bar_off + 28);
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + bar_off + 32);
+    int* abort_flag = reinterpret_cast<int*>(sm + bar_off + 36);
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) tc::mbar_init(&bars[i], 1);
+        for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&maps.q); tc::tma_prefetch_desc(&maps.k); tc::tma_prefetch_desc(&maps.la);

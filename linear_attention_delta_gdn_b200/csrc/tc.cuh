@@ -277,6 +277,8 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until the shared-memory sources of all committed bulk stores may be reused
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// same, for all but the most recently committed bulk group
+__device__ __forceinline__ void bulk_wait_read_but1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // wait until all committed bulk stores are complete
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -297,6 +299,11 @@ __device__ __forceinline__ void flag_release(unsigned int* flag, unsigned int va
 // them before the thread's generic accesses (proxy fence), then release the flag.
 __device__ __forceinline__ void flag_release_after_bulk(unsigned int* flag, unsigned int value) {
     asm volatile("cp.async.bulk.wait_group 0;\n\tfence.proxy.async.global;\n\tfence.acq_rel.gpu;\n\t"
+                 "st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(value) : "memory");
+}
+// Same, when the most recent bulk group belongs to later data: waits for all groups but that one.
+__device__ __forceinline__ void flag_release_after_bulk_but1(unsigned int* flag, unsigned int value) {
+    asm volatile("cp.async.bulk.wait_group 1;\n\tfence.proxy.async.global;\n\tfence.acq_rel.gpu;\n\t"
                  "st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(value) : "memory");
 }
 __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* flag) {
