@@ -59,7 +59,7 @@ __device__ __forceinline__ void tmem_rows_to_tile(uint32_t lane_base_col, unsign
     const int row = 32 * tm_quarter(warp) + lane, c0 = (NCOL / BPARTS) * tm_part(warp);
     float v[16];
     tc::tmem_ld16(lane_base_col + c0, v);
-    tc::tmem_wait_ld();
+    tc::tmem_wait_ld(v);
     tc::st_row8(dst, 128, row, (c0 >> 3), v);
     tc::st_row8(dst, 128, row, (c0 >> 3) + 1, v + 8);
 }
@@ -271,7 +271,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
 #pragma unroll 1
             for (int i0 = cpart; i0 < cpart + 32; i0 += 32) {
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
-                tc::tmem_wait_ld();
+                tc::tmem_wait_ld(v);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
                 tc::tmem_st32(lane_base + TM_S + i0, v);
@@ -345,7 +345,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
 #pragma unroll 1
         for (int i0 = cpart; i0 < cpart + 32; i0 += 32) {
             tc::tmem_ld32(lane_base + TM_S + i0, v);
-            tc::tmem_wait_ld();
+            tc::tmem_wait_ld(v);
 #pragma unroll
             for (int u = 0; u < 32; ++u) p.dS0[(head * D + i0 + u) * D + j] = v[u];
         }
@@ -513,7 +513,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         float v[32];
         const int c0 = cpart;
         tc::tmem_ld32(lane_base + TM_DU + c0, v);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(v);
         if (lane < 16) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
@@ -565,7 +565,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         const int s_ = m64_row(warp, lane), c0 = 16 * tm_part(warp);
         float v[16];
         tc::tmem_ld16(lane_base + TM_AP + c0, v);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(v);
         if (lane < 16) {
 #pragma unroll
             for (int u = 0; u < 16; ++u) v[u] = (s_ <= c0 + u) ? v[u] : 0.f;   // dP[t][s], t >= s
@@ -573,7 +573,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             for (int g = 0; g < 2; ++g) tc::st_row8(PP, C, s_, (c0 >> 3) + g, v + 8 * g);
         }
         tc::tmem_ld16(lane_base + TM_W + c0, v);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(v);
         if (lane < 16) {
 #pragma unroll
             for (int u = 0; u < 16; ++u) v[u] = (s_ < c0 + u) ? v[u] : 0.f;    // dA[t][s], t > s
@@ -656,7 +656,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::tmem_ld8(lane_base + TM_G4 + tq, g4);
         tc::tmem_ld8(lane_base + TM_GV + tq, gv);
         tc::tmem_ld8(lane_base + TM_IGV + tq, igv);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(g1, g2, g3, g4, gv, igv);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const uint32_t t = (uint32_t)(tq + u);

@@ -257,7 +257,7 @@ __device__ __forceinline__ void extract_AP(uint32_t lane_base_ap, float* sA, uns
     const int q = tm_quarter(warp), c0 = 32 * tm_part(warp);
     float v[32];
     tc::tmem_ld32(lane_base_ap + c0, v);
-    tc::tmem_wait_ld();
+    tc::tmem_wait_ld(v);
     if (q < 2) {
         const int t = 32 * q + lane;
 #pragma unroll
@@ -451,7 +451,7 @@ __device__ __forceinline__ void tmem_to_tile_rows(uint32_t lane_base_col, unsign
 #pragma unroll
     for (int cc = 0; cc < NCOL / 2; cc += 32) {
         tc::tmem_ld32(lane_base_col + c0 + cc, v);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(v);
 #pragma unroll
         for (int g = 0; g < 4; ++g) tc::st_row8(dst, 128, row, ((c0 + cc) >> 3) + g, v + 8 * g);
     }
@@ -469,7 +469,7 @@ __device__ __forceinline__ void tmem_m64_to_tile(uint32_t lane_base_col, unsigne
 #pragma unroll
     for (int cc = 0; cc < 64; cc += 32) {
         tc::tmem_ld32(lane_base_col + c0 + cc, v);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(v);
         if (lane < 16) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) tc::st_row8(dst, C, r, ((c0 + cc) >> 3) + g, v + 8 * g);

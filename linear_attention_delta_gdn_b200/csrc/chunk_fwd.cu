@@ -166,7 +166,7 @@ __device__ __forceinline__ void extract_AP_wg(uint32_t lane_base_ap, float* sA, 
     for (int hf = 0; hf < 2; ++hf) {
         const int c0 = 32 * hf;
         tc::tmem_ld32(lane_base_ap + c0, v);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(v);
         if (wq < 2) {
             const int t = 32 * wq + lane;
 #pragma unroll
@@ -258,7 +258,7 @@ __device__ __forceinline__ void tmem_m64_to_tile_wg(uint32_t lane_base_col, unsi
 #pragma unroll
     for (int c0 = 0; c0 < 128; c0 += 32) {
         tc::tmem_ld32(lane_base_col + c0, v);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(v);
         if (lane < 16) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) tc::st_row8(dst, R, r, (c0 >> 3) + g, v + 8 * g);
@@ -286,7 +286,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     const uint32_t sQE = tc::smem_u32(QE), sKT = tc::smem_u32(KT), sTT = tc::smem_u32(TT);
     constexpr uint32_t ID_M1 = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_M2 = tc::idesc_bf16(64, 128, false, true);
-    auto wg_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); };
+    auto wg_sync = [&]() { tc::named_sync(1 + wg, 128); };
     auto sync_for_mma_wg = [&]() {
         tc::fence_async_smem();
         tc::tc_fence_before();
@@ -469,7 +469,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
 #pragma unroll
             for (int c0 = cpart; c0 < cpart + 64; c0 += 32) {
                 tc::tmem_ld32(ob + c0, v);
-                tc::tmem_wait_ld();
+                tc::tmem_wait_ld(v);
                 if (lane < 16 && t < L) {
                     uint4* dst = reinterpret_cast<uint4*>(p.o + tok_off(b, t0 + t, h, T, H, D) + c0);
 #pragma unroll
@@ -580,7 +580,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
 #pragma unroll 1
                 for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
                     tc::tmem_ld32(lane_base + TM_S + i0, v);
-                    tc::tmem_wait_ld();
+                    tc::tmem_wait_ld(v);
 #pragma unroll
                     for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
                     tc::tmem_st32(lane_base + TM_S + i0, v);
@@ -609,7 +609,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
 #pragma unroll 1
             for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
-                tc::tmem_wait_ld();
+                tc::tmem_wait_ld(v);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) p.ST[(head * D + i0 + u) * D + j] = v[u];
             }

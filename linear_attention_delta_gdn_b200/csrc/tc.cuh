@@ -149,29 +149,38 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// tcgen05.ld fills its destination registers asynchronously: they may be read only after
+// tcgen05.wait::ld. The wait takes the arrays that the outstanding loads fill and, after the wait
+// instruction, marks each of their registers as rewritten (an empty asm), so that the compiler cannot
+// schedule any use of them (a conversion, a multiply) above the wait.
+template <int N>
+__device__ __forceinline__ void reg_fence(float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+template <typename... Arrays>
+__device__ __forceinline__ void tmem_wait_ld(Arrays&... arrays) {
+    static_assert(sizeof...(Arrays) > 0, "name the registers the loads fill");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    (reg_fence(arrays), ...);
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Warp-wide: each thread reads 16 / 32 consecutive 32-bit columns of its own lane.
+// Warp-wide: each thread reads 8 / 16 / 32 consecutive 32-bit columns of its own lane. The loads write
+// straight into the caller's float registers (no copy that could be scheduled before the wait).
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
-    uint32_t r[8];
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
                  : "r"(taddr)
                  : "memory");
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-    uint32_t r[16];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+          "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
         : "r"(taddr)
         : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     tmem_ld16(taddr, v);
@@ -236,6 +245,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
         if (done) return true;
         if (global_timer_ns() - t0 > 2000000000ull) return false;
     }
+}
+// Named barrier `id` over `count` threads (a multiple of 32), in the non-aligned form: every thread
+// counts on its own, so it is correct even when a warp arrives diverged, e.g. right after a block that
+// only one of its threads executes (the aligned bar.sync would count the whole warp at once).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 // Make generic-proxy shared-memory writes visible to the async proxy (UMMA, TMA).
 __device__ __forceinline__ void fence_async_smem() {
