@@ -300,8 +300,9 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     };
     const int units = p.BH * p.nc, npipe = 2 * p.nprod;
     // The WY image of a unit is written by bulk stores of the pipeline's thread 0 in two groups: Qt, Kt and
-    // gC right after the prep, T | P | Wm at the end of the unit. The same thread sets the unit's flag one
-    // unit later (once the stores are complete). The next unit's tiles are loaded as soon as their
+    // gC right after the prep, T | P | Wm at the end of the unit. The same thread sets the unit's flag at
+    // the end of the pipeline's next unit, when its stores have long completed (the wait for them and the
+    // release fence then cost little). The next unit's tiles are loaded as soon as their
     // buffers are free: q and log_alpha (over Qt, Kt) once M1 and the first group have read them, k (over
     // A) after the solve, b (over Et) once M2 has read it. Before the solve writes T | P | Wm, the previous
     // unit's second group has read them (thread 0 waits for that before issuing M1, whose completion the
@@ -344,15 +345,13 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             tc::bulk_store(img + TC_WY_GC, gC, 512u);                       // gC
             tc::bulk_commit();
         }
-        if (wt == 0) {   // [A; P] = [Et; Qt] Kt^T ; then the previous unit's flag (its stores have completed)
+        if (wt == 0) {   // [A; P] = [Et; Qt] Kt^T
             tc::bulk_wait_read_but1();   // the previous unit's T | P | Wm may be overwritten
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_bf16(tm_ap, tc::desc_k(sQE, 2 * C, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_M1, kk > 0);
             tc::mma_commit(bar_mma);
-            if (unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk_but1(p.flags + unreleased, 1u);
-            unreleased = -1;
         }
         wait_mma();
         if (wt == 0 && next) {   // the next unit's q and log_alpha over Qt, Kt
@@ -379,7 +378,9 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         if (wt == 0 && next) tma_tile(QE, 2 * C, 0, &m.b, nb, nh, nt0, bar_in);   // the next unit's b over Et
         tmem_m64_to_tile_wg(lane_base + (tm_w - tmem), pb + wy::TF, C, wq, lane);   // Wm over the fp32 T
         sync_for_mma_wg();
-        if (wt == 0) {   // second image group: T | P | Wm
+        if (wt == 0) {   // the previous unit's flag (all its stores are older than this unit's first group);
+                         // second image group: T | P | Wm
+            if (unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk_but1(p.flags + unreleased, 1u);
             const size_t unit = (size_t)head * p.nc + c;
             tc::bulk_store(p.wyimg + unit * TC_WY_BYTES + TC_WY_T, TT, 32768u);
             tc::bulk_commit();
