@@ -39,14 +39,17 @@ using namespace chunk;
 namespace sp {
 constexpr uint32_t QQ = 0;          // 2 x [64 x 128] Qt from the WY image (by chunk parity)
 constexpr uint32_t KT = 32768;      // 2 x [64 x 128] Kt from the WY image (by chunk parity)
-constexpr uint32_t UU = 65536;      // [64 x 128] v -> U
-constexpr uint32_t WW = 81920;      // [64 x 128] w
+constexpr uint32_t UU = 65536;      // [64 x 128] v -> U (even chunks)
+constexpr uint32_t WW = 81920;      // [64 x 128] w (even chunks)
 constexpr uint32_t WY = 98304;      // WY image head: T [64 x 64] | P [64 x 64] | Wm [64 x 128]
 constexpr uint32_t TT = WY, PP = WY + 8192, WM = WY + 16384;
 constexpr uint32_t ST = 131072;     // [128 x 128] S^T (bf16)
 constexpr uint32_t DT = 163840;     // [128 x 64] Delta^T (bf16)
 constexpr uint32_t GC = 180224;     // 2 x fp32 gC[128] from the WY image (by chunk parity)
-constexpr uint32_t BAR = 181248;    // 4 mbarriers (load, mma, 2 unused), tmem base, abort flag
+constexpr uint32_t BAR = 181248;    // 4 mbarriers (load even, mma, load odd, unused), tmem base, abort flag
+constexpr uint32_t UU1 = 182272;    // [64 x 128] v -> U (odd chunks)
+constexpr uint32_t WW1 = 198656;    // [64 x 128] w (odd chunks)
+constexpr uint32_t END = 215040;
 }  // namespace sp
 // ---- producer (WY) shared memory: two independent pipelines of one warpgroup (4 warps) each, so that one
 // unit's tensor-core round trips and barriers overlap the other unit's work
@@ -62,8 +65,8 @@ constexpr uint32_t SX = 98304;      // solve temporaries (4 warps x 16 x XS fp32
 constexpr uint32_t GC = 104448;     // 2 x fp32 gC[128] (by unit parity)
 constexpr uint32_t BAR = 2 * PIPE;  // 4 mbarriers (inputs, mma per pipeline), tmem base, abort flag
 }  // namespace wy
-constexpr uint32_t SMEM_BYTES = wy::BAR + 64 + 1024;
-static_assert(sp::BAR + 64 <= wy::BAR + 64, "consumer layout fits");
+constexpr uint32_t SMEM_BYTES = (sp::END > wy::BAR + 64 ? sp::END : wy::BAR + 64) + 1024;
+static_assert(sp::BAR + 64 <= sp::UU1 && sp::UU1 % 1024 == 0 && sp::WW1 % 1024 == 0, "consumer layout");
 static_assert(4 * 16 * XS * 4 <= wy::GC - wy::SX && 8 * 128 * 4 <= wy::GC - wy::SX, "producer scratch fits");
 static_assert(TC_WY_QT == 32768 && TC_WY_KT == 49152 && TC_WY_GC == 65536, "WY image: T | P | Wm | Qt | Kt | gC");
 static_assert(wy::TF == wy::IMG + TC_WY_WM, "T | P | Wm contiguous in shared memory as in the image");
@@ -399,26 +402,28 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
 // ------------------------------------------------------------------ consumer
 __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int cid) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    unsigned char* UU = sm + sp::UU;
-    unsigned char* WW = sm + sp::WW;
+    // v and w tiles by chunk parity: chunk c + 2 is loaded while chunk c + 1's tiles wait in the other pair
+    auto UUp = [&](int c) { return sm + ((c & 1) ? sp::UU1 : sp::UU); };
+    auto WWp = [&](int c) { return sm + ((c & 1) ? sp::WW1 : sp::WW); };
     unsigned char* STt = sm + sp::ST;
     unsigned char* DT = sm + sp::DT;
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + sp::BAR);
-    uint64_t* bar_mma = bar_load + 1;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + sp::BAR);
+    uint64_t* bar_mma = bars + 1;
+    auto bar_ld = [&](int c) { return bars + ((c & 1) ? 2 : 0); };
     int* abort_flag = reinterpret_cast<int*>(sm + sp::BAR + 36);
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);   // this warp's TMEM lanes
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
     const int T = p.T, H = p.H, nc = p.nc;
     const bool want_o = (p.o != nullptr);
 
-    const uint32_t sUU = tc::smem_u32(UU), sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
+    const uint32_t sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
                    sTT = tc::smem_u32(sm + sp::TT), sPP = tc::smem_u32(sm + sp::PP), sWM = tc::smem_u32(sm + sp::WM);
     constexpr uint32_t ID_M3 = tc::idesc_bf16(128, 64, true, false);
     constexpr uint32_t ID_M4 = tc::idesc_bf16(128, 64, false, false, true);
     constexpr uint32_t ID_M56 = tc::idesc_bf16(64, 128, false, false);
     constexpr uint32_t ID_M7 = tc::idesc_bf16(128, 128, false, true);
 
-    uint32_t ph_load = 0, ph_mma = 0;
+    uint32_t ph_load = 0, ph_mma = 0;   // ph_load: bit p is the phase of the load barrier of parity p
     auto wait_mma = [&]() {
         if (!tc::mbar_wait(bar_mma, ph_mma)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 1u); }
         ph_mma ^= 1;
@@ -455,10 +460,10 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             if (lane != 0 || warp > 1) return;
             const int t0 = c * C;
             if (warp == 0) {
-                tc::mbar_arrive_expect_tx(bar_load, CONS_LOAD_BYTES);
-                tma_tile(UU, C, 0, &m.v, b, h, t0, bar_load);
+                tc::mbar_arrive_expect_tx(bar_ld(c), CONS_LOAD_BYTES);
+                tma_tile(UUp(c), C, 0, &m.v, b, h, t0, bar_ld(c));
             } else {
-                tma_tile(WW, C, 0, &m.w, b, h, t0, bar_load);
+                tma_tile(WWp(c), C, 0, &m.w, b, h, t0, bar_ld(c));
             }
         };
         // o rows of chunk c from its M=64 accumulator (16-byte stores)
@@ -481,6 +486,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             }
         };
         issue_loads(0);
+        if (nc > 1) issue_loads(1);
         if (tid == 0) wait_wy(head, 0);
         // initial state: S^T row j = column j of S0
         {
@@ -513,8 +519,11 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                            sKT = tc::smem_u32(sm + sp::KT + par * TILE_64x128);
             const float* sGC = reinterpret_cast<const float*>(sm + sp::GC + par * 512);
             const uint32_t tm_o = tmem + TM_O + 128 * par;
-            if (!tc::mbar_wait(bar_load, ph_load)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
-            ph_load ^= 1;
+            unsigned char* UU = UUp(c);
+            const unsigned char* WW = WWp(c);
+            const uint32_t sUU = tc::smem_u32(UU);
+            if (!tc::mbar_wait(bar_ld(c), (ph_load >> par) & 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
+            ph_load ^= 1u << par;
 
             // ---- U = w * v (Qt, Kt and gC come with the WY image): 4 row chunks of 8 values per thread
 #pragma unroll
@@ -549,8 +558,8 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             }
             if (want_o && c > 0) store_o(c - 1);      // previous chunk's output, in the MMAs' shadow
             wait_mma();
-            // v (read by M3) and w are free: prefetch the next chunk's
-            if (c + 1 < nc) issue_loads(c + 1);
+            // this chunk's v (read by M3) and w buffers are free: chunk c + 2's tiles go there
+            if (c + 2 < nc) issue_loads(c + 2);
             tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
             sync_for_mma();
             if (p.deltas && tid == 0) {   // Delta^T of this chunk for the backward
@@ -597,7 +606,8 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 tc::bulk_commit();
             }
             if (*abort_flag) {   // let the next chunk's loads land before leaving
-                if (tid == 0 && c + 1 < nc) (void)tc::mbar_wait(bar_load, ph_load);
+                if (tid == 0 && c + 1 < nc) (void)tc::mbar_wait(bar_ld(c + 1), (ph_load >> ((c + 1) & 1)) & 1u);
+                if (tid == 0 && c + 2 < nc) (void)tc::mbar_wait(bar_ld(c + 2), ((ph_load >> (c & 1)) & 1u));
                 break;
             }
         }
