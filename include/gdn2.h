@@ -45,7 +45,10 @@
  *     flags in the workspace), else as two ordinary launches with the same
  *     results. Setting the environment variable GDN2_NO_COOPERATIVE (to any
  *     value but "0") selects the two-launch form, e.g. for tools that do not
- *     support cooperative launches.
+ *     support cooperative launches. GDN2_TEST_SKIP_PRODUCERS (same rule) is a
+ *     test hook of the forward's two-launch form: the producer launch is left
+ *     out, so the consumers' ready-flag waits run out and gdn2_device_status
+ *     reports GDN2_ERR_TIMEOUT; outputs are then not valid.
  */
 #ifndef GDN2_H
 #define GDN2_H
@@ -62,7 +65,7 @@ typedef enum gdn2_status {
     GDN2_ERR_UNSUPPORTED = 2, /* valid but not built for this shape/dtype; nothing launched */
     GDN2_ERR_WORKSPACE = 3,   /* workspace missing or too small; nothing launched */
     GDN2_ERR_CUDA = 4,        /* CUDA runtime error (see gdn2_last_error) */
-    GDN2_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (reserved) */
+    GDN2_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (reported by gdn2_device_status) */
 } gdn2_status;
 
 typedef enum gdn2_dtype {
@@ -186,6 +189,19 @@ size_t gdn2_no_alloc_scratch_bytes(void);
  */
 void gdn2_trace_enable(int on);
 int gdn2_trace_read(char* names, size_t names_cap, int* launches, double* ms, int max_kernels);
+
+/* Device-side status of the tensor-core kernels. Every wait inside them (on an
+ * mbarrier or on a ready flag written by another CTA) gives up after ~2 s; the
+ * kernel then records the event in device memory, lets its own copies in flight
+ * land, skips the rest of its work and exits (the outputs of that call are not
+ * valid, the CUDA context stays usable). This call synchronises `stream` (a
+ * cudaStream_t, NULL for the default stream), returns GDN2_ERR_TIMEOUT if such
+ * an event was recorded since the previous call (gdn2_last_error names the
+ * kernel and the kind of wait) and clears the record; GDN2_ERR_CUDA if the
+ * stream holds a CUDA error. The entry points above never synchronise, so this
+ * is the call that checks a finished step after the fact.
+ */
+gdn2_status gdn2_device_status(void* stream);
 
 /* Static description of a status code. */
 const char* gdn2_status_string(gdn2_status s);

@@ -22,13 +22,14 @@ _lib = None
 
 GDN2_F32, GDN2_BF16 = 0, 1
 GDN2_OP_FWD, GDN2_OP_FWD_SAVE, GDN2_OP_BWD = 0, 1, 2
+GDN2_OK, GDN2_ERR_TIMEOUT = 0, 5
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_WORKSPACE",
           4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT"}
 
 #: exported symbols, as declared in include/gdn2.h
 EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "gdn2_status_string",
            "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes",
-           "gdn2_trace_enable", "gdn2_trace_read")
+           "gdn2_trace_enable", "gdn2_trace_read", "gdn2_device_status")
 
 
 class Gdn2Error(RuntimeError):
@@ -65,6 +66,8 @@ def lib(path: Optional[str] = None) -> ctypes.CDLL:
     L.gdn2_bwd_no_alloc.restype = I
     L.gdn2_no_alloc_scratch_bytes.argtypes = []
     L.gdn2_no_alloc_scratch_bytes.restype = Z
+    L.gdn2_device_status.argtypes = [P]
+    L.gdn2_device_status.restype = I
     L.gdn2_trace_enable.argtypes = [I]
     L.gdn2_trace_enable.restype = None
     L.gdn2_trace_read.argtypes = [ctypes.c_char_p, Z, P, P, I]
@@ -186,6 +189,18 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None):
                                 B, H, Dk, Dv, _dt(q), _stream(q.device))
     _check("gdn2_decode_step", rc)
     return o
+
+
+def gdn2_device_status(device=None) -> int:
+    """Synchronise the current stream and return the device-side status of the tensor-core kernels
+    (0, or GDN2_ERR_TIMEOUT if a bounded wait inside them gave up since the previous call; the record is
+    cleared). The detail is in :func:`last_error`."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(lib().gdn2_device_status(_stream(dev)))
+
+
+def last_error() -> str:
+    return lib().gdn2_last_error().decode()
 
 
 def trace_enable(on: bool = True) -> None:

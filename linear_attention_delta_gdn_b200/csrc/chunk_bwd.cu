@@ -727,7 +727,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     }
     if (!ok) atomicOr(&g_bwd_error, 4u);
     tc::tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok) != 0;   // the same answer on every thread: the CTA leaves the loop together
     tc::tc_fence_after();
     return ok;
 }
@@ -840,6 +840,13 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     pg.nrev = 0; pg.join = 0; pg.grad = 1;
     chunk_bwd_kernel<<<units < slots ? units : slots, BT, SMEM_BYTES_ALL, s>>>(maps, pg);
     return cudaGetLastError();
+}
+
+cudaError_t chunk_bwd_take_errors(unsigned int* bits) {
+    cudaError_t e = cudaMemcpyFromSymbol(bits, g_bwd_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_bwd_error, &zero, sizeof(unsigned int));
 }
 
 }  // namespace gdn2

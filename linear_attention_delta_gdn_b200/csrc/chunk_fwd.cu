@@ -389,7 +389,9 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             tc::bulk_commit();
             unreleased = (long long)unit;
         }
-        if (*abort_flag) break;
+        // all 128 threads leave together if any has seen the abort flag (the other pipeline may set it at
+        // any time, so separate reads could split the threads that synchronise on this barrier)
+        if (tc::named_sync_or(1 + wg, 128, *abort_flag != 0)) break;
     }
     if (wt == 0) {   // the last unit's flag; every image store completes before the CTA leaves
         if (unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk(p.flags + unreleased, 1u);
@@ -700,7 +702,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     TraceScope trace(K_CHUNK_FWD, s);
     // Heads share the launch with the producers while the producers keep pace: per chunk step the
     // BH consumer chunks take about as long as BH WY units spread over the remaining CTAs.
-    if (coop && !cooperative_disabled() && slots >= 2 && 16 * BH <= 9 * slots) {
+    if (coop && !cooperative_disabled() && !test_skip_producers() && slots >= 2 && 16 * BH <= 9 * slots) {
         p.ncons = BH;
         p.nprod = slots - BH < units ? slots - BH : units;
         void* args[2] = {&maps, &p};
@@ -712,13 +714,22 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     FwdParams pp = p;   // producers only
     pp.ncons = 0;
     pp.nprod = units < slots ? units : slots;
-    chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (!test_skip_producers()) {
+        chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     FwdParams pc = p;   // consumers only; every flag is set when they start
     pc.ncons = BH;
     pc.nprod = 0;
     chunk_fwd_kernel<<<BH, NT, SMEM_BYTES, s>>>(maps, pc);
     return cudaGetLastError();
+}
+
+cudaError_t chunk_fwd_take_errors(unsigned int* bits) {
+    cudaError_t e = cudaMemcpyFromSymbol(bits, g_fwd_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_fwd_error, &zero, sizeof(unsigned int));
 }
 
 }  // namespace gdn2

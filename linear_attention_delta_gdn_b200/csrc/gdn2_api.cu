@@ -104,10 +104,12 @@ gdn2_status copy_or_zero_state(float* dst, const float* src, const Dims& d, cuda
 
 namespace gdn2 {
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
-bool cooperative_disabled() {
-    const char* v = getenv("GDN2_NO_COOPERATIVE");
+static bool env_flag(const char* name) {
+    const char* v = getenv(name);
     return v && v[0] && !(v[0] == '0' && v[1] == 0);
 }
+bool cooperative_disabled() { return env_flag("GDN2_NO_COOPERATIVE"); }
+bool test_skip_producers() { return env_flag("GDN2_TEST_SKIP_PRODUCERS"); }
 }  // namespace gdn2
 
 extern "C" {
@@ -127,6 +129,20 @@ const char* gdn2_status_string(gdn2_status s) {
 }
 
 const char* gdn2_last_error(void) { return g_err; }
+
+gdn2_status gdn2_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e, "gdn2_device_status (stream)");
+    unsigned int fwd = 0, bwd = 0;
+    if ((e = chunk_fwd_take_errors(&fwd)) != cudaSuccess) return cuda_status(e, "gdn2_device_status (forward record)");
+    if ((e = chunk_bwd_take_errors(&bwd)) != cudaSuccess) return cuda_status(e, "gdn2_device_status (backward record)");
+    if (fwd | bwd)
+        return fail(GDN2_ERR_TIMEOUT,
+                    "device wait gave up: chunk_fwd_kernel bits 0x%x, chunk_bwd_kernel bits 0x%x "
+                    "(1 MMA completion, 2 tile loads, 4 forward ready flag / gradient unit, 8 backward ready flag)",
+                    fwd, bwd);
+    return GDN2_OK;
+}
 
 size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt) {
     if (check_dims(B, T, H, Dk, Dv, chunk, dt, true) != GDN2_OK) return 0;

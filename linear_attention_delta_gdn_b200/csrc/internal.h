@@ -88,6 +88,10 @@ class TraceScope {
 // True when the environment variable GDN2_NO_COOPERATIVE is set: the chunkwise kernels then run
 // their producer and consumer work as two ordinary launches instead of one cooperative launch.
 bool cooperative_disabled();
+bool test_skip_producers();   // host-side fault injection for the forward's two-launch form
+// Read and clear the device-side error words of the tensor-core kernels (bit set: a bounded wait gave up).
+cudaError_t chunk_fwd_take_errors(unsigned int* bits);
+cudaError_t chunk_bwd_take_errors(unsigned int* bits);
 
 // Sets the detail string returned by gdn2_last_error() on this host thread.
 void set_last_error(const char* msg);

@@ -252,6 +252,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
     asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Named barrier that also returns whether `pred` held on any participating thread (the same answer on
+// every thread, so a loop can leave on it without splitting the threads that synchronise on `id`).
+__device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbarrier.red.or.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
 // Make generic-proxy shared-memory writes visible to the async proxy (UMMA, TMA).
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
