@@ -681,8 +681,20 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][4 quarters][128]
     xch[(0 * BPARTS + qt) * 128 + i] = Epart;
     xch[(1 * BPARTS + qt) * 128 + i] = dGsum;
-    tc::fence_async_smem();   // every read of S^T and dZ^T (G MMAs, rowsum) precedes the prefetch below
+    tc::fence_async_smem();   // every read of S^T and dZ^T (G MMAs, rowsum) precedes the prefetch below, and
+                              // dq, dk, db (final after pass 1) are visible to the tensor stores
     __syncthreads();          // also orders warp 9's acquire before every thread's copy of the next dZ^T
+    if (tid == 0) {   // dq, dk, db go out while pass 2 runs; rows past the end of the sequence are skipped
+        const CUtensorMap* maps[3] = {mdq, mdk, mdb};
+        const unsigned char* tiles[3] = {DU, DT, DDT};
+        const uint32_t panel[3] = {2 * C * 128, C * 128, C * 128};   // second 64 channels
+#pragma unroll
+        for (int o = 0; o < 3; ++o) {
+            tc::tma_store_4d(maps[o], 0, h, t0, b, tiles[o]);
+            tc::tma_store_4d(maps[o], 64, h, t0, b, tiles[o] + panel[o]);
+        }
+        tc::bulk_commit();
+    }
     if (tid == 0 && nxt->prefetched) {   // S^T and T of the next unit into the tiles this unit has finished with
         const int nu_ = nxt->unit;
         const size_t nu = (size_t)(nu_ % p.BH) * nc + (nc - 1 - nu_ / p.BH);
@@ -713,15 +725,9 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     }
     tc::fence_async_smem();
     __syncthreads();
-    if (tid == 0) {   // rows past the end of the sequence are skipped by the tensor store
-        const CUtensorMap* maps[4] = {mdq, mdk, mdb, mdla};
-        const unsigned char* tiles[4] = {DU, DT, DDT, DU + C * 128};
-        const uint32_t panel[4] = {2 * C * 128, C * 128, C * 128, 2 * C * 128};   // second 64 channels
-#pragma unroll
-        for (int o = 0; o < 4; ++o) {
-            tc::tma_store_4d(maps[o], 0, h, t0, b, tiles[o]);
-            tc::tma_store_4d(maps[o], 64, h, t0, b, tiles[o] + panel[o]);
-        }
+    if (tid == 0) {   // dlog_alpha; every store has read its tile before the next unit's loads reuse them
+        tc::tma_store_4d(mdla, 0, h, t0, b, DU + C * 128);
+        tc::tma_store_4d(mdla, 64, h, t0, b, DU + C * 128 + 2 * C * 128);
         tc::bulk_commit();
         tc::bulk_wait_read();
     }
