@@ -10,9 +10,10 @@
 // The WY step does not depend on S; the state step is a chain over the chunks of a head.
 //
 // One launch, two kinds of CTA (256 threads each, one CTA per SM):
-//   * producers walk the chunks of all heads in chunk-major order and compute the WY step; each
-//     writes T, P and Wm of its chunk ("WY image", 32 KB) to the workspace and then sets the
-//     chunk's ready flag (release);
+//   * producers run two independent WY pipelines each (one warpgroup per pipeline, its own named
+//     barrier, mbarriers and TMEM columns), over the chunks of all heads in chunk-major order; a
+//     pipeline writes T, P, Wm, Qt, Kt and gC of its chunk ("WY image", 65 KB) to the workspace
+//     with bulk stores and sets the chunk's ready flag (release) once they have completed;
 //   * consumers (one per head, or several heads each when heads outnumber them) walk their head's
 //     chunks in order: they wait for the chunk's flag (acquire), copy its WY image into shared
 //     memory and run the state step. The state S^T lives in TMEM (lane j = value channel, column
