@@ -10,7 +10,9 @@ entries never interact, so there is no data-path collective (weak scaling).
 Rank 0 prints one JSON line.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
-sample of the same workload (rank 0 only).
+sample of the same workload (rank 0 only). ``--sweep`` prints, instead of the
+headline line, one line per sequence length (fwd+bwd at 16K tokens per step,
+T = 1K..16K) and one for the long forward (B=1, H=16, T=64K, S0 given).
 """
 from __future__ import annotations
 
@@ -214,6 +216,83 @@ def bench_decode(binding, dev, steps=1024, pool=64):
             "launches": kern[0]}
 
 
+def run_sweep(args):
+    """Opt-in measurements beside the headline step (one JSON line each, 1 GPU): the fwd+bwd step at a
+    fixed 16K tokens per step for sequence lengths 1K..16K, and the long inference forward (B=1, H=16,
+    T=64K, S0 given). Inputs are drawn on the device with the recipe's distributions (seeded torch
+    generator), since the long case holds ~0.8 GB of token tensors."""
+    import torch
+    from linear_attention_delta_gdn_b200 import binding, build
+    from linear_attention_delta_gdn_b200.inputs import make_decode_stream
+    build.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    pk = peaks()
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    D = 128
+
+    def device_inputs(B, T, H, seed, with_do):
+        xs = make_decode_stream(T, B, H, D, D, seed, "bf16", device=dev)   # [T, B, H, D] -> [B, T, H, D]
+        d = {n: xs[n].permute(1, 0, 2, 3).contiguous() for n in names}
+        d["S0"] = xs["S0"]
+        if with_do:
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(seed + 1)
+            d["dout"] = torch.randn((B, T, H, D), generator=gen, device=dev).to(torch.bfloat16)
+        return d
+
+    def timed(fn, steps, warmup=3):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        e.record()
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(e) / steps
+
+    H = 16
+    for T in (1024, 2048, 4096, 8192, 16384):
+        B = 16384 // T
+        d = device_inputs(B, T, H, 3000 + T, True)
+        ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_BWD, B, T, H, D, D, 64, binding.GDN2_BF16),
+                         dtype=torch.uint8, device=dev)
+        o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+        ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+        grads = {n: torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+                 for n in ("dq", "dk", "dlog_alpha", "db", "dv", "dw")}
+        grads["dS0"] = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+
+        def step():
+            binding.gdn2_fwd(*(d[n] for n in names), None, save_states=True, ws=ws, o=o, ST=ST)
+            binding.gdn2_bwd(*(d[n] for n in names), d["dout"], None, None, states_saved=True, ws=ws, grads=grads)
+
+        ms = timed(step, max(3, args.steps))
+        alg = B * T * H * STEP_BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
+        print(json.dumps({"mode": "sweep", "workload": "fwdbwd-bf16-b%dh%dt%dd128" % (B, H, T), "B": B, "T": T,
+                          "H": H, "ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
+                          "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                          "status": binding.gdn2_device_status()}), flush=True)
+        del d, ws, o, ST, grads
+        torch.cuda.empty_cache()
+
+    B, T = 1, 65536   # the long inference forward, initial state given
+    d = device_inputs(B, T, H, 4000, False)
+    ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_FWD, B, T, H, D, D, 64, binding.GDN2_BF16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    ms = timed(lambda: binding.gdn2_fwd(*(d[n] for n in names), d["S0"], ws=ws, o=o, ST=ST), max(3, args.steps))
+    alg = B * T * H * KERNEL_BYTES_PER_TOKEN_HEAD["chunk_fwd_kernel"] + 2 * B * H * D * D * 4
+    print(json.dumps({"mode": "sweep", "workload": "fwd-bf16-b1h16t65536d128-S0", "B": B, "T": T, "H": H,
+                      "ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
+                      "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                      "status": binding.gdn2_device_status()}), flush=True)
+    return 0
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -246,9 +325,14 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
     ap.add_argument("--B", type=int, default=None, help="override the batch size (small profiling cases)")
     ap.add_argument("--T", type=int, default=None, help="override the sequence length (small profiling cases)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the headline line: fwd+bwd at 16K tokens per step for T = 1K..16K, and "
+                         "the long forward B1 H16 T64K with S0 (one JSON line each, 1 GPU)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
 
     import torch
     import torch.distributed as dist
