@@ -135,3 +135,12 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         binding.gdn2_fwd(x, x, x, x, x, x)
+
+
+def test_device_status_reports_a_cuda_error_without_a_device(L):
+    """On a host without a usable GPU the status call returns GDN2_ERR_CUDA with a detail, not a crash."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present (the GPU tests cover the status call)")
+    assert L.gdn2_device_status(None) == 4
+    assert b"gdn2_device_status" in L.gdn2_last_error()
