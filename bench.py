@@ -376,7 +376,9 @@ def main():
     torch.cuda.synchronize(dev)
 
     # ---- device-timed region: inputs resident in HBM (470 MB per step, larger than L2)
-    clock_log = os.path.join(ROOT, "gpurun_out", "bench_clocks_rank%d.csv" % rank)
+    # nvidia-smi samples of the timed region (summarised in the JSON line); GDN2_BENCH_LOG_DIR moves the CSV
+    clock_log = os.path.join(os.environ.get("GDN2_BENCH_LOG_DIR", os.path.join(ROOT, "bench_logs")),
+                             "bench_clocks_rank%d.csv" % rank)
     os.makedirs(os.path.dirname(clock_log), exist_ok=True)
     binding.trace_read()
     if world > 1:
