@@ -26,7 +26,8 @@
  *     token gradients dq, dk, dv, dlog_alpha, db, dw. States and their
  *     gradients are always float32.
  *   - stream is a cudaStream_t (NULL: the legacy default stream). All work is
- *     enqueued on it; no call synchronises the host or allocates memory.
+ *     enqueued on it; no call allocates memory, and none but
+ *     gdn2_device_status synchronises the host.
  *   - The caller owns every buffer, including the workspace.
  *   - Arguments are checked on the host before anything is launched. On an
  *     error status nothing has been launched and no output was touched, except
@@ -85,9 +86,10 @@ typedef enum gdn2_op {
  * fills, so one buffer of gdn2_workspace_size(GDN2_OP_BWD, ...) bytes serves a
  * gdn2_fwd(save_states = 1) followed by a gdn2_bwd(states_saved = 1).
  * GDN2_OP_FWD needs a workspace only on the tensor-core path (dt = GDN2_BF16,
- * Dk = Dv = 128, chunk = 64): there the forward keeps, per chunk, the
- * T | P | Wm tiles of the WY step and a ready flag that hands them from the CTAs
- * that compute them to the CTAs that walk the chunks of a head.
+ * Dk = Dv = 128, chunk = 64): there the forward keeps, per chunk, the image of
+ * the WY step (the T, P and Wm tiles, the scaled query and key tiles and the
+ * chunk's decay) and a ready flag that hands it from the CTAs that compute it
+ * to the CTAs that walk the chunks of a head.
  * Returns 0 for an invalid or unsupported problem and for a forward that needs
  * no workspace. The workspace must be 256-byte aligned; its contents on entry
  * do not matter.
