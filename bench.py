@@ -9,10 +9,19 @@ process per GPU under torchrun) every rank runs its own batch: heads and batch
 entries never interact, so there is no data-path collective (weak scaling).
 Rank 0 prints one JSON line.
 
+Besides the headline step, the line carries (rank 0, N=1):
+  * ``configs``: the forward-only 1.3B layer (B=4, H=16, T=4K, no saved states)
+    and the long forward (B=1, H=16, T=64K, random S0), each with ms, tokens/s
+    and the fraction of its HBM roofline;
+  * ``sweep``: fwd+bwd at a fixed 64K tokens per step for T = 1K..64K
+    (B = 64K / T), the same figures per point;
+  * ``decode``: 1024 in-place decode steps (batch 256, 16 heads, d = 128);
+  * ``cpu_baseline``: the fp64 oracle timed on a bounded sample of the headline
+    workload on the host cores, with the GPU outputs of those same sequences
+    compared against the oracle's (relative L2, whole sample and worst head).
+
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
-sample of the same workload (rank 0 only). ``--sweep`` prints, instead of the
-headline line, one line per sequence length (fwd+bwd at 16K tokens per step,
-T = 1K..16K) and one for the long forward (B=1, H=16, T=64K, S0 given).
+sample of the same workload (rank 0 only).
 """
 from __future__ import annotations
 
@@ -141,8 +150,13 @@ def make_host_inputs(rank, B=None, T=None):
     return wl, make_inputs(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, rank_seed(wl.seed, rank), wl.dtype, with_do=True)
 
 
-def cpu_baseline(wl, x, budget_s=20.0, steps=1):
-    """Time the fp64 oracle (fwd + bwd) on a bounded sample of the workload."""
+def cpu_baseline(wl, x, budget_s=20.0, steps=1, gpu=None):
+    """Time the fp64 oracle (fwd + bwd) on a bounded sample of the workload.
+
+    ``gpu`` (optional): the GPU's outputs of the same step (o and the gradients, CPU tensors of the full
+    workload); the sampled sequences are then compared against the oracle's results on them (relative L2
+    over the sample and the worst single sequence). The forward output is compared at any sample length
+    (it is causal); the gradients only when the sample covers the whole sequence."""
     import oracle
     from linear_attention_delta_gdn_b200.inputs import to_f64
     cores = oracle.threads()
@@ -166,15 +180,29 @@ def cpu_baseline(wl, x, budget_s=20.0, steps=1):
     times = []
     for _ in range(steps):
         t0 = time.perf_counter()
-        oracle.fwd(*(sub[n] for n in names))
-        oracle.bwd(*(sub[n] for n in names), dout=sub["dout"])
+        o_ref, _ = oracle.fwd(*(sub[n] for n in names))
+        g_ref = oracle.bwd(*(sub[n] for n in names), dout=sub["dout"])
         times.append(time.perf_counter() - t0)
     dt = statistics.median(times)
     tokens = nheads * T / wl.H            # token = one position of the 16-head layer
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "fp64 oracle fwd+bwd on %d of %d (batch, head) sequences x %d tokens; tokens = "
-                      "sequences x tokens / %d heads" % (nheads, wl.B * wl.H, T, wl.H),
-            "seconds": dt}
+    out = {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": "fp64 oracle fwd+bwd on %d of %d (batch, head) sequences x %d tokens; tokens = "
+                     "sequences x tokens / %d heads" % (nheads, wl.B * wl.H, T, wl.H),
+           "seconds": dt}
+    if gpu is not None:
+        def rel(a, r):
+            return float(np.linalg.norm((a - r).ravel()) / max(np.linalg.norm(r.ravel()), 1e-300))
+
+        refs = {"o": o_ref}
+        if T == wl.T:
+            refs.update({n: g_ref[n] for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw")})
+        par = {}
+        for n, r in refs.items():
+            a = np.stack([to_f64(gpu[n][b, :T, h]) for b, h in heads])[:, :, None]
+            par[n] = {"rel_l2": rel(a, r), "worst_sequence": max(rel(a[i], r[i]) for i in range(len(heads)))}
+        out["parity"] = {"sequences": nheads, "tokens": T, "errors": par,
+                         "tolerance": {"o": 2e-2, "gradients": 3e-2}}
+    return out
 
 
 def bench_decode(binding, dev, steps=1024, pool=64):
@@ -216,80 +244,129 @@ def bench_decode(binding, dev, steps=1024, pool=64):
             "launches": kern[0]}
 
 
-def run_sweep(args):
-    """Opt-in measurements beside the headline step (one JSON line each, 1 GPU): the fwd+bwd step at a
-    fixed 16K tokens per step for sequence lengths 1K..16K, and the long inference forward (B=1, H=16,
-    T=64K, S0 given). Inputs are drawn on the device with the recipe's distributions (seeded torch
-    generator), since the long case holds ~0.8 GB of token tensors."""
+def device_inputs(B, T, H, D, seed, with_do, dev):
+    """Token inputs drawn on the device with the recipe's distributions (seeded torch generator): the long
+    and swept workloads hold up to ~2 GB of token tensors."""
     import torch
-    from linear_attention_delta_gdn_b200 import binding, build
     from linear_attention_delta_gdn_b200.inputs import make_decode_stream
-    build.build()
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
-    pk = peaks()
     names = ("q", "k", "v", "log_alpha", "b", "w")
+    xs = make_decode_stream(T, B, H, D, D, seed, "bf16", device=dev)   # [T, B, H, D] -> [B, T, H, D]
+    d = {n: xs[n].permute(1, 0, 2, 3).contiguous() for n in names}
+    d["S0"] = xs["S0"]
+    del xs
+    if with_do:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed + 1)
+        d["dout"] = torch.randn((B, T, H, D), generator=gen, device=dev).to(torch.bfloat16)
+    return d
+
+
+def timed_ms(fn, steps, dev, warmup=3):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize(dev)
+    return a.elapsed_time(e) / steps
+
+
+def fwdbwd_point(binding, dev, B, T, H, steps, seed):
+    """fwd (keeping the states) + bwd at one (B, T): ms per step, tokens/s and fraction of the HBM roofline."""
+    import torch
     D = 128
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    pk = peaks()
+    d = device_inputs(B, T, H, D, seed, True, dev)
+    ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_BWD, B, T, H, D, D, 64, binding.GDN2_BF16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    grads = {n: torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+             for n in ("dq", "dk", "dlog_alpha", "db", "dv", "dw")}
+    grads["dS0"] = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
 
-    def device_inputs(B, T, H, seed, with_do):
-        xs = make_decode_stream(T, B, H, D, D, seed, "bf16", device=dev)   # [T, B, H, D] -> [B, T, H, D]
-        d = {n: xs[n].permute(1, 0, 2, 3).contiguous() for n in names}
-        d["S0"] = xs["S0"]
-        if with_do:
-            gen = torch.Generator(device=dev)
-            gen.manual_seed(seed + 1)
-            d["dout"] = torch.randn((B, T, H, D), generator=gen, device=dev).to(torch.bfloat16)
-        return d
+    def step():
+        binding.gdn2_fwd(*(d[n] for n in names), None, save_states=True, ws=ws, o=o, ST=ST)
+        binding.gdn2_bwd(*(d[n] for n in names), d["dout"], None, None, states_saved=True, ws=ws, grads=grads)
 
-    def timed(fn, steps, warmup=3):
-        for _ in range(warmup):
-            fn()
-        torch.cuda.synchronize(dev)
-        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(steps):
-            fn()
-        e.record()
-        torch.cuda.synchronize(dev)
-        return a.elapsed_time(e) / steps
+    ms = timed_ms(step, steps, dev)
+    alg = B * T * H * STEP_BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
+    out = {"workload": "fwdbwd-bf16-b%dh%dt%dd128" % (B, H, T), "B": B, "T": T, "H": H, "ms_per_step": ms,
+           "tokens_per_s": B * T / (ms / 1e3), "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+           "status": binding.gdn2_device_status()}
+    del d, ws, o, ST, grads
+    torch.cuda.empty_cache()
+    return out
 
-    H = 16
-    for T in (1024, 2048, 4096, 8192, 16384):
-        B = 16384 // T
-        d = device_inputs(B, T, H, 3000 + T, True)
-        ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_BWD, B, T, H, D, D, 64, binding.GDN2_BF16),
-                         dtype=torch.uint8, device=dev)
-        o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
-        ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
-        grads = {n: torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
-                 for n in ("dq", "dk", "dlog_alpha", "db", "dv", "dw")}
-        grads["dS0"] = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
 
-        def step():
-            binding.gdn2_fwd(*(d[n] for n in names), None, save_states=True, ws=ws, o=o, ST=ST)
-            binding.gdn2_bwd(*(d[n] for n in names), d["dout"], None, None, states_saved=True, ws=ws, grads=grads)
-
-        ms = timed(step, max(3, args.steps))
-        alg = B * T * H * STEP_BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
-        print(json.dumps({"mode": "sweep", "workload": "fwdbwd-bf16-b%dh%dt%dd128" % (B, H, T), "B": B, "T": T,
-                          "H": H, "ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
-                          "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                          "status": binding.gdn2_device_status()}), flush=True)
-        del d, ws, o, ST, grads
-        torch.cuda.empty_cache()
-
-    B, T = 1, 65536   # the long inference forward, initial state given
-    d = device_inputs(B, T, H, 4000, False)
+def measure_configs(binding, dev, args, fwd_inputs):
+    """The forward-only 1.3B layer (the headline inputs, no saved states) and the long forward (B=1, H=16,
+    T=64K, random S0): ms, tokens/s and the fraction of each one's HBM roofline (its inputs read, o written,
+    the fp32 states read and written)."""
+    import torch
+    D = 128
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    pk = peaks()
+    out = {}
+    B, T, H = fwd_inputs["q"].shape[0], fwd_inputs["q"].shape[1], fwd_inputs["q"].shape[2]
     ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_FWD, B, T, H, D, D, 64, binding.GDN2_BF16),
                      dtype=torch.uint8, device=dev)
     o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
     ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
-    ms = timed(lambda: binding.gdn2_fwd(*(d[n] for n in names), d["S0"], ws=ws, o=o, ST=ST), max(3, args.steps))
+    ms = timed_ms(lambda: binding.gdn2_fwd(*(fwd_inputs[n] for n in names), None, ws=ws, o=o, ST=ST),
+                  max(5, args.steps), dev)
+    alg = B * T * H * KERNEL_BYTES_PER_TOKEN_HEAD["chunk_fwd_kernel"] + B * H * D * D * 4
+    out["fwd-bf16-b%dh%dt%dd128" % (B, H, T)] = {
+        "mode": "forward only (no saved states), zero S0, o and S_T returned", "ms": ms,
+        "tokens_per_s": B * T / (ms / 1e3), "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+        "status": binding.gdn2_device_status()}
+    del ws, o, ST
+
+    B, T = 1, 65536
+    d = device_inputs(B, T, H, D, 4000, False, dev)
+    ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_FWD, B, T, H, D, D, 64, binding.GDN2_BF16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    ms = timed_ms(lambda: binding.gdn2_fwd(*(d[n] for n in names), d["S0"], ws=ws, o=o, ST=ST),
+                  max(5, args.steps // 2), dev)
     alg = B * T * H * KERNEL_BYTES_PER_TOKEN_HEAD["chunk_fwd_kernel"] + 2 * B * H * D * D * 4
-    print(json.dumps({"mode": "sweep", "workload": "fwd-bf16-b1h16t65536d128-S0", "B": B, "T": T, "H": H,
-                      "ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
-                      "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                      "status": binding.gdn2_device_status()}), flush=True)
+    out["fwd-bf16-b1h16t65536d128-s0"] = {
+        "mode": "forward, random S0 ~ N(0, 0.02^2), o and S_T returned", "ms": ms,
+        "tokens_per_s": B * T / (ms / 1e3), "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+        "status": binding.gdn2_device_status()}
+    del d, ws, o, ST
+    torch.cuda.empty_cache()
+    return out
+
+
+SWEEP_TOKENS = 65536
+SWEEP_T = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
+
+
+def measure_sweep(binding, dev, args):
+    """fwd+bwd throughput against sequence length at a fixed 64K tokens per step (B = 64K / T), H = 16."""
+    return [fwdbwd_point(binding, dev, SWEEP_TOKENS // T, T, 16, max(3, args.steps // 4), 3000 + T)
+            for T in SWEEP_T]
+
+
+def run_sweep(args):
+    """The sweep and the extra configs alone, one JSON line each (1 GPU)."""
+    import torch
+    from linear_attention_delta_gdn_b200 import binding, build
+    build.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    for pt in measure_sweep(binding, dev, args):
+        print(json.dumps(dict(mode="sweep", **pt)), flush=True)
+    d = device_inputs(4, 4096, 16, 128, 5000, False, dev)
+    for name, r in measure_configs(binding, dev, args, d).items():
+        print(json.dumps(dict(mode="config", workload=name, **r)), flush=True)
     return 0
 
 
@@ -323,11 +400,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
+    ap.add_argument("--no-extra", action="store_true", help="skip the extra configs and the length sweep")
     ap.add_argument("--B", type=int, default=None, help="override the batch size (small profiling cases)")
     ap.add_argument("--T", type=int, default=None, help="override the sequence length (small profiling cases)")
     ap.add_argument("--sweep", action="store_true",
-                    help="instead of the headline line: fwd+bwd at 16K tokens per step for T = 1K..16K, and "
-                         "the long forward B1 H16 T64K with S0 (one JSON line each, 1 GPU)")
+                    help="instead of the headline line: the length sweep (fwd+bwd at 64K tokens per step, "
+                         "T = 1K..64K) and the extra configs, one JSON line each (1 GPU)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -441,16 +519,22 @@ def main():
                 / (ms_per_step / 1e3) / 1e9 / pk["hbm_gbs"]}
     launches_in_timed_region = sum(v[0] for v in kernels.values())
 
-    decode = None
-    if not args.no_decode and args.B is None and args.T is None:
+    decode = configs = sweep = None
+    full = args.B is None and args.T is None
+    if not args.no_decode and full:
         decode = bench_decode(binding, dev)
+    if not args.no_extra and full and world == 1:
+        configs = measure_configs(binding, dev, args, d)
+        sweep = measure_sweep(binding, dev, args)
 
     line = None
     if rank == 0:
         cb = None
         if not args.no_cpu_baseline and world == 1:
-            cb = cpu_baseline(wl, xh)
-            cb = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            gpu_out = {"o": o.cpu()}
+            gpu_out.update({n: grads[n].cpu() for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw")})
+            cb = cpu_baseline(wl, xh, gpu=gpu_out)
+            cb = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "parity")}
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -463,7 +547,7 @@ def main():
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_in_timed_region,
-                "decode": decode}
+                "decode": decode, "configs": configs, "sweep": sweep}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

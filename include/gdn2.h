@@ -34,10 +34,17 @@
  *     GDN2_ERR_CUDA, which reports a launch failure or an earlier asynchronous
  *     error of the device (outputs are then undefined).
  *   - Gate values are not range-checked (that would cost a pass over HBM).
+ *   - Decay range of the tensor-core path: for every channel, the sum of
+ *     log_alpha over each 64-token chunk must stay above about -88. Below that
+ *     the chunk factors exp(-sum) overflow float and the outputs become
+ *     inf/NaN without an error status. The recurrent kernels have no limit.
  *   - Supported sizes: Dk, Dv in {16, 32, 64, 128}; chunk in {16, 32, 64};
  *     any T >= 0 (a ragged last chunk is allowed); B, H >= 1.
- *     The tensor-core path runs for dt = GDN2_BF16, Dk = Dv = 128, chunk = 64;
- *     every other supported combination runs on the fp32 recurrent kernels.
+ *     The tensor-core path runs for dt = GDN2_BF16, Dk = Dv = 128, with any
+ *     chunk argument: its kernels always use 64-token chunks (the chunkwise
+ *     algorithm is exact, so the chunk length does not change the result).
+ *     Every other supported combination runs on the fp32 recurrent kernels,
+ *     where chunk is the spacing of the state checkpoints of the backward.
  *   - Thread safety: calls may be made from several host threads; error
  *     detail strings are per thread.
  *   - Launches: on the tensor-core path the forward and the backward each run
@@ -163,8 +170,15 @@ gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const 
  *   - Problems whose gdn2_workspace_size(GDN2_OP_BWD, ...) exceeds that size
  *     are rejected with GDN2_ERR_WORKSPACE before anything is launched.
  *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture on the device.
+ *     device, with that device current). Under lazy module loading
+ *     (CUDA_MODULE_LOADING=LAZY, the default) that first lookup also loads the
+ *     library's device code and commits the array's memory, so it can fail for
+ *     lack of memory and it can synchronise: make the first call on each device
+ *     during start-up, and before any stream capture on the device.
+ *   - The looked-up address is kept for the life of the process. After a reset
+ *     of the device (cudaDeviceReset, or a primary context that was released
+ *     and created again) it is stale, and this entry point must not be used on
+ *     that device any more.
  *   - All calls on a device share the array and it keeps the last call's
  *     contents (nothing in it needs to start at zero). Calls whose work overlaps
  *     on the GPU -- other streams or host threads on the same device -- race on

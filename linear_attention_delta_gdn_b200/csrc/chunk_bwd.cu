@@ -50,6 +50,10 @@ __device__ unsigned int g_bwd_error;
 // 32 (w % 4) .. + 31; the four warps of a quarter, part = w / 4, split the columns of a read-out).
 constexpr int BT = 512;
 constexpr int BPARTS = BT / 128;
+// The copy loops move whole images in 16-byte pieces per thread and the gate chain maps thread tid to
+// (key channel tid % 128, token quarter tid / 128): both need exactly BT threads (checked at kernel entry).
+static_assert(TC_STATE_BYTES % (16 * BT) == 0 && TC_DELTA_BYTES % (16 * BT) == 0 && BPARTS * 16 == 64,
+              "BT-thread loops");
 
 // Copy a [128 lanes x NCOL] fp32 accumulator into a bf16 row tile of 128 rows (row = lane); each of
 // the four warps of a lane quarter takes NCOL / 4 columns.
@@ -746,6 +750,10 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 32);
     int* abort_flag = reinterpret_cast<int*>(sm + OFF_BARS + 36);
     NextUnit* nxt = reinterpret_cast<NextUnit*>(sm + OFF_BARS + 40);
+    if (blockDim.x != BT) {   // the index arithmetic assumes BT threads: refuse any other launch shape
+        if (tid == 0) atomicOr(&g_bwd_error, 16u);
+        return;
+    }
     if (tid == 0) {
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
         tc::mbar_init(reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48), 1);

@@ -71,6 +71,9 @@ static_assert(sp::BAR + 64 <= sp::UU1 && sp::UU1 % 1024 == 0 && sp::WW1 % 1024 =
 static_assert(4 * 16 * XS * 4 <= wy::GC - wy::SX && 8 * 128 * 4 <= wy::GC - wy::SX, "producer scratch fits");
 static_assert(TC_WY_QT == 32768 && TC_WY_KT == 49152 && TC_WY_GC == 65536, "WY image: T | P | Wm | Qt | Kt | gC");
 static_assert(wy::TF == wy::IMG + TC_WY_WM, "T | P | Wm contiguous in shared memory as in the image");
+// The per-thread copy loops below are written for NT threads: copy_wy moves 8 (T | P | Wm) and 4 (Qt, Kt)
+// 16-byte pieces per thread, the U = w*v loop 4 rows of 8 values. The kernel checks blockDim.x == NT.
+static_assert(8 * 16 * NT == TC_WY_QT && 4 * 16 * NT == TILE_64x128 && 4 * NT * 8 == C * D, "NT-thread loops");
 
 // TMEM columns. Consumer: S^T (fp32 state), Ut^T -> Delta^T, O x 2 (M=64). Producer pipeline g: [A; P] at
 // 256 g, Wm (M=64) at 256 g + 64.
@@ -641,6 +644,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
     const int tid = threadIdx.x, warp = tid >> 5;
+    if (blockDim.x != NT) {   // the index arithmetic assumes NT threads: refuse any other launch shape
+        if (tid == 0) atomicOr(&g_fwd_error, 16u);
+        return;
+    }
     const bool consumer = (int)blockIdx.x < p.ncons;
     const uint32_t bar_off = consumer ? sp::BAR : wy::BAR;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + bar_off);

@@ -64,7 +64,7 @@ size_t tc_wy_bytes(const Dims& d) { return tc_units(d) * TC_WY_BYTES + align256(
 // Forward-saved region: chunk-start states (and, on the tensor-core path, Delta^T, the WY images and flags).
 size_t states_bytes(const Dims& d, gdn2_dtype dt) {
     const size_t units = tc_units(d);
-    return tc_train_path(dt, d.Dk, d.Dv, d.chunk) ? units * (TC_STATE_BYTES + TC_DELTA_BYTES) + tc_wy_bytes(d)
+    return tc_path(dt, d.Dk, d.Dv) ? units * (TC_STATE_BYTES + TC_DELTA_BYTES) + tc_wy_bytes(d)
                                                   : units * d.Dk * d.Dv * sizeof(float);
 }
 size_t tc_delta_offset(const Dims& d) { return tc_units(d) * TC_STATE_BYTES; }
@@ -74,7 +74,7 @@ size_t tc_flags_offset(const Dims& d, bool with_states) {
 }
 
 size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
-    if (tc_train_path(dt, d.Dk, d.Dv, d.chunk))   // dZ and dDelta images, ready flags, work counter, abort word
+    if (tc_path(dt, d.Dk, d.Dv))   // dZ and dDelta images, ready flags, work counter, abort word
         return tc_units(d) * (TC_STATE_BYTES + TC_DELTA_BYTES) + align256((tc_units(d) + 2) * sizeof(unsigned int));
     const size_t seg = (size_t)d.B * d.H * d.chunk * d.Dk * d.Dv * sizeof(float);
     const size_t del = (size_t)d.B * d.H * d.chunk * d.Dv * sizeof(float);
@@ -139,16 +139,17 @@ gdn2_status gdn2_device_status(void* stream) {
     if (fwd | bwd)
         return fail(GDN2_ERR_TIMEOUT,
                     "device wait gave up: chunk_fwd_kernel bits 0x%x, chunk_bwd_kernel bits 0x%x "
-                    "(1 MMA completion, 2 tile loads, 4 forward ready flag / gradient unit, 8 backward ready flag)",
+                    "(1 MMA completion, 2 tile loads, 4 forward ready flag / gradient unit, 8 backward ready flag, "
+                    "16 launched with a block size the kernel is not built for)",
                     fwd, bwd);
     return GDN2_OK;
 }
 
 size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt) {
     if (check_dims(B, T, H, Dk, Dv, chunk, dt, true) != GDN2_OK) return 0;
-    const Dims d{B, T, H, Dk, Dv, chunk};
+    const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
     switch (op) {
-    case GDN2_OP_FWD: return tc_path(dt, Dk, Dv, chunk) ? align256(tc_wy_bytes(d)) : 0;
+    case GDN2_OP_FWD: return tc_path(dt, Dk, Dv) ? align256(tc_wy_bytes(d)) : 0;
     case GDN2_OP_FWD_SAVE: return align256(states_bytes(d, dt));
     case GDN2_OP_BWD: return align256(states_bytes(d, dt)) + align256(bwd_extra_bytes(d, dt));
     }
@@ -161,7 +162,7 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
                      void* stream) {
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
-    const Dims d{B, T, H, Dk, Dv, chunk};
+    const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     OPTIONAL_PTR(S0);
     OPTIONAL_PTR(ST);
@@ -175,7 +176,7 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
                         save_states ? " with save_states" : "", need, ws ? ws_bytes : 0);
         if (need && !aligned(ws, 256)) return fail(GDN2_ERR_INVALID, "ws must be 256-byte aligned");
     }
-    if (save_states ? tc_train_path(dt, Dk, Dv, chunk) : tc_path(dt, Dk, Dv, chunk)) {
+    if (tc_path(dt, Dk, Dv)) {
         ChunkFwdArgs a{};
         a.d = d;
         a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
@@ -205,7 +206,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
                      size_t ws_bytes, void* stream) {
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
-    const Dims d{B, T, H, Dk, Dv, chunk};
+    const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     OPTIONAL_PTR(S0);
     OPTIONAL_PTR(dST);
@@ -222,7 +223,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     unsigned char* extra = wsb + align256(states_bytes(d, dt));
 
-    if (tc_train_path(dt, Dk, Dv, chunk)) {
+    if (tc_path(dt, Dk, Dv)) {
         if (!states_saved) {
             ChunkFwdArgs f{};
             f.d = d;
@@ -263,7 +264,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
     a.op = RecurrentArgs::BWD;
     a.dout = dout; a.dST = dST;
     a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.db = db; a.dw = dw; a.dS0 = dS0;
-    const size_t seg = (size_t)B * H * chunk * Dk * Dv * sizeof(float);
+    const size_t seg = (size_t)B * H * d.chunk * Dk * Dv * sizeof(float);
     a.seg = reinterpret_cast<float*>(extra);
     a.segdelta = reinterpret_cast<float*>(extra + align256(seg));
     return cuda_status(recurrent_launch(a, s), "gdn2_bwd (recurrent path)");

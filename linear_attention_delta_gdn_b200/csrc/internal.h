@@ -96,15 +96,13 @@ cudaError_t chunk_bwd_take_errors(unsigned int* bits);
 // Sets the detail string returned by gdn2_last_error() on this host thread.
 void set_last_error(const char* msg);
 
-// Whether the tensor-core forward handles this problem.
-inline bool tc_path(gdn2_dtype dt, int Dk, int Dv, int chunk) {
-    return dt == GDN2_BF16 && Dk == TC_D && Dv == TC_D && chunk == TC_C;
-}
-// Whether the tensor-core backward is built.
-constexpr bool kTcBackward = true;
-// Whether training (fwd with saved states + bwd) runs on the tensor-core kernels.
-inline bool tc_train_path(gdn2_dtype dt, int Dk, int Dv, int chunk) {
-    return kTcBackward && tc_path(dt, Dk, Dv, chunk);
+// Whether the tensor-core kernels handle this problem: bf16 with d_k = d_v = 128. They always run the
+// WY algorithm on 64-token chunks; the result does not depend on the chunk length in exact arithmetic,
+// so a requested chunk of 16 or 32 is served by the same kernels.
+inline bool tc_path(gdn2_dtype dt, int Dk, int Dv) { return dt == GDN2_BF16 && Dk == TC_D && Dv == TC_D; }
+// The sizes a call runs with: on the tensor-core path the chunk is the kernels' 64.
+inline Dims run_dims(int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt) {
+    return Dims{B, T, H, Dk, Dv, tc_path(dt, Dk, Dv) ? TC_C : chunk};
 }
 
 }  // namespace gdn2

@@ -24,6 +24,27 @@ def rel_l2(x, ref):
     return num / den if den > 0 else num
 
 
+def worst_head_rel_l2(x, ref, state=False):
+    """Largest per-(batch, head) relative L2 error: token tensors are [B, T, H, D], states [B, H, Dk, Dv].
+
+    A whole-tensor figure can hide one bad head (or one bad stretch of chunks of one head); this one
+    cannot. Heads whose reference is zero use the absolute L2, as rel_l2 does."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    worst = 0.0
+    if state:
+        for b in range(ref.shape[0]):
+            for h in range(ref.shape[1]):
+                worst = max(worst, rel_l2(x[b, h], ref[b, h]))
+    else:
+        if ref.shape[1] == 0:
+            return 0.0
+        for b in range(ref.shape[0]):
+            for h in range(ref.shape[2]):
+                worst = max(worst, rel_l2(x[b, :, h], ref[b, :, h]))
+    return worst
+
+
 @pytest.fixture(scope="session")
 def oracle_mod():
     import oracle

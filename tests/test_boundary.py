@@ -65,6 +65,10 @@ def test_workspace_sizes(L):
     assert b == f + units * (32768 + 16384) + (units * 4 + 256)
     # ragged T rounds the chunk count up
     assert ws(1, 1, 65, 1, 128, 128, 64, 1) == ws(1, 1, 128, 1, 128, 128, 64, 1)
+    # bf16 d = 128 runs the tensor-core kernels (64-token chunks) whatever chunk is requested
+    for op in (0, 1, 2):
+        for c in (16, 32):
+            assert ws(op, 2, 300, 3, 128, 128, c, 1) == ws(op, 2, 300, 3, 128, 128, 64, 1)
     # invalid problems report zero
     assert ws(1, 0, 16, 1, 64, 64, 64, 1) == 0
     assert ws(1, 1, 16, 1, 96, 64, 64, 1) == 0

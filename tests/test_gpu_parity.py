@@ -1,18 +1,19 @@
 """GPU parity: libgdn2 (through its C ABI) against the fp64 oracle on the same
 seeded inputs.
 
-Tolerances (relative L2 over a whole tensor, ||x - ref|| / ||ref||):
+Tolerances (relative L2, ||x - ref|| / ||ref||), applied to the whole tensor AND to
+every (batch, head) slice on its own, so that one bad head cannot hide among good ones:
   fp32 inputs: o, S_T and every gradient <= 1e-4
   bf16 inputs (fp32 state and accumulation): o, S_T <= 2e-2; gradients <= 3e-2
-The oracle consumes exactly the dtype-rounded inputs, widened to fp64. Full-size
-workloads are checked on sampled (batch, head) pairs, which the oracle computes
+The oracle consumes exactly the dtype-rounded inputs, widened to fp64. The full-size
+workloads are checked on every (batch, head) pair; the oracle computes each pair
 independently of the others (heads never interact).
 """
 import numpy as np
 import pytest
 import torch
 
-from conftest import rel_l2
+from conftest import rel_l2, worst_head_rel_l2
 from linear_attention_delta_gdn_b200 import binding
 from linear_attention_delta_gdn_b200.inputs import WORKLOADS, make_inputs, make_workload_inputs, make_decode_stream, to_f64
 
@@ -84,10 +85,12 @@ def pick(arr, heads, state=False):
 def check_fwd(oracle_mod, x, chunk, dtype, heads=None):
     o, ST = gpu_fwd(x, chunk)
     o_ref, ST_ref = oracle_fwd(oracle_mod, x, heads)
-    eo, es = rel_l2(pick(o, heads), o_ref), rel_l2(pick(ST, heads, True), ST_ref)
+    o, ST = pick(o, heads), pick(ST, heads, True)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(ST))
-    assert eo <= TOL_OUT[dtype], "o rel err %.3g" % eo
-    assert es <= TOL_OUT[dtype], "S_T rel err %.3g" % es
+    eo, es = rel_l2(o, o_ref), rel_l2(ST, ST_ref)
+    wo, ws = worst_head_rel_l2(o, o_ref), worst_head_rel_l2(ST, ST_ref, state=True)
+    assert eo <= TOL_OUT[dtype] and wo <= TOL_OUT[dtype], "o rel err %.3g (worst head %.3g)" % (eo, wo)
+    assert es <= TOL_OUT[dtype] and ws <= TOL_OUT[dtype], "S_T rel err %.3g (worst head %.3g)" % (es, ws)
     return eo, es
 
 
@@ -147,10 +150,34 @@ def test_fwd_bf16_d128(oracle_mod, T, with_S0):
     check_fwd(oracle_mod, x, 64, "bf16")
 
 
-@pytest.mark.parametrize("Dk,Dv,chunk", [(64, 64, 64), (128, 128, 32), (64, 128, 16)])
+# bf16 shapes off the tensor-core shape (d_k = d_v = 128) run on the recurrent kernels (bf16 in, fp32 math);
+# bf16 at d = 128 with chunk 16 or 32 runs on the tensor-core kernels (64-token chunks inside).
+BF16_SHAPES = [(64, 64, 64), (128, 128, 32), (128, 128, 16), (64, 128, 16), (128, 64, 32), (16, 16, 64),
+               (32, 128, 64)]
+
+
+@pytest.mark.parametrize("Dk,Dv,chunk", BF16_SHAPES)
 def test_fwd_bf16_other_shapes(oracle_mod, Dk, Dv, chunk):
     x = make_inputs(2, 97, 2, Dk, Dv, seed=200 + Dk + chunk, dtype="bf16", with_S0=True)
     check_fwd(oracle_mod, x, chunk, "bf16")
+
+
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_bf16_d128_small_chunk_runs_on_tensor_cores(oracle_mod, chunk):
+    """The chunk length does not change the result, so bf16 d = 128 with chunk 16 or 32 takes the tensor-core
+    kernels (64-token chunks) instead of the token-recurrent ones."""
+    x = make_inputs(1, 150, 3, 128, 128, seed=210 + chunk, dtype="bf16", with_do=True, with_S0=True)
+    binding.trace_read()
+    binding.trace_enable(True)
+    try:
+        check_fwd(oracle_mod, x, chunk, "bf16")
+        check_bwd(oracle_mod, x, chunk, "bf16", with_dST=True)
+        check_bwd(oracle_mod, x, chunk, "bf16", with_dST=True, saved=True)
+    finally:
+        binding.trace_enable(False)
+    names = set(binding.trace_read())
+    assert {"chunk_fwd_kernel", "chunk_bwd_kernel"} <= names, names
+    assert not names & {"recurrent_fwd_kernel", "recurrent_bwd_kernel"}, names
 
 
 def test_fwd_workload_fp32(oracle_mod):
@@ -158,13 +185,11 @@ def test_fwd_workload_fp32(oracle_mod):
     check_fwd(oracle_mod, make_workload_inputs(wl), wl.chunk, wl.dtype)
 
 
-@pytest.mark.parametrize("name,heads", [
-    ("fwd-bf16-b4h16t4096d128", [(0, 0), (1, 7), (2, 13), (3, 15)]),
-    ("fwd-bf16-b1h16t65536d128-s0", [(0, 0), (0, 9), (0, 15)]),
-])
-def test_fwd_workload_sampled(oracle_mod, name, heads):
+@pytest.mark.parametrize("name", ["fwd-bf16-b4h16t4096d128", "fwd-bf16-b1h16t65536d128-s0"])
+def test_fwd_workload_all_heads(oracle_mod, name):
+    """The full-size forward workloads, every (batch, head) pair against the oracle."""
     wl = WORKLOADS[name]
-    check_fwd(oracle_mod, make_workload_inputs(wl), wl.chunk, wl.dtype, heads=heads)
+    check_fwd(oracle_mod, make_workload_inputs(wl), wl.chunk, wl.dtype)
 
 
 def test_fwd_resume_from_state(oracle_mod):
@@ -192,9 +217,17 @@ def test_fwd_state_in_place(oracle_mod):
 
 # ---------------------------------------------------------------- backward
 
+# Exact retrieval (b = 1, q = k, unit keys): the outputs do not depend on the state, so the gradient reaching
+# S0 is only the incoming dST carried back through the decays and erases, ~1/2700 of it at these shapes. There
+# dS0 is ill-conditioned: perturbing the inputs by half a bf16 ulp moves the oracle's own dS0 by more than its
+# norm, ~5e-4 of ||dST|| (tests/test_oracle_pins.py::test_exact_retrieval_dS0_is_ill_conditioned). Its error
+# is therefore measured against ||dST||, with a bound a few times that input-level sensitivity.
+DS0_VS_DST_TOL = 3e-3
+
+
 def check_bwd(oracle_mod, x, chunk, dtype, heads=None, with_dST=False, saved=False, ds0_vs_dST=False):
-    """Gradients against the oracle. With ds0_vs_dST the error of dS0 is measured against the norm of the
-    incoming state gradient dST instead of its own (for inputs where dS0 is a near-cancellation)."""
+    """Gradients against the oracle, whole tensor and worst (batch, head). With ds0_vs_dST the error of dS0 is
+    measured against the norm of the incoming state gradient dST (see DS0_VS_DST_TOL)."""
     d = dev(x)
     dST = None
     if with_dST:
@@ -213,19 +246,25 @@ def check_bwd(oracle_mod, x, chunk, dtype, heads=None, with_dST=False, saved=Fal
                              None if dST is None else dST.cuda(), chunk=chunk)
     torch.cuda.synchronize()
     ref = oracle_bwd(oracle_mod, x, None if dST is None else dST.double().numpy(), heads)
-    errs = {}
+    errs, worst = {}, {}
     for n in GRADS:
-        got = to_f64(g[n])
+        got = pick(to_f64(g[n]), heads)
         assert np.all(np.isfinite(got)), n
-        errs[n] = rel_l2(pick(got, heads), ref[n])
+        errs[n] = rel_l2(got, ref[n])
+        worst[n] = worst_head_rel_l2(got, ref[n])
+    got = pick(to_f64(g["dS0"]), heads, True)
+    assert np.all(np.isfinite(got)), "dS0"
     if ds0_vs_dST:
         assert dST is not None
-        errs["dS0"] = float(np.linalg.norm((pick(to_f64(g["dS0"]), heads, True) - ref["dS0"]).ravel())
-                            / np.linalg.norm(dST.double().numpy().ravel()))
+        dST_ref = pick(dST.double().numpy(), heads, True)
+        e = float(np.linalg.norm((got - ref["dS0"]).ravel()) / np.linalg.norm(dST_ref.ravel()))
+        assert e <= DS0_VS_DST_TOL, "dS0 error %.3g of ||dST|| (bound %g)" % (e, DS0_VS_DST_TOL)
     else:
-        errs["dS0"] = rel_l2(pick(to_f64(g["dS0"]), heads, True), ref["dS0"])
-    bad = {n: e for n, e in errs.items() if e > TOL_GRAD[dtype]}
-    assert not bad, "gradient rel errors above %g: %s (all: %s)" % (TOL_GRAD[dtype], bad, errs)
+        errs["dS0"] = rel_l2(got, ref["dS0"])
+        worst["dS0"] = worst_head_rel_l2(got, ref["dS0"], state=True)
+    bad = {n: (errs[n], worst[n]) for n in errs if max(errs[n], worst[n]) > TOL_GRAD[dtype]}
+    assert not bad, "gradient rel errors (whole, worst head) above %g: %s (all: %s; worst heads: %s)" % (
+        TOL_GRAD[dtype], bad, errs, worst)
     return errs
 
 
@@ -249,11 +288,22 @@ def test_bwd_saved_states(oracle_mod, saved):
     check_bwd(oracle_mod, x, 64, "bf16", with_dST=True, saved=saved)
 
 
-def test_bwd_workload_sampled(oracle_mod):
+def test_bwd_workload_all_heads(oracle_mod):
+    """The full-size training workload (the bench step: forward keeping the states, then the backward), every
+    (batch, head) pair against the oracle."""
     wl = WORKLOADS["fwdbwd-bf16-b4h16t4096d128"]
     x = make_workload_inputs(wl)
-    errs = check_bwd(oracle_mod, x, wl.chunk, wl.dtype, heads=[(0, 0), (1, 6), (2, 11), (3, 15)], saved=True)
-    print("sampled-head gradient rel errors:", errs)
+    errs = check_bwd(oracle_mod, x, wl.chunk, wl.dtype, saved=True)
+    print("gradient rel errors:", errs)
+
+
+@pytest.mark.parametrize("Dk,Dv,chunk", BF16_SHAPES)
+@pytest.mark.parametrize("saved", [False, True])
+def test_bwd_bf16_other_shapes(oracle_mod, Dk, Dv, chunk, saved):
+    """bf16 backward off the tensor-core shape (the bf16 instantiation of the recurrent backward), and bf16
+    d = 128 with chunk 16 or 32 (tensor-core kernels)."""
+    x = make_inputs(2, 97, 2, Dk, Dv, seed=220 + Dk + Dv + chunk, dtype="bf16", with_do=True, with_S0=True)
+    check_bwd(oracle_mod, x, chunk, "bf16", with_dST=True, saved=saved)
 
 
 def test_autograd_matches_direct():

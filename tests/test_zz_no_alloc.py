@@ -78,3 +78,33 @@ def test_no_alloc_rejects_problems_larger_than_the_array():
                              4, 4096, 16, 128, 128, 64, binding.GDN2_BF16, None)
     assert rc == 3
     assert b"fixed array holds" in L.gdn2_last_error()
+
+
+def test_no_alloc_accepts_exactly_the_problems_that_fit():
+    """The size check sits exactly at the array's capacity: on the tensor-core shape (bf16, d = 128), the
+    largest sequence of one head whose backward scratch fits passes the size check (on a host without a GPU
+    the call then stops at the device lookup with GDN2_ERR_CUDA; with a GPU present that call is not made,
+    since it would launch on the placeholder pointers), and one more 64-token chunk is refused with
+    GDN2_ERR_WORKSPACE before anything runs."""
+    from linear_attention_delta_gdn_b200 import build
+    build.build()
+    L = binding.lib()
+    cap = L.gdn2_no_alloc_scratch_bytes()
+
+    def need(n):   # backward scratch of one head of n 64-token chunks
+        return binding.gdn2_workspace_size(binding.GDN2_OP_BWD, 1, 64 * n, 1, 128, 128, 64, binding.GDN2_BF16)
+
+    n = 1
+    while need(n + 1) <= cap:
+        n += 1
+    assert need(n) <= cap < need(n + 1)
+    assert n >= 300      # a few hundred 64-token chunk-heads fit in the array
+    p = ctypes.c_void_p(1 << 20)
+    cases = [(n + 1, False)] + ([] if torch.cuda.is_available() else [(n, True)])
+    for chunks, fits in cases:
+        rc = L.gdn2_bwd_no_alloc(*([p] * 6), None, p, None, p, p, p, p, p, p, None,
+                                 1, 64 * chunks, 1, 128, 128, 64, binding.GDN2_BF16, None)
+        if fits:
+            assert rc == 4, L.gdn2_last_error()      # past the size check, stopped at the device lookup
+        else:
+            assert rc == 3 and b"fixed array holds" in L.gdn2_last_error()
