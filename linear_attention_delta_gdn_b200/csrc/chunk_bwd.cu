@@ -4,29 +4,31 @@
 // "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention" (arXiv
 // abstract) names a gate-aware backward that keeps training parallel; the page
 // prints no equations. The adjoint of the chunk form (see chunk_common.cuh), for
-// one chunk with start state S, S' = Diag(gC) (S + Kt^T Delta), next-state gradient dS'
-// and output gradient dO; write dZ = Diag(gC) dS' (the gradient of S + Kt^T Delta):
-//   dDelta = Kt dZ + P^T dO                          (P = tril(Qt Kt^T))
-//   dS     = dZ + Qt^T dO - Wm^T dDelta              -> gradient of the chunk-start state
+// one chunk with start state S, S' = Diag(gC) S + Kh^T Delta, next-state gradient dS'
+// and output gradient dO:
+//   dDelta = Kh dS' + P^T dO                         (P = tril(Qt Kt^T))
+//   dS     = Diag(gC) dS' + Qt^T dO - Wm^T dDelta    -> gradient of the chunk-start state
 //   dU     = T^T dDelta                              -> dv = dU*w, dw = dU*v
 //   dP     = (dO Delta^T) * incl,  dA = -(dU Delta^T) * strict
 //   dQt    = dO S^T + dP Kt,       dEt = -dU S^T + dA Kt
-//   dKt    = dP^T Qt + dA^T Et + Delta dZ^T
+//   dKt    = dP^T Qt + dA^T Et,    dKh = Delta dS'^T
 // (dA uses T^T dT T^T = dU Delta^T, since dT = dDelta (U - Et S)^T = dDelta Delta^T (I + A)^T.)
-// Gate chain through g = exp(G), G = in-chunk cumsum of log_alpha:
-//   dq = g*dQt;  dE = g*dEt;  db = dE*k;  dk = dKt/g + dE*b
-//   dG_t = Qt*dQt + Et*dEt - Kt*dKt;  the last position also gets
-//   E = rowsum(dZ * S) + sum_t Kt_t * (Delta dZ^T)_t   (the dependence of S' on gC)
+// Gate chain through g = exp(G), h = exp(G_C - G) (G = in-chunk cumsum of log_alpha):
+//   dq = g*dQt;  dE = g*dEt;  dkK = dKt/g + h*dKh;  db = dE*k;  dk = dkK + dE*b
+//   dG_t = q*dq + e*dE - k*dkK   (e = b*k);  the last position also gets
+//   E = gC * rowsum(dS' * S) + sum_t Kh_t * dKh_t   (the dependence of S' on gC)
 //   dlog_alpha_t = sum_{tau >= t} dG_tau + E
+// Untame channels (chunk_common.cuh) have Kt = 0 in the tensor-core products; their pair terms of
+// dq, dE and dkK are summed exactly on CUDA cores with exp(G_t - G_s) as a running product of alpha.
 //
 // One launch, two kinds of work, both reading the forward's per-chunk T and P tiles instead of
 // redoing the solve:
 //   reverse pass    one CTA per (batch, head) walks the chunks backwards carrying dS^T in TMEM
-//                   (fp32); per chunk it writes dZ^T as a bf16 image and then sets the chunk's
+//                   (fp32); per chunk it writes dS'^T as a bf16 image and then sets the chunk's
 //                   ready flag (release);
 //   chunk gradients every other CTA takes (head, chunk) units from a shared counter, in the
 //                   order the reverse pass produces them, waits for the unit's flag (acquire) and
-//                   computes every gradient of the chunk from the saved S, Delta (forward), dZ,
+//                   computes every gradient of the chunk from the saved S, Delta (forward), dS',
 //                   dDelta (reverse pass), T, P, the inputs and dout. Reverse-pass CTAs join them
 //                   once their head is done.
 // With few heads this is one cooperative launch (all CTAs resident, so every wait ends; each wait is
@@ -71,29 +73,45 @@ __device__ __forceinline__ void tmem_rows_to_tile(uint32_t lane_base_col, unsign
 // Gradient-unit prep, thread = (key channel i = tid % 128, token quarter qt = tid / 128: tokens
 // 16 qt .. 16 qt + 15):
 //   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127)
-//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT (k stays in KH);
-//   g[t][i] = exp(G) and 1/g go to TMEM at tmem_g and tmem_ig (lane i, column t) for the gate chain.
-//   Quarter sums of log_alpha are exchanged through qsum (fp32 [4][128]). Contains one __syncthreads.
-__device__ __forceinline__ void grad_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
-                                          float* qsum, int tid, uint32_t tmem_g, uint32_t tmem_ig) {
+//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT (zero on untame channels; k stays in KH);
+//   g[t][i] = exp(G) and h[t][i] = exp(G_C - G) go to TMEM at tmem_g and tmem_h (lane i, column t) for the
+//   gate chain. Quarter sums of log_alpha and of |log_alpha| are exchanged through qsum (fp32 [2][4][128]).
+//   Sets *any_untame when channel i is untame. Contains one __syncthreads.
+struct PrepOut {
+    float gC;       // exp(G_C) of channel i
+    bool untame;    // channel i is left out of the tensor-core pair products
+};
+__device__ __forceinline__ PrepOut grad_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
+                                             float* qsum, int tid, uint32_t tmem_g, uint32_t tmem_h,
+                                             int* any_untame) {
     const int i = tid & 127, qt = tid >> 7;
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chunk = (uint32_t)((i & 63) >> 3);
     float la[16];
-    float s0 = 0.f, s1 = 0.f;
+    float s0 = 0.f, s1 = 0.f, m = 0.f;
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
         const uint32_t t = (uint32_t)(16 * qt + u);
         la[u] = tc::ld_bf16(KT, col64 + t * 128 + ((chunk ^ (t & 7)) << 4));
         if (u & 1) s1 += la[u]; else s0 += la[u];
+        m += fabsf(la[u]);
     }
     qsum[qt * 128 + i] = s0 + s1;
+    qsum[512 + qt * 128 + i] = m;
     __syncthreads();   // also: every log_alpha is read before Kt overwrites it
-    float G = 0.f;
-#pragma unroll 1
-    for (int q = 0; q < qt; ++q) G += qsum[q * 128 + i];
-    float gvals[16], igvals[16];
+    float G = 0.f, tot = 0.f, mass = 0.f;
+#pragma unroll
+    for (int q = 0; q < BPARTS; ++q) {
+        const float x = qsum[q * 128 + i];
+        tot += x;
+        if (q < qt) G += x;
+        mass += qsum[512 + q * 128 + i];
+    }
+    const bool untame = mass > TAME_LOG_DECAY;
+    if (untame && qt == 0) *reinterpret_cast<volatile int*>(any_untame) = 1;
+    const float gC = fast_exp(tot), igC = 1.f / gC;
+    float gvals[16], hvals[16];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         float kk[8], bb[8], qq[8];
@@ -111,23 +129,25 @@ __device__ __forceinline__ void grad_prep(unsigned char* QE, const unsigned char
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             G += la[8 * half + u];
-            const float g = fast_exp(G), ig = fast_exp(-G);
+            const float g = fast_exp(G), h = fast_exp(tot - G);
             gvals[8 * half + u] = g;
-            igvals[8 * half + u] = ig;
-            tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);          // Et
-            tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);        // Qt
-            tc::st_bf16(KT, o64[u], kk[u] * ig);                  // Kt
+            hvals[8 * half + u] = h;
+            tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);                  // Et
+            tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);                // Qt
+            tc::st_bf16(KT, o64[u], untame ? 0.f : kk[u] * h * igC);      // Kt = k/g
         }
     }
     tc::tmem_st16(tmem_g + 16 * qt, gvals);
-    tc::tmem_st16(tmem_ig + 16 * qt, igvals);
+    tc::tmem_st16(tmem_h + 16 * qt, hvals);
     tc::tmem_wait_st();
+    return PrepOut{gC, untame};
 }
 
 constexpr uint32_t TILE_C = 64 * 64 * 2;   // bytes of a 64 x 64 bf16 tile
 
 // Barrier block shared by both kinds of work (above every tile of either layout):
-// 4 mbarriers (load, mma, k, b), TMEM base, abort flag, next unit (2 ints), prefetch mbarrier at +48.
+// 4 mbarriers (load, mma, k, b), TMEM base, abort flag, next unit (2 ints), prefetch mbarrier at +48,
+// "this unit has an untame channel" flag at +56.
 constexpr uint32_t OFF_BARS = 229888;
 constexpr uint32_t SMEM_BYTES_ALL = 229952 + 1024;
 
@@ -136,6 +156,7 @@ struct BwdMaps {
 };
 struct BwdParams {
     int T, H, BH, nc;
+    const __nv_bfloat16 *q_raw, *la_raw;   // raw inputs, read directly only for untame channels
     int nrev;                        // CTAs [0, nrev) run the reverse pass of head blockIdx.x
     int join;                        // reverse-pass CTAs take gradient units afterwards
     int grad;                        // this launch computes gradient units
@@ -145,9 +166,9 @@ struct BwdParams {
     const unsigned char* states;     // chunk-start state images
     const unsigned char* deltas;     // Delta^T images of the forward
     const unsigned char* tp;         // WY images (T | P | Wm)
-    unsigned char* dstates;          // dZ^T images
+    unsigned char* dstates;          // dS'^T images
     unsigned char* ddeltas;          // dDelta^T images
-    unsigned int* flags;             // [BH, nc] dZ ready flags (zero at launch)
+    unsigned int* flags;             // [BH, nc] dS' ready flags (zero at launch)
     unsigned int* counter;           // [0]: next gradient unit, [1]: abort word (zero at launch)
 };
 // mbarrier parities carried across the units a CTA works on
@@ -155,7 +176,7 @@ struct Phases {
     uint32_t load = 0, mma = 0, k = 0, b = 0, pre = 0;
 };
 // The next gradient unit of a CTA, handed between units through shared memory (OFF_BARS + 40):
-// [0] unit index, [1] nonzero once its S, T and dZ^T images are being prefetched (flag acquired).
+// [0] unit index, [1] nonzero once its S, T and dS'^T images are being prefetched (flag acquired).
 struct NextUnit {
     int unit, prefetched;
 };
@@ -163,22 +184,22 @@ struct NextUnit {
 // ====================================================================== reverse state pass
 
 namespace rs {
-// Qt, Kt, dout, Wm and gC alternate between two buffers by chunk parity, so the next chunk's tiles
-// can land while this chunk's MMAs read the current ones; P has one buffer. Qt, Kt, Wm, P and gC come
+// Qt, Kh, dout, Wm and gC alternate between two buffers by chunk parity, so the next chunk's tiles
+// can land while this chunk's MMAs read the current ones; P has one buffer. Qt, Kh, Wm, P and gC come
 // from the forward's WY image.
 constexpr uint32_t OFF_QQ = 0;           // 2 x Qt (64 rows), at +0 / +16384
-constexpr uint32_t OFF_KT0 = 49152;      // Kt (even chunks)
+constexpr uint32_t OFF_KT0 = 49152;      // Kh (even chunks)
 constexpr uint32_t OFF_DO0 = 65536;      // dout (even chunks)
 constexpr uint32_t OFF_WW0 = 81920;      // Wm (even chunks)
-constexpr uint32_t OFF_ST = 98304;       // dZ^T (bf16)
+constexpr uint32_t OFF_ST = 98304;       // dS'^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16)
 constexpr uint32_t OFF_PP = 147456;      // P
 constexpr uint32_t OFF_DO1 = 163840;     // dout (odd chunks)
 constexpr uint32_t OFF_WW1 = 180224;     // Wm (odd chunks)
-constexpr uint32_t OFF_KT1 = 196608;     // Kt (odd chunks)
+constexpr uint32_t OFF_KT1 = 196608;     // Kh (odd chunks)
 constexpr uint32_t OFF_GC = 212992;      // 2 x fp32 gC[128] (by parity)
 constexpr uint32_t TM_S = 0, TM_D = 128;
-constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 512;   // Qt, Kt, dout, Wm, P, gC
+constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 512;   // Qt, Kh, dout, Wm, P, gC
 }  // namespace rs
 static_assert(rs::OFF_GC + 1024 <= OFF_BARS, "reverse-pass layout lies below the barrier block");
 
@@ -205,7 +226,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 32 * tm_part(warp);      // lane row, column quarter
 
     // chunk c's tiles arrive on one barrier phase, issued in three groups as their buffers free up
-    // dout, Qt, Kt, Wm, gC (buffers of this parity are free): issued by lane 0 of warps 0-4 at once
+    // dout, Qt, Kh, Wm, gC (buffers of this parity are free): issued by lane 0 of warps 0-4 at once
     auto issue_first = [&](int c) {
         if (lane != 0 || warp > 4) return;
         const unsigned char* img = p.tp + (head * nc + c) * TC_WY_BYTES;
@@ -215,7 +236,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             tma_tile(DO(c), C, 0, &m.dout, b, h, c * C, bar_load);
             break;
         case 1: tc::bulk_load(QQ(c), img + TC_WY_QT, 64 * 128 * 2, bar_load); break;
-        case 2: tc::bulk_load(KT(c), img + TC_WY_KT, 64 * 128 * 2, bar_load); break;
+        case 2: tc::bulk_load(KT(c), img + TC_WY_KH, 64 * 128 * 2, bar_load); break;
         case 3: tc::bulk_load(WW(c), img + TC_WY_WM, 64 * 128 * 2, bar_load); break;
         default: tc::bulk_load(GC(c), img + TC_WY_GC, 512, bar_load); break;
         }
@@ -258,7 +279,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         __syncthreads();
     };
 
-    int unreleased = -1;   // chunk whose dZ image is written but whose flag is not yet set
+    int unreleased = -1;   // chunk whose dS' image is written but whose flag is not yet set
     for (int c = nc - 1; c >= 0; --c) {
         const uint32_t sQQ = tc::smem_u32(QQ(c)), sKT = tc::smem_u32(KT(c)), sDO = tc::smem_u32(DO(c)),
                        sWW = tc::smem_u32(WW(c));
@@ -267,8 +288,9 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         // the other parity's buffers were last read by chunk c + 1, whose MMAs are complete
         if (c > 0) issue_first(c - 1);
 
-        const float* sGC = GC(c);   // Qt, Kt, gC came with the forward's WY image
-        // dZ^T = dS'^T Diag(gC): scale the fp32 gradient in place and keep a bf16 copy
+        const float* sGC = GC(c);   // Qt, Kh, gC came with the forward's WY image
+        // a bf16 copy of dS'^T (the operand of dDelta and the image for the gradient units), then the fp32
+        // gradient scaled in place, dS'^T Diag(gC), the first term of dS^T
         {
             const int j = jrow;
             float v[32];
@@ -277,16 +299,16 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
                 tc::tmem_wait_ld(v);
 #pragma unroll
+                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+#pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
                 tc::tmem_st32(lane_base + TM_S + i0, v);
-#pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
             }
             tc::tmem_wait_st();
         }
         sync_for_mma();
 
-        // dDelta^T = dZ^T Kt^T + dO^T P (commit) ;  dS^T = dZ^T + dO^T Qt (continues below)
+        // dDelta^T = dS'^T Kh^T + dO^T P (commit) ;  dS^T = dS'^T Diag(gC) + dO^T Qt (continues below)
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
@@ -300,9 +322,9 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQQ, C, 0, kk), ID_N2a, 1);
         }
-        // the previous chunk's dZ image stores have drained: publish it while the MMAs run
+        // the previous chunk's dS' image stores have drained: publish it while the MMAs run
         if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
-        // this chunk's dZ^T image for the gradient units (plain stores, published one chunk later)
+        // this chunk's dS'^T image for the gradient units (plain stores, published one chunk later)
         {
             uint4* dst = reinterpret_cast<uint4*>(p.dstates + (head * nc + c) * TC_STATE_BYTES);
             const uint4* src = reinterpret_cast<const uint4*>(STt);
@@ -314,7 +336,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         if (tid == 0 && c > 0) issue_p(c - 1);
         tmem_rows_to_tile<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
-        {   // dDelta^T image for the gradient units (published with the dZ^T image)
+        {   // dDelta^T image for the gradient units (published with the dS'^T image)
             uint4* dst = reinterpret_cast<uint4*>(p.ddeltas + (head * nc + c) * TC_DELTA_BYTES);
             const uint4* src = reinterpret_cast<const uint4*>(DT);
 #pragma unroll
@@ -369,7 +391,7 @@ constexpr uint32_t OFF_DU = 65536;       // [128 x 128]: rows 0..63 dout (later 
                                          // v -> -dU (later staged dlog_alpha): one N = 128 operand
 constexpr uint32_t OFF_WW = 98304;       // w, later b (reloaded)
 constexpr uint32_t OFF_ST = 114688;      // S^T image (chunk start)
-constexpr uint32_t OFF_DS = 147456;      // dZ^T image
+constexpr uint32_t OFF_DS = 147456;      // dS'^T image
 constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64] (forward image), later staged dk
 constexpr uint32_t OFF_DDT = 196608;     // dDelta^T [128 x 64] (reverse-pass image), later staged db
 constexpr uint32_t OFF_PP = 212992;      // prep scratch, then dP^T [64 x 64]; with TT: dw staging, and
@@ -378,17 +400,17 @@ constexpr uint32_t OFF_TT = 221184;      // T, later dA^T   [dP^T | dA^T] as one
 constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_W = 64,                     // dA^T (M=64, 64 columns)
     TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
-    TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,   // G3 = dKt^T (P and A paths), G4 = (Delta dZ^T)^T
+    TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,   // G3 = dKt^T (P and A paths), G4 = (Delta dS'^T)^T = dKh^T
     TM_GV = 448,                   // g[t] = exp(G) per key channel
-    TM_IGV = 128;                  // 1/g[t]
+    TM_HV = 128;                   // h[t] = exp(G_C - G)
 constexpr uint32_t LOAD_TOK = 7 * 64 * 128 * 2 + (uint32_t)TC_DELTA_BYTES;   // 7 token tiles, Delta^T
-constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dZ^T: cp.async)
+constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dS'^T: cp.async)
 }  // namespace cg
 
 // Gradients of chunk c of head `headi`; returns false if a bounded wait gave up. `prefetched`: the S, T
-// and dZ^T images of this unit were requested by the previous unit (S, T on the prefetch barrier).
+// and dS'^T images of this unit were requested by the previous unit (S, T on the prefetch barrier).
 // Lane 0 of warp 9 takes the CTA's next unit from the counter while this one runs and acquires its flag
-// while the G MMAs run; once this unit has finished with the S^T, T and dZ^T tiles, the next unit's
+// while the G MMAs run; once this unit has finished with the S^T, T and dS'^T tiles, the next unit's
 // images are requested into them. The next unit is published in *nxt.
 __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi, int c,
                           Phases& ph, bool prefetched, NextUnit* nxt) {
@@ -408,6 +430,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     uint64_t* bar_mma = bar_load + 1;
     uint64_t* bar_b = bar_load + 3;
     uint64_t* bar_pre = reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48);
+    int* untame_flag = reinterpret_cast<int*>(sm + OFF_BARS + 56);   // set by the prep, read after barriers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T, H = p.H, nc = p.nc;
@@ -450,15 +473,16 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         default: break;
         }
     }
-    if (tid == 0 && !prefetched) {   // dZ^T of this chunk comes from the reverse pass: wait for its flag
+    if (tid == 0) *untame_flag = 0;   // the previous unit's last read of it preceded its final barrier
+    if (tid == 0 && !prefetched) {   // dS'^T of this chunk comes from the reverse pass: wait for its flag
         if (!tc::flag_wait(p.flags + head * nc + c, 1u)) {
             ok = false;
             atomicOr(&g_bwd_error, 8u);
             atomicExch(p.counter + 1, 1u);
         }
     }
-    __syncthreads();   // orders thread 0's acquire before every thread's copy of the dZ^T image
-    {   // the reverse pass's images of this chunk: dZ^T (unless prefetched) and dDelta^T
+    __syncthreads();   // orders thread 0's acquire before every thread's copy of the dS'^T image
+    {   // the reverse pass's images of this chunk: dS'^T (unless prefetched) and dDelta^T
         if (!prefetched) {
             const unsigned char* src = p.dstates + (head * nc + c) * TC_STATE_BYTES;
 #pragma unroll
@@ -498,7 +522,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
     // ---- factors (G kept in TMEM)
-    grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV, lane_base + TM_IGV);   // PP: scratch
+    const PrepOut prep = grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV,
+                                   lane_base + TM_HV, untame_flag);   // PP: scratch
     sync_for_mma();
 
     // ---- dU = T^T dDelta (M=64)
@@ -613,18 +638,18 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mma_commit(bar_mma);
     }
 
-    // rowsum(dZ * S) for key channel i over this quarter's value channels (both images hold row j =
-    // value channel)
+    // rowsum(dS' * S) for key channel i over this quarter's value channels (both images hold row j =
+    // value channel); times gC below
     const int i = tid & 127, qt = tid >> 7;
     float Epart = 0.f;
     {
-        float e2 = 0.f;
+        float e1 = 0.f, e2 = 0.f;
 #pragma unroll 8
         for (int j = 32 * qt; j < 32 * qt + 32; j += 2) {
-            Epart += tc::ld_bf16(DS, tc::tile_off(D, j, i)) * tc::ld_bf16(STt, tc::tile_off(D, j, i));
+            e1 += tc::ld_bf16(DS, tc::tile_off(D, j, i)) * tc::ld_bf16(STt, tc::tile_off(D, j, i));
             e2 += tc::ld_bf16(DS, tc::tile_off(D, j + 1, i)) * tc::ld_bf16(STt, tc::tile_off(D, j + 1, i));
         }
-        Epart += e2;
+        Epart = (e1 + e2) * prep.gC;
     }
     if (warp == 9 && lane == 0) {   // while the G MMAs run: the CTA's next unit, published at the next barrier
         if (*reinterpret_cast<volatile unsigned int*>(p.counter + 1)) next_unit = units;   // a CTA gave up
@@ -640,54 +665,102 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     ok = tc::mbar_wait(bar_b, ph.b) && ok;
     ph.b ^= 1;
 
+    // ---- untame channels: their pair terms are summed exactly below, from alpha and the raw q of the chunk
+    // (fp32 [64 tokens][128 channels] tables over the S^T and dS'^T tiles, which the G MMAs and the rowsum
+    // have finished with; the next unit's images are fetched into them only after pass 1)
+    const bool slow = *reinterpret_cast<volatile int*>(untame_flag) != 0;   // the same on every thread
+    float* atab = reinterpret_cast<float*>(STt);
+    float* qtab = reinterpret_cast<float*>(DS);
+    if (slow) {
+        __syncthreads();   // every thread's rowsum has read S^T and dS'^T
+        for (int x = tid; x < C * D; x += BT) {
+            const int tau = x >> 7, ch = x & 127;
+            float al = 1.f, qq = 0.f;
+            if (tau < L) {
+                const size_t off = tok_off(b, t0 + tau, h, T, H, D) + ch;
+                al = fast_exp(__bfloat162float(p.la_raw[off]));
+                qq = __bfloat162float(p.q_raw[off]);
+            }
+            atab[x] = al;
+            qtab[x] = qq;
+        }
+        __syncthreads();
+    }
+
     // ---- gate chain, thread = (key channel i, token quarter qt: tokens 16 qt .. 16 qt + 15). Pass 1: dq,
-    // dk, db and dG_t; partial sums of Kt*G4 and dG are exchanged between the quarters (in the consumed
-    // dP^T tile). Pass 2: dlog_alpha_t = sum_{tau >= t} dG_tau + E, E = rowsum(dZ*S) + sum_t Kt*G4.
-    // Results go to bf16 row tiles (dq -> DU rows 0..63, dk -> DT, db -> DDT, dlog_alpha -> DU rows
-    // 64..127), stored by TMA.
+    // dk, db and dG_t; partial sums of E and dG are exchanged between the quarters (in the consumed dP^T
+    // tile). Pass 2: dlog_alpha_t = sum_{tau >= t} dG_tau + E. Results go to bf16 row tiles (dq -> DU rows
+    // 0..63, dk -> DT, db -> DDT, dlog_alpha -> DU rows 64..127), stored by TMA.
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chk = (uint32_t)((i & 63) >> 3);
+    const float igC = prep.untame ? 0.f : 1.f / prep.gC;
     float dG[16];
     float dGsum = 0.f;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {   // two halves of 8 tokens (keeps the TMEM read-outs in registers)
         const int tq = 16 * qt + 8 * hh;
-        float g1[8], g2[8], g3[8], g4[8], gv[8], igv[8];
+        float g1[8], g2[8], g3[8], g4[8], gv[8], hv[8];
         tc::tmem_ld8(lane_base + TM_G1 + tq, g1);
         tc::tmem_ld8(lane_base + TM_G2 + tq, g2);
         tc::tmem_ld8(lane_base + TM_G3 + tq, g3);
         tc::tmem_ld8(lane_base + TM_G4 + tq, g4);
         tc::tmem_ld8(lane_base + TM_GV + tq, gv);
-        tc::tmem_ld8(lane_base + TM_IGV + tq, igv);
-        tc::tmem_wait_ld(g1, g2, g3, g4, gv, igv);
+        tc::tmem_ld8(lane_base + TM_HV + tq, hv);
+        tc::tmem_wait_ld(g1, g2, g3, g4, gv, hv);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const uint32_t t = (uint32_t)(tq + u);
-            const uint32_t sw = t * 128 + ((chk ^ (t & 7)) << 4);
-            const float qv = tc::ld_bf16(QE, col128 + C * 128 + sw);
-            const float et = tc::ld_bf16(QE, col128 + sw);
-            const float kt = tc::ld_bf16(KT, col64 + sw);
+            const int t = tq + u;
+            const uint32_t sw = (uint32_t)t * 128 + ((chk ^ ((uint32_t)t & 7)) << 4);
             const float kk = tc::ld_bf16(KH, col64 + sw);
             const float bb = tc::ld_bf16(WW, col64 + sw);
-            const float g = gv[u], ig = igv[u];
-            const float dKt = g3[u] + g4[u];
-            const float dGt = qv * g1[u] + et * g2[u] - kt * dKt;
+            const float g = gv[u], hh_ = hv[u];
+            float dq, dE, dkK, dGt;
+            if (!prep.untame) {
+                const float qv = tc::ld_bf16(QE, col128 + C * 128 + sw);   // Qt
+                const float et = tc::ld_bf16(QE, col128 + sw);             // Et
+                dq = g * g1[u];
+                dE = g * g2[u];
+                dkK = (g3[u] * igC + g4[u]) * hh_;                         // dKt/g + h dKh
+                dGt = qv * g1[u] + et * g2[u] - kk * dkK;
+            } else {
+                // exact pair terms of channel i at token t, L = exp(G_t - G_s) as a running product:
+                //   fq = sum_{s<=t} dP_ts k_s L,  fe = sum_{s<t} dA_ts k_s L,
+                //   fk = sum_{t2>=t} (dP_{t2,t} q_t2 + dA_{t2,t} e_t2) exp(G_t2 - G_t)
+                float fq = 0.f, fe = 0.f, fk = 0.f, Lr = 1.f;
+                for (int s2 = t; s2 >= 0; --s2) {
+                    if (s2 < t) Lr *= atab[(s2 + 1) * 128 + i];
+                    const float ks = tc::ld_bf16(KH, tc::tile_off(C, s2, i)) * Lr;
+                    fq += tc::ld_bf16(PP, tc::tile_off(C, s2, t)) * ks;
+                    fe += tc::ld_bf16(TT, tc::tile_off(C, s2, t)) * ks;   // dA_tt = 0
+                }
+                Lr = 1.f;
+                for (int t2 = t; t2 < C; ++t2) {
+                    if (t2 > t) Lr *= atab[t2 * 128 + i];
+                    const float e2_ = tc::ld_bf16(WW, tc::tile_off(C, t2, i)) * tc::ld_bf16(KH, tc::tile_off(C, t2, i));
+                    fk += (tc::ld_bf16(PP, tc::tile_off(C, t, t2)) * qtab[t2 * 128 + i] +
+                           tc::ld_bf16(TT, tc::tile_off(C, t, t2)) * e2_) * Lr;
+                }
+                dq = g * g1[u] + fq;
+                dE = g * g2[u] + fe;
+                dkK = fk + hh_ * g4[u];
+                dGt = qtab[t * 128 + i] * dq + bb * kk * dE - kk * dkK;
+            }
             dG[8 * hh + u] = dGt;
             dGsum += dGt;
-            Epart += kt * g4[u];
-            const float dE = g * g2[u];
-            tc::st_bf16(DU, col128 + sw, g * g1[u]);                // dq
-            tc::st_bf16(DT, col64 + sw, dKt * ig + dE * bb);        // dk
-            tc::st_bf16(DDT, col64 + sw, dE * kk);                  // db
+            Epart += kk * hh_ * g4[u];                                     // Kh * dKh
+            tc::st_bf16(DU, col128 + sw, dq);                               // dq
+            tc::st_bf16(DT, col64 + sw, dkK + dE * bb);                     // dk
+            tc::st_bf16(DDT, col64 + sw, dE * kk);                          // db
         }
     }
+    if (slow) __syncthreads();   // every exact sum has read dP^T before it becomes the exchange area
     float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][4 quarters][128]
     xch[(0 * BPARTS + qt) * 128 + i] = Epart;
     xch[(1 * BPARTS + qt) * 128 + i] = dGsum;
-    tc::fence_async_smem();   // every read of S^T and dZ^T (G MMAs, rowsum) precedes the prefetch below, and
+    tc::fence_async_smem();   // every read of S^T and dS'^T (G MMAs, rowsum) precedes the prefetch below, and
                               // dq, dk, db (final after pass 1) are visible to the tensor stores
-    __syncthreads();          // also orders warp 9's acquire before every thread's copy of the next dZ^T
+    __syncthreads();          // also orders warp 9's acquire before every thread's copy of the next dS'^T
     if (tid == 0) {   // dq, dk, db go out while pass 2 runs; rows past the end of the sequence are skipped
         const CUtensorMap* maps[3] = {mdq, mdk, mdb};
         const unsigned char* tiles[3] = {DU, DT, DDT};
@@ -831,6 +904,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
 
     BwdParams p{};
     p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
+    p.q_raw = static_cast<const __nv_bfloat16*>(a.q); p.la_raw = static_cast<const __nv_bfloat16*>(a.la);
     p.dST = a.dST; p.dS0 = a.dS0;
     p.dv = static_cast<__nv_bfloat16*>(a.dv); p.dw = static_cast<__nv_bfloat16*>(a.dw);
     p.states = a.states; p.deltas = a.deltas; p.tp = a.tp; p.dstates = a.dstates; p.ddeltas = a.ddeltas;

@@ -11,11 +11,21 @@
 //   Qt = g*q,  Kh = (gC/g)*k = gC*Kt,  U = w*v
 //   A  = strictly_lower(Et Kt^T),  T = (I + A)^{-1},  Wm = T Et,  Ut = T U
 //   Delta = Ut - Wm S;   O = Qt S + tril(Qt Kt^T) Delta;   S' = Diag(gC) S + Kh^T Delta
-// The kernels apply the last step as S' = Diag(gC) (S + Kt^T Delta) (Kh = gC*Kt), scaling the
-// fp32 accumulator after the contraction, so no Kh tile is formed.
+// The kernels scale the fp32 state by gC, then let the contraction add Kh^T Delta to it; the WY image
+// of a chunk carries Kh (bounded) in place of Kt.
 // Rows past the end of the sequence are zero-filled by TMA: they give zero
 // factors, a flat cumulative decay and an identity block of T, so a ragged
 // last chunk needs no special case except masked stores.
+//
+// Range of the factors. Qt, Et and Kh carry exp(G_t) or exp(G_C - G_t) <= 1 (log_alpha <= 0), but Kt
+// carries exp(-G_t), which overflows once a channel decays by more than ~e^88 inside one chunk. A channel
+// is "tame" in a chunk when the sum of |log_alpha| over the chunk is at most TAME_LOG_DECAY: then every
+// factor stays within e^{+-60} and the products inside the fp32 accumulators stay finite. For the other
+// ("untame") channels Kt is set to zero, so the tensor-core products that pair two tokens of the chunk
+// (A, P in the forward; dQt, dEt, dKt in the backward) leave them out, and their exact contribution,
+// sum over channels of x_t y_s exp(G_t - G_s), is added on CUDA cores with exp(G_t - G_s) formed as the
+// running product of alpha over (s, t] (every factor <= 1). The state updates use Kh, so they need no
+// fix-up. Typical decays (|G| of a few units per chunk) never take the exact path.
 #pragma once
 
 #include <cuda.h>
@@ -32,6 +42,7 @@ namespace chunk {
 constexpr int D = 128;        // d_k = d_v
 constexpr int C = 64;         // chunk length
 constexpr int NT = 256;       // threads per CTA (two warpgroups)
+constexpr float TAME_LOG_DECAY = 60.f;   // largest sum of |log_alpha| over a chunk on the tensor-core products
 // TMEM access: warp w reads lane quarter (w % 4), i.e. lanes 32 (w % 4) .. +31; the two warps of a
 // quarter (w and w + 4) split the columns of each read-out between them (part = w / 4).
 __device__ __forceinline__ int tm_quarter(int warp) { return warp & 3; }

@@ -6,9 +6,13 @@ The degenerate cases are the ones the oracle is pinned on (closed forms and the 
   no erase         b = 0 (gated linear attention)
   no write         w = 0 and S0 = 0: o and S_T are exactly zero
   exact retrieval  b = 1 and q = k (unit norm): o_t = w_t * v_t
-and a strong uniform decay, log_alpha = -1.2 per token, whose in-chunk cumulative decay (down to
-exp(-77) over 64 tokens) pushes the asymmetric factors exp(+G) and exp(-G) of the chunk form close to the
-ends of the fp32 / bf16 exponent range.
+and decays strong enough that the asymmetric factor exp(-G) of the chunk form would overflow (the kernels
+then leave those channels out of the tensor-core pair products and sum their terms exactly):
+  strong_decay     log_alpha = -1.2 per token (exp(-77) over a 64-token chunk)
+  decay_3          log_alpha = -3 per token on every channel (exp(-192) over a chunk)
+  mixed_20         three channels at -20 per token, the rest from the recipe's distribution
+  spike            the recipe's distribution plus one token per chunk at -100 on every channel
+  tame_edge        log_alpha = -0.9 per token (a chunk's decay mass 57.6, just inside the tensor-core range)
 """
 import numpy as np
 import pytest
@@ -20,7 +24,8 @@ from linear_attention_delta_gdn_b200.inputs import make_inputs
 
 pytestmark = pytest.mark.gpu
 
-CASES = ("no_decay", "no_erase", "no_write", "exact_retrieval", "strong_decay")
+CASES = ("no_decay", "no_erase", "no_write", "exact_retrieval", "strong_decay", "decay_3", "mixed_20", "spike",
+         "tame_edge")
 
 
 def _inputs(case):
@@ -37,6 +42,14 @@ def _inputs(case):
         x["q"] = x["k"].clone()
     elif case == "strong_decay":
         x["log_alpha"].fill_(-1.2)
+    elif case == "decay_3":
+        x["log_alpha"].fill_(-3.0)
+    elif case == "mixed_20":
+        x["log_alpha"][..., [5, 77, 100]] = -20.0
+    elif case == "spike":
+        x["log_alpha"][:, 10::64] = -100.0
+    elif case == "tame_edge":
+        x["log_alpha"].fill_(-0.9)
     return x
 
 
