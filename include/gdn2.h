@@ -34,10 +34,14 @@
  *     GDN2_ERR_CUDA, which reports a launch failure or an earlier asynchronous
  *     error of the device (outputs are then undefined).
  *   - Gate values are not range-checked (that would cost a pass over HBM).
- *   - Decay range of the tensor-core path: for every channel, the sum of
- *     log_alpha over each 64-token chunk must stay above about -88. Below that
- *     the chunk factors exp(-sum) overflow float and the outputs become
- *     inf/NaN without an error status. The recurrent kernels have no limit.
+ *   - log_alpha is a log-decay (alpha in (0, 1]); any value <= 0 is handled,
+ *     however strong. On the tensor-core path a channel whose log-decay over
+ *     a 64-token chunk exceeds 60 is left out of that chunk's tensor-core
+ *     products and its terms are summed exactly on CUDA cores instead (same
+ *     results, slower: such chunks cost several times a typical one).
+ *     Positive log_alpha (growth) is accepted as long as the cumulative sum
+ *     inside a chunk stays below about +60; beyond that the tensor-core path
+ *     overflows (the recurrent kernels have no such limit).
  *   - Supported sizes: Dk, Dv in {16, 32, 64, 128}; chunk in {16, 32, 64};
  *     any T >= 0 (a ragged last chunk is allowed); B, H >= 1.
  *     The tensor-core path runs for dt = GDN2_BF16, Dk = Dv = 128, with any
@@ -93,13 +97,15 @@ typedef enum gdn2_op {
  * fills, so one buffer of gdn2_workspace_size(GDN2_OP_BWD, ...) bytes serves a
  * gdn2_fwd(save_states = 1) followed by a gdn2_bwd(states_saved = 1).
  * GDN2_OP_FWD needs a workspace only on the tensor-core path (dt = GDN2_BF16,
- * Dk = Dv = 128, chunk = 64): there the forward keeps, per chunk, the image of
- * the WY step (the T, P and Wm tiles, the scaled query and key tiles and the
- * chunk's decay) and a ready flag that hands it from the CTAs that compute it
- * to the CTAs that walk the chunks of a head.
+ * Dk = Dv = 128): there the forward keeps, per chunk, the image of the WY step
+ * (the T, P and Wm tiles, the scaled query and key tiles, the chunk's decay and
+ * its strongly decaying channels) and a ready flag that hands it from the CTAs
+ * that compute it to the CTAs that walk the chunks of a head.
  * Returns 0 for an invalid or unsupported problem and for a forward that needs
  * no workspace. The workspace must be 256-byte aligned; its contents on entry
- * do not matter.
+ * do not matter. On the tensor-core path it is about 81 KB per 64-token
+ * chunk and head for GDN2_OP_FWD, 129 KB for GDN2_OP_FWD_SAVE and 177 KB for
+ * GDN2_OP_BWD.
  */
 size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk,
                            gdn2_dtype dt);

@@ -4,31 +4,34 @@
 // "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention" (arXiv
 // abstract) names a gate-aware backward that keeps training parallel; the page
 // prints no equations. The adjoint of the chunk form (see chunk_common.cuh), for
-// one chunk with start state S, S' = Diag(gC) S + Kh^T Delta, next-state gradient dS'
-// and output gradient dO:
-//   dDelta = Kh dS' + P^T dO                         (P = tril(Qt Kt^T))
-//   dS     = Diag(gC) dS' + Qt^T dO - Wm^T dDelta    -> gradient of the chunk-start state
+// one chunk with start state S, S' = Diag(gC) S + Kh^T Delta (Kh = gC*Kt), next-state gradient
+// dS' and output gradient dO; dZ = Diag(gC) dS':
+//   dDelta = Kh dS' + P^T dO = Kt dZ + P^T dO        (P = tril(Qt Kt^T))
+//   dS     = dZ + Qt^T dO - Wm^T dDelta              -> gradient of the chunk-start state
 //   dU     = T^T dDelta                              -> dv = dU*w, dw = dU*v
 //   dP     = (dO Delta^T) * incl,  dA = -(dU Delta^T) * strict
 //   dQt    = dO S^T + dP Kt,       dEt = -dU S^T + dA Kt
-//   dKt    = dP^T Qt + dA^T Et,    dKh = Delta dS'^T
+//   dKt    = dP^T Qt + dA^T Et,    dKh = Delta dS'^T  (so Delta dZ^T = gC*dKh)
 // (dA uses T^T dT T^T = dU Delta^T, since dT = dDelta (U - Et S)^T = dDelta Delta^T (I + A)^T.)
-// Gate chain through g = exp(G), h = exp(G_C - G) (G = in-chunk cumsum of log_alpha):
-//   dq = g*dQt;  dE = g*dEt;  dkK = dKt/g + h*dKh;  db = dE*k;  dk = dkK + dE*b
+// Gate chain through g = exp(G) (G = in-chunk cumsum of log_alpha):
+//   dq = g*dQt;  dE = g*dEt;  dkK = dKt/g + (gC/g)*dKh;  db = dE*k;  dk = dkK + dE*b
 //   dG_t = q*dq + e*dE - k*dkK   (e = b*k);  the last position also gets
-//   E = gC * rowsum(dS' * S) + sum_t Kh_t * dKh_t   (the dependence of S' on gC)
+//   E = rowsum(dZ * S) + sum_t Kh_t * dKh_t   (the dependence of S' on gC)
 //   dlog_alpha_t = sum_{tau >= t} dG_tau + E
-// Untame channels (chunk_common.cuh) have Kt = 0 in the tensor-core products; their pair terms of
-// dq, dE and dkK are summed exactly on CUDA cores with exp(G_t - G_s) as a running product of alpha.
+// Chunks without untame channels (chunk_common.cuh) carry dZ (reverse pass image), Kt and 1/g; chunks
+// with untame channels carry dS', Kh and h = gC/g instead (Kt = k/g would overflow), and the pair terms of
+// dq, dE and dkK of their untame channels (left out of the tensor-core products) are summed exactly on
+// CUDA cores with exp(G_t - G_s) as a running product of alpha. The forward's WY image of the chunk
+// records which channels are untame.
 //
 // One launch, two kinds of work, both reading the forward's per-chunk T and P tiles instead of
 // redoing the solve:
 //   reverse pass    one CTA per (batch, head) walks the chunks backwards carrying dS^T in TMEM
-//                   (fp32); per chunk it writes dS'^T as a bf16 image and then sets the chunk's
+//                   (fp32); per chunk it writes dZ^T (dS'^T) as a bf16 image and then sets the chunk's
 //                   ready flag (release);
 //   chunk gradients every other CTA takes (head, chunk) units from a shared counter, in the
 //                   order the reverse pass produces them, waits for the unit's flag (acquire) and
-//                   computes every gradient of the chunk from the saved S, Delta (forward), dS',
+//                   computes every gradient of the chunk from the saved S, Delta (forward), dZ (dS'),
 //                   dDelta (reverse pass), T, P, the inputs and dout. Reverse-pass CTAs join them
 //                   once their head is done.
 // With few heads this is one cooperative launch (all CTAs resident, so every wait ends; each wait is
@@ -70,48 +73,109 @@ __device__ __forceinline__ void tmem_rows_to_tile(uint32_t lane_base_col, unsign
     tc::st_row8(dst, 128, row, (c0 >> 3) + 1, v + 8);
 }
 
+// Exact pair terms of an untame channel i at token t (see the gate chain): with L = exp(G_t - G_s) as a
+// running product of alpha (tables of alpha and of the raw q, fp32 [64 tokens][128 channels]),
+//   fq = sum_{s<=t} dP_ts k_s L,  fe = sum_{s<t} dA_ts k_s L,
+//   fk = sum_{t2>=t} (dP_{t2,t} q_t2 + dA_{t2,t} e_t2) exp(G_t2 - G_t)      (e = b*k)
+// dP^T and dA^T are the bf16 tiles PP and TT (row s, column t); k and b the raw tiles KH and WW.
+struct PairTerms {
+    float fq, fe, fk;
+};
+__device__ __noinline__ PairTerms untame_pair_terms(const unsigned char* KH, const unsigned char* WW,
+                                                    const unsigned char* PP, const unsigned char* TT,
+                                                    const float* atab, const float* qtab, int i, int t) {
+    float fq = 0.f, fe = 0.f, fk = 0.f, L = 1.f;
+    for (int s = t; s >= 0; --s) {
+        if (s < t) L *= atab[(s + 1) * 128 + i];
+        const float ks = tc::ld_bf16(KH, tc::tile_off(C, s, i)) * L;
+        fq += tc::ld_bf16(PP, tc::tile_off(C, s, t)) * ks;
+        fe += tc::ld_bf16(TT, tc::tile_off(C, s, t)) * ks;   // dA_tt = 0
+    }
+    L = 1.f;
+    for (int t2 = t; t2 < C; ++t2) {
+        if (t2 > t) L *= atab[t2 * 128 + i];
+        const float e2 = tc::ld_bf16(WW, tc::tile_off(C, t2, i)) * tc::ld_bf16(KH, tc::tile_off(C, t2, i));
+        fk += (tc::ld_bf16(PP, tc::tile_off(C, t, t2)) * qtab[t2 * 128 + i] + tc::ld_bf16(TT, tc::tile_off(C, t, t2)) * e2) * L;
+    }
+    return PairTerms{fq, fe, fk};
+}
+
+// For a chunk with untame channels, before the gate chain: thread (channel i, token quarter qt) of an
+// untame channel replaces, for its 16 tokens, G1 by dq = g G1 + fq, G2 by dE = g G2 + fe, G3 by fk and g by 1
+// in TMEM, and Qt, Et by the raw q and e = b*k in QE, so that the gate chain's uniform formulas give the
+// exact gradients (see untame_pair_terms). Whole warps (the TMEM accesses are warp-wide).
+__device__ __noinline__ void untame_prepass(uint32_t lane_base, unsigned char* QE, const unsigned char* KH,
+                                            const unsigned char* WW, const unsigned char* PP, const unsigned char* TT,
+                                            const float* atab, const float* qtab, int i, int qt, bool untame,
+                                            uint32_t tm_g1, uint32_t tm_g2, uint32_t tm_g3, uint32_t tm_gv) {
+    const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
+    const uint32_t chk = (uint32_t)((i & 63) >> 3);
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+        const int tq = 16 * qt + 8 * hh;
+        float g1[8], g2[8], g3[8], gv[8];
+        tc::tmem_ld8(lane_base + tm_g1 + tq, g1);
+        tc::tmem_ld8(lane_base + tm_g2 + tq, g2);
+        tc::tmem_ld8(lane_base + tm_g3 + tq, g3);
+        tc::tmem_ld8(lane_base + tm_gv + tq, gv);
+        tc::tmem_wait_ld(g1, g2, g3, gv);
+        if (untame) {
+#pragma unroll 1
+            for (int u = 0; u < 8; ++u) {
+                const int t = tq + u;
+                const PairTerms f = untame_pair_terms(KH, WW, PP, TT, atab, qtab, i, t);
+                g1[u] = gv[u] * g1[u] + f.fq;
+                g2[u] = gv[u] * g2[u] + f.fe;
+                g3[u] = f.fk;
+                gv[u] = 1.f;
+                const uint32_t sw = (uint32_t)t * 128 + ((chk ^ ((uint32_t)t & 7)) << 4);
+                tc::st_bf16(QE, col128 + C * 128 + sw, qtab[t * 128 + i]);                          // q
+                tc::st_bf16(QE, col128 + sw, tc::ld_bf16(WW, tc::tile_off(C, t, i)) *
+                                                 tc::ld_bf16(KH, tc::tile_off(C, t, i)));           // e = b*k
+            }
+        }
+        tc::tmem_st8(lane_base + tm_g1 + tq, g1);
+        tc::tmem_st8(lane_base + tm_g2 + tq, g2);
+        tc::tmem_st8(lane_base + tm_g3 + tq, g3);
+        tc::tmem_st8(lane_base + tm_gv + tq, gv);
+    }
+    tc::tmem_wait_st();
+}
+
 // Gradient-unit prep, thread = (key channel i = tid % 128, token quarter qt = tid / 128: tokens
 // 16 qt .. 16 qt + 15):
 //   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127)
-//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT (zero on untame channels; k stays in KH);
-//   g[t][i] = exp(G) and h[t][i] = exp(G_C - G) go to TMEM at tmem_g and tmem_h (lane i, column t) for the
-//   gate chain. Quarter sums of log_alpha and of |log_alpha| are exchanged through qsum (fp32 [2][4][128]).
-//   Sets *any_untame when channel i is untame. Contains one __syncthreads.
-struct PrepOut {
-    float gC;       // exp(G_C) of channel i
-    bool untame;    // channel i is left out of the tensor-core pair products
-};
-__device__ __forceinline__ PrepOut grad_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
-                                             float* qsum, int tid, uint32_t tmem_g, uint32_t tmem_h,
-                                             int* any_untame) {
+//   writes Et -> QE rows 0..63, Qt -> QE rows 64..127, Kt -> KT (zero when channel i is untame; k stays in
+//   KH); g[t][i] = exp(G) and r[t][i] go to TMEM at tmem_g and tmem_r (lane i, column t) for the gate chain,
+//   r = 1/g, or h = exp(G_C - G) when the chunk has untame channels (khm). Quarter sums of log_alpha are
+//   exchanged through qsum (fp32 [4][128]). Returns gC = exp(G_C) of channel i. Contains one __syncthreads.
+__device__ __forceinline__ float grad_prep(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
+                                           float* qsum, int tid, uint32_t tmem_g, uint32_t tmem_r, bool untame,
+                                           bool khm) {
     const int i = tid & 127, qt = tid >> 7;
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chunk = (uint32_t)((i & 63) >> 3);
     float la[16];
-    float s0 = 0.f, s1 = 0.f, m = 0.f;
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
         const uint32_t t = (uint32_t)(16 * qt + u);
         la[u] = tc::ld_bf16(KT, col64 + t * 128 + ((chunk ^ (t & 7)) << 4));
         if (u & 1) s1 += la[u]; else s0 += la[u];
-        m += fabsf(la[u]);
     }
     qsum[qt * 128 + i] = s0 + s1;
-    qsum[512 + qt * 128 + i] = m;
     __syncthreads();   // also: every log_alpha is read before Kt overwrites it
-    float G = 0.f, tot = 0.f, mass = 0.f;
+    float G = 0.f, tot = 0.f;
 #pragma unroll
     for (int q = 0; q < BPARTS; ++q) {
         const float x = qsum[q * 128 + i];
         tot += x;
         if (q < qt) G += x;
-        mass += qsum[512 + q * 128 + i];
     }
-    const bool untame = mass > TAME_LOG_DECAY;
-    if (untame && qt == 0) *reinterpret_cast<volatile int*>(any_untame) = 1;
-    const float gC = fast_exp(tot), igC = 1.f / gC;
-    float gvals[16], hvals[16];
+    const float shift = khm ? tot : 0.f;   // r = exp(shift - G)
+    const float igC = khm ? 1.f / fast_exp(tot) : 1.f;   // 1/g = r * igC (used on tame channels only)
+    float gvals[16], rvals[16];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         float kk[8], bb[8], qq[8];
@@ -129,18 +193,18 @@ __device__ __forceinline__ PrepOut grad_prep(unsigned char* QE, const unsigned c
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             G += la[8 * half + u];
-            const float g = fast_exp(G), h = fast_exp(tot - G);
+            const float g = fast_exp(G), r = fast_exp(shift - G), ig = r * igC;
             gvals[8 * half + u] = g;
-            hvals[8 * half + u] = h;
+            rvals[8 * half + u] = r;
             tc::st_bf16(QE, o128[u], g * bb[u] * kk[u]);                  // Et
             tc::st_bf16(QE, o128[u] + C * 128, g * qq[u]);                // Qt
-            tc::st_bf16(KT, o64[u], untame ? 0.f : kk[u] * h * igC);      // Kt = k/g
+            tc::st_bf16(KT, o64[u], untame ? 0.f : kk[u] * ig);           // Kt = k/g
         }
     }
     tc::tmem_st16(tmem_g + 16 * qt, gvals);
-    tc::tmem_st16(tmem_h + 16 * qt, hvals);
+    tc::tmem_st16(tmem_r + 16 * qt, rvals);
     tc::tmem_wait_st();
-    return PrepOut{gC, untame};
+    return fast_exp(tot);
 }
 
 constexpr uint32_t TILE_C = 64 * 64 * 2;   // bytes of a 64 x 64 bf16 tile
@@ -181,27 +245,48 @@ struct NextUnit {
     int unit, prefetched;
 };
 
+// Kh of a chunk with untame channels, in place of its Kt tile (bf16 [64 x 128] row tile): Kt * gC on the
+// tame columns, and on the untame ones (bits of msk) the values that the forward wrote to the image's Kh tile
+// (kh_img, global memory). BT threads, 2 pieces of 8 columns each.
+__device__ __noinline__ void kh_from_kt(unsigned char* KT, const unsigned char* kh_img, const float* gC, uint4 msk,
+                                        int tid) {
+    const unsigned int mw[4] = {msk.x, msk.y, msk.z, msk.w};
+#pragma unroll 1
+    for (int e = 0; e < 2; ++e) {
+        const int idx = tid + BT * e, row = idx >> 4, g = idx & 15;
+        float x[8];
+        tc::ld_row8(KT, C, row, g, x);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int col = 8 * g + c;
+            x[c] = ((mw[col >> 5] >> (col & 31)) & 1u) ? tc::ld_bf16(kh_img, tc::tile_off(C, row, col)) : x[c] * gC[col];
+        }
+        tc::st_row8(KT, C, row, g, x);
+    }
+}
+
 // ====================================================================== reverse state pass
 
 namespace rs {
-// Qt, Kh, dout, Wm and gC alternate between two buffers by chunk parity, so the next chunk's tiles
-// can land while this chunk's MMAs read the current ones; P has one buffer. Qt, Kh, Wm, P and gC come
-// from the forward's WY image.
+// Qt, Kt, dout, Wm, gC and the mask alternate between two buffers by chunk parity, so the next chunk's
+// tiles can land while this chunk's MMAs read the current ones; P has one buffer. Qt, Kt (Kh), Wm, P, gC
+// and the mask come from the forward's WY image.
 constexpr uint32_t OFF_QQ = 0;           // 2 x Qt (64 rows), at +0 / +16384
-constexpr uint32_t OFF_KT0 = 49152;      // Kh (even chunks)
+constexpr uint32_t OFF_KT0 = 49152;      // Kt or Kh (even chunks)
 constexpr uint32_t OFF_DO0 = 65536;      // dout (even chunks)
 constexpr uint32_t OFF_WW0 = 81920;      // Wm (even chunks)
-constexpr uint32_t OFF_ST = 98304;       // dS'^T (bf16)
+constexpr uint32_t OFF_ST = 98304;       // dZ^T or dS'^T (bf16)
 constexpr uint32_t OFF_DT = 131072;      // dDelta^T (bf16)
 constexpr uint32_t OFF_PP = 147456;      // P
 constexpr uint32_t OFF_DO1 = 163840;     // dout (odd chunks)
 constexpr uint32_t OFF_WW1 = 180224;     // Wm (odd chunks)
-constexpr uint32_t OFF_KT1 = 196608;     // Kh (odd chunks)
+constexpr uint32_t OFF_KT1 = 196608;     // Kt or Kh (odd chunks)
 constexpr uint32_t OFF_GC = 212992;      // 2 x fp32 gC[128] (by parity)
+constexpr uint32_t OFF_MASK = 214016;    // 2 x untame-channel mask (4 words, by parity)
 constexpr uint32_t TM_S = 0, TM_D = 128;
-constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 512;   // Qt, Kh, dout, Wm, P, gC
+constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 512 + 16;   // Qt, Kt, dout, Wm, P, gC, mask
 }  // namespace rs
-static_assert(rs::OFF_GC + 1024 <= OFF_BARS, "reverse-pass layout lies below the barrier block");
+static_assert(rs::OFF_MASK + 32 <= OFF_BARS, "reverse-pass layout lies below the barrier block");
 
 __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi,
                             Phases& ph) {
@@ -217,6 +302,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     auto DO = [&](int c) { return sm + ((c & 1) ? OFF_DO1 : OFF_DO0); };
     auto WW = [&](int c) { return sm + ((c & 1) ? OFF_WW1 : OFF_WW0); };
     auto GC = [&](int c) { return reinterpret_cast<float*>(sm + OFF_GC + (c & 1) * 512); };
+    auto MASK = [&](int c) { return sm + OFF_MASK + (c & 1) * 16; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = headi % p.H, b = headi / p.H;
@@ -226,9 +312,9 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 32 * tm_part(warp);      // lane row, column quarter
 
     // chunk c's tiles arrive on one barrier phase, issued in three groups as their buffers free up
-    // dout, Qt, Kh, Wm, gC (buffers of this parity are free): issued by lane 0 of warps 0-4 at once
+    // dout, Qt, Kt, Wm, gC, mask (buffers of this parity are free): issued by lane 0 of warps 0-5 at once
     auto issue_first = [&](int c) {
-        if (lane != 0 || warp > 4) return;
+        if (lane != 0 || warp > 5) return;
         const unsigned char* img = p.tp + (head * nc + c) * TC_WY_BYTES;
         switch (warp) {
         case 0:
@@ -236,9 +322,10 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             tma_tile(DO(c), C, 0, &m.dout, b, h, c * C, bar_load);
             break;
         case 1: tc::bulk_load(QQ(c), img + TC_WY_QT, 64 * 128 * 2, bar_load); break;
-        case 2: tc::bulk_load(KT(c), img + TC_WY_KH, 64 * 128 * 2, bar_load); break;
+        case 2: tc::bulk_load(KT(c), img + TC_WY_KT, 64 * 128 * 2, bar_load); break;
         case 3: tc::bulk_load(WW(c), img + TC_WY_WM, 64 * 128 * 2, bar_load); break;
-        default: tc::bulk_load(GC(c), img + TC_WY_GC, 512, bar_load); break;
+        case 4: tc::bulk_load(GC(c), img + TC_WY_GC, 512, bar_load); break;
+        default: tc::bulk_load(MASK(c), img + TC_WY_MASK, 16, bar_load); break;
         }
     };
     auto issue_p = [&](int c) {   // after the MMAs that read P
@@ -288,9 +375,14 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         // the other parity's buffers were last read by chunk c + 1, whose MMAs are complete
         if (c > 0) issue_first(c - 1);
 
-        const float* sGC = GC(c);   // Qt, Kh, gC came with the forward's WY image
-        // a bf16 copy of dS'^T (the operand of dDelta and the image for the gradient units), then the fp32
-        // gradient scaled in place, dS'^T Diag(gC), the first term of dS^T
+        const float* sGC = GC(c);   // Qt, Kt, gC and the mask came with the forward's WY image
+        const uint4 msk = *reinterpret_cast<const uint4*>(MASK(c));
+        const bool khm = (msk.x | msk.y | msk.z | msk.w) != 0u;   // the same on every thread
+        if (khm)   // untame channels in this chunk: Kh replaces Kt, dS' replaces dZ
+            kh_from_kt(KT(c), p.tp + (head * nc + c) * TC_WY_BYTES + TC_WY_KH, sGC, msk, tid);
+        // the fp32 gradient scaled in place, dZ^T = dS'^T Diag(gC) (the first term of dS^T), and a bf16 copy of
+        // dZ^T, or of dS'^T (taken before the scaling) in a chunk with untame channels: the operand of dDelta
+        // and the image for the gradient units
         {
             const int j = jrow;
             float v[32];
@@ -298,17 +390,23 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             for (int i0 = cpart; i0 < cpart + 32; i0 += 32) {
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
                 tc::tmem_wait_ld(v);
+                if (khm) {
 #pragma unroll
-                for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+                    for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+                }
 #pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
                 tc::tmem_st32(lane_base + TM_S + i0, v);
+                if (!khm) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
+                }
             }
             tc::tmem_wait_st();
         }
         sync_for_mma();
 
-        // dDelta^T = dS'^T Kh^T + dO^T P (commit) ;  dS^T = dS'^T Diag(gC) + dO^T Qt (continues below)
+        // dDelta^T = dZ^T Kt^T (= dS'^T Kh^T) + dO^T P (commit) ;  dS^T = dZ^T + dO^T Qt (continues below)
         if (tid == 0) {
             tc::tc_fence_after();
 #pragma unroll
@@ -322,9 +420,9 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQQ, C, 0, kk), ID_N2a, 1);
         }
-        // the previous chunk's dS' image stores have drained: publish it while the MMAs run
+        // the previous chunk's dZ image stores have drained: publish it while the MMAs run
         if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
-        // this chunk's dS'^T image for the gradient units (plain stores, published one chunk later)
+        // this chunk's dZ^T (dS'^T) image for the gradient units (plain stores, published one chunk later)
         {
             uint4* dst = reinterpret_cast<uint4*>(p.dstates + (head * nc + c) * TC_STATE_BYTES);
             const uint4* src = reinterpret_cast<const uint4*>(STt);
@@ -336,7 +434,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         if (tid == 0 && c > 0) issue_p(c - 1);
         tmem_rows_to_tile<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
-        {   // dDelta^T image for the gradient units (published with the dS'^T image)
+        {   // dDelta^T image for the gradient units (published with the dZ^T image)
             uint4* dst = reinterpret_cast<uint4*>(p.ddeltas + (head * nc + c) * TC_DELTA_BYTES);
             const uint4* src = reinterpret_cast<const uint4*>(DT);
 #pragma unroll
@@ -402,7 +500,7 @@ constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_DU = 320,                   // dU (M=64, 128 columns), later G1 = dQt^T, G2 = dEt^T
     TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,   // G3 = dKt^T (P and A paths), G4 = (Delta dS'^T)^T = dKh^T
     TM_GV = 448,                   // g[t] = exp(G) per key channel
-    TM_HV = 128;                   // h[t] = exp(G_C - G)
+    TM_HV = 128;                   // r[t] = 1/g, or exp(G_C - G) in a chunk with untame channels
 constexpr uint32_t LOAD_TOK = 7 * 64 * 128 * 2 + (uint32_t)TC_DELTA_BYTES;   // 7 token tiles, Delta^T
 constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dS'^T: cp.async)
 }  // namespace cg
@@ -430,7 +528,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     uint64_t* bar_mma = bar_load + 1;
     uint64_t* bar_b = bar_load + 3;
     uint64_t* bar_pre = reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48);
-    int* untame_flag = reinterpret_cast<int*>(sm + OFF_BARS + 56);   // set by the prep, read after barriers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T, H = p.H, nc = p.nc;
@@ -442,6 +539,9 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const CUtensorMap *mq = &m.q, *mk = &m.k, *mv = &m.v, *mla = &m.la, *mb = &m.b, *mw = &m.w, *mdo = &m.dout;
     const CUtensorMap *mdq = &m.dq, *mdk = &m.dk, *mdb = &m.db, *mdla = &m.dla;
 
+    // the chunk's untame channels, as recorded by the forward (a chunk with any takes the Kh / dS' form); loaded
+    // first, used after the tile loads
+    const uint4 msk = *reinterpret_cast<const uint4*>(p.tp + (head * nc + c) * TC_WY_BYTES + TC_WY_MASK);
     bool ok = true;
     int next_unit = units;    // lane 0 of warp 9: the CTA's next unit (its atomic returns while this unit runs)
     // The loads are issued by lane 0 of several warps at once (a TMA issue takes ~100 cycles); the
@@ -473,7 +573,6 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         default: break;
         }
     }
-    if (tid == 0) *untame_flag = 0;   // the previous unit's last read of it preceded its final barrier
     if (tid == 0 && !prefetched) {   // dS'^T of this chunk comes from the reverse pass: wait for its flag
         if (!tc::flag_wait(p.flags + head * nc + c, 1u)) {
             ok = false;
@@ -522,8 +621,11 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
                    sTT = tc::smem_u32(TT), sPP = tc::smem_u32(PP);
 
     // ---- factors (G kept in TMEM)
-    const PrepOut prep = grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV,
-                                   lane_base + TM_HV, untame_flag);   // PP: scratch
+    const bool khm = (msk.x | msk.y | msk.z | msk.w) != 0u;   // the same on every thread
+    const int ich = tid & 127;
+    const bool untame = ((ich < 64 ? (ich < 32 ? msk.x : msk.y) : (ich < 96 ? msk.z : msk.w)) >> (ich & 31)) & 1u;
+    const float gC = grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV, lane_base + TM_HV,
+                               untame, khm);   // PP: scratch
     sync_for_mma();
 
     // ---- dU = T^T dDelta (M=64)
@@ -638,8 +740,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::mma_commit(bar_mma);
     }
 
-    // rowsum(dS' * S) for key channel i over this quarter's value channels (both images hold row j =
-    // value channel); times gC below
+    // rowsum(dZ * S) (or gC rowsum(dS' * S)) for key channel i over this quarter's value channels (both images
+    // hold row j = value channel)
     const int i = tid & 127, qt = tid >> 7;
     float Epart = 0.f;
     {
@@ -649,7 +751,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             e1 += tc::ld_bf16(DS, tc::tile_off(D, j, i)) * tc::ld_bf16(STt, tc::tile_off(D, j, i));
             e2 += tc::ld_bf16(DS, tc::tile_off(D, j + 1, i)) * tc::ld_bf16(STt, tc::tile_off(D, j + 1, i));
         }
-        Epart = (e1 + e2) * prep.gC;
+        Epart = (e1 + e2) * (khm ? gC : 1.f);
     }
     if (warp == 9 && lane == 0) {   // while the G MMAs run: the CTA's next unit, published at the next barrier
         if (*reinterpret_cast<volatile unsigned int*>(p.counter + 1)) next_unit = units;   // a CTA gave up
@@ -668,7 +770,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     // ---- untame channels: their pair terms are summed exactly below, from alpha and the raw q of the chunk
     // (fp32 [64 tokens][128 channels] tables over the S^T and dS'^T tiles, which the G MMAs and the rowsum
     // have finished with; the next unit's images are fetched into them only after pass 1)
-    const bool slow = *reinterpret_cast<volatile int*>(untame_flag) != 0;   // the same on every thread
+    const bool slow = khm;
     float* atab = reinterpret_cast<float*>(STt);
     float* qtab = reinterpret_cast<float*>(DS);
     if (slow) {
@@ -685,6 +787,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             qtab[x] = qq;
         }
         __syncthreads();
+        untame_prepass(lane_base, QE, KH, WW, PP, TT, atab, qtab, i, qt, untame, TM_G1, TM_G2, TM_G3, TM_GV);
+        __syncthreads();   // every exact sum has read dP^T (PP) before the gate chain's exchange reuses it
     }
 
     // ---- gate chain, thread = (key channel i, token quarter qt: tokens 16 qt .. 16 qt + 15). Pass 1: dq,
@@ -694,7 +798,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const uint32_t col64 = (uint32_t)((i >> 6) * 64 * 128 + ((i & 7) << 1));
     const uint32_t col128 = (uint32_t)((i >> 6) * 128 * 128 + ((i & 7) << 1));
     const uint32_t chk = (uint32_t)((i & 63) >> 3);
-    const float igC = prep.untame ? 0.f : 1.f / prep.gC;
+    // tame channels: dkK = (G3 a + G4) r with r = 1/g, a = 1 (G4 = Delta dZ^T), or r = gC/g, a = 1/gC (G4 = dKh)
+    const float a_ = khm ? (untame ? 0.f : 1.f / gC) : 1.f;
     float dG[16];
     float dGsum = 0.f;
 #pragma unroll
@@ -714,47 +819,20 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             const uint32_t sw = (uint32_t)t * 128 + ((chk ^ ((uint32_t)t & 7)) << 4);
             const float kk = tc::ld_bf16(KH, col64 + sw);
             const float bb = tc::ld_bf16(WW, col64 + sw);
-            const float g = gv[u], hh_ = hv[u];
-            float dq, dE, dkK, dGt;
-            if (!prep.untame) {
-                const float qv = tc::ld_bf16(QE, col128 + C * 128 + sw);   // Qt
-                const float et = tc::ld_bf16(QE, col128 + sw);             // Et
-                dq = g * g1[u];
-                dE = g * g2[u];
-                dkK = (g3[u] * igC + g4[u]) * hh_;                         // dKt/g + h dKh
-                dGt = qv * g1[u] + et * g2[u] - kk * dkK;
-            } else {
-                // exact pair terms of channel i at token t, L = exp(G_t - G_s) as a running product:
-                //   fq = sum_{s<=t} dP_ts k_s L,  fe = sum_{s<t} dA_ts k_s L,
-                //   fk = sum_{t2>=t} (dP_{t2,t} q_t2 + dA_{t2,t} e_t2) exp(G_t2 - G_t)
-                float fq = 0.f, fe = 0.f, fk = 0.f, Lr = 1.f;
-                for (int s2 = t; s2 >= 0; --s2) {
-                    if (s2 < t) Lr *= atab[(s2 + 1) * 128 + i];
-                    const float ks = tc::ld_bf16(KH, tc::tile_off(C, s2, i)) * Lr;
-                    fq += tc::ld_bf16(PP, tc::tile_off(C, s2, t)) * ks;
-                    fe += tc::ld_bf16(TT, tc::tile_off(C, s2, t)) * ks;   // dA_tt = 0
-                }
-                Lr = 1.f;
-                for (int t2 = t; t2 < C; ++t2) {
-                    if (t2 > t) Lr *= atab[t2 * 128 + i];
-                    const float e2_ = tc::ld_bf16(WW, tc::tile_off(C, t2, i)) * tc::ld_bf16(KH, tc::tile_off(C, t2, i));
-                    fk += (tc::ld_bf16(PP, tc::tile_off(C, t, t2)) * qtab[t2 * 128 + i] +
-                           tc::ld_bf16(TT, tc::tile_off(C, t, t2)) * e2_) * Lr;
-                }
-                dq = g * g1[u] + fq;
-                dE = g * g2[u] + fe;
-                dkK = fk + hh_ * g4[u];
-                dGt = qtab[t * 128 + i] * dq + bb * kk * dE - kk * dkK;
-            }
+            const float g = gv[u], r = hv[u];
+            const float qv = tc::ld_bf16(QE, col128 + C * 128 + sw);   // Qt (raw q on an untame channel)
+            const float et = tc::ld_bf16(QE, col128 + sw);             // Et (raw e on an untame channel)
+            const float dq = g * g1[u], dE = g * g2[u];
+            const float dkK = g3[u] * (untame ? 1.f : r * a_) + g4[u] * r;   // dKt/g + (gC/g) dKh
+            const float dGt = qv * g1[u] + et * g2[u] - kk * dkK;
             dG[8 * hh + u] = dGt;
             dGsum += dGt;
-            Epart += kk * hh_ * g4[u];                                     // Kh * dKh
+            Epart += kk * r * g4[u];                                        // Kh dKh (= Kt Delta dZ^T)
             tc::st_bf16(DU, col128 + sw, dq);                               // dq
             tc::st_bf16(DT, col64 + sw, dkK + dE * bb);                     // dk
             tc::st_bf16(DDT, col64 + sw, dE * kk);                          // db
         }
     }
-    if (slow) __syncthreads();   // every exact sum has read dP^T before it becomes the exchange area
     float* xch = reinterpret_cast<float*>(PP);                      // [2 quantities][4 quarters][128]
     xch[(0 * BPARTS + qt) * 128 + i] = Epart;
     xch[(1 * BPARTS + qt) * 128 + i] = dGsum;

@@ -4,19 +4,20 @@
 // Chunk algebra ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
 // Attention", arXiv abstract: chunkwise WY algorithm, decay absorbed into
 // asymmetric erase factors), per head and chunk of 64 tokens starting from S:
-//   prep     Et = g*b*k, Qt = g*q, Kt = k/g, Kh = gC*Kt, U = w*v  (g = exp(cumsum log_alpha))
+//   prep     Et = g*b*k, Qt = g*q, Kt = k/g, U = w*v          (g = exp(cumsum log_alpha))
 //   WY       [A; P] = [Et; Qt] Kt^T,  T = (I + strict_lower(A))^{-1},  Wm = T Et
-//   state    Delta^T = U^T T^T - S^T Wm^T,  O = Qt S + P Delta,  S'^T = S^T Diag(gC) + Delta^T Kh
-// (channels whose decay inside the chunk is too strong for the factor Kt = k/g are left out of
-// [A; P] = [Et; Qt] Kt^T and added exactly on CUDA cores; see chunk_common.cuh).
+//   state    Delta^T = U^T T^T - S^T Wm^T,  O = Qt S + P Delta,  S'^T = (S^T + Delta^T Kt) Diag(gC)
+// Chunks with untame channels (see chunk_common.cuh) leave those channels out of [A; P] = [Et; Qt] Kt^T,
+// add their terms exactly on CUDA cores, and update the state as S'^T = S^T Diag(gC) + Delta^T Kh with
+// Kh = k*exp(G_C - G) (an extra tile of their WY image), since Kt itself would overflow.
 // The WY step does not depend on S; the state step is a chain over the chunks of a head.
 //
 // One launch, two kinds of CTA (256 threads each, one CTA per SM):
 //   * producers run two independent WY pipelines each (one warpgroup per pipeline, its own named
 //     barrier, mbarriers and TMEM columns), over the chunks of all heads in chunk-major order; a
-//     pipeline writes T, P, Wm, Qt, Kh and gC of its chunk ("WY image", 65 KB) to the workspace
-//     (bulk stores, Kh by plain stores from the prep) and sets the chunk's ready flag (release) once
-//     they have completed;
+//     pipeline writes T, P, Wm, Qt, Kt, gC and the untame-channel mask of its chunk ("WY image", 65 KB,
+//     plus Kh for chunks with untame channels) to the workspace and sets the chunk's ready flag (release)
+//     once those stores have completed;
 //   * consumers (one per head, or several heads each when heads outnumber them) walk their head's
 //     chunks in order: they wait for the chunk's flag (acquire), copy its WY image into shared
 //     memory and run the state step. The state S^T lives in TMEM (lane j = value channel, column
@@ -42,7 +43,7 @@ using namespace chunk;
 // ---- consumer (state pass) shared memory, bytes from a 1024-aligned base
 namespace sp {
 constexpr uint32_t QQ = 0;          // 2 x [64 x 128] Qt from the WY image (by chunk parity)
-constexpr uint32_t KT = 32768;      // 2 x [64 x 128] Kh from the WY image (by chunk parity)
+constexpr uint32_t KT = 32768;      // 2 x [64 x 128] Kt (Kh for chunks with untame channels) from the WY image
 constexpr uint32_t UU = 65536;      // [64 x 128] v -> U (even chunks)
 constexpr uint32_t WW = 81920;      // [64 x 128] w (even chunks)
 constexpr uint32_t WY = 98304;      // WY image head: T [64 x 64] | P [64 x 64] | Wm [64 x 128]
@@ -51,6 +52,7 @@ constexpr uint32_t ST = 131072;     // [128 x 128] S^T (bf16)
 constexpr uint32_t DT = 163840;     // [128 x 64] Delta^T (bf16)
 constexpr uint32_t GC = 180224;     // 2 x fp32 gC[128] from the WY image (by chunk parity)
 constexpr uint32_t BAR = 181248;    // 4 mbarriers (load even, mma, load odd, unused), tmem base, abort flag
+constexpr uint32_t MASK = BAR + 64; // 2 x untame-channel mask (4 words) from the WY image (by chunk parity)
 constexpr uint32_t UU1 = 182272;    // [64 x 128] v -> U (odd chunks)
 constexpr uint32_t WW1 = 198656;    // [64 x 128] w (odd chunks)
 constexpr uint32_t END = 215040;
@@ -65,20 +67,21 @@ constexpr uint32_t KT = 49152;      // log_alpha -> Kt
 constexpr uint32_t IMG = 65536;     // T | P (bf16 64 x 64 each), then Wm (bf16 64 x 128): the image's first 48 KB
 constexpr uint32_t TT = IMG, PP = IMG + 8192;
 constexpr uint32_t TF = 81920;      // fp32 T [64 x 64] (sq_idx), then Wm once the solve is done
-constexpr uint32_t SX = 98304;      // solve temporaries (4 warps x 16 x XS fp32) | prep scan scratch (fp32 [8][128]
-                                    // cumulative log-decay, then bf16 [8][128] sums of |log_alpha|) | untame list
+constexpr uint32_t SX = 98304;      // solve temporaries (4 warps x 16 x XS fp32) | prep scan scratch (fp32 [8][128])
+                                    // | list of the untame channels (exact path)
 constexpr uint32_t GC = 104448;     // 2 x fp32 gC[128] (by unit parity)
 constexpr uint32_t STAGE = TF;      // exact path for untame channels: fp32 [4][64][16] raw-input stage
 constexpr uint32_t BAR = 2 * PIPE;  // 4 mbarriers (inputs, mma per pipeline), tmem base, abort flag
 constexpr uint32_t UMASK = BAR + 64;  // untame-channel masks: [pipeline][unit parity][4 words]
 }  // namespace wy
 constexpr uint32_t SMEM_BYTES = (sp::END > wy::UMASK + 64 ? sp::END : wy::UMASK + 64) + 1024;
-static_assert(sp::BAR + 64 <= sp::UU1 && sp::UU1 % 1024 == 0 && sp::WW1 % 1024 == 0, "consumer layout");
-static_assert(4 * 16 * XS * 4 <= wy::GC - wy::SX && 8 * 128 * 6 <= wy::GC - wy::SX, "producer scratch fits");
+static_assert(sp::MASK + 32 <= sp::UU1 && sp::UU1 % 1024 == 0 && sp::WW1 % 1024 == 0, "consumer layout");
+static_assert(4 * 16 * XS * 4 <= wy::GC - wy::SX && 8 * 128 * 4 <= wy::GC - wy::SX, "producer scratch fits");
 static_assert(4 * 64 * 16 * 4 == TILE_64x128 && wy::STAGE + 4 * 64 * 16 * 4 <= wy::SX, "untame stage fits");
-static_assert(TC_WY_QT == 32768 && TC_WY_KH == 49152 && TC_WY_GC == 65536, "WY image: T | P | Wm | Qt | Kh | gC");
+static_assert(TC_WY_QT == 32768 && TC_WY_KT == 49152 && TC_WY_GC == 65536 && TC_WY_MASK == 66048 &&
+              TC_WY_KH == 66560, "WY image: T | P | Wm | Qt | Kt | gC | mask | (Kh)");
 static_assert(wy::TF == wy::IMG + TC_WY_WM, "T | P | Wm contiguous in shared memory as in the image");
-// The per-thread copy loops below are written for NT threads: copy_wy moves 8 (T | P | Wm) and 4 (Qt, Kh)
+// The per-thread copy loops below are written for NT threads: copy_wy moves 8 (T | P | Wm) and 4 (Qt, Kt)
 // 16-byte pieces per thread, the U = w*v loop 4 rows of 8 values. The kernel checks blockDim.x == NT.
 static_assert(8 * 16 * NT == TC_WY_QT && 4 * 16 * NT == TILE_64x128 && 4 * NT * 8 == C * D, "NT-thread loops");
 
@@ -121,100 +124,91 @@ __device__ __forceinline__ void sync_for_mma() {   // smem written by threads + 
 
 // Gate prep of one chunk: thread = (8-token block tb = wt / 16, 8-channel group cg = wt % 16);
 //   reads  log_alpha (KT), k (KH), b (QE rows 0..63), q (QE rows 64..127)
-//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127, Kt = k/g -> KT (zero on untame channels),
-//          gC, and Kh = (gC/g)*k with plain 16-byte stores straight into the chunk's WY image (kh_img);
-//   block totals of the cumsum (fp32) and of |log_alpha| (bf16) go through red / red_abs; the untame
-//   channels (sum of |log_alpha| over the chunk above TAME_LOG_DECAY) are OR-ed into umask (bit = channel).
+//   writes Et = g*b*k -> QE rows 0..63, Qt = g*q -> QE rows 64..127, Kt = k/g -> KT, gC;
+//   block totals of the cumsum go through red (fp32 [8][128]). The threads of the last token block, which
+//   hold G_C, OR the untame channels (log-decay over the chunk, -G_C, above TAME_LOG_DECAY) into umask
+//   (bit = channel); their Kt is still written here and cleared afterwards (untame chunks only).
 template <typename Sync>
 __device__ __forceinline__ void gate_prep_wg(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
-                                             float* gC_out, float* red, __nv_bfloat16* red_abs, unsigned int* umask,
-                                             unsigned char* kh_img, int wt, Sync&& wg_sync) {
+                                             float* gC_out, float* red, unsigned int* umask, int wt, Sync&& wg_sync) {
     constexpr int RB = 8;
     const int cg = wt & 15, tb = wt >> 4;
-    float G[RB][8], A[8];
+    float G[RB][8];
 #pragma unroll
     for (int u = 0; u < RB; ++u) {
         tc::ld_row8(KT, C, RB * tb + u, cg, G[u]);
+        if (u > 0) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            A[c] = (u == 0) ? fabsf(G[0][c]) : A[c] + fabsf(G[u][c]);
-            if (u > 0) G[u][c] += G[u - 1][c];
+            for (int c = 0; c < 8; ++c) G[u][c] += G[u - 1][c];
         }
     }
     *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg) = make_float4(G[RB - 1][0], G[RB - 1][1], G[RB - 1][2], G[RB - 1][3]);
     *reinterpret_cast<float4*>(red + tb * 128 + 8 * cg + 4) = make_float4(G[RB - 1][4], G[RB - 1][5], G[RB - 1][6], G[RB - 1][7]);
-    *reinterpret_cast<uint4*>(red_abs + tb * 128 + 8 * cg) =
-        make_uint4(tc::pack_bf16x2(A[0], A[1]), tc::pack_bf16x2(A[2], A[3]), tc::pack_bf16x2(A[4], A[5]),
-                   tc::pack_bf16x2(A[6], A[7]));
     wg_sync();
-    float pre[8], tot[8], mass[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) pre[c] = tot[c] = mass[c] = 0.f;
-#pragma unroll
-    for (int q = 0; q < C / RB; ++q) {
+    float pre[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int q = 0; q < tb; ++q) {
         const float4 x0 = *reinterpret_cast<const float4*>(red + q * 128 + 8 * cg);
         const float4 x1 = *reinterpret_cast<const float4*>(red + q * 128 + 8 * cg + 4);
-        const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        const uint4 ab = *reinterpret_cast<const uint4*>(red_abs + q * 128 + 8 * cg);
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ab);
+        pre[0] += x0.x; pre[1] += x0.y; pre[2] += x0.z; pre[3] += x0.w;
+        pre[4] += x1.x; pre[5] += x1.y; pre[6] += x1.z; pre[7] += x1.w;
+    }
+    if (tb == C / RB - 1) {
+        unsigned int bits = 0;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            tot[c] += x[c];
-            if (q < tb) pre[c] += x[c];
-            const float2 f = __bfloat1622float2(a2[c >> 1]);
-            mass[c] += (c & 1) ? f.y : f.x;
+            const float tot = pre[c] + G[RB - 1][c];
+            gC_out[8 * cg + c] = fast_exp(tot);
+            bits |= (tot < -TAME_LOG_DECAY ? 1u : 0u) << c;
         }
-    }
-    unsigned int bits = 0;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) bits |= (mass[c] > TAME_LOG_DECAY ? 1u : 0u) << c;
-    if (tb == 0 && bits) atomicOr(umask + (cg >> 2), bits << (8 * (cg & 3)));
-    float gCv[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) gCv[c] = fast_exp(tot[c]);
-    if (tb == C / RB - 1) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) gC_out[8 * cg + c] = gCv[c];
+        if (bits) atomicOr(umask + (cg >> 2), bits << (8 * (cg & 3)));
     }
 #pragma unroll
     for (int u = 0; u < RB; ++u) {
         const int row = RB * tb + u;
-        float kk[8], bb[8], qq[8], e[8], kt[8], kh[8];
+        float kk[8], bb[8], qq[8], e[8], kt[8];
         tc::ld_row8(KH, C, row, cg, kk);
         tc::ld_row8(QE, 2 * C, row, cg, bb);
         tc::ld_row8(QE, 2 * C, C + row, cg, qq);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float Gv = pre[c] + G[u][c];
-            const float g = fast_exp(Gv);
+            const float g = fast_exp(Gv), ig = fast_exp(-Gv);
             e[c] = g * bb[c] * kk[c];
+            kt[c] = kk[c] * ig;
             qq[c] *= g;
-            if ((bits >> c) & 1u) {   // untame: left out of the tensor-core products; Kh from its own exponent
-                kt[c] = 0.f;
-                kh[c] = kk[c] * fast_exp(tot[c] - Gv);
-            } else {
-                kt[c] = kk[c] * fast_exp(-Gv);
-                kh[c] = kt[c] * gCv[c];
-            }
         }
         tc::st_row8(QE, 2 * C, row, cg, e);
         tc::st_row8(KT, C, row, cg, kt);
         tc::st_row8(QE, 2 * C, C + row, cg, qq);
-        *reinterpret_cast<uint4*>(kh_img + tc::tile_chunk_off(C, row, cg)) =
-            make_uint4(tc::pack_bf16x2(kh[0], kh[1]), tc::pack_bf16x2(kh[2], kh[3]), tc::pack_bf16x2(kh[4], kh[5]),
-                       tc::pack_bf16x2(kh[6], kh[7]));
     }
+}
+
+// Clears the Kt columns of the untame channels (umask) of the thread's 8 x 8 block (prep mapping), so that the
+// tensor-core pair products leave them out.
+__device__ __noinline__ void clear_untame_kt(unsigned char* KT, const unsigned int* umask, int wt) {
+    const int cg = wt & 15, tb = wt >> 4;
+    const unsigned int bits = (umask[cg >> 2] >> (8 * (cg & 3))) & 0xFFu;
+    if (!bits) return;
+#pragma unroll 1
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if ((bits >> c) & 1u) tc::st_bf16(KT, tc::tile_off(C, 8 * tb + u, 8 * cg + c), 0.f);
 }
 
 // Exact contributions of the untame channels (bits of umask) to A (sA: fp32, strictly lower) and P (PP: bf16,
 // lower with the diagonal): for each such channel i and pair s <= t of the chunk,
 //   A_ts += e_ti k_si L,  P_ts += q_ti k_si L,   L = prod_{s < tau <= t} alpha_tau,i = exp(G_ti - G_si) <= 1,
-// e = b*k. The chunk's raw inputs are read from global memory, 16 channels at a time, into an fp32 stage
-// ([alpha | k | e | q][64 tokens][16]); thread (column s = wt % 64, A or P = wt / 64) keeps its 64 sums in
-// registers and adds them at the end. Called by the whole warpgroup; ends with a barrier.
-template <typename Sync>
-__device__ void untame_fixup_wg(const FwdParams& p, int b, int h, int t0, const unsigned int* umask, float* sA,
-                                unsigned char* PP, float* stage, unsigned char* list, int wt, Sync&& wg_sync) {
+// e = b*k; and their column of the image's Kh tile, Kh_ti = k_ti prod_{tau > t} alpha_tau,i. The chunk's raw
+// inputs are read from global memory, 16 channels at a time, into an fp32 stage ([alpha | k | e | q][64
+// tokens][16]); thread (column s = wt % 64, A or P = wt / 64) keeps its 64 sums in registers and adds them at
+// the end. Called by the whole warpgroup; ends with a barrier.
+__device__ __noinline__ void untame_fixup_wg(int T, int H, const __nv_bfloat16* gq, const __nv_bfloat16* gk,
+                                             const __nv_bfloat16* gla, const __nv_bfloat16* gb, int b, int h, int t0,
+                                             const unsigned int* umask, float* sA, unsigned char* PP, float* stage,
+                                             unsigned char* list, unsigned char* kh_img, int wt, int wg) {
+    auto wg_sync = [&]() { tc::named_sync(1 + wg, 128); };
     const int w = wt >> 5, bit = wt & 31;
     int before = 0;
     for (int i = 0; i < w; ++i) before += __popc(umask[i]);
@@ -222,7 +216,7 @@ __device__ void untame_fixup_wg(const FwdParams& p, int b, int h, int t0, const 
     if ((umask[w] >> bit) & 1u) list[before + __popc(umask[w] & ((1u << bit) - 1u))] = (unsigned char)wt;
     const int s = wt & 63;
     const bool isP = wt >= 64;
-    const int L = min(C, p.T - t0);
+    const int L = min(C, T - t0);
     float* sAl = stage;
     float* sK = stage + 64 * 16;
     float* sE = stage + 2 * 64 * 16;
@@ -240,11 +234,11 @@ __device__ void untame_fixup_wg(const FwdParams& p, int b, int h, int t0, const 
                 const int tau = 8 * tb + u;
                 float al = 1.f, kk = 0.f, ee = 0.f, qq = 0.f;
                 if (ch >= 0 && tau < L) {
-                    const size_t off = tok_off(b, t0 + tau, h, p.T, p.H, D) + ch;
-                    al = fast_exp(__bfloat162float(p.la[off]));
-                    kk = __bfloat162float(p.k[off]);
-                    ee = __bfloat162float(p.b[off]) * kk;
-                    qq = __bfloat162float(p.q[off]);
+                    const size_t off = tok_off(b, t0 + tau, h, T, H, D) + ch;
+                    al = fast_exp(__bfloat162float(gla[off]));
+                    kk = __bfloat162float(gk[off]);
+                    ee = __bfloat162float(gb[off]) * kk;
+                    qq = __bfloat162float(gq[off]);
                 }
                 sAl[tau * 16 + c] = al;
                 sK[tau * 16 + c] = kk;
@@ -253,6 +247,14 @@ __device__ void untame_fixup_wg(const FwdParams& p, int b, int h, int t0, const 
             }
         }
         wg_sync();
+        if (wt < 16 && g0 + wt < nU) {   // Kh of channel list[g0 + wt]: suffix products of alpha
+            const int ch = list[g0 + wt];
+            float suf = 1.f;
+            for (int t = C - 1; t >= 0; --t) {
+                tc::st_bf16(kh_img, tc::tile_off(C, t, ch), sK[t * 16 + wt] * suf);
+                suf *= sAl[t * 16 + wt];
+            }
+        }
         const float* X = isP ? sQ : sE;
         for (int c = 0; c < 16; ++c) {
             const float ks = sK[s * 16 + c];
@@ -416,9 +418,10 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         tc::tc_fence_after();
     };
     const int units = p.BH * p.nc, npipe = 2 * p.nprod;
-    // The WY image of a unit is written by bulk stores of the pipeline's thread 0 in two groups: Qt and gC
-    // right after the prep (Kh is stored by every thread from the prep itself), T | P | Wm at the end of the
-    // unit. The same thread sets the unit's flag at
+    // The WY image of a unit is written by bulk stores of the pipeline's thread 0 in two groups: Qt, Kt and
+    // gC right after the prep (with the untame mask, a plain store; the Kh tile of a chunk with untame
+    // channels comes from the prep's own plain stores), T | P | Wm at the end of the unit. The same thread
+    // sets the unit's flag at
     // the end of the pipeline's next unit, when its stores have long completed (the wait for them and the
     // release fence then cost little). The next unit's tiles are loaded as soon as their
     // buffers are free: q and log_alpha (over Qt, Kt) once M1 and the first group have read them, k (over
@@ -457,15 +460,20 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         unsigned int* umask = reinterpret_cast<unsigned int*>(sm + wy::UMASK) + 8 * wg + 4 * (kunit & 1);
         if (wt < 4) reinterpret_cast<unsigned int*>(sm + wy::UMASK)[8 * wg + 4 * ((kunit + 1) & 1) + wt] = 0u;
         unsigned char* img = p.wyimg + ((size_t)head * p.nc + c) * TC_WY_BYTES;
-        gate_prep_wg(QE, KH, KT, gC, sX, reinterpret_cast<__nv_bfloat16*>(sX + 8 * 128), umask, img + TC_WY_KH, wt,
-                     wg_sync);
+        gate_prep_wg(QE, KH, KT, gC, sX, umask, wt, wg_sync);
         sync_for_mma_wg();
-        const bool untame = (umask[0] | umask[1] | umask[2] | umask[3]) != 0u;   // same answer on every thread
-        if (wt == 0) {   // first image group: Qt, gC (final after the prep)
+        const bool untame = (umask[0] | umask[1] | umask[2] | umask[3]) != 0u;   // the same on every thread
+        if (untame) {   // their Kt columns are cleared before the image's Kt and M1 read KT
+            clear_untame_kt(KT, umask, wt);
+            sync_for_mma_wg();
+        }
+        if (wt == 0) {   // first image group: Qt, Kt, gC (final after the prep), and the untame mask
             tc::bulk_store(img + TC_WY_QT, QE + 8192, 8192u);               // Qt (two 64-row halves of the
             tc::bulk_store(img + TC_WY_QT + 8192, QE + 24576, 8192u);       //  128-row tile, 16 KB apart)
+            tc::bulk_store(img + TC_WY_KT, KT, 16384u);                     // Kt
             tc::bulk_store(img + TC_WY_GC, gC, 512u);                       // gC
             tc::bulk_commit();
+            *reinterpret_cast<uint4*>(img + TC_WY_MASK) = make_uint4(umask[0], umask[1], umask[2], umask[3]);
         }
         if (wt == 0) {   // [A; P] = [Et; Qt] Kt^T
             tc::bulk_wait_read_but1();   // the previous unit's T | P | Wm may be overwritten
@@ -489,8 +497,9 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         if (untame) {   // exact terms of the channels left out of M1 (TF is free until the solve)
             int b, h, t0;
             coords(u, b, h, t0);
-            untame_fixup_wg(p, b, h, t0, umask, sA, PP, reinterpret_cast<float*>(pb + wy::STAGE),
-                            reinterpret_cast<unsigned char*>(sX), wt, wg_sync);
+            untame_fixup_wg(p.T, p.H, p.q, p.k, p.la, p.b, b, h, t0, umask, sA, PP,
+                            reinterpret_cast<float*>(pb + wy::STAGE), reinterpret_cast<unsigned char*>(sX),
+                            img + TC_WY_KH, wt, wg);
         }
         solve_unit_lower_wg(sA, sTf, sX, TT, wq, lane, wg_sync);   // T = (I + A)^{-1}
         sync_for_mma_wg();
@@ -527,6 +536,27 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
 }
 
 // ------------------------------------------------------------------ consumer
+
+// Kh of a chunk with untame channels, in place of its Kt tile (bf16 [64 x 128] row tile): Kt * gC on the
+// tame columns, and on the untame ones (bits of msk) the values that the producer wrote to the image's Kh
+// tile (kh_img, global memory). NT threads, 4 pieces of 8 columns each.
+__device__ __noinline__ void kh_from_kt(unsigned char* KT, const unsigned char* kh_img, const float* gC, uint4 msk,
+                                        int tid) {
+    const unsigned int mw[4] = {msk.x, msk.y, msk.z, msk.w};
+#pragma unroll 1
+    for (int e = 0; e < 4; ++e) {
+        const int idx = tid + NT * e, row = idx >> 4, g = idx & 15;
+        float x[8];
+        tc::ld_row8(KT, C, row, g, x);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int col = 8 * g + c;
+            x[c] = ((mw[col >> 5] >> (col & 31)) & 1u) ? tc::ld_bf16(kh_img, tc::tile_off(C, row, col)) : x[c] * gC[col];
+        }
+        tc::st_row8(KT, C, row, g, x);
+    }
+}
+
 __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int cid) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // v and w tiles by chunk parity: chunk c + 2 is loaded while chunk c + 1's tiles wait in the other pair
@@ -560,7 +590,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     auto wait_wy = [&](size_t head, int c) {
         if (!tc::flag_wait(p.flags + head * nc + c, 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 4u); }
     };
-    // the WY image of (head, c): T | P | Wm to WY, Qt and Kh to this chunk's parity buffers, gC
+    // the WY image of (head, c): T | P | Wm to WY, Qt and Kt to this chunk's parity buffers, gC and the mask
     auto copy_wy = [&](size_t head, int c) {
         const unsigned char* src = p.wyimg + (head * nc + c) * TC_WY_BYTES;
         const int par = c & 1;
@@ -573,9 +603,10 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
         for (int i = 0; i < 4; ++i) {
             const int o = 16 * (tid + NT * i);
             tc::cp_async16_cg(sm + sp::QQ + par * TILE_64x128 + o, src + TC_WY_QT + o);
-            tc::cp_async16_cg(sm + sp::KT + par * TILE_64x128 + o, src + TC_WY_KH + o);
+            tc::cp_async16_cg(sm + sp::KT + par * TILE_64x128 + o, src + TC_WY_KT + o);
         }
         if (tid < 32) tc::cp_async16_cg(sm + sp::GC + par * 512 + 16 * tid, src + TC_WY_GC + 16 * tid);
+        if (tid == 32) tc::cp_async16_cg(sm + sp::MASK + par * 16, src + TC_WY_MASK);
         tc::cp_async_commit();
     };
 
@@ -652,7 +683,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             if (!tc::mbar_wait(bar_ld(c), (ph_load >> par) & 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
             ph_load ^= 1u << par;
 
-            // ---- U = w * v (Qt, Kh and gC come with the WY image): 4 row chunks of 8 values per thread
+            // ---- U = w * v (Qt, Kt and gC come with the WY image): 4 row chunks of 8 values per thread
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int idx = tid + NT * e, row = idx >> 4, g = idx & 15;
@@ -665,6 +696,12 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             }
             tc::cp_async_wait_all();   // this chunk's WY image
             sync_for_mma();
+            // a chunk with untame channels updates the state with Kh on a state scaled by gC first, the others
+            // with Kt and a scaling afterwards
+            const uint4 msk = *reinterpret_cast<const uint4*>(sm + sp::MASK + par * 16);
+            const bool khm = (msk.x | msk.y | msk.z | msk.w) != 0u;   // the same on every thread
+            if (khm) kh_from_kt(sm + sp::KT + par * TILE_64x128, p.wyimg + (head * nc + c) * TC_WY_BYTES + TC_WY_KH,
+                                sGC, msk, tid);   // in the shadow of M3-M5, which do not read it
 
             // ---- M3: Delta^T := U^T T^T ;  M4: Delta^T -= S^T Wm^T  (commit) ;  M5: O = Qt S
             if (tid == 0) {
@@ -684,8 +721,8 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 if (c + 1 < nc) wait_wy(head, c + 1);   // overlaps the MMAs
             }
             if (want_o && c > 0) store_o(c - 1);      // previous chunk's output, in the MMAs' shadow
-            {   // S^T := S^T Diag(gC) on the fp32 state, in the MMAs' shadow (M3-M5 read its bf16 copy); M7 then
-                // adds Delta^T Kh
+            if (khm) {   // S^T := S^T Diag(gC) on the fp32 state, in the MMAs' shadow (M3-M5 read its bf16 copy); M7
+                         // then adds Delta^T Kh
                 float v[32];
 #pragma unroll 1
                 for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
@@ -707,7 +744,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 tc::bulk_commit();
             }
 
-            // ---- M6: O += P Delta ;  M7: S'^T = S^T Diag(gC) + Delta^T Kh
+            // ---- M6: O += P Delta ;  M7: Z^T = S^T + Delta^T Kt  (or S'^T = S^T Diag(gC) + Delta^T Kh)
             if (tid == 0) {
                 tc::tc_fence_after();
 #pragma unroll
@@ -719,8 +756,8 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 tc::mma_commit(bar_mma);
             }
             wait_mma();
-            // bf16 copy of the new state for the next chunk (the bulk stores of the previous state image and of
-            // this chunk's Delta^T must have read their tiles)
+            // S'^T = Z^T Diag(gC) (unless already scaled), and a bf16 copy of the new state for the next chunk
+            // (the bulk stores of the previous state image and of this chunk's Delta^T must have read their tiles)
             if (p.states && tid == 0) tc::bulk_wait_read();
             __syncthreads();   // also orders thread 0's flag acquire before the image copy
             if (c + 1 < nc) copy_wy(head, c + 1);
@@ -731,9 +768,15 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
                     tc::tmem_ld32(lane_base + TM_S + i0, v);
                     tc::tmem_wait_ld(v);
+                    if (!khm) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) v[u] *= sGC[i0 + u];
+                        tc::tmem_st32(lane_base + TM_S + i0, v);
+                    }
 #pragma unroll
                     for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
                 }
+                if (!khm) tc::tmem_wait_st();
             }
             sync_for_mma();
             tc::tc_fence_after();

@@ -31,12 +31,12 @@ constexpr int TC_C = 64;
 // bytes of one saved state image (bf16 128 x 128, 128B-swizzled panels)
 constexpr size_t TC_STATE_BYTES = (size_t)TC_D * TC_D * 2;
 // One WY image per chunk, written by the forward's producers: bf16 row tiles T [64 x 64], P [64 x 64],
-// Wm, Qt, Kh [64 x 128 each] (Kh = k * exp(G_C - G_t), the key scaled to the chunk's end), then gC
-// (fp32 [128]) and padding to a 1 KB multiple.
-constexpr size_t TC_TP_BYTES = (size_t)2 * TC_C * TC_C * 2;
-constexpr size_t TC_WY_T = 0, TC_WY_P = 8192, TC_WY_WM = 16384, TC_WY_QT = 32768, TC_WY_KH = 49152,
-                 TC_WY_GC = 65536;
-constexpr size_t TC_WY_BYTES = 66560;
+// Wm, Qt, Kt [64 x 128 each], then gC (fp32 [128]), the chunk's untame-channel mask (4 x 32 bits, bit =
+// key channel) and padding to a 1 KB multiple, then a Kh = k * exp(G_C - G_t) tile [64 x 128] that is
+// written (and read) only for chunks whose mask is not zero.
+constexpr size_t TC_WY_T = 0, TC_WY_P = 8192, TC_WY_WM = 16384, TC_WY_QT = 32768, TC_WY_KT = 49152,
+                 TC_WY_GC = 65536, TC_WY_MASK = 66048, TC_WY_KH = 66560;
+constexpr size_t TC_WY_BYTES = 82944;
 // bytes of one saved Delta^T (forward) or dDelta^T (backward) image: bf16 128 x 64 row tile
 constexpr size_t TC_DELTA_BYTES = (size_t)TC_D * TC_C * 2;
 

@@ -53,12 +53,12 @@ def test_workspace_sizes(L):
     assert fs >= 1 * 2 * 4 * 64 * 64 * 4 and fs % 256 == 0
     assert ws(2, 1, 256, 2, 64, 64, 64, 0) > fs
     # bf16 shape of the 1.3B training layer: the inference forward keeps a WY image
-    # (T | P | Wm | Qt | Kt | gC, 65 KB) and a ready flag per chunk; training adds the state (32 KB) and
-    # Delta (16 KB) images; the backward adds the dZ (32 KB) and dDelta (16 KB) images, its
-    # ready flags, a work counter and an abort word
+    # (T | P | Wm | Qt | Kt | gC | untame mask, 65 KB, plus a 16 KB Kh tile used by chunks with untame channels)
+    # and a ready flag per chunk; training adds the state (32 KB) and Delta (16 KB) images; the backward adds
+    # the dZ (32 KB) and dDelta (16 KB) images, its ready flags, a work counter and an abort word
     units = 4 * 16 * 64
     i = ws(0, 4, 4096, 16, 128, 128, 64, 1)
-    assert i == units * 66560 + units * 4
+    assert i == units * 82944 + units * 4
     f = ws(1, 4, 4096, 16, 128, 128, 64, 1)
     b = ws(2, 4, 4096, 16, 128, 128, 64, 1)
     assert f == units * (32768 + 16384) + i
