@@ -16,6 +16,8 @@ Besides the headline step, the line carries (rank 0, N=1):
   * ``sweep``: fwd+bwd at a fixed 64K tokens per step for T = 1K..64K
     (B = 64K / T), the same figures per point;
   * ``decode``: 1024 in-place decode steps (batch 256, 16 heads, d = 128);
+  * ``kda_overhead``: the KDA and Gated DeltaNet reductions through the same
+    kernels at the headline shape, against the GDN-2 step;
   * ``cpu_baseline``: the fp64 oracle timed on a bounded sample of the headline
     workload on the host cores, with the GPU outputs of those same sequences
     compared against the oracle's (relative L2, whole sample and worst head).
@@ -345,6 +347,44 @@ def measure_configs(binding, dev, args, fwd_inputs):
     return out
 
 
+def measure_reductions(binding, dev, d, args, gdn2_ms):
+    """The pages' reductions through the same kernels at the headline shape: KDA (b = w = beta * 1) and Gated
+    DeltaNet (also a scalar decay), fwd (keeping the states) + bwd, against the GDN-2 step. Both run the GDN-2
+    kernels on broadcast gates plus a broadcast and a gate-sum kernel; `overhead_of_gdn2` is
+    gdn2_ms / reduced_ms - 1."""
+    import torch
+    names = ("q", "k", "v")
+    B, T, H, D = d["q"].shape
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6000)
+    beta = torch.sigmoid(torch.randn((B, T, H), generator=gen, device=dev)).to(torch.bfloat16)
+    log_a = (-torch.nn.functional.softplus(torch.randn((B, T, H), generator=gen, device=dev)) / 16.0).to(torch.bfloat16)
+    out = {"gdn2_ms": gdn2_ms}
+    for name, gate, la in (("kda", binding.GDN2_GATE_KDA, d["log_alpha"]), ("gated_deltanet", binding.GDN2_GATE_GDN, log_a)):
+        ws = torch.empty(binding.gdn2_beta_workspace_size(gate, binding.GDN2_OP_BWD, B, T, H, D, D, 64,
+                                                          binding.GDN2_BF16), dtype=torch.uint8, device=dev)
+        o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+        ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+        grads = {"dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]), "dv": torch.empty_like(d["v"]),
+                 "dlog_alpha": torch.empty_like(la), "dbeta": torch.empty_like(beta),
+                 "dS0": torch.empty((B, H, D, D), dtype=torch.float32, device=dev)}
+
+        def step():
+            binding.gdn2_beta_fwd(gate, *(d[n] for n in names), la, beta, None, save_states=True, ws=ws, o=o, ST=ST)
+            binding.gdn2_beta_bwd(gate, *(d[n] for n in names), la, beta, d["dout"], None, None, states_saved=True,
+                                  ws=ws, grads=grads)
+
+        ms = timed_ms(step, max(5, args.steps), dev)
+        out[name + "_ms"] = ms
+        out["overhead_of_gdn2_over_" + name] = gdn2_ms / ms - 1.0
+        out[name + "_status"] = binding.gdn2_device_status()
+        del ws, o, ST, grads
+    out["note"] = ("KDA and Gated DeltaNet run the GDN-2 kernels on gates broadcast into the workspace, plus a "
+                   "broadcast and a gate-sum kernel; a negative overhead means the reduced model costs more here")
+    torch.cuda.empty_cache()
+    return out
+
+
 SWEEP_TOKENS = 65536
 SWEEP_T = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
 
@@ -523,9 +563,11 @@ def main():
     full = args.B is None and args.T is None
     if not args.no_decode and full:
         decode = bench_decode(binding, dev)
+    reductions = None
     if not args.no_extra and full and world == 1:
         configs = measure_configs(binding, dev, args, d)
         sweep = measure_sweep(binding, dev, args)
+        reductions = measure_reductions(binding, dev, d, args, ms_per_step)
 
     line = None
     if rank == 0:
@@ -547,7 +589,7 @@ def main():
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_in_timed_region,
-                "decode": decode, "configs": configs, "sweep": sweep}
+                "decode": decode, "configs": configs, "sweep": sweep, "kda_overhead": reductions}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -162,6 +162,46 @@ gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const 
                              int Dk, int Dv, gdn2_dtype dt, void* stream);
 
 /*
+ * The two recurrences that the operator generalises, run through the same
+ * kernels (README "Strict Generalization" bullet, arXiv abstract). With the
+ * erase and write gates one scalar beta_t per head and token, b_t = w_t =
+ * beta_t 1, the operator is KDA,
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ * and with the decay also one scalar per head and token it is Gated DeltaNet
+ * (published with the state transposed, d_v x d_k; here the state keeps the
+ * [B, H, Dk, Dv] layout of gdn2_fwd, the transpose of the published one).
+ *   gate       GDN2_GATE_KDA: log_alpha [B, T, H, Dk] (channel-wise decay)
+ *              GDN2_GATE_GDN: log_alpha [B, T, H]     (one decay per head and token)
+ *   beta       [B, T, H] dt
+ *   dbeta      [B, T, H] dt (output of the backward); for GDN2_GATE_GDN dlog_alpha
+ *              is [B, T, H], else [B, T, H, Dk]
+ * Everything else as gdn2_fwd / gdn2_bwd, including the chunk and the paths
+ * taken. The calls broadcast beta (and a scalar decay) into the workspace,
+ * run gdn2_fwd / gdn2_bwd on it, and (backward) sum the gradients of the
+ * broadcast gates back over their channels: dbeta_t = sum_i db_ti +
+ * sum_j dw_tj, dlog_a_t = sum_i dlog_alpha_ti.
+ * Workspace: gdn2_beta_workspace_size(gate, op, ...) bytes, 256-byte aligned;
+ * one buffer of the GDN2_OP_BWD size serves gdn2_beta_fwd(save_states = 1)
+ * followed by gdn2_beta_bwd(states_saved = 1). Returns 0 for an invalid gate
+ * or problem.
+ */
+typedef enum gdn2_gate {
+    GDN2_GATE_KDA = 1,   /* beta per head and token, channel-wise decay */
+    GDN2_GATE_GDN = 2    /* beta and the decay per head and token */
+} gdn2_gate;
+size_t gdn2_beta_workspace_size(gdn2_gate gate, gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk,
+                                gdn2_dtype dt);
+gdn2_status gdn2_beta_fwd(gdn2_gate gate, const void* q, const void* k, const void* v, const void* log_alpha,
+                          const void* beta, const float* S0, void* o, float* ST, int B, int T, int H, int Dk,
+                          int Dv, int chunk, gdn2_dtype dt, int save_states, void* ws, size_t ws_bytes,
+                          void* stream);
+gdn2_status gdn2_beta_bwd(gdn2_gate gate, const void* q, const void* k, const void* v, const void* log_alpha,
+                          const void* beta, const float* S0, const void* dout, const float* dST, void* dq,
+                          void* dk, void* dv, void* dlog_alpha, void* dbeta, float* dS0, int B, int T, int H,
+                          int Dk, int Dv, int chunk, gdn2_dtype dt, int states_saved, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/*
  * Backward without a caller-supplied workspace. The paper has no counterpart:
  * this entry point exists for callers that cannot call cudaMalloc where they
  * need gradients -- code running inside another component's memory management

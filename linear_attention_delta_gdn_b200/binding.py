@@ -29,7 +29,9 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GD
 #: exported symbols, as declared in include/gdn2.h
 EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "gdn2_status_string",
            "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes",
-           "gdn2_trace_enable", "gdn2_trace_read", "gdn2_device_status")
+           "gdn2_trace_enable", "gdn2_trace_read", "gdn2_device_status", "gdn2_beta_workspace_size",
+           "gdn2_beta_fwd", "gdn2_beta_bwd")
+GDN2_GATE_KDA, GDN2_GATE_GDN = 1, 2
 
 
 class Gdn2Error(RuntimeError):
@@ -66,6 +68,12 @@ def lib(path: Optional[str] = None) -> ctypes.CDLL:
     L.gdn2_bwd_no_alloc.restype = I
     L.gdn2_no_alloc_scratch_bytes.argtypes = []
     L.gdn2_no_alloc_scratch_bytes.restype = Z
+    L.gdn2_beta_workspace_size.argtypes = [I] * 9
+    L.gdn2_beta_workspace_size.restype = Z
+    L.gdn2_beta_fwd.argtypes = [I] + [P] * 8 + [I] * 8 + [P, Z, P]
+    L.gdn2_beta_fwd.restype = I
+    L.gdn2_beta_bwd.argtypes = [I] + [P] * 14 + [I] * 8 + [P, Z, P]
+    L.gdn2_beta_bwd.restype = I
     L.gdn2_device_status.argtypes = [P]
     L.gdn2_device_status.restype = I
     L.gdn2_trace_enable.argtypes = [I]
@@ -175,6 +183,64 @@ def gdn2_bwd(q, k, v, log_alpha, b, w, dout, S0=None, dST=None, chunk: int = 64,
                         _ptr(g["db"]), _ptr(g["dw"]), _ptr(g.get("dS0")), B, T, H, Dk, Dv, chunk, dt,
                         int(states_saved), _ptr(ws), ws.numel(), _stream(q.device))
     _check("gdn2_bwd", rc)
+    return grads
+
+
+def gdn2_beta_workspace_size(gate: int, op: int, B: int, T: int, H: int, Dk: int, Dv: int, chunk: int,
+                             dt: int) -> int:
+    return int(lib().gdn2_beta_workspace_size(gate, op, B, T, H, Dk, Dv, chunk, dt))
+
+
+def gdn2_beta_fwd(gate, q, k, v, log_alpha, beta, S0=None, chunk: int = 64, want_state: bool = True,
+                  save_states: bool = False, ws: Optional[torch.Tensor] = None, o=None, ST=None):
+    """KDA (gate=GDN2_GATE_KDA, log_alpha [B,T,H,Dk]) or Gated DeltaNet (GDN2_GATE_GDN, log_alpha [B,T,H])
+    forward through the Gated Delta Rule-2 kernels; beta [B,T,H]. Returns ``(o, ST)``."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    la_shape = (B, T, H, Dk) if gate == GDN2_GATE_KDA else (B, T, H)
+    for name, t, shp in (("k", k, (B, T, H, Dk)), ("v", v, (B, T, H, Dv)), ("log_alpha", log_alpha, la_shape),
+                         ("beta", beta, (B, T, H))):
+        if t.dtype != q.dtype or tuple(t.shape) != shp:
+            raise ValueError("%s must be %s %s" % (name, q.dtype, shp))
+    _state(S0, q, B, H, Dk, Dv)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
+    if ST is None and want_state:
+        ST = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    op = GDN2_OP_FWD_SAVE if save_states else GDN2_OP_FWD
+    need = gdn2_beta_workspace_size(gate, op, B, T, H, Dk, Dv, chunk, dt)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rc = lib().gdn2_beta_fwd(gate, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(o),
+                             _ptr(ST), B, T, H, Dk, Dv, chunk, dt, int(save_states), _ptr(ws), ws.numel(),
+                             _stream(q.device))
+    _check("gdn2_beta_fwd", rc)
+    return o, ST
+
+
+def gdn2_beta_bwd(gate, q, k, v, log_alpha, beta, dout, S0=None, dST=None, chunk: int = 64, want_dS0: bool = True,
+                  states_saved: bool = False, ws: Optional[torch.Tensor] = None, grads=None):
+    """Backward of :func:`gdn2_beta_fwd`: dict with dq, dk, dv, dlog_alpha (shape of log_alpha), dbeta
+    [B,T,H] and dS0."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    _state(S0, q, B, H, Dk, Dv)
+    _state(dST, q, B, H, Dk, Dv)
+    if grads is None:
+        grads = {"dq": torch.empty_like(q), "dk": torch.empty_like(q), "dv": torch.empty_like(v),
+                 "dlog_alpha": torch.empty_like(log_alpha), "dbeta": torch.empty_like(beta),
+                 "dS0": torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device) if want_dS0 else None}
+    need = gdn2_beta_workspace_size(gate, GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    g = grads
+    rc = lib().gdn2_beta_bwd(gate, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(dout),
+                             _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]),
+                             _ptr(g["dbeta"]), _ptr(g.get("dS0")), B, T, H, Dk, Dv, chunk, dt, int(states_saved),
+                             _ptr(ws), ws.numel(), _stream(q.device))
+    _check("gdn2_beta_bwd", rc)
     return grads
 
 

@@ -1,0 +1,259 @@
+// beta_gates.cu -- KDA and Gated DeltaNet through the Gated Delta Rule-2 kernels.
+//
+// "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention" (README "Strict Generalization"
+// bullet, arXiv abstract) states that the operator reduces to KDA when the erase and write gates are one
+// scalar beta_t per head and token (b_t = w_t = beta_t 1), and further to Gated DeltaNet when the decay is
+// also one scalar per head and token. These entry points take the reduced gates, broadcast them into the
+// workspace (b, w and, for the scalar decay, log_alpha), run gdn2_fwd / gdn2_bwd, and sum the gradients
+// of the broadcast gates back over their channels:
+//   dbeta_t = sum_i db_ti + sum_j dw_tj,    dlog_a_t = sum_i dlog_alpha_ti   (scalar decay).
+// Both steps are memory-bound elementwise kernels (16-byte accesses, one warp per row for the sums).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "gdn2.h"
+#include "internal.h"
+
+namespace gdn2 {
+namespace {
+
+size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// 8 copies of one value at dst (16-byte aligned), in 16-byte stores
+__device__ __forceinline__ void store8(__nv_bfloat16* dst, __nv_bfloat16 v) {
+    const uint32_t x = (uint32_t)__bfloat16_as_ushort(v) * 0x10001u;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(x, x, x, x);
+}
+__device__ __forceinline__ void store8(float* dst, float v) {
+    *reinterpret_cast<float4*>(dst) = make_float4(v, v, v, v);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(v, v, v, v);
+}
+
+// Per-row broadcast: row r = (b, t, h); b[r][0:Dk] = beta[r], w[r][0:Dv] = beta[r], la[r][0:Dk] = la_s[r]
+// (scalar decay only). One thread per 8 consecutive elements of the row's [b | w | la] concatenation.
+template <typename Tin>
+__global__ void expand_kernel(const Tin* __restrict__ beta, const Tin* __restrict__ la_s, Tin* __restrict__ b,
+                              Tin* __restrict__ w, Tin* __restrict__ la, long long rows, int Dk, int Dv) {
+    const int nb = Dk / 8, nw = Dv / 8, nl = la_s ? Dk / 8 : 0, per = nb + nw + nl;
+    const long long total = rows * per;
+    for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
+         x += (long long)gridDim.x * blockDim.x) {
+        const long long r = x / per;
+        const int p = (int)(x - r * per);
+        Tin val;
+        Tin* dst;
+        if (p < nb) {
+            val = beta[r];
+            dst = b + r * Dk + 8 * p;
+        } else if (p < nb + nw) {
+            val = beta[r];
+            dst = w + r * Dv + 8 * (p - nb);
+        } else {
+            val = la_s[r];
+            dst = la + r * Dk + 8 * (p - nb - nw);
+        }
+        store8(dst, val);
+    }
+}
+
+// Per-row sums: dbeta[r] = sum db[r] + sum dw[r]; dla_s[r] = sum dla[r] (scalar decay only). One warp per row.
+template <typename Tin>
+__global__ void reduce_kernel(const Tin* __restrict__ db, const Tin* __restrict__ dw, const Tin* __restrict__ dla,
+                              Tin* __restrict__ dbeta, Tin* __restrict__ dla_s, long long rows, int Dk, int Dv) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        float sb = 0.f, sl = 0.f;
+        for (int i = lane; i < Dk; i += 32) {
+            sb += to_f32(db[r * Dk + i]);
+            if (dla) sl += to_f32(dla[r * Dk + i]);
+        }
+        for (int j = lane; j < Dv; j += 32) sb += to_f32(dw[r * Dv + j]);
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+            sb += __shfl_xor_sync(0xffffffffu, sb, m);
+            sl += __shfl_xor_sync(0xffffffffu, sl, m);
+        }
+        if (lane == 0) {
+            dbeta[r] = from_f32<Tin>(sb);
+            if (dla) dla_s[r] = from_f32<Tin>(sl);
+        }
+    }
+}
+
+int grid_for(long long work, int block) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long want = (work + block - 1) / block;
+    const long long cap = (long long)sms * 8;
+    return (int)(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+template <typename Tin>
+cudaError_t launch_expand(const void* beta, const void* la_s, void* b, void* w, void* la, long long rows, int Dk,
+                          int Dv, cudaStream_t s) {
+    const long long work = rows * (Dk / 8 + Dv / 8 + (la_s ? Dk / 8 : 0));
+    TraceScope trace(K_GATE_EXPAND, s);
+    expand_kernel<Tin><<<grid_for(work, 256), 256, 0, s>>>(static_cast<const Tin*>(beta), static_cast<const Tin*>(la_s),
+                                                          static_cast<Tin*>(b), static_cast<Tin*>(w),
+                                                          static_cast<Tin*>(la), rows, Dk, Dv);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_reduce(const void* db, const void* dw, const void* dla, void* dbeta, void* dla_s, long long rows,
+                          int Dk, int Dv, cudaStream_t s) {
+    TraceScope trace(K_GATE_REDUCE, s);
+    reduce_kernel<Tin><<<grid_for(rows * 32, 256), 256, 0, s>>>(
+        static_cast<const Tin*>(db), static_cast<const Tin*>(dw), static_cast<const Tin*>(dla),
+        static_cast<Tin*>(dbeta), static_cast<Tin*>(dla_s), rows, Dk, Dv);
+    return cudaGetLastError();
+}
+
+// Workspace of the reduced-gate calls (each region 256-byte aligned):
+//   [gdn2 workspace: gdn2_workspace_size(GDN2_OP_FWD) for a plain forward, else of GDN2_OP_BWD]
+//   [b: rows x Dk][w: rows x Dv][log_alpha: rows x Dk (scalar decay)]
+//   backward only: [db: rows x Dk][dw: rows x Dv][dlog_alpha: rows x Dk (scalar decay)]
+struct Layout {
+    size_t base, b, w, la, db, dw, dla, total;
+};
+Layout layout(gdn2_gate gate, gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt) {
+    Layout L{};
+    const size_t es = dt == GDN2_BF16 ? 2 : 4;
+    const size_t rows = (size_t)B * T * H;
+    const bool scalar = gate == GDN2_GATE_GDN;
+    L.base = al256(gdn2_workspace_size(op == GDN2_OP_FWD ? GDN2_OP_FWD : GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt));
+    L.b = L.base;
+    L.w = L.b + al256(rows * Dk * es);
+    L.la = L.w + al256(rows * Dv * es);
+    L.db = L.la + (scalar ? al256(rows * Dk * es) : 0);
+    L.dw = L.db + al256(rows * Dk * es);
+    L.dla = L.dw + al256(rows * Dv * es);
+    L.total = op == GDN2_OP_BWD ? L.dla + (scalar ? al256(rows * Dk * es) : 0) : L.db;
+    return L;
+}
+
+thread_local char g_err[256];
+gdn2_status report(gdn2_status s) {
+    set_last_error(g_err);
+    return s;
+}
+
+}  // namespace
+}  // namespace gdn2
+
+using namespace gdn2;
+
+extern "C" {
+
+size_t gdn2_beta_workspace_size(gdn2_gate gate, gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk,
+                                gdn2_dtype dt) {
+    if (gate != GDN2_GATE_KDA && gate != GDN2_GATE_GDN) return 0;
+    if (gdn2_workspace_size(GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt) == 0 && T > 0) return 0;
+    return layout(gate, op, B, T, H, Dk, Dv, chunk, dt).total;
+}
+
+gdn2_status gdn2_beta_fwd(gdn2_gate gate, const void* q, const void* k, const void* v, const void* log_alpha,
+                          const void* beta, const float* S0, void* o, float* ST, int B, int T, int H, int Dk, int Dv,
+                          int chunk, gdn2_dtype dt, int save_states, void* ws, size_t ws_bytes, void* stream) {
+    if (gate != GDN2_GATE_KDA && gate != GDN2_GATE_GDN) {
+        snprintf(g_err, sizeof(g_err), "gate=%d is not GDN2_GATE_KDA or GDN2_GATE_GDN", (int)gate);
+        return report(GDN2_ERR_INVALID);
+    }
+    if (T > 0 && (!beta || !log_alpha)) {
+        snprintf(g_err, sizeof(g_err), "%s must not be NULL", beta ? "log_alpha" : "beta");
+        return report(GDN2_ERR_INVALID);
+    }
+    const gdn2_op op = save_states ? GDN2_OP_FWD_SAVE : GDN2_OP_FWD;
+    const Layout L = layout(gate, op, B, T, H, Dk, Dv, chunk, dt);
+    if (T > 0) {
+        if (gdn2_workspace_size(GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt) == 0)   // invalid sizes: let gdn2_fwd say why
+            return gdn2_fwd(q, k, v, log_alpha, log_alpha, log_alpha, S0, o, ST, B, T, H, Dk, Dv, chunk, dt,
+                            save_states, ws, ws_bytes, stream);
+        if (!ws || ws_bytes < L.total || ((uintptr_t)ws & 255)) {
+            snprintf(g_err, sizeof(g_err), "gdn2_beta_fwd needs a 256-byte aligned workspace of %zu bytes, got %zu",
+                     L.total, ws ? ws_bytes : 0);
+            return report(ws && ws_bytes >= L.total ? GDN2_ERR_INVALID : GDN2_ERR_WORKSPACE);
+        }
+    }
+    unsigned char* w8 = static_cast<unsigned char*>(ws);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool scalar = gate == GDN2_GATE_GDN;
+    const void* la_full = log_alpha;
+    if (T > 0) {
+        const long long rows = (long long)B * T * H;
+        cudaError_t e = dt == GDN2_BF16
+                            ? launch_expand<__nv_bfloat16>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w,
+                                                           w8 + L.la, rows, Dk, Dv, s)
+                            : launch_expand<float>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w, w8 + L.la,
+                                                   rows, Dk, Dv, s);
+        if (e != cudaSuccess) {
+            snprintf(g_err, sizeof(g_err), "gdn2_beta_fwd (gate broadcast): %s", cudaGetErrorString(e));
+            return report(GDN2_ERR_CUDA);
+        }
+        if (scalar) la_full = w8 + L.la;
+    }
+    return gdn2_fwd(q, k, v, la_full, T > 0 ? w8 + L.b : nullptr, T > 0 ? w8 + L.w : nullptr, S0, o, ST, B, T, H,
+                    Dk, Dv, chunk, dt, save_states, ws, L.base, stream);
+}
+
+gdn2_status gdn2_beta_bwd(gdn2_gate gate, const void* q, const void* k, const void* v, const void* log_alpha,
+                          const void* beta, const float* S0, const void* dout, const float* dST, void* dq, void* dk,
+                          void* dv, void* dlog_alpha, void* dbeta, float* dS0, int B, int T, int H, int Dk, int Dv,
+                          int chunk, gdn2_dtype dt, int states_saved, void* ws, size_t ws_bytes, void* stream) {
+    if (gate != GDN2_GATE_KDA && gate != GDN2_GATE_GDN) {
+        snprintf(g_err, sizeof(g_err), "gate=%d is not GDN2_GATE_KDA or GDN2_GATE_GDN", (int)gate);
+        return report(GDN2_ERR_INVALID);
+    }
+    const Layout L = layout(gate, GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt);
+    if (T > 0) {
+        if (!beta || !log_alpha || !dbeta || !dlog_alpha) {
+            snprintf(g_err, sizeof(g_err), "beta, log_alpha, dbeta and dlog_alpha must not be NULL");
+            return report(GDN2_ERR_INVALID);
+        }
+        if (gdn2_workspace_size(GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt) == 0)
+            return gdn2_bwd(q, k, v, log_alpha, log_alpha, log_alpha, S0, dout, dST, dq, dk, dv, dlog_alpha, dbeta,
+                            dbeta, dS0, B, T, H, Dk, Dv, chunk, dt, states_saved, ws, ws_bytes, stream);
+        if (!ws || ws_bytes < L.total || ((uintptr_t)ws & 255)) {
+            snprintf(g_err, sizeof(g_err), "gdn2_beta_bwd needs a 256-byte aligned workspace of %zu bytes, got %zu",
+                     L.total, ws ? ws_bytes : 0);
+            return report(ws && ws_bytes >= L.total ? GDN2_ERR_INVALID : GDN2_ERR_WORKSPACE);
+        }
+    }
+    unsigned char* w8 = static_cast<unsigned char*>(ws);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool scalar = gate == GDN2_GATE_GDN;
+    const long long rows = (long long)B * T * H;
+    if (T > 0) {   // the broadcast gates (again: the forward may have run with another workspace)
+        cudaError_t e = dt == GDN2_BF16
+                            ? launch_expand<__nv_bfloat16>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w,
+                                                           w8 + L.la, rows, Dk, Dv, s)
+                            : launch_expand<float>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w, w8 + L.la,
+                                                   rows, Dk, Dv, s);
+        if (e != cudaSuccess) {
+            snprintf(g_err, sizeof(g_err), "gdn2_beta_bwd (gate broadcast): %s", cudaGetErrorString(e));
+            return report(GDN2_ERR_CUDA);
+        }
+    }
+    void* dla_full = scalar ? static_cast<void*>(w8 + L.dla) : dlog_alpha;
+    gdn2_status st = gdn2_bwd(q, k, v, scalar ? static_cast<const void*>(w8 + L.la) : log_alpha,
+                              T > 0 ? w8 + L.b : nullptr, T > 0 ? w8 + L.w : nullptr, S0, dout, dST, dq, dk, dv,
+                              T > 0 ? dla_full : dlog_alpha, T > 0 ? w8 + L.db : dbeta, T > 0 ? w8 + L.dw : dbeta,
+                              dS0, B, T, H, Dk, Dv, chunk, dt, states_saved, ws, L.base, stream);
+    if (st != GDN2_OK || T == 0) return st;
+    cudaError_t e = dt == GDN2_BF16
+                        ? launch_reduce<__nv_bfloat16>(w8 + L.db, w8 + L.dw, scalar ? w8 + L.dla : nullptr, dbeta,
+                                                       scalar ? dlog_alpha : nullptr, rows, Dk, Dv, s)
+                        : launch_reduce<float>(w8 + L.db, w8 + L.dw, scalar ? w8 + L.dla : nullptr, dbeta,
+                                               scalar ? dlog_alpha : nullptr, rows, Dk, Dv, s);
+    if (e != cudaSuccess) {
+        snprintf(g_err, sizeof(g_err), "gdn2_beta_bwd (gate sums): %s", cudaGetErrorString(e));
+        return report(GDN2_ERR_CUDA);
+    }
+    return GDN2_OK;
+}
+
+}  // extern "C"

@@ -69,7 +69,8 @@ struct ChunkBwdArgs {
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 
 // Kernels of the library, for gdn2_trace_read().
-enum KernelId { K_CHUNK_FWD = 0, K_CHUNK_BWD, K_REC_FWD, K_REC_BWD, K_DECODE, KERNEL_COUNT };
+enum KernelId { K_CHUNK_FWD = 0, K_CHUNK_BWD, K_REC_FWD, K_REC_BWD, K_DECODE, K_GATE_EXPAND, K_GATE_REDUCE,
+                KERNEL_COUNT };
 
 // Brackets one kernel launch with CUDA events on its stream while tracing is on.
 class TraceScope {

@@ -104,6 +104,16 @@ def make_inputs(B, T, H, Dk, Dv, seed, dtype="f32", with_do=False, with_S0=False
     return out
 
 
+def make_reduced_gates(B, T, H, seed, dtype="f32"):
+    """Gates of the two reductions (KDA, Gated DeltaNet), drawn with the recipe's distributions but one value
+    per head and token: beta = sigmoid(N(0, 1)) and log_a = -softplus(N(0, 1)) / 16, both [B, T, H], from
+    numpy PCG64(seed), in that order."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    beta = _sigmoid(rng.standard_normal(size=(B, T, H)))
+    log_a = -_softplus(rng.standard_normal(size=(B, T, H))) / 16.0
+    return {"beta": _round(beta, dtype), "log_a": _round(log_a, dtype)}
+
+
 def make_workload_inputs(wl: Workload):
     """Inputs of a sequence workload (``mode`` fwd or fwd_bwd)."""
     return make_inputs(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, wl.seed, wl.dtype,

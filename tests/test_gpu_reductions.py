@@ -1,0 +1,108 @@
+"""KDA and Gated DeltaNet through the Gated Delta Rule-2 kernels (gdn2_beta_fwd / gdn2_beta_bwd), against the
+fp64 oracle run with the broadcast gates b = w = beta * 1 (and, for Gated DeltaNet, log_alpha = log_a * 1).
+
+The oracle's agreement with the two published recurrences is pinned on the CPU
+(tests/test_oracle_pins.py::test_reduces_to_kda, ::test_reduces_to_gated_deltanet). Gradients of the reduced
+gates follow from the chain rule through the broadcast: dbeta_t = sum_i db_ti + sum_j dw_tj and
+dlog_a_t = sum_i dlog_alpha_ti. Tolerances as for the operator (relative L2, whole tensor and worst head):
+fp32 1e-4; bf16 o, S_T 2e-2 and gradients 3e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import rel_l2, worst_head_rel_l2
+from linear_attention_delta_gdn_b200 import binding
+from linear_attention_delta_gdn_b200.inputs import make_inputs, make_reduced_gates, to_f64
+
+pytestmark = pytest.mark.gpu
+
+TOL_OUT = {"f32": 1e-4, "bf16": 2e-2}
+TOL_GRAD = {"f32": 1e-4, "bf16": 3e-2}
+GATES = {"kda": binding.GDN2_GATE_KDA, "gdn": binding.GDN2_GATE_GDN}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from linear_attention_delta_gdn_b200 import build
+    build.build()
+
+
+def _case(gate, B, T, H, Dk, Dv, dtype, seed):
+    x = make_inputs(B, T, H, Dk, Dv, seed=seed, dtype=dtype, with_do=True, with_S0=True)
+    r = make_reduced_gates(B, T, H, seed + 1, dtype)
+    la = x["log_alpha"] if gate == "kda" else r["log_a"]
+    return x, r["beta"], la
+
+
+def _check(got, ref, tol, name, state=False):
+    got = np.asarray(got)
+    assert np.all(np.isfinite(got)), name
+    e = rel_l2(got, ref)
+    wh = worst_head_rel_l2(got, ref, state=state) if got.ndim == 4 else e
+    assert e <= tol and wh <= tol, "%s: rel err %.3g (worst head %.3g) > %g" % (name, e, wh, tol)
+
+
+def _worst_rows(got, ref):
+    """[B, T, H] tensors: worst per-(b, h) relative error."""
+    worst = 0.0
+    for b in range(ref.shape[0]):
+        for h in range(ref.shape[2]):
+            worst = max(worst, rel_l2(got[b, :, h], ref[b, :, h]))
+    return worst
+
+
+@pytest.mark.parametrize("gate", ["kda", "gdn"])
+@pytest.mark.parametrize("dtype,T,Dk,Dv,chunk", [("bf16", 150, 128, 128, 64), ("bf16", 300, 128, 128, 64),
+                                                 ("f32", 70, 64, 64, 32), ("bf16", 97, 64, 128, 64)])
+def test_reduced_gates_against_oracle(oracle_mod, gate, dtype, T, Dk, Dv, chunk):
+    B, H = 2, 3
+    x, beta, la = _case(gate, B, T, H, Dk, Dv, dtype, seed=1200 + T + Dk)
+    d = {n: t.cuda() for n, t in x.items()}
+    dST = torch.randn((B, H, Dk, Dv), generator=torch.Generator().manual_seed(9))
+    g_beta, g_la = beta.cuda(), la.cuda()
+    ws = torch.empty(binding.gdn2_beta_workspace_size(GATES[gate], binding.GDN2_OP_BWD, B, T, H, Dk, Dv, chunk,
+                                                      binding._dt(d["q"])), dtype=torch.uint8, device="cuda")
+    o, ST = binding.gdn2_beta_fwd(GATES[gate], d["q"], d["k"], d["v"], g_la, g_beta, d["S0"], chunk=chunk,
+                                  save_states=True, ws=ws)
+    g = binding.gdn2_beta_bwd(GATES[gate], d["q"], d["k"], d["v"], g_la, g_beta, d["dout"], d["S0"], dST.cuda(),
+                              chunk=chunk, states_saved=True, ws=ws)
+    torch.cuda.synchronize()
+
+    f = {n: to_f64(t) for n, t in x.items()}
+    be, lae = to_f64(beta), to_f64(la)
+    b_full = np.repeat(be[..., None], Dk, axis=-1)
+    w_full = np.repeat(be[..., None], Dv, axis=-1)
+    la_full = lae if gate == "kda" else np.repeat(lae[..., None], Dk, axis=-1)
+    o_ref, ST_ref = oracle_mod.fwd(f["q"], f["k"], f["v"], la_full, b_full, w_full, S0=f["S0"])
+    ref = oracle_mod.bwd(f["q"], f["k"], f["v"], la_full, b_full, w_full, dout=f["dout"], S0=f["S0"],
+                         dST=dST.double().numpy())
+    _check(to_f64(o), o_ref, TOL_OUT[dtype], "o")
+    _check(to_f64(ST), ST_ref, TOL_OUT[dtype], "S_T", state=True)
+    for n in ("dq", "dk", "dv"):
+        _check(to_f64(g[n]), ref[n], TOL_GRAD[dtype], n)
+    _check(to_f64(g["dS0"]), ref["dS0"], TOL_GRAD[dtype], "dS0", state=True)
+    dbeta_ref = ref["db"].sum(-1) + ref["dw"].sum(-1)
+    got = to_f64(g["dbeta"])
+    assert rel_l2(got, dbeta_ref) <= TOL_GRAD[dtype] and _worst_rows(got, dbeta_ref) <= TOL_GRAD[dtype], \
+        "dbeta %.3g" % rel_l2(got, dbeta_ref)
+    if gate == "kda":
+        _check(to_f64(g["dlog_alpha"]), ref["dlog_alpha"], TOL_GRAD[dtype], "dlog_alpha")
+    else:
+        dla_ref = ref["dlog_alpha"].sum(-1)
+        got = to_f64(g["dlog_alpha"])
+        assert rel_l2(got, dla_ref) <= TOL_GRAD[dtype] and _worst_rows(got, dla_ref) <= TOL_GRAD[dtype], \
+            "dlog_a %.3g" % rel_l2(got, dla_ref)
+
+
+def test_reduced_gates_empty_sequence():
+    B, T, H, D = 1, 0, 2, 128
+    x = make_inputs(B, T, H, D, D, seed=5, dtype="bf16", with_do=True, with_S0=True)
+    r = make_reduced_gates(B, T, H, 6, "bf16")
+    d = {n: t.cuda() for n, t in x.items()}
+    o, ST = binding.gdn2_beta_fwd(binding.GDN2_GATE_GDN, d["q"], d["k"], d["v"], r["log_a"].cuda(),
+                                  r["beta"].cuda(), d["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(ST, d["S0"])
