@@ -57,7 +57,7 @@ STEP_FLOPS_PER_TOKEN_HEAD = 3 * 180224
 KERNEL_BYTES_PER_TOKEN_HEAD = {"chunk_fwd_kernel": 1792, "chunk_bwd_kernel": 3328,
                                "recurrent_fwd_kernel": 1792, "recurrent_bwd_kernel": 3328}
 KERNEL_SOURCES = {"chunk_fwd_kernel": ["chunk_fwd.cu"], "chunk_bwd_kernel": ["chunk_bwd.cu"]}
-COMMON_SOURCES = ["chunk_common.cuh", "tc.cuh", "common.cuh"]
+COMMON_SOURCES = ["chunk_common.cuh", "tc.cuh", "common.cuh", "internal.h"]
 
 
 def kernel_source_hash(kernel):
