@@ -952,11 +952,6 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
     }
 }
 
-template <typename K>
-cudaError_t set_smem(K kernel, uint32_t bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-}
-
 }  // namespace
 
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
@@ -968,14 +963,10 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
                            &maps.dq, &maps.dk, &maps.db, &maps.dla, &maps.dv, &maps.dw};
     for (int i = 0; i < 13; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    cudaError_t e = set_smem(chunk_bwd_kernel, SMEM_BYTES_ALL);
+    LaunchFacts lf{};
+    cudaError_t e = launch_facts(chunk_bwd_kernel, BT, SMEM_BYTES_ALL, &lf);
     if (e != cudaSuccess) return e;
-    int dev = 0, nsm = 0, coop = 0, occ = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, chunk_bwd_kernel, BT, SMEM_BYTES_ALL)) != cudaSuccess)
-        return e;
+    const int nsm = lf.nsm, coop = lf.coop, occ = lf.occ;
     const int BH = d.B * d.H, nc = d.nchunks();
     const int units = BH * nc;
     const int slots = nsm * occ;

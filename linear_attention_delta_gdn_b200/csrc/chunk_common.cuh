@@ -33,6 +33,8 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -53,7 +55,7 @@ constexpr uint32_t TILE_64x128 = 64 * 128 * 2;    // bytes of a [64 x 128] bf16 
 
 // Tensor map of a [B, T, H, 128] bf16 tensor; box = 64 channels x 1 head x 64 tokens x 1,
 // 128-byte swizzle, zero fill past the end of the sequence.
-inline CUresult make_token_map(CUtensorMap* map, const void* ptr, int B, int T, int H) {
+inline CUresult encode_token_map(CUtensorMap* map, const void* ptr, int B, int T, int H) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         cudaDriverEntryPointQueryResult q;
@@ -70,6 +72,62 @@ inline CUresult make_token_map(CUtensorMap* map, const void* ptr, int B, int T, 
     return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// The same, from a small per-thread cache keyed by (pointer, B, T, H): a training step passes the same
+// tensors call after call, and encoding a map is host work on every launch otherwise. A map describes
+// only addresses and sizes, so a hit is exact; the cache never dereferences the pointer.
+inline CUresult make_token_map(CUtensorMap* map, const void* ptr, int B, int T, int H) {
+    struct Entry {
+        const void* ptr;
+        int B, T, H;
+        CUtensorMap map;
+    };
+    constexpr int N = 64;
+    thread_local Entry cache[N] = {};
+    const uintptr_t key = reinterpret_cast<uintptr_t>(ptr);
+    const int slot = (int)(((key >> 8) ^ (key >> 20) ^ (uintptr_t)T * 31u ^ (uintptr_t)B * 7u ^ (uintptr_t)H) % N);
+    Entry& e = cache[slot];
+    if (e.ptr == ptr && e.B == B && e.T == T && e.H == H && ptr) {
+        *map = e.map;
+        return CUDA_SUCCESS;
+    }
+    const CUresult r = encode_token_map(map, ptr, B, T, H);
+    if (r == CUDA_SUCCESS) e = Entry{ptr, B, T, H, *map};
+    return r;
+}
+
+// Per-device launch facts of a kernel that never change once known: SM count, cooperative-launch support,
+// resident CTAs per SM at the kernel's shared-memory size. The shared-memory attribute itself is set on every
+// call (a device reset clears it).
+struct LaunchFacts {
+    int nsm, coop, occ;
+};
+template <typename Kernel>
+inline cudaError_t launch_facts(Kernel kernel, int threads, uint32_t smem, LaunchFacts* out) {
+    constexpr int kMaxDev = 64;
+    static LaunchFacts facts[kMaxDev];
+    static bool known[kMaxDev];
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < kMaxDev && known[dev]) {
+        *out = facts[dev];
+        return cudaSuccess;
+    }
+    LaunchFacts f{};
+    if ((e = cudaDeviceGetAttribute(&f.nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&f.coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.occ, kernel, threads, smem)) != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev) {
+        facts[dev] = f;
+        known[dev] = true;
+    }
+    *out = f;
+    return cudaSuccess;
 }
 
 // ------------------------------------------------------------ device

@@ -864,14 +864,10 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     CUtensorMap* mp[6] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w};
     for (int i = 0; i < 6; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    LaunchFacts lf{};
+    cudaError_t e = launch_facts(chunk_fwd_kernel, NT, SMEM_BYTES, &lf);
     if (e != cudaSuccess) return e;
-    int dev = 0, nsm = 0, coop = 0, occ = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, chunk_fwd_kernel, NT, SMEM_BYTES)) != cudaSuccess)
-        return e;
+    const int nsm = lf.nsm, coop = lf.coop, occ = lf.occ;
     const int BH = d.B * d.H, nc = d.nchunks();
     const int units = BH * nc;
     const int slots = nsm * occ;

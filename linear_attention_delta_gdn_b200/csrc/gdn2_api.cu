@@ -11,10 +11,22 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "gdn2.h"
 #include "internal.h"
 
 using namespace gdn2;
+
+namespace {
+// An NVTX range around an entry point (visible in Nsight timelines; free when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace
 
 namespace {
 
@@ -160,6 +172,7 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
                      const void* w, const float* S0, void* o, float* ST, int B, int T, int H, int Dk,
                      int Dv, int chunk, gdn2_dtype dt, int save_states, void* ws, size_t ws_bytes,
                      void* stream) {
+    NvtxRange nvtx("gdn2_fwd");
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
     const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
@@ -204,6 +217,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
                      void* dk, void* dv, void* dlog_alpha, void* db, void* dw, float* dS0, int B, int T,
                      int H, int Dk, int Dv, int chunk, gdn2_dtype dt, int states_saved, void* ws,
                      size_t ws_bytes, void* stream) {
+    NvtxRange nvtx("gdn2_bwd");
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
     const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
@@ -273,6 +287,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
 gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
                              const void* b, const void* w, float* S, void* o, int B, int H, int Dk,
                              int Dv, gdn2_dtype dt, void* stream) {
+    NvtxRange nvtx("gdn2_decode_step");
     gdn2_status st = check_dims(B, 1, H, Dk, Dv, 64, dt, false);
     if (st != GDN2_OK) return st;
     REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(log_alpha);
