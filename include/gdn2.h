@@ -202,6 +202,38 @@ gdn2_status gdn2_beta_bwd(gdn2_gate gate, const void* q, const void* k, const vo
                           size_t ws_bytes, void* stream);
 
 /*
+ * Sequences of different lengths packed along the token axis. Sequence n
+ * holds packed tokens cu_seqlens[n] .. cu_seqlens[n+1] - 1 and has its own
+ * initial and final state; the state does not pass from one sequence to the
+ * next.
+ *   q, k, log_alpha, b : [Ttot, H, Dk] dt ;  v, w, o, dout : [Ttot, H, Dv] dt
+ *   cu_seqlens         : [N + 1] int32, DEVICE memory, non-decreasing, from 0
+ *   N, Tmax, Ttot      : number of sequences, a bound on their lengths (host
+ *                        ints; the work is sized by N x Tmax), packed length
+ *   S0, ST, dST, dS0   : [N, H, Dk, Dv] float32 (nullable as in gdn2_fwd/bwd)
+ * Token gradients are packed like the inputs. The calls copy the packed
+ * tensors into a zero-padded [N, Tmax, H, D] layout in the workspace, run
+ * gdn2_fwd / gdn2_bwd on it and copy the results back (a zero token maps the
+ * state to itself, so the padding changes no result). cu_seqlens is not read
+ * on the host: a sequence longer than Tmax is cut at Tmax, one outside
+ * [0, Ttot) is skipped, and gdn2_device_status then returns GDN2_ERR_INVALID
+ * with the detail "cu_seqlens".
+ * Workspace: gdn2_varlen_workspace_size(op, ...) bytes, 256-byte aligned; the
+ * GDN2_OP_BWD size serves gdn2_varlen_fwd(save_states = 1) followed by
+ * gdn2_varlen_bwd(states_saved = 1).
+ */
+size_t gdn2_varlen_workspace_size(gdn2_op op, int N, int Tmax, int H, int Dk, int Dv, int chunk, gdn2_dtype dt);
+gdn2_status gdn2_varlen_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                            const void* w, const int* cu_seqlens, int N, int Tmax, long long Ttot, const float* S0,
+                            void* o, float* ST, int H, int Dk, int Dv, int chunk, gdn2_dtype dt, int save_states,
+                            void* ws, size_t ws_bytes, void* stream);
+gdn2_status gdn2_varlen_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                            const void* w, const int* cu_seqlens, int N, int Tmax, long long Ttot, const float* S0,
+                            const void* dout, const float* dST, void* dq, void* dk, void* dv, void* dlog_alpha,
+                            void* db, void* dw, float* dS0, int H, int Dk, int Dv, int chunk, gdn2_dtype dt,
+                            int states_saved, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Backward without a caller-supplied workspace. The paper has no counterpart:
  * this entry point exists for callers that cannot call cudaMalloc where they
  * need gradients -- code running inside another component's memory management
@@ -260,8 +292,9 @@ int gdn2_trace_read(char* names, size_t names_cap, int* launches, double* ms, in
  * cudaStream_t, NULL for the default stream), returns GDN2_ERR_TIMEOUT if such
  * an event was recorded since the previous call (gdn2_last_error names the
  * kernel and the kind of wait) and clears the record; GDN2_ERR_CUDA if the
- * stream holds a CUDA error. The entry points above never synchronise, so this
- * is the call that checks a finished step after the fact.
+ * stream holds a CUDA error, and GDN2_ERR_INVALID if a packed-sequence call met
+ * an inconsistent cu_seqlens (see gdn2_varlen_fwd). The entry points above never
+ * synchronise, so this is the call that checks a finished step after the fact.
  */
 gdn2_status gdn2_device_status(void* stream);
 

@@ -22,7 +22,7 @@ _lib = None
 
 GDN2_F32, GDN2_BF16 = 0, 1
 GDN2_OP_FWD, GDN2_OP_FWD_SAVE, GDN2_OP_BWD = 0, 1, 2
-GDN2_OK, GDN2_ERR_TIMEOUT = 0, 5
+GDN2_OK, GDN2_ERR_INVALID, GDN2_ERR_TIMEOUT = 0, 1, 5
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_WORKSPACE",
           4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT"}
 
@@ -30,7 +30,7 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GD
 EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "gdn2_status_string",
            "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes",
            "gdn2_trace_enable", "gdn2_trace_read", "gdn2_device_status", "gdn2_beta_workspace_size",
-           "gdn2_beta_fwd", "gdn2_beta_bwd")
+           "gdn2_beta_fwd", "gdn2_beta_bwd", "gdn2_varlen_workspace_size", "gdn2_varlen_fwd", "gdn2_varlen_bwd")
 GDN2_GATE_KDA, GDN2_GATE_GDN = 1, 2
 
 
@@ -74,6 +74,13 @@ def lib(path: Optional[str] = None) -> ctypes.CDLL:
     L.gdn2_beta_fwd.restype = I
     L.gdn2_beta_bwd.argtypes = [I] + [P] * 14 + [I] * 8 + [P, Z, P]
     L.gdn2_beta_bwd.restype = I
+    LL = ctypes.c_longlong
+    L.gdn2_varlen_workspace_size.argtypes = [I] * 8
+    L.gdn2_varlen_workspace_size.restype = Z
+    L.gdn2_varlen_fwd.argtypes = [P] * 7 + [I, I, LL] + [P] * 3 + [I] * 6 + [P, Z, P]
+    L.gdn2_varlen_fwd.restype = I
+    L.gdn2_varlen_bwd.argtypes = [P] * 7 + [I, I, LL] + [P] * 10 + [I] * 6 + [P, Z, P]
+    L.gdn2_varlen_bwd.restype = I
     L.gdn2_device_status.argtypes = [P]
     L.gdn2_device_status.restype = I
     L.gdn2_trace_enable.argtypes = [I]
@@ -242,6 +249,56 @@ def gdn2_beta_bwd(gate, q, k, v, log_alpha, beta, dout, S0=None, dST=None, chunk
                              _ptr(ws), ws.numel(), _stream(q.device))
     _check("gdn2_beta_bwd", rc)
     return grads
+
+
+def gdn2_varlen_workspace_size(op: int, N: int, Tmax: int, H: int, Dk: int, Dv: int, chunk: int, dt: int) -> int:
+    return int(lib().gdn2_varlen_workspace_size(op, N, Tmax, H, Dk, Dv, chunk, dt))
+
+
+def gdn2_varlen_fwd(q, k, v, log_alpha, b, w, cu_seqlens, Tmax: int, S0=None, chunk: int = 64,
+                    want_state: bool = True, save_states: bool = False, ws: Optional[torch.Tensor] = None):
+    """Packed sequences: tensors [Ttot, H, D], cu_seqlens int32 [N + 1] on the device, Tmax >= every length.
+    Returns ``(o [Ttot, H, Dv], ST [N, H, Dk, Dv] or None)``."""
+    Ttot, H, Dk = q.shape
+    Dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    dt = _dt(q)
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+        raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+    _state(S0, q, N, H, Dk, Dv)
+    o = torch.empty((Ttot, H, Dv), dtype=q.dtype, device=q.device)
+    ST = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=q.device) if want_state else None
+    need = gdn2_varlen_workspace_size(GDN2_OP_FWD_SAVE if save_states else GDN2_OP_FWD, N, Tmax, H, Dk, Dv, chunk, dt)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rc = lib().gdn2_varlen_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(cu_seqlens), N,
+                               Tmax, Ttot, _ptr(S0), _ptr(o), _ptr(ST), H, Dk, Dv, chunk, dt, int(save_states),
+                               _ptr(ws), ws.numel(), _stream(q.device))
+    _check("gdn2_varlen_fwd", rc)
+    return o, ST
+
+
+def gdn2_varlen_bwd(q, k, v, log_alpha, b, w, dout, cu_seqlens, Tmax: int, S0=None, dST=None, chunk: int = 64,
+                    want_dS0: bool = True, states_saved: bool = False, ws: Optional[torch.Tensor] = None):
+    """Backward of :func:`gdn2_varlen_fwd`: dict of packed dq, dk, dv, dlog_alpha, db, dw and dS0 [N, ...]."""
+    Ttot, H, Dk = q.shape
+    Dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    dt = _dt(q)
+    _state(S0, q, N, H, Dk, Dv)
+    _state(dST, q, N, H, Dk, Dv)
+    g = {n: torch.empty_like(q) for n in ("dq", "dk", "dlog_alpha", "db")}
+    g.update({n: torch.empty_like(v) for n in ("dv", "dw")})
+    g["dS0"] = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=q.device) if want_dS0 else None
+    need = gdn2_varlen_workspace_size(GDN2_OP_BWD, N, Tmax, H, Dk, Dv, chunk, dt)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rc = lib().gdn2_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(cu_seqlens), N,
+                               Tmax, Ttot, _ptr(S0), _ptr(dout), _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                               _ptr(g["dlog_alpha"]), _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), H, Dk, Dv, chunk,
+                               dt, int(states_saved), _ptr(ws), ws.numel(), _stream(q.device))
+    _check("gdn2_varlen_bwd", rc)
+    return g
 
 
 def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None):

@@ -148,6 +148,11 @@ gdn2_status gdn2_device_status(void* stream) {
     unsigned int fwd = 0, bwd = 0;
     if ((e = chunk_fwd_take_errors(&fwd)) != cudaSuccess) return cuda_status(e, "gdn2_device_status (forward record)");
     if ((e = chunk_bwd_take_errors(&bwd)) != cudaSuccess) return cuda_status(e, "gdn2_device_status (backward record)");
+    unsigned int vl = 0;
+    if ((e = varlen_take_errors(&vl)) != cudaSuccess) return cuda_status(e, "gdn2_device_status (varlen record)");
+    if (vl)
+        return fail(GDN2_ERR_INVALID, "cu_seqlens: %s%s", (vl & 1u) ? "a sequence was longer than Tmax (cut) " : "",
+                    (vl & 2u) ? "a sequence lay outside [0, Ttot) or had a negative length (dropped)" : "");
     if (fwd | bwd)
         return fail(GDN2_ERR_TIMEOUT,
                     "device wait gave up: chunk_fwd_kernel bits 0x%x, chunk_bwd_kernel bits 0x%x "

@@ -70,7 +70,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 
 // Kernels of the library, for gdn2_trace_read().
 enum KernelId { K_CHUNK_FWD = 0, K_CHUNK_BWD, K_REC_FWD, K_REC_BWD, K_DECODE, K_GATE_EXPAND, K_GATE_REDUCE,
-                KERNEL_COUNT };
+                K_VARLEN_COPY, KERNEL_COUNT };
 
 // Brackets one kernel launch with CUDA events on its stream while tracing is on.
 class TraceScope {
@@ -94,6 +94,7 @@ bool test_skip_producers();   // host-side fault injection for the forward's two
 // Read and clear the device-side error words of the tensor-core kernels (bit set: a bounded wait gave up).
 cudaError_t chunk_fwd_take_errors(unsigned int* bits);
 cudaError_t chunk_bwd_take_errors(unsigned int* bits);
+cudaError_t varlen_take_errors(unsigned int* bits);   // bit 1: a sequence longer than Tmax; 2: outside [0, Ttot)
 
 // Sets the detail string returned by gdn2_last_error() on this host thread.
 void set_last_error(const char* msg);
