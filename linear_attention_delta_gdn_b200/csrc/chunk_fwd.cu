@@ -106,7 +106,67 @@ struct FwdParams {
     unsigned char* deltas;         // [BH, nc] Delta^T images, or null
     unsigned char* wyimg;          // [BH, nc] WY images
     unsigned int* flags;           // [BH, nc] ready flags (zero at launch)
+    int split_R;                   // > 0: the chunks of a head are cut into split_R segments (long sequences)
+    int phase;                     // with split_R: 1 (first segment, segment maps) or 3 (the other segments)
+    float* sbuf;                   // with split_R: per head, segment start states, then the maps N and M
 };
+
+// ---- consumer tasks
+// Without a split, task t walks every chunk of head t from S0 (zero if none) and writes o, S_T and, for training,
+// the chunk-start state and Delta images. A long sequence with few heads is cut into R segments instead; with
+// the state after segment s-1 written S_s, a segment is an affine map S_{s+1} = M_s S_s + N_s, where N_s is the
+// segment's final state from a zero start and M_s (d_k x d_k) the one from an identity start with no input
+// (U = 0). Phase 1 walks segment 0 for real (its end is S_1) and, for s = 1 .. R-2, N_s and M_s as separate
+// tasks; a prefix kernel then forms S_2 .. S_{R-1}; phase 3 walks segments 1 .. R-1 for real from S_s.
+struct Task {
+    int head, c0, c1;
+    const float* start;   // start state [D][D] (row = key), or null: zero, or identity when ident
+    bool ident;           // start from the identity (a segment's M)
+    bool zero_u;          // no input: U = 0 (a segment's M)
+    bool out;             // the real chain: o and, if requested, the training images
+    float* fin;           // where the final state goes [D][D], or null
+};
+// per head: R-1 start states S_1 .. S_{R-1}, then N_1 .. N_{R-2}, then M_1 .. M_{R-2}
+constexpr int SPLIT_R_MAX = 8;
+constexpr size_t SPLIT_MATS_PER_HEAD = (SPLIT_R_MAX - 1) + 2 * (SPLIT_R_MAX - 2);
+__host__ __device__ inline int seg_begin(int s, int nc, int R) { return (int)((long long)s * nc / R); }
+__device__ __forceinline__ float* split_mat(const FwdParams& p, int head, int kind, int s) {   // kind 0: S, 1: N, 2: M
+    const int R = p.split_R;
+    const int idx = kind == 0 ? s - 1 : (kind == 1 ? (R - 1) + (s - 1) : (R - 1) + (R - 2) + (s - 1));
+    return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
+}
+__device__ __forceinline__ int task_count(const FwdParams& p) {
+    if (!p.split_R) return p.BH;
+    return p.phase == 1 ? p.BH * (1 + 2 * (p.split_R - 2)) : p.BH * (p.split_R - 1);
+}
+__device__ Task task_at(const FwdParams& p, int t) {
+    Task k{};
+    k.head = t % p.BH;
+    const size_t hd = (size_t)k.head * D * D;
+    if (!p.split_R) {
+        k.c0 = 0; k.c1 = p.nc; k.start = p.S0 ? p.S0 + hd : nullptr; k.out = true; k.fin = p.ST ? p.ST + hd : nullptr;
+        return k;
+    }
+    const int R = p.split_R, j = t / p.BH;
+    if (p.phase == 1) {
+        if (j == 0) {
+            k.c0 = 0; k.c1 = seg_begin(1, p.nc, R); k.start = p.S0 ? p.S0 + hd : nullptr; k.out = true;
+            k.fin = split_mat(p, k.head, 0, 1);
+        } else if (j <= R - 2) {
+            k.c0 = seg_begin(j, p.nc, R); k.c1 = seg_begin(j + 1, p.nc, R); k.fin = split_mat(p, k.head, 1, j);
+        } else {
+            const int s2 = j - (R - 2);
+            k.c0 = seg_begin(s2, p.nc, R); k.c1 = seg_begin(s2 + 1, p.nc, R); k.ident = true; k.zero_u = true;
+            k.fin = split_mat(p, k.head, 2, s2);
+        }
+    } else {
+        const int s2 = 1 + j;
+        k.c0 = seg_begin(s2, p.nc, R); k.c1 = s2 == R - 1 ? p.nc : seg_begin(s2 + 1, p.nc, R);
+        k.start = split_mat(p, k.head, 0, s2); k.out = true;
+        k.fin = (s2 == R - 1 && p.ST) ? p.ST + hd : nullptr;
+    }
+    return k;
+}
 
 struct Maps {
     CUtensorMap q, k, v, la, b, w;
@@ -571,7 +631,6 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);   // this warp's TMEM lanes
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 64 * tm_part(warp);      // lane row, column half
     const int T = p.T, H = p.H, nc = p.nc;
-    const bool want_o = (p.o != nullptr);
 
     const uint32_t sST = tc::smem_u32(STt), sDT = tc::smem_u32(DT),
                    sTT = tc::smem_u32(sm + sp::TT), sPP = tc::smem_u32(sm + sp::PP), sWM = tc::smem_u32(sm + sp::WM);
@@ -610,9 +669,16 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
         tc::cp_async_commit();
     };
 
-    for (int headi = cid; headi < p.BH; headi += p.ncons) {
+    const int ntasks = task_count(p);
+    for (int ti = cid; ti < ntasks; ti += p.ncons) {
+        const Task task = task_at(p, ti);
+        const int headi = task.head, c0 = task.c0, c1 = task.c1;
         const size_t head = (size_t)headi;
         const int h = headi % H, b = headi / H;
+        const bool want_o = task.out && p.o != nullptr;
+        unsigned char* const states = task.out ? p.states : nullptr;   // training images: real chains only
+        unsigned char* const deltas = task.out ? p.deltas : nullptr;
+        const bool zero_u = task.zero_u;
         // v and w of chunk c (issued by lane 0 of warps 0 and 1 at once; a TMA issue takes ~100 cycles)
         auto issue_loads = [&](int c) {
             if (lane != 0 || warp > 1) return;
@@ -643,17 +709,20 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 }
             }
         };
-        issue_loads(0);
-        if (nc > 1) issue_loads(1);
-        if (tid == 0) wait_wy(head, 0);
-        // initial state: S^T row j = column j of S0
+        if (!zero_u) {
+            issue_loads(c0);
+            if (c0 + 1 < c1) issue_loads(c0 + 1);
+        }
+        if (tid == 0) wait_wy(head, c0);
+        // start state: S^T row j = column j of the start matrix (zero if none, or the identity)
         {
             const int j = jrow;
             float v[32];
 #pragma unroll 1
             for (int i0 = cpart; i0 < cpart + 64; i0 += 32) {
 #pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] = p.S0 ? p.S0[(head * D + i0 + u) * D + j] : 0.f;
+                for (int u = 0; u < 32; ++u)
+                    v[u] = task.start ? task.start[(i0 + u) * D + j] : (task.ident && i0 + u == j ? 1.f : 0.f);
                 tc::tmem_st32(lane_base + TM_S + i0, v);
 #pragma unroll
                 for (int g = 0; g < 4; ++g) tc::st_row8(STt, D, j, (i0 >> 3) + g, v + 8 * g);
@@ -664,14 +733,14 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
-        copy_wy(head, 0);
-        if (p.states && tid == 0) {
-            tc::bulk_store(p.states + (head * nc + 0) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
+        copy_wy(head, c0);
+        if (states && tid == 0) {
+            tc::bulk_store(states + (head * nc + c0) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
             tc::bulk_commit();
         }
 
-        int c = 0;
-        for (; c < nc; ++c) {
+        int c = c0;
+        for (; c < c1; ++c) {
             const int par = c & 1;
             const uint32_t sQQ = tc::smem_u32(sm + sp::QQ + par * TILE_64x128),
                            sKT = tc::smem_u32(sm + sp::KT + par * TILE_64x128);
@@ -680,12 +749,14 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             unsigned char* UU = UUp(c);
             const unsigned char* WW = WWp(c);
             const uint32_t sUU = tc::smem_u32(UU);
-            if (!tc::mbar_wait(bar_ld(c), (ph_load >> par) & 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
-            ph_load ^= 1u << par;
+            if (!zero_u) {
+                if (!tc::mbar_wait(bar_ld(c), (ph_load >> par) & 1u)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
+                ph_load ^= 1u << par;
+            }
 
             // ---- U = w * v (Qt, Kt and gC come with the WY image): 4 row chunks of 8 values per thread
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 4 && !zero_u; ++e) {
                 const int idx = tid + NT * e, row = idx >> 4, g = idx & 15;
                 float vv[8], ww[8];
                 tc::ld_row8(UU, C, row, g, vv);
@@ -706,21 +777,24 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             // ---- M3: Delta^T := U^T T^T ;  M4: Delta^T -= S^T Wm^T  (commit) ;  M5: O = Qt S
             if (tid == 0) {
                 tc::tc_fence_after();
+                if (!zero_u) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M3, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tmem + TM_D, tc::desc_mn(sUU, C, 0, kk), tc::desc_k(sTT, C, 0, kk), ID_M3, kk > 0);
+                }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWM, C, 0, kk), ID_M4, 1);
+                    tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sWM, C, 0, kk), ID_M4,
+                                 (zero_u && kk == 0) ? 0u : 1u);
                 tc::mma_commit(bar_mma);
                 if (want_o) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         tc::mma_bf16(tm_o, tc::desc_k(sQQ, C, 0, kk), tc::desc_k(sST, D, 0, kk), ID_M56, kk > 0);
                 }
-                if (c + 1 < nc) wait_wy(head, c + 1);   // overlaps the MMAs
+                if (c + 1 < c1) wait_wy(head, c + 1);   // overlaps the MMAs
             }
-            if (want_o && c > 0) store_o(c - 1);      // previous chunk's output, in the MMAs' shadow
+            if (want_o && c > c0) store_o(c - 1);     // previous chunk's output, in the MMAs' shadow
             if (khm) {   // S^T := S^T Diag(gC) on the fp32 state, in the MMAs' shadow (M3-M5 read its bf16 copy); M7
                          // then adds Delta^T Kh
                 float v[32];
@@ -736,11 +810,11 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             }
             wait_mma();
             // this chunk's v (read by M3) and w buffers are free: chunk c + 2's tiles go there
-            if (c + 2 < nc) issue_loads(c + 2);
+            if (!zero_u && c + 2 < c1) issue_loads(c + 2);
             tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
             sync_for_mma();
-            if (p.deltas && tid == 0) {   // Delta^T of this chunk for the backward
-                tc::bulk_store(p.deltas + (head * nc + c) * TC_DELTA_BYTES, DT, (uint32_t)TC_DELTA_BYTES);
+            if (deltas && tid == 0) {   // Delta^T of this chunk for the backward
+                tc::bulk_store(deltas + (head * nc + c) * TC_DELTA_BYTES, DT, (uint32_t)TC_DELTA_BYTES);
                 tc::bulk_commit();
             }
 
@@ -758,9 +832,9 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             wait_mma();
             // S'^T = Z^T Diag(gC) (unless already scaled), and a bf16 copy of the new state for the next chunk
             // (the bulk stores of the previous state image and of this chunk's Delta^T must have read their tiles)
-            if (p.states && tid == 0) tc::bulk_wait_read();
+            if (states && tid == 0) tc::bulk_wait_read();
             __syncthreads();   // also orders thread 0's flag acquire before the image copy
-            if (c + 1 < nc) copy_wy(head, c + 1);
+            if (c + 1 < c1) copy_wy(head, c + 1);
             {
                 const int j = jrow;
                 float v[32];
@@ -780,20 +854,20 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             }
             sync_for_mma();
             tc::tc_fence_after();
-            if (p.states && tid == 0 && c + 1 < nc) {
-                tc::bulk_store(p.states + (head * nc + c + 1) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
+            if (states && tid == 0 && c + 1 < c1) {
+                tc::bulk_store(states + (head * nc + c + 1) * TC_STATE_BYTES, STt, (uint32_t)TC_STATE_BYTES);
                 tc::bulk_commit();
             }
             if (*abort_flag) {   // let the next chunk's loads land before leaving
-                if (tid == 0 && c + 1 < nc) (void)tc::mbar_wait(bar_ld(c + 1), (ph_load >> ((c + 1) & 1)) & 1u);
-                if (tid == 0 && c + 2 < nc) (void)tc::mbar_wait(bar_ld(c + 2), ((ph_load >> (c & 1)) & 1u));
+                if (!zero_u && tid == 0 && c + 1 < c1) (void)tc::mbar_wait(bar_ld(c + 1), (ph_load >> ((c + 1) & 1)) & 1u);
+                if (!zero_u && tid == 0 && c + 2 < c1) (void)tc::mbar_wait(bar_ld(c + 2), ((ph_load >> (c & 1)) & 1u));
                 break;
             }
         }
-        if (want_o && c == nc) store_o(nc - 1);
+        if (want_o && c == c1) store_o(c1 - 1);
 
-        // final state (fp32): ST[i][j] from S^T (lane j)
-        if (p.ST) {
+        // final state (fp32): fin[i][j] from S^T (lane j)
+        if (task.fin) {
             const int j = jrow;
             float v[32];
 #pragma unroll 1
@@ -801,11 +875,11 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 tc::tmem_ld32(lane_base + TM_S + i0, v);
                 tc::tmem_wait_ld(v);
 #pragma unroll
-                for (int u = 0; u < 32; ++u) p.ST[(head * D + i0 + u) * D + j] = v[u];
+                for (int u = 0; u < 32; ++u) task.fin[(i0 + u) * D + j] = v[u];
             }
         }
         tc::cp_async_wait_all();
-        if (p.states && tid == 0) tc::bulk_wait_all();
+        if (states && tid == 0) tc::bulk_wait_all();
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
@@ -854,7 +928,60 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     }
 }
 
+// Segment start states S_2 .. S_{R-1} from S_1 and the segment maps, S_{s+1} = M_s S_s + N_s, in fp32. The value
+// columns of a state never mix, so CTA (head, block of 16 columns) runs the whole prefix for its columns; thread
+// (row i = tid / 2, 8 columns) keeps its sums in registers.
+__global__ void __launch_bounds__(256) split_prefix_kernel(float* sbuf, int R) {
+    __shared__ float Sc[D][16];
+    const int head = blockIdx.x / (D / 16), j0 = (blockIdx.x % (D / 16)) * 16;
+    const int tid = threadIdx.x, i = tid >> 1, jh = (tid & 1) * 8;
+    float* base = sbuf + (size_t)head * SPLIT_MATS_PER_HEAD * D * D;
+    auto mat = [&](int kind, int s) { return base + (size_t)((kind == 0 ? 0 : (kind == 1 ? R - 1 : 2 * R - 3)) + s - 1) * D * D; };
+    const float* S1 = mat(0, 1);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) Sc[i][jh + e] = S1[i * D + j0 + jh + e];
+    for (int s = 1; s <= R - 2; ++s) {
+        __syncthreads();
+        const float* N = mat(1, s);
+        const float* M = mat(2, s);
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = N[i * D + j0 + jh + e];
+#pragma unroll 4
+        for (int l = 0; l < D; l += 4) {
+            const float4 m = *reinterpret_cast<const float4*>(M + i * D + l);
+            const float mv[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] += mv[u] * Sc[l + u][jh + e];
+        }
+        __syncthreads();
+        float* Sn = mat(0, s + 1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            Sc[i][jh + e] = acc[e];
+            Sn[i * D + j0 + jh + e] = acc[e];
+        }
+    }
+}
+
+// Number of segments a head's chunks are cut into (0: none). Only when the heads leave most CTA slots idle
+// and every segment keeps a few dozen chunks; bounded by the workspace reserved for the maps.
+int split_segments(int BH, int nc, int slots, bool have_buf) {
+    if (!have_buf || split_disabled() || BH <= 0 || BH > TC_SPLIT_MAX_BH) return 0;
+    int R = (slots / BH - 1) / 2 + 2;   // phase 1 runs BH (1 + 2 (R - 2)) chains at once
+    if (R > SPLIT_R_MAX) R = SPLIT_R_MAX;
+    if (R > nc / TC_SPLIT_MIN_CHUNKS_PER_SEG) R = nc / TC_SPLIT_MIN_CHUNKS_PER_SEG;
+    return R < 4 ? 0 : R;
+}
+
 }  // namespace
+
+size_t chunk_fwd_split_bytes(int BH, int nc) {
+    if (BH > TC_SPLIT_MAX_BH || nc < TC_SPLIT_MIN_CHUNKS_PER_SEG * 4) return 0;
+    return (size_t)BH * SPLIT_MATS_PER_HEAD * TC_D * TC_D * sizeof(float);
+}
 
 cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
@@ -879,6 +1006,40 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     p.S0 = a.S0; p.o = static_cast<__nv_bfloat16*>(a.o); p.ST = a.ST;
     p.states = a.states; p.deltas = a.deltas; p.wyimg = a.wy; p.flags = a.flags;
     if ((e = cudaMemsetAsync(a.flags, 0, (size_t)units * sizeof(unsigned int), s)) != cudaSuccess) return e;
+
+    const int R = split_segments(BH, nc, slots, a.sbuf != nullptr);
+    if (R) {   // producers, then the first segments and the segment maps, the prefix, then the other segments
+        p.split_R = R;
+        p.sbuf = a.sbuf;
+        FwdParams pp = p;
+        pp.ncons = 0;
+        pp.nprod = units < slots ? units : slots;
+        {
+            TraceScope trace(K_CHUNK_FWD, s);
+            if (!test_skip_producers()) {
+                chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+        }
+        for (int phase = 1; phase <= 3; phase += 2) {
+            FwdParams pc = p;
+            pc.phase = phase;
+            pc.nprod = 0;
+            const int ntasks = phase == 1 ? BH * (1 + 2 * (R - 2)) : BH * (R - 1);
+            pc.ncons = ntasks < slots ? ntasks : slots;
+            {
+                TraceScope trace(K_CHUNK_FWD, s);
+                chunk_fwd_kernel<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+            if (phase == 1) {
+                TraceScope trace(K_SPLIT_PREFIX, s);
+                split_prefix_kernel<<<BH * (D / 16), 256, 0, s>>>(a.sbuf, R);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+        }
+        return cudaSuccess;
+    }
 
     TraceScope trace(K_CHUNK_FWD, s);
     // Heads share the launch with the producers while the producers keep pace: per chunk step the

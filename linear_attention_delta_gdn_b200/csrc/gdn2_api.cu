@@ -71,7 +71,11 @@ gdn2_status check_dims(int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtyp
 //   [WY images: units x TC_WY_BYTES][ready flags]
 //   then, for the backward, [dZ^T: units x TC_STATE_BYTES][dDelta^T: units x TC_DELTA_BYTES][flags].
 size_t tc_units(const Dims& d) { return (size_t)d.B * d.H * (size_t)d.nchunks(); }
-size_t tc_wy_bytes(const Dims& d) { return tc_units(d) * TC_WY_BYTES + align256(tc_units(d) * sizeof(unsigned int)); }
+size_t tc_split_bytes(const Dims& d) { return align256(chunk_fwd_split_bytes(d.B * d.H, d.nchunks())); }
+// WY images, ready flags, then the segment states and maps of a long sequence (if it can be cut)
+size_t tc_wy_bytes(const Dims& d) {
+    return tc_units(d) * TC_WY_BYTES + align256(tc_units(d) * sizeof(unsigned int)) + tc_split_bytes(d);
+}
 
 // Forward-saved region: chunk-start states (and, on the tensor-core path, Delta^T, the WY images and flags).
 size_t states_bytes(const Dims& d, gdn2_dtype dt) {
@@ -83,6 +87,9 @@ size_t tc_delta_offset(const Dims& d) { return tc_units(d) * TC_STATE_BYTES; }
 size_t tc_tp_offset(const Dims& d) { return tc_units(d) * (TC_STATE_BYTES + TC_DELTA_BYTES); }
 size_t tc_flags_offset(const Dims& d, bool with_states) {
     return (with_states ? tc_tp_offset(d) : 0) + tc_units(d) * TC_WY_BYTES;
+}
+size_t tc_split_offset(const Dims& d, bool with_states) {
+    return tc_flags_offset(d, with_states) + align256(tc_units(d) * sizeof(unsigned int));
 }
 
 size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
@@ -122,6 +129,7 @@ static bool env_flag(const char* name) {
 }
 bool cooperative_disabled() { return env_flag("GDN2_NO_COOPERATIVE"); }
 bool test_skip_producers() { return env_flag("GDN2_TEST_SKIP_PRODUCERS"); }
+bool split_disabled() { return env_flag("GDN2_NO_SPLIT"); }
 }  // namespace gdn2
 
 extern "C" {
@@ -205,6 +213,7 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
         a.deltas = keep ? wsb + tc_delta_offset(d) : nullptr;
         a.wy = wsb + (keep ? tc_tp_offset(d) : 0);
         a.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, keep));
+        a.sbuf = tc_split_bytes(d) ? reinterpret_cast<float*>(wsb + tc_split_offset(d, keep)) : nullptr;
         return cuda_status(chunk_fwd_launch(a, s), "gdn2_fwd (tensor-core path)");
     }
     RecurrentArgs a{};
@@ -250,6 +259,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
             f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.deltas = wsb + tc_delta_offset(d);
             f.wy = wsb + tc_tp_offset(d);
             f.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, true));
+            f.sbuf = tc_split_bytes(d) ? reinterpret_cast<float*>(wsb + tc_split_offset(d, true)) : nullptr;
             gdn2_status e = cuda_status(chunk_fwd_launch(f, s), "gdn2_bwd state recompute");
             if (e != GDN2_OK) return e;
         }

@@ -50,8 +50,16 @@ struct ChunkFwdArgs {
     unsigned char* deltas; // [B,H,NC] Delta^T images (with states), or null
     unsigned char* wy;     // [B,H,NC] WY images (T | P | Wm), always written
     unsigned int* flags;   // [B,H,NC] ready flags (scratch)
+    float* sbuf;           // segment states and maps of long sequences (chunk_fwd_split_bytes), or null
 };
 cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s);
+// Long sequences with few heads: a head's chunks may be cut into segments that run on separate CTAs (segment
+// maps, a prefix over them, then the segments again from their start states). Workspace for that, 0 if the
+// problem never qualifies.
+constexpr int TC_SPLIT_MAX_BH = 32;
+constexpr int TC_SPLIT_MIN_CHUNKS_PER_SEG = 16;
+size_t chunk_fwd_split_bytes(int BH, int nc);
+bool split_disabled();   // environment variable GDN2_NO_SPLIT set: keep every head on one chain
 
 struct ChunkBwdArgs {
     Dims d;
@@ -70,7 +78,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 
 // Kernels of the library, for gdn2_trace_read().
 enum KernelId { K_CHUNK_FWD = 0, K_CHUNK_BWD, K_REC_FWD, K_REC_BWD, K_DECODE, K_GATE_EXPAND, K_GATE_REDUCE,
-                K_VARLEN_COPY, KERNEL_COUNT };
+                K_VARLEN_COPY, K_SPLIT_PREFIX, KERNEL_COUNT };
 
 // Brackets one kernel launch with CUDA events on its stream while tracing is on.
 class TraceScope {

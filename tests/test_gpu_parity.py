@@ -317,3 +317,32 @@ def test_autograd_matches_direct():
     for n, gn in zip(NAMES, GRADS):
         assert rel_l2(to_f64(leaves[n].grad), to_f64(g[gn])) < 1e-6, n
     assert rel_l2(to_f64(S0.grad), to_f64(g["dS0"])) < 1e-6
+
+
+@pytest.mark.parametrize("B,T,H,S0", [(1, 8192, 4, True), (1, 6000, 2, False), (2, 4100, 3, True)])
+def test_long_sequence_segments(oracle_mod, B, T, H, S0):
+    """With few heads and long sequences the forward cuts each head's chunks into segments (segment maps, a prefix
+    over them, the segments again from their start states). Same results as one chain per head (GDN2_NO_SPLIT)
+    and as the oracle, for the output, the final state and, through the backward's recompute and through the
+    saved states, the gradients."""
+    import os
+    x = make_inputs(B, T, H, 128, 128, seed=1700 + T, dtype="bf16", with_do=True, with_S0=S0)
+    d = dev(x)
+    binding.trace_read()
+    binding.trace_enable(True)
+    try:
+        o, ST = binding.gdn2_fwd(*(d[n] for n in NAMES), d.get("S0"))
+    finally:
+        binding.trace_enable(False)
+    assert "split_prefix_kernel" in binding.trace_read()      # the segmented form ran
+    os.environ["GDN2_NO_SPLIT"] = "1"
+    try:
+        o1, ST1 = binding.gdn2_fwd(*(d[n] for n in NAMES), d.get("S0"))
+    finally:
+        del os.environ["GDN2_NO_SPLIT"]
+    torch.cuda.synchronize()
+    assert rel_l2(to_f64(o), to_f64(o1)) < 1e-2 and rel_l2(to_f64(ST), to_f64(ST1)) < 1e-2
+    check_fwd(oracle_mod, x, 64, "bf16")
+    check_bwd(oracle_mod, x, 64, "bf16", with_dST=True)
+    check_bwd(oracle_mod, x, 64, "bf16", with_dST=True, saved=True)
+    assert binding.gdn2_device_status() == binding.GDN2_OK, binding.last_error()
