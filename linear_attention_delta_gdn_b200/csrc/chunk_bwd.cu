@@ -234,7 +234,101 @@ struct BwdParams {
     unsigned char* ddeltas;          // dDelta^T images
     unsigned int* flags;             // [BH, nc] dS' ready flags (zero at launch)
     unsigned int* counter;           // [0]: next gradient unit, [1]: abort word (zero at launch)
+    int split_R;                     // > 0: the reverse pass of a head is cut into split_R segments
+    int phase;                       // with split_R: 1 (last segment, segment maps) or 3 (the other segments)
+    float* sbuf;                     // with split_R: per head, segment end gradients, then the maps B and A
 };
+
+// ---- reverse-pass tasks
+// Without a split, task t walks every chunk of head t backwards from dST (zero if none). A long sequence with
+// few heads is cut into R segments as in the forward; with E_s the gradient at the end of segment s (E_{R-1} =
+// dST), walking a segment backwards is an affine map E_{s-1} = A_s E_s + B_s, where B_s is the result from a
+// zero end gradient and A_s (d_k x d_k) the one from an identity end gradient without output gradients (dO =
+// 0). Phase 1 walks the last segment for real (its start gradient is E_{R-2}) and, for s = 1 .. R-2, B_s and
+// A_s as separate tasks; the forward's prefix kernel then forms E_{R-3} .. E_0 (its slot k holds E_{R-1-k},
+// its maps those of segment R-1-k); phase 3 walks segments 0 .. R-2 for real, next to the gradient workers.
+struct RevTask {
+    int head, c_hi, c_lo;    // chunks c_hi down to c_lo
+    const float* start;      // end gradient [D][D] (row = key), or null: zero, or identity when ident
+    bool ident, zero_do;     // A_s: identity start, no output gradient
+    bool real;               // the real chain: dZ and dDelta images, ready flags
+    float* fin;              // where the gradient at chunk c_lo's start goes, or null
+};
+constexpr int SPLIT_R_MAX = 8;
+constexpr size_t SPLIT_MATS_PER_HEAD = (SPLIT_R_MAX - 1) + 2 * (SPLIT_R_MAX - 2);
+__host__ __device__ inline int seg_begin(int s, int nc, int R) { return (int)((long long)s * nc / R); }
+__device__ __forceinline__ float* rsplit_mat(const BwdParams& p, int head, int kind, int k) {   // 0: E, 1: B, 2: A
+    const int R = p.split_R;
+    const int idx = kind == 0 ? k - 1 : (kind == 1 ? (R - 1) + (k - 1) : (R - 1) + (R - 2) + (k - 1));
+    return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
+}
+__device__ __forceinline__ int rev_task_count(const BwdParams& p) {
+    if (!p.split_R) return p.BH;
+    return p.phase == 1 ? p.BH * (1 + 2 * (p.split_R - 2)) : p.BH * (p.split_R - 1);
+}
+__device__ RevTask rev_task_at(const BwdParams& p, int t) {
+    RevTask k{};
+    k.head = t % p.BH;
+    const size_t hd = (size_t)k.head * D * D;
+    if (!p.split_R) {
+        k.c_hi = p.nc - 1; k.c_lo = 0; k.start = p.dST ? p.dST + hd : nullptr; k.real = true;
+        k.fin = p.dS0 ? p.dS0 + hd : nullptr;
+        return k;
+    }
+    const int R = p.split_R, j = t / p.BH;
+    auto seg_lo = [&](int s2) { return seg_begin(s2, p.nc, R); };
+    auto seg_hi = [&](int s2) { return (s2 == R - 1 ? p.nc : seg_begin(s2 + 1, p.nc, R)) - 1; };
+    if (p.phase == 1) {
+        if (j == 0) {   // the last segment, for real, from dST; its start gradient is E_{R-2} = slot 1
+            k.c_hi = seg_hi(R - 1); k.c_lo = seg_lo(R - 1); k.start = p.dST ? p.dST + hd : nullptr; k.real = true;
+            k.fin = rsplit_mat(p, k.head, 0, 1);
+        } else if (j <= R - 2) {   // B of segment s2 = R-1-j into slot j
+            const int s2 = R - 1 - j;
+            k.c_hi = seg_hi(s2); k.c_lo = seg_lo(s2); k.fin = rsplit_mat(p, k.head, 1, j);
+        } else {   // A of segment s2 into slot j - (R-2)
+            const int kk = j - (R - 2), s2 = R - 1 - kk;
+            k.c_hi = seg_hi(s2); k.c_lo = seg_lo(s2); k.ident = true; k.zero_do = true;
+            k.fin = rsplit_mat(p, k.head, 2, kk);
+        }
+    } else {   // segment s2 = j (0 .. R-2) for real from E_{s2} = slot R-1-s2
+        const int s2 = j;
+        k.c_hi = seg_hi(s2); k.c_lo = seg_lo(s2); k.start = rsplit_mat(p, k.head, 0, R - 1 - s2); k.real = true;
+        k.fin = (s2 == 0 && p.dS0) ? p.dS0 + hd : nullptr;
+    }
+    return k;
+}
+// Gradient units in the order the reverse pass produces them. Without a split: chunks from the last, heads
+// inside. With a split (phase 3): the last segment's units first (ready from phase 1), then the other
+// segments' units interleaved by position from their ends. Returns false for an index that names no unit
+// (segments of unequal length).
+__device__ __forceinline__ int unit_slots(const BwdParams& p) {
+    if (!p.split_R) return p.BH * p.nc;
+    const int R = p.split_R, last = p.nc - seg_begin(R - 1, p.nc, R);
+    int lmax = 0;
+    for (int s2 = 0; s2 < R - 1; ++s2) {
+        const int l = seg_begin(s2 + 1, p.nc, R) - seg_begin(s2, p.nc, R);
+        lmax = l > lmax ? l : lmax;
+    }
+    return p.BH * last + p.BH * (R - 1) * lmax;
+}
+__device__ __forceinline__ bool unit_at(const BwdParams& p, int u, int* head, int* c) {
+    if (!p.split_R) {
+        *c = p.nc - 1 - u / p.BH;
+        *head = u % p.BH;
+        return true;
+    }
+    const int R = p.split_R, lo_last = seg_begin(R - 1, p.nc, R), nlast = p.BH * (p.nc - lo_last);
+    if (u < nlast) {
+        *c = p.nc - 1 - u / p.BH;
+        *head = u % p.BH;
+        return true;
+    }
+    const int v = u - nlast, per = p.BH * (R - 1), jpos = v / per, rem = v % per, s2 = rem / p.BH;
+    *head = rem % p.BH;
+    const int lo = seg_begin(s2, p.nc, R), hi = seg_begin(s2 + 1, p.nc, R) - 1;
+    *c = hi - jpos;
+    return *c >= lo;
+}
 // mbarrier parities carried across the units a CTA works on
 struct Phases {
     uint32_t load = 0, mma = 0, k = 0, b = 0, pre = 0;
@@ -288,8 +382,8 @@ constexpr uint32_t LOAD_BYTES = 4 * 64 * 128 * 2 + TILE_C + 512 + 16;   // Qt, K
 }  // namespace rs
 static_assert(rs::OFF_MASK + 32 <= OFF_BARS, "reverse-pass layout lies below the barrier block");
 
-__device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi,
-                            Phases& ph) {
+__device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem,
+                            const RevTask& task, Phases& ph) {
     using namespace rs;
     unsigned char* STt = sm + OFF_ST;
     unsigned char* DT = sm + OFF_DT;
@@ -305,6 +399,8 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     auto MASK = [&](int c) { return sm + OFF_MASK + (c & 1) * 16; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int headi = task.head, c_hi = task.c_hi, c_lo = task.c_lo;
+    const bool zero_do = task.zero_do, real = task.real;
     const int h = headi % p.H, b = headi / p.H;
     const size_t head = (size_t)headi;
     const int nc = p.nc;
@@ -313,15 +409,16 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
 
     // chunk c's tiles arrive on one barrier phase, issued in three groups as their buffers free up
     // dout, Qt, Kt, Wm, gC, mask (buffers of this parity are free): issued by lane 0 of warps 0-5 at once
+    // (a task without output gradients, zero_do, needs neither dout, nor Qt and P)
     auto issue_first = [&](int c) {
         if (lane != 0 || warp > 5) return;
         const unsigned char* img = p.tp + (head * nc + c) * TC_WY_BYTES;
         switch (warp) {
         case 0:
-            tc::mbar_arrive_expect_tx(bar_load, LOAD_BYTES);
-            tma_tile(DO(c), C, 0, &m.dout, b, h, c * C, bar_load);
+            tc::mbar_arrive_expect_tx(bar_load, zero_do ? LOAD_BYTES - 2 * 64 * 128 * 2 - TILE_C : LOAD_BYTES);
+            if (!zero_do) tma_tile(DO(c), C, 0, &m.dout, b, h, c * C, bar_load);
             break;
-        case 1: tc::bulk_load(QQ(c), img + TC_WY_QT, 64 * 128 * 2, bar_load); break;
+        case 1: if (!zero_do) tc::bulk_load(QQ(c), img + TC_WY_QT, 64 * 128 * 2, bar_load); break;
         case 2: tc::bulk_load(KT(c), img + TC_WY_KT, 64 * 128 * 2, bar_load); break;
         case 3: tc::bulk_load(WW(c), img + TC_WY_WM, 64 * 128 * 2, bar_load); break;
         case 4: tc::bulk_load(GC(c), img + TC_WY_GC, 512, bar_load); break;
@@ -331,16 +428,17 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     auto issue_p = [&](int c) {   // after the MMAs that read P
         tc::bulk_load(PP, p.tp + (head * nc + c) * TC_WY_BYTES + TILE_C, TILE_C, bar_load);
     };
-    issue_first(nc - 1);
-    if (tid == 0) issue_p(nc - 1);
+    issue_first(c_hi);
+    if (tid == 0 && !zero_do) issue_p(c_hi);
 
-    {   // dS_{NC}^T = dST^T (or zero): lane j holds column j of dST
+    {   // the gradient at the end of the range: lane j holds column j of the start matrix (dST, zero or I)
         const int j = jrow;
         float v[32];
 #pragma unroll 1
         for (int i0 = cpart; i0 < cpart + 32; i0 += 32) {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] = p.dST ? p.dST[(head * D + i0 + u) * D + j] : 0.f;
+            for (int u = 0; u < 32; ++u)
+                v[u] = task.start ? task.start[(i0 + u) * D + j] : (task.ident && i0 + u == j ? 1.f : 0.f);
             tc::tmem_st32(lane_base + TM_S + i0, v);
         }
         tc::tmem_wait_st();
@@ -367,13 +465,13 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
     };
 
     int unreleased = -1;   // chunk whose dS' image is written but whose flag is not yet set
-    for (int c = nc - 1; c >= 0; --c) {
+    for (int c = c_hi; c >= c_lo; --c) {
         const uint32_t sQQ = tc::smem_u32(QQ(c)), sKT = tc::smem_u32(KT(c)), sDO = tc::smem_u32(DO(c)),
                        sWW = tc::smem_u32(WW(c));
         if (!tc::mbar_wait(bar_load, ph.load)) { atomicExch(abort_flag, 1); atomicOr(&g_bwd_error, 2u); }
         ph.load ^= 1;
         // the other parity's buffers were last read by chunk c + 1, whose MMAs are complete
-        if (c > 0) issue_first(c - 1);
+        if (c > c_lo) issue_first(c - 1);
 
         const float* sGC = GC(c);   // Qt, Kt, gC and the mask came with the forward's WY image
         const uint4 msk = *reinterpret_cast<const uint4*>(MASK(c));
@@ -412,29 +510,32 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_bf16(tmem + TM_D, tc::desc_k(sST, D, 0, kk), tc::desc_k(sKT, C, 0, kk), ID_N1a, kk > 0);
+            if (!zero_do) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_D, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), ID_N1b, 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_D, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sPP, C, 0, kk), ID_N1b, 1);
+            }
             tc::mma_commit(bar_mma);
+            if (!zero_do) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQQ, C, 0, kk), ID_N2a, 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_S, tc::desc_mn(sDO, C, 0, kk), tc::desc_mn(sQQ, C, 0, kk), ID_N2a, 1);
+            }
         }
         // the previous chunk's dZ image stores have drained: publish it while the MMAs run
-        if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
-        // this chunk's dZ^T (dS'^T) image for the gradient units (plain stores, published one chunk later)
-        {
+        if (real && tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
+        if (real) {   // this chunk's dZ^T (dS'^T) image for the gradient units (plain stores, published one chunk later)
             uint4* dst = reinterpret_cast<uint4*>(p.dstates + (head * nc + c) * TC_STATE_BYTES);
             const uint4* src = reinterpret_cast<const uint4*>(STt);
 #pragma unroll
             for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i) dst[tid + BT * i] = src[tid + BT * i];
+            unreleased = c;
         }
-        unreleased = c;
         wait_mma();
-        if (tid == 0 && c > 0) issue_p(c - 1);
+        if (tid == 0 && c > c_lo && !zero_do) issue_p(c - 1);
         tmem_rows_to_tile<64>(lane_base + TM_D, DT, warp, lane);   // dDelta^T rows
         sync_for_mma();
-        {   // dDelta^T image for the gradient units (published with the dZ^T image)
+        if (real) {   // dDelta^T image for the gradient units (published with the dZ^T image)
             uint4* dst = reinterpret_cast<uint4*>(p.ddeltas + (head * nc + c) * TC_DELTA_BYTES);
             const uint4* src = reinterpret_cast<const uint4*>(DT);
 #pragma unroll
@@ -456,14 +557,14 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
         if (*abort_flag) {   // let the next chunk's loads land before leaving
             if (tid == 0) {
                 atomicExch(p.counter + 1, 1u);   // gradient units of this head will never be ready
-                if (c > 0) (void)tc::mbar_wait(bar_load, ph.load);
+                if (c > c_lo) (void)tc::mbar_wait(bar_load, ph.load);
             }
             break;
         }
     }
     if (tid == 32 && unreleased >= 0 && !*abort_flag) tc::flag_release(p.flags + head * nc + unreleased, 1u);
 
-    if (p.dS0) {   // dS0[i][j] from dS^T (lane j)
+    if (task.fin) {   // the gradient at the start of the range, fin[i][j] from dS^T (lane j): dS0 or a segment's
         const int j = jrow;
         float v[32];
 #pragma unroll 1
@@ -471,7 +572,7 @@ __device__ void run_reverse(const BwdMaps& m, const BwdParams& p, unsigned char*
             tc::tmem_ld32(lane_base + TM_S + i0, v);
             tc::tmem_wait_ld(v);
 #pragma unroll
-            for (int u = 0; u < 32; ++u) p.dS0[(head * D + i0 + u) * D + j] = v[u];
+            for (int u = 0; u < 32; ++u) task.fin[(i0 + u) * D + j] = v[u];
         }
     }
     tc::tc_fence_before();
@@ -531,7 +632,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T, H = p.H, nc = p.nc;
-    const int units = p.BH * nc;
+    const int units = unit_slots(p);
     const int h = headi % H, b = headi / H;
     const size_t head = (size_t)headi;
     const int t0 = c * C;
@@ -756,10 +857,9 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     if (warp == 9 && lane == 0) {   // while the G MMAs run: the CTA's next unit, published at the next barrier
         if (*reinterpret_cast<volatile unsigned int*>(p.counter + 1)) next_unit = units;   // a CTA gave up
         int ready = 0;
-        if (next_unit < units) {   // acquire: usually the flag has been set for long
-            const int nc_ = nc - 1 - next_unit / p.BH, nh = next_unit % p.BH;
+        int nh = 0, nc_ = 0;
+        if (next_unit < units && unit_at(p, next_unit, &nh, &nc_))   // acquire: usually set long ago
             ready = tc::ld_acquire(p.flags + (size_t)nh * nc + nc_) == 1u;
-        }
         nxt->unit = next_unit;
         nxt->prefetched = ready;
     }
@@ -850,16 +950,16 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         }
         tc::bulk_commit();
     }
+    int nxt_head = 0, nxt_c = 0;
+    if (nxt->prefetched) unit_at(p, nxt->unit, &nxt_head, &nxt_c);
     if (tid == 0 && nxt->prefetched) {   // S^T and T of the next unit into the tiles this unit has finished with
-        const int nu_ = nxt->unit;
-        const size_t nu = (size_t)(nu_ % p.BH) * nc + (nc - 1 - nu_ / p.BH);
+        const size_t nu = (size_t)nxt_head * nc + nxt_c;
         tc::mbar_arrive_expect_tx(bar_pre, LOAD_PRE);
         tc::bulk_load(STt, p.states + nu * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_pre);
         tc::bulk_load(TT, p.tp + nu * TC_WY_BYTES, TILE_C, bar_pre);
     }
     if (nxt->prefetched) {
-        const int nu_ = nxt->unit;
-        const size_t nu = (size_t)(nu_ % p.BH) * nc + (nc - 1 - nu_ / p.BH);
+        const size_t nu = (size_t)nxt_head * nc + nxt_c;
         const unsigned char* src = p.dstates + nu * TC_STATE_BYTES;
 #pragma unroll
         for (int i = 0; i < (int)(TC_STATE_BYTES / 16 / BT); ++i)
@@ -921,9 +1021,12 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_base_ptr;
     Phases ph;
     const bool reverse = (int)blockIdx.x < p.nrev;
-    if (reverse) run_reverse(maps, p, sm, tmem, blockIdx.x, ph);
+    if (reverse) {   // the CTA's reverse-pass tasks (one each in a launch with gradient workers)
+        const int ntasks = rev_task_count(p);
+        for (int t = blockIdx.x; t < ntasks && !*abort_flag; t += p.nrev) run_reverse(maps, p, sm, tmem, rev_task_at(p, t), ph);
+    }
     if (p.grad && (!reverse || p.join) && !*abort_flag) {
-        const int units = p.BH * p.nc;
+        const int units = unit_slots(p);
         if (tid == 0) {   // stop taking units once any CTA of the launch has given up
             nxt->unit = *reinterpret_cast<volatile unsigned int*>(p.counter + 1) ? units : (int)atomicAdd(p.counter, 1u);
             nxt->prefetched = 0;
@@ -932,8 +1035,19 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
         int u = nxt->unit;
         bool pre = false;
         while (u < units) {
-            // units in the order the reverse pass produces them: chunks from the last, heads inside
-            const int c = p.nc - 1 - u / p.BH, headi = u % p.BH;
+            // units in the order the reverse pass produces them (unit_at)
+            int c = 0, headi = 0;
+            if (!unit_at(p, u, &headi, &c)) {   // an index that names no unit: take the next one
+                if (tid == 0) {
+                    nxt->unit = *reinterpret_cast<volatile unsigned int*>(p.counter + 1) ? units : (int)atomicAdd(p.counter, 1u);
+                    nxt->prefetched = 0;
+                }
+                __syncthreads();
+                u = nxt->unit;
+                pre = false;
+                __syncthreads();
+                continue;
+            }
             if (!grad_unit(maps, p, sm, tmem, headi, c, ph, pre, nxt)) {
                 // a bounded wait gave up: let a prefetch in flight land before leaving
                 if (tid == 0 && nxt->prefetched) (void)tc::mbar_wait(reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48), ph.pre);
@@ -979,6 +1093,41 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     p.states = a.states; p.deltas = a.deltas; p.tp = a.tp; p.dstates = a.dstates; p.ddeltas = a.ddeltas;
     p.flags = a.flags; p.counter = a.flags + units;
     if ((e = cudaMemsetAsync(a.flags, 0, ((size_t)units + 2) * sizeof(unsigned int), s)) != cudaSuccess) return e;
+
+    const int R = split_segments_for(BH, nc, slots, a.sbuf != nullptr);
+    if (R) {   // the last segments and the segment maps, the prefix, then the other segments with the gradients
+        p.split_R = R;
+        p.sbuf = a.sbuf;
+        BwdParams p1 = p;
+        p1.phase = 1; p1.grad = 0; p1.join = 0;
+        const int n1 = BH * (1 + 2 * (R - 2));
+        p1.nrev = n1 < slots ? n1 : slots;
+        {
+            TraceScope trace(K_CHUNK_BWD, s);
+            chunk_bwd_kernel<<<p1.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, p1);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if ((e = split_prefix_launch(a.sbuf, R, BH, s)) != cudaSuccess) return e;
+        BwdParams p3 = p;
+        p3.phase = 3;
+        const int n3 = BH * (R - 1);
+        TraceScope trace(K_CHUNK_BWD, s);
+        if (coop && !cooperative_disabled() && n3 < slots) {
+            p3.nrev = n3; p3.join = 1; p3.grad = 1;
+            void* args[2] = {&maps, &p3};
+            e = cudaLaunchCooperativeKernel((const void*)chunk_bwd_kernel, dim3(slots), dim3(BT), args, SMEM_BYTES_ALL, s);
+            if (e == cudaSuccess) return cudaSuccess;
+            (void)cudaGetLastError();
+        }
+        BwdParams pr = p3;
+        pr.nrev = n3 < slots ? n3 : slots; pr.join = 0; pr.grad = 0;
+        chunk_bwd_kernel<<<pr.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        BwdParams pg = p3;
+        pg.nrev = 0; pg.join = 0; pg.grad = 1;
+        chunk_bwd_kernel<<<units < slots ? units : slots, BT, SMEM_BYTES_ALL, s>>>(maps, pg);
+        return cudaGetLastError();
+    }
 
     TraceScope trace(K_CHUNK_BWD, s);
     // Every head's reverse pass plus at least one gradient worker resident at once: one launch.

@@ -978,6 +978,14 @@ int split_segments(int BH, int nc, int slots, bool have_buf) {
 
 }  // namespace
 
+cudaError_t split_prefix_launch(float* sbuf, int R, int BH, cudaStream_t s) {
+    TraceScope trace(K_SPLIT_PREFIX, s);
+    split_prefix_kernel<<<BH * (D / 16), 256, 0, s>>>(sbuf, R);
+    return cudaGetLastError();
+}
+
+int split_segments_for(int BH, int nc, int slots, bool have_buf) { return split_segments(BH, nc, slots, have_buf); }
+
 size_t chunk_fwd_split_bytes(int BH, int nc) {
     if (BH > TC_SPLIT_MAX_BH || nc < TC_SPLIT_MIN_CHUNKS_PER_SEG * 4) return 0;
     return (size_t)BH * SPLIT_MATS_PER_HEAD * TC_D * TC_D * sizeof(float);
@@ -1032,11 +1040,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
                 chunk_fwd_kernel<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
-            if (phase == 1) {
-                TraceScope trace(K_SPLIT_PREFIX, s);
-                split_prefix_kernel<<<BH * (D / 16), 256, 0, s>>>(a.sbuf, R);
-                if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            }
+            if (phase == 1 && (e = split_prefix_launch(a.sbuf, R, BH, s)) != cudaSuccess) return e;
         }
         return cudaSuccess;
     }

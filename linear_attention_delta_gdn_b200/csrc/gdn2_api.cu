@@ -274,6 +274,8 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
         a.dstates = extra;
         a.ddeltas = extra + tc_units(d) * TC_STATE_BYTES;
         a.flags = reinterpret_cast<unsigned int*>(extra + tc_units(d) * (TC_STATE_BYTES + TC_DELTA_BYTES));
+        // the forward's segment region (dead once the forward is done) serves the backward's segments
+        a.sbuf = tc_split_bytes(d) ? reinterpret_cast<float*>(wsb + tc_split_offset(d, true)) : nullptr;
         return cuda_status(chunk_bwd_launch(a, s), "gdn2_bwd (tensor-core path)");
     }
 

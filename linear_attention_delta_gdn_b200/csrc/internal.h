@@ -59,6 +59,10 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s);
 constexpr int TC_SPLIT_MAX_BH = 32;
 constexpr int TC_SPLIT_MIN_CHUNKS_PER_SEG = 16;
 size_t chunk_fwd_split_bytes(int BH, int nc);
+// The segment count for a problem (0: no split), and the fp32 prefix over the segment maps, shared by the
+// forward and the backward (whose reverse segments use the same per-head layout of states and maps).
+int split_segments_for(int BH, int nc, int slots, bool have_buf);
+cudaError_t split_prefix_launch(float* sbuf, int R, int BH, cudaStream_t s);
 bool split_disabled();   // environment variable GDN2_NO_SPLIT set: keep every head on one chain
 
 struct ChunkBwdArgs {
@@ -73,6 +77,7 @@ struct ChunkBwdArgs {
     unsigned char* dstates;       // [B,H,NC] images of Diag(gC) dL/dS' per chunk (scratch)
     unsigned char* ddeltas;       // [B,H,NC] dDelta^T images (scratch)
     unsigned int* flags;          // [B,H,NC] ready flags, then work counter and abort word (scratch)
+    float* sbuf;                  // segment gradients and maps of long sequences (chunk_fwd_split_bytes), or null
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 
