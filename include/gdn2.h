@@ -88,7 +88,8 @@ typedef enum gdn2_dtype {
 typedef enum gdn2_op {
     GDN2_OP_FWD = 0,      /* gdn2_fwd with save_states = 0 */
     GDN2_OP_FWD_SAVE = 1, /* gdn2_fwd with save_states = 1 */
-    GDN2_OP_BWD = 2       /* gdn2_bwd (either value of states_saved) */
+    GDN2_OP_BWD = 2,      /* gdn2_bwd (either value of states_saved) */
+    GDN2_OP_MAP = 3       /* gdn2_fwd_map and gdn2_bwd_map */
 } gdn2_op;
 
 /*
@@ -271,6 +272,41 @@ gdn2_status gdn2_bwd_no_alloc(const void* q, const void* k, const void* v, const
 
 /* Size in bytes of the fixed scratch array used by gdn2_bwd_no_alloc. */
 size_t gdn2_no_alloc_scratch_bytes(void);
+
+/*
+ * Affine maps of a sequence piece, for one sequence cut into pieces that run on
+ * several devices (context parallelism). The recurrence is linear in the state
+ * (S_t = (I - k_t (b_t*k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t*v_t)^T, the
+ * state update of the GitHub README's introduction; the abstract's fixed-size
+ * state is what crosses a piece boundary), so a piece maps its start state to its end
+ * state as S_end = M S_start + N, and its backward maps the end gradient to the
+ * start gradient as dS_start = A dS_end + B (A = M^T in exact arithmetic; B is
+ * the start gradient from a zero end gradient). With the maps of the pieces
+ * before it, a device forms its start state (and with those after it, its end
+ * gradient) and then runs gdn2_fwd / gdn2_bwd on its own piece.
+ *   q .. w, dout : one piece [B, T, H, D] dt, as in gdn2_fwd / gdn2_bwd
+ *   M, A         : [B, H, Dk, Dk] float32 out
+ *   N, Bm        : [B, H, Dk, Dv] float32 out
+ * Tensor-core path only (dt = GDN2_BF16, Dk = Dv = 128); other problems return
+ * GDN2_ERR_UNSUPPORTED. T = 0 gives M = A = I and N = Bm = 0. Workspace:
+ * gdn2_workspace_size(GDN2_OP_MAP, ...) bytes, 256-byte aligned (the WY images
+ * of the piece and their flags). The maps go to the caller's buffers; nothing
+ * else is written.
+ */
+gdn2_status gdn2_fwd_map(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                         const void* w, float* M, float* N, int B, int T, int H, int Dk, int Dv, int chunk,
+                         gdn2_dtype dt, void* ws, size_t ws_bytes, void* stream);
+gdn2_status gdn2_bwd_map(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                         const void* w, const void* dout, float* A, float* Bm, int B, int T, int H, int Dk,
+                         int Dv, int chunk, gdn2_dtype dt, void* ws, size_t ws_bytes, void* stream);
+/*
+ * S_out = M S_in + N per (batch, head), in float32: the step that chains the
+ * maps above. M: [B, H, Dk, Dk]; S_in, N, S_out: [B, H, Dk, Dv]; S_in NULL
+ * reads as zero, N NULL as zero. S_out may alias S_in or N (not M). Device
+ * pointers, 16-byte aligned.
+ */
+gdn2_status gdn2_state_affine(const float* M, const float* N, const float* S_in, float* S_out, int B, int H,
+                              int Dk, int Dv, void* stream);
 
 /*
  * Per-kernel timing, for profiling. gdn2_trace_enable(1) makes every later

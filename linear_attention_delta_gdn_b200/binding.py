@@ -21,8 +21,9 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn2.so
 _lib = None
 
 GDN2_F32, GDN2_BF16 = 0, 1
-GDN2_OP_FWD, GDN2_OP_FWD_SAVE, GDN2_OP_BWD = 0, 1, 2
+GDN2_OP_FWD, GDN2_OP_FWD_SAVE, GDN2_OP_BWD, GDN2_OP_MAP = 0, 1, 2, 3
 GDN2_OK, GDN2_ERR_INVALID, GDN2_ERR_TIMEOUT = 0, 1, 5
+GDN2_ERR_UNSUPPORTED = 2
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_WORKSPACE",
           4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT"}
 
@@ -30,7 +31,8 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID", 2: "GDN2_ERR_UNSUPPORTED", 3: "GD
 EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "gdn2_status_string",
            "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes",
            "gdn2_trace_enable", "gdn2_trace_read", "gdn2_device_status", "gdn2_beta_workspace_size",
-           "gdn2_beta_fwd", "gdn2_beta_bwd", "gdn2_varlen_workspace_size", "gdn2_varlen_fwd", "gdn2_varlen_bwd")
+           "gdn2_beta_fwd", "gdn2_beta_bwd", "gdn2_varlen_workspace_size", "gdn2_varlen_fwd", "gdn2_varlen_bwd",
+           "gdn2_fwd_map", "gdn2_bwd_map", "gdn2_state_affine")
 GDN2_GATE_KDA, GDN2_GATE_GDN = 1, 2
 
 
@@ -81,6 +83,12 @@ def lib(path: Optional[str] = None) -> ctypes.CDLL:
     L.gdn2_varlen_fwd.restype = I
     L.gdn2_varlen_bwd.argtypes = [P] * 7 + [I, I, LL] + [P] * 10 + [I] * 6 + [P, Z, P]
     L.gdn2_varlen_bwd.restype = I
+    L.gdn2_fwd_map.argtypes = [P] * 8 + [I] * 7 + [P, Z, P]
+    L.gdn2_fwd_map.restype = I
+    L.gdn2_bwd_map.argtypes = [P] * 9 + [I] * 7 + [P, Z, P]
+    L.gdn2_bwd_map.restype = I
+    L.gdn2_state_affine.argtypes = [P] * 4 + [I] * 4 + [P]
+    L.gdn2_state_affine.restype = I
     L.gdn2_device_status.argtypes = [P]
     L.gdn2_device_status.restype = I
     L.gdn2_trace_enable.argtypes = [I]
@@ -191,6 +199,53 @@ def gdn2_bwd(q, k, v, log_alpha, b, w, dout, S0=None, dST=None, chunk: int = 64,
                         int(states_saved), _ptr(ws), ws.numel(), _stream(q.device))
     _check("gdn2_bwd", rc)
     return grads
+
+
+def _map_ws(q, v, chunk, ws):
+    B, T, H, Dk = q.shape
+    need = gdn2_workspace_size(GDN2_OP_MAP, B, T, H, Dk, v.shape[-1], chunk, _dt(q))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    return ws
+
+
+def gdn2_fwd_map(q, k, v, log_alpha, b, w, chunk: int = 64, ws: Optional[torch.Tensor] = None):
+    """Affine map of a sequence piece, ``S_end = M S_start + N``: returns ``(M, N)``, fp32
+    ``[B, H, Dk, Dk]`` and ``[B, H, Dk, Dv]``."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    M = torch.empty((B, H, Dk, Dk), dtype=torch.float32, device=q.device)
+    N = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    ws = _map_ws(q, v, chunk, ws)
+    rc = lib().gdn2_fwd_map(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(M), _ptr(N),
+                            B, T, H, Dk, Dv, chunk, _dt(q), _ptr(ws), ws.numel(), _stream(q.device))
+    _check("gdn2_fwd_map", rc)
+    return M, N
+
+
+def gdn2_bwd_map(q, k, v, log_alpha, b, w, dout, chunk: int = 64, ws: Optional[torch.Tensor] = None):
+    """Reverse affine map of a sequence piece, ``dS_start = A dS_end + B``: returns ``(A, B)``."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    A = torch.empty((B, H, Dk, Dk), dtype=torch.float32, device=q.device)
+    Bm = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    ws = _map_ws(q, v, chunk, ws)
+    rc = lib().gdn2_bwd_map(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(dout), _ptr(A),
+                            _ptr(Bm), B, T, H, Dk, Dv, chunk, _dt(q), _ptr(ws), ws.numel(), _stream(q.device))
+    _check("gdn2_bwd_map", rc)
+    return A, Bm
+
+
+def gdn2_state_affine(M, N, S_in, out=None):
+    """``M S_in + N`` per (batch, head) in fp32 (``N`` or ``S_in`` may be None: zero)."""
+    B, H, Dk, _ = M.shape
+    ref = N if N is not None else S_in
+    Dv = ref.shape[-1] if ref is not None else Dk
+    if out is None:
+        out = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=M.device)
+    rc = lib().gdn2_state_affine(_ptr(M), _ptr(N), _ptr(S_in), _ptr(out), B, H, Dk, Dv, _stream(M.device))
+    _check("gdn2_state_affine", rc)
+    return out
 
 
 def gdn2_beta_workspace_size(gate: int, op: int, B: int, T: int, H: int, Dk: int, Dv: int, chunk: int,

@@ -235,8 +235,10 @@ struct BwdParams {
     unsigned int* flags;             // [BH, nc] dS' ready flags (zero at launch)
     unsigned int* counter;           // [0]: next gradient unit, [1]: abort word (zero at launch)
     int split_R;                     // > 0: the reverse pass of a head is cut into split_R segments
-    int phase;                       // with split_R: 1 (last segment, segment maps) or 3 (the other segments)
+    int phase;                       // with split_R: 1 (last segment, segment maps) or 3 (the other segments);
+                                     // 5: the reverse maps of every head's whole sequence (map_B, map_A)
     float* sbuf;                     // with split_R: per head, segment end gradients, then the maps B and A
+    float *map_B, *map_A;            // phase 5: [BH][D][D] each
 };
 
 // ---- reverse-pass tasks
@@ -263,6 +265,7 @@ __device__ __forceinline__ float* rsplit_mat(const BwdParams& p, int head, int k
     return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
 }
 __device__ __forceinline__ int rev_task_count(const BwdParams& p) {
+    if (p.phase == 5) return 2 * p.BH;
     if (!p.split_R) return p.BH;
     return p.phase == 1 ? p.BH * (1 + 2 * (p.split_R - 2)) : p.BH * (p.split_R - 1);
 }
@@ -270,6 +273,15 @@ __device__ RevTask rev_task_at(const BwdParams& p, int t) {
     RevTask k{};
     k.head = t % p.BH;
     const size_t hd = (size_t)k.head * D * D;
+    if (p.phase == 5) {   // the whole sequence as one piece: B from a zero end gradient, A from the identity
+        k.c_hi = p.nc - 1; k.c_lo = 0;
+        if (t < p.BH) {
+            k.fin = p.map_B + hd;
+        } else {
+            k.ident = true; k.zero_do = true; k.fin = p.map_A + hd;
+        }
+        return k;
+    }
     if (!p.split_R) {
         k.c_hi = p.nc - 1; k.c_lo = 0; k.start = p.dST ? p.dST + hd : nullptr; k.real = true;
         k.fin = p.dS0 ? p.dS0 + hd : nullptr;
@@ -1075,6 +1087,8 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     const void* ptrs[13] = {a.q, a.k, a.v, a.la, a.b, a.w, a.dout, a.dq, a.dk, a.db, a.dla, a.dv, a.dw};
     CUtensorMap* mp[13] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w, &maps.dout,
                            &maps.dq, &maps.dk, &maps.db, &maps.dla, &maps.dv, &maps.dw};
+    if (a.map_A && a.map_B)   // no gradient units run: their output maps only need a valid address
+        for (int i = 7; i < 13; ++i) ptrs[i] = a.dout;
     for (int i = 0; i < 13; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     LaunchFacts lf{};
@@ -1094,6 +1108,14 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     p.flags = a.flags; p.counter = a.flags + units;
     if ((e = cudaMemsetAsync(a.flags, 0, ((size_t)units + 2) * sizeof(unsigned int), s)) != cudaSuccess) return e;
 
+    if (a.map_A && a.map_B) {   // reverse maps only: the reverse pass of every head twice, no gradients
+        BwdParams pm = p;
+        pm.phase = 5; pm.grad = 0; pm.join = 0; pm.map_A = a.map_A; pm.map_B = a.map_B;
+        pm.nrev = 2 * BH < slots ? 2 * BH : slots;
+        TraceScope trace(K_CHUNK_BWD, s);
+        chunk_bwd_kernel<<<pm.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pm);
+        return cudaGetLastError();
+    }
     const int R = split_segments_for(BH, nc, slots, a.sbuf != nullptr);
     if (R) {   // the last segments and the segment maps, the prefix, then the other segments with the gradients
         p.split_R = R;

@@ -107,8 +107,10 @@ struct FwdParams {
     unsigned char* wyimg;          // [BH, nc] WY images
     unsigned int* flags;           // [BH, nc] ready flags (zero at launch)
     int split_R;                   // > 0: the chunks of a head are cut into split_R segments (long sequences)
-    int phase;                     // with split_R: 1 (first segment, segment maps) or 3 (the other segments)
+    int phase;                     // with split_R: 1 (first segment, segment maps) or 3 (the other segments);
+                                   // 5: the maps of the whole sequence of every head (map_N, map_M)
     float* sbuf;                   // with split_R: per head, segment start states, then the maps N and M
+    float *map_N, *map_M;          // phase 5: [BH][D][D] each
 };
 
 // ---- consumer tasks
@@ -136,6 +138,7 @@ __device__ __forceinline__ float* split_mat(const FwdParams& p, int head, int ki
     return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
 }
 __device__ __forceinline__ int task_count(const FwdParams& p) {
+    if (p.phase == 5) return 2 * p.BH;
     if (!p.split_R) return p.BH;
     return p.phase == 1 ? p.BH * (1 + 2 * (p.split_R - 2)) : p.BH * (p.split_R - 1);
 }
@@ -143,6 +146,15 @@ __device__ Task task_at(const FwdParams& p, int t) {
     Task k{};
     k.head = t % p.BH;
     const size_t hd = (size_t)k.head * D * D;
+    if (p.phase == 5) {   // the whole sequence as one piece: N from a zero start, M from the identity without input
+        k.c0 = 0; k.c1 = p.nc;
+        if (t < p.BH) {
+            k.fin = p.map_N + hd;
+        } else {
+            k.ident = true; k.zero_u = true; k.fin = p.map_M + hd;
+        }
+        return k;
+    }
     if (!p.split_R) {
         k.c0 = 0; k.c1 = p.nc; k.start = p.S0 ? p.S0 + hd : nullptr; k.out = true; k.fin = p.ST ? p.ST + hd : nullptr;
         return k;
@@ -986,12 +998,53 @@ cudaError_t split_prefix_launch(float* sbuf, int R, int BH, cudaStream_t s) {
 
 int split_segments_for(int BH, int nc, int slots, bool have_buf) { return split_segments(BH, nc, slots, have_buf); }
 
+// The producers alone (with_maps: then per head two chains over the whole sequence, a piece of a longer one:
+// N from a zero start with the inputs, M from the identity without input).
+static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool with_maps) {
+    const Dims& d = a.d;
+    if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
+    Maps maps;
+    const void* ptrs[6] = {a.q, a.k, a.v, a.la, a.b, a.w};
+    CUtensorMap* mp[6] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w};
+    for (int i = 0; i < 6; ++i)
+        if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    LaunchFacts lf{};
+    cudaError_t e = launch_facts(chunk_fwd_kernel, NT, SMEM_BYTES, &lf);
+    if (e != cudaSuccess) return e;
+    const int BH = d.B * d.H, nc = d.nchunks(), units = BH * nc, slots = lf.nsm * lf.occ;
+    FwdParams p{};
+    p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
+    p.q = static_cast<const __nv_bfloat16*>(a.q); p.k = static_cast<const __nv_bfloat16*>(a.k);
+    p.la = static_cast<const __nv_bfloat16*>(a.la); p.b = static_cast<const __nv_bfloat16*>(a.b);
+    p.wyimg = a.wy; p.flags = a.flags;
+    if ((e = cudaMemsetAsync(a.flags, 0, (size_t)units * sizeof(unsigned int), s)) != cudaSuccess) return e;
+    FwdParams pp = p;
+    pp.ncons = 0;
+    pp.nprod = units < slots ? units : slots;
+    {
+        TraceScope trace(K_CHUNK_FWD, s);
+        chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (!with_maps) return cudaSuccess;
+    FwdParams pc = p;
+    pc.phase = 5; pc.nprod = 0; pc.map_N = a.map_N; pc.map_M = a.map_M;
+    pc.ncons = 2 * BH < slots ? 2 * BH : slots;
+    TraceScope trace(K_CHUNK_FWD, s);
+    chunk_fwd_kernel<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
+    return cudaGetLastError();
+}
+
+cudaError_t chunk_fwd_map_launch(const ChunkFwdArgs& a, cudaStream_t s) { return fwd_pieces_launch(a, s, true); }
+cudaError_t chunk_fwd_wy_launch(const ChunkFwdArgs& a, cudaStream_t s) { return fwd_pieces_launch(a, s, false); }
+
 size_t chunk_fwd_split_bytes(int BH, int nc) {
     if (BH > TC_SPLIT_MAX_BH || nc < TC_SPLIT_MIN_CHUNKS_PER_SEG * 4) return 0;
     return (size_t)BH * SPLIT_MATS_PER_HEAD * TC_D * TC_D * sizeof(float);
 }
 
 cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
+    if (a.map_N && a.map_M) return chunk_fwd_map_launch(a, s);
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
     Maps maps;

@@ -177,6 +177,9 @@ size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int 
     case GDN2_OP_FWD: return tc_path(dt, Dk, Dv) ? align256(tc_wy_bytes(d)) : 0;
     case GDN2_OP_FWD_SAVE: return align256(states_bytes(d, dt));
     case GDN2_OP_BWD: return align256(states_bytes(d, dt)) + align256(bwd_extra_bytes(d, dt));
+    case GDN2_OP_MAP:   // WY images, then ready flags with the backward's work counter and abort word
+        return tc_path(dt, Dk, Dv) ? align256(tc_units(d) * TC_WY_BYTES) + align256((tc_units(d) + 2) * sizeof(unsigned int))
+                                   : 0;
     }
     return 0;
 }
@@ -299,6 +302,93 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
     a.seg = reinterpret_cast<float*>(extra);
     a.segdelta = reinterpret_cast<float*>(extra + align256(seg));
     return cuda_status(recurrent_launch(a, s), "gdn2_bwd (recurrent path)");
+}
+
+// Shared checks of gdn2_fwd_map / gdn2_bwd_map; T == 0 writes the maps of an empty piece.
+static gdn2_status map_prologue(const char* name, const void* q, const void* k, const void* v, const void* la,
+                                const void* b, const void* w, const void* dout, bool need_dout, float* Mx, float* Nx,
+                                int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt, void* ws, size_t ws_bytes,
+                                cudaStream_t s, bool* done) {
+    *done = false;
+    gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
+    if (st != GDN2_OK) return st;
+    if (!tc_path(dt, Dk, Dv))
+        return fail(GDN2_ERR_UNSUPPORTED, "%s: maps are computed on the tensor-core path only (bf16, Dk = Dv = 128)", name);
+    if (!Mx || !aligned(Mx, 16) || !Nx || !aligned(Nx, 16))
+        return fail(GDN2_ERR_INVALID, "%s: both map outputs must be non-NULL and 16-byte aligned", name);
+    const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
+    if (T == 0) {
+        *done = true;
+        cudaError_t e = state_identity_launch(Mx, B * H, Dk, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(Nx, 0, (size_t)B * H * Dk * Dv * sizeof(float), s);
+        return cuda_status(e, name);
+    }
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(la); REQUIRE_PTR(b); REQUIRE_PTR(w);
+    if (need_dout) REQUIRE_PTR(dout);
+    const size_t need = gdn2_workspace_size(GDN2_OP_MAP, B, T, H, Dk, Dv, chunk, dt);
+    if (!ws || ws_bytes < need) return fail(GDN2_ERR_WORKSPACE, "%s needs %zu workspace bytes, got %zu", name, need, ws ? ws_bytes : 0);
+    if (!aligned(ws, 256)) return fail(GDN2_ERR_INVALID, "ws must be 256-byte aligned");
+    (void)d;
+    return GDN2_OK;
+}
+
+gdn2_status gdn2_fwd_map(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                         const void* w, float* M, float* N, int B, int T, int H, int Dk, int Dv, int chunk,
+                         gdn2_dtype dt, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx("gdn2_fwd_map");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bool done = false;
+    gdn2_status st = map_prologue("gdn2_fwd_map", q, k, v, log_alpha, b, w, nullptr, false, M, N, B, T, H, Dk, Dv,
+                                  chunk, dt, ws, ws_bytes, s, &done);
+    if (st != GDN2_OK || done) return st;
+    const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    ChunkFwdArgs a{};
+    a.d = d;
+    a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
+    a.wy = wsb;
+    a.flags = reinterpret_cast<unsigned int*>(wsb + align256(tc_units(d) * TC_WY_BYTES));
+    a.map_N = N; a.map_M = M;
+    return cuda_status(chunk_fwd_launch(a, s), "gdn2_fwd_map");
+}
+
+gdn2_status gdn2_bwd_map(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                         const void* w, const void* dout, float* A, float* Bm, int B, int T, int H, int Dk,
+                         int Dv, int chunk, gdn2_dtype dt, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx("gdn2_bwd_map");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bool done = false;
+    gdn2_status st = map_prologue("gdn2_bwd_map", q, k, v, log_alpha, b, w, dout, true, A, Bm, B, T, H, Dk, Dv,
+                                  chunk, dt, ws, ws_bytes, s, &done);
+    if (st != GDN2_OK || done) return st;
+    const Dims d = run_dims(B, T, H, Dk, Dv, chunk, dt);
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    unsigned int* flags = reinterpret_cast<unsigned int*>(wsb + align256(tc_units(d) * TC_WY_BYTES));
+    // the WY images of the piece (the forward's producers alone), then the reverse pass twice per head
+    ChunkFwdArgs f{};
+    f.d = d;
+    f.q = q; f.k = k; f.v = v; f.la = log_alpha; f.b = b; f.w = w;
+    f.wy = wsb; f.flags = flags;
+    cudaError_t e = chunk_fwd_wy_launch(f, s);
+    if (e != cudaSuccess) return cuda_status(e, "gdn2_bwd_map (WY images)");
+    ChunkBwdArgs a{};
+    a.d = d;
+    a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w; a.dout = dout;
+    a.tp = wsb; a.flags = flags;
+    a.map_A = A; a.map_B = Bm;
+    return cuda_status(chunk_bwd_launch(a, s), "gdn2_bwd_map");
+}
+
+gdn2_status gdn2_state_affine(const float* M, const float* N, const float* S_in, float* S_out, int B, int H, int Dk,
+                              int Dv, void* stream) {
+    NvtxRange nvtx("gdn2_state_affine");
+    gdn2_status st = check_dims(B, 1, H, Dk, Dv, 64, GDN2_F32, false);
+    if (st != GDN2_OK) return st;
+    REQUIRE_PTR(M); REQUIRE_PTR(S_out);
+    OPTIONAL_PTR(N); OPTIONAL_PTR(S_in);
+    if ((const float*)S_out == M) return fail(GDN2_ERR_INVALID, "S_out must not alias M");
+    return cuda_status(state_affine_launch(M, N, S_in, S_out, B * H, Dk, Dv, static_cast<cudaStream_t>(stream)),
+                       "gdn2_state_affine");
 }
 
 gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,

@@ -51,8 +51,11 @@ struct ChunkFwdArgs {
     unsigned char* wy;     // [B,H,NC] WY images (T | P | Wm), always written
     unsigned int* flags;   // [B,H,NC] ready flags (scratch)
     float* sbuf;           // segment states and maps of long sequences (chunk_fwd_split_bytes), or null
+    float *map_N, *map_M;  // both set: compute the affine map of each head's sequence instead ([BH][128][128])
 };
 cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s);
+cudaError_t chunk_fwd_map_launch(const ChunkFwdArgs& a, cudaStream_t s);   // map_N / map_M of every head
+cudaError_t chunk_fwd_wy_launch(const ChunkFwdArgs& a, cudaStream_t s);    // the WY images (and flags) alone
 // Long sequences with few heads: a head's chunks may be cut into segments that run on separate CTAs (segment
 // maps, a prefix over them, then the segments again from their start states). Workspace for that, 0 if the
 // problem never qualifies.
@@ -78,12 +81,17 @@ struct ChunkBwdArgs {
     unsigned char* ddeltas;       // [B,H,NC] dDelta^T images (scratch)
     unsigned int* flags;          // [B,H,NC] ready flags, then work counter and abort word (scratch)
     float* sbuf;                  // segment gradients and maps of long sequences (chunk_fwd_split_bytes), or null
+    float *map_B, *map_A;         // both set: compute the reverse affine map of each head's sequence instead
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
+// dst = M src + N per head, fp32 [BH][128][128] operands, in place allowed for src == dst
+cudaError_t state_affine_launch(const float* M, const float* N, const float* src, float* dst, int BH, int Dk, int Dv,
+                                cudaStream_t s);
+cudaError_t state_identity_launch(float* dst, int BH, int Dk, cudaStream_t s);   // dst = I per head [Dk][Dk]
 
 // Kernels of the library, for gdn2_trace_read().
 enum KernelId { K_CHUNK_FWD = 0, K_CHUNK_BWD, K_REC_FWD, K_REC_BWD, K_DECODE, K_GATE_EXPAND, K_GATE_REDUCE,
-                K_VARLEN_COPY, K_SPLIT_PREFIX, KERNEL_COUNT };
+                K_VARLEN_COPY, K_SPLIT_PREFIX, K_STATE_AFFINE, KERNEL_COUNT };
 
 // Brackets one kernel launch with CUDA events on its stream while tracing is on.
 class TraceScope {

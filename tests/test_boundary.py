@@ -69,6 +69,9 @@ def test_workspace_sizes(L):
     for op in (0, 1, 2):
         for c in (16, 32):
             assert ws(op, 2, 300, 3, 128, 128, c, 1) == ws(op, 2, 300, 3, 128, 128, 64, 1)
+    # the maps of a sequence piece: WY images, then flags with the work counter and abort word
+    assert ws(3, 4, 4096, 16, 128, 128, 64, 1) == units * 82944 + units * 4 + 256
+    assert ws(3, 1, 256, 2, 64, 64, 64, 0) == 0
     # invalid problems report zero
     assert ws(1, 0, 16, 1, 64, 64, 64, 1) == 0
     assert ws(1, 1, 16, 1, 96, 64, 64, 1) == 0
@@ -148,3 +151,16 @@ def test_device_status_reports_a_cuda_error_without_a_device(L):
         pytest.skip("a CUDA device is present (the GPU tests cover the status call)")
     assert L.gdn2_device_status(None) == 4
     assert b"gdn2_device_status" in L.gdn2_last_error()
+
+
+def test_maps_are_computed_on_the_tensor_core_path_only(L):
+    from linear_attention_delta_gdn_b200 import binding
+    for fn, nptr in ((L.gdn2_fwd_map, 8), (L.gdn2_bwd_map, 9)):
+        rc = fn(*([None] * nptr), 1, 64, 2, 64, 64, 64, binding.GDN2_F32, None, 0, None)
+        assert rc == binding.GDN2_ERR_UNSUPPORTED
+        assert "tensor-core path" in L.gdn2_last_error().decode()
+    # missing map outputs are refused before any launch
+    rc = L.gdn2_fwd_map(*([None] * 8), 1, 64, 2, 128, 128, 64, binding.GDN2_BF16, None, 0, None)
+    assert rc == binding.GDN2_ERR_INVALID
+    rc = L.gdn2_state_affine(None, None, None, None, 1, 1, 128, 128, None)
+    assert rc == binding.GDN2_ERR_INVALID
