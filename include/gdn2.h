@@ -309,6 +309,31 @@ gdn2_status gdn2_state_affine(const float* M, const float* N, const float* S_in,
                               int Dk, int Dv, void* stream);
 
 /*
+ * Gate activations of a Gated DeltaNet-2 layer: the operator's inputs from one
+ * projection of the hidden state. The pages name the two per-channel gate
+ * computations (GitHub README method bullets; the aiexpert.news article puts
+ * the overhead over KDA on them) but not their parameterisation; the plainest
+ * reading is used. Per token and head, z = [z_q | z_k | z_v | z_b | z_w | z_a]
+ * (widths Dk, Dk, Dv, Dk, Dv, Dk) gives
+ *   q = z_q / ||z_q||,  k = z_k / ||z_k||   (L2 over the head's channels, 1e-6
+ *                                            added under the root)
+ *   v = z_v,  b = sigmoid(z_b),  w = sigmoid(z_w),
+ *   log_alpha = -softplus(z_a + a_bias)
+ *   z                   : [B, T, H, 4 Dk + 2 Dv] dt
+ *   a_bias              : [H, Dk] float32 decay bias, or NULL for none
+ *   q, k, b, log_alpha  : [B, T, H, Dk] dt ;  v, w : [B, T, H, Dv] dt
+ * gdn2_layer_gates_bwd writes dz (same layout as z) from z and the gradients of
+ * the six outputs (as gdn2_bwd returns them); the gradient of a_bias is the sum
+ * of dz_a over batch and tokens. Device pointers, 16-byte aligned;
+ * no workspace; any Dk, Dv the operator supports; fp32 arithmetic.
+ */
+gdn2_status gdn2_layer_gates_fwd(const void* z, const float* a_bias, void* q, void* k, void* v, void* b, void* w,
+                                 void* log_alpha, int B, int T, int H, int Dk, int Dv, gdn2_dtype dt, void* stream);
+gdn2_status gdn2_layer_gates_bwd(const void* z, const float* a_bias, const void* dq, const void* dk, const void* dv,
+                                 const void* db, const void* dw, const void* dlog_alpha, void* dz, int B, int T, int H,
+                                 int Dk, int Dv, gdn2_dtype dt, void* stream);
+
+/*
  * Per-kernel timing, for profiling. gdn2_trace_enable(1) makes every later
  * kernel launch of the library record a CUDA event before and after it on the
  * launch's stream (gdn2_trace_enable(0) stops it; off by default).

@@ -17,7 +17,10 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn2.so")
+_DEBUG_BUILD = os.environ.get("GDN2_DEBUG", "") not in ("", "0")
+#: the library this process loads: the debug build (index checks, see build.py) when GDN2_DEBUG is set
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libgdn2_debug.so" if _DEBUG_BUILD else "libgdn2.so")
 _lib = None
 
 GDN2_F32, GDN2_BF16 = 0, 1
@@ -32,7 +35,7 @@ EXPORTS = ("gdn2_workspace_size", "gdn2_fwd", "gdn2_bwd", "gdn2_decode_step", "g
            "gdn2_last_error", "gdn2_version", "gdn2_bwd_no_alloc", "gdn2_no_alloc_scratch_bytes",
            "gdn2_trace_enable", "gdn2_trace_read", "gdn2_device_status", "gdn2_beta_workspace_size",
            "gdn2_beta_fwd", "gdn2_beta_bwd", "gdn2_varlen_workspace_size", "gdn2_varlen_fwd", "gdn2_varlen_bwd",
-           "gdn2_fwd_map", "gdn2_bwd_map", "gdn2_state_affine")
+           "gdn2_fwd_map", "gdn2_bwd_map", "gdn2_state_affine", "gdn2_layer_gates_fwd", "gdn2_layer_gates_bwd")
 GDN2_GATE_KDA, GDN2_GATE_GDN = 1, 2
 
 
@@ -89,6 +92,10 @@ def lib(path: Optional[str] = None) -> ctypes.CDLL:
     L.gdn2_bwd_map.restype = I
     L.gdn2_state_affine.argtypes = [P] * 4 + [I] * 4 + [P]
     L.gdn2_state_affine.restype = I
+    L.gdn2_layer_gates_fwd.argtypes = [P] * 8 + [I] * 6 + [P]
+    L.gdn2_layer_gates_fwd.restype = I
+    L.gdn2_layer_gates_bwd.argtypes = [P] * 9 + [I] * 6 + [P]
+    L.gdn2_layer_gates_bwd.restype = I
     L.gdn2_device_status.argtypes = [P]
     L.gdn2_device_status.restype = I
     L.gdn2_trace_enable.argtypes = [I]
@@ -246,6 +253,32 @@ def gdn2_state_affine(M, N, S_in, out=None):
     rc = lib().gdn2_state_affine(_ptr(M), _ptr(N), _ptr(S_in), _ptr(out), B, H, Dk, Dv, _stream(M.device))
     _check("gdn2_state_affine", rc)
     return out
+
+
+def gdn2_layer_gates_fwd(z, Dk: int, Dv: int, a_bias=None):
+    """Operator inputs from the layer's pre-activations ``z [B, T, H, 4 Dk + 2 Dv]``: returns
+    ``(q, k, v, b, w, log_alpha)`` in z's dtype (``a_bias``: fp32 [H, Dk] decay bias or None)."""
+    B, T, H, W = z.shape
+    if W != 4 * Dk + 2 * Dv:
+        raise ValueError("z must be [B, T, H, 4 Dk + 2 Dv]")
+    if a_bias is not None and (a_bias.dtype != torch.float32 or tuple(a_bias.shape) != (H, Dk)):
+        raise ValueError("a_bias must be float32 [H, Dk]")
+    mk = lambda D: torch.empty((B, T, H, D), dtype=z.dtype, device=z.device)
+    q, k, v, b, w, la = mk(Dk), mk(Dk), mk(Dv), mk(Dk), mk(Dv), mk(Dk)
+    rc = lib().gdn2_layer_gates_fwd(_ptr(z), _ptr(a_bias), _ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(la),
+                                    B, T, H, Dk, Dv, _dt(z), _stream(z.device))
+    _check("gdn2_layer_gates_fwd", rc)
+    return q, k, v, b, w, la
+
+
+def gdn2_layer_gates_bwd(z, dq, dk, dv, db, dw, dlog_alpha, Dk: int, Dv: int, a_bias=None):
+    """dz (z's layout) from z and the gradients of the six operator inputs."""
+    B, T, H, _ = z.shape
+    dz = torch.empty_like(z)
+    rc = lib().gdn2_layer_gates_bwd(_ptr(z), _ptr(a_bias), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(db), _ptr(dw),
+                                    _ptr(dlog_alpha), _ptr(dz), B, T, H, Dk, Dv, _dt(z), _stream(z.device))
+    _check("gdn2_layer_gates_bwd", rc)
+    return dz
 
 
 def gdn2_beta_workspace_size(gate: int, op: int, B: int, T: int, H: int, Dk: int, Dv: int, chunk: int,

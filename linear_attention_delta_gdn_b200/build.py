@@ -1,11 +1,16 @@
 """Build libgdn2.so in-tree with nvcc for sm_100a (B200).
 
-    python -m linear_attention_delta_gdn_b200.build [--force]
+    python -m linear_attention_delta_gdn_b200.build [--force] [--debug]
 
 Each ``csrc/*.cu`` is compiled to an object in ``_build/`` (in parallel), then
 linked into ``linear_attention_delta_gdn_b200/libgdn2.so`` with the CUDA runtime
 linked statically, so the library loads on a host without a GPU driver (the
 driver entry points it needs are looked up at run time).
+
+``--debug`` builds ``libgdn2_debug.so`` instead (objects in ``_build_debug/``),
+compiled with ``-DGDN2_DEBUG``: the kernels' index checks then record failures
+for ``gdn2_device_status`` and skip the guarded accesses. The binding loads it
+when the environment variable ``GDN2_DEBUG`` is set.
 """
 from __future__ import annotations
 
@@ -23,6 +28,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgdn2.so")
+LIB_DEBUG = os.path.join(PKG, "libgdn2_debug.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I", INCLUDE,
@@ -45,22 +52,24 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib, bdir = (LIB_DEBUG, BUILD_DEBUG) if debug else (LIB, BUILD)
+    if not force and not stale(lib):
+        return lib
+    os.makedirs(bdir, exist_ok=True)
     cc = nvcc()
+    flags = NVCC_FLAGS + (["-DGDN2_DEBUG"] if debug else [])
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [cc, *NVCC_FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [cc, *flags, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("nvcc failed on %s:\n%s\n%s" % (src, r.stdout, r.stderr))
@@ -71,18 +80,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         for _, log in results:
             sys.stderr.write(log)
-    tmp = LIB + ".tmp%d" % os.getpid()
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", tmp] + [o for o, _ in results]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s\n%s" % (r.stdout, r.stderr))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libgdn2_debug.so with the index checks")
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose))
+    print(build(force=args.force, verbose=args.verbose, debug=args.debug))

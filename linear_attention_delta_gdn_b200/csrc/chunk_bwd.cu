@@ -262,6 +262,7 @@ __host__ __device__ inline int seg_begin(int s, int nc, int R) { return (int)((l
 __device__ __forceinline__ float* rsplit_mat(const BwdParams& p, int head, int kind, int k) {   // 0: E, 1: B, 2: A
     const int R = p.split_R;
     const int idx = kind == 0 ? k - 1 : (kind == 1 ? (R - 1) + (k - 1) : (R - 1) + (R - 2) + (k - 1));
+    if (!GDN2_IN(g_bwd_error, idx >= 0 && idx < (int)SPLIT_MATS_PER_HEAD && head < p.BH)) return nullptr;
     return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
 }
 __device__ __forceinline__ int rev_task_count(const BwdParams& p) {
@@ -323,7 +324,7 @@ __device__ __forceinline__ int unit_slots(const BwdParams& p) {
     }
     return p.BH * last + p.BH * (R - 1) * lmax;
 }
-__device__ __forceinline__ bool unit_at(const BwdParams& p, int u, int* head, int* c) {
+__device__ __forceinline__ bool unit_at_unchecked(const BwdParams& p, int u, int* head, int* c) {
     if (!p.split_R) {
         *c = p.nc - 1 - u / p.BH;
         *head = u % p.BH;
@@ -340,6 +341,9 @@ __device__ __forceinline__ bool unit_at(const BwdParams& p, int u, int* head, in
     const int lo = seg_begin(s2, p.nc, R), hi = seg_begin(s2 + 1, p.nc, R) - 1;
     *c = hi - jpos;
     return *c >= lo;
+}
+__device__ __forceinline__ bool unit_at(const BwdParams& p, int u, int* head, int* c) {
+    return unit_at_unchecked(p, u, head, c) && GDN2_IN(g_bwd_error, *head >= 0 && *head < p.BH && *c >= 0 && *c < p.nc);
 }
 // mbarrier parities carried across the units a CTA works on
 struct Phases {
@@ -1035,7 +1039,12 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
     const bool reverse = (int)blockIdx.x < p.nrev;
     if (reverse) {   // the CTA's reverse-pass tasks (one each in a launch with gradient workers)
         const int ntasks = rev_task_count(p);
-        for (int t = blockIdx.x; t < ntasks && !*abort_flag; t += p.nrev) run_reverse(maps, p, sm, tmem, rev_task_at(p, t), ph);
+        for (int t = blockIdx.x; t < ntasks && !*abort_flag; t += p.nrev) {
+            const RevTask task = rev_task_at(p, t);
+            if (GDN2_IN(g_bwd_error, task.head >= 0 && task.head < p.BH && 0 <= task.c_lo && task.c_lo <= task.c_hi &&
+                                         task.c_hi < p.nc))
+                run_reverse(maps, p, sm, tmem, task, ph);
+        }
     }
     if (p.grad && (!reverse || p.join) && !*abort_flag) {
         const int units = unit_slots(p);

@@ -135,6 +135,7 @@ __host__ __device__ inline int seg_begin(int s, int nc, int R) { return (int)((l
 __device__ __forceinline__ float* split_mat(const FwdParams& p, int head, int kind, int s) {   // kind 0: S, 1: N, 2: M
     const int R = p.split_R;
     const int idx = kind == 0 ? s - 1 : (kind == 1 ? (R - 1) + (s - 1) : (R - 1) + (R - 2) + (s - 1));
+    if (!GDN2_IN(g_fwd_error, idx >= 0 && idx < (int)SPLIT_MATS_PER_HEAD && head < p.BH)) return nullptr;
     return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
 }
 __device__ __forceinline__ int task_count(const FwdParams& p) {
@@ -532,6 +533,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         unsigned int* umask = reinterpret_cast<unsigned int*>(sm + wy::UMASK) + 8 * wg + 4 * (kunit & 1);
         if (wt < 4) reinterpret_cast<unsigned int*>(sm + wy::UMASK)[8 * wg + 4 * ((kunit + 1) & 1) + wt] = 0u;
         unsigned char* img = p.wyimg + ((size_t)head * p.nc + c) * TC_WY_BYTES;
+        const bool img_ok = GDN2_IN(g_fwd_error, head < p.BH && c < p.nc);   // else the image is not written
         gate_prep_wg(QE, KH, KT, gC, sX, umask, wt, wg_sync);
         sync_for_mma_wg();
         const bool untame = (umask[0] | umask[1] | umask[2] | umask[3]) != 0u;   // the same on every thread
@@ -539,7 +541,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             clear_untame_kt(KT, umask, wt);
             sync_for_mma_wg();
         }
-        if (wt == 0) {   // first image group: Qt, Kt, gC (final after the prep), and the untame mask
+        if (wt == 0 && img_ok) {   // first image group: Qt, Kt, gC (final after the prep), and the untame mask
             tc::bulk_store(img + TC_WY_QT, QE + 8192, 8192u);               // Qt (two 64-row halves of the
             tc::bulk_store(img + TC_WY_QT + 8192, QE + 24576, 8192u);       //  128-row tile, 16 KB apart)
             tc::bulk_store(img + TC_WY_KT, KT, 16384u);                     // Kt
@@ -566,7 +568,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         extract_AP_wg(lane_base + (tm_ap - tmem), sA, PP, wq, lane);   // A over k: the prep has read k
         tc::tc_fence_before();
         wg_sync();
-        if (untame) {   // exact terms of the channels left out of M1 (TF is free until the solve)
+        if (untame && img_ok) {   // exact terms of the channels left out of M1 (TF is free until the solve)
             int b, h, t0;
             coords(u, b, h, t0);
             untame_fixup_wg(p.T, p.H, p.q, p.k, p.la, p.b, b, h, t0, umask, sA, PP,
@@ -591,7 +593,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
                          // second image group: T | P | Wm
             if (unreleased >= 0 && !*abort_flag) tc::flag_release_after_bulk_but1(p.flags + unreleased, 1u);
             const size_t unit = (size_t)head * p.nc + c;
-            tc::bulk_store(p.wyimg + unit * TC_WY_BYTES + TC_WY_T, TT, 32768u);
+            if (img_ok) tc::bulk_store(p.wyimg + unit * TC_WY_BYTES + TC_WY_T, TT, 32768u);
             tc::bulk_commit();
             unreleased = (long long)unit;
         }
@@ -684,6 +686,9 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     const int ntasks = task_count(p);
     for (int ti = cid; ti < ntasks; ti += p.ncons) {
         const Task task = task_at(p, ti);
+        if (!GDN2_IN(g_fwd_error, task.head >= 0 && task.head < p.BH && 0 <= task.c0 && task.c0 < task.c1 &&
+                                      task.c1 <= nc))
+            continue;   // the same on every thread, before any barrier of the task
         const int headi = task.head, c0 = task.c0, c1 = task.c1;
         const size_t head = (size_t)headi;
         const int h = headi % H, b = headi / H;
@@ -945,6 +950,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 // (row i = tid / 2, 8 columns) keeps its sums in registers.
 __global__ void __launch_bounds__(256) split_prefix_kernel(float* sbuf, int R) {
     __shared__ float Sc[D][16];
+    if (!GDN2_IN(g_fwd_error, R >= 4 && R <= SPLIT_R_MAX)) return;   // the slots of a head hold R <= SPLIT_R_MAX
     const int head = blockIdx.x / (D / 16), j0 = (blockIdx.x % (D / 16)) * 16;
     const int tid = threadIdx.x, i = tid >> 1, jh = (tid & 1) * 8;
     float* base = sbuf + (size_t)head * SPLIT_MATS_PER_HEAD * D * D;

@@ -31,4 +31,15 @@ __host__ __device__ __forceinline__ size_t tok_off(int b, int t, int h, int T, i
 
 __device__ __forceinline__ float fast_exp(float x) { return exp2f(x * 1.4426950408889634f); }
 
+// Index checks of the debug build (compiled with -DGDN2_DEBUG into libgdn2_debug.so). GDN2_IN(word, cond) is
+// true when cond holds; otherwise it sets GDN2_DBG_BIT in the kernel's error word and is false, and the caller
+// skips the access it guards, so the kernel returns normally and gdn2_device_status reports the failure.
+// Nothing traps. In release builds every check is the constant true and costs nothing.
+constexpr unsigned int GDN2_DBG_BIT = 1u << 30;
+#ifdef GDN2_DEBUG
+#define GDN2_IN(word, cond) ((cond) ? true : (atomicOr(&(word), ::gdn2::GDN2_DBG_BIT), false))
+#else
+#define GDN2_IN(word, cond) true
+#endif
+
 }  // namespace gdn2

@@ -161,6 +161,11 @@ gdn2_status gdn2_device_status(void* stream) {
     if (vl)
         return fail(GDN2_ERR_INVALID, "cu_seqlens: %s%s", (vl & 1u) ? "a sequence was longer than Tmax (cut) " : "",
                     (vl & 2u) ? "a sequence lay outside [0, Ttot) or had a negative length (dropped)" : "");
+    if ((fwd | bwd) & GDN2_DBG_BIT)
+        return fail(GDN2_ERR_INVALID,
+                    "index check failed (debug build; the accesses it guarded were skipped): chunk_fwd_kernel bits "
+                    "0x%x, chunk_bwd_kernel bits 0x%x",
+                    fwd, bwd);
     if (fwd | bwd)
         return fail(GDN2_ERR_TIMEOUT,
                     "device wait gave up: chunk_fwd_kernel bits 0x%x, chunk_bwd_kernel bits 0x%x "
@@ -389,6 +394,33 @@ gdn2_status gdn2_state_affine(const float* M, const float* N, const float* S_in,
     if ((const float*)S_out == M) return fail(GDN2_ERR_INVALID, "S_out must not alias M");
     return cuda_status(state_affine_launch(M, N, S_in, S_out, B * H, Dk, Dv, static_cast<cudaStream_t>(stream)),
                        "gdn2_state_affine");
+}
+
+gdn2_status gdn2_layer_gates_fwd(const void* z, const float* a_bias, void* q, void* k, void* v, void* b, void* w,
+                                 void* log_alpha, int B, int T, int H, int Dk, int Dv, gdn2_dtype dt, void* stream) {
+    NvtxRange nvtx("gdn2_layer_gates_fwd");
+    gdn2_status st = check_dims(B, T, H, Dk, Dv, 64, dt, true);
+    if (st != GDN2_OK) return st;
+    if (T == 0) return GDN2_OK;
+    REQUIRE_PTR(z); REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(b); REQUIRE_PTR(w);
+    REQUIRE_PTR(log_alpha); OPTIONAL_PTR(a_bias);
+    return cuda_status(gates_fwd_launch(z, q, k, v, b, w, log_alpha, a_bias, (long long)B * T * H, H, Dk, Dv, dt,
+                                        static_cast<cudaStream_t>(stream)),
+                       "gdn2_layer_gates_fwd");
+}
+
+gdn2_status gdn2_layer_gates_bwd(const void* z, const float* a_bias, const void* dq, const void* dk, const void* dv,
+                                 const void* db, const void* dw, const void* dlog_alpha, void* dz, int B, int T, int H,
+                                 int Dk, int Dv, gdn2_dtype dt, void* stream) {
+    NvtxRange nvtx("gdn2_layer_gates_bwd");
+    gdn2_status st = check_dims(B, T, H, Dk, Dv, 64, dt, true);
+    if (st != GDN2_OK) return st;
+    if (T == 0) return GDN2_OK;
+    REQUIRE_PTR(z); REQUIRE_PTR(dq); REQUIRE_PTR(dk); REQUIRE_PTR(dv); REQUIRE_PTR(db); REQUIRE_PTR(dw);
+    REQUIRE_PTR(dlog_alpha); REQUIRE_PTR(dz); OPTIONAL_PTR(a_bias);
+    return cuda_status(gates_bwd_launch(z, dq, dk, dv, db, dw, dlog_alpha, a_bias, dz, (long long)B * T * H, H, Dk, Dv, dt,
+                                        static_cast<cudaStream_t>(stream)),
+                       "gdn2_layer_gates_bwd");
 }
 
 gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,

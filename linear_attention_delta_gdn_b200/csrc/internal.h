@@ -89,9 +89,16 @@ cudaError_t state_affine_launch(const float* M, const float* N, const float* src
                                 cudaStream_t s);
 cudaError_t state_identity_launch(float* dst, int BH, int Dk, cudaStream_t s);   // dst = I per head [Dk][Dk]
 
+// Gate activations of the layer (layer_gates.cu): z [rows][4 Dk + 2 Dv] -> q, k, v, b, w, log_alpha and back.
+cudaError_t gates_fwd_launch(const void* z, void* q, void* k, void* v, void* b, void* w, void* la, const float* abias,
+                             long long rows, int H, int Dk, int Dv, gdn2_dtype dt, cudaStream_t s);
+cudaError_t gates_bwd_launch(const void* z, const void* dq, const void* dk, const void* dv, const void* db, const void* dw,
+                             const void* dla, const float* abias, void* dz, long long rows, int H, int Dk, int Dv,
+                             gdn2_dtype dt, cudaStream_t s);
+
 // Kernels of the library, for gdn2_trace_read().
 enum KernelId { K_CHUNK_FWD = 0, K_CHUNK_BWD, K_REC_FWD, K_REC_BWD, K_DECODE, K_GATE_EXPAND, K_GATE_REDUCE,
-                K_VARLEN_COPY, K_SPLIT_PREFIX, K_STATE_AFFINE, KERNEL_COUNT };
+                K_VARLEN_COPY, K_SPLIT_PREFIX, K_STATE_AFFINE, K_LAYER_GATES, K_LAYER_GATES_BWD, KERNEL_COUNT };
 
 // Brackets one kernel launch with CUDA events on its stream while tracing is on.
 class TraceScope {

@@ -22,7 +22,7 @@ namespace {
 const char* kNames[KERNEL_COUNT] = {"chunk_fwd_kernel", "chunk_bwd_kernel", "recurrent_fwd_kernel",
                                     "recurrent_bwd_kernel", "decode_kernel", "gate_expand_kernel",
                                     "gate_reduce_kernel", "pad_copy_kernel", "split_prefix_kernel",
-                                    "state_affine_kernel"};
+                                    "state_affine_kernel", "gates_fwd_kernel", "gates_bwd_kernel"};
 
 std::atomic<int> g_on{0};
 std::mutex g_mu;

@@ -50,3 +50,17 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _debug_build_index_checks(request):
+    """Under the debug build (environment GDN2_DEBUG set), every GPU test ends with no failed index check."""
+    yield
+    if os.environ.get("GDN2_DEBUG", "") in ("", "0") or request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    from linear_attention_delta_gdn_b200 import binding
+    if binding.gdn2_device_status() != binding.GDN2_OK:
+        assert "index check" not in binding.last_error(), binding.last_error()
