@@ -18,6 +18,10 @@ Besides the headline step, the line carries (rank 0, N=1):
   * ``decode``: 1024 in-place decode steps (batch 256, 16 heads, d = 128);
   * ``kda_overhead``: the KDA and Gated DeltaNet reductions through the same
     kernels at the headline shape, against the GDN-2 step;
+  * ``layer_gates``: the layer's gate-activation kernels (forward and backward)
+    at the headline shape, against the HBM roofline;
+  * ``context_parallel_maps``: a context-parallel rank's map kernels on one
+    16K-token piece, beside that piece's own forward and fwd+bwd;
   * ``cpu_baseline``: the fp64 oracle timed on a bounded sample of the headline
     workload on the host cores, with the GPU outputs of those same sequences
     compared against the oracle's (relative L2, whole sample and worst head).
@@ -385,6 +389,58 @@ def measure_reductions(binding, dev, d, args, gdn2_ms):
     return out
 
 
+def measure_layer_gates(binding, dev, args, B, T, H, D=128):
+    """The layer's gate-activation kernels at the headline shape: z [B, T, H, 6 D] bf16 drawn on the device.
+    Algorithmic bytes per token-head: forward z in + six outputs = 2 x 6D x 2 B; backward z and six gradients
+    in, dz out = 3 x 6D x 2 B."""
+    import torch
+    pk = peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7000)
+    z = torch.randn((B, T, H, 6 * D), generator=gen, device=dev).to(torch.bfloat16)
+    bias = torch.full((H, D), -4.0, device=dev)
+    outs = binding.gdn2_layer_gates_fwd(z, D, D, bias)
+    steps = max(5, args.steps)
+    f_ms = timed_ms(lambda: binding.gdn2_layer_gates_fwd(z, D, D, bias), steps, dev)
+    b_ms = timed_ms(lambda: binding.gdn2_layer_gates_bwd(z, *outs, D, D, bias), steps, dev)
+    th = B * T * H
+    fb, bb = th * 2 * 6 * D * 2, th * 3 * 6 * D * 2
+    out = {"workload": "layer-gates-bf16-b%dh%dt%dd%d" % (B, H, T, D), "fwd_ms": f_ms, "bwd_ms": b_ms,
+           "fwd_frac_of_hbm": fb / (f_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+           "bwd_frac_of_hbm": bb / (b_ms / 1e3) / 1e9 / pk["hbm_gbs"], "status": binding.gdn2_device_status()}
+    del z, outs
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_context_maps(binding, dev, args, T=16384, H=16, D=128):
+    """Per-rank cost of context parallelism on one piece (B = 1, T tokens, H heads): the piece's forward and
+    reverse maps against its own forward and fwd+bwd (what a rank runs anyway)."""
+    import torch
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    d = device_inputs(1, T, H, D, 8000, True, dev)
+    steps = max(3, args.steps // 4)
+    ws_map = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_MAP, 1, T, H, D, D, 64, binding.GDN2_BF16),
+                         dtype=torch.uint8, device=dev)
+    x = [d[n] for n in names]
+    fm = timed_ms(lambda: binding.gdn2_fwd_map(*x, ws=ws_map), steps, dev)
+    bm = timed_ms(lambda: binding.gdn2_bwd_map(*x, d["dout"], ws=ws_map), steps, dev)
+    M, N = binding.gdn2_fwd_map(*x, ws=ws_map)
+    af = timed_ms(lambda: binding.gdn2_state_affine(M, N, d["S0"]), steps, dev)
+    ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_BWD, 1, T, H, D, D, 64, binding.GDN2_BF16),
+                     dtype=torch.uint8, device=dev)
+    f = timed_ms(lambda: binding.gdn2_fwd(*x, d["S0"], save_states=True, ws=ws), steps, dev)
+    fb = timed_ms(lambda: (binding.gdn2_fwd(*x, d["S0"], save_states=True, ws=ws),
+                           binding.gdn2_bwd(*x, d["dout"], d["S0"], None, states_saved=True, ws=ws)), steps, dev)
+    out = {"piece": "b1h%dt%dd%d" % (H, T, D), "fwd_map_ms": fm, "bwd_map_ms": bm, "state_affine_ms": af,
+           "piece_fwd_ms": f, "piece_fwdbwd_ms": fb, "status": binding.gdn2_device_status(),
+           "note": "a rank of a context-parallel step runs its maps, one all-gather, P - 1 state_affine chain steps "
+                   "and its piece's forward (and backward); one GPU per call here, so no multi-GPU time"}
+    del d, ws, ws_map, M, N
+    torch.cuda.empty_cache()
+    return out
+
+
 SWEEP_TOKENS = 65536
 SWEEP_T = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
 
@@ -563,11 +619,13 @@ def main():
     full = args.B is None and args.T is None
     if not args.no_decode and full:
         decode = bench_decode(binding, dev)
-    reductions = None
+    reductions = layer_gates = cp_maps = None
     if not args.no_extra and full and world == 1:
         configs = measure_configs(binding, dev, args, d)
         sweep = measure_sweep(binding, dev, args)
         reductions = measure_reductions(binding, dev, d, args, ms_per_step)
+        layer_gates = measure_layer_gates(binding, dev, args, B, T, H)
+        cp_maps = measure_context_maps(binding, dev, args)
 
     line = None
     if rank == 0:
@@ -589,7 +647,8 @@ def main():
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_in_timed_region,
-                "decode": decode, "configs": configs, "sweep": sweep, "kda_overhead": reductions}
+                "decode": decode, "configs": configs, "sweep": sweep, "kda_overhead": reductions,
+                "layer_gates": layer_gates, "context_parallel_maps": cp_maps}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
