@@ -618,7 +618,8 @@ constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_G1 = 320, TM_G2 = 384, TM_G3 = 256, TM_G4 = 192,   // G3 = dKt^T (P and A paths), G4 = (Delta dS'^T)^T = dKh^T
     TM_GV = 448,                   // g[t] = exp(G) per key channel
     TM_HV = 128;                   // r[t] = 1/g, or exp(G_C - G) in a chunk with untame channels
-constexpr uint32_t LOAD_TOK = 7 * 64 * 128 * 2 + (uint32_t)TC_DELTA_BYTES;   // 7 token tiles, Delta^T
+constexpr uint32_t LOAD_GATE = 4 * 64 * 128 * 2;                             // b, q, k, log_alpha: the prep's
+constexpr uint32_t LOAD_REST = 3 * 64 * 128 * 2 + (uint32_t)TC_DELTA_BYTES;   // v, w, dout, Delta^T
 constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dS'^T: cp.async)
 }  // namespace cg
 
@@ -643,6 +644,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     unsigned char* PP = sm + OFF_PP;
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_load + 1;
+    uint64_t* bar_rest = bar_load + 2;
     uint64_t* bar_b = bar_load + 3;
     uint64_t* bar_pre = reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48);
 
@@ -661,43 +663,55 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const uint4 msk = *reinterpret_cast<const uint4*>(p.tp + (head * nc + c) * TC_WY_BYTES + TC_WY_MASK);
     bool ok = true;
     int next_unit = units;    // lane 0 of warp 9: the CTA's next unit (its atomic returns while this unit runs)
-    // The loads are issued by lane 0 of several warps at once (a TMA issue takes ~100 cycles); the
-    // barrier phase cannot complete before thread 0's arrival, which carries the expected bytes.
+    // The loads are issued by lane 0 of several warps at once (a TMA issue takes ~100 cycles); a barrier
+    // phase cannot complete before the arrival that carries its expected bytes. Two groups: the prep's
+    // inputs (b, q, k, log_alpha, into tiles no output is staged in) go out at once; the rest (v, w, dout,
+    // Delta^T, and S^T, T unless prefetched) after thread 0 has seen the previous unit's output stores read
+    // DU, DT and DDT, and land while the prep runs.
     // (*nxt is rewritten only after the next barriers: every thread has read it by then.)
     if (lane == 0) {
-        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
         switch (warp) {
         case 0:
-            tc::mbar_arrive_expect_tx(bar_load, prefetched ? LOAD_TOK : LOAD_TOK + LOAD_PRE);
+            tc::mbar_arrive_expect_tx(bar_load, LOAD_GATE);
             tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
             break;
         case 1: tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load); break;
         case 2: tma_tile(KH, C, 0, mk, b, h, t0, bar_load); break;
         case 3: tma_tile(KT, C, 0, mla, b, h, t0, bar_load); break;
-        case 4: tma_tile(DU, 2 * C, C, mv, b, h, t0, bar_load); break;
-        case 5: tma_tile(WW, C, 0, mw, b, h, t0, bar_load); break;
-        case 6: tma_tile(DU, 2 * C, 0, mdo, b, h, t0, bar_load); break;
-        case 7:
-            tc::bulk_load(DT, p.deltas + (head * nc + c) * TC_DELTA_BYTES, (uint32_t)TC_DELTA_BYTES, bar_load);
-            break;
         case 9: next_unit = (int)atomicAdd(p.counter, 1u); break;   // first needed at the G MMAs
+        default: break;
+        }
+    }
+    if (tid == 0) {
+        if (!prefetched && !tc::flag_wait(p.flags + head * nc + c, 1u)) {   // dS'^T of this chunk: the reverse pass
+            ok = false;
+            atomicOr(&g_bwd_error, 8u);
+            atomicExch(p.counter + 1, 1u);
+        }
+        tc::bulk_wait_read();   // the previous unit's dq, dk, db, dlog_alpha stores have read DU, DT, DDT
+    }
+    __syncthreads();   // orders thread 0's acquire and its wait before the loads and copies below
+    if (lane == 0) {
+        const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
+        switch (warp) {
+        case 4:
+            tc::mbar_arrive_expect_tx(bar_rest, prefetched ? LOAD_REST : LOAD_REST + LOAD_PRE);
+            tma_tile(DU, 2 * C, C, mv, b, h, t0, bar_rest);
+            break;
+        case 5: tma_tile(WW, C, 0, mw, b, h, t0, bar_rest); break;
+        case 6: tma_tile(DU, 2 * C, 0, mdo, b, h, t0, bar_rest); break;
+        case 7:
+            tc::bulk_load(DT, p.deltas + (head * nc + c) * TC_DELTA_BYTES, (uint32_t)TC_DELTA_BYTES, bar_rest);
+            break;
         case 8:
             if (!prefetched) {
-                tc::bulk_load(STt, p.states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_load);
-                tc::bulk_load(TT, src, TILE_C, bar_load);
+                tc::bulk_load(STt, p.states + (head * nc + c) * TC_STATE_BYTES, (uint32_t)TC_STATE_BYTES, bar_rest);
+                tc::bulk_load(TT, src, TILE_C, bar_rest);
             }
             break;
         default: break;
         }
     }
-    if (tid == 0 && !prefetched) {   // dS'^T of this chunk comes from the reverse pass: wait for its flag
-        if (!tc::flag_wait(p.flags + head * nc + c, 1u)) {
-            ok = false;
-            atomicOr(&g_bwd_error, 8u);
-            atomicExch(p.counter + 1, 1u);
-        }
-    }
-    __syncthreads();   // orders thread 0's acquire before every thread's copy of the dS'^T image
     {   // the reverse pass's images of this chunk: dS'^T (unless prefetched) and dDelta^T
         if (!prefetched) {
             const unsigned char* src = p.dstates + (head * nc + c) * TC_STATE_BYTES;
@@ -714,13 +728,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const uint32_t lane_base = tmem + ((uint32_t)(tm_quarter(warp) * 32) << 16);
     const int jrow = 32 * tm_quarter(warp) + lane, cpart = 32 * tm_part(warp);      // lane row, column quarter
     (void)jrow;
-    ok = tc::mbar_wait(bar_load, ph.load) && ok;
+    ok = tc::mbar_wait(bar_load, ph.load) && ok;   // the prep's inputs
     ph.load ^= 1;
-    if (prefetched) {
-        ok = tc::mbar_wait(bar_pre, ph.pre) && ok;
-        ph.pre ^= 1;
-    }
-    tc::cp_async_wait_all();
     auto wait_mma = [&]() {
         ok = tc::mbar_wait(bar_mma, ph.mma) && ok;
         ph.mma ^= 1;
@@ -743,6 +752,13 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const bool untame = ((ich < 64 ? (ich < 32 ? msk.x : msk.y) : (ich < 96 ? msk.z : msk.w)) >> (ich & 31)) & 1u;
     const float gC = grad_prep(QE, KH, KT, reinterpret_cast<float*>(PP), tid, lane_base + TM_GV, lane_base + TM_HV,
                                untame, khm);   // PP: scratch
+    ok = tc::mbar_wait(bar_rest, ph.k) && ok;   // the rest of the unit's tiles, loaded during the prep
+    ph.k ^= 1;
+    if (prefetched) {
+        ok = tc::mbar_wait(bar_pre, ph.pre) && ok;
+        ph.pre ^= 1;
+    }
+    tc::cp_async_wait_all();
     sync_for_mma();
 
     // ---- dU = T^T dDelta (M=64)
@@ -996,11 +1012,10 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     }
     tc::fence_async_smem();
     __syncthreads();
-    if (tid == 0) {   // dlog_alpha; every store has read its tile before the next unit's loads reuse them
+    if (tid == 0) {   // dlog_alpha; the next unit waits for the stores' reads before it reuses their tiles
         tc::tma_store_4d(mdla, 0, h, t0, b, DU + C * 128);
         tc::tma_store_4d(mdla, 64, h, t0, b, DU + C * 128 + 2 * C * 128);
         tc::bulk_commit();
-        tc::bulk_wait_read();
     }
     if (!ok) atomicOr(&g_bwd_error, 4u);
     tc::tc_fence_before();
@@ -1078,6 +1093,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
             u = nxt->unit;   // written by thread 0 before the unit's last barrier
             pre = nxt->prefetched != 0;
         }
+        if (tid == 0) tc::bulk_wait_read();   // the last unit's output stores have read their tiles
     }
     tc::tc_fence_before();
     __syncthreads();
