@@ -946,42 +946,83 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 }
 
 // Segment start states S_2 .. S_{R-1} from S_1 and the segment maps, S_{s+1} = M_s S_s + N_s, in fp32. The value
-// columns of a state never mix, so CTA (head, block of 16 columns) runs the whole prefix for its columns; thread
-// (row i = tid / 2, 8 columns) keeps its sums in registers.
-__global__ void __launch_bounds__(256) split_prefix_kernel(float* sbuf, int R) {
-    __shared__ float Sc[D][16];
+// columns of a state never mix, so CTA (head, block of 16 columns) runs the whole prefix for its columns. Thread
+// (row group rq = tid / 4: rows rq + 32 r, r < 4; column quarter cq = tid % 4: 4 columns) keeps a 4 x 4 block of
+// sums in registers, so one pass over the 128 terms of a product costs 8 shared-memory vector loads per 64
+// FMAs. M_s goes to shared memory by cp.async, the next step's while this one runs (two buffers; rows padded
+// to 132 floats so that the 8 rows a warp reads at once fall in distinct bank groups).
+constexpr int PREFIX_LD = D + 4;
+constexpr int PREFIX_THREADS = 128;
+constexpr uint32_t PREFIX_SMEM = (uint32_t)(2 * D * PREFIX_LD + D * 16) * sizeof(float);
+static_assert(D * D / 4 == 32 * PREFIX_THREADS && D == 4 * 32, "prefix thread mapping");
+__global__ void __launch_bounds__(PREFIX_THREADS) split_prefix_kernel(float* sbuf, int R) {
+    extern __shared__ float4 prefix_smem[];
+    float* Mbuf = reinterpret_cast<float*>(prefix_smem);   // 2 x [D][PREFIX_LD]
+    float(*Sc)[16] = reinterpret_cast<float(*)[16]>(Mbuf + 2 * D * PREFIX_LD);
     if (!GDN2_IN(g_fwd_error, R >= 4 && R <= SPLIT_R_MAX)) return;   // the slots of a head hold R <= SPLIT_R_MAX
     const int head = blockIdx.x / (D / 16), j0 = (blockIdx.x % (D / 16)) * 16;
-    const int tid = threadIdx.x, i = tid >> 1, jh = (tid & 1) * 8;
+    const int tid = threadIdx.x, cq = tid & 3, rq = tid >> 2;
     float* base = sbuf + (size_t)head * SPLIT_MATS_PER_HEAD * D * D;
     auto mat = [&](int kind, int s) { return base + (size_t)((kind == 0 ? 0 : (kind == 1 ? R - 1 : 2 * R - 3)) + s - 1) * D * D; };
-    const float* S1 = mat(0, 1);
+    auto stage = [&](int s, int buf) {   // M_s -> buffer buf, 32 16-byte copies per thread
+        const float4* src = reinterpret_cast<const float4*>(mat(2, s));
+        float* dst = Mbuf + buf * D * PREFIX_LD;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) Sc[i][jh + e] = S1[i * D + j0 + jh + e];
-    for (int s = 1; s <= R - 2; ++s) {
-        __syncthreads();
-        const float* N = mat(1, s);
-        const float* M = mat(2, s);
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = N[i * D + j0 + jh + e];
-#pragma unroll 4
-        for (int l = 0; l < D; l += 4) {
-            const float4 m = *reinterpret_cast<const float4*>(M + i * D + l);
-            const float mv[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] += mv[u] * Sc[l + u][jh + e];
+        for (int e = 0; e < 32; ++e) {
+            const int idx = tid + PREFIX_THREADS * e, r = idx >> 5, c4 = idx & 31;
+            tc::cp_async16_cg(dst + r * PREFIX_LD + 4 * c4, src + idx);
         }
-        __syncthreads();
+        tc::cp_async_commit();
+    };
+    stage(1, 0);
+    const float* S1 = mat(0, 1);
+    for (int e = tid; e < D * 16; e += PREFIX_THREADS) Sc[e >> 4][e & 15] = S1[(e >> 4) * D + j0 + (e & 15)];
+    for (int s = 1; s <= R - 2; ++s) {
+        const int buf = (s - 1) & 1;
+        const float* N = mat(1, s);
+        float acc[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float4 n = *reinterpret_cast<const float4*>(N + (size_t)(rq + 32 * r) * D + j0 + 4 * cq);
+            acc[r][0] = n.x; acc[r][1] = n.y; acc[r][2] = n.z; acc[r][3] = n.w;
+        }
+        if (s + 1 <= R - 2) {   // the next step's M goes to the other buffer (read last in step s - 1)
+            stage(s + 1, buf ^ 1);
+            tc::cp_async_wait_but1();
+        } else {
+            tc::cp_async_wait_all();
+        }
+        __syncthreads();   // every thread's copies of M_s, and S_s in Sc
+        const float* Ms = Mbuf + buf * D * PREFIX_LD;
+#pragma unroll 2
+        for (int l = 0; l < D; l += 4) {
+            float4 m[4], sv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) m[r] = *reinterpret_cast<const float4*>(Ms + (rq + 32 * r) * PREFIX_LD + l);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) sv[u] = *reinterpret_cast<const float4*>(&Sc[l + u][4 * cq]);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float mr[4] = {m[r].x, m[r].y, m[r].z, m[r].w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    acc[r][0] += mr[u] * sv[u].x;
+                    acc[r][1] += mr[u] * sv[u].y;
+                    acc[r][2] += mr[u] * sv[u].z;
+                    acc[r][3] += mr[u] * sv[u].w;
+                }
+            }
+        }
+        __syncthreads();   // every thread has read Sc and this buffer
         float* Sn = mat(0, s + 1);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            Sc[i][jh + e] = acc[e];
-            Sn[i * D + j0 + jh + e] = acc[e];
+        for (int r = 0; r < 4; ++r) {
+            const int i = rq + 32 * r;
+            *reinterpret_cast<float4*>(&Sc[i][4 * cq]) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+            *reinterpret_cast<float4*>(Sn + (size_t)i * D + j0 + 4 * cq) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
         }
     }
+    tc::cp_async_wait_all();
 }
 
 // Number of segments a head's chunks are cut into (0: none). Only when the heads leave most CTA slots idle
@@ -997,8 +1038,10 @@ int split_segments(int BH, int nc, int slots, bool have_buf) {
 }  // namespace
 
 cudaError_t split_prefix_launch(float* sbuf, int R, int BH, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(split_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREFIX_SMEM);
+    if (e != cudaSuccess) return e;
     TraceScope trace(K_SPLIT_PREFIX, s);
-    split_prefix_kernel<<<BH * (D / 16), 256, 0, s>>>(sbuf, R);
+    split_prefix_kernel<<<BH * (D / 16), PREFIX_THREADS, PREFIX_SMEM, s>>>(sbuf, R);
     return cudaGetLastError();
 }
 

@@ -322,6 +322,8 @@ __device__ __forceinline__ void cp_async16_cg(void* dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// all committed groups but the most recent one are complete
+__device__ __forceinline__ void cp_async_wait_but1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // ------------------------------------------------------------ flags between CTAs of one launch
 // Publishing: every thread writes its data, __syncthreads(), then one thread calls flag_release
