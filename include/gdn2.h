@@ -290,8 +290,9 @@ size_t gdn2_no_alloc_scratch_bytes(void);
  * Tensor-core path only (dt = GDN2_BF16, Dk = Dv = 128); other problems return
  * GDN2_ERR_UNSUPPORTED. T = 0 gives M = A = I and N = Bm = 0. Workspace:
  * gdn2_workspace_size(GDN2_OP_MAP, ...) bytes, 256-byte aligned (the WY images
- * of the piece and their flags). The maps go to the caller's buffers; nothing
- * else is written.
+ * of the piece and their flags; with few heads and a long piece also the maps
+ * of its segments, which run in parallel and are then composed). The maps go
+ * to the caller's buffers; nothing else outside the workspace is written.
  */
 gdn2_status gdn2_fwd_map(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
                          const void* w, float* M, float* N, int B, int T, int H, int Dk, int Dv, int chunk,

@@ -266,7 +266,7 @@ __device__ __forceinline__ float* rsplit_mat(const BwdParams& p, int head, int k
     return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
 }
 __device__ __forceinline__ int rev_task_count(const BwdParams& p) {
-    if (p.phase == 5) return 2 * p.BH;
+    if (p.phase == 5) return 2 * p.BH * (p.split_R ? p.split_R : 1);
     if (!p.split_R) return p.BH;
     return p.phase == 1 ? p.BH * (1 + 2 * (p.split_R - 2)) : p.BH * (p.split_R - 1);
 }
@@ -275,6 +275,14 @@ __device__ RevTask rev_task_at(const BwdParams& p, int t) {
     k.head = t % p.BH;
     const size_t hd = (size_t)k.head * D * D;
     if (p.phase == 5) {   // the whole sequence as one piece: B from a zero end gradient, A from the identity
+        if (p.split_R) {      // per segment j: B_j into slot j, A_j into slot R + j (slot-major: [slot][BH][D][D])
+            const int R = p.split_R, j = t / p.BH, s2 = j < R ? j : j - R;
+            k.c_lo = seg_begin(s2, p.nc, R);
+            k.c_hi = (s2 == R - 1 ? p.nc : seg_begin(s2 + 1, p.nc, R)) - 1;
+            if (j >= R) { k.ident = true; k.zero_do = true; }
+            k.fin = p.sbuf + ((size_t)j * p.BH + k.head) * D * D;
+            return k;
+        }
         k.c_hi = p.nc - 1; k.c_lo = 0;
         if (t < p.BH) {
             k.fin = p.map_B + hd;
@@ -1133,13 +1141,33 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     p.flags = a.flags; p.counter = a.flags + units;
     if ((e = cudaMemsetAsync(a.flags, 0, ((size_t)units + 2) * sizeof(unsigned int), s)) != cudaSuccess) return e;
 
-    if (a.map_A && a.map_B) {   // reverse maps only: the reverse pass of every head twice, no gradients
+    if (a.map_A && a.map_B) {   // reverse maps only: the reverse pass of every head (or segment) twice, no gradients
         BwdParams pm = p;
         pm.phase = 5; pm.grad = 0; pm.join = 0; pm.map_A = a.map_A; pm.map_B = a.map_B;
-        pm.nrev = 2 * BH < slots ? 2 * BH : slots;
-        TraceScope trace(K_CHUNK_BWD, s);
-        chunk_bwd_kernel<<<pm.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pm);
-        return cudaGetLastError();
+        const int R = map_segments_for(BH, nc, slots, a.sbuf != nullptr);
+        pm.split_R = R;
+        pm.sbuf = a.sbuf;
+        const int ntasks = 2 * BH * (R ? R : 1);
+        pm.nrev = ntasks < slots ? ntasks : slots;
+        {
+            TraceScope trace(K_CHUNK_BWD, s);
+            chunk_bwd_kernel<<<pm.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pm);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (!R) return cudaSuccess;
+        // compose from the last segment: B = A_0 (... (A_{R-2} B_{R-1} + B_{R-2}) ...) + B_0, A = A_0 A_1 ... A_{R-1}
+        const size_t DD = (size_t)D * D;
+        auto slot = [&](int j) { return a.sbuf + (size_t)j * BH * DD; };
+        for (int s2 = R - 2; s2 >= 0; --s2) {
+            const bool first = s2 == R - 2;
+            if ((e = state_affine_launch(slot(R + s2), slot(s2), first ? slot(R - 1) : a.map_B, a.map_B, BH, D, D, s)) !=
+                cudaSuccess)
+                return e;
+            if ((e = state_affine_launch(slot(R + s2), nullptr, first ? slot(2 * R - 1) : a.map_A, a.map_A, BH, D, D, s)) !=
+                cudaSuccess)
+                return e;
+        }
+        return cudaSuccess;
     }
     const int R = split_segments_for(BH, nc, slots, a.sbuf != nullptr);
     if (R) {   // the last segments and the segment maps, the prefix, then the other segments with the gradients

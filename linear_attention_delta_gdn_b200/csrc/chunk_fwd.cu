@@ -139,7 +139,7 @@ __device__ __forceinline__ float* split_mat(const FwdParams& p, int head, int ki
     return p.sbuf + ((size_t)head * SPLIT_MATS_PER_HEAD + idx) * D * D;
 }
 __device__ __forceinline__ int task_count(const FwdParams& p) {
-    if (p.phase == 5) return 2 * p.BH;
+    if (p.phase == 5) return 2 * p.BH * (p.split_R ? p.split_R : 1);
     if (!p.split_R) return p.BH;
     return p.phase == 1 ? p.BH * (1 + 2 * (p.split_R - 2)) : p.BH * (p.split_R - 1);
 }
@@ -148,6 +148,13 @@ __device__ Task task_at(const FwdParams& p, int t) {
     k.head = t % p.BH;
     const size_t hd = (size_t)k.head * D * D;
     if (p.phase == 5) {   // the whole sequence as one piece: N from a zero start, M from the identity without input
+        if (p.split_R) {      // per segment j: N_j into slot j, M_j into slot R + j (slot-major: [slot][BH][D][D])
+            const int R = p.split_R, j = t / p.BH, s2 = j < R ? j : j - R;
+            k.c0 = seg_begin(s2, p.nc, R); k.c1 = s2 == R - 1 ? p.nc : seg_begin(s2 + 1, p.nc, R);
+            if (j >= R) { k.ident = true; k.zero_u = true; }
+            k.fin = p.sbuf + ((size_t)j * p.BH + k.head) * D * D;
+            return k;
+        }
         k.c0 = 0; k.c1 = p.nc;
         if (t < p.BH) {
             k.fin = p.map_N + hd;
@@ -1032,7 +1039,7 @@ int split_segments(int BH, int nc, int slots, bool have_buf) {
     int R = (slots / BH - 1) / 2 + 2;   // phase 1 runs BH (1 + 2 (R - 2)) chains at once
     if (R > SPLIT_R_MAX) R = SPLIT_R_MAX;
     if (R > nc / TC_SPLIT_MIN_CHUNKS_PER_SEG) R = nc / TC_SPLIT_MIN_CHUNKS_PER_SEG;
-    return R < 4 ? 0 : R;
+    return R < 4 ? 0 : R;   // three segments lose in the backward (measured at B2 H16 T32K)
 }
 
 }  // namespace
@@ -1046,6 +1053,16 @@ cudaError_t split_prefix_launch(float* sbuf, int R, int BH, cudaStream_t s) {
 }
 
 int split_segments_for(int BH, int nc, int slots, bool have_buf) { return split_segments(BH, nc, slots, have_buf); }
+
+// Segments of a piece's map computation: its 2 B*H chains (N and M, or B and A) become 2 B*H R chains over
+// R segments, composed afterwards (R - 1 steps of gdn2_state_affine per map); as many as the CTA slots hold.
+int map_segments_for(int BH, int nc, int slots, bool have_buf) {
+    if (!have_buf || split_disabled() || BH <= 0 || BH > TC_SPLIT_MAX_BH) return 0;
+    int R = slots / (2 * BH);
+    if (R > SPLIT_R_MAX) R = SPLIT_R_MAX;
+    if (R > nc / TC_SPLIT_MIN_CHUNKS_PER_SEG) R = nc / TC_SPLIT_MIN_CHUNKS_PER_SEG;
+    return R < 2 ? 0 : R;
+}
 
 // The producers alone (with_maps: then per head two chains over the whole sequence, a piece of a longer one:
 // N from a zero start with the inputs, M from the identity without input).
@@ -1078,17 +1095,34 @@ static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool
     if (!with_maps) return cudaSuccess;
     FwdParams pc = p;
     pc.phase = 5; pc.nprod = 0; pc.map_N = a.map_N; pc.map_M = a.map_M;
-    pc.ncons = 2 * BH < slots ? 2 * BH : slots;
-    TraceScope trace(K_CHUNK_FWD, s);
-    chunk_fwd_kernel<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
-    return cudaGetLastError();
+    const int R = map_segments_for(BH, nc, slots, a.sbuf != nullptr);
+    pc.split_R = R;
+    pc.sbuf = a.sbuf;
+    const int ntasks = 2 * BH * (R ? R : 1);
+    pc.ncons = ntasks < slots ? ntasks : slots;
+    {
+        TraceScope trace(K_CHUNK_FWD, s);
+        chunk_fwd_kernel<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (!R) return cudaSuccess;
+    // compose the segments in order: N = M_{R-1} (... (M_1 N_0 + N_1) ...) + N_{R-1}, M = M_{R-1} ... M_1 M_0
+    const size_t DD = (size_t)D * D;
+    auto slot = [&](int j) { return a.sbuf + (size_t)j * BH * DD; };
+    for (int s2 = 1; s2 < R; ++s2) {
+        if ((e = state_affine_launch(slot(R + s2), slot(s2), s2 == 1 ? slot(0) : a.map_N, a.map_N, BH, D, D, s)) != cudaSuccess)
+            return e;
+        if ((e = state_affine_launch(slot(R + s2), nullptr, s2 == 1 ? slot(R) : a.map_M, a.map_M, BH, D, D, s)) != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t chunk_fwd_map_launch(const ChunkFwdArgs& a, cudaStream_t s) { return fwd_pieces_launch(a, s, true); }
 cudaError_t chunk_fwd_wy_launch(const ChunkFwdArgs& a, cudaStream_t s) { return fwd_pieces_launch(a, s, false); }
 
 size_t chunk_fwd_split_bytes(int BH, int nc) {
-    if (BH > TC_SPLIT_MAX_BH || nc < TC_SPLIT_MIN_CHUNKS_PER_SEG * 4) return 0;
+    if (BH > TC_SPLIT_MAX_BH || nc < TC_SPLIT_MIN_CHUNKS_PER_SEG * 2) return 0;   // also the maps' segments (R >= 2)
     return (size_t)BH * SPLIT_MATS_PER_HEAD * TC_D * TC_D * sizeof(float);
 }
 

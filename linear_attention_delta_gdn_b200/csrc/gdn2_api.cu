@@ -92,6 +92,11 @@ size_t tc_split_offset(const Dims& d, bool with_states) {
     return tc_flags_offset(d, with_states) + align256(tc_units(d) * sizeof(unsigned int));
 }
 
+// GDN2_OP_MAP: [WY images][flags, work counter, abort word][segment maps of a long piece]
+size_t map_sbuf_offset(const Dims& d) {
+    return align256(tc_units(d) * TC_WY_BYTES) + align256((tc_units(d) + 2) * sizeof(unsigned int));
+}
+
 size_t bwd_extra_bytes(const Dims& d, gdn2_dtype dt) {
     if (tc_path(dt, d.Dk, d.Dv))   // dZ and dDelta images, ready flags, work counter, abort word
         return tc_units(d) * (TC_STATE_BYTES + TC_DELTA_BYTES) + align256((tc_units(d) + 2) * sizeof(unsigned int));
@@ -182,9 +187,8 @@ size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int 
     case GDN2_OP_FWD: return tc_path(dt, Dk, Dv) ? align256(tc_wy_bytes(d)) : 0;
     case GDN2_OP_FWD_SAVE: return align256(states_bytes(d, dt));
     case GDN2_OP_BWD: return align256(states_bytes(d, dt)) + align256(bwd_extra_bytes(d, dt));
-    case GDN2_OP_MAP:   // WY images, then ready flags with the backward's work counter and abort word
-        return tc_path(dt, Dk, Dv) ? align256(tc_units(d) * TC_WY_BYTES) + align256((tc_units(d) + 2) * sizeof(unsigned int))
-                                   : 0;
+    case GDN2_OP_MAP:   // WY images, ready flags with the backward's work counter and abort word, segment maps
+        return tc_path(dt, Dk, Dv) ? map_sbuf_offset(d) + tc_split_bytes(d) : 0;
     }
     return 0;
 }
@@ -353,6 +357,7 @@ gdn2_status gdn2_fwd_map(const void* q, const void* k, const void* v, const void
     a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
     a.wy = wsb;
     a.flags = reinterpret_cast<unsigned int*>(wsb + align256(tc_units(d) * TC_WY_BYTES));
+    a.sbuf = tc_split_bytes(d) ? reinterpret_cast<float*>(wsb + map_sbuf_offset(d)) : nullptr;
     a.map_N = N; a.map_M = M;
     return cuda_status(chunk_fwd_launch(a, s), "gdn2_fwd_map");
 }
@@ -380,6 +385,7 @@ gdn2_status gdn2_bwd_map(const void* q, const void* k, const void* v, const void
     a.d = d;
     a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w; a.dout = dout;
     a.tp = wsb; a.flags = flags;
+    a.sbuf = tc_split_bytes(d) ? reinterpret_cast<float*>(wsb + map_sbuf_offset(d)) : nullptr;
     a.map_A = A; a.map_B = Bm;
     return cuda_status(chunk_bwd_launch(a, s), "gdn2_bwd_map");
 }

@@ -65,6 +65,9 @@ size_t chunk_fwd_split_bytes(int BH, int nc);
 // The segment count for a problem (0: no split), and the fp32 prefix over the segment maps, shared by the
 // forward and the backward (whose reverse segments use the same per-head layout of states and maps).
 int split_segments_for(int BH, int nc, int slots, bool have_buf);
+// Segments of the maps of a piece (gdn2_fwd_map / gdn2_bwd_map), in the same workspace region, slot-major
+// ([slot][B*H][128][128]): 0 for none.
+int map_segments_for(int BH, int nc, int slots, bool have_buf);
 cudaError_t split_prefix_launch(float* sbuf, int R, int BH, cudaStream_t s);
 bool split_disabled();   // environment variable GDN2_NO_SPLIT set: keep every head on one chain
 

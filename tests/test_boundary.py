@@ -71,6 +71,9 @@ def test_workspace_sizes(L):
             assert ws(op, 2, 300, 3, 128, 128, c, 1) == ws(op, 2, 300, 3, 128, 128, 64, 1)
     # the maps of a sequence piece: WY images, then flags with the work counter and abort word
     assert ws(3, 4, 4096, 16, 128, 128, 64, 1) == units * 82944 + units * 4 + 256
+    # a long piece with few heads adds its segment maps (19 fp32 128 x 128 matrices per head)
+    u1 = 1 * 2 * 256
+    assert ws(3, 1, 16384, 2, 128, 128, 64, 1) == u1 * 82944 + u1 * 4 + 256 + 2 * 19 * 128 * 128 * 4
     assert ws(3, 1, 256, 2, 64, 64, 64, 0) == 0
     # invalid problems report zero
     assert ws(1, 0, 16, 1, 64, 64, 64, 1) == 0

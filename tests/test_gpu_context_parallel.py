@@ -39,13 +39,19 @@ def _oracle_maps(oracle_mod, f):
     return M, N, A, Bm
 
 
-@pytest.mark.parametrize("T,strong", [(700, False), (64, False), (1, False), (300, True)])
-def test_maps_against_oracle(oracle_mod, T, strong):
-    x = make_inputs(2, T, 2, 128, 128, seed=2100 + T, dtype="bf16", with_do=True)
-    if strong:   # a few channels decay by e^-20 per token (exact pair terms on the tensor-core path)
+@pytest.mark.parametrize("B,T,H,decay", [(2, 700, 2, "recipe"), (2, 64, 2, "recipe"), (2, 1, 2, "recipe"),
+                                         (2, 300, 2, "strong"), (1, 4100, 3, "slow")])
+def test_maps_against_oracle(oracle_mod, B, T, H, decay):
+    """The maps against the oracle's. The "slow" case is a 65-chunk piece with 3 heads, whose maps are computed
+    over segments and composed; its decay is the recipe's / 100 so that M (a product of 4100 transitions) stays
+    far from fp32 underflow."""
+    x = make_inputs(B, T, H, 128, 128, seed=2100 + T, dtype="bf16", with_do=True)
+    if decay == "strong":   # a few channels decay by e^-20 per token (exact pair terms on the tensor-core path)
         la = x["log_alpha"].float()
         la[..., [3, 64, 101]] = -20.0
         x["log_alpha"] = la.to(torch.bfloat16)
+    elif decay == "slow":
+        x["log_alpha"] = (x["log_alpha"].float() / 100.0).to(torch.bfloat16)
     d = {n: t.cuda() for n, t in x.items()}
     M, N = binding.gdn2_fwd_map(*(d[n] for n in NAMES))
     A, Bm = binding.gdn2_bwd_map(*(d[n] for n in NAMES), d["dout"])
