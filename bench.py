@@ -494,7 +494,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
     ap.add_argument("--no-extra", action="store_true", help="skip the extra configs and the length sweep")
     ap.add_argument("--B", type=int, default=None, help="override the batch size (small profiling cases)")
@@ -540,10 +540,10 @@ def main():
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(inp):
-        binding.gdn2_fwd(*(inp[n] for n in names), None, chunk=chunk, save_states=True, ws=ws, o=o, ST=ST)
+    def step(inp, o_=o, grads_=grads):
+        binding.gdn2_fwd(*(inp[n] for n in names), None, chunk=chunk, save_states=True, ws=ws, o=o_, ST=ST)
         binding.gdn2_bwd(*(inp[n] for n in names), inp["dout"], None, None, chunk=chunk, states_saved=True,
-                         ws=ws, grads=grads)
+                         ws=ws, grads=grads_)
 
     for _ in range(max(3, args.warmup)):
         step(d)
@@ -578,23 +578,44 @@ def main():
     tokens_per_step = B * T
     value = aggregate_tokens_per_s(world, tokens_per_step, ms_per_step)
 
-    # ---- end to end through host buffers: H2D inputs, fwd + bwd, D2H o and gradients
+    # ---- end to end through host buffers: every step copies its inputs in from pinned host memory, runs fwd + bwd
+    # and copies o and the six gradients back. A training loop's pipeline: two device buffer sets and three streams
+    # (copy in, compute, copy out), so that one step's copies overlap the neighbouring steps' kernels and the two
+    # copy directions overlap each other.
+    gnames = ("dq", "dk", "dv", "dlog_alpha", "db", "dw")
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    outs = [o] + [grads[n] for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw")]
-    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    d2h = sum(t.numel() * t.element_size() for t in outs)
+    d2h = (o.numel() + sum(grads[n].numel() for n in gnames)) * o.element_size()
+    dsets = [d, {n: torch.empty_like(t) for n, t in d.items()}]
+    osets = [(o, grads), (torch.empty_like(o), {n: torch.empty_like(t) for n, t in grads.items()})]
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in [o] + [grads[n] for n in gnames]]
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nsteps = max(1, args.e2e_steps)
+    ev = {k: [torch.cuda.Event() for _ in range(nsteps)] for k in ("in", "cmp", "out")}
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
-    e_start.record(stream)
-    for _ in range(args.e2e_steps):
-        for n in pinned:
-            d[n].copy_(pinned[n], non_blocking=True)
-        step(d)
-        for h_, t in zip(host_out, outs):
-            h_.copy_(t, non_blocking=True)
-    e_end.record(stream)
+    e_start.record(s_in)
+    for i in range(nsteps):
+        k = i % 2
+        if i >= 2:
+            s_in.wait_event(ev["cmp"][i - 2])    # the set's inputs have been consumed
+        with torch.cuda.stream(s_in):
+            for n in pinned:
+                dsets[k][n].copy_(pinned[n], non_blocking=True)
+            ev["in"][i].record(s_in)
+        s_cmp.wait_event(ev["in"][i])
+        if i >= 2:
+            s_cmp.wait_event(ev["out"][i - 2])   # the set's outputs have been copied out
+        with torch.cuda.stream(s_cmp):
+            step(dsets[k], osets[k][0], osets[k][1])
+            ev["cmp"][i].record(s_cmp)
+        s_out.wait_event(ev["cmp"][i])
+        with torch.cuda.stream(s_out):
+            for h_, t in zip(host_out, [osets[k][0]] + [osets[k][1][n] for n in gnames]):
+                h_.copy_(t, non_blocking=True)
+            ev["out"][i].record(s_out)
+    e_end.record(s_out)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / max(1, args.e2e_steps), dist, dev)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / nsteps, dist, dev)
     e2e_value = aggregate_tokens_per_s(world, tokens_per_step, e2e_ms)
 
     # ---- roofline of the dominant kernel (device time summed over the timed region)
