@@ -61,6 +61,15 @@
  *     test hook of the forward's two-launch form: the producer launch is left
  *     out, so the consumers' ready-flag waits run out and gdn2_device_status
  *     reports GDN2_ERR_TIMEOUT; outputs are then not valid.
+ *     With few heads (B*H <= 32) and long sequences (at least 64 chunks) each
+ *     head's chunks are cut into 4 to 8 segments that run on separate CTAs
+ *     (the segments' affine state maps, a prefix over them, then the segments
+ *     from their start states): more launches per call, the same results up
+ *     to rounding. GDN2_NO_SPLIT (same rule) keeps one chain per head.
+ *   - A debug build of the library (libgdn2_debug.so, compiled with
+ *     -DGDN2_DEBUG) checks the kernels' task, segment and unit indexes; a
+ *     failed check skips the access and gdn2_device_status reports it as
+ *     GDN2_ERR_INVALID ("index check"). The release build has no such checks.
  */
 #ifndef GDN2_H
 #define GDN2_H
@@ -105,8 +114,9 @@ typedef enum gdn2_op {
  * Returns 0 for an invalid or unsupported problem and for a forward that needs
  * no workspace. The workspace must be 256-byte aligned; its contents on entry
  * do not matter. On the tensor-core path it is about 81 KB per 64-token
- * chunk and head for GDN2_OP_FWD, 129 KB for GDN2_OP_FWD_SAVE and 177 KB for
- * GDN2_OP_BWD.
+ * chunk and head for GDN2_OP_FWD and GDN2_OP_MAP, 129 KB for GDN2_OP_FWD_SAVE
+ * and 177 KB for GDN2_OP_BWD; with B*H <= 32 and at least 32 chunks, 1.2 MB
+ * per head is added for the segment states and maps of long sequences.
  */
 size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int chunk,
                            gdn2_dtype dt);
