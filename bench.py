@@ -20,6 +20,8 @@ Besides the headline step, the line carries (rank 0, N=1):
     kernels at the headline shape, against the GDN-2 step;
   * ``layer_gates``: the layer's gate-activation kernels (forward and backward)
     at the headline shape, against the HBM roofline;
+  * ``layer_step``: the whole layer (projections on cuBLAS, gate kernels, the
+    operator) forward + backward at d_model = 2048, with the library's share;
   * ``context_parallel_maps``: a context-parallel rank's map kernels on one
     16K-token piece, beside that piece's own forward and fwd+bwd;
   * ``cpu_baseline``: the fp64 oracle timed on a bounded sample of the headline
@@ -413,6 +415,48 @@ def measure_layer_gates(binding, dev, args, B, T, H, D=128):
     return out
 
 
+def measure_layer_step(binding, dev, args, B, T, H, D=128):
+    """The layer around the operator (Gdn2Layer: input projection on cuBLAS, gate kernels, the operator,
+    output projection) forward + backward through autograd at d_model = H * D, bf16: ms per step, tokens/s, the
+    projections' tensor-core throughput and the library kernels' share of the step (trace)."""
+    import torch
+    from linear_attention_delta_gdn_b200.layer import Gdn2Layer
+    pk = peaks()
+    torch.manual_seed(9000)
+    dm = H * D
+    layer = Gdn2Layer(dm, H, D, D, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(9001)
+    x = torch.randn((B, T, dm), generator=gen, device=dev).to(torch.bfloat16).requires_grad_(True)
+    dy = torch.randn((B, T, dm), generator=gen, device=dev).to(torch.bfloat16)
+
+    def step():
+        y, _ = layer(x)
+        y.backward(dy)
+
+    steps = max(3, args.steps // 4)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    binding.trace_read()
+    binding.trace_enable(True)
+    ms = timed_ms(step, steps, dev, warmup=0)
+    binding.trace_enable(False)
+    kern = {k: v[1] / steps for k, v in binding.trace_read().items()}   # device ms per step of each library kernel
+    ntok = B * T
+    proj_flop = 3 * 2 * ntok * dm * (H * (4 * D + 2 * D) + dm)   # in + out projections, forward and two backward GEMMs
+    lib_ms = sum(kern.values())
+    out = {"workload": "layer-bf16-b%dt%dh%dd%d-dmodel%d" % (B, T, H, D, dm), "ms": ms, "tokens_per_s": ntok / (ms / 1e3),
+           "library_kernels_ms": kern, "library_share": lib_ms / ms,
+           "projection_tflops": proj_flop / ((ms - lib_ms) / 1e3) / 1e12 if ms > lib_ms else None,
+           "peak_bf16_tflops": pk.get("bf16_tflops"), "status": binding.gdn2_device_status(),
+           "note": "projections are cuBLAS GEMMs through torch.matmul (their throughput is over the step time the "
+                   "library's kernels leave); the gates, the operator and their backward are the library's kernels"}
+    del layer, x, dy
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_context_maps(binding, dev, args, T=16384, H=16, D=128):
     """Per-rank cost of context parallelism on one piece (B = 1, T tokens, H heads): the piece's forward and
     reverse maps against its own forward and fwd+bwd (what a rank runs anyway)."""
@@ -640,12 +684,13 @@ def main():
     full = args.B is None and args.T is None
     if not args.no_decode and full:
         decode = bench_decode(binding, dev)
-    reductions = layer_gates = cp_maps = None
+    reductions = layer_gates = cp_maps = layer_step = None
     if not args.no_extra and full and world == 1:
         configs = measure_configs(binding, dev, args, d)
         sweep = measure_sweep(binding, dev, args)
         reductions = measure_reductions(binding, dev, d, args, ms_per_step)
         layer_gates = measure_layer_gates(binding, dev, args, B, T, H)
+        layer_step = measure_layer_step(binding, dev, args, B, T, H)
         cp_maps = measure_context_maps(binding, dev, args)
 
     line = None
@@ -669,7 +714,7 @@ def main():
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_in_timed_region,
                 "decode": decode, "configs": configs, "sweep": sweep, "kda_overhead": reductions,
-                "layer_gates": layer_gates, "context_parallel_maps": cp_maps}
+                "layer_gates": layer_gates, "layer_step": layer_step, "context_parallel_maps": cp_maps}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
