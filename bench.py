@@ -26,7 +26,9 @@ Besides the headline step, the line carries (rank 0, N=1):
     16K-token piece, beside that piece's own forward and fwd+bwd;
   * ``cpu_baseline``: the fp64 oracle timed on a bounded sample of the headline
     workload on the host cores, with the GPU outputs of those same sequences
-    compared against the oracle's (relative L2, whole sample and worst head).
+    compared against the oracle's (relative L2, whole sample and worst head);
+    the same leg gives every ``configs`` and ``sweep`` entry a ``parity`` object
+    (o and the worst gradient of one sampled head against the oracle).
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (rank 0 only).
@@ -252,6 +254,45 @@ def bench_decode(binding, dev, steps=1024, pool=64):
             "launches": kern[0]}
 
 
+# One sampled (batch, head) sequence of each extra measurement: its inputs and the GPU's outputs, copied to the host
+# during the measurement; the CPU-baseline leg compares them with the oracle (sample_parity).
+SAMPLES = []
+
+
+def keep_sample(entry, inputs, outputs, b, h, with_do):
+    """Store sequence (b, h) of a measurement's inputs and outputs (host copies) for sample_parity."""
+    names = ("q", "k", "v", "log_alpha", "b", "w") + (("dout",) if with_do else ())
+    x = {n: inputs[n][b, :, h].detach().cpu() for n in names}
+    if inputs.get("S0") is not None and entry.get("with_S0"):
+        x["S0"] = inputs["S0"][b, h].detach().cpu()
+    y = {n: t[b, :, h].detach().cpu() for n, t in outputs.items() if t is not None and t.dim() == 4}
+    SAMPLES.append((entry, x, y, [b, h]))
+
+
+def sample_parity():
+    """Oracle results of every kept sample; each measurement's entry gets ``parity``: relative L2 of o (and of
+    every gradient when the measurement ran the backward) on its sampled head."""
+    import oracle
+    from linear_attention_delta_gdn_b200.inputs import to_f64
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+
+    def rel(a, r):
+        return float(np.linalg.norm((a - r).ravel()) / max(np.linalg.norm(r.ravel()), 1e-300))
+
+    for entry, x, y, bh in SAMPLES:
+        f = {n: to_f64(t)[None, :, None] for n, t in x.items() if n != "S0"}
+        S0 = to_f64(x["S0"])[None, None] if "S0" in x else None
+        o_ref, _ = oracle.fwd(*(f[n] for n in names), S0=S0)
+        par = {"sampled_head": bh, "o": rel(to_f64(y["o"])[None, :, None], o_ref)}
+        if "dout" in f:
+            g = oracle.bwd(*(f[n] for n in names), dout=f["dout"], S0=S0)
+            par["gradients_worst"] = max(rel(to_f64(y[n])[None, :, None], g[n])
+                                         for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw"))
+        par["tolerance"] = {"o": 2e-2, "gradients": 3e-2}
+        entry["parity"] = par
+    SAMPLES.clear()
+
+
 def device_inputs(B, T, H, D, seed, with_do, dev):
     """Token inputs drawn on the device with the recipe's distributions (seeded torch generator): the long
     and swept workloads hold up to ~2 GB of token tensors."""
@@ -307,6 +348,8 @@ def fwdbwd_point(binding, dev, B, T, H, steps, seed):
     out = {"workload": "fwdbwd-bf16-b%dh%dt%dd128" % (B, H, T), "B": B, "T": T, "H": H, "ms_per_step": ms,
            "tokens_per_s": B * T / (ms / 1e3), "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
            "status": binding.gdn2_device_status()}
+    keep_sample(out, d, dict(o=o, **{n: grads[n] for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw")}),
+                B - 1, H // 2, True)
     del d, ws, o, ST, grads
     torch.cuda.empty_cache()
     return out
@@ -333,6 +376,7 @@ def measure_configs(binding, dev, args, fwd_inputs):
         "mode": "forward only (no saved states), zero S0, o and S_T returned", "ms": ms,
         "tokens_per_s": B * T / (ms / 1e3), "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
         "status": binding.gdn2_device_status()}
+    keep_sample(out["fwd-bf16-b%dh%dt%dd128" % (B, H, T)], fwd_inputs, {"o": o}, B - 1, H // 2, False)
     del ws, o, ST
 
     B, T = 1, 65536
@@ -347,7 +391,8 @@ def measure_configs(binding, dev, args, fwd_inputs):
     out["fwd-bf16-b1h16t65536d128-s0"] = {
         "mode": "forward, random S0 ~ N(0, 0.02^2), o and S_T returned", "ms": ms,
         "tokens_per_s": B * T / (ms / 1e3), "frac_of_roofline": alg / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
-        "status": binding.gdn2_device_status()}
+        "status": binding.gdn2_device_status(), "with_S0": True}
+    keep_sample(out["fwd-bf16-b1h16t65536d128-s0"], d, {"o": o}, 0, H // 2, False)
     del d, ws, o, ST
     torch.cuda.empty_cache()
     return out
@@ -701,6 +746,7 @@ def main():
             gpu_out.update({n: grads[n].cpu() for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw")})
             cb = cpu_baseline(wl, xh, gpu=gpu_out)
             cb = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "parity")}
+            sample_parity()   # one sampled head of each extra measurement against the oracle
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
