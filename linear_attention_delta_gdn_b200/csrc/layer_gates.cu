@@ -12,8 +12,8 @@
 // Backward: dz_q = (dq - q (q.dq)) / ||z_q|| (same for k), dz_v = dv, dz_b = db b (1 - b),
 // dz_w = dw w (1 - w), dz_a = -dlog_alpha sigmoid(z_a + a_bias) (the bias gradient is the sum of dz_a).
 //
-// One warp per (token, head): HBM-bound elementwise work with two warp reductions (the norms); every lane
-// moves 8-byte (bf16) or 16-byte (fp32) pieces, so a warp's accesses are contiguous 256 / 512 byte runs.
+// Two (token, head) rows per warp, one per half-warp: HBM-bound elementwise work with two half-warp reductions
+// (the norms); every lane moves 16-byte pieces, a row's loads all in flight before any arithmetic.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -30,6 +30,105 @@ __device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf
 // the small values
 __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x))); }
 
+// 16-byte pieces of a row: E = 8 bf16 or 4 fp32 values.
+template <typename T> struct Vec16;
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int E = 8;
+    __device__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+        }
+    }
+    __device__ static void store(__nv_bfloat16* p, const float (&v)[8]) {
+        uint4 u;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        *reinterpret_cast<uint4*>(p) = u;
+    }
+};
+template <> struct Vec16<float> {
+    static constexpr int E = 4;
+    __device__ static void load(const float* p, float (&v)[4]) {
+        const float4 u = *reinterpret_cast<const float4*>(p);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    }
+    __device__ static void store(float* p, const float (&v)[4]) { *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]); }
+};
+
+// sum over the 16 lanes of a half-warp (the lanes of one row)
+__device__ __forceinline__ float half_sum(float x) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Two rows per warp, one per half-warp: lane hl = lane % 16 of a half takes the 16-byte pieces hl + 16 m of every
+// segment of its row, so each warp instruction works on one segment (one activation, no divergence) and moves
+// 2 x 16 x 16 contiguous bytes; the six segments' pieces are loaded before any arithmetic. M = pieces per lane
+// and segment for d <= 128 (1 for bf16, 2 for fp32).
+template <typename Tin>
+__global__ void __launch_bounds__(32 * GT_WARPS) gates_fwd_kernel(const Tin* __restrict__ z, Tin* __restrict__ q,
+                                                                  Tin* __restrict__ k, Tin* __restrict__ v,
+                                                                  Tin* __restrict__ b, Tin* __restrict__ w,
+                                                                  Tin* __restrict__ la, const float* __restrict__ abias,
+                                                                  long long rows, int H, int Dk, int Dv) {
+    constexpr int E = Vec16<Tin>::E, M = 128 / E / 16;
+    const int hl = threadIdx.x & 15;
+    const int W = 4 * Dk + 2 * Dv;
+    const int width[6] = {Dk, Dk, Dv, Dk, Dv, Dk};
+    const int start[6] = {0, Dk, 2 * Dk, 2 * Dk + Dv, 3 * Dk + Dv, 3 * Dk + 2 * Dv};
+    Tin* const outs[6] = {q, k, v, b, w, la};
+    const long long nwarps = (long long)gridDim.x * GT_WARPS;
+    for (long long r2 = (long long)blockIdx.x * GT_WARPS + (threadIdx.x >> 5); 2 * r2 < rows; r2 += nwarps) {
+        const long long r = 2 * r2 + ((threadIdx.x >> 4) & 1);
+        const bool live = r < rows;
+        const Tin* zr = z + (live ? r : 0) * W;
+        float x[6][M][E];
+#pragma unroll
+        for (int s = 0; s < 6; ++s)
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                const int pc = hl + 16 * m;
+                if (live && pc * E < width[s]) Vec16<Tin>::load(zr + start[s] + pc * E, x[s][m]);
+                else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) x[s][m][e] = 0.f;
+                }
+            }
+        float nq = 0.f, nk = 0.f;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+#pragma unroll
+            for (int e = 0; e < E; ++e) { nq += x[0][m][e] * x[0][m][e]; nk += x[1][m][e] * x[1][m][e]; }
+        const float iq = rsqrtf(half_sum(nq) + GT_EPS), ik = rsqrtf(half_sum(nk) + GT_EPS);
+        if (!live) continue;
+        const float* bb = abias ? abias + (size_t)(r % H) * Dk : nullptr;
+#pragma unroll
+        for (int s = 0; s < 6; ++s)
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                const int pc = hl + 16 * m;
+                if (pc * E >= width[s]) continue;
+                float y[E];
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const float t = x[s][m][e];
+                    y[e] = s == 0 ? t * iq : s == 1 ? t * ik : s == 2 ? t : (s == 3 || s == 4) ? sigmoid_f(t)
+                                                                                              : -softplus_f(t + (bb ? bb[pc * E + e] : 0.f));
+                }
+                Vec16<Tin>::store(outs[s] + r * width[s] + pc * E, y);
+            }
+    }
+}
+
+// The backward: one warp per row (8-byte pieces per lane, 4 values per segment and lane): with the z and
+// gradient pieces of a whole row held at once (as the forward does), its registers would leave half the warps.
 template <typename T> struct Vec4;
 template <> struct Vec4<__nv_bfloat16> {
     __device__ static void load(const __nv_bfloat16* p, float (&v)[4]) {
@@ -71,52 +170,6 @@ struct Seg {
         return o;
     }
 };
-
-// z: [rows = B*T*H][4 Dk + 2 Dv]; outputs [rows][Dk] (q, k, b, la) and [rows][Dv] (v, w).
-template <typename Tin>
-__global__ void __launch_bounds__(32 * GT_WARPS) gates_fwd_kernel(const Tin* __restrict__ z, Tin* __restrict__ q,
-                                                                  Tin* __restrict__ k, Tin* __restrict__ v,
-                                                                  Tin* __restrict__ b, Tin* __restrict__ w,
-                                                                  Tin* __restrict__ la, const float* __restrict__ abias,
-                                                                  long long rows, int H, int Dk, int Dv) {
-    const int lane = threadIdx.x & 31;
-    const Seg sg{Dk, Dv};
-    const int W = 4 * Dk + 2 * Dv;
-    for (long long r = (long long)blockIdx.x * GT_WARPS + (threadIdx.x >> 5); r < rows;
-         r += (long long)gridDim.x * GT_WARPS) {
-        const Tin* zr = z + r * W;
-        // the norms of z_q and z_k
-        float nq = 0.f, nk = 0.f;
-        for (int j = 4 * lane; j < Dk; j += 128) {
-            float a[4], c[4];
-            Vec4<Tin>::load(zr + j, a);
-            Vec4<Tin>::load(zr + Dk + j, c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) { nq += a[e] * a[e]; nk += c[e] * c[e]; }
-        }
-        const float iq = rsqrtf(warp_sum(nq) + GT_EPS), ik = rsqrtf(warp_sum(nk) + GT_EPS);
-        Tin* const outs[6] = {q, k, v, b, w, la};
-#pragma unroll
-        for (int s = 0; s < 6; ++s) {   // unrolled: the segment, its offset and its activation are constants
-            const int D = sg.width(s), o = sg.begin(s);
-            for (int j = 4 * lane; j < D; j += 128) {
-                float x[4];
-                Vec4<Tin>::load(zr + o + j, x);
-                if (s == 5 && abias) {
-                    const float* bb = abias + (size_t)(r % H) * Dk + j;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) x[e] += bb[e];
-                }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float t = x[e];
-                    x[e] = s == 0 ? t * iq : s == 1 ? t * ik : s == 2 ? t : (s == 3 || s == 4) ? sigmoid_f(t) : -softplus_f(t);
-                }
-                Vec4<Tin>::store(outs[s] + r * D + j, x);
-            }
-        }
-    }
-}
 
 // dz from z, the outputs q, k, b, w (recomputed from z) and their gradients.
 template <typename Tin>
@@ -185,7 +238,7 @@ int gates_grid(long long rows) {
         if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             nsm = 148;
     }
-    const long long want = (rows + GT_WARPS - 1) / GT_WARPS;
+    const long long want = ((rows + 1) / 2 + GT_WARPS - 1) / GT_WARPS;   // a warp takes two rows
     const long long cap = (long long)nsm * 16;   // 16 CTAs of 8 warps per SM: full occupancy, grid-stride beyond
     return (int)(want < cap ? want : cap);
 }
