@@ -696,8 +696,9 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             atomicOr(&g_bwd_error, 8u);
             atomicExch(p.counter + 1, 1u);
         }
-        tc::bulk_wait_read();   // the previous unit's dq, dk, db, dlog_alpha stores have read DU, DT, DDT
+        tc::bulk_wait_read();   // the previous unit's dq, dlog_alpha stores have read DU
     }
+    if (lane == 0 && (warp == 1 || warp == 2)) tc::bulk_wait_read();   // its dk, db stores: DT, DDT
     __syncthreads();   // orders thread 0's acquire and its wait before the loads and copies below
     if (lane == 0) {
         const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
@@ -806,29 +807,32 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         }
     }
     sync_for_mma();
-    if (tid == 0) {     // store dv, dw (rows past the end of the sequence are skipped); bring b back for
-                        // the gate chain (w is consumed)
-        tc::tma_store_4d(&m.dv, 0, h, t0, b, DDT);
-        tc::tma_store_4d(&m.dv, 64, h, t0, b, DDT + C * 128);
-        tc::tma_store_4d(&m.dw, 0, h, t0, b, PP);
-        tc::tma_store_4d(&m.dw, 64, h, t0, b, PP + C * 128);
-        tc::bulk_commit();
-        tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
-        tma_tile(WW, C, 0, mb, b, h, t0, bar_b);
+    // store dv (lane 0 of warp 1) and dw (warp 2; rows past the end of the sequence are skipped), and bring b
+    // back for the gate chain (warp 3; w is consumed), while thread 0 issues the MMAs below
+    if (lane == 0 && warp >= 1 && warp <= 3) {
+        if (warp == 3) {
+            tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
+            tma_tile(WW, C, 0, mb, b, h, t0, bar_b);
+        } else {
+            const CUtensorMap* map = warp == 1 ? &m.dv : &m.dw;
+            unsigned char* tile = warp == 1 ? DDT : PP;
+            tc::tma_store_4d(map, 0, h, t0, b, tile);
+            tc::tma_store_4d(map, 64, h, t0, b, tile + C * 128);
+            tc::bulk_commit();
+        }
     }
 
     // ---- dP^T = Delta dO^T (M=64), dA^T = -Delta dU^T (M=64)
     if (tid == 0) {
         tc::tc_fence_after();
-        constexpr uint32_t id_pa = tc::idesc_bf16(64, 64, true, false);   // the tile holds -dU: no negation
+        constexpr uint32_t id_pa = tc::idesc_bf16(64, 128, true, false);   // the tile holds -dU: no negation
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 8; ++kk)   // [dP^T | dA^T] (TM_AP, TM_W adjacent) as one N = 128 product over DU
             tc::mma_bf16(tmem + TM_AP, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sDU, 2 * C, 0, kk), id_pa, kk > 0);
-            tc::mma_bf16(tmem + TM_W, tc::desc_mn(sDT, D, 0, kk), tc::desc_k(sDU, 2 * C, C, kk), id_pa, kk > 0);
-        }
         tc::mma_commit(bar_mma);
-        tc::bulk_wait_read();   // the dv, dw stores have read their tiles (TT, PP are overwritten below)
     }
+    if (lane == 0 && (warp == 1 || warp == 2))
+        tc::bulk_wait_read();   // the dv, dw stores have read their tiles (DDT, TT, PP are overwritten below)
     wait_mma();
     tc::tc_fence_before();
     __syncthreads();
@@ -979,15 +983,13 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     tc::fence_async_smem();   // every read of S^T and dS'^T (G MMAs, rowsum) precedes the prefetch below, and
                               // dq, dk, db (final after pass 1) are visible to the tensor stores
     __syncthreads();          // also orders warp 9's acquire before every thread's copy of the next dS'^T
-    if (tid == 0) {   // dq, dk, db go out while pass 2 runs; rows past the end of the sequence are skipped
-        const CUtensorMap* maps[3] = {mdq, mdk, mdb};
-        const unsigned char* tiles[3] = {DU, DT, DDT};
-        const uint32_t panel[3] = {2 * C * 128, C * 128, C * 128};   // second 64 channels
-#pragma unroll
-        for (int o = 0; o < 3; ++o) {
-            tc::tma_store_4d(maps[o], 0, h, t0, b, tiles[o]);
-            tc::tma_store_4d(maps[o], 64, h, t0, b, tiles[o] + panel[o]);
-        }
+    if (lane == 0 && warp < 3) {   // dq, dk, db (lane 0 of warps 0, 1, 2) go out while pass 2 runs; rows past
+                                   // the end of the sequence are skipped
+        const CUtensorMap* map = warp == 0 ? mdq : (warp == 1 ? mdk : mdb);
+        const unsigned char* tile = warp == 0 ? DU : (warp == 1 ? DT : DDT);
+        const uint32_t panel = warp == 0 ? 2 * C * 128 : C * 128;   // second 64 channels
+        tc::tma_store_4d(map, 0, h, t0, b, tile);
+        tc::tma_store_4d(map, 64, h, t0, b, tile + panel);
         tc::bulk_commit();
     }
     int nxt_head = 0, nxt_c = 0;
@@ -1101,7 +1103,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
             u = nxt->unit;   // written by thread 0 before the unit's last barrier
             pre = nxt->prefetched != 0;
         }
-        if (tid == 0) tc::bulk_wait_read();   // the last unit's output stores have read their tiles
+        if ((tid & 31) == 0 && warp < 3) tc::bulk_wait_read();   // the last unit's output stores have read their tiles
     }
     tc::tc_fence_before();
     __syncthreads();
