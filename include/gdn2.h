@@ -194,7 +194,10 @@ gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const 
  * Workspace: gdn2_beta_workspace_size(gate, op, ...) bytes, 256-byte aligned;
  * one buffer of the GDN2_OP_BWD size serves gdn2_beta_fwd(save_states = 1)
  * followed by gdn2_beta_bwd(states_saved = 1). Returns 0 for an invalid gate
- * or problem.
+ * or problem. With states_saved = 1 the backward also reuses the broadcast
+ * gates that gdn2_beta_fwd(save_states = 1) left in that buffer (the same
+ * gate, beta and log_alpha, like the other inputs), so a training step
+ * broadcasts once; with states_saved = 0 it broadcasts them itself.
  */
 typedef enum gdn2_gate {
     GDN2_GATE_KDA = 1,   /* beta per head and token, channel-wise decay */

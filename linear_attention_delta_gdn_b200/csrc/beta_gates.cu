@@ -7,7 +7,9 @@
 // workspace (b, w and, for the scalar decay, log_alpha), run gdn2_fwd / gdn2_bwd, and sum the gradients
 // of the broadcast gates back over their channels:
 //   dbeta_t = sum_i db_ti + sum_j dw_tj,    dlog_a_t = sum_i dlog_alpha_ti   (scalar decay).
-// Both steps are memory-bound elementwise kernels (16-byte accesses, one warp per row for the sums).
+// Both steps are memory-bound elementwise kernels: one warp per row, 16-byte pieces, a few rows in flight
+// per warp. A backward on saved states reuses the forward's broadcast gates (they sit at the same place in
+// the workspace for both calls), so a training step broadcasts once and sums once.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -22,64 +24,108 @@ namespace {
 
 size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// 8 copies of one value at dst (16-byte aligned), in 16-byte stores
-__device__ __forceinline__ void store8(__nv_bfloat16* dst, __nv_bfloat16 v) {
+// One 16-byte piece of copies of v (8 bf16 or 4 fp32)
+__device__ __forceinline__ void store_piece(__nv_bfloat16* dst, __nv_bfloat16 v) {
     const uint32_t x = (uint32_t)__bfloat16_as_ushort(v) * 0x10001u;
     *reinterpret_cast<uint4*>(dst) = make_uint4(x, x, x, x);
 }
-__device__ __forceinline__ void store8(float* dst, float v) {
+__device__ __forceinline__ void store_piece(float* dst, float v) {
     *reinterpret_cast<float4*>(dst) = make_float4(v, v, v, v);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(v, v, v, v);
+}
+// The sum of one 16-byte piece
+__device__ __forceinline__ float sum_piece(const __nv_bfloat16* src) {
+    const uint4 x = *reinterpret_cast<const uint4*>(src);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        s += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xFFFF0000u);
+    return s;
+}
+__device__ __forceinline__ float sum_piece(const float* src) {
+    const float4 x = *reinterpret_cast<const float4*>(src);
+    return (x.x + x.y) + (x.z + x.w);
 }
 
+constexpr int ROWS_PER_WARP = 4;   // rows a warp has in flight (their loads issued before any store)
+
 // Per-row broadcast: row r = (b, t, h); b[r][0:Dk] = beta[r], w[r][0:Dv] = beta[r], la[r][0:Dk] = la_s[r]
-// (scalar decay only). One thread per 8 consecutive elements of the row's [b | w | la] concatenation.
+// (scalar decay only). A warp takes ROWS_PER_WARP rows at a time; lane l writes the 16-byte pieces l, l + 32,
+// ... of each row's [b | w | la] concatenation (Dk, Dv are multiples of 16: whole pieces).
 template <typename Tin>
 __global__ void expand_kernel(const Tin* __restrict__ beta, const Tin* __restrict__ la_s, Tin* __restrict__ b,
                               Tin* __restrict__ w, Tin* __restrict__ la, long long rows, int Dk, int Dv) {
-    const int nb = Dk / 8, nw = Dv / 8, nl = la_s ? Dk / 8 : 0, per = nb + nw + nl;
-    const long long total = rows * per;
-    for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
-         x += (long long)gridDim.x * blockDim.x) {
-        const long long r = x / per;
-        const int p = (int)(x - r * per);
-        Tin val;
-        Tin* dst;
-        if (p < nb) {
-            val = beta[r];
-            dst = b + r * Dk + 8 * p;
-        } else if (p < nb + nw) {
-            val = beta[r];
-            dst = w + r * Dv + 8 * (p - nb);
-        } else {
-            val = la_s[r];
-            dst = la + r * Dk + 8 * (p - nb - nw);
+    constexpr int E = 16 / (int)sizeof(Tin);
+    const int lane = threadIdx.x & 31;
+    const int nb = Dk / E, nw = Dv / E, per = nb + nw + (la_s ? Dk / E : 0);
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * ROWS_PER_WARP; r0 < rows;
+         r0 += warps * ROWS_PER_WARP) {
+        Tin bv[ROWS_PER_WARP], lv[ROWS_PER_WARP];
+#pragma unroll
+        for (int j = 0; j < ROWS_PER_WARP; ++j) {
+            const long long r = r0 + j < rows ? r0 + j : rows - 1;
+            bv[j] = beta[r];
+            lv[j] = la_s ? la_s[r] : bv[j];
         }
-        store8(dst, val);
+#pragma unroll
+        for (int j = 0; j < ROWS_PER_WARP; ++j) {
+            const long long r = r0 + j;
+            if (r >= rows) break;
+            for (int p = lane; p < per; p += 32) {
+                if (p < nb)
+                    store_piece(b + r * Dk + E * p, bv[j]);
+                else if (p < nb + nw)
+                    store_piece(w + r * Dv + E * (p - nb), bv[j]);
+                else
+                    store_piece(la + r * Dk + E * (p - nb - nw), lv[j]);
+            }
+        }
     }
 }
 
-// Per-row sums: dbeta[r] = sum db[r] + sum dw[r]; dla_s[r] = sum dla[r] (scalar decay only). One warp per row.
+// Per-row sums: dbeta[r] = sum db[r] + sum dw[r]; dla_s[r] = sum dla[r] (scalar decay only). A warp takes
+// ROWS_PER_WARP rows at a time (all their 16-byte pieces loaded before the warp sums).
 template <typename Tin>
 __global__ void reduce_kernel(const Tin* __restrict__ db, const Tin* __restrict__ dw, const Tin* __restrict__ dla,
                               Tin* __restrict__ dbeta, Tin* __restrict__ dla_s, long long rows, int Dk, int Dv) {
+    constexpr int E = 16 / (int)sizeof(Tin);
     const int lane = threadIdx.x & 31;
+    const int nb = Dk / E, nw = Dv / E, per = nb + nw + (dla ? Dk / E : 0);
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-    for (long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
-        float sb = 0.f, sl = 0.f;
-        for (int i = lane; i < Dk; i += 32) {
-            sb += to_f32(db[r * Dk + i]);
-            if (dla) sl += to_f32(dla[r * Dk + i]);
-        }
-        for (int j = lane; j < Dv; j += 32) sb += to_f32(dw[r * Dv + j]);
+    for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * ROWS_PER_WARP; r0 < rows;
+         r0 += warps * ROWS_PER_WARP) {
+        float sb[ROWS_PER_WARP], sl[ROWS_PER_WARP];
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) {
-            sb += __shfl_xor_sync(0xffffffffu, sb, m);
-            sl += __shfl_xor_sync(0xffffffffu, sl, m);
+        for (int j = 0; j < ROWS_PER_WARP; ++j) {
+            sb[j] = 0.f;
+            sl[j] = 0.f;
+            const long long r = r0 + j;
+            if (r >= rows) continue;
+            for (int p = lane; p < per; p += 32) {
+                if (p < nb)
+                    sb[j] += sum_piece(db + r * Dk + E * p);
+                else if (p < nb + nw)
+                    sb[j] += sum_piece(dw + r * Dv + E * (p - nb));
+                else
+                    sl[j] += sum_piece(dla + r * Dk + E * (p - nb - nw));
+            }
         }
-        if (lane == 0) {
-            dbeta[r] = from_f32<Tin>(sb);
-            if (dla) dla_s[r] = from_f32<Tin>(sl);
+#pragma unroll
+        for (int j = 0; j < ROWS_PER_WARP; ++j) {
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) {
+                sb[j] += __shfl_xor_sync(0xffffffffu, sb[j], m);
+                sl[j] += __shfl_xor_sync(0xffffffffu, sl[j], m);
+            }
+        }
+        if (lane < ROWS_PER_WARP && r0 + lane < rows) {
+            float b_ = sb[0], l_ = sl[0];
+#pragma unroll
+            for (int j = 1; j < ROWS_PER_WARP; ++j)
+                if (lane == j) { b_ = sb[j]; l_ = sl[j]; }
+            dbeta[r0 + lane] = from_f32<Tin>(b_);
+            if (dla) dla_s[r0 + lane] = from_f32<Tin>(l_);
         }
     }
 }
@@ -95,9 +141,8 @@ int grid_for(long long work, int block) {
 template <typename Tin>
 cudaError_t launch_expand(const void* beta, const void* la_s, void* b, void* w, void* la, long long rows, int Dk,
                           int Dv, cudaStream_t s) {
-    const long long work = rows * (Dk / 8 + Dv / 8 + (la_s ? Dk / 8 : 0));
     TraceScope trace(K_GATE_EXPAND, s);
-    expand_kernel<Tin><<<grid_for(work, 256), 256, 0, s>>>(static_cast<const Tin*>(beta), static_cast<const Tin*>(la_s),
+    expand_kernel<Tin><<<grid_for(rows * 32 / ROWS_PER_WARP, 256), 256, 0, s>>>(static_cast<const Tin*>(beta), static_cast<const Tin*>(la_s),
                                                           static_cast<Tin*>(b), static_cast<Tin*>(w),
                                                           static_cast<Tin*>(la), rows, Dk, Dv);
     return cudaGetLastError();
@@ -107,14 +152,16 @@ template <typename Tin>
 cudaError_t launch_reduce(const void* db, const void* dw, const void* dla, void* dbeta, void* dla_s, long long rows,
                           int Dk, int Dv, cudaStream_t s) {
     TraceScope trace(K_GATE_REDUCE, s);
-    reduce_kernel<Tin><<<grid_for(rows * 32, 256), 256, 0, s>>>(
+    reduce_kernel<Tin><<<grid_for(rows * 32 / ROWS_PER_WARP, 256), 256, 0, s>>>(
         static_cast<const Tin*>(db), static_cast<const Tin*>(dw), static_cast<const Tin*>(dla),
         static_cast<Tin*>(dbeta), static_cast<Tin*>(dla_s), rows, Dk, Dv);
     return cudaGetLastError();
 }
 
 // Workspace of the reduced-gate calls (each region 256-byte aligned):
-//   [gdn2 workspace: gdn2_workspace_size(GDN2_OP_FWD) for a plain forward, else of GDN2_OP_BWD]
+//   [gdn2 workspace: gdn2_workspace_size(GDN2_OP_FWD) for a plain forward, else the larger of the
+//    GDN2_OP_FWD_SAVE and GDN2_OP_BWD sizes, so that a forward that saves its states and the backward on
+//    them find the broadcast gates at the same offsets]
 //   [b: rows x Dk][w: rows x Dv][log_alpha: rows x Dk (scalar decay)]
 //   backward only: [db: rows x Dk][dw: rows x Dv][dlog_alpha: rows x Dk (scalar decay)]
 struct Layout {
@@ -125,7 +172,13 @@ Layout layout(gdn2_gate gate, gdn2_op op, int B, int T, int H, int Dk, int Dv, i
     const size_t es = dt == GDN2_BF16 ? 2 : 4;
     const size_t rows = (size_t)B * T * H;
     const bool scalar = gate == GDN2_GATE_GDN;
-    L.base = al256(gdn2_workspace_size(op == GDN2_OP_FWD ? GDN2_OP_FWD : GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt));
+    if (op == GDN2_OP_FWD) {
+        L.base = al256(gdn2_workspace_size(GDN2_OP_FWD, B, T, H, Dk, Dv, chunk, dt));
+    } else {
+        const size_t save = gdn2_workspace_size(GDN2_OP_FWD_SAVE, B, T, H, Dk, Dv, chunk, dt);
+        const size_t bwd = gdn2_workspace_size(GDN2_OP_BWD, B, T, H, Dk, Dv, chunk, dt);
+        L.base = al256(save > bwd ? save : bwd);
+    }
     L.b = L.base;
     L.w = L.b + al256(rows * Dk * es);
     L.la = L.w + al256(rows * Dv * es);
@@ -227,7 +280,7 @@ gdn2_status gdn2_beta_bwd(gdn2_gate gate, const void* q, const void* k, const vo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool scalar = gate == GDN2_GATE_GDN;
     const long long rows = (long long)B * T * H;
-    if (T > 0) {   // the broadcast gates (again: the forward may have run with another workspace)
+    if (T > 0 && !states_saved) {   // the broadcast gates (on saved states, the forward's are still there)
         cudaError_t e = dt == GDN2_BF16
                             ? launch_expand<__nv_bfloat16>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w,
                                                            w8 + L.la, rows, Dk, Dv, s)

@@ -55,9 +55,14 @@ def _worst_rows(got, ref):
 
 
 @pytest.mark.parametrize("gate", ["kda", "gdn"])
-@pytest.mark.parametrize("dtype,T,Dk,Dv,chunk", [("bf16", 150, 128, 128, 64), ("bf16", 300, 128, 128, 64),
-                                                 ("f32", 70, 64, 64, 32), ("bf16", 97, 64, 128, 64)])
-def test_reduced_gates_against_oracle(oracle_mod, gate, dtype, T, Dk, Dv, chunk):
+@pytest.mark.parametrize("dtype,T,Dk,Dv,chunk,saved", [("bf16", 150, 128, 128, 64, True),
+                                                       ("bf16", 300, 128, 128, 64, True),
+                                                       ("bf16", 300, 128, 128, 64, False),
+                                                       ("f32", 70, 64, 64, 32, True), ("f32", 70, 64, 64, 32, False),
+                                                       ("bf16", 97, 64, 128, 64, True)])
+def test_reduced_gates_against_oracle(oracle_mod, gate, dtype, T, Dk, Dv, chunk, saved):
+    """saved: the backward runs on the forward's workspace (its saved states and broadcast gates); else on a
+    workspace of its own, filled with 0xFF bytes first, so it must broadcast the gates itself."""
     B, H = 2, 3
     x, beta, la = _case(gate, B, T, H, Dk, Dv, dtype, seed=1200 + T + Dk)
     d = {n: t.cuda() for n, t in x.items()}
@@ -67,8 +72,10 @@ def test_reduced_gates_against_oracle(oracle_mod, gate, dtype, T, Dk, Dv, chunk)
                                                       binding._dt(d["q"])), dtype=torch.uint8, device="cuda")
     o, ST = binding.gdn2_beta_fwd(GATES[gate], d["q"], d["k"], d["v"], g_la, g_beta, d["S0"], chunk=chunk,
                                   save_states=True, ws=ws)
+    if not saved:
+        ws = torch.full_like(ws, 255)
     g = binding.gdn2_beta_bwd(GATES[gate], d["q"], d["k"], d["v"], g_la, g_beta, d["dout"], d["S0"], dST.cuda(),
-                              chunk=chunk, states_saved=True, ws=ws)
+                              chunk=chunk, states_saved=saved, ws=ws)
     torch.cuda.synchronize()
 
     f = {n: to_f64(t) for n, t in x.items()}
