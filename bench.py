@@ -400,8 +400,9 @@ def measure_configs(binding, dev, args, fwd_inputs):
 
 def measure_reductions(binding, dev, d, args, gdn2_ms):
     """The pages' reductions through the same kernels at the headline shape: KDA (b = w = beta * 1) and Gated
-    DeltaNet (also a scalar decay), fwd (keeping the states) + bwd, against the GDN-2 step. Both run the GDN-2
-    kernels on broadcast gates plus a broadcast and a gate-sum kernel; `overhead_of_gdn2` is
+    DeltaNet (also a scalar decay), fwd (keeping the states) + bwd, against the GDN-2 step. Both run the chunk
+    kernels' scalar-gate instances (beta read per token, dbeta summed in the gradient units); Gated DeltaNet's
+    scalar decay is broadcast and its gradient summed by two elementwise kernels. `overhead_of_gdn2` is
     gdn2_ms / reduced_ms - 1."""
     import torch
     names = ("q", "k", "v")
@@ -430,8 +431,9 @@ def measure_reductions(binding, dev, d, args, gdn2_ms):
         out["overhead_of_gdn2_over_" + name] = gdn2_ms / ms - 1.0
         out[name + "_status"] = binding.gdn2_device_status()
         del ws, o, ST, grads
-    out["note"] = ("KDA and Gated DeltaNet run the GDN-2 kernels on gates broadcast into the workspace, plus a "
-                   "broadcast and a gate-sum kernel; a negative overhead means the reduced model costs more here")
+    out["note"] = ("KDA and Gated DeltaNet run the chunk kernels' scalar-gate instances (no b or w tiles; dbeta "
+                   "from the gradient units); Gated DeltaNet's scalar decay is broadcast and its gradient summed by "
+                   "two elementwise kernels")
     torch.cuda.empty_cache()
     return out
 

@@ -3,13 +3,14 @@
 // "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention" (README "Strict Generalization"
 // bullet, arXiv abstract) states that the operator reduces to KDA when the erase and write gates are one
 // scalar beta_t per head and token (b_t = w_t = beta_t 1), and further to Gated DeltaNet when the decay is
-// also one scalar per head and token. These entry points take the reduced gates, broadcast them into the
-// workspace (b, w and, for the scalar decay, log_alpha), run gdn2_fwd / gdn2_bwd, and sum the gradients
-// of the broadcast gates back over their channels:
-//   dbeta_t = sum_i db_ti + sum_j dw_tj,    dlog_a_t = sum_i dlog_alpha_ti   (scalar decay).
-// Both steps are memory-bound elementwise kernels: one warp per row, 16-byte pieces, a few rows in flight
-// per warp. A backward on saved states reuses the forward's broadcast gates (they sit at the same place in
-// the workspace for both calls), so a training step broadcasts once and sums once.
+// also one scalar per head and token. These entry points take the reduced gates. On the tensor-core path
+// (bf16, Dk = Dv = 128) the chunk kernels have an instance for a scalar erase and write gate: beta goes in as
+// it is, and dbeta_t = sum_i db_ti + sum_j dw_tj comes out of the backward's gradient units. Elsewhere the
+// gates are broadcast into the workspace (b, w), gdn2_fwd / gdn2_bwd run on them, and their gradients are
+// summed back over the channels. A scalar decay (Gated DeltaNet) is broadcast on both paths and its gradient
+// summed, dlog_a_t = sum_i dlog_alpha_ti. Both steps are memory-bound elementwise kernels: one warp per row,
+// 16-byte pieces, a few rows in flight per warp. A backward on saved states reuses the forward's broadcast
+// gates (they sit at the same place in the workspace for both calls), so a training step broadcasts once.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -47,32 +48,43 @@ __device__ __forceinline__ float sum_piece(const float* src) {
     return (x.x + x.y) + (x.z + x.w);
 }
 
-constexpr int ROWS_PER_WARP = 4;   // rows a warp has in flight (their loads issued before any store)
+constexpr int ROWS_PER_WARP = 4;   // row steps a warp has in flight (their loads issued before any store)
 
-// Per-row broadcast: row r = (b, t, h); b[r][0:Dk] = beta[r], w[r][0:Dv] = beta[r], la[r][0:Dk] = la_s[r]
-// (scalar decay only). A warp takes ROWS_PER_WARP rows at a time; lane l writes the 16-byte pieces l, l + 32,
-// ... of each row's [b | w | la] concatenation (Dk, Dv are multiples of 16: whole pieces).
+// Lanes that share a row: the pieces per row rounded up to a power of two, at most the warp.
+__device__ __forceinline__ int lanes_per_row(int per) {
+    int g = 1;
+    while (g < per && g < 32) g <<= 1;
+    return g;
+}
+
+// Per-row broadcast: row r = (b, t, h); b[r][0:Dk] = beta[r], w[r][0:Dv] = beta[r] (unless b, w are null),
+// la[r][0:Dk] = la_s[r] (scalar decay only). G lanes share a row (32 / G rows per warp at a time, ROWS_PER_WARP
+// times over); lane g of a row writes the 16-byte pieces g, g + G, ... of its [b | w | la] concatenation (Dk,
+// Dv are multiples of 16: whole pieces).
 template <typename Tin>
 __global__ void expand_kernel(const Tin* __restrict__ beta, const Tin* __restrict__ la_s, Tin* __restrict__ b,
                               Tin* __restrict__ w, Tin* __restrict__ la, long long rows, int Dk, int Dv) {
     constexpr int E = 16 / (int)sizeof(Tin);
     const int lane = threadIdx.x & 31;
-    const int nb = Dk / E, nw = Dv / E, per = nb + nw + (la_s ? Dk / E : 0);
+    const int nb = b ? Dk / E : 0, nw = w ? Dv / E : 0, per = nb + nw + (la_s ? Dk / E : 0);
+    const int G = lanes_per_row(per), rps = 32 / G, sub = lane / G, gl = lane % G;
+    const long long step = (long long)ROWS_PER_WARP * rps;   // rows per warp and pass
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-    for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * ROWS_PER_WARP; r0 < rows;
-         r0 += warps * ROWS_PER_WARP) {
+    for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * step; r0 < rows;
+         r0 += warps * step) {
         Tin bv[ROWS_PER_WARP], lv[ROWS_PER_WARP];
 #pragma unroll
         for (int j = 0; j < ROWS_PER_WARP; ++j) {
-            const long long r = r0 + j < rows ? r0 + j : rows - 1;
-            bv[j] = beta[r];
+            long long r = r0 + j * rps + sub;
+            if (r >= rows) r = rows - 1;
+            bv[j] = nb + nw ? beta[r] : Tin{};
             lv[j] = la_s ? la_s[r] : bv[j];
         }
 #pragma unroll
         for (int j = 0; j < ROWS_PER_WARP; ++j) {
-            const long long r = r0 + j;
+            const long long r = r0 + j * rps + sub;
             if (r >= rows) break;
-            for (int p = lane; p < per; p += 32) {
+            for (int p = gl; p < per; p += G) {
                 if (p < nb)
                     store_piece(b + r * Dk + E * p, bv[j]);
                 else if (p < nb + nw)
@@ -84,25 +96,27 @@ __global__ void expand_kernel(const Tin* __restrict__ beta, const Tin* __restric
     }
 }
 
-// Per-row sums: dbeta[r] = sum db[r] + sum dw[r]; dla_s[r] = sum dla[r] (scalar decay only). A warp takes
-// ROWS_PER_WARP rows at a time (all their 16-byte pieces loaded before the warp sums).
+// Per-row sums: dbeta[r] = sum db[r] + sum dw[r] (unless db, dw are null); dla_s[r] = sum dla[r] (scalar decay
+// only). Rows shared out as in expand_kernel; all of a pass's 16-byte pieces are loaded before the sums.
 template <typename Tin>
 __global__ void reduce_kernel(const Tin* __restrict__ db, const Tin* __restrict__ dw, const Tin* __restrict__ dla,
                               Tin* __restrict__ dbeta, Tin* __restrict__ dla_s, long long rows, int Dk, int Dv) {
     constexpr int E = 16 / (int)sizeof(Tin);
     const int lane = threadIdx.x & 31;
-    const int nb = Dk / E, nw = Dv / E, per = nb + nw + (dla ? Dk / E : 0);
+    const int nb = db ? Dk / E : 0, nw = dw ? Dv / E : 0, per = nb + nw + (dla ? Dk / E : 0);
+    const int G = lanes_per_row(per), rps = 32 / G, sub = lane / G, gl = lane % G;
+    const long long step = (long long)ROWS_PER_WARP * rps;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-    for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * ROWS_PER_WARP; r0 < rows;
-         r0 += warps * ROWS_PER_WARP) {
+    for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * step; r0 < rows;
+         r0 += warps * step) {
         float sb[ROWS_PER_WARP], sl[ROWS_PER_WARP];
 #pragma unroll
         for (int j = 0; j < ROWS_PER_WARP; ++j) {
             sb[j] = 0.f;
             sl[j] = 0.f;
-            const long long r = r0 + j;
+            const long long r = r0 + j * rps + sub;
             if (r >= rows) continue;
-            for (int p = lane; p < per; p += 32) {
+            for (int p = gl; p < per; p += G) {
                 if (p < nb)
                     sb[j] += sum_piece(db + r * Dk + E * p);
                 else if (p < nb + nw)
@@ -113,28 +127,29 @@ __global__ void reduce_kernel(const Tin* __restrict__ db, const Tin* __restrict_
         }
 #pragma unroll
         for (int j = 0; j < ROWS_PER_WARP; ++j) {
-#pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) {
+            for (int m = G >> 1; m >= 1; m >>= 1) {   // within the G lanes of the row
                 sb[j] += __shfl_xor_sync(0xffffffffu, sb[j], m);
                 sl[j] += __shfl_xor_sync(0xffffffffu, sl[j], m);
             }
-        }
-        if (lane < ROWS_PER_WARP && r0 + lane < rows) {
-            float b_ = sb[0], l_ = sl[0];
-#pragma unroll
-            for (int j = 1; j < ROWS_PER_WARP; ++j)
-                if (lane == j) { b_ = sb[j]; l_ = sl[j]; }
-            dbeta[r0 + lane] = from_f32<Tin>(b_);
-            if (dla) dla_s[r0 + lane] = from_f32<Tin>(l_);
+            const long long r = r0 + j * rps + sub;
+            if (gl == 0 && r < rows) {
+                if (nb + nw) dbeta[r] = from_f32<Tin>(sb[j]);
+                if (dla) dla_s[r] = from_f32<Tin>(sl[j]);
+            }
         }
     }
 }
 
-int grid_for(long long work, int block) {
-    int dev = 0, sms = 148;
+// Enough blocks of `block` threads for `work` threads, at most as many as are resident at once (a whole
+// number of waves: the kernels are grid-stride loops)
+template <typename K>
+int grid_for(K kernel, long long work, int block) {
+    int dev = 0, sms = 148, per_sm = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, block, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
     const long long want = (work + block - 1) / block;
-    const long long cap = (long long)sms * 8;
+    const long long cap = (long long)sms * per_sm;
     return (int)(want < 1 ? 1 : (want > cap ? cap : want));
 }
 
@@ -142,7 +157,7 @@ template <typename Tin>
 cudaError_t launch_expand(const void* beta, const void* la_s, void* b, void* w, void* la, long long rows, int Dk,
                           int Dv, cudaStream_t s) {
     TraceScope trace(K_GATE_EXPAND, s);
-    expand_kernel<Tin><<<grid_for(rows * 32 / ROWS_PER_WARP, 256), 256, 0, s>>>(static_cast<const Tin*>(beta), static_cast<const Tin*>(la_s),
+    expand_kernel<Tin><<<grid_for(expand_kernel<Tin>, rows * 32 / ROWS_PER_WARP, 256), 256, 0, s>>>(static_cast<const Tin*>(beta), static_cast<const Tin*>(la_s),
                                                           static_cast<Tin*>(b), static_cast<Tin*>(w),
                                                           static_cast<Tin*>(la), rows, Dk, Dv);
     return cudaGetLastError();
@@ -152,7 +167,7 @@ template <typename Tin>
 cudaError_t launch_reduce(const void* db, const void* dw, const void* dla, void* dbeta, void* dla_s, long long rows,
                           int Dk, int Dv, cudaStream_t s) {
     TraceScope trace(K_GATE_REDUCE, s);
-    reduce_kernel<Tin><<<grid_for(rows * 32 / ROWS_PER_WARP, 256), 256, 0, s>>>(
+    reduce_kernel<Tin><<<grid_for(reduce_kernel<Tin>, rows * 32 / ROWS_PER_WARP, 256), 256, 0, s>>>(
         static_cast<const Tin*>(db), static_cast<const Tin*>(dw), static_cast<const Tin*>(dla),
         static_cast<Tin*>(dbeta), static_cast<Tin*>(dla_s), rows, Dk, Dv);
     return cudaGetLastError();
@@ -235,20 +250,26 @@ gdn2_status gdn2_beta_fwd(gdn2_gate gate, const void* q, const void* k, const vo
     unsigned char* w8 = static_cast<unsigned char*>(ws);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool scalar = gate == GDN2_GATE_GDN;
+    const bool tc = tc_path(dt, Dk, Dv) && ((uintptr_t)beta & 3) == 0;   // the chunk kernels take beta as it is
     const void* la_full = log_alpha;
-    if (T > 0) {
+    if (T > 0 && (!tc || scalar)) {
         const long long rows = (long long)B * T * H;
+        void* bf = tc ? nullptr : w8 + L.b;
+        void* wf = tc ? nullptr : w8 + L.w;
         cudaError_t e = dt == GDN2_BF16
-                            ? launch_expand<__nv_bfloat16>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w,
-                                                           w8 + L.la, rows, Dk, Dv, s)
-                            : launch_expand<float>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w, w8 + L.la,
-                                                   rows, Dk, Dv, s);
+                            ? launch_expand<__nv_bfloat16>(beta, scalar ? log_alpha : nullptr, bf, wf, w8 + L.la, rows,
+                                                           Dk, Dv, s)
+                            : launch_expand<float>(beta, scalar ? log_alpha : nullptr, bf, wf, w8 + L.la, rows, Dk, Dv,
+                                                   s);
         if (e != cudaSuccess) {
             snprintf(g_err, sizeof(g_err), "gdn2_beta_fwd (gate broadcast): %s", cudaGetErrorString(e));
             return report(GDN2_ERR_CUDA);
         }
         if (scalar) la_full = w8 + L.la;
     }
+    if (T > 0 && tc)
+        return fwd_impl(q, k, v, la_full, beta, beta, S0, o, ST, B, T, H, Dk, Dv, chunk, dt, save_states, ws, L.base,
+                        stream, beta);
     return gdn2_fwd(q, k, v, la_full, T > 0 ? w8 + L.b : nullptr, T > 0 ? w8 + L.w : nullptr, S0, o, ST, B, T, H,
                     Dk, Dv, chunk, dt, save_states, ws, L.base, stream);
 }
@@ -279,19 +300,34 @@ gdn2_status gdn2_beta_bwd(gdn2_gate gate, const void* q, const void* k, const vo
     unsigned char* w8 = static_cast<unsigned char*>(ws);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool scalar = gate == GDN2_GATE_GDN;
+    const bool tc = tc_path(dt, Dk, Dv) && ((uintptr_t)beta & 3) == 0;   // the chunk kernels take beta as it is
     const long long rows = (long long)B * T * H;
-    if (T > 0 && !states_saved) {   // the broadcast gates (on saved states, the forward's are still there)
+    if (T > 0 && !states_saved && (!tc || scalar)) {   // the broadcast gates (on saved states, the forward's)
+        void* bf = tc ? nullptr : w8 + L.b;
+        void* wf = tc ? nullptr : w8 + L.w;
         cudaError_t e = dt == GDN2_BF16
-                            ? launch_expand<__nv_bfloat16>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w,
-                                                           w8 + L.la, rows, Dk, Dv, s)
-                            : launch_expand<float>(beta, scalar ? log_alpha : nullptr, w8 + L.b, w8 + L.w, w8 + L.la,
-                                                   rows, Dk, Dv, s);
+                            ? launch_expand<__nv_bfloat16>(beta, scalar ? log_alpha : nullptr, bf, wf, w8 + L.la, rows,
+                                                           Dk, Dv, s)
+                            : launch_expand<float>(beta, scalar ? log_alpha : nullptr, bf, wf, w8 + L.la, rows, Dk, Dv,
+                                                   s);
         if (e != cudaSuccess) {
             snprintf(g_err, sizeof(g_err), "gdn2_beta_bwd (gate broadcast): %s", cudaGetErrorString(e));
             return report(GDN2_ERR_CUDA);
         }
     }
     void* dla_full = scalar ? static_cast<void*>(w8 + L.dla) : dlog_alpha;
+    if (T > 0 && tc) {
+        gdn2_status st = bwd_impl(q, k, v, scalar ? static_cast<const void*>(w8 + L.la) : log_alpha, beta, beta, S0,
+                                  dout, dST, dq, dk, dv, dla_full, dbeta, dbeta, dS0, B, T, H, Dk, Dv, chunk, dt,
+                                  states_saved, ws, L.base, stream, beta, dbeta);
+        if (st != GDN2_OK || !scalar) return st;
+        cudaError_t e = launch_reduce<__nv_bfloat16>(nullptr, nullptr, w8 + L.dla, dbeta, dlog_alpha, rows, Dk, Dv, s);
+        if (e != cudaSuccess) {
+            snprintf(g_err, sizeof(g_err), "gdn2_beta_bwd (decay gradient sum): %s", cudaGetErrorString(e));
+            return report(GDN2_ERR_CUDA);
+        }
+        return GDN2_OK;
+    }
     gdn2_status st = gdn2_bwd(q, k, v, scalar ? static_cast<const void*>(w8 + L.la) : log_alpha,
                               T > 0 ? w8 + L.b : nullptr, T > 0 ? w8 + L.w : nullptr, S0, dout, dST, dq, dk, dv,
                               T > 0 ? dla_full : dlog_alpha, T > 0 ? w8 + L.db : dbeta, T > 0 ? w8 + L.dw : dbeta,

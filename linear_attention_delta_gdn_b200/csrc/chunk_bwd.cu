@@ -60,6 +60,16 @@ constexpr int BPARTS = BT / 128;
 static_assert(TC_STATE_BYTES % (16 * BT) == 0 && TC_DELTA_BYTES % (16 * BT) == 0 && BPARTS * 16 == 64,
               "BT-thread loops");
 
+// The sum of the 8 bf16 values of a 16-byte piece of shared memory
+__device__ __forceinline__ float row8_sum(const unsigned char* src) {
+    const uint4 x = *reinterpret_cast<const uint4*>(src);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xFFFF0000u);
+    return s;
+}
+
 // Copy a [128 lanes x NCOL] fp32 accumulator into a bf16 row tile of 128 rows (row = lane); each of
 // the four warps of a lane quarter takes NCOL / 4 columns.
 template <int NCOL>
@@ -221,6 +231,8 @@ struct BwdMaps {
 struct BwdParams {
     int T, H, BH, nc;
     const __nv_bfloat16 *q_raw, *la_raw;   // raw inputs, read directly only for untame channels
+    const __nv_bfloat16* beta;       // [B, T, H] erase and write gates b = w = beta 1 (kernels instantiated for
+    __nv_bfloat16* dbeta;            // them), and their gradient sum_i db_ti + sum_j dw_tj; else null
     int nrev;                        // CTAs [0, nrev) run the reverse pass of head blockIdx.x
     int join;                        // reverse-pass CTAs take gradient units afterwards
     int grad;                        // this launch computes gradient units
@@ -619,6 +631,7 @@ constexpr uint32_t OFF_DT = 180224;      // Delta^T [128 x 64] (forward image), 
 constexpr uint32_t OFF_DDT = 196608;     // dDelta^T [128 x 64] (reverse-pass image), later staged db
 constexpr uint32_t OFF_PP = 212992;      // prep scratch, then dP^T [64 x 64]; with TT: dw staging, and
 constexpr uint32_t OFF_TT = 221184;      // T, later dA^T   [dP^T | dA^T] as one N = 128 operand
+constexpr uint32_t OFF_SDBW = 229376;    // one scalar gate per token: the dw tile's row sums (64 floats)
 // TMEM columns (M=64 accumulators use lanes 0-15 of each 32-lane quarter)
 constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
     TM_W = 64,                     // dA^T (M=64, 64 columns)
@@ -629,6 +642,7 @@ constexpr uint32_t TM_AP = 0,      // dP^T (M=64)
 constexpr uint32_t LOAD_GATE = 4 * 64 * 128 * 2;                             // b, q, k, log_alpha: the prep's
 constexpr uint32_t LOAD_REST = 3 * 64 * 128 * 2 + (uint32_t)TC_DELTA_BYTES;   // v, w, dout, Delta^T
 constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image, T (dS'^T: cp.async)
+static_assert(OFF_TT + TILE_C <= OFF_SDBW && OFF_SDBW + 64 * 4 <= OFF_BARS, "gradient-unit layout below the barriers");
 }  // namespace cg
 
 // Gradients of chunk c of head `headi`; returns false if a bounded wait gave up. `prefetched`: the S, T
@@ -636,6 +650,10 @@ constexpr uint32_t LOAD_PRE = (uint32_t)TC_STATE_BYTES + TILE_C;     // S image,
 // Lane 0 of warp 9 takes the CTA's next unit from the counter while this one runs and acquires its flag
 // while the G MMAs run; once this unit has finished with the S^T, T and dS'^T tiles, the next unit's
 // images are requested into them. The next unit is published in *nxt.
+// BETA (b = w = beta 1): the b rows of QE and the w tile hold the gate of each token, written by the threads
+// at the start of the unit (no b or w tiles are loaded and b is not reloaded); dw and db are not stored, their
+// row sums (over the value and key channels) go out as dbeta.
+template <bool BETA>
 __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi, int c,
                           Phases& ph, bool prefetched, NextUnit* nxt) {
     using namespace cg;
@@ -671,6 +689,16 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     const uint4 msk = *reinterpret_cast<const uint4*>(p.tp + (head * nc + c) * TC_WY_BYTES + TC_WY_MASK);
     bool ok = true;
     int next_unit = units;    // lane 0 of warp 9: the CTA's next unit (its atomic returns while this unit runs)
+    // BETA: the gates of rows tid / 16 and tid / 16 + 32 (bf16 bits, 0 past the end of the sequence), loaded
+    // first and written out as b and w rows below
+    uint32_t bet16[2] = {0u, 0u};
+    if constexpr (BETA) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const int row = (tid >> 4) + 32 * x;
+            if (t0 + row < T) bet16[x] = __bfloat16_as_ushort(p.beta[((size_t)b * T + t0 + row) * H + h]);
+        }
+    }
     // The loads are issued by lane 0 of several warps at once (a TMA issue takes ~100 cycles); a barrier
     // phase cannot complete before the arrival that carries its expected bytes. Two groups: the prep's
     // inputs (b, q, k, log_alpha, into tiles no output is staged in) go out at once; the rest (v, w, dout,
@@ -680,8 +708,8 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     if (lane == 0) {
         switch (warp) {
         case 0:
-            tc::mbar_arrive_expect_tx(bar_load, LOAD_GATE);
-            tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
+            tc::mbar_arrive_expect_tx(bar_load, LOAD_GATE - (BETA ? 64u * 128u * 2u : 0u));
+            if (!BETA) tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
             break;
         case 1: tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load); break;
         case 2: tma_tile(KH, C, 0, mk, b, h, t0, bar_load); break;
@@ -699,15 +727,27 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::bulk_wait_read();   // the previous unit's dq, dlog_alpha stores have read DU
     }
     if (lane == 0 && (warp == 1 || warp == 2)) tc::bulk_wait_read();   // its dk, db stores: DT, DDT
+    if constexpr (BETA) {   // rows r and r + 32 of b (QE rows 0..63) and w (WW): 8 copies of beta per piece
+        const int r = tid >> 4, panel = (tid >> 3) & 1, chunk = tid & 7;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const int row = r + 32 * x;
+            const uint32_t v16 = bet16[x] * 0x10001u;
+            const uint4 v = make_uint4(v16, v16, v16, v16);
+            *reinterpret_cast<uint4*>(QE + panel * (2 * C * 128) + row * 128 + chunk * 16) = v;
+            *reinterpret_cast<uint4*>(WW + panel * (C * 128) + row * 128 + chunk * 16) = v;
+        }
+    }
     __syncthreads();   // orders thread 0's acquire and its wait before the loads and copies below
     if (lane == 0) {
         const unsigned char* src = p.tp + (head * nc + c) * TC_WY_BYTES;   // T | P | Wm
         switch (warp) {
         case 4:
-            tc::mbar_arrive_expect_tx(bar_rest, prefetched ? LOAD_REST : LOAD_REST + LOAD_PRE);
+            tc::mbar_arrive_expect_tx(bar_rest, (prefetched ? LOAD_REST : LOAD_REST + LOAD_PRE) -
+                                                    (BETA ? 64u * 128u * 2u : 0u));
             tma_tile(DU, 2 * C, C, mv, b, h, t0, bar_rest);
             break;
-        case 5: tma_tile(WW, C, 0, mw, b, h, t0, bar_rest); break;
+        case 5: if (!BETA) tma_tile(WW, C, 0, mw, b, h, t0, bar_rest); break;
         case 6: tma_tile(DU, 2 * C, 0, mdo, b, h, t0, bar_rest); break;
         case 7:
             tc::bulk_load(DT, p.deltas + (head * nc + c) * TC_DELTA_BYTES, (uint32_t)TC_DELTA_BYTES, bar_rest);
@@ -809,7 +849,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     sync_for_mma();
     // store dv (lane 0 of warp 1) and dw (warp 2; rows past the end of the sequence are skipped), and bring b
     // back for the gate chain (warp 3; w is consumed), while thread 0 issues the MMAs below
-    if (lane == 0 && warp >= 1 && warp <= 3) {
+    if (lane == 0 && (warp == 1 || (!BETA && (warp == 2 || warp == 3)))) {
         if (warp == 3) {
             tc::mbar_arrive_expect_tx(bar_b, 64 * 128 * 2);
             tma_tile(WW, C, 0, mb, b, h, t0, bar_b);
@@ -833,6 +873,14 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     }
     if (lane == 0 && (warp == 1 || warp == 2))
         tc::bulk_wait_read();   // the dv, dw stores have read their tiles (DDT, TT, PP are overwritten below)
+    if constexpr (BETA) {   // row t of the dw tile (PP | TT) summed over the value channels, while the MMAs run
+        const int t = tid >> 3, part = tid & 7;
+        float sdw = row8_sum(PP + t * 128 + part * 16) + row8_sum(PP + C * 128 + t * 128 + part * 16);
+        sdw += __shfl_xor_sync(0xffffffffu, sdw, 1);
+        sdw += __shfl_xor_sync(0xffffffffu, sdw, 2);
+        sdw += __shfl_xor_sync(0xffffffffu, sdw, 4);
+        if (part == 0) reinterpret_cast<float*>(sm + OFF_SDBW)[t] = sdw;
+    }
     wait_mma();
     tc::tc_fence_before();
     __syncthreads();
@@ -908,8 +956,10 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         nxt->prefetched = ready;
     }
     wait_mma();
-    ok = tc::mbar_wait(bar_b, ph.b) && ok;
-    ph.b ^= 1;
+    if (!BETA) {
+        ok = tc::mbar_wait(bar_b, ph.b) && ok;
+        ph.b ^= 1;
+    }
 
     // ---- untame channels: their pair terms are summed exactly below, from alpha and the raw q of the chunk
     // (fp32 [64 tokens][128 channels] tables over the S^T and dS'^T tiles, which the G MMAs and the rowsum
@@ -983,7 +1033,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     tc::fence_async_smem();   // every read of S^T and dS'^T (G MMAs, rowsum) precedes the prefetch below, and
                               // dq, dk, db (final after pass 1) are visible to the tensor stores
     __syncthreads();          // also orders warp 9's acquire before every thread's copy of the next dS'^T
-    if (lane == 0 && warp < 3) {   // dq, dk, db (lane 0 of warps 0, 1, 2) go out while pass 2 runs; rows past
+    if (lane == 0 && warp < (BETA ? 2 : 3)) {   // dq, dk, db (lane 0 of warps 0, 1, 2) go out while pass 2 runs; rows past
                                    // the end of the sequence are skipped
         const CUtensorMap* map = warp == 0 ? mdq : (warp == 1 ? mdk : mdb);
         const unsigned char* tile = warp == 0 ? DU : (warp == 1 ? DT : DDT);
@@ -991,6 +1041,16 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
         tc::tma_store_4d(map, 0, h, t0, b, tile);
         tc::tma_store_4d(map, 64, h, t0, b, tile + panel);
         tc::bulk_commit();
+    }
+    if constexpr (BETA) {   // dbeta_t: row t of the db tile (DDT) summed over the key channels, plus the dw sum
+        const int t = tid >> 3, part = tid & 7;
+        float sdb = row8_sum(DDT + t * 128 + part * 16) + row8_sum(DDT + C * 128 + t * 128 + part * 16);
+        sdb += __shfl_xor_sync(0xffffffffu, sdb, 1);
+        sdb += __shfl_xor_sync(0xffffffffu, sdb, 2);
+        sdb += __shfl_xor_sync(0xffffffffu, sdb, 4);
+        if (part == 0 && t < L)
+            p.dbeta[((size_t)b * T + t0 + t) * H + h] =
+                __float2bfloat16(sdb + reinterpret_cast<const float*>(sm + OFF_SDBW)[t]);
     }
     int nxt_head = 0, nxt_c = 0;
     if (nxt->prefetched) unit_at(p, nxt->unit, &nxt_head, &nxt_c);
@@ -1034,6 +1094,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     return ok;
 }
 
+template <bool BETA>
 __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
@@ -1094,7 +1155,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
                 __syncthreads();
                 continue;
             }
-            if (!grad_unit(maps, p, sm, tmem, headi, c, ph, pre, nxt)) {
+            if (!grad_unit<BETA>(maps, p, sm, tmem, headi, c, ph, pre, nxt)) {
                 // a bounded wait gave up: let a prefetch in flight land before leaving
                 if (tid == 0 && nxt->prefetched) (void)tc::mbar_wait(reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48), ph.pre);
                 tc::cp_async_wait_all();
@@ -1118,8 +1179,12 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
+    // one scalar gate per head and token: the kernels built for it (the b, w, db and dw maps are never used)
+    const bool beta = a.beta != nullptr && !(a.map_A && a.map_B);
+    void (*kern)(const BwdMaps, const BwdParams) = beta ? chunk_bwd_kernel<true> : chunk_bwd_kernel<false>;
     BwdMaps maps;
-    const void* ptrs[13] = {a.q, a.k, a.v, a.la, a.b, a.w, a.dout, a.dq, a.dk, a.db, a.dla, a.dv, a.dw};
+    const void* ptrs[13] = {a.q, a.k, a.v, a.la, beta ? a.q : a.b, beta ? a.v : a.w, a.dout, a.dq, a.dk,
+                            beta ? a.dq : a.db, a.dla, a.dv, beta ? a.dv : a.dw};
     CUtensorMap* mp[13] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w, &maps.dout,
                            &maps.dq, &maps.dk, &maps.db, &maps.dla, &maps.dv, &maps.dw};
     if (a.map_A && a.map_B)   // no gradient units run: their output maps only need a valid address
@@ -1127,7 +1192,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     for (int i = 0; i < 13; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     LaunchFacts lf{};
-    cudaError_t e = launch_facts(chunk_bwd_kernel, BT, SMEM_BYTES_ALL, &lf);
+    cudaError_t e = launch_facts(kern, BT, SMEM_BYTES_ALL, &lf);
     if (e != cudaSuccess) return e;
     const int nsm = lf.nsm, coop = lf.coop, occ = lf.occ;
     const int BH = d.B * d.H, nc = d.nchunks();
@@ -1137,6 +1202,10 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     BwdParams p{};
     p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
     p.q_raw = static_cast<const __nv_bfloat16*>(a.q); p.la_raw = static_cast<const __nv_bfloat16*>(a.la);
+    if (beta) {
+        p.beta = static_cast<const __nv_bfloat16*>(a.beta);
+        p.dbeta = static_cast<__nv_bfloat16*>(a.dbeta);
+    }
     p.dST = a.dST; p.dS0 = a.dS0;
     p.dv = static_cast<__nv_bfloat16*>(a.dv); p.dw = static_cast<__nv_bfloat16*>(a.dw);
     p.states = a.states; p.deltas = a.deltas; p.tp = a.tp; p.dstates = a.dstates; p.ddeltas = a.ddeltas;
@@ -1153,7 +1222,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
         pm.nrev = ntasks < slots ? ntasks : slots;
         {
             TraceScope trace(K_CHUNK_BWD, s);
-            chunk_bwd_kernel<<<pm.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pm);
+            kern<<<pm.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pm);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         if (!R) return cudaSuccess;
@@ -1181,7 +1250,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
         p1.nrev = n1 < slots ? n1 : slots;
         {
             TraceScope trace(K_CHUNK_BWD, s);
-            chunk_bwd_kernel<<<p1.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, p1);
+            kern<<<p1.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, p1);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         if ((e = split_prefix_launch(a.sbuf, R, BH, s)) != cudaSuccess) return e;
@@ -1192,17 +1261,17 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
         if (coop && !cooperative_disabled() && n3 < slots) {
             p3.nrev = n3; p3.join = 1; p3.grad = 1;
             void* args[2] = {&maps, &p3};
-            e = cudaLaunchCooperativeKernel((const void*)chunk_bwd_kernel, dim3(slots), dim3(BT), args, SMEM_BYTES_ALL, s);
+            e = cudaLaunchCooperativeKernel((const void*)kern, dim3(slots), dim3(BT), args, SMEM_BYTES_ALL, s);
             if (e == cudaSuccess) return cudaSuccess;
             (void)cudaGetLastError();
         }
         BwdParams pr = p3;
         pr.nrev = n3 < slots ? n3 : slots; pr.join = 0; pr.grad = 0;
-        chunk_bwd_kernel<<<pr.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pr);
+        kern<<<pr.nrev, BT, SMEM_BYTES_ALL, s>>>(maps, pr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         BwdParams pg = p3;
         pg.nrev = 0; pg.join = 0; pg.grad = 1;
-        chunk_bwd_kernel<<<units < slots ? units : slots, BT, SMEM_BYTES_ALL, s>>>(maps, pg);
+        kern<<<units < slots ? units : slots, BT, SMEM_BYTES_ALL, s>>>(maps, pg);
         return cudaGetLastError();
     }
 
@@ -1211,17 +1280,17 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     if (coop && !cooperative_disabled() && BH < slots) {
         p.nrev = BH; p.join = 1; p.grad = 1;
         void* args[2] = {&maps, &p};
-        e = cudaLaunchCooperativeKernel((const void*)chunk_bwd_kernel, dim3(slots), dim3(BT), args, SMEM_BYTES_ALL, s);
+        e = cudaLaunchCooperativeKernel((const void*)kern, dim3(slots), dim3(BT), args, SMEM_BYTES_ALL, s);
         if (e == cudaSuccess) return cudaSuccess;
         (void)cudaGetLastError();   // not launched: fall back to two launches
     }
     BwdParams pr = p;   // reverse pass only
     pr.nrev = BH; pr.join = 0; pr.grad = 0;
-    chunk_bwd_kernel<<<BH, BT, SMEM_BYTES_ALL, s>>>(maps, pr);
+    kern<<<BH, BT, SMEM_BYTES_ALL, s>>>(maps, pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     BwdParams pg = p;   // gradient units only; every flag is set when they start
     pg.nrev = 0; pg.join = 0; pg.grad = 1;
-    chunk_bwd_kernel<<<units < slots ? units : slots, BT, SMEM_BYTES_ALL, s>>>(maps, pg);
+    kern<<<units < slots ? units : slots, BT, SMEM_BYTES_ALL, s>>>(maps, pg);
     return cudaGetLastError();
 }
 

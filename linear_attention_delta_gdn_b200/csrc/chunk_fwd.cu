@@ -73,8 +73,9 @@ constexpr uint32_t GC = 104448;     // 2 x fp32 gC[128] (by unit parity)
 constexpr uint32_t STAGE = TF;      // exact path for untame channels: fp32 [4][64][16] raw-input stage
 constexpr uint32_t BAR = 2 * PIPE;  // 4 mbarriers (inputs, mma per pipeline), tmem base, abort flag
 constexpr uint32_t UMASK = BAR + 64;  // untame-channel masks: [pipeline][unit parity][4 words]
+constexpr uint32_t BETA = UMASK + 64; // scalar gates: [pipeline][unit parity][64 tokens] 32-bit words holding them
 }  // namespace wy
-constexpr uint32_t SMEM_BYTES = (sp::END > wy::UMASK + 64 ? sp::END : wy::UMASK + 64) + 1024;
+constexpr uint32_t SMEM_BYTES = (sp::END > wy::BETA + 1024 ? sp::END : wy::BETA + 1024) + 1024;
 static_assert(sp::MASK + 32 <= sp::UU1 && sp::UU1 % 1024 == 0 && sp::WW1 % 1024 == 0, "consumer layout");
 static_assert(4 * 16 * XS * 4 <= wy::GC - wy::SX && 8 * 128 * 4 <= wy::GC - wy::SX, "producer scratch fits");
 static_assert(4 * 64 * 16 * 4 == TILE_64x128 && wy::STAGE + 4 * 64 * 16 * 4 <= wy::SX, "untame stage fits");
@@ -111,6 +112,8 @@ struct FwdParams {
                                    // 5: the maps of the whole sequence of every head (map_N, map_M)
     float* sbuf;                   // with split_R: per head, segment start states, then the maps N and M
     float *map_N, *map_M;          // phase 5: [BH][D][D] each
+    const __nv_bfloat16* beta;     // [B, T, H] erase and write gates b = w = beta 1 (kernels instantiated for
+                                   // them: no b or w tiles are loaded), else null
 };
 
 // ---- consumer tasks
@@ -208,9 +211,27 @@ __device__ __forceinline__ void sync_for_mma() {   // smem written by threads + 
 //   block totals of the cumsum go through red (fp32 [8][128]). The threads of the last token block, which
 //   hold G_C, OR the untame channels (log-decay over the chunk, -G_C, above TAME_LOG_DECAY) into umask
 //   (bit = channel); their Kt is still written here and cleared afterwards (untame chunks only).
-template <typename Sync>
+// One scalar gate per head and token (beta [B, T, H] bf16, 4-byte aligned): the 64 tokens of a chunk are copied
+// into shared memory as the 32-bit words that hold them (cp.async, 4 bytes each, zeros past the end of the
+// sequence); token row r of a chunk whose first element is e0 = (b T + t0) H + h sits in the high half of its
+// word when e0 + r H is odd.
+__device__ __forceinline__ void beta_words_copy(uint32_t* dst, const __nv_bfloat16* beta, int b, int h, int t0, int T,
+                                                int H, int row) {
+    const size_t e = ((size_t)b * T + t0 + row) * H + h;
+    const bool valid = t0 + row < T;
+    tc::cp_async4(dst + row, valid ? beta + (e & ~(size_t)1) : beta, valid);
+}
+__device__ __forceinline__ float beta_word_value(const uint32_t* words, int row, int e0_odd, int H_odd) {
+    const uint32_t w = words[row];
+    return __uint_as_float(((e0_odd ^ (row & H_odd)) ? w >> 16 : w & 0xFFFFu) << 16);
+}
+
+// With BETA, b is one value per token, read from the chunk's beta words (bw, e0_odd, H_odd: beta_word_value)
+// after the barrier below (QE rows 0..63 hold no b tile).
+template <bool BETA, typename Sync>
 __device__ __forceinline__ void gate_prep_wg(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
-                                             float* gC_out, float* red, unsigned int* umask, int wt, Sync&& wg_sync) {
+                                             float* gC_out, float* red, unsigned int* umask, int wt, const uint32_t* bw,
+                                             int e0_odd, int H_odd, Sync&& wg_sync) {
     constexpr int RB = 8;
     const int cg = wt & 15, tb = wt >> 4;
     float G[RB][8];
@@ -248,7 +269,13 @@ __device__ __forceinline__ void gate_prep_wg(unsigned char* QE, const unsigned c
         const int row = RB * tb + u;
         float kk[8], bb[8], qq[8], e[8], kt[8];
         tc::ld_row8(KH, C, row, cg, kk);
-        tc::ld_row8(QE, 2 * C, row, cg, bb);
+        if constexpr (BETA) {
+            const float bv = beta_word_value(bw, row, e0_odd, H_odd);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) bb[c] = bv;
+        } else {
+            tc::ld_row8(QE, 2 * C, row, cg, bb);
+        }
         tc::ld_row8(QE, 2 * C, C + row, cg, qq);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -285,7 +312,8 @@ __device__ __noinline__ void clear_untame_kt(unsigned char* KT, const unsigned i
 // tokens][16]); thread (column s = wt % 64, A or P = wt / 64) keeps its 64 sums in registers and adds them at
 // the end. Called by the whole warpgroup; ends with a barrier.
 __device__ __noinline__ void untame_fixup_wg(int T, int H, const __nv_bfloat16* gq, const __nv_bfloat16* gk,
-                                             const __nv_bfloat16* gla, const __nv_bfloat16* gb, int b, int h, int t0,
+                                             const __nv_bfloat16* gla, const __nv_bfloat16* gb,
+                                             const __nv_bfloat16* gbeta, int b, int h, int t0,
                                              const unsigned int* umask, float* sA, unsigned char* PP, float* stage,
                                              unsigned char* list, unsigned char* kh_img, int wt, int wg) {
     auto wg_sync = [&]() { tc::named_sync(1 + wg, 128); };
@@ -317,7 +345,8 @@ __device__ __noinline__ void untame_fixup_wg(int T, int H, const __nv_bfloat16* 
                     const size_t off = tok_off(b, t0 + tau, h, T, H, D) + ch;
                     al = fast_exp(__bfloat162float(gla[off]));
                     kk = __bfloat162float(gk[off]);
-                    ee = __bfloat162float(gb[off]) * kk;
+                    ee = (gbeta ? __bfloat162float(gbeta[((size_t)b * T + t0 + tau) * H + h])
+                                : __bfloat162float(gb[off])) * kk;
                     qq = __bfloat162float(gq[off]);
                 }
                 sAl[tau * 16 + c] = al;
@@ -465,7 +494,9 @@ __device__ __forceinline__ void tmem_m64_to_tile_wg(uint32_t lane_base_col, unsi
     }
 }
 
+template <bool BETA>
 __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int pid) {
+    constexpr uint32_t LOAD_BYTES = PROD_LOAD_BYTES - (BETA ? 64u * 128u * 2u : 0u);   // no b tile with BETA
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wg = warp >> 2, wq = warp & 3, wt = tid & 127;   // pipeline, warp and thread in it
     unsigned char* pb = sm + wg * wy::PIPE;
@@ -519,17 +550,34 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     if (u0 < units && wt == 0) {   // the first unit's tiles
         int b, h, t0;
         coords(u0, b, h, t0);
-        tc::mbar_arrive_expect_tx(bar_in, PROD_LOAD_BYTES);
+        tc::mbar_arrive_expect_tx(bar_in, LOAD_BYTES);
         tma_tile(QE, 2 * C, C, &m.q, b, h, t0, bar_in);
         tma_tile(KT, C, 0, &m.la, b, h, t0, bar_in);
         tma_tile(KH, C, 0, &m.k, b, h, t0, bar_in);
-        tma_tile(QE, 2 * C, 0, &m.b, b, h, t0, bar_in);
+        if (!BETA) tma_tile(QE, 2 * C, 0, &m.b, b, h, t0, bar_in);
     }
+    // BETA: a unit's beta words (by unit parity), copied one unit ahead by threads 0..63 of the pipeline
+    uint32_t* betaw = reinterpret_cast<uint32_t*>(sm + wy::BETA) + 128 * wg;
+    auto copy_beta = [&](int u, int par) {
+        int b_, h_, t0_;
+        coords(u, b_, h_, t0_);
+        beta_words_copy(betaw + 64 * par, p.beta, b_, h_, t0_, p.T, p.H, wt);
+        tc::cp_async_commit();
+    };
+    if (BETA && u0 < units && wt < 64) copy_beta(u0, 0);
     for (int u = u0; u < units; u += npipe, ++kunit) {
         const int c = u / p.BH, head = u % p.BH;
         const bool next = u + npipe < units;
         int nb = 0, nh = 0, nt0 = 0;
         if (next) coords(u + npipe, nb, nh, nt0);
+        if (BETA && wt < 64) {   // this unit's words complete (the prep reads them after its first barrier)
+            if (next) {
+                copy_beta(u + npipe, (kunit + 1) & 1);
+                tc::cp_async_wait_but1();
+            } else {
+                tc::cp_async_wait_all();
+            }
+        }
         float* gC = reinterpret_cast<float*>(pb + wy::GC + (kunit & 1) * 512);
         if (!tc::mbar_wait(bar_in, ph_in)) { atomicExch(abort_flag, 1); atomicOr(&g_fwd_error, 2u); }
         ph_in ^= 1;
@@ -541,7 +589,10 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         if (wt < 4) reinterpret_cast<unsigned int*>(sm + wy::UMASK)[8 * wg + 4 * ((kunit + 1) & 1) + wt] = 0u;
         unsigned char* img = p.wyimg + ((size_t)head * p.nc + c) * TC_WY_BYTES;
         const bool img_ok = GDN2_IN(g_fwd_error, head < p.BH && c < p.nc);   // else the image is not written
-        gate_prep_wg(QE, KH, KT, gC, sX, umask, wt, wg_sync);
+        {
+            const int e0 = (int)((((size_t)(head / p.H) * p.T + (size_t)c * C) * p.H + head % p.H) & 1);
+            gate_prep_wg<BETA>(QE, KH, KT, gC, sX, umask, wt, betaw + 64 * (kunit & 1), e0, p.H & 1, wg_sync);
+        }
         sync_for_mma_wg();
         const bool untame = (umask[0] | umask[1] | umask[2] | umask[3]) != 0u;   // the same on every thread
         if (untame) {   // their Kt columns are cleared before the image's Kt and M1 read KT
@@ -567,7 +618,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         wait_mma();
         if (wt == 0 && next) {   // the next unit's q and log_alpha over Qt, Kt
             tc::bulk_wait_read();
-            tc::mbar_arrive_expect_tx(bar_in, PROD_LOAD_BYTES);
+            tc::mbar_arrive_expect_tx(bar_in, LOAD_BYTES);
             tma_tile(QE, 2 * C, C, &m.q, nb, nh, nt0, bar_in);
             tma_tile(KT, C, 0, &m.la, nb, nh, nt0, bar_in);
             inflight = true;
@@ -578,7 +629,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         if (untame && img_ok) {   // exact terms of the channels left out of M1 (TF is free until the solve)
             int b, h, t0;
             coords(u, b, h, t0);
-            untame_fixup_wg(p.T, p.H, p.q, p.k, p.la, p.b, b, h, t0, umask, sA, PP,
+            untame_fixup_wg(p.T, p.H, p.q, p.k, p.la, p.b, BETA ? p.beta : nullptr, b, h, t0, umask, sA, PP,
                             reinterpret_cast<float*>(pb + wy::STAGE), reinterpret_cast<unsigned char*>(sX),
                             img + TC_WY_KH, wt, wg);
         }
@@ -593,7 +644,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             tc::mma_commit(bar_mma);
         }
         wait_mma();
-        if (wt == 0 && next) tma_tile(QE, 2 * C, 0, &m.b, nb, nh, nt0, bar_in);   // the next unit's b over Et
+        if (!BETA && wt == 0 && next) tma_tile(QE, 2 * C, 0, &m.b, nb, nh, nt0, bar_in);   // the next unit's b over Et
         tmem_m64_to_tile_wg(lane_base + (tm_w - tmem), pb + wy::TF, C, wq, lane);   // Wm over the fp32 T
         sync_for_mma_wg();
         if (wt == 0) {   // the previous unit's flag (all its stores are older than this unit's first group);
@@ -614,6 +665,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
     }
     // after an abort: the next unit's loads land before the CTA's shared memory is released
     if (wt == 0 && inflight) (void)tc::mbar_wait(bar_in, ph_in);
+    if (BETA) tc::cp_async_wait_all();   // and the beta words in flight
 }
 
 // ------------------------------------------------------------------ consumer
@@ -638,6 +690,7 @@ __device__ __noinline__ void kh_from_kt(unsigned char* KT, const unsigned char* 
     }
 }
 
+template <bool BETA>
 __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int cid) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // v and w tiles by chunk parity: chunk c + 2 is loaded while chunk c + 1's tiles wait in the other pair
@@ -708,9 +761,9 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             if (lane != 0 || warp > 1) return;
             const int t0 = c * C;
             if (warp == 0) {
-                tc::mbar_arrive_expect_tx(bar_ld(c), CONS_LOAD_BYTES);
+                tc::mbar_arrive_expect_tx(bar_ld(c), CONS_LOAD_BYTES - (BETA ? 64u * 128u * 2u : 0u));
                 tma_tile(UUp(c), C, 0, &m.v, b, h, t0, bar_ld(c));
-            } else {
+            } else if (!BETA) {
                 tma_tile(WWp(c), C, 0, &m.w, b, h, t0, bar_ld(c));
             }
         };
@@ -736,6 +789,19 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
         if (!zero_u) {
             issue_loads(c0);
             if (c0 + 1 < c1) issue_loads(c0 + 1);
+        }
+        // BETA: w is the gate of the token; chunk c's beta words go into its (unused) w tile, copied with its v
+        // tile two chunks ahead and complete at the cp.async wait of the chunk before
+        auto copy_beta = [&](int c) {
+            if (tid < 64) {
+                beta_words_copy(reinterpret_cast<uint32_t*>(WWp(c)), p.beta, b, h, c * C, T, H, tid);
+                tc::cp_async_commit();
+            }
+        };
+        if (BETA && !zero_u) {
+            copy_beta(c0);
+            if (c0 + 1 < c1) copy_beta(c0 + 1);
+            tc::cp_async_wait_all();   // chunk c0's words, before the barrier below
         }
         if (tid == 0) wait_wy(head, c0);
         // start state: S^T row j = column j of the start matrix (zero if none, or the identity)
@@ -784,11 +850,19 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
                 const int idx = tid + NT * e, row = idx >> 4, g = idx & 15;
                 float vv[8], ww[8];
                 tc::ld_row8(UU, C, row, g, vv);
-                tc::ld_row8(WW, C, row, g, ww);
+                if constexpr (BETA) {
+                    const float bv = beta_word_value(reinterpret_cast<const uint32_t*>(WW), row,
+                                                     (int)((((size_t)b * T + (size_t)c * C) * H + h) & 1), H & 1);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) ww[x] = bv;
+                } else {
+                    tc::ld_row8(WW, C, row, g, ww);
+                }
 #pragma unroll
                 for (int x = 0; x < 8; ++x) vv[x] *= ww[x];
                 tc::st_row8(UU, C, row, g, vv);
             }
+
             tc::cp_async_wait_all();   // this chunk's WY image
             sync_for_mma();
             // a chunk with untame channels updates the state with Kh on a state scaled by gC first, the others
@@ -834,7 +908,10 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
             }
             wait_mma();
             // this chunk's v (read by M3) and w buffers are free: chunk c + 2's tiles go there
-            if (!zero_u && c + 2 < c1) issue_loads(c + 2);
+            if (!zero_u && c + 2 < c1) {
+                issue_loads(c + 2);
+                if (BETA) copy_beta(c + 2);
+            }
             tmem_to_tile_rows<64>(lane_base + TM_D, DT, warp, lane);   // Delta^T (lane j) -> bf16 rows
             sync_for_mma();
             if (deltas && tid == 0) {   // Delta^T of this chunk for the backward
@@ -911,6 +988,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     }
 }
 
+template <bool BETA>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant__ Maps maps, const FwdParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
@@ -931,8 +1009,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             for (int i = 0; i < 16; ++i) reinterpret_cast<unsigned int*>(sm + wy::UMASK)[i] = 0u;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&maps.q); tc::tma_prefetch_desc(&maps.k); tc::tma_prefetch_desc(&maps.la);
-        if (consumer) { tc::tma_prefetch_desc(&maps.v); tc::tma_prefetch_desc(&maps.w); }
-        else tc::tma_prefetch_desc(&maps.b);
+        if (consumer) {
+            tc::tma_prefetch_desc(&maps.v);
+            if (!BETA) tc::tma_prefetch_desc(&maps.w);
+        } else if (!BETA) {
+            tc::tma_prefetch_desc(&maps.b);
+        }
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_base_ptr, TM_COLS);
@@ -942,8 +1024,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_base_ptr;
-    if (consumer) run_consumer(maps, p, sm, tmem, blockIdx.x);
-    else run_producer(maps, p, sm, tmem, blockIdx.x - p.ncons);
+    if (consumer) run_consumer<BETA>(maps, p, sm, tmem, blockIdx.x);
+    else run_producer<BETA>(maps, p, sm, tmem, blockIdx.x - p.ncons);
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -1075,7 +1157,7 @@ static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool
     for (int i = 0; i < 6; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     LaunchFacts lf{};
-    cudaError_t e = launch_facts(chunk_fwd_kernel, NT, SMEM_BYTES, &lf);
+    cudaError_t e = launch_facts(chunk_fwd_kernel<false>, NT, SMEM_BYTES, &lf);
     if (e != cudaSuccess) return e;
     const int BH = d.B * d.H, nc = d.nchunks(), units = BH * nc, slots = lf.nsm * lf.occ;
     FwdParams p{};
@@ -1089,7 +1171,7 @@ static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool
     pp.nprod = units < slots ? units : slots;
     {
         TraceScope trace(K_CHUNK_FWD, s);
-        chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+        chunk_fwd_kernel<false><<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (!with_maps) return cudaSuccess;
@@ -1102,7 +1184,7 @@ static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool
     pc.ncons = ntasks < slots ? ntasks : slots;
     {
         TraceScope trace(K_CHUNK_FWD, s);
-        chunk_fwd_kernel<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
+        chunk_fwd_kernel<false><<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (!R) return cudaSuccess;
@@ -1130,13 +1212,15 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     if (a.map_N && a.map_M) return chunk_fwd_map_launch(a, s);
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
+    // one scalar gate per head and token: the kernels built for it (the b and w maps are then never read)
+    void (*kern)(const Maps, const FwdParams) = a.beta ? chunk_fwd_kernel<true> : chunk_fwd_kernel<false>;
     Maps maps;
-    const void* ptrs[6] = {a.q, a.k, a.v, a.la, a.b, a.w};
+    const void* ptrs[6] = {a.q, a.k, a.v, a.la, a.beta ? a.q : a.b, a.beta ? a.v : a.w};
     CUtensorMap* mp[6] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w};
     for (int i = 0; i < 6; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     LaunchFacts lf{};
-    cudaError_t e = launch_facts(chunk_fwd_kernel, NT, SMEM_BYTES, &lf);
+    cudaError_t e = launch_facts(kern, NT, SMEM_BYTES, &lf);
     if (e != cudaSuccess) return e;
     const int nsm = lf.nsm, coop = lf.coop, occ = lf.occ;
     const int BH = d.B * d.H, nc = d.nchunks();
@@ -1147,6 +1231,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     p.T = d.T; p.H = d.H; p.BH = BH; p.nc = nc;
     p.q = static_cast<const __nv_bfloat16*>(a.q); p.k = static_cast<const __nv_bfloat16*>(a.k);
     p.la = static_cast<const __nv_bfloat16*>(a.la); p.b = static_cast<const __nv_bfloat16*>(a.b);
+    p.beta = static_cast<const __nv_bfloat16*>(a.beta);
     p.S0 = a.S0; p.o = static_cast<__nv_bfloat16*>(a.o); p.ST = a.ST;
     p.states = a.states; p.deltas = a.deltas; p.wyimg = a.wy; p.flags = a.flags;
     if ((e = cudaMemsetAsync(a.flags, 0, (size_t)units * sizeof(unsigned int), s)) != cudaSuccess) return e;
@@ -1161,7 +1246,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
         {
             TraceScope trace(K_CHUNK_FWD, s);
             if (!test_skip_producers()) {
-                chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+                kern<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
         }
@@ -1173,7 +1258,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
             pc.ncons = ntasks < slots ? ntasks : slots;
             {
                 TraceScope trace(K_CHUNK_FWD, s);
-                chunk_fwd_kernel<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
+                kern<<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
             if (phase == 1 && (e = split_prefix_launch(a.sbuf, R, BH, s)) != cudaSuccess) return e;
@@ -1188,7 +1273,7 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
         p.ncons = BH;
         p.nprod = slots - BH < units ? slots - BH : units;
         void* args[2] = {&maps, &p};
-        e = cudaLaunchCooperativeKernel((const void*)chunk_fwd_kernel, dim3(p.ncons + p.nprod), dim3(NT), args,
+        e = cudaLaunchCooperativeKernel((const void*)kern, dim3(p.ncons + p.nprod), dim3(NT), args,
                                         SMEM_BYTES, s);
         if (e == cudaSuccess) return cudaSuccess;
         (void)cudaGetLastError();   // not launched: fall back to two launches
@@ -1197,13 +1282,13 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     pp.ncons = 0;
     pp.nprod = units < slots ? units : slots;
     if (!test_skip_producers()) {
-        chunk_fwd_kernel<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+        kern<<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     FwdParams pc = p;   // consumers only; every flag is set when they start
     pc.ncons = BH;
     pc.nprod = 0;
-    chunk_fwd_kernel<<<BH, NT, SMEM_BYTES, s>>>(maps, pc);
+    kern<<<BH, NT, SMEM_BYTES, s>>>(maps, pc);
     return cudaGetLastError();
 }
 

@@ -193,10 +193,14 @@ size_t gdn2_workspace_size(gdn2_op op, int B, int T, int H, int Dk, int Dv, int 
     return 0;
 }
 
-gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+}  // extern "C"
+
+namespace gdn2 {
+
+gdn2_status fwd_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
                      const void* w, const float* S0, void* o, float* ST, int B, int T, int H, int Dk,
                      int Dv, int chunk, gdn2_dtype dt, int save_states, void* ws, size_t ws_bytes,
-                     void* stream) {
+                     void* stream, const void* beta) {
     NvtxRange nvtx("gdn2_fwd");
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
@@ -218,6 +222,7 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
         ChunkFwdArgs a{};
         a.d = d;
         a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
+        a.beta = beta;
         a.S0 = S0; a.o = o; a.ST = ST;
         unsigned char* wsb = static_cast<unsigned char*>(ws);
         const bool keep = save_states != 0;
@@ -238,11 +243,11 @@ gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* lo
     return cuda_status(recurrent_launch(a, s), "gdn2_fwd (recurrent path)");
 }
 
-gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+gdn2_status bwd_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
                      const void* w, const float* S0, const void* dout, const float* dST, void* dq,
                      void* dk, void* dv, void* dlog_alpha, void* db, void* dw, float* dS0, int B, int T,
                      int H, int Dk, int Dv, int chunk, gdn2_dtype dt, int states_saved, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     size_t ws_bytes, void* stream, const void* beta, void* dbeta) {
     NvtxRange nvtx("gdn2_bwd");
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
@@ -268,6 +273,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
             ChunkFwdArgs f{};
             f.d = d;
             f.q = q; f.k = k; f.v = v; f.la = log_alpha; f.b = b; f.w = w;
+            f.beta = beta;
             f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.deltas = wsb + tc_delta_offset(d);
             f.wy = wsb + tc_tp_offset(d);
             f.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, true));
@@ -280,6 +286,7 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
         a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w; a.dout = dout;
         a.dST = dST;
         a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.db = db; a.dw = dw; a.dS0 = dS0;
+        a.beta = beta; a.dbeta = dbeta;
         a.states = wsb;
         a.tp = wsb + tc_tp_offset(d);
         a.deltas = wsb + tc_delta_offset(d);
@@ -311,6 +318,27 @@ gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* lo
     a.seg = reinterpret_cast<float*>(extra);
     a.segdelta = reinterpret_cast<float*>(extra + align256(seg));
     return cuda_status(recurrent_launch(a, s), "gdn2_bwd (recurrent path)");
+}
+
+}  // namespace gdn2
+
+extern "C" {
+
+gdn2_status gdn2_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                     const void* w, const float* S0, void* o, float* ST, int B, int T, int H, int Dk,
+                     int Dv, int chunk, gdn2_dtype dt, int save_states, void* ws, size_t ws_bytes,
+                     void* stream) {
+    return fwd_impl(q, k, v, log_alpha, b, w, S0, o, ST, B, T, H, Dk, Dv, chunk, dt, save_states, ws, ws_bytes,
+                    stream, nullptr);
+}
+
+gdn2_status gdn2_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
+                     const void* w, const float* S0, const void* dout, const float* dST, void* dq,
+                     void* dk, void* dv, void* dlog_alpha, void* db, void* dw, float* dS0, int B, int T,
+                     int H, int Dk, int Dv, int chunk, gdn2_dtype dt, int states_saved, void* ws,
+                     size_t ws_bytes, void* stream) {
+    return bwd_impl(q, k, v, log_alpha, b, w, S0, dout, dST, dq, dk, dv, dlog_alpha, db, dw, dS0, B, T, H, Dk, Dv,
+                    chunk, dt, states_saved, ws, ws_bytes, stream, nullptr, nullptr);
 }
 
 // Shared checks of gdn2_fwd_map / gdn2_bwd_map; T == 0 writes the maps of an empty piece.

@@ -104,6 +104,50 @@ def test_reduced_gates_against_oracle(oracle_mod, gate, dtype, T, Dk, Dv, chunk,
             "dlog_a %.3g" % rel_l2(got, dla_ref)
 
 
+@pytest.mark.parametrize("gate,B,T,H,strong", [("kda", 1, 4200, 2, False), ("gdn", 1, 4200, 2, False),
+                                                ("kda", 2, 300, 2, True)])
+def test_reduced_gates_tensor_core_paths(oracle_mod, gate, B, T, H, strong):
+    """The scalar-gate kernel instances on the tensor-core path where it branches: a long sequence with few heads
+    (cut into segments) and, for KDA, a few channels decaying by e^-20 per token (exact pair terms, which read b
+    from the gate); both against the oracle, dbeta on every (b, h)."""
+    D = 128
+    x, beta, la = _case(gate, B, T, H, D, D, "bf16", seed=1300 + T)
+    if strong:
+        la = la.float()
+        la[..., [5, 70, 127]] = -20.0
+        la = la.to(torch.bfloat16)
+    d = {n: t.cuda() for n, t in x.items()}
+    g_beta, g_la = beta.cuda(), la.cuda()
+    ws = torch.empty(binding.gdn2_beta_workspace_size(GATES[gate], binding.GDN2_OP_BWD, B, T, H, D, D, 64,
+                                                      binding.GDN2_BF16), dtype=torch.uint8, device="cuda")
+    o, ST = binding.gdn2_beta_fwd(GATES[gate], d["q"], d["k"], d["v"], g_la, g_beta, d["S0"], save_states=True, ws=ws)
+    g = binding.gdn2_beta_bwd(GATES[gate], d["q"], d["k"], d["v"], g_la, g_beta, d["dout"], d["S0"], None,
+                              states_saved=True, ws=ws)
+    torch.cuda.synchronize()
+    assert binding.gdn2_device_status() == binding.GDN2_OK, binding.last_error()
+    f = {n: to_f64(t) for n, t in x.items()}
+    be, lae = to_f64(beta), to_f64(la)
+    b_full = np.repeat(be[..., None], D, axis=-1)
+    la_full = lae if gate == "kda" else np.repeat(lae[..., None], D, axis=-1)
+    o_ref, ST_ref = oracle_mod.fwd(f["q"], f["k"], f["v"], la_full, b_full, b_full, S0=f["S0"])
+    ref = oracle_mod.bwd(f["q"], f["k"], f["v"], la_full, b_full, b_full, dout=f["dout"], S0=f["S0"])
+    _check(to_f64(o), o_ref, TOL_OUT["bf16"], "o")
+    _check(to_f64(ST), ST_ref, TOL_OUT["bf16"], "S_T", state=True)
+    for n in ("dq", "dk", "dv"):
+        _check(to_f64(g[n]), ref[n], TOL_GRAD["bf16"], n)
+    dbeta_ref = ref["db"].sum(-1) + ref["dw"].sum(-1)
+    got = to_f64(g["dbeta"])
+    assert np.all(np.isfinite(got))
+    assert rel_l2(got, dbeta_ref) <= TOL_GRAD["bf16"] and _worst_rows(got, dbeta_ref) <= TOL_GRAD["bf16"], \
+        "dbeta %.3g (worst row %.3g)" % (rel_l2(got, dbeta_ref), _worst_rows(got, dbeta_ref))
+    dla_ref = ref["dlog_alpha"] if gate == "kda" else ref["dlog_alpha"].sum(-1)
+    got = to_f64(g["dlog_alpha"])
+    if gate == "kda":
+        _check(got, dla_ref, TOL_GRAD["bf16"], "dlog_alpha")
+    else:
+        assert rel_l2(got, dla_ref) <= TOL_GRAD["bf16"] and _worst_rows(got, dla_ref) <= TOL_GRAD["bf16"]
+
+
 def test_reduced_gates_empty_sequence():
     B, T, H, D = 1, 0, 2, 128
     x = make_inputs(B, T, H, D, D, seed=5, dtype="bf16", with_do=True, with_S0=True)
