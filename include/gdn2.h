@@ -187,10 +187,13 @@ gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const 
  *   dbeta      [B, T, H] dt (output of the backward); for GDN2_GATE_GDN dlog_alpha
  *              is [B, T, H], else [B, T, H, Dk]
  * Everything else as gdn2_fwd / gdn2_bwd, including the chunk and the paths
- * taken. The calls broadcast beta (and a scalar decay) into the workspace,
- * run gdn2_fwd / gdn2_bwd on it, and (backward) sum the gradients of the
- * broadcast gates back over their channels: dbeta_t = sum_i db_ti +
- * sum_j dw_tj, dlog_a_t = sum_i dlog_alpha_ti.
+ * taken. On the tensor-core path (bf16, Dk = Dv = 128) with beta 4-byte
+ * aligned, the chunk kernels' scalar-gate instances read beta per token and
+ * the backward sums dbeta_t = sum_i db_ti + sum_j dw_tj itself; otherwise
+ * beta is broadcast into the workspace as b and w, gdn2_fwd / gdn2_bwd run
+ * on it and the gradients are summed back. A scalar decay (GDN2_GATE_GDN)
+ * is broadcast on both paths and its gradient summed, dlog_a_t =
+ * sum_i dlog_alpha_ti.
  * Workspace: gdn2_beta_workspace_size(gate, op, ...) bytes, 256-byte aligned;
  * one buffer of the GDN2_OP_BWD size serves gdn2_beta_fwd(save_states = 1)
  * followed by gdn2_beta_bwd(states_saved = 1). Returns 0 for an invalid gate
