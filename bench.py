@@ -401,9 +401,8 @@ def measure_configs(binding, dev, args, fwd_inputs):
 def measure_reductions(binding, dev, d, args, gdn2_ms):
     """The pages' reductions through the same kernels at the headline shape: KDA (b = w = beta * 1) and Gated
     DeltaNet (also a scalar decay), fwd (keeping the states) + bwd, against the GDN-2 step. Both run the chunk
-    kernels' scalar-gate instances (beta read per token, dbeta summed in the gradient units); Gated DeltaNet's
-    scalar decay is broadcast and its gradient summed by two elementwise kernels. `overhead_of_gdn2` is
-    gdn2_ms / reduced_ms - 1."""
+    kernels' scalar-gate instances (beta, and Gated DeltaNet's decay, read per token; dbeta and the decay's
+    gradient summed in the gradient units). `overhead_of_gdn2` is gdn2_ms / reduced_ms - 1."""
     import torch
     names = ("q", "k", "v")
     B, T, H, D = d["q"].shape
@@ -431,9 +430,9 @@ def measure_reductions(binding, dev, d, args, gdn2_ms):
         out["overhead_of_gdn2_over_" + name] = gdn2_ms / ms - 1.0
         out[name + "_status"] = binding.gdn2_device_status()
         del ws, o, ST, grads
-    out["note"] = ("KDA and Gated DeltaNet run the chunk kernels' scalar-gate instances (no b or w tiles; dbeta "
-                   "from the gradient units); Gated DeltaNet's scalar decay is broadcast and its gradient summed by "
-                   "two elementwise kernels")
+    out["note"] = ("KDA and Gated DeltaNet run the chunk kernels' scalar-gate instances: no b or w tiles (nor a "
+                   "log_alpha tile for Gated DeltaNet's scalar decay); dbeta (and dlog_a) summed in the gradient "
+                   "units")
     torch.cuda.empty_cache()
     return out
 

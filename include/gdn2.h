@@ -189,18 +189,15 @@ gdn2_status gdn2_decode_step(const void* q, const void* k, const void* v, const 
  * Everything else as gdn2_fwd / gdn2_bwd, including the chunk and the paths
  * taken. On the tensor-core path (bf16, Dk = Dv = 128) with beta 4-byte
  * aligned, the chunk kernels' scalar-gate instances read beta per token and
- * the backward sums dbeta_t = sum_i db_ti + sum_j dw_tj itself; otherwise
- * beta is broadcast into the workspace as b and w, gdn2_fwd / gdn2_bwd run
- * on it and the gradients are summed back. A scalar decay (GDN2_GATE_GDN)
- * is broadcast on both paths and its gradient summed, dlog_a_t =
- * sum_i dlog_alpha_ti.
+ * the backward sums dbeta_t = sum_i db_ti + sum_j dw_tj itself, and likewise
+ * a scalar decay (GDN2_GATE_GDN, log_alpha 4-byte aligned): dlog_a_t =
+ * sum_i dlog_alpha_ti. Otherwise the reduced gates are broadcast into the
+ * workspace, gdn2_fwd / gdn2_bwd run on them and their gradients are summed
+ * back (each call broadcasts what it needs).
  * Workspace: gdn2_beta_workspace_size(gate, op, ...) bytes, 256-byte aligned;
  * one buffer of the GDN2_OP_BWD size serves gdn2_beta_fwd(save_states = 1)
  * followed by gdn2_beta_bwd(states_saved = 1). Returns 0 for an invalid gate
- * or problem. With states_saved = 1 the backward also reuses the broadcast
- * gates that gdn2_beta_fwd(save_states = 1) left in that buffer (the same
- * gate, beta and log_alpha, like the other inputs), so a training step
- * broadcasts once; with states_saved = 0 it broadcasts them itself.
+ * or problem.
  */
 typedef enum gdn2_gate {
     GDN2_GATE_KDA = 1,   /* beta per head and token, channel-wise decay */

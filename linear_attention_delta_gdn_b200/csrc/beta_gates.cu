@@ -4,13 +4,12 @@
 // bullet, arXiv abstract) states that the operator reduces to KDA when the erase and write gates are one
 // scalar beta_t per head and token (b_t = w_t = beta_t 1), and further to Gated DeltaNet when the decay is
 // also one scalar per head and token. These entry points take the reduced gates. On the tensor-core path
-// (bf16, Dk = Dv = 128) the chunk kernels have an instance for a scalar erase and write gate: beta goes in as
-// it is, and dbeta_t = sum_i db_ti + sum_j dw_tj comes out of the backward's gradient units. Elsewhere the
-// gates are broadcast into the workspace (b, w), gdn2_fwd / gdn2_bwd run on them, and their gradients are
-// summed back over the channels. A scalar decay (Gated DeltaNet) is broadcast on both paths and its gradient
-// summed, dlog_a_t = sum_i dlog_alpha_ti. Both steps are memory-bound elementwise kernels: one warp per row,
-// 16-byte pieces, a few rows in flight per warp. A backward on saved states reuses the forward's broadcast
-// gates (they sit at the same place in the workspace for both calls), so a training step broadcasts once.
+// (bf16, Dk = Dv = 128) the chunk kernels have instances for a scalar erase and write gate and for a scalar
+// decay too: beta (and log_a) go in as they are, and dbeta_t = sum_i db_ti + sum_j dw_tj (and dlog_a_t =
+// sum_i dlog_alpha_ti) come out of the backward's gradient units. Elsewhere (or with beta, log_a not 4-byte
+// aligned) the gates are broadcast into the workspace, gdn2_fwd / gdn2_bwd run on them, and their gradients
+// are summed back over the channels, by memory-bound elementwise kernels (a row per lane group, 16-byte
+// pieces, a few rows in flight per warp); each call broadcasts what it needs.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -251,8 +250,9 @@ gdn2_status gdn2_beta_fwd(gdn2_gate gate, const void* q, const void* k, const vo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool scalar = gate == GDN2_GATE_GDN;
     const bool tc = tc_path(dt, Dk, Dv) && ((uintptr_t)beta & 3) == 0;   // the chunk kernels take beta as it is
+    const bool tc_la = tc && scalar && ((uintptr_t)log_alpha & 3) == 0;    // and the scalar decay
     const void* la_full = log_alpha;
-    if (T > 0 && (!tc || scalar)) {
+    if (T > 0 && (!tc || (scalar && !tc_la))) {
         const long long rows = (long long)B * T * H;
         void* bf = tc ? nullptr : w8 + L.b;
         void* wf = tc ? nullptr : w8 + L.w;
@@ -269,7 +269,7 @@ gdn2_status gdn2_beta_fwd(gdn2_gate gate, const void* q, const void* k, const vo
     }
     if (T > 0 && tc)
         return fwd_impl(q, k, v, la_full, beta, beta, S0, o, ST, B, T, H, Dk, Dv, chunk, dt, save_states, ws, L.base,
-                        stream, beta);
+                        stream, beta, tc_la);
     return gdn2_fwd(q, k, v, la_full, T > 0 ? w8 + L.b : nullptr, T > 0 ? w8 + L.w : nullptr, S0, o, ST, B, T, H,
                     Dk, Dv, chunk, dt, save_states, ws, L.base, stream);
 }
@@ -301,8 +301,9 @@ gdn2_status gdn2_beta_bwd(gdn2_gate gate, const void* q, const void* k, const vo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool scalar = gate == GDN2_GATE_GDN;
     const bool tc = tc_path(dt, Dk, Dv) && ((uintptr_t)beta & 3) == 0;   // the chunk kernels take beta as it is
+    const bool tc_la = tc && scalar && ((uintptr_t)log_alpha & 3) == 0;    // and the scalar decay
     const long long rows = (long long)B * T * H;
-    if (T > 0 && !states_saved && (!tc || scalar)) {   // the broadcast gates (on saved states, the forward's)
+    if (T > 0 && (!tc || (scalar && !tc_la))) {   // the broadcast gates
         void* bf = tc ? nullptr : w8 + L.b;
         void* wf = tc ? nullptr : w8 + L.w;
         cudaError_t e = dt == GDN2_BF16
@@ -317,10 +318,11 @@ gdn2_status gdn2_beta_bwd(gdn2_gate gate, const void* q, const void* k, const vo
     }
     void* dla_full = scalar ? static_cast<void*>(w8 + L.dla) : dlog_alpha;
     if (T > 0 && tc) {
-        gdn2_status st = bwd_impl(q, k, v, scalar ? static_cast<const void*>(w8 + L.la) : log_alpha, beta, beta, S0,
-                                  dout, dST, dq, dk, dv, dla_full, dbeta, dbeta, dS0, B, T, H, Dk, Dv, chunk, dt,
-                                  states_saved, ws, L.base, stream, beta, dbeta);
-        if (st != GDN2_OK || !scalar) return st;
+        const bool bcast_la = scalar && !tc_la;
+        gdn2_status st = bwd_impl(q, k, v, bcast_la ? static_cast<const void*>(w8 + L.la) : log_alpha, beta, beta, S0,
+                                  dout, dST, dq, dk, dv, bcast_la ? dla_full : dlog_alpha, dbeta, dbeta, dS0, B, T, H,
+                                  Dk, Dv, chunk, dt, states_saved, ws, L.base, stream, beta, dbeta, tc_la);
+        if (st != GDN2_OK || !bcast_la) return st;
         cudaError_t e = launch_reduce<__nv_bfloat16>(nullptr, nullptr, w8 + L.dla, dbeta, dlog_alpha, rows, Dk, Dv, s);
         if (e != cudaSuccess) {
             snprintf(g_err, sizeof(g_err), "gdn2_beta_bwd (decay gradient sum): %s", cudaGetErrorString(e));

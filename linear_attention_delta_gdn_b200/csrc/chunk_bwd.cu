@@ -233,6 +233,7 @@ struct BwdParams {
     const __nv_bfloat16 *q_raw, *la_raw;   // raw inputs, read directly only for untame channels
     const __nv_bfloat16* beta;       // [B, T, H] erase and write gates b = w = beta 1 (kernels instantiated for
     __nv_bfloat16* dbeta;            // them), and their gradient sum_i db_ti + sum_j dw_tj; else null
+    __nv_bfloat16* dla_s;            // one decay per head and token (la_raw [B, T, H]): its gradient [B, T, H]
     int nrev;                        // CTAs [0, nrev) run the reverse pass of head blockIdx.x
     int join;                        // reverse-pass CTAs take gradient units afterwards
     int grad;                        // this launch computes gradient units
@@ -652,8 +653,9 @@ static_assert(OFF_TT + TILE_C <= OFF_SDBW && OFF_SDBW + 64 * 4 <= OFF_BARS, "gra
 // images are requested into them. The next unit is published in *nxt.
 // BETA (b = w = beta 1): the b rows of QE and the w tile hold the gate of each token, written by the threads
 // at the start of the unit (no b or w tiles are loaded and b is not reloaded); dw and db are not stored, their
-// row sums (over the value and key channels) go out as dbeta.
-template <bool BETA>
+// row sums (over the value and key channels) go out as dbeta. SDEC (with BETA; one decay per head and token):
+// the log_alpha tile is written the same way, and dlog_alpha goes out as its row sums.
+template <bool BETA, bool SDEC>
 __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* sm, uint32_t tmem, int headi, int c,
                           Phases& ph, bool prefetched, NextUnit* nxt) {
     using namespace cg;
@@ -691,12 +693,15 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     int next_unit = units;    // lane 0 of warp 9: the CTA's next unit (its atomic returns while this unit runs)
     // BETA: the gates of rows tid / 16 and tid / 16 + 32 (bf16 bits, 0 past the end of the sequence), loaded
     // first and written out as b and w rows below
-    uint32_t bet16[2] = {0u, 0u};
+    uint32_t bet16[2] = {0u, 0u}, la16[2] = {0u, 0u};
     if constexpr (BETA) {
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
             const int row = (tid >> 4) + 32 * x;
-            if (t0 + row < T) bet16[x] = __bfloat16_as_ushort(p.beta[((size_t)b * T + t0 + row) * H + h]);
+            if (t0 + row < T) {
+                bet16[x] = __bfloat16_as_ushort(p.beta[((size_t)b * T + t0 + row) * H + h]);
+                if (SDEC) la16[x] = __bfloat16_as_ushort(p.la_raw[((size_t)b * T + t0 + row) * H + h]);
+            }
         }
     }
     // The loads are issued by lane 0 of several warps at once (a TMA issue takes ~100 cycles); a barrier
@@ -708,12 +713,12 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     if (lane == 0) {
         switch (warp) {
         case 0:
-            tc::mbar_arrive_expect_tx(bar_load, LOAD_GATE - (BETA ? 64u * 128u * 2u : 0u));
+            tc::mbar_arrive_expect_tx(bar_load, LOAD_GATE - (BETA ? 64u * 128u * 2u : 0u) - (SDEC ? 64u * 128u * 2u : 0u));
             if (!BETA) tma_tile(QE, 2 * C, 0, mb, b, h, t0, bar_load);
             break;
         case 1: tma_tile(QE, 2 * C, C, mq, b, h, t0, bar_load); break;
         case 2: tma_tile(KH, C, 0, mk, b, h, t0, bar_load); break;
-        case 3: tma_tile(KT, C, 0, mla, b, h, t0, bar_load); break;
+        case 3: if (!SDEC) tma_tile(KT, C, 0, mla, b, h, t0, bar_load); break;
         case 9: next_unit = (int)atomicAdd(p.counter, 1u); break;   // first needed at the G MMAs
         default: break;
         }
@@ -736,6 +741,11 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             const uint4 v = make_uint4(v16, v16, v16, v16);
             *reinterpret_cast<uint4*>(QE + panel * (2 * C * 128) + row * 128 + chunk * 16) = v;
             *reinterpret_cast<uint4*>(WW + panel * (C * 128) + row * 128 + chunk * 16) = v;
+            if (SDEC) {
+                const uint32_t l16 = la16[x] * 0x10001u;
+                *reinterpret_cast<uint4*>(KT + panel * (C * 128) + row * 128 + chunk * 16) =
+                    make_uint4(l16, l16, l16, l16);
+            }
         }
     }
     __syncthreads();   // orders thread 0's acquire and its wait before the loads and copies below
@@ -974,7 +984,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
             float al = 1.f, qq = 0.f;
             if (tau < L) {
                 const size_t off = tok_off(b, t0 + tau, h, T, H, D) + ch;
-                al = fast_exp(__bfloat162float(p.la_raw[off]));
+                al = fast_exp(__bfloat162float(SDEC ? p.la_raw[((size_t)b * T + t0 + tau) * H + h] : p.la_raw[off]));
                 qq = __bfloat162float(p.q_raw[off]);
             }
             atab[x] = al;
@@ -1082,10 +1092,18 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     }
     tc::fence_async_smem();
     __syncthreads();
-    if (tid == 0) {   // dlog_alpha; the next unit waits for the stores' reads before it reuses their tiles
+    if (!SDEC && tid == 0) {   // dlog_alpha; the next unit waits for the stores' reads before it reuses their tiles
         tc::tma_store_4d(mdla, 0, h, t0, b, DU + C * 128);
         tc::tma_store_4d(mdla, 64, h, t0, b, DU + C * 128 + 2 * C * 128);
         tc::bulk_commit();
+    }
+    if constexpr (SDEC) {   // one decay per token: row t of the dlog_alpha tile (DU rows 64..127) summed
+        const int t = tid >> 3, part = tid & 7;
+        float sla = row8_sum(DU + C * 128 + t * 128 + part * 16) + row8_sum(DU + 3 * C * 128 + t * 128 + part * 16);
+        sla += __shfl_xor_sync(0xffffffffu, sla, 1);
+        sla += __shfl_xor_sync(0xffffffffu, sla, 2);
+        sla += __shfl_xor_sync(0xffffffffu, sla, 4);
+        if (part == 0 && t < L) p.dla_s[((size_t)b * T + t0 + t) * H + h] = __float2bfloat16(sla);
     }
     if (!ok) atomicOr(&g_bwd_error, 4u);
     tc::tc_fence_before();
@@ -1094,7 +1112,7 @@ __device__ bool grad_unit(const BwdMaps& m, const BwdParams& p, unsigned char* s
     return ok;
 }
 
-template <bool BETA>
+template <bool BETA, bool SDEC>
 __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
@@ -1155,7 +1173,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(const __grid_constant_
                 __syncthreads();
                 continue;
             }
-            if (!grad_unit<BETA>(maps, p, sm, tmem, headi, c, ph, pre, nxt)) {
+            if (!grad_unit<BETA, SDEC>(maps, p, sm, tmem, headi, c, ph, pre, nxt)) {
                 // a bounded wait gave up: let a prefetch in flight land before leaving
                 if (tid == 0 && nxt->prefetched) (void)tc::mbar_wait(reinterpret_cast<uint64_t*>(sm + OFF_BARS + 48), ph.pre);
                 tc::cp_async_wait_all();
@@ -1180,11 +1198,14 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
     // one scalar gate per head and token: the kernels built for it (the b, w, db and dw maps are never used)
+    // (and one decay per head and token: the la and dla maps are then never used either)
     const bool beta = a.beta != nullptr && !(a.map_A && a.map_B);
-    void (*kern)(const BwdMaps, const BwdParams) = beta ? chunk_bwd_kernel<true> : chunk_bwd_kernel<false>;
+    const bool sdec = beta && a.scalar_decay;
+    void (*kern)(const BwdMaps, const BwdParams) = !beta ? chunk_bwd_kernel<false, false>
+                                                   : (sdec ? chunk_bwd_kernel<true, true> : chunk_bwd_kernel<true, false>);
     BwdMaps maps;
-    const void* ptrs[13] = {a.q, a.k, a.v, a.la, beta ? a.q : a.b, beta ? a.v : a.w, a.dout, a.dq, a.dk,
-                            beta ? a.dq : a.db, a.dla, a.dv, beta ? a.dv : a.dw};
+    const void* ptrs[13] = {a.q, a.k, a.v, sdec ? a.q : a.la, beta ? a.q : a.b, beta ? a.v : a.w, a.dout, a.dq, a.dk,
+                            beta ? a.dq : a.db, sdec ? a.dq : a.dla, a.dv, beta ? a.dv : a.dw};
     CUtensorMap* mp[13] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w, &maps.dout,
                            &maps.dq, &maps.dk, &maps.db, &maps.dla, &maps.dv, &maps.dw};
     if (a.map_A && a.map_B)   // no gradient units run: their output maps only need a valid address
@@ -1205,6 +1226,7 @@ cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s) {
     if (beta) {
         p.beta = static_cast<const __nv_bfloat16*>(a.beta);
         p.dbeta = static_cast<__nv_bfloat16*>(a.dbeta);
+        if (sdec) p.dla_s = static_cast<__nv_bfloat16*>(a.dla);
     }
     p.dST = a.dST; p.dS0 = a.dS0;
     p.dv = static_cast<__nv_bfloat16*>(a.dv); p.dw = static_cast<__nv_bfloat16*>(a.dw);

@@ -73,9 +73,10 @@ constexpr uint32_t GC = 104448;     // 2 x fp32 gC[128] (by unit parity)
 constexpr uint32_t STAGE = TF;      // exact path for untame channels: fp32 [4][64][16] raw-input stage
 constexpr uint32_t BAR = 2 * PIPE;  // 4 mbarriers (inputs, mma per pipeline), tmem base, abort flag
 constexpr uint32_t UMASK = BAR + 64;  // untame-channel masks: [pipeline][unit parity][4 words]
-constexpr uint32_t BETA = UMASK + 64; // scalar gates: [pipeline][unit parity][64 tokens] 32-bit words holding them
+constexpr uint32_t BETA = UMASK + 64; // scalar gates (and a scalar decay): [pipeline][unit parity][beta | log_alpha]
+                                      // [64 tokens] 32-bit words holding them
 }  // namespace wy
-constexpr uint32_t SMEM_BYTES = (sp::END > wy::BETA + 1024 ? sp::END : wy::BETA + 1024) + 1024;
+constexpr uint32_t SMEM_BYTES = (sp::END > wy::BETA + 2048 ? sp::END : wy::BETA + 2048) + 1024;
 static_assert(sp::MASK + 32 <= sp::UU1 && sp::UU1 % 1024 == 0 && sp::WW1 % 1024 == 0, "consumer layout");
 static_assert(4 * 16 * XS * 4 <= wy::GC - wy::SX && 8 * 128 * 4 <= wy::GC - wy::SX, "producer scratch fits");
 static_assert(4 * 64 * 16 * 4 == TILE_64x128 && wy::STAGE + 4 * 64 * 16 * 4 <= wy::SX, "untame stage fits");
@@ -226,8 +227,8 @@ __device__ __forceinline__ float beta_word_value(const uint32_t* words, int row,
     return __uint_as_float(((e0_odd ^ (row & H_odd)) ? w >> 16 : w & 0xFFFFu) << 16);
 }
 
-// With BETA, b is one value per token, read from the chunk's beta words (bw, e0_odd, H_odd: beta_word_value)
-// after the barrier below (QE rows 0..63 hold no b tile).
+// With BETA, b is one value per token, read from the chunk's beta words (bw, e0_odd, H_odd: beta_word_value;
+// QE rows 0..63 hold no b tile).
 template <bool BETA, typename Sync>
 __device__ __forceinline__ void gate_prep_wg(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
                                              float* gC_out, float* red, unsigned int* umask, int wt, const uint32_t* bw,
@@ -291,6 +292,53 @@ __device__ __forceinline__ void gate_prep_wg(unsigned char* QE, const unsigned c
     }
 }
 
+// The same prep with one decay and one erase / write gate per token (Gated DeltaNet): the cumulative log-decay
+// G_t and g_t = exp(G_t) are the same for every channel, so each thread keeps one value per row; log_alpha
+// and beta come from their words (lw, bw), not from tiles. Every channel is untame or none is.
+template <typename Sync>
+__device__ __forceinline__ void gate_prep_scalar_wg(unsigned char* QE, const unsigned char* KH, unsigned char* KT,
+                                                    float* gC_out, float* red, unsigned int* umask, int wt,
+                                                    const uint32_t* bw, const uint32_t* lw, int e0_odd, int H_odd,
+                                                    Sync&& wg_sync) {
+    constexpr int RB = 8;
+    const int cg = wt & 15, tb = wt >> 4;
+    float G[RB];
+#pragma unroll
+    for (int u = 0; u < RB; ++u) G[u] = beta_word_value(lw, RB * tb + u, e0_odd, H_odd) + (u > 0 ? G[u - 1] : 0.f);
+    if (cg == 0) red[tb] = G[RB - 1];
+    wg_sync();
+    float pre = 0.f;
+#pragma unroll 1
+    for (int q = 0; q < tb; ++q) pre += red[q];
+    if (tb == C / RB - 1) {
+        const float tot = pre + G[RB - 1];
+        const float gc = fast_exp(tot);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) gC_out[8 * cg + c] = gc;
+        if (tot < -TAME_LOG_DECAY && cg == 0)
+            for (int w = 0; w < 4; ++w) atomicOr(umask + w, 0xFFFFFFFFu);
+    }
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+        const int row = RB * tb + u;
+        float kk[8], qq[8], e[8], kt[8];
+        tc::ld_row8(KH, C, row, cg, kk);
+        tc::ld_row8(QE, 2 * C, C + row, cg, qq);
+        const float Gv = pre + G[u];
+        const float g = fast_exp(Gv), ig = fast_exp(-Gv);
+        const float gb = g * beta_word_value(bw, row, e0_odd, H_odd);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            e[c] = gb * kk[c];
+            kt[c] = kk[c] * ig;
+            qq[c] *= g;
+        }
+        tc::st_row8(QE, 2 * C, row, cg, e);
+        tc::st_row8(KT, C, row, cg, kt);
+        tc::st_row8(QE, 2 * C, C + row, cg, qq);
+    }
+}
+
 // Clears the Kt columns of the untame channels (umask) of the thread's 8 x 8 block (prep mapping), so that the
 // tensor-core pair products leave them out.
 __device__ __noinline__ void clear_untame_kt(unsigned char* KT, const unsigned int* umask, int wt) {
@@ -313,7 +361,7 @@ __device__ __noinline__ void clear_untame_kt(unsigned char* KT, const unsigned i
 // the end. Called by the whole warpgroup; ends with a barrier.
 __device__ __noinline__ void untame_fixup_wg(int T, int H, const __nv_bfloat16* gq, const __nv_bfloat16* gk,
                                              const __nv_bfloat16* gla, const __nv_bfloat16* gb,
-                                             const __nv_bfloat16* gbeta, int b, int h, int t0,
+                                             const __nv_bfloat16* gbeta, bool sdec, int b, int h, int t0,
                                              const unsigned int* umask, float* sA, unsigned char* PP, float* stage,
                                              unsigned char* list, unsigned char* kh_img, int wt, int wg) {
     auto wg_sync = [&]() { tc::named_sync(1 + wg, 128); };
@@ -343,7 +391,7 @@ __device__ __noinline__ void untame_fixup_wg(int T, int H, const __nv_bfloat16* 
                 float al = 1.f, kk = 0.f, ee = 0.f, qq = 0.f;
                 if (ch >= 0 && tau < L) {
                     const size_t off = tok_off(b, t0 + tau, h, T, H, D) + ch;
-                    al = fast_exp(__bfloat162float(gla[off]));
+                    al = fast_exp(__bfloat162float(sdec ? gla[((size_t)b * T + t0 + tau) * H + h] : gla[off]));
                     kk = __bfloat162float(gk[off]);
                     ee = (gbeta ? __bfloat162float(gbeta[((size_t)b * T + t0 + tau) * H + h])
                                 : __bfloat162float(gb[off])) * kk;
@@ -494,9 +542,10 @@ __device__ __forceinline__ void tmem_m64_to_tile_wg(uint32_t lane_base_col, unsi
     }
 }
 
-template <bool BETA>
+template <bool BETA, bool SDEC>
 __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* sm, uint32_t tmem, int pid) {
-    constexpr uint32_t LOAD_BYTES = PROD_LOAD_BYTES - (BETA ? 64u * 128u * 2u : 0u);   // no b tile with BETA
+    // no b tile with BETA, no log_alpha tile with SDEC
+    constexpr uint32_t LOAD_BYTES = PROD_LOAD_BYTES - (BETA ? 64u * 128u * 2u : 0u) - (SDEC ? 64u * 128u * 2u : 0u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wg = warp >> 2, wq = warp & 3, wt = tid & 127;   // pipeline, warp and thread in it
     unsigned char* pb = sm + wg * wy::PIPE;
@@ -552,30 +601,39 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         coords(u0, b, h, t0);
         tc::mbar_arrive_expect_tx(bar_in, LOAD_BYTES);
         tma_tile(QE, 2 * C, C, &m.q, b, h, t0, bar_in);
-        tma_tile(KT, C, 0, &m.la, b, h, t0, bar_in);
+        if (!SDEC) tma_tile(KT, C, 0, &m.la, b, h, t0, bar_in);
         tma_tile(KH, C, 0, &m.k, b, h, t0, bar_in);
         if (!BETA) tma_tile(QE, 2 * C, 0, &m.b, b, h, t0, bar_in);
     }
-    // BETA: a unit's beta words (by unit parity), copied one unit ahead by threads 0..63 of the pipeline
-    uint32_t* betaw = reinterpret_cast<uint32_t*>(sm + wy::BETA) + 128 * wg;
+    // BETA: a unit's beta words (and with SDEC its log_alpha words), by unit parity, copied by threads 0..63 of
+    // the pipeline at the start of the unit before. The beta words are read after the prep's first barrier:
+    // those threads wait for them at the start of the unit; the log_alpha words are read before it: with SDEC
+    // they wait at the end of the unit before, ahead of its last barrier.
+    uint32_t* betaw = reinterpret_cast<uint32_t*>(sm + wy::BETA) + 256 * wg;
     auto copy_beta = [&](int u, int par) {
         int b_, h_, t0_;
         coords(u, b_, h_, t0_);
-        beta_words_copy(betaw + 64 * par, p.beta, b_, h_, t0_, p.T, p.H, wt);
+        beta_words_copy(betaw + 128 * par, p.beta, b_, h_, t0_, p.T, p.H, wt);
+        if (SDEC) beta_words_copy(betaw + 128 * par + 64, p.la, b_, h_, t0_, p.T, p.H, wt);
         tc::cp_async_commit();
     };
-    if (BETA && u0 < units && wt < 64) copy_beta(u0, 0);
+    if (BETA && u0 < units) {
+        if (wt < 64) copy_beta(u0, 0);
+        if (SDEC) {
+            if (wt < 64) tc::cp_async_wait_all();
+            wg_sync();
+        }
+    }
     for (int u = u0; u < units; u += npipe, ++kunit) {
         const int c = u / p.BH, head = u % p.BH;
         const bool next = u + npipe < units;
         int nb = 0, nh = 0, nt0 = 0;
         if (next) coords(u + npipe, nb, nh, nt0);
-        if (BETA && wt < 64) {   // this unit's words complete (the prep reads them after its first barrier)
-            if (next) {
-                copy_beta(u + npipe, (kunit + 1) & 1);
-                tc::cp_async_wait_but1();
-            } else {
-                tc::cp_async_wait_all();
+        if (BETA && wt < 64) {
+            if (next) copy_beta(u + npipe, (kunit + 1) & 1);
+            if (!SDEC) {   // this unit's words
+                if (next) tc::cp_async_wait_but1();
+                else tc::cp_async_wait_all();
             }
         }
         float* gC = reinterpret_cast<float*>(pb + wy::GC + (kunit & 1) * 512);
@@ -591,7 +649,11 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         const bool img_ok = GDN2_IN(g_fwd_error, head < p.BH && c < p.nc);   // else the image is not written
         {
             const int e0 = (int)((((size_t)(head / p.H) * p.T + (size_t)c * C) * p.H + head % p.H) & 1);
-            gate_prep_wg<BETA>(QE, KH, KT, gC, sX, umask, wt, betaw + 64 * (kunit & 1), e0, p.H & 1, wg_sync);
+            if constexpr (SDEC)
+                gate_prep_scalar_wg(QE, KH, KT, gC, sX, umask, wt, betaw + 128 * (kunit & 1),
+                                    betaw + 128 * (kunit & 1) + 64, e0, p.H & 1, wg_sync);
+            else
+                gate_prep_wg<BETA>(QE, KH, KT, gC, sX, umask, wt, betaw + 128 * (kunit & 1), e0, p.H & 1, wg_sync);
         }
         sync_for_mma_wg();
         const bool untame = (umask[0] | umask[1] | umask[2] | umask[3]) != 0u;   // the same on every thread
@@ -620,7 +682,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             tc::bulk_wait_read();
             tc::mbar_arrive_expect_tx(bar_in, LOAD_BYTES);
             tma_tile(QE, 2 * C, C, &m.q, nb, nh, nt0, bar_in);
-            tma_tile(KT, C, 0, &m.la, nb, nh, nt0, bar_in);
+            if (!SDEC) tma_tile(KT, C, 0, &m.la, nb, nh, nt0, bar_in);
             inflight = true;
         }
         extract_AP_wg(lane_base + (tm_ap - tmem), sA, PP, wq, lane);   // A over k: the prep has read k
@@ -629,7 +691,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
         if (untame && img_ok) {   // exact terms of the channels left out of M1 (TF is free until the solve)
             int b, h, t0;
             coords(u, b, h, t0);
-            untame_fixup_wg(p.T, p.H, p.q, p.k, p.la, p.b, BETA ? p.beta : nullptr, b, h, t0, umask, sA, PP,
+            untame_fixup_wg(p.T, p.H, p.q, p.k, p.la, p.b, BETA ? p.beta : nullptr, SDEC, b, h, t0, umask, sA, PP,
                             reinterpret_cast<float*>(pb + wy::STAGE), reinterpret_cast<unsigned char*>(sX),
                             img + TC_WY_KH, wt, wg);
         }
@@ -655,6 +717,7 @@ __device__ void run_producer(const Maps& m, const FwdParams& p, unsigned char* s
             tc::bulk_commit();
             unreleased = (long long)unit;
         }
+        if (SDEC && wt < 64) tc::cp_async_wait_all();   // the next unit's words (published by the barrier)
         // all 128 threads leave together if any has seen the abort flag (the other pipeline may set it at
         // any time, so separate reads could split the threads that synchronise on this barrier)
         if (tc::named_sync_or(1 + wg, 128, *abort_flag != 0)) break;
@@ -988,7 +1051,7 @@ __device__ void run_consumer(const Maps& m, const FwdParams& p, unsigned char* s
     }
 }
 
-template <bool BETA>
+template <bool BETA, bool SDEC>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant__ Maps maps, const FwdParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays in the shared window
@@ -1008,7 +1071,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
         if (!consumer)
             for (int i = 0; i < 16; ++i) reinterpret_cast<unsigned int*>(sm + wy::UMASK)[i] = 0u;
         tc::fence_mbar_init();
-        tc::tma_prefetch_desc(&maps.q); tc::tma_prefetch_desc(&maps.k); tc::tma_prefetch_desc(&maps.la);
+        tc::tma_prefetch_desc(&maps.q); tc::tma_prefetch_desc(&maps.k);
+        if (!SDEC) tc::tma_prefetch_desc(&maps.la);
         if (consumer) {
             tc::tma_prefetch_desc(&maps.v);
             if (!BETA) tc::tma_prefetch_desc(&maps.w);
@@ -1025,7 +1089,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_base_ptr;
     if (consumer) run_consumer<BETA>(maps, p, sm, tmem, blockIdx.x);
-    else run_producer<BETA>(maps, p, sm, tmem, blockIdx.x - p.ncons);
+    else run_producer<BETA, SDEC>(maps, p, sm, tmem, blockIdx.x - p.ncons);
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -1157,7 +1221,7 @@ static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool
     for (int i = 0; i < 6; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     LaunchFacts lf{};
-    cudaError_t e = launch_facts(chunk_fwd_kernel<false>, NT, SMEM_BYTES, &lf);
+    cudaError_t e = launch_facts(chunk_fwd_kernel<false, false>, NT, SMEM_BYTES, &lf);
     if (e != cudaSuccess) return e;
     const int BH = d.B * d.H, nc = d.nchunks(), units = BH * nc, slots = lf.nsm * lf.occ;
     FwdParams p{};
@@ -1171,7 +1235,7 @@ static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool
     pp.nprod = units < slots ? units : slots;
     {
         TraceScope trace(K_CHUNK_FWD, s);
-        chunk_fwd_kernel<false><<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
+        chunk_fwd_kernel<false, false><<<pp.nprod, NT, SMEM_BYTES, s>>>(maps, pp);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (!with_maps) return cudaSuccess;
@@ -1184,7 +1248,7 @@ static cudaError_t fwd_pieces_launch(const ChunkFwdArgs& a, cudaStream_t s, bool
     pc.ncons = ntasks < slots ? ntasks : slots;
     {
         TraceScope trace(K_CHUNK_FWD, s);
-        chunk_fwd_kernel<false><<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
+        chunk_fwd_kernel<false, false><<<pc.ncons, NT, SMEM_BYTES, s>>>(maps, pc);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (!R) return cudaSuccess;
@@ -1213,9 +1277,12 @@ cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s) {
     const Dims& d = a.d;
     if (d.T == 0 || d.B * d.H == 0) return cudaSuccess;
     // one scalar gate per head and token: the kernels built for it (the b and w maps are then never read)
-    void (*kern)(const Maps, const FwdParams) = a.beta ? chunk_fwd_kernel<true> : chunk_fwd_kernel<false>;
+    // (and one decay per head and token: the la map is then never read either)
+    const bool sdec = a.beta && a.scalar_decay;
+    void (*kern)(const Maps, const FwdParams) = !a.beta ? chunk_fwd_kernel<false, false>
+                                                : (sdec ? chunk_fwd_kernel<true, true> : chunk_fwd_kernel<true, false>);
     Maps maps;
-    const void* ptrs[6] = {a.q, a.k, a.v, a.la, a.beta ? a.q : a.b, a.beta ? a.v : a.w};
+    const void* ptrs[6] = {a.q, a.k, a.v, sdec ? a.q : a.la, a.beta ? a.q : a.b, a.beta ? a.v : a.w};
     CUtensorMap* mp[6] = {&maps.q, &maps.k, &maps.v, &maps.la, &maps.b, &maps.w};
     for (int i = 0; i < 6; ++i)
         if (make_token_map(mp[i], ptrs[i], d.B, d.T, d.H) != CUDA_SUCCESS) return cudaErrorInvalidValue;

@@ -200,7 +200,7 @@ namespace gdn2 {
 gdn2_status fwd_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* b,
                      const void* w, const float* S0, void* o, float* ST, int B, int T, int H, int Dk,
                      int Dv, int chunk, gdn2_dtype dt, int save_states, void* ws, size_t ws_bytes,
-                     void* stream, const void* beta) {
+                     void* stream, const void* beta, bool scalar_decay) {
     NvtxRange nvtx("gdn2_fwd");
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
@@ -223,6 +223,7 @@ gdn2_status fwd_impl(const void* q, const void* k, const void* v, const void* lo
         a.d = d;
         a.q = q; a.k = k; a.v = v; a.la = log_alpha; a.b = b; a.w = w;
         a.beta = beta;
+        a.scalar_decay = beta != nullptr && scalar_decay;
         a.S0 = S0; a.o = o; a.ST = ST;
         unsigned char* wsb = static_cast<unsigned char*>(ws);
         const bool keep = save_states != 0;
@@ -247,7 +248,7 @@ gdn2_status bwd_impl(const void* q, const void* k, const void* v, const void* lo
                      const void* w, const float* S0, const void* dout, const float* dST, void* dq,
                      void* dk, void* dv, void* dlog_alpha, void* db, void* dw, float* dS0, int B, int T,
                      int H, int Dk, int Dv, int chunk, gdn2_dtype dt, int states_saved, void* ws,
-                     size_t ws_bytes, void* stream, const void* beta, void* dbeta) {
+                     size_t ws_bytes, void* stream, const void* beta, void* dbeta, bool scalar_decay) {
     NvtxRange nvtx("gdn2_bwd");
     gdn2_status st = check_dims(B, T, H, Dk, Dv, chunk, dt, true);
     if (st != GDN2_OK) return st;
@@ -274,6 +275,7 @@ gdn2_status bwd_impl(const void* q, const void* k, const void* v, const void* lo
             f.d = d;
             f.q = q; f.k = k; f.v = v; f.la = log_alpha; f.b = b; f.w = w;
             f.beta = beta;
+            f.scalar_decay = beta != nullptr && scalar_decay;
             f.S0 = S0; f.o = nullptr; f.ST = nullptr; f.states = wsb; f.deltas = wsb + tc_delta_offset(d);
             f.wy = wsb + tc_tp_offset(d);
             f.flags = reinterpret_cast<unsigned int*>(wsb + tc_flags_offset(d, true));
@@ -287,6 +289,7 @@ gdn2_status bwd_impl(const void* q, const void* k, const void* v, const void* lo
         a.dST = dST;
         a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.db = db; a.dw = dw; a.dS0 = dS0;
         a.beta = beta; a.dbeta = dbeta;
+        a.scalar_decay = beta != nullptr && scalar_decay;
         a.states = wsb;
         a.tp = wsb + tc_tp_offset(d);
         a.deltas = wsb + tc_delta_offset(d);

@@ -54,6 +54,7 @@ struct ChunkFwdArgs {
     float *map_N, *map_M;  // both set: compute the affine map of each head's sequence instead ([BH][128][128])
     const void* beta;      // [B,T,H] bf16, or null: erase and write gates one scalar per head and token
                            // (b = w = beta 1; b and w are then not read)
+    bool scalar_decay;     // with beta: la is [B,T,H] (one decay per head and token, broadcast over Dk)
 };
 cudaError_t chunk_fwd_launch(const ChunkFwdArgs& a, cudaStream_t s);
 cudaError_t chunk_fwd_map_launch(const ChunkFwdArgs& a, cudaStream_t s);   // map_N / map_M of every head
@@ -89,18 +90,21 @@ struct ChunkBwdArgs {
     float *map_B, *map_A;         // both set: compute the reverse affine map of each head's sequence instead
     const void* beta;             // [B,T,H] bf16, or null: b = w = beta 1 (b and w are then not read, db and dw
     void* dbeta;                  // not written; dbeta [B,T,H] bf16 = sum_i db_ti + sum_j dw_tj instead)
+    bool scalar_decay;            // with beta: la and dla are [B,T,H] (dla_t = sum_i dlog_alpha_ti)
 };
 cudaError_t chunk_bwd_launch(const ChunkBwdArgs& a, cudaStream_t s);
 // gdn2_fwd / gdn2_bwd with one scalar erase and write gate per head and token (beta [B,T,H], dbeta), taken on
 // the tensor-core path only (tc_path); b and w must be non-null but are not read there, nor db and dw written.
+// scalar_decay (with beta): log_alpha and dlog_alpha are [B,T,H]; beta and log_alpha 4-byte aligned.
 gdn2_status fwd_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* b, const void* w,
                      const float* S0, void* o, float* ST, int B, int T, int H, int Dk, int Dv, int chunk, gdn2_dtype dt,
-                     int save_states, void* ws, size_t ws_bytes, void* stream, const void* beta);
+                     int save_states, void* ws, size_t ws_bytes, void* stream, const void* beta,
+                     bool scalar_decay = false);
 gdn2_status bwd_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* b, const void* w,
                      const float* S0, const void* dout, const float* dST, void* dq, void* dk, void* dv,
                      void* dlog_alpha, void* db, void* dw, float* dS0, int B, int T, int H, int Dk, int Dv, int chunk,
                      gdn2_dtype dt, int states_saved, void* ws, size_t ws_bytes, void* stream, const void* beta,
-                     void* dbeta);
+                     void* dbeta, bool scalar_decay = false);
 // dst = M src + N per head, fp32 [BH][128][128] operands, in place allowed for src == dst
 cudaError_t state_affine_launch(const float* M, const float* N, const float* src, float* dst, int BH, int Dk, int Dv,
                                 cudaStream_t s);

@@ -148,6 +148,36 @@ def test_reduced_gates_tensor_core_paths(oracle_mod, gate, B, T, H, strong):
         assert rel_l2(got, dla_ref) <= TOL_GRAD["bf16"] and _worst_rows(got, dla_ref) <= TOL_GRAD["bf16"]
 
 
+@pytest.mark.parametrize("gate", ["kda", "gdn"])
+def test_unaligned_beta_takes_the_broadcast_path(gate):
+    """The scalar-gate kernel instances read beta as 4-byte words; a beta that is only 2-byte aligned goes through
+    the broadcast path instead, with the same results (to rounding: the gate sums run in another order)."""
+    B, T, H, D = 2, 200, 2, 128
+    x, beta, la = _case(gate, B, T, H, D, D, "bf16", seed=1400)
+    d = {n: t.cuda() for n, t in x.items()}
+    g_la = la.cuda()
+    store = torch.empty(beta.numel() + 1, dtype=torch.bfloat16, device="cuda")
+    shifted = store[1:].view(beta.shape)          # 2 bytes past a 256-byte boundary
+    shifted.copy_(beta.cuda())
+    aligned = beta.cuda()
+    assert shifted.data_ptr() % 4 == 2 and aligned.data_ptr() % 4 == 0
+    out = {}
+    for name, bt in (("aligned", aligned), ("shifted", shifted)):
+        ws = torch.empty(binding.gdn2_beta_workspace_size(GATES[gate], binding.GDN2_OP_BWD, B, T, H, D, D, 64,
+                                                          binding.GDN2_BF16), dtype=torch.uint8, device="cuda")
+        o, ST = binding.gdn2_beta_fwd(GATES[gate], d["q"], d["k"], d["v"], g_la, bt, d["S0"], save_states=True,
+                                      ws=ws)
+        g = binding.gdn2_beta_bwd(GATES[gate], d["q"], d["k"], d["v"], g_la, bt, d["dout"], d["S0"], None,
+                                  states_saved=True, ws=ws)
+        out[name] = {"o": o, "ST": ST, **g}
+    torch.cuda.synchronize()
+    assert binding.gdn2_device_status() == binding.GDN2_OK, binding.last_error()
+    for n in ("o", "ST", "dq", "dk", "dv", "dbeta", "dlog_alpha", "dS0"):
+        a_, b_ = to_f64(out["aligned"][n]), to_f64(out["shifted"][n])
+        assert np.all(np.isfinite(b_)), n
+        assert rel_l2(b_, a_) <= 1e-2, (n, rel_l2(b_, a_))
+
+
 def test_reduced_gates_empty_sequence():
     B, T, H, D = 1, 0, 2, 128
     x = make_inputs(B, T, H, D, D, seed=5, dtype="bf16", with_do=True, with_S0=True)
