@@ -24,6 +24,8 @@ Besides the headline step, the line carries (rank 0, N=1):
     operator) forward + backward at d_model = 2048, with the library's share;
   * ``context_parallel_maps``: a context-parallel rank's map kernels on one
     16K-token piece, beside that piece's own forward and fwd+bwd;
+  * ``host_overhead``: host time to issue one fwd + bwd step through the binding
+    at a one-chunk problem, beside its device time;
   * ``cpu_baseline``: the fp64 oracle timed on a bounded sample of the headline
     workload on the host cores, with the GPU outputs of those same sequences
     compared against the oracle's (relative L2, whole sample and worst head);
@@ -503,6 +505,46 @@ def measure_layer_step(binding, dev, args, B, T, H, D=128):
     return out
 
 
+def measure_host_overhead(binding, dev, calls=200):
+    """Host time per call of the C ABI through the binding (gdn2_fwd keeping its states + gdn2_bwd on them) at a
+    one-chunk problem, B=1 H=1 T=64, where the device work is a few microseconds: the wall time to issue `calls`
+    steps back to back (no synchronisation inside; workspace, outputs and gradients preallocated), beside the
+    device time per step from CUDA events. The entry points cache the tensor maps (per pointer and shape) and the
+    launch facts, so a repeated call does argument checks, a flag memset and the launches."""
+    import torch
+    B, T, H, D = 1, 64, 1, 128
+    d = device_inputs(B, T, H, D, 4242, True, dev)
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    ws = torch.empty(binding.gdn2_workspace_size(binding.GDN2_OP_BWD, B, T, H, D, D, 64, binding.GDN2_BF16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    grads = {n: torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+             for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw")}
+    grads["dS0"] = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+
+    def step():
+        binding.gdn2_fwd(*(d[n] for n in names), None, save_states=True, ws=ws, o=o, ST=ST)
+        binding.gdn2_bwd(*(d[n] for n in names), d["dout"], None, None, states_saved=True, ws=ws, grads=grads)
+
+    for _ in range(10):
+        step()
+    torch.cuda.synchronize(dev)
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        step()
+    t1 = time.perf_counter()
+    e.record()
+    torch.cuda.synchronize(dev)
+    return {"workload": "fwdbwd-bf16-b1h1t64d128", "steps": calls,
+            "host_us_per_step": (t1 - t0) / calls * 1e6, "device_us_per_step": a.elapsed_time(e) / calls * 1e3,
+            "status": binding.gdn2_device_status(),
+            "note": "host time to issue one fwd (keeping its states) + bwd through the Python binding and the C ABI, "
+                    "and the device time per step when the steps run back to back"}
+
+
 def measure_context_maps(binding, dev, args, T=16384, H=16, D=128):
     """Per-rank cost of context parallelism on one piece (B = 1, T tokens, H heads): the piece's forward and
     reverse maps against its own forward and fwd+bwd (what a rank runs anyway)."""
@@ -730,7 +772,7 @@ def main():
     full = args.B is None and args.T is None
     if not args.no_decode and full:
         decode = bench_decode(binding, dev)
-    reductions = layer_gates = cp_maps = layer_step = None
+    reductions = layer_gates = cp_maps = layer_step = host = None
     if not args.no_extra and full and world == 1:
         configs = measure_configs(binding, dev, args, d)
         sweep = measure_sweep(binding, dev, args)
@@ -738,6 +780,7 @@ def main():
         layer_gates = measure_layer_gates(binding, dev, args, B, T, H)
         layer_step = measure_layer_step(binding, dev, args, B, T, H)
         cp_maps = measure_context_maps(binding, dev, args)
+        host = measure_host_overhead(binding, dev)
 
     line = None
     if rank == 0:
@@ -761,7 +804,8 @@ def main():
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_in_timed_region,
                 "decode": decode, "configs": configs, "sweep": sweep, "kda_overhead": reductions,
-                "layer_gates": layer_gates, "layer_step": layer_step, "context_parallel_maps": cp_maps}
+                "layer_gates": layer_gates, "layer_step": layer_step, "context_parallel_maps": cp_maps,
+                "host_overhead": host}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
