@@ -105,16 +105,20 @@ def test_reduced_gates_against_oracle(oracle_mod, gate, dtype, T, Dk, Dv, chunk,
 
 
 @pytest.mark.parametrize("gate,B,T,H,strong", [("kda", 1, 4200, 2, False), ("gdn", 1, 4200, 2, False),
-                                                ("kda", 2, 300, 2, True)])
+                                                ("kda", 2, 300, 2, True), ("gdn", 2, 300, 2, True)])
 def test_reduced_gates_tensor_core_paths(oracle_mod, gate, B, T, H, strong):
     """The scalar-gate kernel instances on the tensor-core path where it branches: a long sequence with few heads
-    (cut into segments) and, for KDA, a few channels decaying by e^-20 per token (exact pair terms, which read b
-    from the gate); both against the oracle, dbeta on every (b, h)."""
+    (cut into segments) and strong decay: for KDA a few channels decaying by e^-20 per token, for Gated DeltaNet
+    one head decaying by e^-20 per token over its second half (every channel of its chunks there takes the exact
+    pair terms, which read b and the decay from the per-token gates); against the oracle, dbeta on every (b, h)."""
     D = 128
     x, beta, la = _case(gate, B, T, H, D, D, "bf16", seed=1300 + T)
     if strong:
         la = la.float()
-        la[..., [5, 70, 127]] = -20.0
+        if gate == "kda":
+            la[..., [5, 70, 127]] = -20.0
+        else:
+            la[:, T // 2:, 1] = -20.0
         la = la.to(torch.bfloat16)
     d = {n: t.cuda() for n, t in x.items()}
     g_beta, g_la = beta.cuda(), la.cuda()
