@@ -72,3 +72,33 @@ def test_more_heads_than_sms_match_the_same_heads_alone():
         small = _run(sl, dST[bsel:bsel + 1].contiguous())
         for n in big:
             assert torch.equal(big[n][bsel:bsel + 1], small[n]), (bsel, n)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("gate", ["kda", "gdn"])
+def test_two_launch_form_matches_for_scalar_gates(request, gate):
+    """The same for the kernels' scalar-gate (KDA) and scalar-decay (Gated DeltaNet) instances."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    B, T, H = 2, 333, 3
+    d, dST = _inputs(B, T, H, seed=4343)
+    g = torch.Generator().manual_seed(17)
+    beta = torch.sigmoid(torch.randn((B, T, H), generator=g)).to(torch.bfloat16).cuda()
+    code = binding.GDN2_GATE_KDA if gate == "kda" else binding.GDN2_GATE_GDN
+    la = d["log_alpha"] if gate == "kda" else \
+        (-torch.nn.functional.softplus(torch.randn((B, T, H), generator=g)) / 16.0).to(torch.bfloat16).cuda()
+
+    def run():
+        need = binding.gdn2_beta_workspace_size(code, binding.GDN2_OP_BWD, B, T, H, 128, 128, 64, binding.GDN2_BF16)
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        o, ST = binding.gdn2_beta_fwd(code, d["q"], d["k"], d["v"], la, beta, d["S0"], save_states=True, ws=ws)
+        gr = binding.gdn2_beta_bwd(code, d["q"], d["k"], d["v"], la, beta, d["dout"], d["S0"], dST,
+                                   states_saved=True, ws=ws)
+        torch.cuda.synchronize()
+        return {"o": o, "ST": ST, **gr}
+
+    coop = run()
+    request.getfixturevalue("no_cooperative")
+    two = run()
+    for n in coop:
+        assert torch.equal(coop[n], two[n]), n
