@@ -167,3 +167,31 @@ def test_maps_are_computed_on_the_tensor_core_path_only(L):
     assert rc == binding.GDN2_ERR_INVALID
     rc = L.gdn2_state_affine(None, None, None, None, 1, 1, 128, 128, None)
     assert rc == binding.GDN2_ERR_INVALID
+
+
+def test_reduced_gate_workspace_sizes_and_checks(L):
+    """gdn2_beta_workspace_size: the GDN-2 workspace, then the broadcast gates (b, w and, for a scalar decay,
+    log_alpha) and, for the backward, their gradients, each region 256-byte aligned. A forward that keeps its
+    states takes the backward's GDN-2 size as its base, so the gates sit at the same offsets in both calls and one
+    buffer of the backward's size serves both. Bad gates and missing pointers are refused before any launch."""
+    from linear_attention_delta_gdn_b200.binding import gdn2_workspace_size as ws
+    from linear_attention_delta_gdn_b200 import binding
+    al = lambda x: (x + 255) // 256 * 256
+    B, T, H, D = 4, 4096, 16, 128
+    rows = B * T * H
+    tile = al(rows * D * 2)
+    for gate, ntiles in ((binding.GDN2_GATE_KDA, 2), (binding.GDN2_GATE_GDN, 3)):
+        bws = lambda op: binding.gdn2_beta_workspace_size(gate, op, B, T, H, D, D, 64, binding.GDN2_BF16)
+        assert bws(0) == al(ws(0, B, T, H, D, D, 64, 1)) + ntiles * tile
+        assert bws(1) == al(ws(2, B, T, H, D, D, 64, 1)) + ntiles * tile
+        assert bws(2) == al(ws(2, B, T, H, D, D, 64, 1)) + 2 * ntiles * tile
+        assert bws(1) <= bws(2)
+    assert binding.gdn2_beta_workspace_size(7, 2, B, T, H, D, D, 64, binding.GDN2_BF16) == 0
+    assert binding.gdn2_beta_workspace_size(binding.GDN2_GATE_KDA, 2, B, T, H, 96, D, 64, binding.GDN2_BF16) == 0
+    p = 1 << 20
+    # gate 7 is neither KDA nor Gated DeltaNet; beta NULL
+    rc = L.gdn2_beta_fwd(7, p, p, p, p, p, None, p, None, 1, 8, 1, 128, 128, 64, 1, 0, p, 1 << 30, None)
+    assert rc == 1 and b"GDN2_GATE_KDA" in L.gdn2_last_error()
+    rc = L.gdn2_beta_fwd(binding.GDN2_GATE_KDA, p, p, p, p, None, None, p, None, 1, 8, 1, 128, 128, 64, 1, 0, p,
+                         1 << 30, None)
+    assert rc == 1 and b"beta" in L.gdn2_last_error()
